@@ -1,0 +1,411 @@
+"""Pins for the CPU oracle: checks against what the pages and the mathematics fix.
+
+None of these re-types the oracle's own formulas.  They use library routines
+(numpy float16, torch bfloat16, numpy matmul, torch scaled_dot_product_attention),
+closed forms, invariants, and the figures the pages print (tests/golden/).
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+MIB = float(1 << 20)
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ----------------------------------------------------------------------------
+# number formats, pinned to library conversions
+# ----------------------------------------------------------------------------
+
+def _edge_floats():
+    v = [0.0, -0.0, 1.0, -1.0, 65504.0, 65519.99, 65520.0, 65536.0, 1e30, -1e30,
+         2.0 ** -14, 2.0 ** -24, 2.0 ** -25, 3 * 2.0 ** -26, 2.0 ** -26, 6.1e-5, 1e-8, 1e-45,
+         float("inf"), -float("inf")]
+    # exact binary16 ties: halfway between neighbours at several binades
+    for e in (-20, -14, -3, 0, 5, 14, 15):
+        ulp = 2.0 ** (e - 10) if e >= -14 else 2.0 ** -24
+        for k in (1024, 1025, 1500, 2046, 2047):
+            base = k * ulp if e >= -14 else (k - 1024) * ulp
+            v += [base + ulp / 2, -(base + ulp / 2)]
+    return np.array(v, np.float32)
+
+
+def test_f32_to_f16_matches_numpy():
+    rng = np.random.default_rng(11)
+    bits = rng.integers(0, 2 ** 32, size=60000, dtype=np.uint64).astype(np.uint32)
+    vals = np.concatenate([bits.view(np.float32), _edge_floats(),
+                           rng.standard_normal(20000).astype(np.float32) * 1e-5,
+                           rng.standard_normal(20000).astype(np.float32) * 3e4])
+    ref = vals.astype(np.float16).view(np.uint16)
+    got = np.array([oracle.f32_to_f16_bits(x) for x in vals], np.uint16)
+    nan = np.isnan(vals)
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert np.all((got[nan] & 0x7C00) == 0x7C00) and np.all((got[nan] & 0x3FF) != 0)
+
+
+def test_f64_to_f16_matches_numpy():
+    rng = np.random.default_rng(12)
+    vals = np.concatenate([rng.standard_normal(30000) * s for s in (1e-7, 1e-3, 1.0, 1e3, 7e4)])
+    vals = np.concatenate([vals, _edge_floats().astype(np.float64),
+                           np.array([1 + 2.0 ** -11 + 2.0 ** -40, 1 + 2.0 ** -11 - 2.0 ** -40])])
+    ref = vals.astype(np.float16).view(np.uint16)
+    got = np.array([oracle.f64_to_f16_bits(x) for x in vals], np.uint16)
+    assert np.array_equal(got, ref)
+
+
+def test_f16_to_f32_matches_numpy_all_codes():
+    codes = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    ref = codes.view(np.float16).astype(np.float32)
+    got = np.array([oracle.f16_bits_to_f32(int(c)) for c in codes], np.float32)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan].view(np.uint32), ref[~nan].view(np.uint32))
+
+
+def test_f32_to_bf16_matches_torch():
+    rng = np.random.default_rng(13)
+    bits = rng.integers(0, 2 ** 32, size=50000, dtype=np.uint64).astype(np.uint32)
+    vals = bits.view(np.float32)
+    vals = vals[~np.isnan(vals)]
+    ties = (np.arange(1, 3000, dtype=np.uint32) << 16 | 0x8000).view(np.float32)
+    vals = np.concatenate([vals, ties, -ties])
+    ref = torch.from_numpy(vals).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = np.array([oracle.f32_to_bf16_bits(x) for x in vals], np.uint16)
+    assert np.array_equal(got, ref)
+
+
+# ----------------------------------------------------------------------------
+# quantiser
+# ----------------------------------------------------------------------------
+
+def _scale_f32(s_bits):
+    return np.asarray(s_bits, np.uint16).view(np.float16).astype(np.float32)
+
+
+def _signed_codes(codes, bits, dim):
+    if bits == 8:
+        return codes.view(np.int8).astype(np.int32)
+    lo = (codes & 0xF).astype(np.int32)
+    hi = (codes >> 4).astype(np.int32)
+    out = np.empty(codes.shape[:-1] + (dim,), np.int32)
+    out[..., 0::2] = lo
+    out[..., 1::2] = hi
+    return np.where(out >= 8, out - 16, out)
+
+
+@pytest.mark.parametrize("bits,group", [(8, 128), (8, 32), (4, 32), (4, 128), (8, 64)])
+def test_quantizer_error_bound_and_code_range(bits, group):
+    rng = np.random.default_rng(100 + bits + group)
+    dim = 128
+    mags = np.array([1e-3, 0.1, 1.0, 7.0, 300.0], np.float32)
+    x = (rng.standard_normal((400, dim)).astype(np.float32)
+         * mags[rng.integers(0, len(mags), 400)][:, None]).astype(np.float16).astype(np.float32)
+    codes, scales = oracle.quantize_rows(x, group, bits)
+    qmax = 127 if bits == 8 else 7
+    c = _signed_codes(codes, bits, dim)
+    s = np.repeat(_scale_f32(scales), group, axis=-1)
+    assert np.all(np.abs(c) <= qmax)
+    # error bound |x - c*s| <= s/2 (plus fp32 rounding of the quotient)
+    err = np.abs(x.astype(np.float64) - c.astype(np.float64) * s.astype(np.float64))
+    assert np.all(err <= s.astype(np.float64) * 0.5 * (1 + 2.0 ** -20))
+    # the scale is the binary16 nearest to fp32(absmax / qmax) (numpy's conversion)
+    a = np.abs(x).reshape(400, dim // group, group).max(-1)
+    want = (a.astype(np.float32) / np.float32(qmax)).astype(np.float16).view(np.uint16)
+    assert np.array_equal(scales, want)
+    # the absmax element of every group maps to +-qmax (normal-range scales)
+    xg = x.reshape(400, dim // group, group)
+    cg = c.reshape(400, dim // group, group)
+    idx = np.abs(xg).argmax(-1)
+    top = np.take_along_axis(cg, idx[..., None], -1)[..., 0]
+    normal = _scale_f32(scales) >= 2.0 ** -14
+    assert np.all(np.abs(top[normal]) == qmax)
+
+
+def test_quantizer_ties_round_half_even_int8():
+    # absmax 127 gives s32 = 1.0 exactly, s16 = 1.0: codes are rne(x)
+    x = np.zeros((1, 32), np.float32)
+    x[0, :10] = [127, 2.5, 3.5, -2.5, -3.5, 0.5, 1.5, -0.5, 126.5, -1.5]
+    codes, scales = oracle.quantize_rows(x, 32, 8)
+    assert scales[0, 0] == 0x3C00
+    c = codes.view(np.int8)[0, :10].tolist()
+    assert c == [127, 2, 4, -2, -4, 0, 2, 0, 126, -2]
+
+
+def test_quantizer_ties_round_half_even_int4_and_nibble_order():
+    x = np.zeros((1, 32), np.float32)
+    x[0, :8] = [7, 2.5, -0.5, 6.5, 1, -2, -7, 5.5]
+    codes, scales = oracle.quantize_rows(x, 32, 4)
+    assert scales[0, 0] == 0x3C00
+    # codes 7, 2, 0, 6, 1, -2, -7, 6 ; element 2j low nibble, 2j+1 high nibble
+    assert codes[0, :4].tolist() == [0x27, 0x60, 0xE1, 0x69]
+
+
+def test_quantizer_zero_group_and_saturation_and_subnormal():
+    x = np.zeros((3, 32), np.float32)
+    x[1, 0] = 1e7          # absmax/127 > 65504: scale saturates to 65504
+    x[1, 1] = -5e6
+    x[2, 0] = 1e-5         # scale is a binary16 subnormal
+    x[2, 1] = -3e-6
+    codes, scales = oracle.quantize_rows(x, 32, 8)
+    assert scales[0, 0] == 0 and np.all(codes[0] == 0)
+    assert scales[1, 0] == 0x7BFF
+    c = codes.view(np.int8)
+    assert c[1, 0] == 127 and c[1, 1] == -76          # 5e6/65504 = 76.3
+    assert 0 < scales[2, 0] < 0x0400                  # subnormal scale kept
+    assert c[2, 0] == 127                              # clamped
+
+
+def test_quantizer_idempotent_when_a_code_reaches_qmax():
+    rng = np.random.default_rng(7)
+    for bits, group in ((8, 128), (4, 32), (8, 32)):
+        x = rng.standard_normal((64, 128)).astype(np.float16).astype(np.float32)
+        codes, scales = oracle.quantize_rows(x, group, bits)
+        xr = oracle.dequantize_rows(codes, scales, 128, group, bits).astype(np.float32)
+        codes2, scales2 = oracle.quantize_rows(xr, group, bits)
+        assert np.array_equal(codes, codes2) and np.array_equal(scales, scales2)
+
+
+def test_dequantize_is_exact_product():
+    rng = np.random.default_rng(8)
+    x = rng.standard_normal((16, 128)).astype(np.float32)
+    codes, scales = oracle.quantize_rows(x, 32, 4)
+    xr = oracle.dequantize_rows(codes, scales, 128, 32, 4)
+    c = _signed_codes(codes, 4, 128).astype(np.float64)
+    s = np.repeat(_scale_f32(scales).astype(np.float64), 32, axis=-1)
+    assert np.array_equal(xr, c * s)
+
+
+# ----------------------------------------------------------------------------
+# attention: closed forms, invariants, library cross-check
+# ----------------------------------------------------------------------------
+
+def _cache(k, v, kb, vb, kg, vg):
+    """k, v: [B, Hkv, L, dh] float32 -> oracle cache arrays in the ABI layout."""
+    def q(x, bits, g):
+        if bits == 16:
+            return x.astype(np.float16).view(np.uint16), None
+        return oracle.quantize_rows(x, g, bits)
+    kc, ks = q(k, kb, kg)
+    vc, vs = q(v, vb, vg)
+    return kc, ks, vc, vs
+
+
+def _deq(c, s, bits, g, dh):
+    if bits == 16:
+        return c.view(np.float16).astype(np.float64)
+    return oracle.dequantize_rows(c, s, dh, g, bits)
+
+
+def _run(q, lens, k, v, kb=8, vb=8, kg=None, vg=None, tau=0.0):
+    B, Hkv, L, dh = k.shape
+    kg = kg or dh
+    vg = vg or dh
+    kc, ks, vc, vs = _cache(k, v, kb, vb, kg, vg)
+    out = oracle.decode_layer(q, lens, kc, ks, kb, kg, vc, vs, vb, vg, Hkv, tau)
+    return out, _deq(kc, ks, kb, kg, dh), _deq(vc, vs, vb, vg, dh)
+
+
+@pytest.mark.parametrize("kb,vb", [(8, 8), (4, 8), (8, 4), (16, 16)])
+def test_single_token_returns_its_value(kb, vb):
+    rng = np.random.default_rng(20)
+    k = rng.standard_normal((2, 3, 1, 64)).astype(np.float32)
+    v = rng.standard_normal((2, 3, 1, 64)).astype(np.float32)
+    q = rng.standard_normal((2, 6, 64)).astype(np.float32)
+    out, _, vh = _run(q, np.array([1, 1], np.int32), k, v, kb, vb, 32, 32)
+    for h in range(6):
+        assert np.array_equal(out[:, h], vh[:, h // 2, 0])
+
+
+def test_zero_query_returns_mean_of_values():
+    rng = np.random.default_rng(21)
+    k = rng.standard_normal((1, 2, 37, 128)).astype(np.float32)
+    v = rng.standard_normal((1, 2, 37, 128)).astype(np.float32)
+    q = np.zeros((1, 2, 128), np.float32)
+    out, _, vh = _run(q, np.array([37], np.int32), k, v, 8, 4, 128, 32)
+    np.testing.assert_allclose(out[0], vh[0].mean(axis=1), rtol=0, atol=1e-13)
+
+
+def test_equal_keys_return_mean_of_values():
+    rng = np.random.default_rng(22)
+    row = rng.standard_normal(64).astype(np.float32)
+    k = np.broadcast_to(row, (1, 1, 50, 64)).copy()
+    v = rng.standard_normal((1, 1, 50, 64)).astype(np.float32)
+    q = rng.standard_normal((1, 1, 64)).astype(np.float32) * 5
+    out, _, vh = _run(q, np.array([50], np.int32), k, v)
+    np.testing.assert_allclose(out[0, 0], vh[0, 0].mean(axis=0), rtol=0, atol=1e-13)
+
+
+def test_two_tokens_closed_form_with_softmax_scale():
+    # out = v0 + (v1 - v0) * logistic(tau * (q.k1 - q.k0)); catches a missing or wrong tau
+    rng = np.random.default_rng(23)
+    k = rng.standard_normal((1, 1, 2, 64)).astype(np.float32)
+    v = rng.standard_normal((1, 1, 2, 64)).astype(np.float32)
+    q = rng.standard_normal((1, 1, 64)).astype(np.float32)
+    for tau in (0.0, 0.37):
+        out, kh, vh = _run(q, np.array([2], np.int32), k, v, 8, 8, tau=tau)
+        t = tau if tau > 0 else 1 / math.sqrt(64)
+        d = t * (q[0, 0].astype(np.float64) @ (kh[0, 0, 1] - kh[0, 0, 0]))
+        w = 1.0 / (1.0 + math.exp(-d))
+        np.testing.assert_allclose(out[0, 0], vh[0, 0, 0] + (vh[0, 0, 1] - vh[0, 0, 0]) * w,
+                                   rtol=0, atol=1e-13)
+
+
+def test_dominant_key_returns_its_value():
+    rng = np.random.default_rng(24)
+    L = 200
+    k = rng.standard_normal((1, 1, L, 128)).astype(np.float32) * 0.01
+    k[0, 0, 77] = 1.0
+    v = rng.standard_normal((1, 1, L, 128)).astype(np.float32)
+    q = np.full((1, 1, 128), 60.0, np.float32)
+    out, _, vh = _run(q, np.array([L], np.int32), k, v)
+    np.testing.assert_allclose(out[0, 0], vh[0, 0, 77], rtol=0, atol=1e-12)
+
+
+def test_gqa_query_head_reads_kv_head_floor_h_over_g():
+    # value heads are constant per KV head; q = 0 averages, so out[h] names its KV head
+    Hkv, G, L = 3, 4, 9
+    k = np.random.default_rng(25).standard_normal((1, Hkv, L, 64)).astype(np.float32)
+    v = np.zeros((1, Hkv, L, 64), np.float32)
+    for j in range(Hkv):
+        v[0, j] = j + 1
+    q = np.zeros((1, Hkv * G, 64), np.float32)
+    out, _, vh = _run(q, np.array([L], np.int32), k, v)
+    for h in range(Hkv * G):
+        np.testing.assert_allclose(out[0, h], vh[0, h // G, 0], rtol=0, atol=1e-12)
+        assert abs(out[0, h, 0] - (h // G + 1)) < 0.01
+
+
+def test_replicated_kv_heads_equal_shared_head():
+    rng = np.random.default_rng(26)
+    k = rng.standard_normal((1, 1, 40, 64)).astype(np.float32)
+    v = rng.standard_normal((1, 1, 40, 64)).astype(np.float32)
+    q = rng.standard_normal((1, 4, 64)).astype(np.float32)
+    shared, _, _ = _run(q, np.array([40], np.int32), k, v, 4, 8, 32, 64)
+    rep, _, _ = _run(q, np.array([40], np.int32), np.repeat(k, 4, 1), np.repeat(v, 4, 1), 4, 8, 32, 64)
+    np.testing.assert_allclose(shared, rep, rtol=0, atol=1e-14)
+
+
+def test_token_permutation_and_duplication_invariance():
+    rng = np.random.default_rng(27)
+    L = 33
+    k = rng.standard_normal((1, 2, L, 64)).astype(np.float32)
+    v = rng.standard_normal((1, 2, L, 64)).astype(np.float32)
+    q = rng.standard_normal((1, 2, 64)).astype(np.float32)
+    base, _, _ = _run(q, np.array([L], np.int32), k, v, 8, 4, 64, 32)
+    perm = rng.permutation(L)
+    p, _, _ = _run(q, np.array([L], np.int32), k[:, :, perm], v[:, :, perm], 8, 4, 64, 32)
+    dup, _, _ = _run(q, np.array([2 * L], np.int32), np.concatenate([k, k], 2),
+                     np.concatenate([v, v], 2), 8, 4, 64, 32)
+    np.testing.assert_allclose(p, base, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dup, base, rtol=0, atol=1e-13)
+
+
+def test_lengths_truncate_and_empty_sequence_is_zero():
+    rng = np.random.default_rng(28)
+    k = rng.standard_normal((2, 1, 20, 64)).astype(np.float32)
+    v = rng.standard_normal((2, 1, 20, 64)).astype(np.float32)
+    q = rng.standard_normal((2, 1, 64)).astype(np.float32)
+    out, _, _ = _run(q, np.array([0, 7], np.int32), k, v)
+    assert np.all(out[0] == 0)
+    short, _, _ = _run(q[1:], np.array([7], np.int32), k[1:, :, :7], v[1:, :, :7])
+    np.testing.assert_allclose(out[1], short[0], rtol=0, atol=1e-14)
+
+
+def test_16bit_mode_matches_torch_sdpa_fp64():
+    rng = np.random.default_rng(29)
+    B, Hkv, G, L, dh = 2, 2, 3, 45, 128
+    k = rng.standard_normal((B, Hkv, L, dh)).astype(np.float16).astype(np.float32)
+    v = rng.standard_normal((B, Hkv, L, dh)).astype(np.float16).astype(np.float32)
+    q = rng.standard_normal((B, Hkv * G, dh)).astype(np.float32)
+    out, _, _ = _run(q, np.array([L, L], np.int32), k, v, 16, 16)
+    kk = torch.from_numpy(np.repeat(k, G, 1)).double()
+    vv = torch.from_numpy(np.repeat(v, G, 1)).double()
+    qq = torch.from_numpy(q).double()[:, :, None, :]
+    ref = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv)[:, :, 0].numpy()
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# h-mode reconstruction
+# ----------------------------------------------------------------------------
+
+def _h_setup(n_tok=48, D=512, N=256, seed=30):
+    rng = np.random.default_rng(seed)
+    r = rng.standard_normal((n_tok, D))
+    h = ((r - r.mean(-1, keepdims=True)) / np.sqrt(r.var(-1, keepdims=True) + 1e-5)).astype(np.float16)
+    W = torch.from_numpy(rng.standard_normal((N, D)) / math.sqrt(D)).float().to(torch.bfloat16)
+    Wb = W.view(torch.int16).numpy().view(np.uint16)
+    return h, Wb, W.double().numpy()
+
+
+def test_h_reconstruct_fp16_h_equals_matmul():
+    h, Wb, W = _h_setup()
+    y64, y16 = oracle.h_reconstruct(h.view(np.uint16), None, 512, 4, 16, Wb, round_bf16=False)
+    ref = h.astype(np.float64) @ W.T
+    np.testing.assert_allclose(y64, ref, rtol=1e-13, atol=1e-13)
+    assert np.array_equal(y16, ref.astype(np.float16).view(np.uint16))
+
+
+@pytest.mark.parametrize("bits,lo,hi", [(8, 0.003, 0.012), (4, 0.05, 0.20)])
+def test_h_quantized_kv_error_band(bits, lo, hi):
+    # TinyLoop docs, mode table: INT8-h K/V relative L2 error ~0.6 %, INT4-h ~10 %
+    h, Wb, W = _h_setup(n_tok=64, D=2048, N=512, seed=31)
+    groups = 16
+    codes, scales = oracle.quantize_rows(h.astype(np.float32), 2048 // groups, bits)
+    y64, _ = oracle.h_reconstruct(codes, scales, 2048, groups, bits, Wb, round_bf16=False)
+    ref = h.astype(np.float64) @ W.T
+    rel = np.linalg.norm(y64 - ref) / np.linalg.norm(ref)
+    assert lo < rel < hi, rel
+
+
+# ----------------------------------------------------------------------------
+# bytes per token per layer: the printed figures
+# ----------------------------------------------------------------------------
+
+def test_tinyloop_bytes_per_token_layer():
+    g = _golden("tinyloop_bytes.json")
+    D, H = g["d_model"], g["n_heads"]
+    dh = D // H
+    b = g["bytes_per_token_per_layer"]
+    assert oracle.bytes_per_token_layer(0, H, dh, 16, 16) == b["fp16_kv"]
+    assert oracle.bytes_per_token_layer(0, H, dh, 8, 8, dh, dh) == b["int8_kv"]
+    assert oracle.bytes_per_token_layer(1, d_model=D, h_bits=16, h_groups=H) == b["fp16_h"]
+    assert oracle.bytes_per_token_layer(1, d_model=D, h_bits=8, h_groups=H) == b["int8_h"]
+    assert oracle.bytes_per_token_layer(1, d_model=D, h_bits=4, h_groups=H) == b["int4_h"]
+    fp = g["footprint"]
+    n = fp["n_layers"] * fp["max_seq_len"]
+    assert round(b["fp16_kv"] * n / MIB) == fp["mib"]["fp16_kv"]
+    assert round(b["int8_kv"] * n / MIB) == fp["mib"]["int8_kv"]
+    assert round(b["fp16_h"] * n / MIB) == fp["mib"]["fp16_h"]
+    assert round(1 - b["int4_h"] / b["fp16_kv"], 2) == g["h_limit"]["saving"]
+
+
+def test_kvsplit_mib_at_8k_tokens():
+    g = _golden("kvsplit_mib.json")
+    n = g["n_layers"] * g["tokens"]
+    H, dh, grp = g["n_kv_heads"], g["head_dim"], g["group"]
+    assert oracle.bytes_per_token_layer(0, H, dh, 16, 16) * n / MIB == g["mib"]["fp16"]
+    for name, (kb, vb) in {"K8V8": (8, 8), "K8V4": (8, 4), "K4V4": (4, 4)}.items():
+        got = oracle.bytes_per_token_layer(0, H, dh, kb, vb, grp, grp) * n / MIB
+        assert got == g["mib"][name], (name, got)
+
+
+def test_ondevice_mib_k4v8_codes():
+    g = _golden("ondevice_mib.json")
+    n = g["n_layers"] * g["tokens"]
+    H, dh = g["n_kv_heads"], g["head_dim"]
+    assert oracle.bytes_per_token_layer(0, H, dh, 16, 16) * n / MIB == g["mib"]["fp16"]
+    with_scales = oracle.bytes_per_token_layer(0, H, dh, 4, 8, dh, dh)
+    codes_only = with_scales - 2 * H * 2          # one fp16 scale per head per tensor
+    assert codes_only * n / MIB == g["mib"]["K4V8_codes"]
+    assert round(1 - g["mib"]["K4V8_codes"] / g["mib"]["fp16"], 2) in (0.62, 0.63)
