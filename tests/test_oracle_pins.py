@@ -409,3 +409,16 @@ def test_ondevice_mib_k4v8_codes():
     codes_only = with_scales - 2 * H * 2          # one fp16 scale per head per tensor
     assert codes_only * n / MIB == g["mib"]["K4V8_codes"]
     assert round(1 - g["mib"]["K4V8_codes"] / g["mib"]["fp16"], 2) in (0.62, 0.63)
+
+
+def test_h_reconstruct_rounds_operand_to_bf16():
+    # the GEMM operand is bf16(h^): pinned against torch's bfloat16 conversion
+    h, Wb, W = _h_setup(n_tok=32, D=512, N=128, seed=32)
+    codes, scales = oracle.quantize_rows(h.astype(np.float32), 128, 4)
+    hd = oracle.dequantize_rows(codes, scales, 512, 128, 4)
+    hb = torch.from_numpy(hd).float().to(torch.bfloat16).double().numpy()
+    assert not np.array_equal(hb, hd)
+    y64, y16 = oracle.h_reconstruct(codes, scales, 512, 4, 4, Wb, round_bf16=True)
+    ref = hb @ W.T
+    np.testing.assert_allclose(y64, ref, rtol=1e-13, atol=1e-13)
+    assert np.array_equal(y16, ref.astype(np.float16).view(np.uint16))
