@@ -1,0 +1,492 @@
+#!/usr/bin/env python
+"""Decode-step benchmark of the quantised-KV decode-attention path on B200.
+
+Workload (default): B=16, 32 layers, 32 query / 8 KV heads, head_dim 128,
+8K context (8191 cached + 1 appended per step), per-(token, head) fp16 scales.
+One step = for every layer: quantize-on-append of the new token's K and V,
+split-KV decode attention, merge of the partials -- captured in one CUDA graph.
+The headline variant is K8V8; K8V4 and K4V4 are reported under "variants".
+
+value  = KV bytes read per step (codes + scales of every attended token, all
+         layers and sequences, summed over ranks) / device time per step.
+e2e    = the same metric through the public API (eager C-ABI calls) with the
+         step's inputs copied from pinned host memory and the outputs copied
+         back inside the timed region.
+roofline = the decode-attention kernel alone, timed live by CUDA event nodes
+         inside the step graph, against the measured HBM copy bandwidth.
+cpu_baseline = the CPU oracle (fp64 attention) on one layer of one step.
+
+Multi-GPU: replicas only (every rank runs the full workload on its own GPU; no
+data-path collective); launched with torch.distributed.run, max time over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attn KV GB/s (% of HBM peak) and steps/s at 8K ctx, K8V8/K8V4/K4V4"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+VARIANTS = {"K8V8": (8, 8, 128, 128), "K8V4": (8, 4, 128, 128), "K4V4": (4, 4, 128, 128)}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def reduce_max(x: float, world: int, device=None) -> float:
+    """Max of a scalar over ranks (identity without a process group)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(x: float, world: int, device=None) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms during a region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def build_variant(w, fmt, device):
+    import torch
+    import quantized_kv_cache_22_b200 as kvq
+    from quantized_kv_cache_22_b200 import Config, LayerCache, Workspace, inputs
+
+    kb, vb, kg, vg = fmt
+    cfg = Config(batch=w.batch, capacity=w.capacity, n_q_heads=w.n_q_heads,
+                 n_kv_heads=w.n_kv_heads, head_dim=w.head_dim, k_bits=kb, v_bits=vb,
+                 k_group=kg, v_group=vg, n_layers=w.n_layers)
+    L = w.context
+    caches = []
+    pos0 = torch.zeros(w.batch, dtype=torch.int32, device=device)
+    for layer in range(w.n_layers):
+        c = LayerCache(cfg, device)
+        k, v = inputs.kv_tokens(w, layer, L - 1, device)
+        kvq.kvq_append(cfg, c, k, v, pos0, 0, L - 1)
+        del k, v
+        caches.append(c)
+    torch.cuda.synchronize(device)
+    st = {"cfg": cfg, "caches": caches,
+          "d_pos": torch.full((w.batch,), L - 1, dtype=torch.int32, device=device),
+          "d_len": torch.full((w.batch,), L, dtype=torch.int32, device=device),
+          "ws": Workspace(cfg, 0, device)}
+    knew, vnew, qs = [], [], []
+    for layer in range(w.n_layers):
+        k1, v1 = inputs.kv_tokens(w, layer, 1, device, offset_seed=1)
+        knew.append(k1)
+        vnew.append(v1)
+        qs.append(inputs.queries(w, layer, 0, device))
+    st["k_new"] = torch.stack(knew)
+    st["v_new"] = torch.stack(vnew)
+    st["q"] = torch.stack(qs)
+    st["out"] = torch.empty_like(st["q"])
+    return st
+
+
+def capture_step(w, st):
+    import torch
+    import quantized_kv_cache_22_b200 as kvq
+    cfg, L = st["cfg"], w.context
+    ev_s = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(w.n_layers)]
+    ev_e = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(w.n_layers)]
+
+    def step(timed_events: bool):
+        for layer in range(w.n_layers):
+            kvq.kvq_append(cfg, st["caches"][layer], st["k_new"][layer], st["v_new"][layer],
+                           st["d_pos"], L - 1, 1)
+            if timed_events:
+                ev_s[layer].record()
+            kvq.kvq_decode_partials(cfg, st["caches"][layer], st["q"][layer], st["d_len"], L,
+                                    st["ws"])
+            if timed_events:
+                ev_e[layer].record()
+            kvq.kvq_merge_partials(cfg, st["d_len"], st["out"][layer], st["ws"])
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step(False)   # warm the host-side memos outside capture
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step(True)
+    torch.cuda.synchronize()
+    return g, ev_s, ev_e, step
+
+
+def time_graph(g, steps, warmup, world, device, sampler=None):
+    import torch
+    import torch.distributed as dist
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    if sampler:
+        sampler.start()
+        time.sleep(0.25)
+    a.record()
+    for _ in range(steps):
+        g.replay()
+    b.record()
+    b.synchronize()
+    clocks = sampler.stop() if sampler else None
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = a.elapsed_time(b) / steps
+    return reduce_max(ms, world, device), clocks
+
+
+def time_e2e(w, st, steps, warmup, world, device):
+    """Public-API step with host buffers: H2D inputs, eager ABI calls, D2H outputs."""
+    import torch
+    import torch.distributed as dist
+    import quantized_kv_cache_22_b200 as kvq
+    cfg, L = st["cfg"], w.context
+    h_q = st["q"].cpu().pin_memory()
+    h_k = st["k_new"].cpu().pin_memory()
+    h_v = st["v_new"].cpu().pin_memory()
+    h_out = torch.empty(st["out"].shape, dtype=st["out"].dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v))
+    d2h = h_out.numel() * h_out.element_size()
+
+    def one():
+        st["q"].copy_(h_q, non_blocking=True)
+        st["k_new"].copy_(h_k, non_blocking=True)
+        st["v_new"].copy_(h_v, non_blocking=True)
+        for layer in range(w.n_layers):
+            kvq.kvq_append(cfg, st["caches"][layer], st["k_new"][layer], st["v_new"][layer],
+                           st["d_pos"], L - 1, 1)
+            kvq.kvq_decode_attn(cfg, st["caches"][layer], st["q"][layer], st["d_len"], L,
+                                st["out"][layer], st["ws"])
+        h_out.copy_(st["out"], non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        one()
+    b.record()
+    b.synchronize()
+    ms = reduce_max(a.elapsed_time(b) / steps, world, device)
+    return ms, h2d, d2h
+
+
+def cpu_oracle_layer(w, fmt, st=None, device=None, reps=1):
+    """Time the oracle on one layer of one decode step: quantize the new token's K/V,
+    then fp64 attention for every (sequence, query head) over the 8K context."""
+    import numpy as np
+    import torch
+    import oracle
+    from quantized_kv_cache_22_b200 import inputs
+
+    kb, vb, kg, vg = fmt
+    L = w.context
+    gen_dev = device if device is not None else "cpu"
+    k, v = inputs.kv_tokens(w, 0, L - 1, gen_dev)
+    k1, v1 = inputs.kv_tokens(w, 0, 1, gen_dev, offset_seed=1)
+    q = inputs.queries(w, 0, 0, gen_dev)
+    kf = k.float().cpu().numpy().transpose(0, 2, 1, 3)
+    vf = v.float().cpu().numpy().transpose(0, 2, 1, 3)
+    del k, v
+    kc = np.zeros((w.batch, w.n_kv_heads, L, w.head_dim * kb // 8), np.uint8)
+    vc = np.zeros((w.batch, w.n_kv_heads, L, w.head_dim * vb // 8), np.uint8)
+    ks = np.zeros((w.batch, w.n_kv_heads, L, w.head_dim // kg), np.uint16)
+    vs = np.zeros((w.batch, w.n_kv_heads, L, w.head_dim // vg), np.uint16)
+    a, b = oracle.quantize_rows(np.ascontiguousarray(kf), kg, kb)
+    kc[:, :, : L - 1], ks[:, :, : L - 1] = a, b
+    a, b = oracle.quantize_rows(np.ascontiguousarray(vf), vg, vb)
+    vc[:, :, : L - 1], vs[:, :, : L - 1] = a, b
+    del kf, vf
+    k1f = np.ascontiguousarray(k1.float().cpu().numpy().transpose(0, 2, 1, 3))
+    v1f = np.ascontiguousarray(v1.float().cpu().numpy().transpose(0, 2, 1, 3))
+    qf = q.float().cpu().numpy()
+    lens = np.full(w.batch, L, np.int32)
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    times = []
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        a, b = oracle.quantize_rows(k1f, kg, kb)
+        kc[:, :, L - 1:], ks[:, :, L - 1:] = a, b
+        a, b = oracle.quantize_rows(v1f, vg, vb)
+        vc[:, :, L - 1:], vs[:, :, L - 1:] = a, b
+        oracle.decode_layer(qf, lens, kc, ks, kb, kg, vc, vs, vb, vg, w.n_kv_heads, 0.0, cores)
+        times.append(time.perf_counter() - t0)
+    return times, cores
+
+
+def run_gpu(args):
+    import torch
+    import quantized_kv_cache_22_b200 as kvq
+    from quantized_kv_cache_22_b200 import inputs
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    w = inputs.WORKLOADS[args.workload]
+    hbm_peak, peak_kind = measured_peaks()
+    uuid = str(torch.cuda.get_device_properties(device).uuid)
+    gpu_id = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+
+    results = {}
+    main_state = None
+    for name in args.variants:
+        fmt = VARIANTS[name]
+        st = build_variant(w, fmt, device)
+        g, ev_s, ev_e, _ = capture_step(w, st)
+        sampler = ClockSampler(gpu_id) if name == args.variants[0] else None
+        ms, clocks = time_graph(g, args.steps, args.warmup, world, device, sampler)
+        dec_ms = statistics.mean(ev_s[i].elapsed_time(ev_e[i]) for i in range(w.n_layers))
+        dec_ms = reduce_max(dec_ms, world, device)
+        per_tok_layer = kvq.kvq_cache_bytes(st["cfg"])[0]
+        kv_bytes_layer = per_tok_layer * w.batch * w.context
+        kv_bytes_step = kv_bytes_layer * w.n_layers
+        results[name] = {
+            "ms_per_step": ms,
+            "steps_per_s": 1e3 / ms,
+            "kv_bytes_per_step": kv_bytes_step,
+            "kv_gbs": world * kv_bytes_step / (ms * 1e-3) / 1e9,
+            "decode_kernel_ms": dec_ms,
+            "decode_kernel_gbs": kv_bytes_layer / (dec_ms * 1e-3) / 1e9,
+            "clocks": clocks,
+        }
+        results[name]["pct_hbm_measured"] = 100.0 * results[name]["decode_kernel_gbs"] / hbm_peak
+        results[name]["pct_hbm_nominal_8tbs"] = 100.0 * results[name]["decode_kernel_gbs"] / NOMINAL_HBM_GBS
+        if name == args.variants[0]:
+            main_state = (st, g)
+            if not args.no_e2e:
+                e2e_steps = max(3, min(args.steps, 50))
+                ems, h2d, d2h = time_e2e(w, st, e2e_steps, max(args.warmup, 3), world, device)
+                results[name]["e2e"] = {"value": world * kv_bytes_step / (ems * 1e-3) / 1e9,
+                                        "unit": "GB/s", "ms_per_step": ems,
+                                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                                        "steps": e2e_steps}
+        else:
+            del g, st
+            torch.cuda.synchronize()
+            torch.cuda.empty_cache()
+
+    head = args.variants[0]
+    r = results[head]
+    line = {
+        "metric": METRIC,
+        "value": round(r["kv_gbs"], 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(r["ms_per_step"], 5),
+        "steps_per_s": round(r["steps_per_s"], 2),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "kv": head, "batch": w.batch, "layers": w.n_layers,
+                   "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
+                   "context": w.context, "scales": "fp16 per (token, head)",
+                   "l2": "inputs larger than L2 (cache >= 4.4 GB per variant)",
+                   "parallelism": f"replicas x{world}", "graph": "one CUDA graph per step"},
+        "pct_hbm_measured": round(r["pct_hbm_measured"], 2),
+        "pct_hbm_nominal_8tbs": round(r["pct_hbm_nominal_8tbs"], 2),
+        "roofline": {"bound": "hbm", "kernel": "decode_kernel (split-KV attention)",
+                     "achieved": round(r["decode_kernel_gbs"], 1), "peak": hbm_peak,
+                     "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": round(r["decode_kernel_gbs"] / hbm_peak, 4),
+                     "traffic": args.traffic_bytes,
+                     "bytes_per_launch": r["kv_bytes_per_step"] // w.n_layers,
+                     "launch_ms": round(r["decode_kernel_ms"], 5)},
+        "variants": {k: {kk: (round(vv, 4) if isinstance(vv, float) else vv)
+                         for kk, vv in v.items() if kk not in ("clocks", "e2e")}
+                     for k, v in results.items()},
+        "gpu_launches": args.steps * 3 * w.n_layers,
+        "clocks": r["clocks"],
+    }
+    if "e2e" in r:
+        line["e2e"] = {k: (round(v, 3) if isinstance(v, float) else v) for k, v in r["e2e"].items()}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        times, cores = cpu_oracle_layer(w, VARIANTS[head], device=device, reps=1)
+        t = min(times)
+        per_layer = r["kv_bytes_per_step"] / w.n_layers
+        line["cpu_baseline"] = {"value": round(per_layer / t / 1e9, 4), "unit": "GB/s",
+                                "steps_per_s": round(1.0 / (t * w.n_layers), 5),
+                                "cores": cores, "kind": "oracle",
+                                "sample": f"1 of {w.n_layers} layers of one {head} step "
+                                          f"(quantize {w.batch}x{w.n_kv_heads} new rows + fp64 "
+                                          f"attention for {w.batch}x{w.n_q_heads} heads over "
+                                          f"{w.context} tokens), {t:.2f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        del main_state
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    """The CPU oracle as it stands, on the same workload and metric (rank 0 only)."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    from quantized_kv_cache_22_b200.inputs import WORKLOADS
+    import quantized_kv_cache_22_b200 as kvq
+    w = WORKLOADS[args.workload]
+    head = args.variants[0]
+    fmt = VARIANTS[head]
+    cfg = kvq.Config(batch=w.batch, capacity=w.capacity, n_q_heads=w.n_q_heads,
+                     n_kv_heads=w.n_kv_heads, head_dim=w.head_dim, k_bits=fmt[0], v_bits=fmt[1],
+                     k_group=fmt[2], v_group=fmt[3], n_layers=w.n_layers)
+    per_layer = kvq.kvq_cache_bytes(cfg)[0] * w.batch * w.context
+    times, cores = cpu_oracle_layer(w, fmt, reps=args.warmup + args.steps)
+    t = statistics.mean(times[args.warmup:]) if len(times) > args.warmup else statistics.mean(times)
+    value = per_layer / t / 1e9
+    sample = (f"each step = 1 of {w.n_layers} layers of one {head} decode step (quantize "
+              f"{w.batch}x{w.n_kv_heads} new rows + fp64 attention, {w.batch}x{w.n_q_heads} heads "
+              f"x {w.context} tokens)")
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(t * 1e3 * w.n_layers, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "kv": head, "batch": w.batch, "layers": w.n_layers,
+                       "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
+                       "head_dim": w.head_dim, "context": w.context},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("kvq", "reference"), default="kvq")
+    ap.add_argument("--workload", type=int, default=4)
+    ap.add_argument("--variants", default="K8V8,K8V4,K4V4")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--traffic-bytes", type=float, default=None,
+                    help="dram bytes per decode launch from an ncu capture of this kernel build")
+    args = ap.parse_args()
+    args.variants = [v.strip() for v in args.variants.split(",") if v.strip()]
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,243 @@
+/*
+ * kvq.h -- C ABI of libkvq: quantised KV cache and single-token decode
+ * attention on NVIDIA B200 (sm_100a).
+ *
+ * Scope.  The library implements the hot path the source pages describe:
+ *   - quantize-on-append of keys and values (or of the hidden state h in
+ *     h-mode) into a fixed-capacity cache with INT8 or nibble-packed INT4
+ *     codes and fp16 scales, independent key/value bit-widths;
+ *   - split-KV decode attention that dequantises in registers inside
+ *     q.K^T -> online softmax -> P.V and merges the partials;
+ *   - in h-mode, the K/V reconstruction GEMM K = W_k h, V = W_v h on tensor
+ *     cores, followed by the same decode attention over 16-bit K/V.
+ *
+ * Sources (web pages; cited by title and section):
+ *   [TL]  TinyLoop docs, "KV Cache 模式": the five cache modes table, the
+ *         memory-formula table "記憶體公式", and "運作原理" (how h-mode works).
+ *   [KS]  KVSplit (vi.news.hada.io topic 20969): independent key/value
+ *         precision K8V8/K8V4/K4V8/K4V4 ("Tính năng chính", flags --kvq-key,
+ *         --kvq-val) and the 8K-token memory table.
+ *   [MNI] "kv-cache-int8-35x-speedup-rust-cuda" (mni-ml/framework): KV cache
+ *         keeps past K/V and computes one new K/V per step; INT8 KV.
+ *   [OD]  gyaansetu.com on-device LLM page: INT4 keys with INT8 values.
+ *
+ * Conventions for every call:
+ *   Ownership.  The caller allocates every buffer (cache, inputs, outputs,
+ *     workspace, h-mode scratch) in device memory.  The library never
+ *     allocates or frees memory and keeps no state between calls.
+ *   Alignment.  Every device pointer must be 16-byte aligned.
+ *   Asynchrony.  Calls that take a stream only enqueue work on it and return;
+ *     a device fault shows up at the caller's next synchronisation.
+ *   Errors.  Every call returns KVQ_OK (0) or a negative KVQ_ERR_* status,
+ *     checks its arguments on the host before launching anything, and never
+ *     aborts or throws.  Non-finite input values give unspecified codes.
+ *   Layout.  "Row" below means one token of one KV head: head_dim elements.
+ *     bits 8: head_dim bytes of int8 codes (two's complement).
+ *     bits 4: head_dim/2 bytes; element 2j in the low nibble and 2j+1 in the
+ *             high nibble of byte j, 4-bit two's complement.
+ *     bits 16: head_dim fp16 values, no scales.
+ *     Scales: head_dim/group fp16 values per row.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KVQ_API __attribute__((visibility("default")))
+#else
+#define KVQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (cudaStream_t / CUstream).  NULL is the legacy default stream. */
+typedef struct CUstream_st *kvq_stream_t;
+
+enum kvq_status {
+    KVQ_OK = 0,
+    KVQ_ERR_INVALID_ARG = -1,  /* null pointer, bad size, bad dtype          */
+    KVQ_ERR_UNSUPPORTED = -2,  /* bit-width / group / head-shape combination */
+    KVQ_ERR_CAPACITY = -3,     /* position or length beyond the capacity     */
+    KVQ_ERR_ALIGN = -4,        /* a pointer is not 16-byte aligned           */
+    KVQ_ERR_WORKSPACE = -5,    /* workspace or scratch too small             */
+    KVQ_ERR_LAUNCH = -6,       /* the CUDA launch itself failed              */
+    KVQ_ERR_DEVICE = -7,       /* no usable sm_100 device / attribute query  */
+    KVQ_ERR_TIMEOUT = -8       /* a kernel gave up a bounded wait (see
+                                  kvq_workspace_status)                       */
+};
+
+enum kvq_mode {
+    KVQ_MODE_KV = 0,  /* the cache stores quantised K and V                  */
+    KVQ_MODE_H = 1    /* the cache stores quantised h = LN(residual) [TL]    */
+};
+
+enum kvq_dtype {
+    KVQ_F16 = 0,
+    KVQ_F32 = 1,
+    KVQ_BF16 = 2
+};
+
+/* Shape and format of a cache.  [TL] "記憶體公式": a cache has a capacity
+ * max_seq_len fixed at creation and n_layers cached-attention layers; the
+ * mode is chosen before use.  [KS]: key and value bit-widths are independent. */
+typedef struct kvq_config {
+    int32_t mode;        /* KVQ_MODE_KV or KVQ_MODE_H                             */
+    int32_t batch;       /* sequences B                                           */
+    int32_t capacity;    /* tokens per sequence; a multiple of 16                 */
+    int32_t n_layers;    /* used by kvq_cache_bytes only                          */
+    int32_t n_q_heads;   /* Hq                                                    */
+    int32_t n_kv_heads;  /* Hkv; Hq is a multiple of Hkv, G = Hq/Hkv              */
+    int32_t head_dim;    /* Dh: 64 or 128                                         */
+    int32_t k_bits;      /* KV mode: 4, 8 or 16                                   */
+    int32_t v_bits;      /* KV mode: 4, 8 or 16                                   */
+    int32_t k_group;     /* elements per key scale: 32, 64 or 128, dividing Dh;
+                            == Dh means one scale per (token, head)               */
+    int32_t v_group;     /* same for values                                       */
+    int32_t d_model;     /* h-mode: D = n_kv_heads * head_dim                     */
+    int32_t h_bits;      /* h-mode: 4, 8 or 16                                    */
+    int32_t h_groups;    /* h-mode: fp16 scales per token (the "per-head" scales
+                            of [TL]); D / h_groups must be 32, 64 or 128          */
+} kvq_config;
+
+/* One layer's cache buffers (device pointers, caller-owned).
+ * KV mode:  k_codes  [B][Hkv][capacity][Dh*k_bits/8] bytes
+ *           k_scales [B][Hkv][capacity][Dh/k_group] fp16   (NULL at 16 bits)
+ *           v_codes / v_scales likewise with v_bits, v_group.
+ * h-mode:   k_codes  [B][capacity][D*h_bits/8] bytes  (the h codes)
+ *           k_scales [B][capacity][h_groups] fp16      (NULL at 16 bits)
+ *           v_codes = v_scales = NULL. */
+typedef struct kvq_layer {
+    void *k_codes;
+    void *k_scales;
+    void *v_codes;
+    void *v_scales;
+} kvq_layer;
+
+/* Cache size.  [TL] "記憶體公式": bytes per token per layer are, at
+ * D = 2048 and 16 heads, 8192 (FP16 KV), 4160 (INT8 KV), 4096 (FP16 h),
+ * 2080 (INT8 h), 1056 (INT4 h); the whole cache costs that times
+ * n_layers * max_seq_len.  Generalised here to separate K/V widths and
+ * scale groups ([KS] 8K-token table):
+ *   KV mode: sum over K and V of Hkv*Dh*bits/8 + Hkv*(Dh/group)*2 (no scale
+ *            term at 16 bits);   h-mode: D*h_bits/8 + h_groups*2 (none at 16).
+ * Outputs (any may be NULL): bytes per token per layer, per layer
+ * (x batch x capacity) and total (x n_layers).  Pure host function: no GPU
+ * needed.  Errors: KVQ_ERR_INVALID_ARG / KVQ_ERR_UNSUPPORTED for a bad config. */
+KVQ_API int kvq_cache_bytes(const kvq_config *cfg, uint64_t *per_token_layer, uint64_t *per_layer,
+                    uint64_t *total);
+
+/* Sizes of the four buffers of one layer in bytes (any output may be NULL;
+ * an unused buffer reports 0).  Pure host function. */
+KVQ_API int kvq_layer_buffer_bytes(const kvq_config *cfg, uint64_t *k_codes, uint64_t *k_scales,
+                           uint64_t *v_codes, uint64_t *v_scales);
+
+/* Quantize-on-append.  [MNI] "Cách KV cache tạo ra tốc độ": each step computes
+ * only the new tokens' K and V and keeps the old ones; [TL] mode table: INT8
+ * codes with one fp16 scale per head, INT4 nibble-packed ("255" vs "15"
+ * symmetric levels); [KS]/[OD]: keys and values at their own widths.
+ *
+ * For every sequence b, new token j < n_new and KV head, each group of
+ * `group` elements x is quantised as
+ *   s = fp16_rne(max|x| / qmax)   (IEEE fp32 division; qmax 127 or 7;
+ *                                  +inf saturates to 65504)
+ *   code = clamp(rne(x / s), -qmax, qmax)   (IEEE fp32 division; 0 if s == 0)
+ * and stored at position d_pos[b] + j.  At 16 bits the value is stored as
+ * fp16 (round to nearest even).
+ *   k, v     device, [B][n_new][Hkv][Dh] in in_dtype (h-mode: k = h,
+ *            [B][n_new][D], and v must be NULL)
+ *   in_dtype KVQ_F16, KVQ_F32 or KVQ_BF16
+ *   d_pos    device int32 [B]: first position written for each sequence
+ *   max_pos_host  host-side upper bound of d_pos[]: the call fails with
+ *            KVQ_ERR_CAPACITY if max_pos_host + n_new > capacity.  Rows whose
+ *            device position still falls outside [0, capacity) are skipped.
+ *   n_new    tokens per sequence (0 is a no-op).
+ * Errors: INVALID_ARG, UNSUPPORTED, CAPACITY, ALIGN, LAUNCH. */
+KVQ_API int kvq_append(const kvq_config *cfg, const kvq_layer *layer, const void *k, const void *v,
+               int32_t in_dtype, const int32_t *d_pos, int32_t max_pos_host, int32_t n_new,
+               kvq_stream_t stream);
+
+/* Workspace bytes kvq_decode_attn needs for this config (KV mode, or the
+ * attention half of h-mode) when launched with `num_ctas` persistent CTAs
+ * (0 = the library's choice for the current device, which needs a CUDA
+ * device; pass an explicit count to size it without one). */
+KVQ_API int kvq_workspace_bytes(const kvq_config *cfg, int32_t num_ctas, uint64_t *bytes);
+
+/* h-mode scratch bytes: reconstructed fp16 K and V for up to max_len
+ * tokens of every sequence ([2][B][Hkv][round_up(max_len,64)][Dh]). */
+KVQ_API int kvq_h_scratch_bytes(const kvq_config *cfg, int32_t max_len, uint64_t *bytes);
+
+/* Decode attention for one query token per sequence (split-KV, dequantised in
+ * registers).  [MNI]: the new token's query attends over every cached K/V;
+ * [KS] "…tích hợp trực tiếp vào kiến trúc FlashAttention": dequantise inside
+ * the attention kernel.  Computes, for query head h (KV head h / G):
+ *   s_t = softmax_scale * q . k^_t,  p = softmax(s) over t < d_len[b],
+ *   out = sum_t p_t v^_t,   k^ = code * scale (exact), v^ likewise,
+ * with fp32 accumulation, then rounds to out_dtype.  A sequence with length
+ * 0 gets zeros.  The token just appended is included (no mask).
+ *   q        device [B][Hq][Dh], q_dtype KVQ_F16, KVQ_F32 or KVQ_BF16
+ *            (f32/bf16 queries need G <= 4; f16 queries G <= 8)
+ *   d_len    device int32 [B]: tokens attended per sequence (clamped to
+ *            [0, capacity] on the device)
+ *   max_len_host  host bound of d_len[] (<= capacity; used for h-mode scratch)
+ *   softmax_scale  0 selects 1/sqrt(Dh)
+ *   out      device [B][Hq][Dh], out_dtype KVQ_F16 or KVQ_F32
+ *   workspace/workspace_bytes  device scratch for split partials, at least
+ *            kvq_workspace_bytes(cfg, num_ctas); need not be initialised
+ *   num_ctas persistent CTAs (0 = library's choice)
+ *   h-mode only: w_kv device bf16 [2*Hkv*Dh][D] (rows of W_k then W_v;
+ *            [TL] "運作原理": rebuild K = W_k h, V = W_v h at every attention
+ *            call, skipping the Q slice), kv_scratch/kv_scratch_bytes at least
+ *            kvq_h_scratch_bytes(cfg, max_len_host).  KV mode: pass NULL / 0.
+ * Errors: INVALID_ARG, UNSUPPORTED, CAPACITY, ALIGN, WORKSPACE, LAUNCH, DEVICE. */
+KVQ_API int kvq_decode_attn(const kvq_config *cfg, const kvq_layer *layer, const void *q, int32_t q_dtype,
+                    const int32_t *d_len, int32_t max_len_host, float softmax_scale, void *out,
+                    int32_t out_dtype, void *workspace, uint64_t workspace_bytes, int32_t num_ctas,
+                    const void *w_kv, void *kv_scratch, uint64_t kv_scratch_bytes,
+                    kvq_stream_t stream);
+
+/* The two halves of kvq_decode_attn in KV mode, for callers that schedule
+ * them separately (e.g. to time the attention kernel alone, or to gather the
+ * partials of several devices before merging).
+ * kvq_decode_partials: the split-KV attention kernel; writes one (m, l, o)
+ *   partial per (CTA, sequence, KV head) segment into `workspace` (arguments
+ *   as kvq_decode_attn).  The partials are unnormalised: o = sum_t p_t v^_t
+ *   and l = sum_t p_t with p_t = 2^(s_t log2(e) - m).
+ * kvq_merge_partials: combines the partials with log-sum-exp weights,
+ *   out = sum_k o_k 2^(m_k - M) / sum_k l_k 2^(m_k - M), and rounds to
+ *   out_dtype.  cfg, d_len, workspace and num_ctas must be those of the
+ *   kvq_decode_partials call it follows on the same stream.
+ * Errors as kvq_decode_attn; KVQ_ERR_INVALID_ARG in h-mode. */
+KVQ_API int kvq_decode_partials(const kvq_config *cfg, const kvq_layer *layer, const void *q,
+                                int32_t q_dtype, const int32_t *d_len, int32_t max_len_host,
+                                float softmax_scale, void *workspace, uint64_t workspace_bytes,
+                                int32_t num_ctas, kvq_stream_t stream);
+KVQ_API int kvq_merge_partials(const kvq_config *cfg, const int32_t *d_len, void *out,
+                               int32_t out_dtype, void *workspace, uint64_t workspace_bytes,
+                               int32_t num_ctas, kvq_stream_t stream);
+
+/* h-mode K/V reconstruction on its own ([TL] "運作原理"; the page's tensor-core
+ * path replaces the scalar one): for every sequence b and token t < len,
+ *   [K_t | V_t] = W_kv . bf16(h^_t)   (fp32 accumulation, rounded to fp16)
+ * written to k_out / v_out, each [B][Hkv][out_capacity][Dh] fp16, with
+ * len = max_len_host for every sequence.  out_capacity is a multiple of 64
+ * and >= max_len_host.  Errors as kvq_decode_attn. */
+KVQ_API int kvq_h_reconstruct(const kvq_config *cfg, const kvq_layer *layer, const void *w_kv,
+                      int32_t max_len_host, void *k_out, void *v_out, int32_t out_capacity,
+                      kvq_stream_t stream);
+
+/* Read and clear the device status word a decode launch leaves in its
+ * workspace: KVQ_OK, or KVQ_ERR_TIMEOUT if a kernel gave up a bounded wait
+ * (its outputs are then invalid).  Synchronises `stream`. */
+KVQ_API int kvq_workspace_status(void *workspace, int32_t *status, kvq_stream_t stream);
+
+/* Static description of a status code. */
+KVQ_API const char *kvq_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

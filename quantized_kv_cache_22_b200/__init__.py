@@ -1,0 +1,239 @@
+"""Python binding of libkvq (quantised KV cache + decode attention on B200).
+
+Argument marshalling only: every step of the path runs in the CUDA kernels of
+``libkvq.so``; PyTorch tensors only provide device memory and streams.  The
+functions carry the C ABI's names (``include/kvq.h``) and raise ``KvqError``
+on a non-zero status.  If the shared library is missing the import fails: there
+is no fallback of any kind.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkvq.so")
+
+KVQ_OK = 0
+KVQ_MODE_KV, KVQ_MODE_H = 0, 1
+KVQ_F16, KVQ_F32, KVQ_BF16 = 0, 1, 2
+
+EXPORTED = ("kvq_cache_bytes", "kvq_layer_buffer_bytes", "kvq_append", "kvq_workspace_bytes",
+            "kvq_h_scratch_bytes", "kvq_decode_attn", "kvq_decode_partials", "kvq_merge_partials",
+            "kvq_h_reconstruct", "kvq_workspace_status", "kvq_status_string")
+
+
+class KvqError(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__(f"{fn} failed: {status} ({status_string(status)})")
+
+
+class KvqConfig(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "mode", "batch", "capacity", "n_layers", "n_q_heads", "n_kv_heads", "head_dim",
+        "k_bits", "v_bits", "k_group", "v_group", "d_model", "h_bits", "h_groups")]
+
+
+class KvqLayer(ctypes.Structure):
+    _fields_ = [("k_codes", ctypes.c_void_p), ("k_scales", ctypes.c_void_p),
+                ("v_codes", ctypes.c_void_p), ("v_scales", ctypes.c_void_p)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libkvq.so not built ({LIB_PATH}); run quantized_kv_cache_22_b200/build.py")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, i32, u64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint64
+    pu64 = ctypes.POINTER(u64)
+    cfgp = ctypes.POINTER(KvqConfig)
+    layp = ctypes.POINTER(KvqLayer)
+    sig = {
+        "kvq_cache_bytes": [cfgp, pu64, pu64, pu64],
+        "kvq_layer_buffer_bytes": [cfgp, pu64, pu64, pu64, pu64],
+        "kvq_append": [cfgp, layp, P, P, i32, P, i32, i32, P],
+        "kvq_workspace_bytes": [cfgp, i32, pu64],
+        "kvq_h_scratch_bytes": [cfgp, i32, pu64],
+        "kvq_decode_attn": [cfgp, layp, P, i32, P, i32, ctypes.c_float, P, i32, P, u64, i32, P, P,
+                            u64, P],
+        "kvq_decode_partials": [cfgp, layp, P, i32, P, i32, ctypes.c_float, P, u64, i32, P],
+        "kvq_merge_partials": [cfgp, P, P, i32, P, u64, i32, P],
+        "kvq_h_reconstruct": [cfgp, layp, P, i32, P, P, i32, P],
+        "kvq_workspace_status": [P, ctypes.POINTER(i32), P],
+    }
+    for name, args in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = ctypes.c_int
+    lib.kvq_status_string.argtypes = [ctypes.c_int]
+    lib.kvq_status_string.restype = ctypes.c_char_p
+    return lib
+
+
+_lib = _load()
+
+
+def lib():
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return _lib.kvq_status_string(int(status)).decode()
+
+
+def _check(fn, rc):
+    if rc != KVQ_OK:
+        raise KvqError(fn, rc)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    return {torch.float16: KVQ_F16, torch.float32: KVQ_F32, torch.bfloat16: KVQ_BF16}[t.dtype]
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+@dataclass
+class Config:
+    """Python view of ``kvq_config`` (see include/kvq.h for the meaning of each field)."""
+    batch: int
+    capacity: int
+    n_q_heads: int = 0
+    n_kv_heads: int = 0
+    head_dim: int = 128
+    k_bits: int = 8
+    v_bits: int = 8
+    k_group: int = 0
+    v_group: int = 0
+    n_layers: int = 1
+    mode: int = KVQ_MODE_KV
+    d_model: int = 0
+    h_bits: int = 4
+    h_groups: int = 0
+
+    def c(self) -> KvqConfig:
+        return KvqConfig(self.mode, self.batch, self.capacity, self.n_layers, self.n_q_heads,
+                         self.n_kv_heads, self.head_dim, self.k_bits, self.v_bits,
+                         self.k_group or self.head_dim, self.v_group or self.head_dim,
+                         self.d_model, self.h_bits, self.h_groups)
+
+
+# ----------------------------------------------------------------------------- host-only calls
+
+def kvq_cache_bytes(cfg: Config):
+    a, b, c = ctypes.c_uint64(), ctypes.c_uint64(), ctypes.c_uint64()
+    _check("kvq_cache_bytes", _lib.kvq_cache_bytes(ctypes.byref(cfg.c()), ctypes.byref(a),
+                                                   ctypes.byref(b), ctypes.byref(c)))
+    return a.value, b.value, c.value
+
+
+def kvq_layer_buffer_bytes(cfg: Config):
+    v = [ctypes.c_uint64() for _ in range(4)]
+    _check("kvq_layer_buffer_bytes",
+           _lib.kvq_layer_buffer_bytes(ctypes.byref(cfg.c()), *[ctypes.byref(x) for x in v]))
+    return tuple(x.value for x in v)
+
+
+def kvq_workspace_bytes(cfg: Config, num_ctas: int = 0) -> int:
+    v = ctypes.c_uint64()
+    _check("kvq_workspace_bytes", _lib.kvq_workspace_bytes(ctypes.byref(cfg.c()), num_ctas,
+                                                           ctypes.byref(v)))
+    return v.value
+
+
+def kvq_h_scratch_bytes(cfg: Config, max_len: int) -> int:
+    v = ctypes.c_uint64()
+    _check("kvq_h_scratch_bytes", _lib.kvq_h_scratch_bytes(ctypes.byref(cfg.c()), max_len,
+                                                           ctypes.byref(v)))
+    return v.value
+
+
+# ----------------------------------------------------------------------------- device buffers
+
+class LayerCache:
+    """One layer's cache buffers, allocated with torch on `device` (caller-owned memory)."""
+
+    def __init__(self, cfg: Config, device="cuda", zero: bool = False):
+        kc, ks, vc, vs = kvq_layer_buffer_bytes(cfg)
+        alloc = torch.zeros if zero else torch.empty
+        self.k_codes = alloc(max(kc, 16), dtype=torch.uint8, device=device)
+        self.k_scales = alloc(max(ks // 2, 8), dtype=torch.float16, device=device) if ks else None
+        self.v_codes = alloc(max(vc, 16), dtype=torch.uint8, device=device) if vc else None
+        self.v_scales = alloc(max(vs // 2, 8), dtype=torch.float16, device=device) if vs else None
+        self.cfg = cfg
+
+    def c(self) -> KvqLayer:
+        return KvqLayer(*(None if t is None else t.data_ptr()
+                          for t in (self.k_codes, self.k_scales, self.v_codes, self.v_scales)))
+
+
+class Workspace:
+    """Split-KV partials buffer sized by kvq_workspace_bytes (status word zeroed)."""
+
+    def __init__(self, cfg: Config, num_ctas: int = 0, device="cuda"):
+        self.nbytes = kvq_workspace_bytes(cfg, num_ctas)
+        self.buf = torch.zeros(self.nbytes // 4 + 64, dtype=torch.float32, device=device)
+
+
+# ----------------------------------------------------------------------------- device calls
+
+def kvq_append(cfg: Config, layer: LayerCache, k: torch.Tensor, v, d_pos: torch.Tensor,
+               max_pos: int, n_new: int, stream=None):
+    _check("kvq_append", _lib.kvq_append(ctypes.byref(cfg.c()), ctypes.byref(layer.c()), _ptr(k),
+                                         _ptr(v), _dtype_code(k), _ptr(d_pos), int(max_pos),
+                                         int(n_new), _stream(stream)))
+
+
+def kvq_decode_attn(cfg: Config, layer: LayerCache, q: torch.Tensor, d_len: torch.Tensor,
+                    max_len: int, out: torch.Tensor, ws: Workspace, softmax_scale: float = 0.0,
+                    num_ctas: int = 0, w_kv=None, kv_scratch=None, stream=None):
+    scratch_bytes = 0 if kv_scratch is None else kv_scratch.numel() * kv_scratch.element_size()
+    _check("kvq_decode_attn",
+           _lib.kvq_decode_attn(ctypes.byref(cfg.c()), ctypes.byref(layer.c()), _ptr(q),
+                                _dtype_code(q), _ptr(d_len), int(max_len), float(softmax_scale),
+                                _ptr(out), _dtype_code(out), _ptr(ws.buf), ws.nbytes,
+                                int(num_ctas), _ptr(w_kv), _ptr(kv_scratch), scratch_bytes,
+                                _stream(stream)))
+
+
+def kvq_decode_partials(cfg: Config, layer: LayerCache, q: torch.Tensor, d_len: torch.Tensor,
+                        max_len: int, ws: Workspace, softmax_scale: float = 0.0, num_ctas: int = 0,
+                        stream=None):
+    _check("kvq_decode_partials",
+           _lib.kvq_decode_partials(ctypes.byref(cfg.c()), ctypes.byref(layer.c()), _ptr(q),
+                                    _dtype_code(q), _ptr(d_len), int(max_len), float(softmax_scale),
+                                    _ptr(ws.buf), ws.nbytes, int(num_ctas), _stream(stream)))
+
+
+def kvq_merge_partials(cfg: Config, d_len: torch.Tensor, out: torch.Tensor, ws: Workspace,
+                       num_ctas: int = 0, stream=None):
+    _check("kvq_merge_partials",
+           _lib.kvq_merge_partials(ctypes.byref(cfg.c()), _ptr(d_len), _ptr(out), _dtype_code(out),
+                                   _ptr(ws.buf), ws.nbytes, int(num_ctas), _stream(stream)))
+
+
+def kvq_h_reconstruct(cfg: Config, layer: LayerCache, w_kv: torch.Tensor, max_len: int,
+                      k_out: torch.Tensor, v_out: torch.Tensor, out_capacity: int, stream=None):
+    _check("kvq_h_reconstruct",
+           _lib.kvq_h_reconstruct(ctypes.byref(cfg.c()), ctypes.byref(layer.c()), _ptr(w_kv),
+                                  int(max_len), _ptr(k_out), _ptr(v_out), int(out_capacity),
+                                  _stream(stream)))
+
+
+def kvq_workspace_status(ws: Workspace, stream=None) -> int:
+    st = ctypes.c_int32()
+    _check("kvq_workspace_status", _lib.kvq_workspace_status(_ptr(ws.buf), ctypes.byref(st),
+                                                             _stream(stream)))
+    return st.value

@@ -1,0 +1,579 @@
+// kvq_api.cu -- the extern "C" boundary of libkvq: argument validation, TMA
+// descriptor encoding and stream-ordered launches.  No allocation, no state
+// that changes results (the only memos are the driver entry point address and
+// per-device attribute / occupancy queries).
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "kvq_internal.h"
+#include "../../include/kvq.h"
+
+using namespace kvq;
+
+namespace {
+
+constexpr uint64_t kTimeoutNs = 1000000000ull;  // bounded waits give up after ~1 s
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_group(int group, int dim)
+{
+    return (group == 32 || group == 64 || group == 128) && dim % group == 0;
+}
+
+bool valid_bits(int b) { return b == 4 || b == 8 || b == 16; }
+
+int check_cfg(const kvq_config *c)
+{
+    if (!c) return KVQ_ERR_INVALID_ARG;
+    if (c->mode != KVQ_MODE_KV && c->mode != KVQ_MODE_H) return KVQ_ERR_INVALID_ARG;
+    if (c->batch < 1 || c->capacity < 16 || c->n_layers < 0) return KVQ_ERR_INVALID_ARG;
+    if (c->capacity % 16 != 0) return KVQ_ERR_UNSUPPORTED;
+    if (c->mode == KVQ_MODE_KV) {
+        if (c->n_kv_heads < 1 || c->n_q_heads < 1 || c->n_q_heads % c->n_kv_heads != 0)
+            return KVQ_ERR_INVALID_ARG;
+        if (c->head_dim != 64 && c->head_dim != 128) return KVQ_ERR_UNSUPPORTED;
+        if (!valid_bits(c->k_bits) || !valid_bits(c->v_bits)) return KVQ_ERR_UNSUPPORTED;
+        if (c->k_bits != 16 && !valid_group(c->k_group, c->head_dim)) return KVQ_ERR_UNSUPPORTED;
+        if (c->v_bits != 16 && !valid_group(c->v_group, c->head_dim)) return KVQ_ERR_UNSUPPORTED;
+    } else {
+        if (c->d_model < 128 || c->d_model % 128 != 0) return KVQ_ERR_UNSUPPORTED;
+        if (!valid_bits(c->h_bits)) return KVQ_ERR_UNSUPPORTED;
+        if (c->h_bits != 16) {
+            if (c->h_groups < 1 || c->d_model % c->h_groups != 0) return KVQ_ERR_UNSUPPORTED;
+            if (!valid_group(c->d_model / c->h_groups, c->d_model)) return KVQ_ERR_UNSUPPORTED;
+        }
+    }
+    return KVQ_OK;
+}
+
+uint64_t tensor_row_bytes(int dim, int bits) { return (uint64_t)dim * bits / 8; }
+
+int scale_groups(int dim, int bits, int group) { return bits == 16 ? 0 : dim / group; }
+
+// ---------------------------------------------------------------- TMA encode
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// Codes of one layer viewed as [bh][cap][R bytes]; a tile of T tokens is one
+// 128-byte-swizzled box (R <= 128: 128/R tokens per 128-byte line) or two
+// 128-byte-wide boxes (R = 256).
+bool encode_codes_map(CUtensorMap *m, const void *codes, int bh, int cap, int R)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3], strides[2];
+    cuuint32_t box[3], estr[3] = {1, 1, 1};
+    if (R <= 128) {
+        dims[0] = 128;
+        dims[1] = (cuuint64_t)cap * R / 128;
+        dims[2] = (cuuint64_t)bh;
+        strides[0] = 128;
+        strides[1] = (cuuint64_t)cap * R;
+        box[0] = 128;
+        box[1] = (cuuint32_t)(kDecodeTileTokens * R / 128);
+        box[2] = 1;
+    } else {
+        dims[0] = (cuuint64_t)R;
+        dims[1] = (cuuint64_t)cap;
+        dims[2] = (cuuint64_t)bh;
+        strides[0] = (cuuint64_t)R;
+        strides[1] = (cuuint64_t)cap * R;
+        box[0] = 128;
+        box[1] = kDecodeTileTokens;
+        box[2] = 1;
+    }
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(codes), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int current_device_props(int *sms, int *max_smem)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return KVQ_ERR_DEVICE;
+    // memo of the three attributes per device (they never change)
+    static std::mutex mu;
+    static int memo[64][3];
+    static bool have[64];
+    if (dev >= 0 && dev < 64) {
+        std::lock_guard<std::mutex> lk(mu);
+        if (have[dev]) {
+            if (memo[dev][0] != 10) return KVQ_ERR_DEVICE;
+            *sms = memo[dev][1];
+            *max_smem = memo[dev][2];
+            return KVQ_OK;
+        }
+    }
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+        return KVQ_ERR_DEVICE;
+    if (major != 10) return KVQ_ERR_DEVICE;  // sm_100a kernels only
+    if (cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return KVQ_ERR_DEVICE;
+    if (cudaDeviceGetAttribute(max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+        cudaSuccess)
+        return KVQ_ERR_DEVICE;
+    if (dev >= 0 && dev < 64) {
+        std::lock_guard<std::mutex> lk(mu);
+        memo[dev][0] = major;
+        memo[dev][1] = *sms;
+        memo[dev][2] = *max_smem;
+        have[dev] = true;
+    }
+    return KVQ_OK;
+}
+
+// Shapes of the attention half (KV mode, or h-mode after reconstruction).
+struct AttnShape {
+    int hkv, hq, G, dh, kb, vb, kg, vg, ngs_k, ngs_v;
+};
+
+AttnShape attn_shape(const kvq_config *c)
+{
+    AttnShape s{};
+    s.hkv = c->n_kv_heads;
+    s.hq = c->n_q_heads;
+    s.G = s.hq / s.hkv;
+    s.dh = c->head_dim;
+    if (c->mode == KVQ_MODE_KV) {
+        s.kb = c->k_bits;
+        s.vb = c->v_bits;
+        s.kg = c->k_group;
+        s.vg = c->v_group;
+    } else {
+        s.kb = s.vb = 16;
+        s.kg = s.vg = s.dh;
+    }
+    s.ngs_k = scale_groups(s.dh, s.kb, s.kg);
+    s.ngs_v = scale_groups(s.dh, s.vb, s.vg);
+    return s;
+}
+
+int resolve_plan(const kvq_config *cfg, int32_t num_ctas, DecodeLaunch *plan, int *ctas)
+{
+    const AttnShape a = attn_shape(cfg);
+    if (a.G > 8) return KVQ_ERR_UNSUPPORTED;
+    int sms = 148, max_smem = 232448;
+    if (num_ctas <= 0) {
+        int rc = current_device_props(&sms, &max_smem);
+        if (rc) return rc;
+    }
+    if (!plan_decode(a.dh, a.kb, a.vb, a.ngs_k, a.ngs_v, a.G, max_smem, plan))
+        return KVQ_ERR_UNSUPPORTED;
+    if (num_ctas > 0) {
+        *ctas = num_ctas;
+        return KVQ_OK;
+    }
+    int per_sm = 0;
+    if (decode_occupancy(*plan, &per_sm) != cudaSuccess || per_sm < 1) return KVQ_ERR_DEVICE;
+    *ctas = sms * per_sm;
+    return KVQ_OK;
+}
+
+uint64_t workspace_need(const kvq_config *cfg, int ctas)
+{
+    const AttnShape a = attn_shape(cfg);
+    return (uint64_t)kWorkspaceHeaderFloats * 4 +
+           slot_count(ctas, cfg->batch, a.hkv) * slot_floats(a.G, a.dh) * 4;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *kvq_status_string(int status)
+{
+    switch (status) {
+    case KVQ_OK: return "ok";
+    case KVQ_ERR_INVALID_ARG: return "invalid argument";
+    case KVQ_ERR_UNSUPPORTED: return "unsupported bit-width, group or head shape";
+    case KVQ_ERR_CAPACITY: return "position or length beyond the cache capacity";
+    case KVQ_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case KVQ_ERR_WORKSPACE: return "workspace or scratch too small";
+    case KVQ_ERR_LAUNCH: return "CUDA launch failed";
+    case KVQ_ERR_DEVICE: return "no usable sm_100 CUDA device";
+    case KVQ_ERR_TIMEOUT: return "a kernel gave up a bounded wait";
+    default: return "unknown status";
+    }
+}
+
+int kvq_cache_bytes(const kvq_config *cfg, uint64_t *per_token_layer, uint64_t *per_layer,
+                    uint64_t *total)
+{
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    uint64_t b = 0;
+    if (cfg->mode == KVQ_MODE_KV) {
+        const int bits[2] = {cfg->k_bits, cfg->v_bits};
+        const int grp[2] = {cfg->k_group, cfg->v_group};
+        for (int i = 0; i < 2; i++) {
+            b += (uint64_t)cfg->n_kv_heads * tensor_row_bytes(cfg->head_dim, bits[i]);
+            b += (uint64_t)cfg->n_kv_heads * scale_groups(cfg->head_dim, bits[i], grp[i]) * 2;
+        }
+    } else {
+        b = tensor_row_bytes(cfg->d_model, cfg->h_bits);
+        if (cfg->h_bits != 16) b += (uint64_t)cfg->h_groups * 2;
+    }
+    const uint64_t layer = b * (uint64_t)cfg->batch * (uint64_t)cfg->capacity;
+    if (per_token_layer) *per_token_layer = b;
+    if (per_layer) *per_layer = layer;
+    if (total) *total = layer * (uint64_t)cfg->n_layers;
+    return KVQ_OK;
+}
+
+int kvq_layer_buffer_bytes(const kvq_config *cfg, uint64_t *k_codes, uint64_t *k_scales,
+                           uint64_t *v_codes, uint64_t *v_scales)
+{
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    const uint64_t rows = (uint64_t)cfg->batch * cfg->capacity;
+    uint64_t kc, ks, vc = 0, vs = 0;
+    if (cfg->mode == KVQ_MODE_KV) {
+        const uint64_t hr = rows * cfg->n_kv_heads;
+        kc = hr * tensor_row_bytes(cfg->head_dim, cfg->k_bits);
+        ks = hr * scale_groups(cfg->head_dim, cfg->k_bits, cfg->k_group) * 2;
+        vc = hr * tensor_row_bytes(cfg->head_dim, cfg->v_bits);
+        vs = hr * scale_groups(cfg->head_dim, cfg->v_bits, cfg->v_group) * 2;
+    } else {
+        kc = rows * tensor_row_bytes(cfg->d_model, cfg->h_bits);
+        ks = cfg->h_bits == 16 ? 0 : rows * (uint64_t)cfg->h_groups * 2;
+    }
+    if (k_codes) *k_codes = kc;
+    if (k_scales) *k_scales = ks;
+    if (v_codes) *v_codes = vc;
+    if (v_scales) *v_scales = vs;
+    return KVQ_OK;
+}
+
+int kvq_append(const kvq_config *cfg, const kvq_layer *layer, const void *k, const void *v,
+               int32_t in_dtype, const int32_t *d_pos, int32_t max_pos_host, int32_t n_new,
+               kvq_stream_t stream)
+{
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (!layer || !d_pos || n_new < 0 || max_pos_host < 0) return KVQ_ERR_INVALID_ARG;
+    if (in_dtype != KVQ_F16 && in_dtype != KVQ_F32 && in_dtype != KVQ_BF16)
+        return KVQ_ERR_INVALID_ARG;
+    if ((int64_t)max_pos_host + n_new > cfg->capacity) return KVQ_ERR_CAPACITY;
+    if (n_new == 0) return KVQ_OK;
+    AppendParams pk{};
+    pk.in_dtype = in_dtype;
+    pk.batch = cfg->batch;
+    pk.n_new = n_new;
+    pk.cap = cfg->capacity;
+    pk.d_pos = d_pos;
+    if (cfg->mode == KVQ_MODE_KV) {
+        if (!k || !v || !layer->k_codes || !layer->v_codes) return KVQ_ERR_INVALID_ARG;
+        if ((cfg->k_bits != 16 && !layer->k_scales) || (cfg->v_bits != 16 && !layer->v_scales))
+            return KVQ_ERR_INVALID_ARG;
+        if (!aligned16(k) || !aligned16(v) || !aligned16(layer->k_codes) ||
+            !aligned16(layer->v_codes) || (layer->k_scales && !aligned16(layer->k_scales)) ||
+            (layer->v_scales && !aligned16(layer->v_scales)))
+            return KVQ_ERR_ALIGN;
+        pk.rows_per_tok = cfg->n_kv_heads;
+        pk.dim = cfg->head_dim;
+        AppendParams pv = pk;
+        pk.x = k;
+        pk.codes = static_cast<uint8_t *>(layer->k_codes);
+        pk.scales = static_cast<__half *>(layer->k_scales);
+        pk.bits = cfg->k_bits;
+        pk.group = cfg->k_bits == 16 ? 32 : cfg->k_group;
+        pv.x = v;
+        pv.codes = static_cast<uint8_t *>(layer->v_codes);
+        pv.scales = static_cast<__half *>(layer->v_scales);
+        pv.bits = cfg->v_bits;
+        pv.group = cfg->v_bits == 16 ? 32 : cfg->v_group;
+        if (launch_append(pk, &pv, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+            return KVQ_ERR_LAUNCH;
+        return KVQ_OK;
+    }
+    if (!k || v || !layer->k_codes) return KVQ_ERR_INVALID_ARG;
+    if (cfg->h_bits != 16 && !layer->k_scales) return KVQ_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(layer->k_codes) ||
+        (layer->k_scales && !aligned16(layer->k_scales)))
+        return KVQ_ERR_ALIGN;
+    pk.rows_per_tok = 1;
+    pk.dim = cfg->d_model;
+    pk.x = k;
+    pk.codes = static_cast<uint8_t *>(layer->k_codes);
+    pk.scales = static_cast<__half *>(layer->k_scales);
+    pk.bits = cfg->h_bits;
+    pk.group = cfg->h_bits == 16 ? 32 : cfg->d_model / cfg->h_groups;
+    if (launch_append(pk, nullptr, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return KVQ_ERR_LAUNCH;
+    return KVQ_OK;
+}
+
+int kvq_workspace_bytes(const kvq_config *cfg, int32_t num_ctas, uint64_t *bytes)
+{
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (!bytes || num_ctas < 0) return KVQ_ERR_INVALID_ARG;
+    if (cfg->mode == KVQ_MODE_H && cfg->n_kv_heads * cfg->head_dim != cfg->d_model)
+        return KVQ_ERR_INVALID_ARG;
+    DecodeLaunch plan;
+    int ctas = 0;
+    rc = resolve_plan(cfg, num_ctas, &plan, &ctas);
+    if (rc) return rc;
+    *bytes = workspace_need(cfg, ctas);
+    return KVQ_OK;
+}
+
+int kvq_h_scratch_bytes(const kvq_config *cfg, int32_t max_len, uint64_t *bytes)
+{
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (cfg->mode != KVQ_MODE_H || !bytes || max_len < 0) return KVQ_ERR_INVALID_ARG;
+    if (max_len > cfg->capacity) return KVQ_ERR_CAPACITY;
+    const uint64_t cap = ((uint64_t)max_len + 63) / 64 * 64;
+    *bytes = 2ull * cfg->batch * cfg->n_kv_heads * cap * cfg->head_dim * 2;
+    return KVQ_OK;
+}
+
+// Validated KV-layout attention: launch the split kernel (do_partials) and/or
+// the merge (do_merge).
+static int decode_kv_layout(const kvq_config *cfg, const void *k_codes, const void *k_scales,
+                            const void *v_codes, const void *v_scales, int cap, const void *q,
+                            int32_t q_dtype, const int32_t *d_len, float softmax_scale, void *out,
+                            int32_t out_dtype, void *workspace, uint64_t workspace_bytes,
+                            int32_t num_ctas, cudaStream_t stream, bool do_partials, bool do_merge)
+{
+    const AttnShape a = attn_shape(cfg);
+    if (q_dtype != KVQ_F16 && a.G > 4) return KVQ_ERR_UNSUPPORTED;
+    DecodeLaunch plan;
+    int ctas = 0;
+    int rc = resolve_plan(cfg, num_ctas, &plan, &ctas);
+    if (rc) return rc;
+    if (workspace_bytes < workspace_need(cfg, ctas)) return KVQ_ERR_WORKSPACE;
+    float *ws = static_cast<float *>(workspace) + kWorkspaceHeaderFloats;
+
+    if (do_partials) {
+        CUtensorMap tm_k, tm_v;
+        const int bh = cfg->batch * a.hkv;
+        if (!encode_codes_map(&tm_k, k_codes, bh, cap, a.dh * a.kb / 8) ||
+            !encode_codes_map(&tm_v, v_codes, bh, cap, a.dh * a.vb / 8))
+            return KVQ_ERR_LAUNCH;
+        DecodeParams p{};
+        p.d_len = d_len;
+        p.q = q;
+        p.k_scales = static_cast<const __half *>(k_scales);
+        p.v_scales = static_cast<const __half *>(v_scales);
+        p.status = static_cast<int *>(workspace);
+        p.ws = ws;
+        p.q_dtype = q_dtype;
+        p.batch = cfg->batch;
+        p.n_q_heads = a.hq;
+        p.n_kv_heads = a.hkv;
+        p.group_size_g = a.G;
+        p.cap = cap;
+        p.ngs_k = a.ngs_k;
+        p.ngs_v = a.ngs_v;
+        p.kshift = a.kb == 16 ? 0 : (a.kg == 32 ? 0 : (a.kg == 64 ? 1 : 2));
+        p.vshift = a.vb == 16 ? 0 : (a.vg == 32 ? 0 : (a.vg == 64 ? 1 : 2));
+        p.num_ctas = ctas;
+        p.stages = plan.stages;
+        p.stage_bytes = plan.stage_bytes;
+        p.off_v = plan.off_v;
+        p.off_sk = plan.off_sk;
+        p.off_sv = plan.off_sv;
+        p.off_meta = plan.off_meta;
+        p.off_bar = plan.off_bar;
+        p.off_merge = plan.off_merge;
+        const float scale = softmax_scale != 0.f ? softmax_scale : 1.f / std::sqrt((float)a.dh);
+        p.tau_log2e = scale * 1.4426950408889634f;
+        p.timeout_ns = kTimeoutNs;
+        if (launch_decode(plan, p, tm_k, tm_v, stream) != cudaSuccess) return KVQ_ERR_LAUNCH;
+    }
+    if (do_merge) {
+        MergeParams mp{};
+        mp.d_len = d_len;
+        mp.ws = ws;
+        mp.out = out;
+        mp.out_f32 = out_dtype == KVQ_F32;
+        mp.batch = cfg->batch;
+        mp.n_q_heads = a.hq;
+        mp.n_kv_heads = a.hkv;
+        mp.group_size_g = a.G;
+        mp.cap = cap;
+        mp.head_dim = a.dh;
+        mp.num_ctas = ctas;
+        if (launch_merge(mp, stream) != cudaSuccess) return KVQ_ERR_LAUNCH;
+    }
+    return KVQ_OK;
+}
+
+static int check_kv_layer(const kvq_config *cfg, const kvq_layer *layer)
+{
+    if (!layer->k_codes || !layer->v_codes) return KVQ_ERR_INVALID_ARG;
+    if ((cfg->k_bits != 16 && !layer->k_scales) || (cfg->v_bits != 16 && !layer->v_scales))
+        return KVQ_ERR_INVALID_ARG;
+    if (!aligned16(layer->k_codes) || !aligned16(layer->v_codes) ||
+        (layer->k_scales && !aligned16(layer->k_scales)) ||
+        (layer->v_scales && !aligned16(layer->v_scales)))
+        return KVQ_ERR_ALIGN;
+    return KVQ_OK;
+}
+
+int kvq_decode_partials(const kvq_config *cfg, const kvq_layer *layer, const void *q,
+                        int32_t q_dtype, const int32_t *d_len, int32_t max_len_host,
+                        float softmax_scale, void *workspace, uint64_t workspace_bytes,
+                        int32_t num_ctas, kvq_stream_t stream)
+{
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (cfg->mode != KVQ_MODE_KV) return KVQ_ERR_INVALID_ARG;
+    if (!layer || !q || !d_len || !workspace || num_ctas < 0) return KVQ_ERR_INVALID_ARG;
+    if (q_dtype != KVQ_F16 && q_dtype != KVQ_F32 && q_dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale) || max_len_host < 0) return KVQ_ERR_INVALID_ARG;
+    if (max_len_host > cfg->capacity) return KVQ_ERR_CAPACITY;
+    if (!aligned16(q) || !aligned16(workspace)) return KVQ_ERR_ALIGN;
+    rc = check_kv_layer(cfg, layer);
+    if (rc) return rc;
+    return decode_kv_layout(cfg, layer->k_codes, layer->k_scales, layer->v_codes, layer->v_scales,
+                            cfg->capacity, q, q_dtype, d_len, softmax_scale, nullptr, KVQ_F32,
+                            workspace, workspace_bytes, num_ctas,
+                            reinterpret_cast<cudaStream_t>(stream), true, false);
+}
+
+int kvq_merge_partials(const kvq_config *cfg, const int32_t *d_len, void *out, int32_t out_dtype,
+                       void *workspace, uint64_t workspace_bytes, int32_t num_ctas,
+                       kvq_stream_t stream)
+{
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (cfg->mode != KVQ_MODE_KV) return KVQ_ERR_INVALID_ARG;
+    if (!d_len || !out || !workspace || num_ctas < 0) return KVQ_ERR_INVALID_ARG;
+    if (out_dtype != KVQ_F16 && out_dtype != KVQ_F32) return KVQ_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(workspace)) return KVQ_ERR_ALIGN;
+    return decode_kv_layout(cfg, nullptr, nullptr, nullptr, nullptr, cfg->capacity, nullptr,
+                            KVQ_F16, d_len, 0.f, out, out_dtype, workspace, workspace_bytes,
+                            num_ctas, reinterpret_cast<cudaStream_t>(stream), false, true);
+}
+
+int kvq_decode_attn(const kvq_config *cfg, const kvq_layer *layer, const void *q, int32_t q_dtype,
+                    const int32_t *d_len, int32_t max_len_host, float softmax_scale, void *out,
+                    int32_t out_dtype, void *workspace, uint64_t workspace_bytes, int32_t num_ctas,
+                    const void *w_kv, void *kv_scratch, uint64_t kv_scratch_bytes,
+                    kvq_stream_t stream)
+{
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (!layer || !q || !d_len || !out || !workspace || num_ctas < 0) return KVQ_ERR_INVALID_ARG;
+    if (q_dtype != KVQ_F16 && q_dtype != KVQ_F32 && q_dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
+    if (out_dtype != KVQ_F16 && out_dtype != KVQ_F32) return KVQ_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale)) return KVQ_ERR_INVALID_ARG;
+    if (max_len_host < 0) return KVQ_ERR_INVALID_ARG;
+    if (max_len_host > cfg->capacity) return KVQ_ERR_CAPACITY;
+    if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return KVQ_ERR_ALIGN;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+    if (cfg->mode == KVQ_MODE_KV) {
+        if (w_kv || kv_scratch || kv_scratch_bytes) return KVQ_ERR_INVALID_ARG;
+        rc = check_kv_layer(cfg, layer);
+        if (rc) return rc;
+        return decode_kv_layout(cfg, layer->k_codes, layer->k_scales, layer->v_codes,
+                                layer->v_scales, cfg->capacity, q, q_dtype, d_len, softmax_scale,
+                                out, out_dtype, workspace, workspace_bytes, num_ctas, st, true,
+                                true);
+    }
+
+    // h-mode: rebuild K, V into the scratch, then attend over 16-bit K/V.
+    if (cfg->n_kv_heads * cfg->head_dim != cfg->d_model) return KVQ_ERR_INVALID_ARG;
+    if (!w_kv || !kv_scratch || !layer->k_codes) return KVQ_ERR_INVALID_ARG;
+    if (!aligned16(w_kv) || !aligned16(kv_scratch)) return KVQ_ERR_ALIGN;
+    if (cfg->head_dim != 128 || cfg->n_q_heads % cfg->n_kv_heads != 0) return KVQ_ERR_UNSUPPORTED;
+    uint64_t need = 0;
+    rc = kvq_h_scratch_bytes(cfg, max_len_host, &need);
+    if (rc) return rc;
+    if (kv_scratch_bytes < need) return KVQ_ERR_WORKSPACE;
+    const int scap = (max_len_host + 63) / 64 * 64;
+    if (scap == 0) {
+        // nothing cached: every output is zero
+        const size_t ob = (size_t)cfg->batch * cfg->n_q_heads * cfg->head_dim *
+                          (out_dtype == KVQ_F32 ? 4 : 2);
+        return cudaMemsetAsync(out, 0, ob, st) == cudaSuccess ? KVQ_OK : KVQ_ERR_LAUNCH;
+    }
+    __half *kout = static_cast<__half *>(kv_scratch);
+    __half *vout = kout + (size_t)cfg->batch * cfg->n_kv_heads * scap * cfg->head_dim;
+    rc = kvq_h_reconstruct(cfg, layer, w_kv, max_len_host, kout, vout, scap, stream);
+    if (rc) return rc;
+    return decode_kv_layout(cfg, kout, nullptr, vout, nullptr, scap, q, q_dtype, d_len,
+                            softmax_scale, out, out_dtype, workspace, workspace_bytes, num_ctas, st,
+                            true, true);
+}
+
+int kvq_h_reconstruct(const kvq_config *cfg, const kvq_layer *layer, const void *w_kv,
+                      int32_t max_len_host, void *k_out, void *v_out, int32_t out_capacity,
+                      kvq_stream_t stream)
+{
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (cfg->mode != KVQ_MODE_H || !layer || !layer->k_codes || !w_kv || !k_out || !v_out)
+        return KVQ_ERR_INVALID_ARG;
+    if (cfg->n_kv_heads * cfg->head_dim != cfg->d_model) return KVQ_ERR_INVALID_ARG;
+    if (cfg->h_bits != 16 && !layer->k_scales) return KVQ_ERR_INVALID_ARG;
+    if (max_len_host < 0 || out_capacity < max_len_host || out_capacity % 64 != 0)
+        return KVQ_ERR_INVALID_ARG;
+    if (max_len_host > cfg->capacity) return KVQ_ERR_CAPACITY;
+    if (!aligned16(layer->k_codes) || !aligned16(w_kv) || !aligned16(k_out) ||
+        !aligned16(v_out) || (layer->k_scales && !aligned16(layer->k_scales)))
+        return KVQ_ERR_ALIGN;
+    if (cfg->head_dim != 128) return KVQ_ERR_UNSUPPORTED;
+    if (max_len_host == 0) return KVQ_OK;
+    HGemmParams p{};
+    p.h_codes = static_cast<const uint8_t *>(layer->k_codes);
+    p.h_scales = static_cast<const __half *>(layer->k_scales);
+    p.w = w_kv;
+    p.k_out = static_cast<__half *>(k_out);
+    p.v_out = static_cast<__half *>(v_out);
+    p.batch = cfg->batch;
+    p.cap = cfg->capacity;
+    p.d_model = cfg->d_model;
+    p.h_bits = cfg->h_bits;
+    p.h_groups = cfg->h_bits == 16 ? 1 : cfg->h_groups;
+    p.n_kv_heads = cfg->n_kv_heads;
+    p.head_dim = cfg->head_dim;
+    p.len = max_len_host;
+    p.out_cap = out_capacity;
+    cudaError_t e = launch_h_reconstruct(p, reinterpret_cast<cudaStream_t>(stream));
+    if (e == cudaErrorNotSupported) return KVQ_ERR_UNSUPPORTED;
+    return e == cudaSuccess ? KVQ_OK : KVQ_ERR_LAUNCH;
+}
+
+int kvq_workspace_status(void *workspace, int32_t *status, kvq_stream_t stream)
+{
+    if (!workspace || !status) return KVQ_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int32_t v = 0;
+    if (cudaMemcpyAsync(&v, workspace, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return KVQ_ERR_LAUNCH;
+    if (cudaMemsetAsync(workspace, 0, 4, st) != cudaSuccess) return KVQ_ERR_LAUNCH;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return KVQ_ERR_LAUNCH;
+    *status = v;
+    return KVQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,88 @@
+// kvq_internal.h -- declarations shared by the libkvq translation units.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+
+namespace kvq {
+
+// ------------------------------------------------------------------ append
+struct AppendParams {
+    const void *x;          // [B][n_new][rows_per_tok][dim] input
+    const int32_t *d_pos;   // [B]
+    uint8_t *codes;         // [B][rows_per_tok][cap][row_bytes]
+    __half *scales;         // [B][rows_per_tok][cap][dim/group] (unused at 16 bits)
+    int32_t in_dtype;       // KVQ_F16 / KVQ_F32 / KVQ_BF16
+    int32_t batch, n_new, rows_per_tok, dim, cap;
+    int32_t bits, group;
+};
+
+cudaError_t launch_append(const AppendParams &k, const AppendParams *v, cudaStream_t stream);
+
+// ------------------------------------------------------------------ decode
+constexpr int kDecodeConsumerWarps = 4;
+constexpr int kDecodeTileTokens = 16 * kDecodeConsumerWarps;   // tokens per stage
+constexpr int kDecodeThreads = 32 * (kDecodeConsumerWarps + 1);
+constexpr int kWorkspaceHeaderFloats = 64;                      // status word + padding
+
+struct DecodeParams {
+    const int32_t *d_len;     // [B]
+    const void *q;            // [B][Hq][Dh]
+    const __half *k_scales;   // [B][Hkv][cap][ngs_k]   (null at 16 bits)
+    const __half *v_scales;
+    float *ws;                // partial slots (after the header)
+    int *status;              // workspace status word
+    int32_t q_dtype;
+    int32_t batch, n_q_heads, n_kv_heads, group_size_g, cap;
+    int32_t ngs_k, ngs_v;     // scales per row
+    int32_t kshift, vshift;   // scale index of 32-element block = blk >> shift
+    int32_t num_ctas;         // persistent CTAs (work split over them)
+    int32_t stages;
+    uint32_t stage_bytes, off_v, off_sk, off_sv, off_meta, off_bar, off_merge;
+    float tau_log2e;
+    uint64_t timeout_ns;
+};
+
+struct MergeParams {
+    const int32_t *d_len;
+    const float *ws;
+    void *out;
+    int32_t out_f32;
+    int32_t batch, n_q_heads, n_kv_heads, group_size_g, cap, head_dim, num_ctas;
+};
+
+// Host helpers implemented in kvq_decode.cu.
+struct DecodeLaunch {
+    int dh, kb, vb;
+    size_t smem_bytes;
+    int stages;
+    uint32_t stage_bytes, off_v, off_sk, off_sv, off_meta, off_bar, off_merge;
+};
+
+// Fill in the shared-memory plan; returns false if the shape is unsupported.
+bool plan_decode(int dh, int kb, int vb, int ngs_k, int ngs_v, int G, int max_smem,
+                 DecodeLaunch *plan);
+cudaError_t decode_occupancy(const DecodeLaunch &plan, int *ctas_per_sm);
+cudaError_t launch_decode(const DecodeLaunch &plan, const DecodeParams &p, const CUtensorMap &tm_k,
+                          const CUtensorMap &tm_v, cudaStream_t stream);
+cudaError_t launch_merge(const MergeParams &p, cudaStream_t stream);
+
+// Floats of one partial slot and slot count for a launch.
+inline uint64_t slot_floats(int G, int dh) { return (uint64_t)G * (uint64_t)(dh + 2); }
+inline uint64_t slot_count(int num_ctas, int batch, int n_kv_heads)
+{
+    return (uint64_t)num_ctas + (uint64_t)batch * (uint64_t)n_kv_heads;
+}
+
+// ------------------------------------------------------------------ h-mode GEMM
+struct HGemmParams {
+    const uint8_t *h_codes;   // [B][cap][D*h_bits/8]
+    const __half *h_scales;   // [B][cap][h_groups]
+    const void *w;            // bf16 [N][D]
+    __half *k_out, *v_out;    // [B][Hkv][out_cap][Dh]
+    int32_t batch, cap, d_model, h_bits, h_groups, n_kv_heads, head_dim, len, out_cap;
+};
+cudaError_t launch_h_reconstruct(const HGemmParams &p, cudaStream_t stream);
+
+}  // namespace kvq

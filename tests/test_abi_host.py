@@ -1,0 +1,133 @@
+"""C-ABI tests that need no GPU: symbols, byte formulas, host-side validation."""
+import ctypes
+import json
+import os
+import re
+
+import pytest
+
+import oracle
+import quantized_kv_cache_22_b200 as kvq
+from quantized_kv_cache_22_b200 import Config, KvqConfig, KvqLayer
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kvq.h")
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"KVQ_API\s+[\w\s\*]*?\b(kvq_\w+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_symbols()
+    assert len(names) >= 9
+    lib = ctypes.CDLL(kvq.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(kvq.EXPORTED)
+
+
+def test_status_strings():
+    assert kvq.status_string(0) == "ok"
+    for rc in range(-8, 0):
+        assert kvq.status_string(rc) != "unknown status"
+
+
+def _mib(x):
+    return x / float(1 << 20)
+
+
+@pytest.mark.parametrize("kb,vb,kg,vg,H,dh", [
+    (8, 8, 128, 128, 16, 128), (16, 16, 0, 0, 16, 128), (8, 4, 128, 32, 8, 128),
+    (4, 8, 32, 128, 8, 128), (4, 4, 32, 32, 4, 64), (8, 8, 64, 64, 4, 64), (4, 16, 64, 0, 2, 128)])
+def test_cache_bytes_matches_oracle(kb, vb, kg, vg, H, dh):
+    cfg = Config(batch=3, capacity=1024, n_q_heads=H, n_kv_heads=H, head_dim=dh, k_bits=kb,
+                 v_bits=vb, k_group=kg, v_group=vg, n_layers=5)
+    per_tok, per_layer, total = kvq.kvq_cache_bytes(cfg)
+    want = oracle.bytes_per_token_layer(0, H, dh, kb, vb, kg or dh, vg or dh)
+    assert per_tok == want
+    assert per_layer == want * 3 * 1024
+    assert total == per_layer * 5
+    kc, ks, vc, vs = kvq.kvq_layer_buffer_bytes(cfg)
+    assert kc + ks + vc + vs == per_layer
+
+
+def test_cache_bytes_tinyloop_figures():
+    g = json.load(open(os.path.join(ROOT, "tests", "golden", "tinyloop_bytes.json")))
+    b = g["bytes_per_token_per_layer"]
+    kv = dict(batch=1, capacity=1024, n_q_heads=16, n_kv_heads=16, head_dim=128, n_layers=34)
+    assert kvq.kvq_cache_bytes(Config(k_bits=16, v_bits=16, **kv))[0] == b["fp16_kv"]
+    int8 = kvq.kvq_cache_bytes(Config(k_bits=8, v_bits=8, **kv))
+    assert int8[0] == b["int8_kv"]
+    assert round(_mib(int8[2])) == g["footprint"]["mib"]["int8_kv"]
+    for name, bits in (("fp16_h", 16), ("int8_h", 8), ("int4_h", 4)):
+        cfg = Config(batch=1, capacity=1024, mode=kvq.KVQ_MODE_H, d_model=2048, h_bits=bits,
+                     h_groups=16, n_q_heads=16, n_kv_heads=16, head_dim=128, n_layers=34)
+        assert kvq.kvq_cache_bytes(cfg)[0] == b[name]
+
+
+def test_cache_bytes_kvsplit_figures():
+    g = json.load(open(os.path.join(ROOT, "tests", "golden", "kvsplit_mib.json")))
+    for name, (kb, vb) in {"K8V8": (8, 8), "K8V4": (8, 4), "K4V4": (4, 4)}.items():
+        cfg = Config(batch=1, capacity=g["tokens"], n_q_heads=32, n_kv_heads=g["n_kv_heads"],
+                     head_dim=g["head_dim"], k_bits=kb, v_bits=vb, k_group=g["group"],
+                     v_group=g["group"], n_layers=g["n_layers"])
+        assert _mib(kvq.kvq_cache_bytes(cfg)[2]) == g["mib"][name]
+
+
+def test_workspace_bytes_explicit_ctas_without_device():
+    cfg = Config(batch=16, capacity=8192, n_q_heads=32, n_kv_heads=8, head_dim=128)
+    a = kvq.kvq_workspace_bytes(cfg, num_ctas=296)
+    b = kvq.kvq_workspace_bytes(cfg, num_ctas=300)
+    # header + (ctas + B*Hkv) slots of G*(Dh+2) floats
+    assert a == 256 + (296 + 128) * 4 * 130 * 4
+    assert b - a == 4 * 4 * 130 * 4
+
+
+def _rc(fn, *args):
+    return getattr(kvq.lib(), fn)(*args)
+
+
+def test_validation_errors_are_returned_on_the_host():
+    good = Config(batch=2, capacity=64, n_q_heads=4, n_kv_heads=2, head_dim=128).c()
+    lay = KvqLayer(16, 16, 32, 48)
+    P = ctypes.c_void_p
+    # bad configs
+    for field, val, want in (("capacity", 40, -2), ("head_dim", 96, -2), ("k_bits", 6, -2),
+                             ("n_q_heads", 3, -1), ("batch", 0, -1), ("k_group", 48, -2),
+                             ("mode", 7, -1)):
+        c = Config(batch=2, capacity=64, n_q_heads=4, n_kv_heads=2, head_dim=128).c()
+        setattr(c, field, val)
+        out = ctypes.c_uint64()
+        assert _rc("kvq_cache_bytes", ctypes.byref(c), ctypes.byref(out), None, None) == want, field
+    # append: capacity overflow, null input, misaligned pointer, bad dtype
+    assert _rc("kvq_append", ctypes.byref(good), ctypes.byref(lay), P(16), P(32), 0, P(64), 60, 8,
+               None) == -3
+    assert _rc("kvq_append", ctypes.byref(good), ctypes.byref(lay), None, P(32), 0, P(64), 0, 1,
+               None) == -1
+    assert _rc("kvq_append", ctypes.byref(good), ctypes.byref(lay), P(17), P(32), 0, P(64), 0, 1,
+               None) == -4
+    assert _rc("kvq_append", ctypes.byref(good), ctypes.byref(lay), P(16), P(32), 9, P(64), 0, 1,
+               None) == -1
+    assert _rc("kvq_append", ctypes.byref(good), ctypes.byref(lay), P(16), P(32), 0, P(64), 0, 0,
+               None) == 0   # zero tokens: nothing to do
+    # decode: length beyond capacity, bad dtype, misaligned out, KV mode with h-mode args
+    args = lambda **kw: [ctypes.byref(good), ctypes.byref(lay), kw.get("q", P(16)), kw.get("qd", 0),
+                         P(64), kw.get("ml", 8), ctypes.c_float(0.0), kw.get("out", P(128)),
+                         kw.get("od", 0), P(256), ctypes.c_uint64(1 << 20), 4, kw.get("w", None),
+                         None, ctypes.c_uint64(0), None]
+    assert _rc("kvq_decode_attn", *args(ml=65)) == -3
+    assert _rc("kvq_decode_attn", *args(qd=5)) == -1
+    assert _rc("kvq_decode_attn", *args(od=2)) == -1
+    assert _rc("kvq_decode_attn", *args(out=P(130))) == -4
+    assert _rc("kvq_decode_attn", *args(w=P(512))) == -1
+    assert _rc("kvq_decode_attn", *args(q=None)) == -1
+    # h-mode reconstruction argument checks
+    hc = Config(batch=1, capacity=64, mode=kvq.KVQ_MODE_H, d_model=256, h_bits=4, h_groups=2,
+                n_q_heads=2, n_kv_heads=2, head_dim=128).c()
+    hl = KvqLayer(16, 32, None, None)
+    assert _rc("kvq_h_reconstruct", ctypes.byref(hc), ctypes.byref(hl), P(64), 65, P(128), P(256),
+               128, None) == -3
+    assert _rc("kvq_h_reconstruct", ctypes.byref(hc), ctypes.byref(hl), P(64), 10, P(128), P(256),
+               100, None) == -1
