@@ -233,6 +233,11 @@ KVQ_API int kvq_h_reconstruct(const kvq_config *cfg, const kvq_layer *layer, con
  * (its outputs are then invalid).  Synchronises `stream`. */
 KVQ_API int kvq_workspace_status(void *workspace, int32_t *status, kvq_stream_t stream);
 
+/* Which step of the last call on this thread that returned KVQ_ERR_LAUNCH
+ * failed, and the CUDA error name ("decode launch: cudaErrorX").  Valid until
+ * the next failing call on the same thread; "" if none. */
+KVQ_API const char *kvq_last_error_detail(void);
+
 /* Static description of a status code. */
 KVQ_API const char *kvq_status_string(int status);
 

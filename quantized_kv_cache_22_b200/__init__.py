@@ -23,13 +23,15 @@ KVQ_F16, KVQ_F32, KVQ_BF16 = 0, 1, 2
 
 EXPORTED = ("kvq_cache_bytes", "kvq_layer_buffer_bytes", "kvq_append", "kvq_workspace_bytes",
             "kvq_h_scratch_bytes", "kvq_decode_attn", "kvq_decode_partials", "kvq_merge_partials",
-            "kvq_h_reconstruct", "kvq_workspace_status", "kvq_status_string")
+            "kvq_h_reconstruct", "kvq_workspace_status", "kvq_status_string",
+            "kvq_last_error_detail")
 
 
 class KvqError(RuntimeError):
     def __init__(self, fn, status):
         self.status = status
-        super().__init__(f"{fn} failed: {status} ({status_string(status)})")
+        detail = _lib.kvq_last_error_detail().decode() if status == -6 else ""
+        super().__init__(f"{fn} failed: {status} ({status_string(status)}) {detail}".rstrip())
 
 
 class KvqConfig(ctypes.Structure):
@@ -70,6 +72,8 @@ def _load():
         f.restype = ctypes.c_int
     lib.kvq_status_string.argtypes = [ctypes.c_int]
     lib.kvq_status_string.restype = ctypes.c_char_p
+    lib.kvq_last_error_detail.argtypes = []
+    lib.kvq_last_error_detail.restype = ctypes.c_char_p
     return lib
 
 

@@ -4,6 +4,7 @@
 // per-device attribute / occupancy queries).
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 #include <cuda.h>
@@ -17,6 +18,15 @@ using namespace kvq;
 namespace {
 
 constexpr uint64_t kTimeoutNs = 1000000000ull;  // bounded waits give up after ~1 s
+
+thread_local char g_detail[160] = "";
+
+// Record which step failed with which CUDA error (read by kvq_last_error_detail).
+int fail(const char *where, cudaError_t e)
+{
+    snprintf(g_detail, sizeof(g_detail), "%s: %s", where, e == cudaSuccess ? "ok" : cudaGetErrorName(e));
+    return KVQ_ERR_LAUNCH;
+}
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -204,6 +214,8 @@ uint64_t workspace_need(const kvq_config *cfg, int ctas)
 
 extern "C" {
 
+const char *kvq_last_error_detail(void) { return g_detail; }
+
 const char *kvq_status_string(int status)
 {
     switch (status) {
@@ -306,9 +318,8 @@ int kvq_append(const kvq_config *cfg, const kvq_layer *layer, const void *k, con
         pv.scales = static_cast<__half *>(layer->v_scales);
         pv.bits = cfg->v_bits;
         pv.group = cfg->v_bits == 16 ? 32 : cfg->v_group;
-        if (launch_append(pk, &pv, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-            return KVQ_ERR_LAUNCH;
-        return KVQ_OK;
+        cudaError_t e = launch_append(pk, &pv, reinterpret_cast<cudaStream_t>(stream));
+        return e == cudaSuccess ? KVQ_OK : fail("append launch", e);
     }
     if (!k || v || !layer->k_codes) return KVQ_ERR_INVALID_ARG;
     if (cfg->h_bits != 16 && !layer->k_scales) return KVQ_ERR_INVALID_ARG;
@@ -322,9 +333,8 @@ int kvq_append(const kvq_config *cfg, const kvq_layer *layer, const void *k, con
     pk.scales = static_cast<__half *>(layer->k_scales);
     pk.bits = cfg->h_bits;
     pk.group = cfg->h_bits == 16 ? 32 : cfg->d_model / cfg->h_groups;
-    if (launch_append(pk, nullptr, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-        return KVQ_ERR_LAUNCH;
-    return KVQ_OK;
+    cudaError_t e = launch_append(pk, nullptr, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KVQ_OK : fail("append launch", e);
 }
 
 int kvq_workspace_bytes(const kvq_config *cfg, int32_t num_ctas, uint64_t *bytes)
@@ -375,7 +385,7 @@ static int decode_kv_layout(const kvq_config *cfg, const void *k_codes, const vo
         const int bh = cfg->batch * a.hkv;
         if (!encode_codes_map(&tm_k, k_codes, bh, cap, a.dh * a.kb / 8) ||
             !encode_codes_map(&tm_v, v_codes, bh, cap, a.dh * a.vb / 8))
-            return KVQ_ERR_LAUNCH;
+            return fail("tensor map encode", cudaErrorInvalidValue);
         DecodeParams p{};
         p.d_len = d_len;
         p.q = q;
@@ -405,7 +415,8 @@ static int decode_kv_layout(const kvq_config *cfg, const void *k_codes, const vo
         const float scale = softmax_scale != 0.f ? softmax_scale : 1.f / std::sqrt((float)a.dh);
         p.tau_log2e = scale * 1.4426950408889634f;
         p.timeout_ns = kTimeoutNs;
-        if (launch_decode(plan, p, tm_k, tm_v, stream) != cudaSuccess) return KVQ_ERR_LAUNCH;
+        cudaError_t e = launch_decode(plan, p, tm_k, tm_v, stream);
+        if (e != cudaSuccess) return fail("decode launch", e);
     }
     if (do_merge) {
         MergeParams mp{};
@@ -420,7 +431,8 @@ static int decode_kv_layout(const kvq_config *cfg, const void *k_codes, const vo
         mp.cap = cap;
         mp.head_dim = a.dh;
         mp.num_ctas = ctas;
-        if (launch_merge(mp, stream) != cudaSuccess) return KVQ_ERR_LAUNCH;
+        cudaError_t e = launch_merge(mp, stream);
+        if (e != cudaSuccess) return fail("merge launch", e);
     }
     return KVQ_OK;
 }
@@ -514,7 +526,8 @@ int kvq_decode_attn(const kvq_config *cfg, const kvq_layer *layer, const void *q
         // nothing cached: every output is zero
         const size_t ob = (size_t)cfg->batch * cfg->n_q_heads * cfg->head_dim *
                           (out_dtype == KVQ_F32 ? 4 : 2);
-        return cudaMemsetAsync(out, 0, ob, st) == cudaSuccess ? KVQ_OK : KVQ_ERR_LAUNCH;
+        cudaError_t e = cudaMemsetAsync(out, 0, ob, st);
+        return e == cudaSuccess ? KVQ_OK : fail("zero output", e);
     }
     __half *kout = static_cast<__half *>(kv_scratch);
     __half *vout = kout + (size_t)cfg->batch * cfg->n_kv_heads * scap * cfg->head_dim;
@@ -560,7 +573,7 @@ int kvq_h_reconstruct(const kvq_config *cfg, const kvq_layer *layer, const void 
     p.out_cap = out_capacity;
     cudaError_t e = launch_h_reconstruct(p, reinterpret_cast<cudaStream_t>(stream));
     if (e == cudaErrorNotSupported) return KVQ_ERR_UNSUPPORTED;
-    return e == cudaSuccess ? KVQ_OK : KVQ_ERR_LAUNCH;
+    return e == cudaSuccess ? KVQ_OK : fail("reconstruction launch", e);
 }
 
 int kvq_workspace_status(void *workspace, int32_t *status, kvq_stream_t stream)
@@ -568,10 +581,12 @@ int kvq_workspace_status(void *workspace, int32_t *status, kvq_stream_t stream)
     if (!workspace || !status) return KVQ_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     int32_t v = 0;
-    if (cudaMemcpyAsync(&v, workspace, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess)
-        return KVQ_ERR_LAUNCH;
-    if (cudaMemsetAsync(workspace, 0, 4, st) != cudaSuccess) return KVQ_ERR_LAUNCH;
-    if (cudaStreamSynchronize(st) != cudaSuccess) return KVQ_ERR_LAUNCH;
+    cudaError_t e = cudaMemcpyAsync(&v, workspace, 4, cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess) return fail("status copy", e);
+    e = cudaMemsetAsync(workspace, 0, 4, st);
+    if (e != cudaSuccess) return fail("status clear", e);
+    e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return fail("status sync", e);
     *status = v;
     return KVQ_OK;
 }

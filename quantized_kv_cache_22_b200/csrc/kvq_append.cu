@@ -125,6 +125,7 @@ cudaError_t launch_append(const AppendParams &k, const AppendParams *v, cudaStre
     AppendPair pp;
     pp.t[0] = k;
     pp.t[1] = v ? *v : k;
+    (void)cudaGetLastError();  // drop a stale, already-reported error of an earlier call
     append_kernel<<<(unsigned)blocks, 256, 0, stream>>>(pp, ntensor);
     return cudaGetLastError();
 }

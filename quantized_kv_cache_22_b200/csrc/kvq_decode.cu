@@ -824,40 +824,59 @@ bool plan_decode(int dh, int kb, int vb, int ngs_k, int ngs_v, int G, int max_sm
     return false;
 }
 
-// Per-device memo of "dynamic shared memory attribute set" and occupancy for a
-// kernel instance and smem size: the queries cost microseconds of host time per
-// call otherwise.  It changes no result.
+// Per-device memos: the dynamic-shared-memory limit of a kernel instance is
+// raised once to the device's opt-in maximum (the attribute is one value per
+// function, so it must never be lowered by a later, smaller plan), and the
+// occupancy of (instance, smem size) is remembered.  Neither changes a result;
+// they only save microseconds of host time per call.
 namespace {
-struct FnMemo {
+struct AttrMemo {
+    int dev;
+    void *fn;
+};
+struct OccMemo {
     int dev;
     void *fn;
     size_t smem;
     int occupancy;
 };
 std::mutex g_memo_mu;
-std::vector<FnMemo> g_memo;
+std::vector<AttrMemo> g_attr;
+std::vector<OccMemo> g_occ;
 
 cudaError_t prepare_fn(void *fn, size_t smem, int *occupancy)
 {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    {
-        std::lock_guard<std::mutex> lk(g_memo_mu);
-        for (const FnMemo &m : g_memo)
-            if (m.dev == dev && m.fn == fn && m.smem == smem) {
-                if (occupancy) *occupancy = m.occupancy;
-                return cudaSuccess;
-            }
+    std::lock_guard<std::mutex> lk(g_memo_mu);
+    bool have_attr = false;
+    for (const AttrMemo &m : g_attr)
+        if (m.dev == dev && m.fn == fn) have_attr = true;
+    if (!have_attr) {
+        int max_optin = 0;
+        e = cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e != cudaSuccess) return e;
+        cudaFuncAttributes fa;
+        e = cudaFuncGetAttributes(&fa, fn);
+        if (e != cudaSuccess) return e;
+        // the opt-in limit covers static + dynamic shared memory
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 max_optin - (int)fa.sharedSizeBytes);
+        if (e != cudaSuccess) return e;
+        g_attr.push_back(AttrMemo{dev, fn});
     }
-    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
+    if (!occupancy) return cudaSuccess;
+    for (const OccMemo &m : g_occ)
+        if (m.dev == dev && m.fn == fn && m.smem == smem) {
+            *occupancy = m.occupancy;
+            return cudaSuccess;
+        }
     int occ = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, NTHR, smem);
     if (e != cudaSuccess) return e;
-    std::lock_guard<std::mutex> lk(g_memo_mu);
-    g_memo.push_back(FnMemo{dev, fn, smem, occ});
-    if (occupancy) *occupancy = occ;
+    g_occ.push_back(OccMemo{dev, fn, smem, occ});
+    *occupancy = occ;
     return cudaSuccess;
 }
 }  // namespace
@@ -883,6 +902,7 @@ cudaError_t launch_merge(const MergeParams &p, cudaStream_t stream)
     const int64_t warps = (int64_t)p.batch * p.n_q_heads;
     if (warps == 0) return cudaSuccess;
     const unsigned blocks = (unsigned)((warps + 7) / 8);
+    (void)cudaGetLastError();  // drop a stale, already-reported error of an earlier call
     if (p.head_dim == 128)
         merge_kernel<128><<<blocks, 256, 0, stream>>>(p);
     else

@@ -135,8 +135,11 @@ def test_decode_split_count_invariance(cuda_device):
         got = gpu_decode(cfg, cache, q, lens, num_ctas=n)
         assert_close_to_oracle(got, want, vmax, G, f"num_ctas={n}")
         outs.append(got)
+    # p * s_V enters the MMA rounded to fp16 relative to the running max, and the
+    # running max depends on where the split boundaries fall: outputs of different
+    # split counts agree to fp16 rounding of the weights, 2^-11 * max|V^|.
     for o in outs[1:]:
-        assert np.abs(o - outs[0]).max() <= 1e-5 * vmax.max()
+        assert np.abs(o - outs[0]).max() <= 2.0 ** -11 * vmax.max()
 
 
 def test_decode_edge_lengths_and_capacity_tail(cuda_device):
@@ -208,11 +211,11 @@ def test_tiny_workload_prompt_then_252_steps(cuda_device):
     oc = oracle_cache(k, v, cfg)
     worst = 0.0
     for step in range(252):
-        L = 4 + step
-        if step > 0:
-            pos.fill_(L - 1)
-            kvq.kvq_append(cfg, cache, k[:, L - 1:L].cuda().contiguous(),
-                           v[:, L - 1:L].cuda().contiguous(), pos, L - 1, 1)
+        # each step appends the newest token (position 4 + step), then attends over all
+        L = 5 + step
+        pos.fill_(L - 1)
+        kvq.kvq_append(cfg, cache, k[:, L - 1:L].cuda().contiguous(),
+                       v[:, L - 1:L].cuda().contiguous(), pos, L - 1, 1)
         q = inputs.queries(w, 0, step)
         d_len = torch.tensor([L], dtype=torch.int32, device="cuda")
         out = torch.empty(1, 4, 64, dtype=torch.float32, device="cuda")
