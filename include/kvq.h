@@ -233,6 +233,36 @@ KVQ_API int kvq_h_reconstruct(const kvq_config *cfg, const kvq_layer *layer, con
  * (its outputs are then invalid).  Synchronises `stream`. */
 KVQ_API int kvq_workspace_status(void *workspace, int32_t *status, kvq_stream_t stream);
 
+/* Bytes of the device array behind kvq_decode_attn_noalloc (2 MiB). */
+#define KVQ_NOALLOC_SCRATCH_BYTES (2u * 1024u * 1024u)
+
+/* kvq_decode_attn (KV mode) for callers that cannot allocate device memory.
+ * The source pages have no counterpart: this is a deployment convenience.
+ * Some callers may not call cudaMalloc at all: code that runs under a host
+ * framework which owns every device allocation, real-time loops that forbid
+ * allocation after start-up because cudaMalloc can stall the device for an
+ * unbounded time, or library code that must not change the process's memory
+ * footprint at run time.  Instead of a caller-provided workspace, this entry
+ * point uses one array of KVQ_NOALLOC_SCRATCH_BYTES in device memory that is
+ * part of libkvq itself; every GPU that loads the library holds it until the
+ * process exits.  The caller still passes the cache, q, d_len and out.
+ *   Set-up: the first call on each device (with that device current) looks up
+ *     the array's device address; make that first call before any stream
+ *     capture.
+ *   Limit: configurations whose kvq_workspace_bytes(cfg, num_ctas) exceeds
+ *     KVQ_NOALLOC_SCRATCH_BYTES are rejected with KVQ_ERR_WORKSPACE before
+ *     anything is launched (for example B=16, Hkv=8, G=4, Dh=128 needs 0.9 MB).
+ *   Sharing: all calls in the process share the one array and it keeps the
+ *     last call's contents; calls that overlap on the GPU (different streams,
+ *     or several host threads) race on it and give wrong results.  Each call
+ *     clears the status word it needs zeroed.
+ * Nothing here allocates or frees memory.  Other arguments and errors as
+ * kvq_decode_attn; h-mode configs return KVQ_ERR_INVALID_ARG. */
+KVQ_API int kvq_decode_attn_noalloc(const kvq_config *cfg, const kvq_layer *layer, const void *q,
+                                    int32_t q_dtype, const int32_t *d_len, int32_t max_len_host,
+                                    float softmax_scale, void *out, int32_t out_dtype,
+                                    int32_t num_ctas, kvq_stream_t stream);
+
 /* Which step of the last call on this thread that returned KVQ_ERR_LAUNCH
  * failed, and the CUDA error name ("decode launch: cudaErrorX").  Valid until
  * the next failing call on the same thread; "" if none. */

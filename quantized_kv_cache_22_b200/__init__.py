@@ -24,7 +24,7 @@ KVQ_F16, KVQ_F32, KVQ_BF16 = 0, 1, 2
 EXPORTED = ("kvq_cache_bytes", "kvq_layer_buffer_bytes", "kvq_append", "kvq_workspace_bytes",
             "kvq_h_scratch_bytes", "kvq_decode_attn", "kvq_decode_partials", "kvq_merge_partials",
             "kvq_h_reconstruct", "kvq_workspace_status", "kvq_status_string",
-            "kvq_last_error_detail")
+            "kvq_last_error_detail", "kvq_decode_attn_noalloc")
 
 
 class KvqError(RuntimeError):
