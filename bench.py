@@ -22,6 +22,7 @@ data-path collective); launched with torch.distributed.run, max time over ranks.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -330,6 +331,8 @@ def run_gpu(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=device)
     w = inputs.WORKLOADS[args.workload]
+    if args.layers:
+        w = dataclasses.replace(w, n_layers=args.layers)
     hbm_peak, peak_kind = measured_peaks()
     uuid = str(torch.cuda.get_device_properties(device).uuid)
     gpu_id = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
@@ -476,6 +479,8 @@ def main():
     ap.add_argument("--variants", default="K8V8,K8V4,K4V4")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="override the layer count (small profiling captures only)")
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="dram bytes per decode launch from an ncu capture of this kernel build")
     args = ap.parse_args()
