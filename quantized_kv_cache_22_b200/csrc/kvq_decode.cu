@@ -60,7 +60,7 @@ struct __align__(16) StageMeta {
 // wrote with 128-byte swizzle.  Rows of R <= 128 bytes are packed 128/R tokens
 // per 128-byte line; R = 256 is stored as two 128-byte-wide boxes.
 template <int R>
-__device__ __forceinline__ uint32_t sw_off(int t, int o)
+__host__ __device__ constexpr uint32_t sw_off(int t, int o)
 {
     if constexpr (R <= 128) {
         constexpr int TPL = 128 / R;
@@ -112,6 +112,51 @@ __device__ __forceinline__ int tiles_of(int len, int cap)
     return (len + T - 1) / T;
 }
 
+// Shared-memory loads at 32-bit shared-window addresses.
+__device__ __forceinline__ uint32_t lds_u16(uint32_t a)
+{
+    uint16_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds_u32(uint32_t a)
+{
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint2 lds_u64(uint32_t a)
+{
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint4 lds_u128(uint32_t a)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(a));
+    return v;
+}
+
+// Address of block `blk` of a row whose block-0 address (stage base + per-lane
+// swizzled offset) is `a0`, for a tile of R-byte rows whose 32-element blocks are
+// STR bytes long: the swizzle is linear in the block index, so block blk sits at
+// a0 ^ sw_off<R>(0, blk*STR).  Rows of 256 bytes keep their second half in a
+// second box T*128 bytes further, which is added rather than XORed because the
+// stage base is only 1024-byte aligned.
+template <int R, int STR>
+__device__ __forceinline__ uint32_t blk_addr(uint32_t a0, int blk)
+{
+    if constexpr (R <= 128) {
+        return a0 ^ sw_off<R>(0, blk * STR);
+    } else {
+        const uint32_t x = sw_off<R>(0, blk * STR);
+        return (a0 ^ (x & (T * 128 - 1))) + (x & ~(uint32_t)(T * 128 - 1));
+    }
+}
+
 template <int DH, int KB, int VB>
 __global__ void __launch_bounds__(NTHR, 2)
     decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -120,8 +165,14 @@ __global__ void __launch_bounds__(NTHR, 2)
     constexpr int NG = DH / 32;                // 32-element blocks along head_dim
     constexpr int RK = DH * KB / 8;            // bytes per key row
     constexpr int RV = DH * VB / 8;
+    constexpr int SK = 32 * KB / 8;            // bytes per 32-element block of a key row
+    constexpr int SV = 32 * VB / 8;
     constexpr float BIAS_K = KB == 8 ? 1152.f : (KB == 4 ? 1032.f : 0.f);
     constexpr float BIAS_V = VB == 8 ? 1152.f : (VB == 4 ? 1032.f : 0.f);
+    // The running max is only raised when a tile beats it by more than 2^LAZY;
+    // weights p * s_V then stay below 2^LAZY, well inside fp16.
+    constexpr float LAZY = 8.f;
+    constexpr unsigned FULL = 0xffffffffu;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -129,7 +180,7 @@ __global__ void __launch_bounds__(NTHR, 2)
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + p.off_bar);
     uint64_t *empty = full + p.stages;
     uint64_t *segbar = empty + p.stages;               // two: [0] partials written, [1] merged
-    int *ctl = reinterpret_cast<int *>(segbar + 2);    // [0] abort, [1] units
+    int *ctl = reinterpret_cast<int *>(segbar + 2);    // [0] abort, [1] units, [2..3] prefix
     float *mbuf = reinterpret_cast<float *>(smem + p.off_merge);
 
     const int tid = threadIdx.x;
@@ -153,11 +204,11 @@ __global__ void __launch_bounds__(NTHR, 2)
 
     // ---- work range of this CTA (computed by the producer warp) -------------
     __shared__ long long sh_u_begin;
-    __shared__ int sh_b, sh_rem;
+    __shared__ int sh_b;
     if (warp == NW) {
         long long total = 0;
         for (int b = lane; b < p.batch; b += 32) total += tiles_of(p.d_len[b], cap);
-        for (int off = 16; off; off >>= 1) total += __shfl_xor_sync(0xffffffffu, total, off);
+        for (int off = 16; off; off >>= 1) total += __shfl_xor_sync(FULL, total, off);
         const long long N = total * p.n_kv_heads;
         const long long P = p.num_ctas;
         const long long ub = (long long)blockIdx.x * N / P;
@@ -168,31 +219,27 @@ __global__ void __launch_bounds__(NTHR, 2)
         long long fpre = 0;
         for (int base = 0; base < p.batch && fb < 0; base += 32) {
             const int b = base + lane;
-            const long long units = (b < p.batch) ? (long long)tiles_of(p.d_len[b], cap) * p.n_kv_heads : 0;
+            const long long units =
+                (b < p.batch) ? (long long)tiles_of(p.d_len[b], cap) * p.n_kv_heads : 0;
             long long incl = units;
             for (int off = 1; off < 32; off <<= 1) {
-                const long long v = __shfl_up_sync(0xffffffffu, incl, off);
+                const long long v = __shfl_up_sync(FULL, incl, off);
                 if (lane >= off) incl += v;
             }
             const long long excl = acc + incl - units;
             const bool hit = units > 0 && excl <= ub && ub < excl + units;
-            const unsigned m = __ballot_sync(0xffffffffu, hit);
+            const unsigned m = __ballot_sync(FULL, hit);
             if (m) {
                 const int src = __ffs(m) - 1;
-                fb = __shfl_sync(0xffffffffu, b, src);
-                fpre = __shfl_sync(0xffffffffu, excl, src);
+                fb = __shfl_sync(FULL, b, src);
+                fpre = __shfl_sync(FULL, excl, src);
             }
-            acc += __shfl_sync(0xffffffffu, incl, 31);
+            acc += __shfl_sync(FULL, incl, 31);
         }
         if (lane == 0) {
             sh_u_begin = ub;
             sh_b = fb;
-            sh_rem = (int)(ue > ub && fb >= 0 ? ue - ub : 0);
-            (void)fpre;
-            ctl[1] = sh_rem;
-        }
-        if (lane == 0) {
-            // stash the prefix of sequence fb for the walk
+            ctl[1] = (int)(ue > ub && fb >= 0 ? ue - ub : 0);
             reinterpret_cast<long long *>(ctl + 2)[0] = fpre;
         }
     }
@@ -206,15 +253,17 @@ __global__ void __launch_bounds__(NTHR, 2)
         prefetch_tensormap(&tm_v);
         int b = sh_b;
         const long long pre = reinterpret_cast<long long *>(ctl + 2)[0];
-        int tiles_b = (b >= 0) ? tiles_of(p.d_len[b], cap) : 0;
-        int off = (int)(sh_u_begin - pre);          // unit offset inside sequence b
+        int len_b = (b >= 0) ? min(max(p.d_len[b], 0), cap) : 0;
+        int tiles_b = (len_b + T - 1) / T;
+        const int off = (int)(sh_u_begin - pre);   // unit offset inside sequence b
         int kvh = tiles_b ? off / tiles_b : 0;
         int tile = tiles_b ? off % tiles_b : 0;
+        int s = 0;
+        uint32_t ph = 0;                            // phase parity of this use of stage s
         int issued = 0;
         for (int i = 0; i < n_units; i++) {
-            const int s = i % S;
             if (i >= S) {
-                if (!mbar_wait_bounded(&empty[s], ((i / S) - 1) & 1, abort_flag, p.timeout_ns)) {
+                if (!mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, p.timeout_ns)) {
                     ctl[0] = 1;
                     atomicExch(p.status, KVQ_ERR_TIMEOUT);
                     break;
@@ -222,13 +271,12 @@ __global__ void __launch_bounds__(NTHR, 2)
             }
             const int bh = b * p.n_kv_heads + kvh;
             const int t0 = tile * T;
-            const int len = min(max(p.d_len[b], 0), cap);
             int flags = 0;
             if (i == 0 || tile == 0) flags |= 1;
             if (i == n_units - 1 || tile == tiles_b - 1) flags |= 2;
             flags |= ((int)blockIdx.x + bh) << 8;
             StageMeta m;
-            m.bh = bh; m.t0 = t0; m.len = len; m.flags = flags;
+            m.bh = bh; m.t0 = t0; m.len = len_b; m.flags = flags;
             meta[s] = m;
 
             uint8_t *st = smem + (size_t)s * p.stage_bytes;
@@ -256,22 +304,34 @@ __global__ void __launch_bounds__(NTHR, 2)
                 bulk_load(st + p.off_sv, p.v_scales + ((int64_t)bh * cap + t0) * p.ngs_v,
                           (uint32_t)(n_s * p.ngs_v * 2), &full[s]);
             issued = i + 1;
-            // advance to the next unit
+            if (++s == S) {
+                s = 0;
+                ph ^= 1u;
+            }
+            // advance to the next unit (the length is re-read only when b changes)
             if (++tile == tiles_b) {
                 tile = 0;
                 if (++kvh == p.n_kv_heads) {
                     kvh = 0;
                     do {
                         ++b;
-                        tiles_b = (b < p.batch) ? tiles_of(p.d_len[b], cap) : 1;
+                        len_b = (b < p.batch) ? min(max(p.d_len[b], 0), cap) : T;
+                        tiles_b = (len_b + T - 1) / T;
                     } while (tiles_b == 0);
                 }
             }
         }
         // never leave with copies in flight: wait for the last issued phases
-        const int first = issued > S ? issued - S : 0;
-        for (int i = first; i < issued; i++)
-            (void)mbar_wait_bounded(&full[i % S], (i / S) & 1, abort_flag, p.timeout_ns);
+        int ss = s;
+        uint32_t pp = ph;
+        for (int j = 0; j < min(S, issued); j++) {
+            if (ss == 0) {
+                ss = S;
+                pp ^= 1u;
+            }
+            --ss;
+            (void)mbar_wait_bounded(&full[ss], pp, abort_flag, p.timeout_ns);
+        }
         return;
     }
 
@@ -281,15 +341,79 @@ __global__ void __launch_bounds__(NTHR, 2)
     const bool qsplit = p.q_dtype != KVQ_F16;
     const bool kgrp = p.ngs_k > 1;
     const bool vgrp = p.ngs_v > 1;
+    const int colmax = qsplit ? 4 : 8;
+    const bool col_ok0 = (2 * tig) < G && (2 * tig) < colmax;
+    const bool col_ok1 = (2 * tig + 1) < G && (2 * tig + 1) < colmax;
+
+    // per-lane swizzled offsets of block 0 of the rows this lane reads (relative
+    // to a stage tile), for the two 16-token sub-tiles of the warp
+    uint32_t kofs[2][2], vofs[2][4];
+#pragma unroll
+    for (int u = 0; u < 2; u++) {
+        const int tw = warp * 32 + u * 16;
+        kofs[u][0] = sw_off<RK>(tw + 2 * gid, tig * (SK / 4));
+        kofs[u][1] = sw_off<RK>(tw + 2 * gid + 1, tig * (SK / 4));
+        const int tv = tw + 2 * tig;
+        vofs[u][0] = p.off_v + sw_off<RV>(tv, gid * (SV / 8));
+        vofs[u][1] = p.off_v + sw_off<RV>(tv + 1, gid * (SV / 8));
+        vofs[u][2] = p.off_v + sw_off<RV>(tv + 8, gid * (SV / 8));
+        vofs[u][3] = p.off_v + sw_off<RV>(tv + 9, gid * (SV / 8));
+    }
+    // source lanes of the P transposition (score layout -> B-fragment layout)
+    const int src0 = tig * 4 + (gid >> 1);
+    const int src1 = (tig + 4) * 4 + (gid >> 1);
+    const bool odd = gid & 1;
 
     uint32_t qb[NG][2][2];              // q B-fragments per (block, k-half)
-    float qsum[NG][2];                  // per block, for score cols 2tig, 2tig+1
+    float qbias[NG][2];                 // BIAS_K * sum(q) per block, score cols 2tig, 2tig+1
     float m_run[2], l_run[2];
-    float psum[NG][2];                  // sum of fp16 p*sV per value block (or [0])
+    float psum[NG][2];                  // sum of fp16 p*s_V per value block (or [0])
     float o_acc[2 * NG][4];             // O^T fragments, m-tile = 2*blk + u
-    int seg_parity = 0;
+    uint32_t seg_parity = 0;
 
-    auto reset_state = [&]() {
+    auto load_q = [&](int bh) {
+        const int b = bh / p.n_kv_heads;
+        const int kvh = bh % p.n_kv_heads;
+        // B-fragment column n = gid: non-split: head n; split: hi (n<4) / lo (n>=4) of head n&3
+        const int head = qsplit ? (gid & 3) : gid;
+        const bool lo_part = qsplit && gid >= 4;
+        const bool valid = head < G;
+        const int64_t qbase = ((int64_t)b * p.n_q_heads + (int64_t)kvh * G + head) * DH;
+#pragma unroll
+        for (int blk = 0; blk < NG; blk++) {
+            float colsum = 0.f;
+#pragma unroll
+            for (int hs = 0; hs < 2; hs++) {
+                __half hv[4];
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    const int d = 32 * blk + 8 * tig + k_elem<KB>(hs, j);
+                    const float x = valid ? load_qf(p.q, p.q_dtype, qbase + d) : 0.f;
+                    __half h = __float2half_rn(x);
+                    if (lo_part) h = __float2half_rn(x - __half2float(h));
+                    hv[j] = h;
+                    colsum += __half2float(h);
+                }
+                __half2 b0 = __halves2half2(hv[0], hv[1]);
+                __half2 b1 = __halves2half2(hv[2], hv[3]);
+                qb[blk][hs][0] = *reinterpret_cast<uint32_t *>(&b0);
+                qb[blk][hs][1] = *reinterpret_cast<uint32_t *>(&b1);
+            }
+            colsum += __shfl_xor_sync(FULL, colsum, 1);
+            colsum += __shfl_xor_sync(FULL, colsum, 2);
+            // score cols of this lane are 2tig and 2tig+1; column n lives on lanes with gid = n
+            qbias[blk][0] = BIAS_K * __shfl_sync(FULL, colsum, (2 * tig) * 4);
+            qbias[blk][1] = BIAS_K * __shfl_sync(FULL, colsum, (2 * tig + 1) * 4);
+        }
+        if (!kgrp) {
+#pragma unroll
+            for (int c = 0; c < 2; c++) {
+                float t = 0.f;
+#pragma unroll
+                for (int blk = 0; blk < NG; blk++) t += qbias[blk][c];
+                qbias[0][c] = t;
+            }
+        }
 #pragma unroll
         for (int c = 0; c < 2; c++) {
             m_run[c] = -INFINITY;
@@ -303,294 +427,261 @@ __global__ void __launch_bounds__(NTHR, 2)
             for (int i = 0; i < 4; i++) o_acc[mt][i] = 0.f;
     };
 
-    auto load_q = [&](int bh) {
-        const int b = bh / p.n_kv_heads;
-        const int kvh = bh % p.n_kv_heads;
-        // B-fragment column n = gid: non-split: head n; split: hi (n<4) / lo (n>=4) of head n&3
-        const int head = qsplit ? (gid & 3) : gid;
-        const bool lo_part = qsplit && gid >= 4;
-        const bool valid = head < G;
-        const int64_t qbase = ((int64_t)b * p.n_q_heads + (int64_t)kvh * G + head) * DH;
-        float colsum[NG];
-#pragma unroll
-        for (int blk = 0; blk < NG; blk++) {
-            colsum[blk] = 0.f;
-#pragma unroll
-            for (int hs = 0; hs < 2; hs++) {
-                __half hv[4];
-#pragma unroll
-                for (int j = 0; j < 4; j++) {
-                    const int d = 32 * blk + 8 * tig + k_elem<KB>(hs, j);
-                    float x = valid ? load_qf(p.q, p.q_dtype, qbase + d) : 0.f;
-                    __half h = __float2half_rn(x);
-                    if (lo_part) h = __float2half_rn(x - __half2float(h));
-                    hv[j] = h;
-                    colsum[blk] += __half2float(h);
-                }
-                __half2 b0 = __halves2half2(hv[0], hv[1]);
-                __half2 b1 = __halves2half2(hv[2], hv[3]);
-                qb[blk][hs][0] = *reinterpret_cast<uint32_t *>(&b0);
-                qb[blk][hs][1] = *reinterpret_cast<uint32_t *>(&b1);
-            }
-            colsum[blk] += __shfl_xor_sync(0xffffffffu, colsum[blk], 1);
-            colsum[blk] += __shfl_xor_sync(0xffffffffu, colsum[blk], 2);
-            // score cols of this lane are 2tig and 2tig+1; column n lives on lanes with gid = n
-            qsum[blk][0] = __shfl_sync(0xffffffffu, colsum[blk], (2 * tig) * 4);
-            qsum[blk][1] = __shfl_sync(0xffffffffu, colsum[blk], (2 * tig + 1) * 4);
+    // A fragments of block blk, k-half hs, for key rows at a[0] (row gid) and a[1] (row gid+8)
+    auto key_frags = [&](uint32_t ra, uint32_t rb, int blk, uint32_t (&fa)[2][4]) {
+        if constexpr (KB == 8) {
+            const uint2 r0 = lds_u64(blk_addr<RK, SK>(ra, blk));
+            const uint2 r1 = lds_u64(blk_addr<RK, SK>(rb, blk));
+            const uint32_t x00 = r0.x ^ 0x80808080u, x01 = r0.y ^ 0x80808080u;
+            const uint32_t x10 = r1.x ^ 0x80808080u, x11 = r1.y ^ 0x80808080u;
+            fa[0][0] = i8_lo_pair(x00); fa[0][2] = i8_hi_pair(x00);
+            fa[0][1] = i8_lo_pair(x10); fa[0][3] = i8_hi_pair(x10);
+            fa[1][0] = i8_lo_pair(x01); fa[1][2] = i8_hi_pair(x01);
+            fa[1][1] = i8_lo_pair(x11); fa[1][3] = i8_hi_pair(x11);
+        } else if constexpr (KB == 4) {
+            const uint32_t r0 = lds_u32(blk_addr<RK, SK>(ra, blk));
+            const uint32_t r1 = lds_u32(blk_addr<RK, SK>(rb, blk));
+            fa[0][0] = i4_pair(r0, 0); fa[0][2] = i4_pair(r0, 1);
+            fa[0][1] = i4_pair(r1, 0); fa[0][3] = i4_pair(r1, 1);
+            fa[1][0] = i4_pair(r0, 2); fa[1][2] = i4_pair(r0, 3);
+            fa[1][1] = i4_pair(r1, 2); fa[1][3] = i4_pair(r1, 3);
+        } else {
+            const uint4 r0 = lds_u128(blk_addr<RK, SK>(ra, blk));
+            const uint4 r1 = lds_u128(blk_addr<RK, SK>(rb, blk));
+            fa[0][0] = r0.x; fa[0][2] = r0.y; fa[0][1] = r1.x; fa[0][3] = r1.y;
+            fa[1][0] = r0.z; fa[1][2] = r0.w; fa[1][1] = r1.z; fa[1][3] = r1.w;
         }
     };
 
     const uint64_t limit = p.timeout_ns;
-    bool ok = true;
+    const uint32_t smem_base = smem_u32(smem);
+    int s = 0;
+    uint32_t ph = 0;
     for (int i = 0; i < n_units; i++) {
-        const int s = i % S;
-        if (!mbar_wait_bounded(&full[s], (i / S) & 1, abort_flag, limit)) {
+        if (!mbar_wait_bounded(&full[s], ph, abort_flag, limit)) {
             ctl[0] = 1;
             atomicExch(p.status, KVQ_ERR_TIMEOUT);
-            ok = false;
             break;
         }
         const StageMeta m = meta[s];
-        if (m.flags & 1) {
-            load_q(m.bh);
-            reset_state();
-        }
-        const uint8_t *st = smem + (size_t)s * p.stage_bytes;
-        const uint8_t *sk = st;
-        const uint8_t *sv = st + p.off_v;
-        const __half *ssk = reinterpret_cast<const __half *>(st + p.off_sk);
-        const __half *ssv = reinterpret_cast<const __half *>(st + p.off_sv);
-        const int tw = warp * 16;                        // first token of this warp in the stage
-        const int tA = tw + 2 * gid;                     // score rows: tokens tA, tA+1
+        if (m.flags & 1) load_q(m.bh);
+        const uint32_t st = smem_base + (uint32_t)s * p.stage_bytes;
+        const __half *ssk = reinterpret_cast<const __half *>(smem + (size_t)s * p.stage_bytes + p.off_sk);
+        const __half *ssv = reinterpret_cast<const __half *>(smem + (size_t)s * p.stage_bytes + p.off_sv);
 
-        // ---------------- scores: S^T = K q^T -------------------------------
-        float acc[NG][4];
 #pragma unroll
-        for (int g = 0; g < NG; g++) acc[g][0] = acc[g][1] = acc[g][2] = acc[g][3] = 0.f;
-#pragma unroll
-        for (int blk = 0; blk < NG; blk++) {
-            uint32_t a[2][4];  // [hs][a0..a3]
-            if constexpr (KB == 8) {
-                const uint2 r0 = *reinterpret_cast<const uint2 *>(sk + sw_off<RK>(tA, 32 * blk + 8 * tig));
-                const uint2 r1 = *reinterpret_cast<const uint2 *>(sk + sw_off<RK>(tA + 1, 32 * blk + 8 * tig));
-                const uint32_t x00 = r0.x ^ 0x80808080u, x01 = r0.y ^ 0x80808080u;
-                const uint32_t x10 = r1.x ^ 0x80808080u, x11 = r1.y ^ 0x80808080u;
-                a[0][0] = i8_lo_pair(x00); a[0][2] = i8_hi_pair(x00);
-                a[0][1] = i8_lo_pair(x10); a[0][3] = i8_hi_pair(x10);
-                a[1][0] = i8_lo_pair(x01); a[1][2] = i8_hi_pair(x01);
-                a[1][1] = i8_lo_pair(x11); a[1][3] = i8_hi_pair(x11);
-            } else if constexpr (KB == 4) {
-                const uint32_t r0 = *reinterpret_cast<const uint32_t *>(sk + sw_off<RK>(tA, 16 * blk + 4 * tig));
-                const uint32_t r1 = *reinterpret_cast<const uint32_t *>(sk + sw_off<RK>(tA + 1, 16 * blk + 4 * tig));
-                a[0][0] = i4_pair(r0, 0); a[0][2] = i4_pair(r0, 1);
-                a[0][1] = i4_pair(r1, 0); a[0][3] = i4_pair(r1, 1);
-                a[1][0] = i4_pair(r0, 2); a[1][2] = i4_pair(r0, 3);
-                a[1][1] = i4_pair(r1, 2); a[1][3] = i4_pair(r1, 3);
-            } else {
-                const uint4 r0 = *reinterpret_cast<const uint4 *>(sk + sw_off<RK>(tA, 64 * blk + 16 * tig));
-                const uint4 r1 = *reinterpret_cast<const uint4 *>(sk + sw_off<RK>(tA + 1, 64 * blk + 16 * tig));
-                a[0][0] = r0.x; a[0][2] = r0.y; a[0][1] = r1.x; a[0][3] = r1.y;
-                a[1][0] = r0.z; a[1][2] = r0.w; a[1][1] = r1.z; a[1][3] = r1.w;
-            }
-#pragma unroll
-            for (int hs = 0; hs < 2; hs++)
-                mma_16816(acc[blk], a[hs][0], a[hs][1], a[hs][2], a[hs][3], qb[blk][hs][0], qb[blk][hs][1]);
-        }
+        for (int u = 0; u < 2; u++) {
+            const int tA = warp * 32 + u * 16 + 2 * gid;       // score rows: tokens tA, tA + 1
+            const bool vt0 = m.t0 + tA < m.len;
+            const bool vt1 = m.t0 + tA + 1 < m.len;
 
-        // score values: idx 0 (tok tA, col 2tig), 1 (tA, 2tig+1), 2 (tA+1, 2tig), 3 (tA+1, 2tig+1)
-        float sc[4];
-        {
-            float sk0[NG], sk1[NG];
-            if (KB == 16) {
+            // ---------------- scores: S^T = K q^T ---------------------------
+            float s2[4];
+            {
+                const uint32_t ra = st + kofs[u][0], rb = st + kofs[u][1];
+                float ks0 = p.tau_log2e, ks1 = p.tau_log2e;
+                if (!kgrp) {
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int g = 0; g < NG; g++) sk0[g] = sk1[g] = 1.f;
-            } else if (!kgrp) {
-                const float2 kk = unpack_half2(*reinterpret_cast<const uint32_t *>(ssk + tA));
+                    for (int blk = 0; blk < NG; blk++) {
+                        uint32_t fa[2][4];
+                        key_frags(ra, rb, blk, fa);
 #pragma unroll
-                for (int g = 0; g < NG; g++) { sk0[g] = kk.x; sk1[g] = kk.y; }
-            } else {
-#pragma unroll
-                for (int g = 0; g < NG; g++) {
-                    sk0[g] = __half2float(ssk[tA * p.ngs_k + (g >> p.kshift)]);
-                    sk1[g] = __half2float(ssk[(tA + 1) * p.ngs_k + (g >> p.kshift)]);
-                }
-            }
-#pragma unroll
-            for (int e = 0; e < 4; e++) {
-                const int c = e & 1;
-                float v = 0.f;
-#pragma unroll
-                for (int g = 0; g < NG; g++) {
-                    const float sc_g = (e < 2) ? sk0[g] : sk1[g];
-                    v = fmaf(sc_g, acc[g][e] - BIAS_K * qsum[g][c], v);
-                }
-                sc[e] = v;
-            }
-            if (qsplit) {
-#pragma unroll
-                for (int e = 0; e < 4; e++) sc[e] += __shfl_xor_sync(0xffffffffu, sc[e], 2);
-            }
-        }
-
-        // ---------------- online softmax ------------------------------------
-        const int tok0 = m.t0 + tA;
-        const bool valid_t0 = tok0 < m.len;
-        const bool valid_t1 = tok0 + 1 < m.len;
-        float sv0[NG], sv1[NG], lsv[2];
-        if (VB == 16) {
-#pragma unroll
-            for (int g = 0; g < NG; g++) sv0[g] = sv1[g] = 1.f;
-        } else if (!vgrp) {
-            const float2 vv = unpack_half2(*reinterpret_cast<const uint32_t *>(ssv + tA));
-#pragma unroll
-            for (int g = 0; g < NG; g++) { sv0[g] = vv.x; sv1[g] = vv.y; }
-        } else {
-#pragma unroll
-            for (int g = 0; g < NG; g++) {
-                sv0[g] = __half2float(ssv[tA * p.ngs_v + (g >> p.vshift)]);
-                sv1[g] = __half2float(ssv[(tA + 1) * p.ngs_v + (g >> p.vshift)]);
-            }
-        }
-        // scales of tokens past the length may be stale shared memory: never use them
-#pragma unroll
-        for (int g = 0; g < NG; g++) {
-            sv0[g] = valid_t0 ? sv0[g] : 0.f;
-            sv1[g] = valid_t1 ? sv1[g] : 0.f;
-        }
-        {
-            float mx0 = 0.f, mx1 = 0.f;
-#pragma unroll
-            for (int g = 0; g < NG; g++) { mx0 = fmaxf(mx0, sv0[g]); mx1 = fmaxf(mx1, sv1[g]); }
-            lsv[0] = mx0 > 0.f ? fmaxf(__log2f(mx0), -32.f) : -32.f;
-            lsv[1] = mx1 > 0.f ? fmaxf(__log2f(mx1), -32.f) : -32.f;
-        }
-        float s2[4];
-        float alpha[2];
-        {
-            const int colmax = qsplit ? 4 : 8;
-#pragma unroll
-            for (int e = 0; e < 4; e++) {
-                const int col = 2 * tig + (e & 1);
-                const bool vt = (e < 2) ? valid_t0 : valid_t1;
-                const bool vc = col < G && col < colmax;
-                s2[e] = (vt && vc) ? sc[e] * p.tau_log2e : -INFINITY;
-            }
-#pragma unroll
-            for (int c = 0; c < 2; c++) {
-                float tmax = fmaxf(s2[c] + lsv[0], s2[2 + c] + lsv[1]);
-                tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
-                tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
-                tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
-                const float mnew = fmaxf(m_run[c], tmax);
-                if (mnew == -INFINITY) {
-                    alpha[c] = 1.f;
+                        for (int hs = 0; hs < 2; hs++)
+                            mma_16816(acc, fa[hs][0], fa[hs][1], fa[hs][2], fa[hs][3],
+                                      qb[blk][hs][0], qb[blk][hs][1]);
+                    }
+                    if (KB != 16) {
+                        const float2 kk = unpack_half2(*reinterpret_cast<const uint32_t *>(ssk + tA));
+                        ks0 *= kk.x;
+                        ks1 *= kk.y;
+                    }
+                    s2[0] = (acc[0] - qbias[0][0]) * ks0;
+                    s2[1] = (acc[1] - qbias[0][1]) * ks0;
+                    s2[2] = (acc[2] - qbias[0][0]) * ks1;
+                    s2[3] = (acc[3] - qbias[0][1]) * ks1;
                 } else {
-                    alpha[c] = exp2f(m_run[c] - mnew);
+                    float acc[NG][4];
+#pragma unroll
+                    for (int blk = 0; blk < NG; blk++) {
+                        acc[blk][0] = acc[blk][1] = acc[blk][2] = acc[blk][3] = 0.f;
+                        uint32_t fa[2][4];
+                        key_frags(ra, rb, blk, fa);
+#pragma unroll
+                        for (int hs = 0; hs < 2; hs++)
+                            mma_16816(acc[blk], fa[hs][0], fa[hs][1], fa[hs][2], fa[hs][3],
+                                      qb[blk][hs][0], qb[blk][hs][1]);
+                    }
+                    float v[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int blk = 0; blk < NG; blk++) {
+                        const float k0 = __half2float(ssk[tA * p.ngs_k + (blk >> p.kshift)]);
+                        const float k1 = __half2float(ssk[(tA + 1) * p.ngs_k + (blk >> p.kshift)]);
+                        v[0] = fmaf(k0, acc[blk][0] - qbias[blk][0], v[0]);
+                        v[1] = fmaf(k0, acc[blk][1] - qbias[blk][1], v[1]);
+                        v[2] = fmaf(k1, acc[blk][2] - qbias[blk][0], v[2]);
+                        v[3] = fmaf(k1, acc[blk][3] - qbias[blk][1], v[3]);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 4; e++) s2[e] = v[e] * p.tau_log2e;
                 }
-                m_run[c] = mnew;
+                if (qsplit) {
+#pragma unroll
+                    for (int e = 0; e < 4; e++) s2[e] += __shfl_xor_sync(FULL, s2[e], 2);
+                }
+                s2[0] = (vt0 && col_ok0) ? s2[0] : -INFINITY;
+                s2[1] = (vt0 && col_ok1) ? s2[1] : -INFINITY;
+                s2[2] = (vt1 && col_ok0) ? s2[2] : -INFINITY;
+                s2[3] = (vt1 && col_ok1) ? s2[3] : -INFINITY;
             }
-        }
-        float pr[4];
+
+            // ---------------- value scales of rows tA, tA+1 -----------------
+            float sv0[NG], sv1[NG], lsv0, lsv1;
+            {
+                if (VB == 16) {
 #pragma unroll
-        for (int e = 0; e < 4; e++) {
-            const int c = e & 1;
-            pr[e] = (s2[e] == -INFINITY) ? 0.f : exp2f(s2[e] - m_run[c]);
-        }
+                    for (int g = 0; g < NG; g++) sv0[g] = sv1[g] = 1.f;
+                } else if (!vgrp) {
+                    const float2 vv = unpack_half2(*reinterpret_cast<const uint32_t *>(ssv + tA));
 #pragma unroll
-        for (int c = 0; c < 2; c++) l_run[c] = l_run[c] * alpha[c] + pr[c] + pr[2 + c];
-        if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
+                    for (int g = 0; g < NG; g++) {
+                        sv0[g] = vv.x;
+                        sv1[g] = vv.y;
+                    }
+                } else {
 #pragma unroll
-            for (int mt = 0; mt < 2 * NG; mt++) {
-                o_acc[mt][0] *= alpha[0];
-                o_acc[mt][1] *= alpha[1];
-                o_acc[mt][2] *= alpha[0];
-                o_acc[mt][3] *= alpha[1];
+                    for (int g = 0; g < NG; g++) {
+                        sv0[g] = __half2float(ssv[tA * p.ngs_v + (g >> p.vshift)]);
+                        sv1[g] = __half2float(ssv[(tA + 1) * p.ngs_v + (g >> p.vshift)]);
+                    }
+                }
+                // scales past the length may be stale shared memory: never use them
+                float mx0 = 0.f, mx1 = 0.f;
+#pragma unroll
+                for (int g = 0; g < NG; g++) {
+                    sv0[g] = vt0 ? sv0[g] : 0.f;
+                    sv1[g] = vt1 ? sv1[g] : 0.f;
+                    mx0 = fmaxf(mx0, sv0[g]);
+                    mx1 = fmaxf(mx1, sv1[g]);
+                }
+                lsv0 = mx0 > 0.f ? fmaxf(__log2f(mx0), -32.f) : -32.f;
+                lsv1 = mx1 > 0.f ? fmaxf(__log2f(mx1), -32.f) : -32.f;
             }
+
+            // ---------------- online softmax (lazy rescale) ------------------
+            {
+                const float loc0 = fmaxf(s2[0] + lsv0, s2[2] + lsv1);
+                const float loc1 = fmaxf(s2[1] + lsv0, s2[3] + lsv1);
+                const bool need = (loc0 > m_run[0] + LAZY) || (loc1 > m_run[1] + LAZY);
+                if (__any_sync(FULL, need)) {
+                    float r0 = loc0, r1 = loc1;
+#pragma unroll
+                    for (int off = 4; off < 32; off <<= 1) {
+                        r0 = fmaxf(r0, __shfl_xor_sync(FULL, r0, off));
+                        r1 = fmaxf(r1, __shfl_xor_sync(FULL, r1, off));
+                    }
+                    const float mn0 = fmaxf(m_run[0], r0), mn1 = fmaxf(m_run[1], r1);
+                    const float a0 = (mn0 == -INFINITY) ? 1.f : exp2f(m_run[0] - mn0);
+                    const float a1 = (mn1 == -INFINITY) ? 1.f : exp2f(m_run[1] - mn1);
+                    m_run[0] = mn0;
+                    m_run[1] = mn1;
+                    l_run[0] *= a0;
+                    l_run[1] *= a1;
+#pragma unroll
+                    for (int g = 0; g < NG; g++) {
+                        psum[g][0] *= a0;
+                        psum[g][1] *= a1;
+                    }
+#pragma unroll
+                    for (int mt = 0; mt < 2 * NG; mt++) {
+                        o_acc[mt][0] *= a0;
+                        o_acc[mt][1] *= a1;
+                        o_acc[mt][2] *= a0;
+                        o_acc[mt][3] *= a1;
+                    }
+                }
+            }
+            float pr[4];
+#pragma unroll
+            for (int e = 0; e < 4; e++)
+                pr[e] = (s2[e] == -INFINITY) ? 0.f : exp2f(s2[e] - m_run[e & 1]);
+            l_run[0] += pr[0] + pr[2];
+            l_run[1] += pr[1] + pr[3];
+
+            // ---------------- P (fp16, value scale folded) -> B fragments ----
+            uint32_t pb[NG][2];
+            const int nvb = vgrp ? NG : 1;
 #pragma unroll
             for (int g = 0; g < NG; g++) {
-                psum[g][0] *= alpha[0];
-                psum[g][1] *= alpha[1];
-            }
-        }
-
-        // ---------------- P (fp16, value scale folded) -> B fragments --------
-        const int src0 = tig * 4 + (gid >> 1);
-        const int src1 = (tig + 4) * 4 + (gid >> 1);
-        const bool odd = gid & 1;
-        uint32_t pb[NG][2];
-        const int nvb = vgrp ? NG : 1;
-#pragma unroll
-        for (int g = 0; g < NG; g++) {
-            if (g < nvb) {
-                const uint32_t ha = pack_half2(pr[0] * sv0[g], pr[2] * sv1[g]);  // col 2tig
-                const uint32_t hb = pack_half2(pr[1] * sv0[g], pr[3] * sv1[g]);  // col 2tig+1
-                const float2 fa = unpack_half2(ha), fb = unpack_half2(hb);
-                psum[g][0] += fa.x + fa.y;
-                psum[g][1] += fb.x + fb.y;
-                const uint32_t x0 = __shfl_sync(0xffffffffu, ha, src0);
-                const uint32_t y0 = __shfl_sync(0xffffffffu, hb, src0);
-                const uint32_t x1 = __shfl_sync(0xffffffffu, ha, src1);
-                const uint32_t y1 = __shfl_sync(0xffffffffu, hb, src1);
-                pb[g][0] = odd ? y0 : x0;
-                pb[g][1] = odd ? y1 : x1;
-            } else {
-                pb[g][0] = pb[0][0];
-                pb[g][1] = pb[0][1];
-            }
-        }
-
-        // ---------------- O^T += V^T P ---------------------------------------
-        const int tv = tw + 2 * tig;   // value tokens tv, tv+1, tv+8, tv+9
-#pragma unroll
-        for (int blk = 0; blk < NG; blk++) {
-            const uint32_t b0 = pb[blk][0], b1 = pb[blk][1];
-            if constexpr (VB == 8) {
-                const int o = 32 * blk + 4 * gid;
-                const uint32_t wA = *reinterpret_cast<const uint32_t *>(sv + sw_off<RV>(tv, o));
-                const uint32_t wB = *reinterpret_cast<const uint32_t *>(sv + sw_off<RV>(tv + 1, o));
-                const uint32_t wC = *reinterpret_cast<const uint32_t *>(sv + sw_off<RV>(tv + 8, o));
-                const uint32_t wE = *reinterpret_cast<const uint32_t *>(sv + sw_off<RV>(tv + 9, o));
-#pragma unroll
-                for (int u = 0; u < 2; u++) {
-                    const uint32_t sel = u ? 0x7632u : 0x5410u;
-                    const uint32_t yAB = prmt(wA, wB, sel), yCE = prmt(wC, wE, sel);
-                    const uint32_t a0 = and_xor(yAB, 0x00FF00FFu, 0x64806480u);
-                    const uint32_t a1 = and_xor(yAB >> 8, 0x00FF00FFu, 0x64806480u);
-                    const uint32_t a2 = and_xor(yCE, 0x00FF00FFu, 0x64806480u);
-                    const uint32_t a3 = and_xor(yCE >> 8, 0x00FF00FFu, 0x64806480u);
-                    mma_16816(o_acc[2 * blk + u], a0, a1, a2, a3, b0, b1);
+                if (g < nvb) {
+                    const uint32_t ha = pack_half2(pr[0] * sv0[g], pr[2] * sv1[g]);  // col 2tig
+                    const uint32_t hb = pack_half2(pr[1] * sv0[g], pr[3] * sv1[g]);  // col 2tig+1
+                    const float2 fa = unpack_half2(ha), fb = unpack_half2(hb);
+                    psum[g][0] += fa.x + fa.y;
+                    psum[g][1] += fb.x + fb.y;
+                    const uint32_t x0 = __shfl_sync(FULL, ha, src0);
+                    const uint32_t y0 = __shfl_sync(FULL, hb, src0);
+                    const uint32_t x1 = __shfl_sync(FULL, ha, src1);
+                    const uint32_t y1 = __shfl_sync(FULL, hb, src1);
+                    pb[g][0] = odd ? y0 : x0;
+                    pb[g][1] = odd ? y1 : x1;
+                } else {
+                    pb[g][0] = pb[0][0];
+                    pb[g][1] = pb[0][1];
                 }
-            } else if constexpr (VB == 4) {
-                const int o = 16 * blk + 2 * gid;
-                const uint32_t hA = *reinterpret_cast<const uint16_t *>(sv + sw_off<RV>(tv, o));
-                const uint32_t hB = *reinterpret_cast<const uint16_t *>(sv + sw_off<RV>(tv + 1, o));
-                const uint32_t hC = *reinterpret_cast<const uint16_t *>(sv + sw_off<RV>(tv + 8, o));
-                const uint32_t hE = *reinterpret_cast<const uint16_t *>(sv + sw_off<RV>(tv + 9, o));
-                const uint32_t yAB = prmt(hA, hB, 0x5410u), yCE = prmt(hC, hE, 0x5410u);
+            }
+
+            // ---------------- O^T += V^T P -----------------------------------
+            const uint32_t va = st + vofs[u][0], vb = st + vofs[u][1];
+            const uint32_t vc = st + vofs[u][2], ve = st + vofs[u][3];
 #pragma unroll
-                for (int u = 0; u < 2; u++) {
-                    const uint32_t a0 = i4_pair(yAB, 2 * u);
-                    const uint32_t a1 = i4_pair(yAB, 2 * u + 1);
-                    const uint32_t a2 = i4_pair(yCE, 2 * u);
-                    const uint32_t a3 = i4_pair(yCE, 2 * u + 1);
-                    mma_16816(o_acc[2 * blk + u], a0, a1, a2, a3, b0, b1);
-                }
-            } else {
-                const int o = 64 * blk + 8 * gid;
-                // fp16 values past the length may be anything (NaN included): zero them
-                const int tg = m.t0 + tv;
-                const uint2 z = make_uint2(0u, 0u);
-                const uint2 wA = tg < m.len ? *reinterpret_cast<const uint2 *>(sv + sw_off<RV>(tv, o)) : z;
-                const uint2 wB = tg + 1 < m.len ? *reinterpret_cast<const uint2 *>(sv + sw_off<RV>(tv + 1, o)) : z;
-                const uint2 wC = tg + 8 < m.len ? *reinterpret_cast<const uint2 *>(sv + sw_off<RV>(tv + 8, o)) : z;
-                const uint2 wE = tg + 9 < m.len ? *reinterpret_cast<const uint2 *>(sv + sw_off<RV>(tv + 9, o)) : z;
+            for (int blk = 0; blk < NG; blk++) {
+                const uint32_t b0 = pb[blk][0], b1 = pb[blk][1];
+                if constexpr (VB == 8) {
+                    const uint32_t wA = lds_u32(blk_addr<RV, SV>(va, blk));
+                    const uint32_t wB = lds_u32(blk_addr<RV, SV>(vb, blk));
+                    const uint32_t wC = lds_u32(blk_addr<RV, SV>(vc, blk));
+                    const uint32_t wE = lds_u32(blk_addr<RV, SV>(ve, blk));
 #pragma unroll
-                for (int u = 0; u < 2; u++) {
-                    const uint32_t A = u ? wA.y : wA.x, Bw = u ? wB.y : wB.x;
-                    const uint32_t C = u ? wC.y : wC.x, E = u ? wE.y : wE.x;
-                    const uint32_t a0 = prmt(A, Bw, 0x5410u), a1 = prmt(A, Bw, 0x7632u);
-                    const uint32_t a2 = prmt(C, E, 0x5410u), a3 = prmt(C, E, 0x7632u);
-                    mma_16816(o_acc[2 * blk + u], a0, a1, a2, a3, b0, b1);
+                    for (int h = 0; h < 2; h++) {
+                        const uint32_t sel = h ? 0x7632u : 0x5410u;
+                        const uint32_t yAB = prmt(wA, wB, sel), yCE = prmt(wC, wE, sel);
+                        const uint32_t a0 = and_xor(yAB, 0x00FF00FFu, 0x64806480u);
+                        const uint32_t a1 = and_xor(yAB >> 8, 0x00FF00FFu, 0x64806480u);
+                        const uint32_t a2 = and_xor(yCE, 0x00FF00FFu, 0x64806480u);
+                        const uint32_t a3 = and_xor(yCE >> 8, 0x00FF00FFu, 0x64806480u);
+                        mma_16816(o_acc[2 * blk + h], a0, a1, a2, a3, b0, b1);
+                    }
+                } else if constexpr (VB == 4) {
+                    const uint32_t hA = lds_u16(blk_addr<RV, SV>(va, blk));
+                    const uint32_t hB = lds_u16(blk_addr<RV, SV>(vb, blk));
+                    const uint32_t hC = lds_u16(blk_addr<RV, SV>(vc, blk));
+                    const uint32_t hE = lds_u16(blk_addr<RV, SV>(ve, blk));
+                    const uint32_t yAB = prmt(hA, hB, 0x5410u), yCE = prmt(hC, hE, 0x5410u);
+#pragma unroll
+                    for (int h = 0; h < 2; h++) {
+                        const uint32_t a0 = i4_pair(yAB, 2 * h);
+                        const uint32_t a1 = i4_pair(yAB, 2 * h + 1);
+                        const uint32_t a2 = i4_pair(yCE, 2 * h);
+                        const uint32_t a3 = i4_pair(yCE, 2 * h + 1);
+                        mma_16816(o_acc[2 * blk + h], a0, a1, a2, a3, b0, b1);
+                    }
+                } else {
+                    // fp16 values past the length may be anything (NaN included): zero them
+                    const int tg = m.t0 + warp * 32 + u * 16 + 2 * tig;
+                    const uint2 z = make_uint2(0u, 0u);
+                    const uint2 wA = tg < m.len ? lds_u64(blk_addr<RV, SV>(va, blk)) : z;
+                    const uint2 wB = tg + 1 < m.len ? lds_u64(blk_addr<RV, SV>(vb, blk)) : z;
+                    const uint2 wC = tg + 8 < m.len ? lds_u64(blk_addr<RV, SV>(vc, blk)) : z;
+                    const uint2 wE = tg + 9 < m.len ? lds_u64(blk_addr<RV, SV>(ve, blk)) : z;
+#pragma unroll
+                    for (int h = 0; h < 2; h++) {
+                        const uint32_t A = h ? wA.y : wA.x, Bw = h ? wB.y : wB.x;
+                        const uint32_t C = h ? wC.y : wC.x, E = h ? wE.y : wE.x;
+                        const uint32_t a0 = prmt(A, Bw, 0x5410u), a1 = prmt(A, Bw, 0x7632u);
+                        const uint32_t a2 = prmt(C, E, 0x5410u), a3 = prmt(C, E, 0x7632u);
+                        mma_16816(o_acc[2 * blk + h], a0, a1, a2, a3, b0, b1);
+                    }
                 }
             }
         }
@@ -598,6 +689,10 @@ __global__ void __launch_bounds__(NTHR, 2)
         // release the stage to the producer
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
+        if (++s == S) {
+            s = 0;
+            ph ^= 1u;
+        }
 
         // ---------------- segment end: merge the warps, write the partial ---
         if (m.flags & 2) {
@@ -605,16 +700,16 @@ __global__ void __launch_bounds__(NTHR, 2)
 #pragma unroll
             for (int c = 0; c < 2; c++) {
                 float v = l_run[c];
-                v += __shfl_xor_sync(0xffffffffu, v, 4);
-                v += __shfl_xor_sync(0xffffffffu, v, 8);
-                v += __shfl_xor_sync(0xffffffffu, v, 16);
+                v += __shfl_xor_sync(FULL, v, 4);
+                v += __shfl_xor_sync(FULL, v, 8);
+                v += __shfl_xor_sync(FULL, v, 16);
                 lt[c] = v;
 #pragma unroll
                 for (int g = 0; g < NG; g++) {
                     float w = psum[g][c];
-                    w += __shfl_xor_sync(0xffffffffu, w, 4);
-                    w += __shfl_xor_sync(0xffffffffu, w, 8);
-                    w += __shfl_xor_sync(0xffffffffu, w, 16);
+                    w += __shfl_xor_sync(FULL, w, 4);
+                    w += __shfl_xor_sync(FULL, w, 8);
+                    w += __shfl_xor_sync(FULL, w, 16);
                     ps[g][c] = w;
                 }
             }
@@ -623,16 +718,16 @@ __global__ void __launch_bounds__(NTHR, 2)
 #pragma unroll
             for (int c = 0; c < 2; c++) {
                 const int col = 2 * tig + c;
-                if (col < G && (!qsplit || col < 4)) {
+                if (c == 0 ? col_ok0 : col_ok1) {
                     float *oc = mine + (size_t)col * (DH + 2);
 #pragma unroll
                     for (int blk = 0; blk < NG; blk++) {
                         const float corr = BIAS_V * ps[vgrp ? blk : 0][c];
 #pragma unroll
-                        for (int u = 0; u < 2; u++) {
-                            const int d = 32 * blk + 4 * gid + 2 * u;
-                            oc[d] = o_acc[2 * blk + u][c] - corr;
-                            oc[d + 1] = o_acc[2 * blk + u][2 + c] - corr;
+                        for (int h = 0; h < 2; h++) {
+                            const int d = 32 * blk + 4 * gid + 2 * h;
+                            oc[d] = o_acc[2 * blk + h][c] - corr;
+                            oc[d + 1] = o_acc[2 * blk + h][2 + c] - corr;
                         }
                     }
                     if (gid == 0) {
@@ -646,14 +741,12 @@ __global__ void __launch_bounds__(NTHR, 2)
             if (!mbar_wait_bounded(&segbar[0], seg_parity, abort_flag, limit)) {
                 ctl[0] = 1;
                 atomicExch(p.status, KVQ_ERR_TIMEOUT);
-                ok = false;
                 break;
             }
-            // combine NW warps deterministically and write the slot
+            // combine the NW warps deterministically and write the slot
             const int slot = m.flags >> 8;
             float *dst = p.ws + (size_t)slot * G * (DH + 2);
-            const int ctid = tid;  // 0 .. 32*NW-1
-            for (int idx = ctid; idx < G * DH; idx += 32 * NW) {
+            for (int idx = tid; idx < G * DH; idx += 32 * NW) {
                 const int col = idx / DH, d = idx % DH;
                 float M = -INFINITY;
 #pragma unroll
@@ -668,8 +761,8 @@ __global__ void __launch_bounds__(NTHR, 2)
                 }
                 dst[(size_t)col * (DH + 2) + d] = O;
             }
-            if (ctid < G) {
-                const int col = ctid;
+            if (tid < G) {
+                const int col = tid;
                 float M = -INFINITY;
 #pragma unroll
                 for (int w = 0; w < NW; w++) M = fmaxf(M, mbuf[((size_t)w * G + col) * (DH + 2) + DH]);
@@ -688,13 +781,11 @@ __global__ void __launch_bounds__(NTHR, 2)
             if (!mbar_wait_bounded(&segbar[1], seg_parity, abort_flag, limit)) {
                 ctl[0] = 1;
                 atomicExch(p.status, KVQ_ERR_TIMEOUT);
-                ok = false;
                 break;
             }
-            seg_parity ^= 1;
+            seg_parity ^= 1u;
         }
     }
-    (void)ok;
 }
 
 // ---------------------------------------------------------------------------

@@ -22,7 +22,7 @@ cudaError_t launch_append(const AppendParams &k, const AppendParams *v, cudaStre
 
 // ------------------------------------------------------------------ decode
 constexpr int kDecodeConsumerWarps = 4;
-constexpr int kDecodeTileTokens = 16 * kDecodeConsumerWarps;   // tokens per stage
+constexpr int kDecodeTileTokens = 32 * kDecodeConsumerWarps;   // tokens per stage (32 per warp)
 constexpr int kDecodeThreads = 32 * (kDecodeConsumerWarps + 1);
 constexpr int kWorkspaceHeaderFloats = 64;                      // status word + padding
 
