@@ -112,31 +112,43 @@ __device__ __forceinline__ int tiles_of(int len, int cap)
     return (len + T - 1) / T;
 }
 
-// Shared-memory loads at 32-bit shared-window addresses.
-__device__ __forceinline__ uint32_t lds_u16(uint32_t a)
+// 2^x with the hardware approximation (relative error ~2^-22); results below
+// 2^-126 flush to zero, which only drops probabilities that are zero anyway.
+__device__ __forceinline__ float fast_exp2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Loads from the stage ring.  `b` is the 32-bit shared-window address of the
+// 1024-aligned ring base and `o` a byte offset from it; explicit ld.shared keeps the
+// address arithmetic 32-bit.  volatile keeps every load after the mbarrier wait
+// that guards its stage (the wait is a volatile asm with a memory clobber).
+__device__ __forceinline__ uint32_t lds_u16(uint32_t b, uint32_t o)
 {
     uint16_t v;
-    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(b + o));
     return v;
 }
-__device__ __forceinline__ uint32_t lds_u32(uint32_t a)
+__device__ __forceinline__ uint32_t lds_u32(uint32_t b, uint32_t o)
 {
     uint32_t v;
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(b + o));
     return v;
 }
-__device__ __forceinline__ uint2 lds_u64(uint32_t a)
+__device__ __forceinline__ uint2 lds_u64(uint32_t b, uint32_t o)
 {
     uint2 v;
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(b + o));
     return v;
 }
-__device__ __forceinline__ uint4 lds_u128(uint32_t a)
+__device__ __forceinline__ uint4 lds_u128(uint32_t b, uint32_t o)
 {
     uint4 v;
     asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "r"(a));
+                 : "r"(b + o));
     return v;
 }
 
@@ -175,7 +187,10 @@ __global__ void __launch_bounds__(NTHR, 2)
     constexpr unsigned FULL = 0xffffffffu;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    // align to 1024 B (128-byte swizzle atoms) by pointer arithmetic on the shared
+    // array itself, so every access below stays a shared-memory access
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(smem);             // 32-bit shared address of the ring
     StageMeta *meta = reinterpret_cast<StageMeta *>(smem + p.off_meta);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + p.off_bar);
     uint64_t *empty = full + p.stages;
@@ -430,8 +445,8 @@ __global__ void __launch_bounds__(NTHR, 2)
     // A fragments of block blk, k-half hs, for key rows at a[0] (row gid) and a[1] (row gid+8)
     auto key_frags = [&](uint32_t ra, uint32_t rb, int blk, uint32_t (&fa)[2][4]) {
         if constexpr (KB == 8) {
-            const uint2 r0 = lds_u64(blk_addr<RK, SK>(ra, blk));
-            const uint2 r1 = lds_u64(blk_addr<RK, SK>(rb, blk));
+            const uint2 r0 = lds_u64(sbase, blk_addr<RK, SK>(ra, blk));
+            const uint2 r1 = lds_u64(sbase, blk_addr<RK, SK>(rb, blk));
             const uint32_t x00 = r0.x ^ 0x80808080u, x01 = r0.y ^ 0x80808080u;
             const uint32_t x10 = r1.x ^ 0x80808080u, x11 = r1.y ^ 0x80808080u;
             fa[0][0] = i8_lo_pair(x00); fa[0][2] = i8_hi_pair(x00);
@@ -439,22 +454,21 @@ __global__ void __launch_bounds__(NTHR, 2)
             fa[1][0] = i8_lo_pair(x01); fa[1][2] = i8_hi_pair(x01);
             fa[1][1] = i8_lo_pair(x11); fa[1][3] = i8_hi_pair(x11);
         } else if constexpr (KB == 4) {
-            const uint32_t r0 = lds_u32(blk_addr<RK, SK>(ra, blk));
-            const uint32_t r1 = lds_u32(blk_addr<RK, SK>(rb, blk));
+            const uint32_t r0 = lds_u32(sbase, blk_addr<RK, SK>(ra, blk));
+            const uint32_t r1 = lds_u32(sbase, blk_addr<RK, SK>(rb, blk));
             fa[0][0] = i4_pair(r0, 0); fa[0][2] = i4_pair(r0, 1);
             fa[0][1] = i4_pair(r1, 0); fa[0][3] = i4_pair(r1, 1);
             fa[1][0] = i4_pair(r0, 2); fa[1][2] = i4_pair(r0, 3);
             fa[1][1] = i4_pair(r1, 2); fa[1][3] = i4_pair(r1, 3);
         } else {
-            const uint4 r0 = lds_u128(blk_addr<RK, SK>(ra, blk));
-            const uint4 r1 = lds_u128(blk_addr<RK, SK>(rb, blk));
+            const uint4 r0 = lds_u128(sbase, blk_addr<RK, SK>(ra, blk));
+            const uint4 r1 = lds_u128(sbase, blk_addr<RK, SK>(rb, blk));
             fa[0][0] = r0.x; fa[0][2] = r0.y; fa[0][1] = r1.x; fa[0][3] = r1.y;
             fa[1][0] = r0.z; fa[1][2] = r0.w; fa[1][1] = r1.z; fa[1][3] = r1.w;
         }
     };
 
     const uint64_t limit = p.timeout_ns;
-    const uint32_t smem_base = smem_u32(smem);
     int s = 0;
     uint32_t ph = 0;
     for (int i = 0; i < n_units; i++) {
@@ -463,159 +477,200 @@ __global__ void __launch_bounds__(NTHR, 2)
             atomicExch(p.status, KVQ_ERR_TIMEOUT);
             break;
         }
-        const StageMeta m = meta[s];
+        StageMeta m;
+        {
+            const uint4 mm = *reinterpret_cast<const uint4 *>(&meta[s]);
+            m.bh = (int)mm.x; m.t0 = (int)mm.y; m.len = (int)mm.z; m.flags = (int)mm.w;
+        }
         if (m.flags & 1) load_q(m.bh);
-        const uint32_t st = smem_base + (uint32_t)s * p.stage_bytes;
-        const __half *ssk = reinterpret_cast<const __half *>(smem + (size_t)s * p.stage_bytes + p.off_sk);
-        const __half *ssv = reinterpret_cast<const __half *>(smem + (size_t)s * p.stage_bytes + p.off_sv);
+        const uint32_t st = (uint32_t)s * p.stage_bytes;   // stage offset from smem
+        const uint32_t ssk = st + p.off_sk;   // fp16 key scales of the stage
+        const uint32_t ssv = st + p.off_sv;   // fp16 value scales
 
+        // Work of this warp on the stage: two 16-token sub-tiles u = 0, 1, processed
+        // phase by phase so that the two sub-tiles give the scheduler independent
+        // instruction streams at every step.
+        int tAu[2];
+        bool vt[2][2];
 #pragma unroll
         for (int u = 0; u < 2; u++) {
-            const int tA = warp * 32 + u * 16 + 2 * gid;       // score rows: tokens tA, tA + 1
-            const bool vt0 = m.t0 + tA < m.len;
-            const bool vt1 = m.t0 + tA + 1 < m.len;
+            tAu[u] = warp * 32 + u * 16 + 2 * gid;               // score rows: tAu, tAu + 1
+            vt[u][0] = m.t0 + tAu[u] < m.len;
+            vt[u][1] = m.t0 + tAu[u] + 1 < m.len;
+        }
 
-            // ---------------- scores: S^T = K q^T ---------------------------
-            float s2[4];
-            {
-                const uint32_t ra = st + kofs[u][0], rb = st + kofs[u][1];
-                float ks0 = p.tau_log2e, ks1 = p.tau_log2e;
-                if (!kgrp) {
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        // ---------------- phase 1: scores S^T = K q^T for both sub-tiles ----------
+        float s2[2][4];
+        if (!kgrp) {
+            // two partial accumulators per sub-tile (even / odd blocks) halve the
+            // dependent MMA chain
+            float acc[2][2][4];
 #pragma unroll
-                    for (int blk = 0; blk < NG; blk++) {
-                        uint32_t fa[2][4];
-                        key_frags(ra, rb, blk, fa);
+            for (int u = 0; u < 2; u++)
 #pragma unroll
-                        for (int hs = 0; hs < 2; hs++)
-                            mma_16816(acc, fa[hs][0], fa[hs][1], fa[hs][2], fa[hs][3],
-                                      qb[blk][hs][0], qb[blk][hs][1]);
-                    }
-                    if (KB != 16) {
-                        const float2 kk = unpack_half2(*reinterpret_cast<const uint32_t *>(ssk + tA));
-                        ks0 *= kk.x;
-                        ks1 *= kk.y;
-                    }
-                    s2[0] = (acc[0] - qbias[0][0]) * ks0;
-                    s2[1] = (acc[1] - qbias[0][1]) * ks0;
-                    s2[2] = (acc[2] - qbias[0][0]) * ks1;
-                    s2[3] = (acc[3] - qbias[0][1]) * ks1;
-                } else {
-                    float acc[NG][4];
+                for (int h = 0; h < 2; h++) acc[u][h][0] = acc[u][h][1] = acc[u][h][2] = acc[u][h][3] = 0.f;
 #pragma unroll
-                    for (int blk = 0; blk < NG; blk++) {
-                        acc[blk][0] = acc[blk][1] = acc[blk][2] = acc[blk][3] = 0.f;
-                        uint32_t fa[2][4];
-                        key_frags(ra, rb, blk, fa);
+            for (int blk = 0; blk < NG; blk++) {
 #pragma unroll
-                        for (int hs = 0; hs < 2; hs++)
-                            mma_16816(acc[blk], fa[hs][0], fa[hs][1], fa[hs][2], fa[hs][3],
-                                      qb[blk][hs][0], qb[blk][hs][1]);
-                    }
-                    float v[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int u = 0; u < 2; u++) {
+                    uint32_t fa[2][4];
+                    key_frags(st + kofs[u][0], st + kofs[u][1], blk, fa);
 #pragma unroll
-                    for (int blk = 0; blk < NG; blk++) {
-                        const float k0 = __half2float(ssk[tA * p.ngs_k + (blk >> p.kshift)]);
-                        const float k1 = __half2float(ssk[(tA + 1) * p.ngs_k + (blk >> p.kshift)]);
-                        v[0] = fmaf(k0, acc[blk][0] - qbias[blk][0], v[0]);
-                        v[1] = fmaf(k0, acc[blk][1] - qbias[blk][1], v[1]);
-                        v[2] = fmaf(k1, acc[blk][2] - qbias[blk][0], v[2]);
-                        v[3] = fmaf(k1, acc[blk][3] - qbias[blk][1], v[3]);
-                    }
-#pragma unroll
-                    for (int e = 0; e < 4; e++) s2[e] = v[e] * p.tau_log2e;
+                    for (int hs = 0; hs < 2; hs++)
+                        mma_16816(acc[u][blk & 1], fa[hs][0], fa[hs][1], fa[hs][2], fa[hs][3],
+                                  qb[blk][hs][0], qb[blk][hs][1]);
                 }
-                if (qsplit) {
-#pragma unroll
-                    for (int e = 0; e < 4; e++) s2[e] += __shfl_xor_sync(FULL, s2[e], 2);
-                }
-                s2[0] = (vt0 && col_ok0) ? s2[0] : -INFINITY;
-                s2[1] = (vt0 && col_ok1) ? s2[1] : -INFINITY;
-                s2[2] = (vt1 && col_ok0) ? s2[2] : -INFINITY;
-                s2[3] = (vt1 && col_ok1) ? s2[3] : -INFINITY;
             }
-
-            // ---------------- value scales of rows tA, tA+1 -----------------
-            float sv0[NG], sv1[NG], lsv0, lsv1;
-            {
-                if (VB == 16) {
 #pragma unroll
-                    for (int g = 0; g < NG; g++) sv0[g] = sv1[g] = 1.f;
-                } else if (!vgrp) {
-                    const float2 vv = unpack_half2(*reinterpret_cast<const uint32_t *>(ssv + tA));
-#pragma unroll
-                    for (int g = 0; g < NG; g++) {
-                        sv0[g] = vv.x;
-                        sv1[g] = vv.y;
-                    }
-                } else {
-#pragma unroll
-                    for (int g = 0; g < NG; g++) {
-                        sv0[g] = __half2float(ssv[tA * p.ngs_v + (g >> p.vshift)]);
-                        sv1[g] = __half2float(ssv[(tA + 1) * p.ngs_v + (g >> p.vshift)]);
-                    }
+            for (int u = 0; u < 2; u++) {
+                float ks0 = p.tau_log2e, ks1 = p.tau_log2e;
+                if (KB != 16) {
+                    const float2 kk = unpack_half2(lds_u32(sbase, ssk + 2 * tAu[u]));
+                    ks0 *= kk.x;
+                    ks1 *= kk.y;
                 }
-                // scales past the length may be stale shared memory: never use them
-                float mx0 = 0.f, mx1 = 0.f;
+                s2[u][0] = (acc[u][0][0] + acc[u][1][0] - qbias[0][0]) * ks0;
+                s2[u][1] = (acc[u][0][1] + acc[u][1][1] - qbias[0][1]) * ks0;
+                s2[u][2] = (acc[u][0][2] + acc[u][1][2] - qbias[0][0]) * ks1;
+                s2[u][3] = (acc[u][0][3] + acc[u][1][3] - qbias[0][1]) * ks1;
+            }
+        } else {
+#pragma unroll
+            for (int u = 0; u < 2; u++) {
+                float acc[NG][4];
+#pragma unroll
+                for (int blk = 0; blk < NG; blk++) {
+                    acc[blk][0] = acc[blk][1] = acc[blk][2] = acc[blk][3] = 0.f;
+                    uint32_t fa[2][4];
+                    key_frags(st + kofs[u][0], st + kofs[u][1], blk, fa);
+#pragma unroll
+                    for (int hs = 0; hs < 2; hs++)
+                        mma_16816(acc[blk], fa[hs][0], fa[hs][1], fa[hs][2], fa[hs][3],
+                                  qb[blk][hs][0], qb[blk][hs][1]);
+                }
+                float v[4] = {0.f, 0.f, 0.f, 0.f};
+                const int tA = tAu[u];
+#pragma unroll
+                for (int blk = 0; blk < NG; blk++) {
+                    const float k0 = __half2float(__ushort_as_half(
+                        (unsigned short)lds_u16(sbase, ssk + 2 * (tA * p.ngs_k + (blk >> p.kshift)))));
+                    const float k1 = __half2float(__ushort_as_half(
+                        (unsigned short)lds_u16(sbase, ssk + 2 * ((tA + 1) * p.ngs_k + (blk >> p.kshift)))));
+                    v[0] = fmaf(k0, acc[blk][0] - qbias[blk][0], v[0]);
+                    v[1] = fmaf(k0, acc[blk][1] - qbias[blk][1], v[1]);
+                    v[2] = fmaf(k1, acc[blk][2] - qbias[blk][0], v[2]);
+                    v[3] = fmaf(k1, acc[blk][3] - qbias[blk][1], v[3]);
+                }
+#pragma unroll
+                for (int e = 0; e < 4; e++) s2[u][e] = v[e] * p.tau_log2e;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; u++) {
+            if (qsplit) {
+#pragma unroll
+                for (int e = 0; e < 4; e++) s2[u][e] += __shfl_xor_sync(FULL, s2[u][e], 2);
+            }
+            // Padding columns (heads >= G, or the hi/lo halves of a split query)
+            // carry finite scores from zero query columns; their outputs are never
+            // written, so only tokens past the length are masked.
+            s2[u][0] = vt[u][0] ? s2[u][0] : -INFINITY;
+            s2[u][1] = vt[u][0] ? s2[u][1] : -INFINITY;
+            s2[u][2] = vt[u][1] ? s2[u][2] : -INFINITY;
+            s2[u][3] = vt[u][1] ? s2[u][3] : -INFINITY;
+        }
+
+        // ---------------- phase 2: value scales of the score rows -----------------
+        float sv[2][2][NG];   // [sub-tile][row][value block]
+        float lsv[2][2];
+#pragma unroll
+        for (int u = 0; u < 2; u++) {
+            const int tA = tAu[u];
+            if (VB == 16) {
+#pragma unroll
+                for (int g = 0; g < NG; g++) sv[u][0][g] = sv[u][1][g] = 1.f;
+            } else if (!vgrp) {
+                const float2 vv = unpack_half2(lds_u32(sbase, ssv + 2 * tA));
 #pragma unroll
                 for (int g = 0; g < NG; g++) {
-                    sv0[g] = vt0 ? sv0[g] : 0.f;
-                    sv1[g] = vt1 ? sv1[g] : 0.f;
-                    mx0 = fmaxf(mx0, sv0[g]);
-                    mx1 = fmaxf(mx1, sv1[g]);
+                    sv[u][0][g] = vv.x;
+                    sv[u][1][g] = vv.y;
                 }
-                lsv0 = mx0 > 0.f ? fmaxf(__log2f(mx0), -32.f) : -32.f;
-                lsv1 = mx1 > 0.f ? fmaxf(__log2f(mx1), -32.f) : -32.f;
+            } else {
+#pragma unroll
+                for (int g = 0; g < NG; g++) {
+                    sv[u][0][g] = __half2float(__ushort_as_half(
+                        (unsigned short)lds_u16(sbase, ssv + 2 * (tA * p.ngs_v + (g >> p.vshift)))));
+                    sv[u][1][g] = __half2float(__ushort_as_half(
+                        (unsigned short)lds_u16(sbase, ssv + 2 * ((tA + 1) * p.ngs_v + (g >> p.vshift)))));
+                }
             }
+            // scales past the length may be stale shared memory: never use them
+#pragma unroll
+            for (int r = 0; r < 2; r++) {
+                float mx = 0.f;
+#pragma unroll
+                for (int g = 0; g < NG; g++) {
+                    sv[u][r][g] = vt[u][r] ? sv[u][r][g] : 0.f;
+                    mx = fmaxf(mx, sv[u][r][g]);
+                }
+                lsv[u][r] = mx > 0.f ? fmaxf(__log2f(mx), -32.f) : -32.f;
+            }
+        }
 
-            // ---------------- online softmax (lazy rescale) ------------------
-            {
-                const float loc0 = fmaxf(s2[0] + lsv0, s2[2] + lsv1);
-                const float loc1 = fmaxf(s2[1] + lsv0, s2[3] + lsv1);
-                const bool need = (loc0 > m_run[0] + LAZY) || (loc1 > m_run[1] + LAZY);
-                if (__any_sync(FULL, need)) {
-                    float r0 = loc0, r1 = loc1;
+        // ---------------- phase 3: online softmax, one lazy check for 32 tokens ---
+        {
+            float loc0 = -INFINITY, loc1 = -INFINITY;
 #pragma unroll
-                    for (int off = 4; off < 32; off <<= 1) {
-                        r0 = fmaxf(r0, __shfl_xor_sync(FULL, r0, off));
-                        r1 = fmaxf(r1, __shfl_xor_sync(FULL, r1, off));
-                    }
-                    const float mn0 = fmaxf(m_run[0], r0), mn1 = fmaxf(m_run[1], r1);
-                    const float a0 = (mn0 == -INFINITY) ? 1.f : exp2f(m_run[0] - mn0);
-                    const float a1 = (mn1 == -INFINITY) ? 1.f : exp2f(m_run[1] - mn1);
-                    m_run[0] = mn0;
-                    m_run[1] = mn1;
-                    l_run[0] *= a0;
-                    l_run[1] *= a1;
+            for (int u = 0; u < 2; u++) {
+                loc0 = fmaxf(loc0, fmaxf(s2[u][0] + lsv[u][0], s2[u][2] + lsv[u][1]));
+                loc1 = fmaxf(loc1, fmaxf(s2[u][1] + lsv[u][0], s2[u][3] + lsv[u][1]));
+            }
+            const bool need = (loc0 > m_run[0] + LAZY) || (loc1 > m_run[1] + LAZY);
+            if (__any_sync(FULL, need)) {
 #pragma unroll
-                    for (int g = 0; g < NG; g++) {
-                        psum[g][0] *= a0;
-                        psum[g][1] *= a1;
-                    }
+                for (int off = 4; off < 32; off <<= 1) {
+                    loc0 = fmaxf(loc0, __shfl_xor_sync(FULL, loc0, off));
+                    loc1 = fmaxf(loc1, __shfl_xor_sync(FULL, loc1, off));
+                }
+                const float mn0 = fmaxf(m_run[0], loc0), mn1 = fmaxf(m_run[1], loc1);
+                const float a0 = (mn0 == -INFINITY) ? 1.f : fast_exp2(m_run[0] - mn0);
+                const float a1 = (mn1 == -INFINITY) ? 1.f : fast_exp2(m_run[1] - mn1);
+                m_run[0] = mn0;
+                m_run[1] = mn1;
+                l_run[0] *= a0;
+                l_run[1] *= a1;
 #pragma unroll
-                    for (int mt = 0; mt < 2 * NG; mt++) {
-                        o_acc[mt][0] *= a0;
-                        o_acc[mt][1] *= a1;
-                        o_acc[mt][2] *= a0;
-                        o_acc[mt][3] *= a1;
-                    }
+                for (int g = 0; g < NG; g++) {
+                    psum[g][0] *= a0;
+                    psum[g][1] *= a1;
+                }
+#pragma unroll
+                for (int mt = 0; mt < 2 * NG; mt++) {
+                    o_acc[mt][0] *= a0;
+                    o_acc[mt][1] *= a1;
+                    o_acc[mt][2] *= a0;
+                    o_acc[mt][3] *= a1;
                 }
             }
+        }
+
+        // ---------------- phase 4: P (fp16, value scale folded) -> B fragments ----
+        uint32_t pb[2][NG][2];
+        const int nvb = vgrp ? NG : 1;
+#pragma unroll
+        for (int u = 0; u < 2; u++) {
             float pr[4];
 #pragma unroll
             for (int e = 0; e < 4; e++)
-                pr[e] = (s2[e] == -INFINITY) ? 0.f : exp2f(s2[e] - m_run[e & 1]);
+                pr[e] = (s2[u][e] == -INFINITY) ? 0.f : fast_exp2(s2[u][e] - m_run[e & 1]);
             l_run[0] += pr[0] + pr[2];
             l_run[1] += pr[1] + pr[3];
-
-            // ---------------- P (fp16, value scale folded) -> B fragments ----
-            uint32_t pb[NG][2];
-            const int nvb = vgrp ? NG : 1;
 #pragma unroll
             for (int g = 0; g < NG; g++) {
                 if (g < nvb) {
-                    const uint32_t ha = pack_half2(pr[0] * sv0[g], pr[2] * sv1[g]);  // col 2tig
-                    const uint32_t hb = pack_half2(pr[1] * sv0[g], pr[3] * sv1[g]);  // col 2tig+1
+                    const uint32_t ha = pack_half2(pr[0] * sv[u][0][g], pr[2] * sv[u][1][g]);  // col 2tig
+                    const uint32_t hb = pack_half2(pr[1] * sv[u][0][g], pr[3] * sv[u][1][g]);  // col 2tig+1
                     const float2 fa = unpack_half2(ha), fb = unpack_half2(hb);
                     psum[g][0] += fa.x + fa.y;
                     psum[g][1] += fb.x + fb.y;
@@ -623,25 +678,28 @@ __global__ void __launch_bounds__(NTHR, 2)
                     const uint32_t y0 = __shfl_sync(FULL, hb, src0);
                     const uint32_t x1 = __shfl_sync(FULL, ha, src1);
                     const uint32_t y1 = __shfl_sync(FULL, hb, src1);
-                    pb[g][0] = odd ? y0 : x0;
-                    pb[g][1] = odd ? y1 : x1;
+                    pb[u][g][0] = odd ? y0 : x0;
+                    pb[u][g][1] = odd ? y1 : x1;
                 } else {
-                    pb[g][0] = pb[0][0];
-                    pb[g][1] = pb[0][1];
+                    pb[u][g][0] = pb[u][0][0];
+                    pb[u][g][1] = pb[u][0][1];
                 }
             }
+        }
 
-            // ---------------- O^T += V^T P -----------------------------------
-            const uint32_t va = st + vofs[u][0], vb = st + vofs[u][1];
-            const uint32_t vc = st + vofs[u][2], ve = st + vofs[u][3];
+        // ---------------- phase 5: O^T += V^T P for both sub-tiles ----------------
 #pragma unroll
-            for (int blk = 0; blk < NG; blk++) {
-                const uint32_t b0 = pb[blk][0], b1 = pb[blk][1];
+        for (int blk = 0; blk < NG; blk++) {
+#pragma unroll
+            for (int u = 0; u < 2; u++) {
+                const uint32_t va = st + vofs[u][0], vb = st + vofs[u][1];
+                const uint32_t vc = st + vofs[u][2], ve = st + vofs[u][3];
+                const uint32_t b0 = pb[u][blk][0], b1 = pb[u][blk][1];
                 if constexpr (VB == 8) {
-                    const uint32_t wA = lds_u32(blk_addr<RV, SV>(va, blk));
-                    const uint32_t wB = lds_u32(blk_addr<RV, SV>(vb, blk));
-                    const uint32_t wC = lds_u32(blk_addr<RV, SV>(vc, blk));
-                    const uint32_t wE = lds_u32(blk_addr<RV, SV>(ve, blk));
+                    const uint32_t wA = lds_u32(sbase, blk_addr<RV, SV>(va, blk));
+                    const uint32_t wB = lds_u32(sbase, blk_addr<RV, SV>(vb, blk));
+                    const uint32_t wC = lds_u32(sbase, blk_addr<RV, SV>(vc, blk));
+                    const uint32_t wE = lds_u32(sbase, blk_addr<RV, SV>(ve, blk));
 #pragma unroll
                     for (int h = 0; h < 2; h++) {
                         const uint32_t sel = h ? 0x7632u : 0x5410u;
@@ -653,10 +711,10 @@ __global__ void __launch_bounds__(NTHR, 2)
                         mma_16816(o_acc[2 * blk + h], a0, a1, a2, a3, b0, b1);
                     }
                 } else if constexpr (VB == 4) {
-                    const uint32_t hA = lds_u16(blk_addr<RV, SV>(va, blk));
-                    const uint32_t hB = lds_u16(blk_addr<RV, SV>(vb, blk));
-                    const uint32_t hC = lds_u16(blk_addr<RV, SV>(vc, blk));
-                    const uint32_t hE = lds_u16(blk_addr<RV, SV>(ve, blk));
+                    const uint32_t hA = lds_u16(sbase, blk_addr<RV, SV>(va, blk));
+                    const uint32_t hB = lds_u16(sbase, blk_addr<RV, SV>(vb, blk));
+                    const uint32_t hC = lds_u16(sbase, blk_addr<RV, SV>(vc, blk));
+                    const uint32_t hE = lds_u16(sbase, blk_addr<RV, SV>(ve, blk));
                     const uint32_t yAB = prmt(hA, hB, 0x5410u), yCE = prmt(hC, hE, 0x5410u);
 #pragma unroll
                     for (int h = 0; h < 2; h++) {
@@ -670,10 +728,10 @@ __global__ void __launch_bounds__(NTHR, 2)
                     // fp16 values past the length may be anything (NaN included): zero them
                     const int tg = m.t0 + warp * 32 + u * 16 + 2 * tig;
                     const uint2 z = make_uint2(0u, 0u);
-                    const uint2 wA = tg < m.len ? lds_u64(blk_addr<RV, SV>(va, blk)) : z;
-                    const uint2 wB = tg + 1 < m.len ? lds_u64(blk_addr<RV, SV>(vb, blk)) : z;
-                    const uint2 wC = tg + 8 < m.len ? lds_u64(blk_addr<RV, SV>(vc, blk)) : z;
-                    const uint2 wE = tg + 9 < m.len ? lds_u64(blk_addr<RV, SV>(ve, blk)) : z;
+                    const uint2 wA = tg < m.len ? lds_u64(sbase, blk_addr<RV, SV>(va, blk)) : z;
+                    const uint2 wB = tg + 1 < m.len ? lds_u64(sbase, blk_addr<RV, SV>(vb, blk)) : z;
+                    const uint2 wC = tg + 8 < m.len ? lds_u64(sbase, blk_addr<RV, SV>(vc, blk)) : z;
+                    const uint2 wE = tg + 9 < m.len ? lds_u64(sbase, blk_addr<RV, SV>(ve, blk)) : z;
 #pragma unroll
                     for (int h = 0; h < 2; h++) {
                         const uint32_t A = h ? wA.y : wA.x, Bw = h ? wB.y : wB.x;
