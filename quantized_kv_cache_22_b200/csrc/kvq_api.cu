@@ -485,6 +485,45 @@ int kvq_merge_partials(const kvq_config *cfg, const int32_t *d_len, void *out, i
                             num_ctas, reinterpret_cast<cudaStream_t>(stream), false, true);
 }
 
+static int h_reconstruct_impl(const kvq_config *cfg, const kvq_layer *layer, const void *w_kv,
+                              int32_t max_len_host, void *k_out, void *v_out,
+                              int32_t out_capacity, int *status, kvq_stream_t stream)
+{
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (cfg->mode != KVQ_MODE_H || !layer || !layer->k_codes || !w_kv || !k_out || !v_out)
+        return KVQ_ERR_INVALID_ARG;
+    if (cfg->n_kv_heads * cfg->head_dim != cfg->d_model) return KVQ_ERR_INVALID_ARG;
+    if (cfg->h_bits != 16 && !layer->k_scales) return KVQ_ERR_INVALID_ARG;
+    if (max_len_host < 0 || out_capacity < max_len_host || out_capacity % 64 != 0)
+        return KVQ_ERR_INVALID_ARG;
+    if (max_len_host > cfg->capacity) return KVQ_ERR_CAPACITY;
+    if (!aligned16(layer->k_codes) || !aligned16(w_kv) || !aligned16(k_out) ||
+        !aligned16(v_out) || (layer->k_scales && !aligned16(layer->k_scales)))
+        return KVQ_ERR_ALIGN;
+    if (cfg->head_dim != 128) return KVQ_ERR_UNSUPPORTED;
+    if (max_len_host == 0) return KVQ_OK;
+    HGemmParams p{};
+    p.h_codes = static_cast<const uint8_t *>(layer->k_codes);
+    p.h_scales = static_cast<const __half *>(layer->k_scales);
+    p.w = w_kv;
+    p.k_out = static_cast<__half *>(k_out);
+    p.v_out = static_cast<__half *>(v_out);
+    p.batch = cfg->batch;
+    p.cap = cfg->capacity;
+    p.d_model = cfg->d_model;
+    p.h_bits = cfg->h_bits;
+    p.h_groups = cfg->h_bits == 16 ? 1 : cfg->h_groups;
+    p.n_kv_heads = cfg->n_kv_heads;
+    p.head_dim = cfg->head_dim;
+    p.len = max_len_host;
+    p.out_cap = out_capacity;
+    p.status = status;
+    cudaError_t e = launch_h_reconstruct(p, reinterpret_cast<cudaStream_t>(stream));
+    if (e == cudaErrorNotSupported) return KVQ_ERR_UNSUPPORTED;
+    return e == cudaSuccess ? KVQ_OK : fail("reconstruction launch", e);
+}
+
 int kvq_decode_attn(const kvq_config *cfg, const kvq_layer *layer, const void *q, int32_t q_dtype,
                     const int32_t *d_len, int32_t max_len_host, float softmax_scale, void *out,
                     int32_t out_dtype, void *workspace, uint64_t workspace_bytes, int32_t num_ctas,
@@ -531,7 +570,8 @@ int kvq_decode_attn(const kvq_config *cfg, const kvq_layer *layer, const void *q
     }
     __half *kout = static_cast<__half *>(kv_scratch);
     __half *vout = kout + (size_t)cfg->batch * cfg->n_kv_heads * scap * cfg->head_dim;
-    rc = kvq_h_reconstruct(cfg, layer, w_kv, max_len_host, kout, vout, scap, stream);
+    rc = h_reconstruct_impl(cfg, layer, w_kv, max_len_host, kout, vout, scap,
+                            static_cast<int *>(workspace), stream);
     if (rc) return rc;
     return decode_kv_layout(cfg, kout, nullptr, vout, nullptr, scap, q, q_dtype, d_len,
                             softmax_scale, out, out_dtype, workspace, workspace_bytes, num_ctas, st,
@@ -542,38 +582,8 @@ int kvq_h_reconstruct(const kvq_config *cfg, const kvq_layer *layer, const void 
                       int32_t max_len_host, void *k_out, void *v_out, int32_t out_capacity,
                       kvq_stream_t stream)
 {
-    int rc = check_cfg(cfg);
-    if (rc) return rc;
-    if (cfg->mode != KVQ_MODE_H || !layer || !layer->k_codes || !w_kv || !k_out || !v_out)
-        return KVQ_ERR_INVALID_ARG;
-    if (cfg->n_kv_heads * cfg->head_dim != cfg->d_model) return KVQ_ERR_INVALID_ARG;
-    if (cfg->h_bits != 16 && !layer->k_scales) return KVQ_ERR_INVALID_ARG;
-    if (max_len_host < 0 || out_capacity < max_len_host || out_capacity % 64 != 0)
-        return KVQ_ERR_INVALID_ARG;
-    if (max_len_host > cfg->capacity) return KVQ_ERR_CAPACITY;
-    if (!aligned16(layer->k_codes) || !aligned16(w_kv) || !aligned16(k_out) ||
-        !aligned16(v_out) || (layer->k_scales && !aligned16(layer->k_scales)))
-        return KVQ_ERR_ALIGN;
-    if (cfg->head_dim != 128) return KVQ_ERR_UNSUPPORTED;
-    if (max_len_host == 0) return KVQ_OK;
-    HGemmParams p{};
-    p.h_codes = static_cast<const uint8_t *>(layer->k_codes);
-    p.h_scales = static_cast<const __half *>(layer->k_scales);
-    p.w = w_kv;
-    p.k_out = static_cast<__half *>(k_out);
-    p.v_out = static_cast<__half *>(v_out);
-    p.batch = cfg->batch;
-    p.cap = cfg->capacity;
-    p.d_model = cfg->d_model;
-    p.h_bits = cfg->h_bits;
-    p.h_groups = cfg->h_bits == 16 ? 1 : cfg->h_groups;
-    p.n_kv_heads = cfg->n_kv_heads;
-    p.head_dim = cfg->head_dim;
-    p.len = max_len_host;
-    p.out_cap = out_capacity;
-    cudaError_t e = launch_h_reconstruct(p, reinterpret_cast<cudaStream_t>(stream));
-    if (e == cudaErrorNotSupported) return KVQ_ERR_UNSUPPORTED;
-    return e == cudaSuccess ? KVQ_OK : fail("reconstruction launch", e);
+    return h_reconstruct_impl(cfg, layer, w_kv, max_len_host, k_out, v_out, out_capacity, nullptr,
+                              stream);
 }
 
 int kvq_workspace_status(void *workspace, int32_t *status, kvq_stream_t stream)

@@ -1,13 +1,480 @@
-// kvq_hgemm.cu -- h-mode K/V reconstruction GEMM (tcgen05).  Not built yet:
-// the launcher reports cudaErrorNotSupported, which the ABI maps to
-// KVQ_ERR_UNSUPPORTED.
+// kvq_hgemm.cu -- h-mode K/V reconstruction GEMM on 5th-generation tensor cores.
+//
+// TinyLoop docs, "KV Cache 模式", section "運作原理": in h-mode the cache holds
+// h = LN(residual) and every attention call rebuilds K = W_k h and V = W_v h for
+// all cached positions, skipping the Q slice of attn_qkv; the page moves this GEMM
+// from a scalar path to tensor cores.  Here, for every sequence b and token t:
+//     [K_t | V_t] = W_kv . bf16(h^_t),   h^ = code * scale (dequantised in the
+//     operand prologue), fp32 accumulation, rounded to fp16,
+// written to K/V [B][Hkv][out_cap][Dh], the layout the 16-bit decode kernel reads.
+//
+// One CTA computes a 128 (tokens) x 256 (output features) tile:
+//   warp 0      TMA producer: W tile (bf16, 128-byte swizzle) and the raw h codes
+//               of each 64-wide K stage into a ring of shared-memory stages;
+//   warp 1      allocates 256 TMEM columns and, from one lane, issues
+//               tcgen05.mma (M=128, N=256, K=16, bf16 x bf16 -> fp32) four times
+//               per stage, committing each stage to its "empty" mbarrier;
+//   warps 2..5  dequantise the raw codes of each stage into the K-major,
+//               128-byte-swizzled bf16 A tile (generic stores + proxy fence),
+//               then read the accumulator back (tcgen05.ld, 32 lanes each) and
+//               store fp16 K/V rows.
+// Every wait is bounded; a give-up sets *status and the CTA drains and frees its
+// TMEM before returning.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
 #include "kvq_internal.h"
+#include "kvq_ptx.cuh"
+#include "../../include/kvq.h"
 
 namespace kvq {
+namespace {
 
-cudaError_t launch_h_reconstruct(const HGemmParams &, cudaStream_t)
+constexpr int BM = 128, BN = 256, BK = 64;
+constexpr int NTHREADS = 192;                    // 6 warps
+constexpr uint32_t A_BYTES = BM * BK * 2;        // 16 KB
+constexpr uint32_t B_BYTES = BN * BK * 2;        // 32 KB
+constexpr uint32_t TMEM_COLS = 256;
+
+struct GemmArgs {
+    const __half *h_scales;   // [B][cap][h_groups] (null at 16 bits)
+    __half *k_out, *v_out;    // [B][Hkv][out_cap][Dh]
+    int *status;              // may be null
+    int32_t cap, d_model, h_bits, h_groups, n_kv_heads, head_dim, len, out_cap, m_tiles;
+    uint32_t raw_bytes, stage_bytes, stages;
+    uint64_t timeout_ns;
+};
+
+// ------------------------------------------------------------ tcgen05 helpers
+__device__ __forceinline__ void tmem_alloc(uint32_t *slot, uint32_t cols)
 {
-    return cudaErrorNotSupported;
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(slot)),
+                 "r"(cols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16 (bf16 operands here).
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t accumulate)
+{
+    uint32_t mask[4] = {0, 0, 0, 0};
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(
+            d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(mask[0]), "r"(mask[1]),
+        "r"(mask[2]), "r"(mask[3])
+        : "memory");
+}
+
+// Arrive on `bar` once every tcgen05.mma issued so far by this thread completes.
+__device__ __forceinline__ void umma_commit(uint64_t *bar)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
+        "%29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row atoms of
+// 1024 bytes (stride-dimension offset), start address in 16-byte units.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);          // start address
+    d |= (uint64_t)1u << 16;                             // leading offset (unused here)
+    d |= (uint64_t)(1024u >> 4) << 32;                   // stride offset: 8 rows x 128 B
+    d |= (uint64_t)1u << 46;                             // descriptor version (sm_100)
+    d |= (uint64_t)2u << 61;                             // layout: 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor: D f32, A/B bf16, both K-major, M = 128, N = 256.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                            ((uint32_t)(BM >> 4) << 24);
+
+// byte offset of bf16 element e (0..63) of row r in a K-major 128-byte-swizzled tile
+__device__ __forceinline__ uint32_t a_off(int r, int chunk16)
+{
+    return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((chunk16 ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ uint32_t bf2(float lo, float hi)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    hgemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_h,
+                 const GemmArgs g)
+{
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t S = g.stages;
+    // stage s: [A 16 KB][B 32 KB][raw codes] ; barriers after the ring
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + S * g.stage_bytes);
+    uint64_t *tma_full = bars;           // W + raw codes landed (TMA tx)
+    uint64_t *a_full = bars + S;         // A tile written (4 converter warps)
+    uint64_t *empty = bars + 2 * S;      // MMAs of the stage finished (tcgen05.commit)
+    uint64_t *acc_full = bars + 3 * S;   // all MMAs finished
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * S + 1);
+    int *abort_flag_p = reinterpret_cast<int *>(tmem_slot + 1);
+    volatile int *abort_flag = abort_flag_p;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * BN;
+    const int b = blockIdx.y / g.m_tiles;
+    const int t0 = (blockIdx.y % g.m_tiles) * BM;
+    const int k_stages = g.d_model / BK;
+    const uint64_t limit = g.timeout_ns;
+
+    if (threadIdx.x == 0) {
+        for (uint32_t s = 0; s < S; s++) {
+            mbar_init(&tma_full[s], 1);
+            mbar_init(&a_full[s], 4);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        *abort_flag_p = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    auto give_up = [&]() {
+        *abort_flag_p = 1;
+        if (g.status) atomicExch(g.status, KVQ_ERR_TIMEOUT);
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            prefetch_tensormap(&tm_w);
+            prefetch_tensormap(&tm_h);
+            uint32_t s = 0, ph = 0;
+            int issued = 0;
+            const int raw_x = BK * g.h_bits / 8;   // raw bytes of one row per stage
+            for (int k = 0; k < k_stages; k++) {
+                if (k >= (int)S && !mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, limit)) {
+                    give_up();
+                    break;
+                }
+                uint8_t *st = smem + s * g.stage_bytes;
+                mbar_arrive_expect_tx(&tma_full[s], B_BYTES + g.raw_bytes);
+                tma_load_2d(st + A_BYTES, &tm_w, &tma_full[s], k * BK, n0);
+                tma_load_3d(st + A_BYTES + B_BYTES, &tm_h, &tma_full[s], k * raw_x, t0, b);
+                issued = k + 1;
+                if (++s == S) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+            // drain: every issued copy must land before the CTA can exit
+            uint32_t ss = s, pp = ph;
+            for (int j = 0; j < min((int)S, issued); j++) {
+                if (ss == 0) {
+                    ss = S;
+                    pp ^= 1u;
+                }
+                --ss;
+                (void)mbar_wait_bounded(&tma_full[ss], pp, abort_flag, limit);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            uint32_t s = 0, ph = 0;
+            int issued = 0;
+            for (int k = 0; k < k_stages; k++) {
+                if (!mbar_wait_bounded(&tma_full[s], ph, abort_flag, limit) ||
+                    !mbar_wait_bounded(&a_full[s], ph, abort_flag, limit)) {
+                    give_up();
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a_base = smem_u32(smem + s * g.stage_bytes);
+                const uint32_t b_base = a_base + A_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; kk++) {
+                    // K = 16 bf16 = 32 bytes further inside the 128-byte swizzle atom
+                    umma_f16(tmem, sw128_desc(a_base + kk * 32), sw128_desc(b_base + kk * 32),
+                             kIdesc, (k > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(&empty[s]);
+                issued = k + 1;
+                if (++s == S) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+            if (issued == k_stages) {
+                umma_commit(acc_full);
+            } else if (issued > 0) {
+                // aborted: wait (bounded) for the MMAs already issued to retire
+                uint32_t ss = s, pp = ph;
+                if (ss == 0) {
+                    ss = S;
+                    pp ^= 1u;
+                }
+                --ss;
+                (void)mbar_wait_bounded(&empty[ss], pp, abort_flag, limit);
+            }
+        }
+    } else {
+        // ------------------------------------------------ converters, then epilogue
+        const int r = threadIdx.x - 64;            // 0..127: tile row handled by this thread
+        const int t = t0 + r;
+        const int gsz = g.d_model / g.h_groups;   // elements per h scale group
+        const bool live = t < g.len;
+        // scales of the two 32-element blocks of stage k, fetched one stage ahead
+        auto load_scales = [&](int k, float (&o)[2]) {
+#pragma unroll
+            for (int q = 0; q < 2; q++) {
+                const int e = k * BK + 32 * q;
+                o[q] = live ? __half2float(g.h_scales[((int64_t)b * g.cap + t) * g.h_groups + e / gsz])
+                            : 0.f;
+            }
+        };
+        float sc_next[2] = {0.f, 0.f};
+        if (g.h_bits != 16) load_scales(0, sc_next);
+        uint32_t s = 0, ph = 0;
+        bool ok = true;
+        for (int k = 0; k < k_stages && ok; k++) {
+            const float sc[2] = {sc_next[0], sc_next[1]};
+            if (g.h_bits != 16 && k + 1 < k_stages) load_scales(k + 1, sc_next);
+            if (!mbar_wait_bounded(&tma_full[s], ph, abort_flag, limit)) {
+                give_up();
+                ok = false;
+                break;
+            }
+            uint8_t *st = smem + s * g.stage_bytes;
+            const uint8_t *raw = st + A_BYTES + B_BYTES + (size_t)r * (BK * g.h_bits / 8);
+            uint8_t *arow = st;
+            if (g.h_bits == 16) {
+                // fp16 h: bf16(h), 8 elements per 16-byte chunk
+#pragma unroll
+                for (int c = 0; c < 8; c++) {
+                    uint4 x = *reinterpret_cast<const uint4 *>(raw + 16 * c);
+                    const __half2 *hx = reinterpret_cast<const __half2 *>(&x);
+                    uint4 o;
+                    uint32_t *ow = reinterpret_cast<uint32_t *>(&o);
+#pragma unroll
+                    for (int j = 0; j < 4; j++) {
+                        const float2 f = __half22float2(hx[j]);
+                        ow[j] = live ? bf2(f.x, f.y) : 0u;
+                    }
+                    *reinterpret_cast<uint4 *>(arow + a_off(r, c)) = o;
+                }
+            } else {
+                if (g.h_bits == 8) {
+#pragma unroll
+                    for (int c = 0; c < 8; c++) {
+                        const uint2 x = *reinterpret_cast<const uint2 *>(raw + 8 * c);
+                        const float sv = sc[c >> 2];
+                        uint4 o;
+                        const uint32_t w[2] = {x.x, x.y};
+                        uint32_t *ow = reinterpret_cast<uint32_t *>(&o);
+#pragma unroll
+                        for (int j = 0; j < 4; j++) {
+                            const uint32_t ww = w[j >> 1];
+                            const int sh = (j & 1) * 16;
+                            const float lo = (float)(int8_t)((ww >> sh) & 0xff);
+                            const float hi = (float)(int8_t)((ww >> (sh + 8)) & 0xff);
+                            ow[j] = bf2(lo * sv, hi * sv);
+                        }
+                        *reinterpret_cast<uint4 *>(arow + a_off(r, c)) = o;
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 8; c++) {
+                        const uint32_t x = *reinterpret_cast<const uint32_t *>(raw + 4 * c);
+                        const float sv = sc[c >> 2];
+                        uint4 o;
+                        uint32_t *ow = reinterpret_cast<uint32_t *>(&o);
+#pragma unroll
+                        for (int j = 0; j < 4; j++) {
+                            // element 2j in the low nibble of byte j, 2j+1 in the high nibble
+                            const int lo = (int)((x >> (8 * j)) & 0xf), hi = (int)((x >> (8 * j + 4)) & 0xf);
+                            const float flo = (float)(lo >= 8 ? lo - 16 : lo);
+                            const float fhi = (float)(hi >= 8 ? hi - 16 : hi);
+                            ow[j] = bf2(flo * sv, fhi * sv);
+                        }
+                        *reinterpret_cast<uint4 *>(arow + a_off(r, c)) = o;
+                    }
+                }
+            }
+            fence_proxy_async_smem();   // generic-proxy stores -> async-proxy MMA reads
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&a_full[s]);
+            if (++s == S) {
+                s = 0;
+                ph ^= 1u;
+            }
+        }
+        // ---------------- epilogue: TMEM -> fp16 K/V rows
+        if (ok && mbar_wait_bounded(acc_full, 0, abort_flag, limit)) {
+            tc_fence_after();
+            const int q = warp & 3;                       // TMEM lane quarter of this warp
+            const int row = 32 * q + lane;                // accumulator row = tile row
+            const int tt = t0 + row;
+            const int hd = g.n_kv_heads * g.head_dim;     // features of K (then of V)
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
+                if (tt < g.len) {
+                    const int n = n0 + c0;
+                    __half *dst = n < hd ? g.k_out : g.v_out;
+                    const int nn = n < hd ? n : n - hd;
+                    const int head = nn / g.head_dim, d = nn % g.head_dim;
+                    __half *p = dst + (((int64_t)b * g.n_kv_heads + head) * g.out_cap + tt) * g.head_dim + d;
+#pragma unroll
+                    for (int j = 0; j < 32; j += 8) {
+                        uint4 o;
+                        o.x = pack_half2(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+                        o.y = pack_half2(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+                        o.z = pack_half2(__uint_as_float(v[j + 4]), __uint_as_float(v[j + 5]));
+                        o.w = pack_half2(__uint_as_float(v[j + 6]), __uint_as_float(v[j + 7]));
+                        *reinterpret_cast<uint4 *>(p + j) = o;
+                    }
+                }
+            }
+        } else if (ok) {
+            give_up();
+        }
+    }
+
+    // every role reaches this point; free TMEM after all tcgen05 work is done
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+}  // namespace
+
+cudaError_t launch_h_reconstruct(const HGemmParams &p, cudaStream_t stream)
+{
+    const int N = 2 * p.n_kv_heads * p.head_dim;
+    if (p.head_dim % 32 != 0 || N % BN != 0 || p.d_model % BK != 0) return cudaErrorNotSupported;
+    if (p.h_bits != 16 && (p.d_model / p.h_groups) % 32 != 0) return cudaErrorNotSupported;
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+
+    // W: bf16 [N][D], boxes of 64 (K) x 256 (N) with 128-byte swizzle
+    CUtensorMap tm_w, tm_h;
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)p.d_model, (cuuint64_t)N};
+        cuuint64_t strides[1] = {(cuuint64_t)p.d_model * 2};
+        cuuint32_t box[2] = {BK, BN}, es[2] = {1, 1};
+        if (fn(&tm_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(p.w), dims, strides,
+               box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    // h codes: bytes [B][cap][D*bits/8], boxes of (64 elements of codes) x 128 tokens
+    const uint32_t row_bytes = (uint32_t)p.d_model * p.h_bits / 8;
+    const uint32_t raw_x = BK * p.h_bits / 8;
+    {
+        cuuint64_t dims[3] = {row_bytes, (cuuint64_t)p.cap, (cuuint64_t)p.batch};
+        cuuint64_t strides[2] = {row_bytes, (cuuint64_t)row_bytes * p.cap};
+        cuuint32_t box[3] = {raw_x, BM, 1}, es[3] = {1, 1, 1};
+        if (fn(&tm_h, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t *>(p.h_codes), dims,
+               strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    GemmArgs g{};
+    g.h_scales = p.h_scales;
+    g.k_out = p.k_out;
+    g.v_out = p.v_out;
+    g.status = p.status;
+    g.cap = p.cap;
+    g.d_model = p.d_model;
+    g.h_bits = p.h_bits;
+    g.h_groups = p.h_groups;
+    g.n_kv_heads = p.n_kv_heads;
+    g.head_dim = p.head_dim;
+    g.len = p.len;
+    g.out_cap = p.out_cap;
+    g.m_tiles = (p.len + BM - 1) / BM;
+    g.raw_bytes = raw_x * BM;
+    g.stage_bytes = ((A_BYTES + B_BYTES + g.raw_bytes) + 1023u) / 1024u * 1024u;
+    const uint32_t budget = 220u * 1024u;
+    g.stages = budget / g.stage_bytes;
+    if (g.stages > 4) g.stages = 4;
+    if (g.stages < 2) return cudaErrorNotSupported;
+    g.timeout_ns = 1000000000ull;
+    const size_t smem = (size_t)g.stages * g.stage_bytes + 1024 + 3 * 8 * g.stages + 64;
+
+    cudaError_t e = cudaFuncSetAttribute(hgemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    const dim3 grid(N / BN, (unsigned)(g.m_tiles * p.batch));
+    void *args[] = {&tm_w, &tm_h, &g};
+    (void)cudaGetLastError();
+    return cudaLaunchKernel(reinterpret_cast<void *>(&hgemm_kernel), grid, dim3(NTHREADS), args,
+                            smem, stream);
 }
 
 }  // namespace kvq
