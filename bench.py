@@ -49,6 +49,33 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+def bf16_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), float(d["bf16_tflops_sustained"]), "measured"
+    return 1590.0, 1400.0, "fallback"
+
+
+def decode_traffic(variant: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was taken on
+    the current decode kernel source (sha256 of kvq_decode.cu); otherwise None."""
+    import hashlib
+    f = os.path.join(ROOT, "profiles", "decode_kernel_traffic.txt")
+    src = os.path.join(ROOT, "quantized_kv_cache_22_b200", "csrc", "kvq_decode.cu")
+    if not os.path.exists(f):
+        return None
+    vals = {}
+    for line in open(f):
+        parts = line.split()
+        if len(parts) == 2 and not line.startswith("#"):
+            vals[parts[0]] = parts[1]
+    if vals.get("sha256") != hashlib.sha256(open(src, "rb").read()).hexdigest():
+        return None
+    return float(vals[variant]) if variant in vals else None
+
+
 def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -317,6 +344,65 @@ def cpu_oracle_layer(w, fmt, st=None, device=None, reps=1):
     return times, cores
 
 
+def run_hmode(args, world, device):
+    """h-mode workload: INT4-h cache of B=8 x 1024 tokens, D=2048, 16 heads x 128;
+    one call = rebuild K/V with the tcgen05 GEMM (137.4 GFLOP) + decode attention."""
+    import torch
+    import quantized_kv_cache_22_b200 as kvq
+    from quantized_kv_cache_22_b200 import Config, LayerCache, Workspace, inputs
+
+    w = inputs.WORKLOADS[5]
+    S, D, H = w.context, w.d_model, w.n_kv_heads
+    cfg = Config(batch=w.batch, capacity=w.capacity, mode=kvq.KVQ_MODE_H, d_model=D, h_bits=4,
+                 h_groups=16, n_q_heads=w.n_q_heads, n_kv_heads=H, head_dim=w.head_dim)
+    h, W = inputs.hmode_inputs(w, S, device)
+    cache = LayerCache(cfg, device)
+    kvq.kvq_append(cfg, cache, h, None, torch.zeros(w.batch, dtype=torch.int32, device=device), 0, S)
+    del h
+    q = inputs.queries(w, 0, 0, device)
+    out = torch.empty_like(q)
+    ws = Workspace(cfg, 0, device)
+    scratch = torch.empty(kvq.kvq_h_scratch_bytes(cfg, S) // 2, dtype=torch.float16, device=device)
+    nkv = w.batch * H * S * w.head_dim
+    k_out = scratch[:nkv].view(w.batch, H, S, w.head_dim)
+    v_out = scratch[nkv:2 * nkv].view(w.batch, H, S, w.head_dim)
+    d_len = torch.full((w.batch,), S, dtype=torch.int32, device=device)
+    flops = 2.0 * w.batch * S * (2 * H * w.head_dim) * D
+
+    operand = torch.empty(kvq.kvq_h_operand_bytes(cfg, S) // 2, dtype=torch.bfloat16, device=device)
+
+    def gemm():
+        kvq.kvq_h_reconstruct(cfg, cache, W, S, k_out, v_out, S, operand)
+
+    def step():
+        kvq.kvq_decode_attn(cfg, cache, q, d_len, S, out, ws, w_kv=W, kv_scratch=scratch)
+
+    res = {"workload": w.name, "h_bits": 4, "gflop_per_call": round(flops / 1e9, 2)}
+    for name, fn in (("gemm", gemm), ("step", step)):
+        for _ in range(max(args.warmup, 3)):
+            fn()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        n = max(3, min(args.steps, 100))
+        a.record()
+        for _ in range(n):
+            fn()
+        b.record()
+        b.synchronize()
+        res[f"{name}_ms"] = round(reduce_max(a.elapsed_time(b) / n, world, device), 5)
+    assert kvq.kvq_workspace_status(ws) == 0
+    burst, sustained, kind = bf16_peaks()
+    tf = flops / (res["gemm_ms"] * 1e-3) / 1e12
+    res["gemm_tflops"] = round(tf, 1)
+    res["roofline"] = {"bound": "tensor", "kernel": "hgemm_kernel (tcgen05 bf16, fp32 acc)",
+                       "achieved": round(tf, 1), "peak": burst, "peak_kind": kind + " burst",
+                       "unit": "TFLOP/s", "frac": round(tf / burst, 4),
+                       "frac_of_sustained": round(tf / sustained, 4)}
+    res["steps_per_s"] = round(world * 1e3 / res["step_ms"], 2)
+    return res
+
+
 def run_gpu(args):
     import torch
     import quantized_kv_cache_22_b200 as kvq
@@ -339,7 +425,8 @@ def run_gpu(args):
 
     results = {}
     main_state = None
-    for name in args.variants:
+    variants = args.variants if "kv" in args.sections else []
+    for name in variants:
         fmt = VARIANTS[name]
         st = build_variant(w, fmt, device)
         g, ev_s, ev_e, _ = capture_step(w, st)
@@ -375,6 +462,11 @@ def run_gpu(args):
             torch.cuda.synchronize()
             torch.cuda.empty_cache()
 
+    hmode = run_hmode(args, world, device) if "hmode" in args.sections else None
+    if not variants:
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": None, "hmode": hmode}), flush=True)
+        return
     head = args.variants[0]
     r = results[head]
     line = {
@@ -402,13 +494,14 @@ def run_gpu(args):
                      "achieved": round(r["decode_kernel_gbs"], 1), "peak": hbm_peak,
                      "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(r["decode_kernel_gbs"] / hbm_peak, 4),
-                     "traffic": args.traffic_bytes,
+                     "traffic": args.traffic_bytes if args.traffic_bytes else decode_traffic(head),
                      "bytes_per_launch": r["kv_bytes_per_step"] // w.n_layers,
                      "launch_ms": round(r["decode_kernel_ms"], 5)},
         "variants": {k: {kk: (round(vv, 4) if isinstance(vv, float) else vv)
                          for kk, vv in v.items() if kk not in ("clocks", "e2e")}
                      for k, v in results.items()},
         "gpu_launches": args.steps * 3 * w.n_layers,
+        "hmode": hmode,
         "clocks": r["clocks"],
     }
     if "e2e" in r:
@@ -479,6 +572,8 @@ def main():
     ap.add_argument("--variants", default="K8V8,K8V4,K4V4")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--sections", default="kv,hmode",
+                    help="kv: the 8K K/V decode step (headline); hmode: the h-mode workload")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the layer count (small profiling captures only)")
     ap.add_argument("--traffic-bytes", type=float, default=None,

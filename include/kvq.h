@@ -165,9 +165,14 @@ KVQ_API int kvq_append(const kvq_config *cfg, const kvq_layer *layer, const void
  * device; pass an explicit count to size it without one). */
 KVQ_API int kvq_workspace_bytes(const kvq_config *cfg, int32_t num_ctas, uint64_t *bytes);
 
-/* h-mode scratch bytes: reconstructed fp16 K and V for up to max_len
- * tokens of every sequence ([2][B][Hkv][round_up(max_len,64)][Dh]). */
+/* h-mode scratch bytes for kvq_decode_attn: the reconstructed fp16 K and V for
+ * up to max_len tokens of every sequence ([2][B][Hkv][round_up(max_len,64)][Dh]),
+ * followed by the bf16 GEMM operand (kvq_h_operand_bytes). */
 KVQ_API int kvq_h_scratch_bytes(const kvq_config *cfg, int32_t max_len, uint64_t *bytes);
+
+/* Bytes of the bf16 operand buffer kvq_h_reconstruct needs: the dequantised
+ * h^ of every sequence, [B][round_up(max_len,128)][D] bf16. */
+KVQ_API int kvq_h_operand_bytes(const kvq_config *cfg, int32_t max_len, uint64_t *bytes);
 
 /* Decode attention for one query token per sequence (split-KV, dequantised in
  * registers).  [MNI]: the new token's query attends over every cached K/V;
@@ -222,11 +227,15 @@ KVQ_API int kvq_merge_partials(const kvq_config *cfg, const int32_t *d_len, void
  * path replaces the scalar one): for every sequence b and token t < len,
  *   [K_t | V_t] = W_kv . bf16(h^_t)   (fp32 accumulation, rounded to fp16)
  * written to k_out / v_out, each [B][Hkv][out_capacity][Dh] fp16, with
- * len = max_len_host for every sequence.  out_capacity is a multiple of 64
- * and >= max_len_host.  Errors as kvq_decode_attn. */
+ * len = max_len_host for every sequence (rows t >= len are not written).
+ * out_capacity is a multiple of 64 and >= max_len_host.  `operand` is device
+ * scratch of at least kvq_h_operand_bytes(cfg, max_len_host) bytes that
+ * receives bf16(h^) first (contents on entry do not matter).
+ * Errors as kvq_decode_attn. */
 KVQ_API int kvq_h_reconstruct(const kvq_config *cfg, const kvq_layer *layer, const void *w_kv,
-                      int32_t max_len_host, void *k_out, void *v_out, int32_t out_capacity,
-                      kvq_stream_t stream);
+                              int32_t max_len_host, void *k_out, void *v_out,
+                              int32_t out_capacity, void *operand, uint64_t operand_bytes,
+                              kvq_stream_t stream);
 
 /* Read and clear the device status word a decode launch leaves in its
  * workspace: KVQ_OK, or KVQ_ERR_TIMEOUT if a kernel gave up a bounded wait

@@ -24,7 +24,7 @@ KVQ_F16, KVQ_F32, KVQ_BF16 = 0, 1, 2
 EXPORTED = ("kvq_cache_bytes", "kvq_layer_buffer_bytes", "kvq_append", "kvq_workspace_bytes",
             "kvq_h_scratch_bytes", "kvq_decode_attn", "kvq_decode_partials", "kvq_merge_partials",
             "kvq_h_reconstruct", "kvq_workspace_status", "kvq_status_string",
-            "kvq_last_error_detail", "kvq_decode_attn_noalloc")
+            "kvq_last_error_detail", "kvq_decode_attn_noalloc", "kvq_h_operand_bytes")
 
 
 class KvqError(RuntimeError):
@@ -63,7 +63,8 @@ def _load():
                             u64, P],
         "kvq_decode_partials": [cfgp, layp, P, i32, P, i32, ctypes.c_float, P, u64, i32, P],
         "kvq_merge_partials": [cfgp, P, P, i32, P, u64, i32, P],
-        "kvq_h_reconstruct": [cfgp, layp, P, i32, P, P, i32, P],
+        "kvq_h_operand_bytes": [cfgp, i32, pu64],
+        "kvq_h_reconstruct": [cfgp, layp, P, i32, P, P, i32, P, u64, P],
         "kvq_workspace_status": [P, ctypes.POINTER(i32), P],
     }
     for name, args in sig.items():
@@ -228,11 +229,20 @@ def kvq_merge_partials(cfg: Config, d_len: torch.Tensor, out: torch.Tensor, ws: 
                                    _ptr(ws.buf), ws.nbytes, int(num_ctas), _stream(stream)))
 
 
+def kvq_h_operand_bytes(cfg: Config, max_len: int) -> int:
+    v = ctypes.c_uint64()
+    _check("kvq_h_operand_bytes", _lib.kvq_h_operand_bytes(ctypes.byref(cfg.c()), max_len,
+                                                           ctypes.byref(v)))
+    return v.value
+
+
 def kvq_h_reconstruct(cfg: Config, layer: LayerCache, w_kv: torch.Tensor, max_len: int,
-                      k_out: torch.Tensor, v_out: torch.Tensor, out_capacity: int, stream=None):
+                      k_out: torch.Tensor, v_out: torch.Tensor, out_capacity: int,
+                      operand: torch.Tensor, stream=None):
     _check("kvq_h_reconstruct",
            _lib.kvq_h_reconstruct(ctypes.byref(cfg.c()), ctypes.byref(layer.c()), _ptr(w_kv),
                                   int(max_len), _ptr(k_out), _ptr(v_out), int(out_capacity),
+                                  _ptr(operand), operand.numel() * operand.element_size(),
                                   _stream(stream)))
 
 

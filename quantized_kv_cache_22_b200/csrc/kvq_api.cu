@@ -352,14 +352,35 @@ int kvq_workspace_bytes(const kvq_config *cfg, int32_t num_ctas, uint64_t *bytes
     return KVQ_OK;
 }
 
+static uint64_t h_operand_need(const kvq_config *cfg, int32_t max_len)
+{
+    const uint64_t pad = ((uint64_t)max_len + kHTileTokens - 1) / kHTileTokens * kHTileTokens;
+    return (uint64_t)cfg->batch * pad * (uint64_t)cfg->d_model * 2;
+}
+
+static uint64_t h_kv_need(const kvq_config *cfg, int32_t max_len)
+{
+    const uint64_t cap = ((uint64_t)max_len + 63) / 64 * 64;
+    return 2ull * cfg->batch * cfg->n_kv_heads * cap * cfg->head_dim * 2;
+}
+
 int kvq_h_scratch_bytes(const kvq_config *cfg, int32_t max_len, uint64_t *bytes)
 {
     int rc = check_cfg(cfg);
     if (rc) return rc;
     if (cfg->mode != KVQ_MODE_H || !bytes || max_len < 0) return KVQ_ERR_INVALID_ARG;
     if (max_len > cfg->capacity) return KVQ_ERR_CAPACITY;
-    const uint64_t cap = ((uint64_t)max_len + 63) / 64 * 64;
-    *bytes = 2ull * cfg->batch * cfg->n_kv_heads * cap * cfg->head_dim * 2;
+    *bytes = h_kv_need(cfg, max_len) + h_operand_need(cfg, max_len);
+    return KVQ_OK;
+}
+
+int kvq_h_operand_bytes(const kvq_config *cfg, int32_t max_len, uint64_t *bytes)
+{
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (cfg->mode != KVQ_MODE_H || !bytes || max_len < 0) return KVQ_ERR_INVALID_ARG;
+    if (max_len > cfg->capacity) return KVQ_ERR_CAPACITY;
+    *bytes = h_operand_need(cfg, max_len);
     return KVQ_OK;
 }
 
@@ -487,11 +508,13 @@ int kvq_merge_partials(const kvq_config *cfg, const int32_t *d_len, void *out, i
 
 static int h_reconstruct_impl(const kvq_config *cfg, const kvq_layer *layer, const void *w_kv,
                               int32_t max_len_host, void *k_out, void *v_out,
-                              int32_t out_capacity, int *status, kvq_stream_t stream)
+                              int32_t out_capacity, void *operand, uint64_t operand_bytes,
+                              int *status, kvq_stream_t stream)
 {
     int rc = check_cfg(cfg);
     if (rc) return rc;
-    if (cfg->mode != KVQ_MODE_H || !layer || !layer->k_codes || !w_kv || !k_out || !v_out)
+    if (cfg->mode != KVQ_MODE_H || !layer || !layer->k_codes || !w_kv || !k_out || !v_out ||
+        !operand)
         return KVQ_ERR_INVALID_ARG;
     if (cfg->n_kv_heads * cfg->head_dim != cfg->d_model) return KVQ_ERR_INVALID_ARG;
     if (cfg->h_bits != 16 && !layer->k_scales) return KVQ_ERR_INVALID_ARG;
@@ -499,9 +522,11 @@ static int h_reconstruct_impl(const kvq_config *cfg, const kvq_layer *layer, con
         return KVQ_ERR_INVALID_ARG;
     if (max_len_host > cfg->capacity) return KVQ_ERR_CAPACITY;
     if (!aligned16(layer->k_codes) || !aligned16(w_kv) || !aligned16(k_out) ||
-        !aligned16(v_out) || (layer->k_scales && !aligned16(layer->k_scales)))
+        !aligned16(v_out) || !aligned16(operand) ||
+        (layer->k_scales && !aligned16(layer->k_scales)))
         return KVQ_ERR_ALIGN;
     if (cfg->head_dim != 128) return KVQ_ERR_UNSUPPORTED;
+    if (operand_bytes < h_operand_need(cfg, max_len_host)) return KVQ_ERR_WORKSPACE;
     if (max_len_host == 0) return KVQ_OK;
     HGemmParams p{};
     p.h_codes = static_cast<const uint8_t *>(layer->k_codes);
@@ -518,6 +543,7 @@ static int h_reconstruct_impl(const kvq_config *cfg, const kvq_layer *layer, con
     p.head_dim = cfg->head_dim;
     p.len = max_len_host;
     p.out_cap = out_capacity;
+    p.operand = operand;
     p.status = status;
     cudaError_t e = launch_h_reconstruct(p, reinterpret_cast<cudaStream_t>(stream));
     if (e == cudaErrorNotSupported) return KVQ_ERR_UNSUPPORTED;
@@ -570,8 +596,10 @@ int kvq_decode_attn(const kvq_config *cfg, const kvq_layer *layer, const void *q
     }
     __half *kout = static_cast<__half *>(kv_scratch);
     __half *vout = kout + (size_t)cfg->batch * cfg->n_kv_heads * scap * cfg->head_dim;
-    rc = h_reconstruct_impl(cfg, layer, w_kv, max_len_host, kout, vout, scap,
-                            static_cast<int *>(workspace), stream);
+    uint8_t *operand = static_cast<uint8_t *>(kv_scratch) + h_kv_need(cfg, max_len_host);
+    rc = h_reconstruct_impl(cfg, layer, w_kv, max_len_host, kout, vout, scap, operand,
+                            h_operand_need(cfg, max_len_host), static_cast<int *>(workspace),
+                            stream);
     if (rc) return rc;
     return decode_kv_layout(cfg, kout, nullptr, vout, nullptr, scap, q, q_dtype, d_len,
                             softmax_scale, out, out_dtype, workspace, workspace_bytes, num_ctas, st,
@@ -580,10 +608,10 @@ int kvq_decode_attn(const kvq_config *cfg, const kvq_layer *layer, const void *q
 
 int kvq_h_reconstruct(const kvq_config *cfg, const kvq_layer *layer, const void *w_kv,
                       int32_t max_len_host, void *k_out, void *v_out, int32_t out_capacity,
-                      kvq_stream_t stream)
+                      void *operand, uint64_t operand_bytes, kvq_stream_t stream)
 {
-    return h_reconstruct_impl(cfg, layer, w_kv, max_len_host, k_out, v_out, out_capacity, nullptr,
-                              stream);
+    return h_reconstruct_impl(cfg, layer, w_kv, max_len_host, k_out, v_out, out_capacity, operand,
+                              operand_bytes, nullptr, stream);
 }
 
 int kvq_workspace_status(void *workspace, int32_t *status, kvq_stream_t stream)

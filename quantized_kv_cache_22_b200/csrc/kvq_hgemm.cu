@@ -8,18 +8,21 @@
 //     operand prologue), fp32 accumulation, rounded to fp16,
 // written to K/V [B][Hkv][out_cap][Dh], the layout the 16-bit decode kernel reads.
 //
-// One CTA computes a 128 (tokens) x 256 (output features) tile:
-//   warp 0      TMA producer: W tile (bf16, 128-byte swizzle) and the raw h codes
-//               of each 64-wide K stage into a ring of shared-memory stages;
-//   warp 1      allocates 256 TMEM columns and, from one lane, issues
-//               tcgen05.mma (M=128, N=256, K=16, bf16 x bf16 -> fp32) four times
-//               per stage, committing each stage to its "empty" mbarrier;
-//   warps 2..5  dequantise the raw codes of each stage into the K-major,
-//               128-byte-swizzled bf16 A tile (generic stores + proxy fence),
-//               then read the accumulator back (tcgen05.ld, 32 lanes each) and
-//               store fp16 K/V rows.
-// Every wait is bounded; a give-up sets *status and the CTA drains and frees its
-// TMEM before returning.
+// Two kernels:
+//   dequant_h_kernel   h^ = code * scale rounded to bf16 (the GEMM operand), once per
+//                      call, into a [B][len_pad][D] bf16 buffer (rows past the length
+//                      are zero); memory-bound.
+//   hgemm_kernel       one CTA per 128 (tokens) x 256 (output features) tile:
+//     warp 0      TMA producer: A (bf16 h^) and W tiles of each 64-wide K stage,
+//                 both with 128-byte swizzle, into a 4-stage shared-memory ring;
+//     warp 1      allocates 256 TMEM columns and, from one lane, issues
+//                 tcgen05.mma (M=128, N=256, K=16, bf16 x bf16 -> fp32) four times
+//                 per stage, committing each stage to its "empty" mbarrier;
+//     warps 2..5  read the accumulator back (tcgen05.ld, one 32-lane quarter each)
+//                 and store fp16 K/V rows.
+// Dequantising once instead of inside every (M, N) tile keeps the 16 N-tiles of a
+// row block from redoing the same conversion.  Every wait is bounded; a give-up
+// sets *status and the CTA drains and frees its TMEM before returning.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -37,12 +40,18 @@ constexpr uint32_t B_BYTES = BN * BK * 2;        // 32 KB
 constexpr uint32_t TMEM_COLS = 256;
 
 struct GemmArgs {
-    const __half *h_scales;   // [B][cap][h_groups] (null at 16 bits)
     __half *k_out, *v_out;    // [B][Hkv][out_cap][Dh]
     int *status;              // may be null
-    int32_t cap, d_model, h_bits, h_groups, n_kv_heads, head_dim, len, out_cap, m_tiles;
-    uint32_t raw_bytes, stage_bytes, stages;
+    int32_t d_model, n_kv_heads, head_dim, len, out_cap, m_tiles;
+    uint32_t stage_bytes, stages;
     uint64_t timeout_ns;
+};
+
+struct DequantArgs {
+    const uint8_t *h_codes;   // [B][cap][D*bits/8]
+    const __half *h_scales;   // [B][cap][h_groups]
+    __nv_bfloat16 *out;       // [B][len_pad][D]
+    int32_t cap, d_model, h_bits, h_groups, len, len_pad;
 };
 
 // ------------------------------------------------------------ tcgen05 helpers
@@ -126,32 +135,73 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr)
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                             ((uint32_t)(BM >> 4) << 24);
 
-// byte offset of bf16 element e (0..63) of row r in a K-major 128-byte-swizzled tile
-__device__ __forceinline__ uint32_t a_off(int r, int chunk16)
-{
-    return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((chunk16 ^ (r & 7)) << 4));
-}
-
 __device__ __forceinline__ uint32_t bf2(float lo, float hi)
 {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// One block per (sequence, token) row, one thread per 8 elements (16 output bytes).
+__global__ void __launch_bounds__(256) dequant_h_kernel(const DequantArgs a)
+{
+    const int row = blockIdx.x;                      // b * len_pad + t
+    const int b = row / a.len_pad, t = row % a.len_pad;
+    const int nchunk = a.d_model / 8;
+    const int gsz = a.d_model / a.h_groups;
+    const bool live = t < a.len;
+    const int64_t src_row = (int64_t)b * a.cap + t;
+    for (int j = threadIdx.x; j < nchunk; j += blockDim.x) {
+        uint4 o = make_uint4(0u, 0u, 0u, 0u);
+        if (live) {
+            uint32_t *ow = reinterpret_cast<uint32_t *>(&o);
+            if (a.h_bits == 16) {
+                const uint4 x = *reinterpret_cast<const uint4 *>(a.h_codes + (src_row * a.d_model + 8 * j) * 2);
+                const __half2 *hx = reinterpret_cast<const __half2 *>(&x);
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    const float2 f = __half22float2(hx[i]);
+                    ow[i] = bf2(f.x, f.y);
+                }
+            } else {
+                const float sv = __half2float(a.h_scales[src_row * a.h_groups + (8 * j) / gsz]);
+                if (a.h_bits == 8) {
+                    const uint2 x = *reinterpret_cast<const uint2 *>(a.h_codes + src_row * a.d_model + 8 * j);
+                    const uint32_t w[2] = {x.x, x.y};
+#pragma unroll
+                    for (int i = 0; i < 4; i++) {
+                        const uint32_t ww = w[i >> 1];
+                        const int sh = (i & 1) * 16;
+                        ow[i] = bf2((float)(int8_t)((ww >> sh) & 0xff) * sv,
+                                    (float)(int8_t)((ww >> (sh + 8)) & 0xff) * sv);
+                    }
+                } else {
+                    // element 2i in the low nibble of byte i, 2i+1 in the high nibble
+                    const uint32_t x = *reinterpret_cast<const uint32_t *>(a.h_codes + src_row * (a.d_model / 2) + 4 * j);
+#pragma unroll
+                    for (int i = 0; i < 4; i++) {
+                        const int lo = (int)((x >> (8 * i)) & 0xf), hi = (int)((x >> (8 * i + 4)) & 0xf);
+                        ow[i] = bf2((float)(lo >= 8 ? lo - 16 : lo) * sv, (float)(hi >= 8 ? hi - 16 : hi) * sv);
+                    }
+                }
+            }
+        }
+        *reinterpret_cast<uint4 *>(a.out + ((int64_t)row * a.d_model + 8 * j)) = o;
+    }
+}
+
 __global__ void __launch_bounds__(NTHREADS, 1)
-    hgemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_h,
+    hgemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_a,
                  const GemmArgs g)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t S = g.stages;
-    // stage s: [A 16 KB][B 32 KB][raw codes] ; barriers after the ring
+    // stage s: [A 16 KB][B 32 KB]; barriers after the ring
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + S * g.stage_bytes);
-    uint64_t *tma_full = bars;           // W + raw codes landed (TMA tx)
-    uint64_t *a_full = bars + S;         // A tile written (4 converter warps)
-    uint64_t *empty = bars + 2 * S;      // MMAs of the stage finished (tcgen05.commit)
-    uint64_t *acc_full = bars + 3 * S;   // all MMAs finished
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * S + 1);
+    uint64_t *full = bars;               // A + W tiles landed (TMA tx)
+    uint64_t *empty = bars + S;          // MMAs of the stage finished (tcgen05.commit)
+    uint64_t *acc_full = bars + 2 * S;   // all MMAs finished
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 1);
     int *abort_flag_p = reinterpret_cast<int *>(tmem_slot + 1);
     volatile int *abort_flag = abort_flag_p;
 
@@ -164,8 +214,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
     if (threadIdx.x == 0) {
         for (uint32_t s = 0; s < S; s++) {
-            mbar_init(&tma_full[s], 1);
-            mbar_init(&a_full[s], 4);
+            mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
         mbar_init(acc_full, 1);
@@ -190,19 +239,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
             prefetch_tensormap(&tm_w);
-            prefetch_tensormap(&tm_h);
+            prefetch_tensormap(&tm_a);
             uint32_t s = 0, ph = 0;
             int issued = 0;
-            const int raw_x = BK * g.h_bits / 8;   // raw bytes of one row per stage
             for (int k = 0; k < k_stages; k++) {
                 if (k >= (int)S && !mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, limit)) {
                     give_up();
                     break;
                 }
                 uint8_t *st = smem + s * g.stage_bytes;
-                mbar_arrive_expect_tx(&tma_full[s], B_BYTES + g.raw_bytes);
-                tma_load_2d(st + A_BYTES, &tm_w, &tma_full[s], k * BK, n0);
-                tma_load_3d(st + A_BYTES + B_BYTES, &tm_h, &tma_full[s], k * raw_x, t0, b);
+                mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES);
+                tma_load_3d(st, &tm_a, &full[s], k * BK, t0, b);
+                tma_load_2d(st + A_BYTES, &tm_w, &full[s], k * BK, n0);
                 issued = k + 1;
                 if (++s == S) {
                     s = 0;
@@ -217,7 +265,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     pp ^= 1u;
                 }
                 --ss;
-                (void)mbar_wait_bounded(&tma_full[ss], pp, abort_flag, limit);
+                (void)mbar_wait_bounded(&full[ss], pp, abort_flag, limit);
             }
         }
     } else if (warp == 1) {
@@ -226,8 +274,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             uint32_t s = 0, ph = 0;
             int issued = 0;
             for (int k = 0; k < k_stages; k++) {
-                if (!mbar_wait_bounded(&tma_full[s], ph, abort_flag, limit) ||
-                    !mbar_wait_bounded(&a_full[s], ph, abort_flag, limit)) {
+                if (!mbar_wait_bounded(&full[s], ph, abort_flag, limit)) {
                     give_up();
                     break;
                 }
@@ -261,98 +308,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
         }
     } else {
-        // ------------------------------------------------ converters, then epilogue
-        const int r = threadIdx.x - 64;            // 0..127: tile row handled by this thread
-        const int t = t0 + r;
-        const int gsz = g.d_model / g.h_groups;   // elements per h scale group
-        const bool live = t < g.len;
-        // scales of the two 32-element blocks of stage k, fetched one stage ahead
-        auto load_scales = [&](int k, float (&o)[2]) {
-#pragma unroll
-            for (int q = 0; q < 2; q++) {
-                const int e = k * BK + 32 * q;
-                o[q] = live ? __half2float(g.h_scales[((int64_t)b * g.cap + t) * g.h_groups + e / gsz])
-                            : 0.f;
-            }
-        };
-        float sc_next[2] = {0.f, 0.f};
-        if (g.h_bits != 16) load_scales(0, sc_next);
-        uint32_t s = 0, ph = 0;
-        bool ok = true;
-        for (int k = 0; k < k_stages && ok; k++) {
-            const float sc[2] = {sc_next[0], sc_next[1]};
-            if (g.h_bits != 16 && k + 1 < k_stages) load_scales(k + 1, sc_next);
-            if (!mbar_wait_bounded(&tma_full[s], ph, abort_flag, limit)) {
-                give_up();
-                ok = false;
-                break;
-            }
-            uint8_t *st = smem + s * g.stage_bytes;
-            const uint8_t *raw = st + A_BYTES + B_BYTES + (size_t)r * (BK * g.h_bits / 8);
-            uint8_t *arow = st;
-            if (g.h_bits == 16) {
-                // fp16 h: bf16(h), 8 elements per 16-byte chunk
-#pragma unroll
-                for (int c = 0; c < 8; c++) {
-                    uint4 x = *reinterpret_cast<const uint4 *>(raw + 16 * c);
-                    const __half2 *hx = reinterpret_cast<const __half2 *>(&x);
-                    uint4 o;
-                    uint32_t *ow = reinterpret_cast<uint32_t *>(&o);
-#pragma unroll
-                    for (int j = 0; j < 4; j++) {
-                        const float2 f = __half22float2(hx[j]);
-                        ow[j] = live ? bf2(f.x, f.y) : 0u;
-                    }
-                    *reinterpret_cast<uint4 *>(arow + a_off(r, c)) = o;
-                }
-            } else {
-                if (g.h_bits == 8) {
-#pragma unroll
-                    for (int c = 0; c < 8; c++) {
-                        const uint2 x = *reinterpret_cast<const uint2 *>(raw + 8 * c);
-                        const float sv = sc[c >> 2];
-                        uint4 o;
-                        const uint32_t w[2] = {x.x, x.y};
-                        uint32_t *ow = reinterpret_cast<uint32_t *>(&o);
-#pragma unroll
-                        for (int j = 0; j < 4; j++) {
-                            const uint32_t ww = w[j >> 1];
-                            const int sh = (j & 1) * 16;
-                            const float lo = (float)(int8_t)((ww >> sh) & 0xff);
-                            const float hi = (float)(int8_t)((ww >> (sh + 8)) & 0xff);
-                            ow[j] = bf2(lo * sv, hi * sv);
-                        }
-                        *reinterpret_cast<uint4 *>(arow + a_off(r, c)) = o;
-                    }
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 8; c++) {
-                        const uint32_t x = *reinterpret_cast<const uint32_t *>(raw + 4 * c);
-                        const float sv = sc[c >> 2];
-                        uint4 o;
-                        uint32_t *ow = reinterpret_cast<uint32_t *>(&o);
-#pragma unroll
-                        for (int j = 0; j < 4; j++) {
-                            // element 2j in the low nibble of byte j, 2j+1 in the high nibble
-                            const int lo = (int)((x >> (8 * j)) & 0xf), hi = (int)((x >> (8 * j + 4)) & 0xf);
-                            const float flo = (float)(lo >= 8 ? lo - 16 : lo);
-                            const float fhi = (float)(hi >= 8 ? hi - 16 : hi);
-                            ow[j] = bf2(flo * sv, fhi * sv);
-                        }
-                        *reinterpret_cast<uint4 *>(arow + a_off(r, c)) = o;
-                    }
-                }
-            }
-            fence_proxy_async_smem();   // generic-proxy stores -> async-proxy MMA reads
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&a_full[s]);
-            if (++s == S) {
-                s = 0;
-                ph ^= 1u;
-            }
-        }
-        // ---------------- epilogue: TMEM -> fp16 K/V rows
-        if (ok && mbar_wait_bounded(acc_full, 0, abort_flag, limit)) {
+        // ------------------------------------------------ epilogue: TMEM -> fp16 K/V rows
+        if (mbar_wait_bounded(acc_full, 0, abort_flag, limit)) {
             tc_fence_after();
             const int q = warp & 3;                       // TMEM lane quarter of this warp
             const int row = 32 * q + lane;                // accumulator row = tile row
@@ -379,7 +336,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                 }
             }
-        } else if (ok) {
+        } else {
             give_up();
         }
     }
@@ -417,12 +374,31 @@ cudaError_t launch_h_reconstruct(const HGemmParams &p, cudaStream_t stream)
 {
     const int N = 2 * p.n_kv_heads * p.head_dim;
     if (p.head_dim % 32 != 0 || N % BN != 0 || p.d_model % BK != 0) return cudaErrorNotSupported;
-    if (p.h_bits != 16 && (p.d_model / p.h_groups) % 32 != 0) return cudaErrorNotSupported;
+    if (p.h_bits != 16 && (p.d_model / p.h_groups) % 8 != 0) return cudaErrorNotSupported;
     EncodeTiledFn fn = encode_fn();
     if (!fn) return cudaErrorNotSupported;
+    const int m_tiles = (p.len + BM - 1) / BM;
+    const int len_pad = m_tiles * BM;
 
-    // W: bf16 [N][D], boxes of 64 (K) x 256 (N) with 128-byte swizzle
-    CUtensorMap tm_w, tm_h;
+    // 1. h^ -> bf16 operand, once per call
+    DequantArgs da{};
+    da.h_codes = p.h_codes;
+    da.h_scales = p.h_scales;
+    da.out = reinterpret_cast<__nv_bfloat16 *>(p.operand);
+    da.cap = p.cap;
+    da.d_model = p.d_model;
+    da.h_bits = p.h_bits;
+    da.h_groups = p.h_groups;
+    da.len = p.len;
+    da.len_pad = len_pad;
+    (void)cudaGetLastError();
+    dequant_h_kernel<<<(unsigned)(p.batch * len_pad), 256, 0, stream>>>(da);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    // 2. tensor maps: W bf16 [N][D] and the operand bf16 [B][len_pad][D], boxes of
+    //    64 (K) x 256 (N) and 64 (K) x 128 (tokens), both with 128-byte swizzle
+    CUtensorMap tm_w, tm_a;
     {
         cuuint64_t dims[2] = {(cuuint64_t)p.d_model, (cuuint64_t)N};
         cuuint64_t strides[1] = {(cuuint64_t)p.d_model * 2};
@@ -432,47 +408,33 @@ cudaError_t launch_h_reconstruct(const HGemmParams &p, cudaStream_t stream)
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
-    // h codes: bytes [B][cap][D*bits/8], boxes of (64 elements of codes) x 128 tokens
-    const uint32_t row_bytes = (uint32_t)p.d_model * p.h_bits / 8;
-    const uint32_t raw_x = BK * p.h_bits / 8;
     {
-        cuuint64_t dims[3] = {row_bytes, (cuuint64_t)p.cap, (cuuint64_t)p.batch};
-        cuuint64_t strides[2] = {row_bytes, (cuuint64_t)row_bytes * p.cap};
-        cuuint32_t box[3] = {raw_x, BM, 1}, es[3] = {1, 1, 1};
-        if (fn(&tm_h, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t *>(p.h_codes), dims,
-               strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+        cuuint64_t dims[3] = {(cuuint64_t)p.d_model, (cuuint64_t)len_pad, (cuuint64_t)p.batch};
+        cuuint64_t strides[2] = {(cuuint64_t)p.d_model * 2, (cuuint64_t)p.d_model * 2 * len_pad};
+        cuuint32_t box[3] = {BK, BM, 1}, es[3] = {1, 1, 1};
+        if (fn(&tm_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.operand, dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
     GemmArgs g{};
-    g.h_scales = p.h_scales;
     g.k_out = p.k_out;
     g.v_out = p.v_out;
     g.status = p.status;
-    g.cap = p.cap;
     g.d_model = p.d_model;
-    g.h_bits = p.h_bits;
-    g.h_groups = p.h_groups;
     g.n_kv_heads = p.n_kv_heads;
     g.head_dim = p.head_dim;
     g.len = p.len;
     g.out_cap = p.out_cap;
-    g.m_tiles = (p.len + BM - 1) / BM;
-    g.raw_bytes = raw_x * BM;
-    g.stage_bytes = ((A_BYTES + B_BYTES + g.raw_bytes) + 1023u) / 1024u * 1024u;
-    const uint32_t budget = 220u * 1024u;
-    g.stages = budget / g.stage_bytes;
-    if (g.stages > 4) g.stages = 4;
-    if (g.stages < 2) return cudaErrorNotSupported;
+    g.m_tiles = m_tiles;
+    g.stage_bytes = A_BYTES + B_BYTES;
+    g.stages = 4;
     g.timeout_ns = 1000000000ull;
-    const size_t smem = (size_t)g.stages * g.stage_bytes + 1024 + 3 * 8 * g.stages + 64;
-
-    cudaError_t e = cudaFuncSetAttribute(hgemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    const size_t smem = (size_t)g.stages * g.stage_bytes + 1024 + 8 * (2 * g.stages + 1) + 16;
+    e = cudaFuncSetAttribute(hgemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const dim3 grid(N / BN, (unsigned)(g.m_tiles * p.batch));
-    void *args[] = {&tm_w, &tm_h, &g};
-    (void)cudaGetLastError();
+    const dim3 grid(N / BN, (unsigned)(m_tiles * p.batch));
+    void *args[] = {&tm_w, &tm_a, &g};
     return cudaLaunchKernel(reinterpret_cast<void *>(&hgemm_kernel), grid, dim3(NTHREADS), args,
                             smem, stream);
 }

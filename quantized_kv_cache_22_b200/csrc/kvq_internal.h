@@ -81,9 +81,11 @@ struct HGemmParams {
     const __half *h_scales;   // [B][cap][h_groups]
     const void *w;            // bf16 [N][D]
     __half *k_out, *v_out;    // [B][Hkv][out_cap][Dh]
+    void *operand;            // bf16 [B][round_up(len, 128)][D] scratch for h^
     int *status;              // set to KVQ_ERR_TIMEOUT if a wait gives up (may be null)
     int32_t batch, cap, d_model, h_bits, h_groups, n_kv_heads, head_dim, len, out_cap;
 };
 cudaError_t launch_h_reconstruct(const HGemmParams &p, cudaStream_t stream);
+constexpr int kHTileTokens = 128;   // token rows of one reconstruction tile
 
 }  // namespace kvq

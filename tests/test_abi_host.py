@@ -128,6 +128,12 @@ def test_validation_errors_are_returned_on_the_host():
                 n_q_heads=2, n_kv_heads=2, head_dim=128).c()
     hl = KvqLayer(16, 32, None, None)
     assert _rc("kvq_h_reconstruct", ctypes.byref(hc), ctypes.byref(hl), P(64), 65, P(128), P(256),
-               128, None) == -3
+               128, P(512), ctypes.c_uint64(1 << 20), None) == -3
     assert _rc("kvq_h_reconstruct", ctypes.byref(hc), ctypes.byref(hl), P(64), 10, P(128), P(256),
-               100, None) == -1
+               100, P(512), ctypes.c_uint64(1 << 20), None) == -1
+    # operand scratch smaller than kvq_h_operand_bytes
+    need = ctypes.c_uint64()
+    assert _rc("kvq_h_operand_bytes", ctypes.byref(hc), 10, ctypes.byref(need)) == 0
+    assert need.value == 1 * 128 * 256 * 2
+    assert _rc("kvq_h_reconstruct", ctypes.byref(hc), ctypes.byref(hl), P(64), 10, P(128), P(256),
+               64, P(512), ctypes.c_uint64(need.value - 16), None) == -5

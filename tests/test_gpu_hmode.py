@@ -61,7 +61,9 @@ def _gpu_kv(cfg, h, W, L, out_cap):
     H = cfg.n_kv_heads
     k_out = torch.full((B, H, out_cap, 128), float("nan"), dtype=torch.float16, device="cuda")
     v_out = torch.full_like(k_out, float("nan"))
-    kvq.kvq_h_reconstruct(cfg, cache, W.cuda(), L, k_out, v_out, out_cap)
+    operand = torch.full((kvq.kvq_h_operand_bytes(cfg, L) // 2,), float("nan"),
+                         dtype=torch.bfloat16, device="cuda")
+    kvq.kvq_h_reconstruct(cfg, cache, W.cuda(), L, k_out, v_out, out_cap, operand)
     torch.cuda.synchronize()
     return cache, k_out.cpu(), v_out.cpu()
 
@@ -151,7 +153,8 @@ def test_hmode_full_size_sampled(cuda_device):
     H = cfg.n_kv_heads
     k_out = torch.empty(B, H, S, 128, dtype=torch.float16, device="cuda")
     v_out = torch.empty_like(k_out)
-    kvq.kvq_h_reconstruct(cfg, cache, W, S, k_out, v_out, S)
+    operand = torch.empty(kvq.kvq_h_operand_bytes(cfg, S) // 2, dtype=torch.bfloat16, device="cuda")
+    kvq.kvq_h_reconstruct(cfg, cache, W, S, k_out, v_out, S, operand)
     torch.cuda.synchronize()
     Wb = W.cpu().view(torch.int16).numpy().view(np.uint16)
     for b, head in ((0, 0), (5, 9), (7, 15)):
