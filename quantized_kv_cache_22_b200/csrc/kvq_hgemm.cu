@@ -12,14 +12,18 @@
 //   dequant_h_kernel   h^ = code * scale rounded to bf16 (the GEMM operand), once per
 //                      call, into a [B][len_pad][D] bf16 buffer (rows past the length
 //                      are zero); memory-bound.
-//   hgemm_kernel       one CTA per 128 (tokens) x 256 (output features) tile:
+//   hgemm_kernel       persistent, one CTA per SM, 128 (tokens) x 256 (output
+//                      features) tiles taken round-robin:
 //     warp 0      TMA producer: A (bf16 h^) and W tiles of each 64-wide K stage,
 //                 both with 128-byte swizzle, into a 4-stage shared-memory ring;
-//     warp 1      allocates 256 TMEM columns and, from one lane, issues
-//                 tcgen05.mma (M=128, N=256, K=16, bf16 x bf16 -> fp32) four times
-//                 per stage, committing each stage to its "empty" mbarrier;
-//     warps 2..5  read the accumulator back (tcgen05.ld, one 32-lane quarter each)
-//                 and store fp16 K/V rows.
+//     warp 1      allocates 2 x 256 TMEM columns (two accumulators) and, from one
+//                 lane, issues tcgen05.mma (M=128, N=256, K=16, bf16 x bf16 ->
+//                 fp32) four times per stage, committing each stage to its
+//                 "empty" mbarrier and each finished tile to its buffer's
+//                 "acc_full" mbarrier;
+//     warps 2..5  drain the other accumulator while the next tile's MMAs run
+//                 (tcgen05.ld, one 32-lane quarter each), store fp16 K/V rows and
+//                 hand the buffer back through "acc_empty".
 // Dequantising once instead of inside every (M, N) tile keeps the 16 N-tiles of a
 // row block from redoing the same conversion.  Every wait is bounded; a give-up
 // sets *status and the CTA drains and frees its TMEM before returning.
@@ -42,7 +46,7 @@ constexpr uint32_t TMEM_COLS = 256;
 struct GemmArgs {
     __half *k_out, *v_out;    // [B][Hkv][out_cap][Dh]
     int *status;              // may be null
-    int32_t d_model, n_kv_heads, head_dim, len, out_cap, m_tiles;
+    int32_t d_model, n_kv_heads, head_dim, len, out_cap, m_tiles, n_tiles, batch;
     uint32_t stage_bytes, stages;
     uint64_t timeout_ns;
 };
@@ -73,10 +77,6 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols)
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void fence_proxy_async_smem()
-{
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 
 // D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16 (bf16 operands here).
 __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
@@ -198,18 +198,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t S = g.stages;
     // stage s: [A 16 KB][B 32 KB]; barriers after the ring
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + S * g.stage_bytes);
-    uint64_t *full = bars;               // A + W tiles landed (TMA tx)
-    uint64_t *empty = bars + S;          // MMAs of the stage finished (tcgen05.commit)
-    uint64_t *acc_full = bars + 2 * S;   // all MMAs finished
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 1);
+    uint64_t *full = bars;               // A + W tiles of a stage landed (TMA tx)
+    uint64_t *empty = bars + S;          // MMAs of a stage finished (tcgen05.commit)
+    uint64_t *acc_full = bars + 2 * S;   // [2] accumulator buffer complete (tcgen05.commit)
+    uint64_t *acc_empty = bars + 2 * S + 2;   // [2] accumulator buffer drained (4 warps)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 4);
     int *abort_flag_p = reinterpret_cast<int *>(tmem_slot + 1);
     volatile int *abort_flag = abort_flag_p;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * BN;
-    const int b = blockIdx.y / g.m_tiles;
-    const int t0 = (blockIdx.y % g.m_tiles) * BM;
     const int k_stages = g.d_model / BK;
+    const int total = g.n_tiles * g.m_tiles * g.batch;
     const uint64_t limit = g.timeout_ns;
 
     if (threadIdx.x == 0) {
@@ -217,12 +216,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(acc_full, 1);
+        mbar_init(&acc_full[0], 1);
+        mbar_init(&acc_full[1], 1);
+        mbar_init(&acc_empty[0], 4);
+        mbar_init(&acc_empty[1], 4);
         *abort_flag_p = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_alloc(tmem_slot, 2 * TMEM_COLS);   // two 256-column accumulators
         tmem_relinquish();
     }
     tc_fence_before();
@@ -234,27 +236,40 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         *abort_flag_p = 1;
         if (g.status) atomicExch(g.status, KVQ_ERR_TIMEOUT);
     };
+    // tile index -> (n0, b, t0); N tiles vary fastest
+    auto tile_coords = [&](int tile, int &n0, int &b, int &t0) {
+        n0 = (tile % g.n_tiles) * BN;
+        const int mt = tile / g.n_tiles;
+        b = mt / g.m_tiles;
+        t0 = (mt % g.m_tiles) * BM;
+    };
 
     if (warp == 0) {
-        // ------------------------------------------------ TMA producer
+        // ------------------------------------------------ TMA producer (all tiles)
         if (lane == 0) {
             prefetch_tensormap(&tm_w);
             prefetch_tensormap(&tm_a);
             uint32_t s = 0, ph = 0;
-            int issued = 0;
-            for (int k = 0; k < k_stages; k++) {
-                if (k >= (int)S && !mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, limit)) {
-                    give_up();
-                    break;
-                }
-                uint8_t *st = smem + s * g.stage_bytes;
-                mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES);
-                tma_load_3d(st, &tm_a, &full[s], k * BK, t0, b);
-                tma_load_2d(st + A_BYTES, &tm_w, &full[s], k * BK, n0);
-                issued = k + 1;
-                if (++s == S) {
-                    s = 0;
-                    ph ^= 1u;
+            int issued = 0;      // stage uses issued so far
+            bool stop = false;
+            for (int tile = blockIdx.x; tile < total && !stop; tile += gridDim.x) {
+                int n0, b, t0;
+                tile_coords(tile, n0, b, t0);
+                for (int k = 0; k < k_stages; k++) {
+                    if (issued >= (int)S && !mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, limit)) {
+                        give_up();
+                        stop = true;
+                        break;
+                    }
+                    uint8_t *st = smem + s * g.stage_bytes;
+                    mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES);
+                    tma_load_3d(st, &tm_a, &full[s], k * BK, t0, b);
+                    tma_load_2d(st + A_BYTES, &tm_w, &full[s], k * BK, n0);
+                    ++issued;
+                    if (++s == S) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
             }
             // drain: every issued copy must land before the CTA can exit
@@ -272,31 +287,44 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
             uint32_t s = 0, ph = 0;
-            int issued = 0;
-            for (int k = 0; k < k_stages; k++) {
-                if (!mbar_wait_bounded(&full[s], ph, abort_flag, limit)) {
+            int done = 0;        // stage uses consumed
+            int local = 0;       // tiles of this CTA
+            bool stop = false;
+            for (int tile = blockIdx.x; tile < total && !stop; tile += gridDim.x, ++local) {
+                const int buf = local & 1;
+                // the epilogue must have drained this buffer (its use two tiles ago)
+                if (local >= 2 &&
+                    !mbar_wait_bounded(&acc_empty[buf], ((local >> 1) - 1) & 1u, abort_flag, limit)) {
                     give_up();
                     break;
                 }
                 tc_fence_after();
-                const uint32_t a_base = smem_u32(smem + s * g.stage_bytes);
-                const uint32_t b_base = a_base + A_BYTES;
+                const uint32_t d_tmem = tmem + (uint32_t)buf * TMEM_COLS;
+                for (int k = 0; k < k_stages; k++) {
+                    if (!mbar_wait_bounded(&full[s], ph, abort_flag, limit)) {
+                        give_up();
+                        stop = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_base = smem_u32(smem + s * g.stage_bytes);
+                    const uint32_t b_base = a_base + A_BYTES;
 #pragma unroll
-                for (int kk = 0; kk < BK / 16; kk++) {
-                    // K = 16 bf16 = 32 bytes further inside the 128-byte swizzle atom
-                    umma_f16(tmem, sw128_desc(a_base + kk * 32), sw128_desc(b_base + kk * 32),
-                             kIdesc, (k > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < BK / 16; kk++) {
+                        // K = 16 bf16 = 32 bytes further inside the 128-byte swizzle atom
+                        umma_f16(d_tmem, sw128_desc(a_base + kk * 32), sw128_desc(b_base + kk * 32),
+                                 kIdesc, (k > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(&empty[s]);
+                    ++done;
+                    if (++s == S) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
-                umma_commit(&empty[s]);
-                issued = k + 1;
-                if (++s == S) {
-                    s = 0;
-                    ph ^= 1u;
-                }
+                if (!stop) umma_commit(&acc_full[buf]);
             }
-            if (issued == k_stages) {
-                umma_commit(acc_full);
-            } else if (issued > 0) {
+            if (*abort_flag && done > 0) {
                 // aborted: wait (bounded) for the MMAs already issued to retire
                 uint32_t ss = s, pp = ph;
                 if (ss == 0) {
@@ -309,16 +337,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
     } else {
         // ------------------------------------------------ epilogue: TMEM -> fp16 K/V rows
-        if (mbar_wait_bounded(acc_full, 0, abort_flag, limit)) {
+        const int q = warp & 3;                       // TMEM lane quarter of this warp
+        const int row = 32 * q + lane;                // accumulator row = tile row
+        const int hd = g.n_kv_heads * g.head_dim;     // features of K (then of V)
+        int local = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
+            const int buf = local & 1;
+            if (!mbar_wait_bounded(&acc_full[buf], (local >> 1) & 1u, abort_flag, limit)) {
+                give_up();
+                break;
+            }
             tc_fence_after();
-            const int q = warp & 3;                       // TMEM lane quarter of this warp
-            const int row = 32 * q + lane;                // accumulator row = tile row
+            int n0, b, t0;
+            tile_coords(tile, n0, b, t0);
             const int tt = t0 + row;
-            const int hd = g.n_kv_heads * g.head_dim;     // features of K (then of V)
 #pragma unroll 1
             for (int c0 = 0; c0 < BN; c0 += 32) {
                 uint32_t v[32];
-                tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
+                tmem_ld32(tmem + (uint32_t)buf * TMEM_COLS + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
                 if (tt < g.len) {
                     const int n = n0 + c0;
                     __half *dst = n < hd ? g.k_out : g.v_out;
@@ -336,8 +372,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                 }
             }
-        } else {
-            give_up();
+            // all TMEM reads of this buffer are done: hand it back to the MMA warp
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
         }
     }
 
@@ -345,7 +383,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+    if (warp == 1) tmem_dealloc(tmem, 2 * TMEM_COLS);
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -430,10 +468,17 @@ cudaError_t launch_h_reconstruct(const HGemmParams &p, cudaStream_t stream)
     g.stage_bytes = A_BYTES + B_BYTES;
     g.stages = 4;
     g.timeout_ns = 1000000000ull;
-    const size_t smem = (size_t)g.stages * g.stage_bytes + 1024 + 8 * (2 * g.stages + 1) + 16;
+    const size_t smem = (size_t)g.stages * g.stage_bytes + 1024 + 8 * (2 * g.stages + 4) + 16;
     e = cudaFuncSetAttribute(hgemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const dim3 grid(N / BN, (unsigned)(m_tiles * p.batch));
+    g.n_tiles = N / BN;
+    g.batch = p.batch;
+    // persistent: one CTA per SM (the 197 KB ring allows no more), tiles round-robin
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        (void)cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int tiles = g.n_tiles * m_tiles * p.batch;
+    const dim3 grid((unsigned)(tiles < sms ? tiles : sms), 1);
     void *args[] = {&tm_w, &tm_a, &g};
     return cudaLaunchKernel(reinterpret_cast<void *>(&hgemm_kernel), grid, dim3(NTHREADS), args,
                             smem, stream);
