@@ -182,15 +182,22 @@ KVQ_API int kvq_h_operand_bytes(const kvq_config *cfg, int32_t max_len, uint64_t
  *   out = sum_t p_t v^_t,   k^ = code * scale (exact), v^ likewise,
  * with fp32 accumulation, then rounds to out_dtype.  A sequence with length
  * 0 gets zeros.  The token just appended is included (no mask).
- *   q        device [B][Hq][Dh], q_dtype KVQ_F16, KVQ_F32 or KVQ_BF16
- *            (f32/bf16 queries need G <= 4; f16 queries G <= 8)
+ *   q        device [B][Hq][Dh], q_dtype KVQ_F16, KVQ_F32 or KVQ_BF16; G <= 8
+ *            (with 16-bit keys, f32/bf16 queries need G <= 4).  With 4- or
+ *            8-bit keys the query enters the int8 tensor-core product as two
+ *            int8 parts per head, q ~ (max|q|/127)(hi + lo/254), i.e. with a
+ *            relative error below 2^-15 of the head's largest element.
  *   d_len    device int32 [B]: tokens attended per sequence (clamped to
  *            [0, capacity] on the device)
  *   max_len_host  host bound of d_len[] (<= capacity; used for h-mode scratch)
  *   softmax_scale  0 selects 1/sqrt(Dh)
  *   out      device [B][Hq][Dh], out_dtype KVQ_F16 or KVQ_F32
- *   workspace/workspace_bytes  device scratch for split partials, at least
- *            kvq_workspace_bytes(cfg, num_ctas); need not be initialised
+ *   workspace/workspace_bytes  device scratch for split partials and the
+ *            merge's arrival counters, at least kvq_workspace_bytes(cfg,
+ *            num_ctas).  Zero-fill it once before its first use; every call
+ *            leaves it ready for the next one, except one that reported
+ *            KVQ_ERR_TIMEOUT (zero-fill it again then).  Calls that overlap
+ *            on the GPU need separate workspaces.
  *   num_ctas persistent CTAs (0 = library's choice)
  *   h-mode only: w_kv device bf16 [2*Hkv*Dh][D] (rows of W_k then W_v;
  *            [TL] "運作原理": rebuild K = W_k h, V = W_v h at every attention
@@ -203,12 +210,28 @@ KVQ_API int kvq_decode_attn(const kvq_config *cfg, const kvq_layer *layer, const
                     const void *w_kv, void *kv_scratch, uint64_t kv_scratch_bytes,
                     kvq_stream_t stream);
 
+/* One decode step of a layer in one launch (KV mode): quantize-on-append of
+ * each sequence's newest token, then decode attention over the cache that
+ * includes it.  For every sequence b with L = d_len[b] >= 1 (clamped to the
+ * capacity), k_new[b] and v_new[b] ([B][Hkv][Dh], in_dtype) are quantised
+ * into position L - 1 exactly as kvq_append(d_pos = L - 1, n_new = 1) would
+ * ([TL] "KV Cache 模式": codes at append time), and the query then attends
+ * over positions [0, L) as in kvq_decode_attn.  Sequences with L = 0 append
+ * nothing and get zeros.  Other arguments and errors as kvq_decode_attn;
+ * h-mode configs return KVQ_ERR_INVALID_ARG. */
+KVQ_API int kvq_append_decode_attn(const kvq_config *cfg, const kvq_layer *layer,
+                                   const void *k_new, const void *v_new, int32_t in_dtype,
+                                   const void *q, int32_t q_dtype, const int32_t *d_len,
+                                   int32_t max_len_host, float softmax_scale, void *out,
+                                   int32_t out_dtype, void *workspace, uint64_t workspace_bytes,
+                                   int32_t num_ctas, kvq_stream_t stream);
+
 /* The two halves of kvq_decode_attn in KV mode, for callers that schedule
  * them separately (e.g. to time the attention kernel alone, or to gather the
  * partials of several devices before merging).
- * kvq_decode_partials: the split-KV attention kernel; writes one (m, l, o)
- *   partial per (CTA, sequence, KV head) segment into `workspace` (arguments
- *   as kvq_decode_attn).  The partials are unnormalised: o = sum_t p_t v^_t
+ * kvq_decode_partials: the split-KV attention kernel alone; writes one
+ *   (m, l, o) partial per (consumer warp, CTA, sequence, KV head) segment into
+ *   `workspace` (arguments as kvq_decode_attn; the counters are not used).  The partials are unnormalised: o = sum_t p_t v^_t
  *   and l = sum_t p_t with p_t = 2^(s_t log2(e) - m).
  * kvq_merge_partials: combines the partials with log-sum-exp weights,
  *   out = sum_k o_k 2^(m_k - M) / sum_k l_k 2^(m_k - M), and rounds to
@@ -242,8 +265,8 @@ KVQ_API int kvq_h_reconstruct(const kvq_config *cfg, const kvq_layer *layer, con
  * (its outputs are then invalid).  Synchronises `stream`. */
 KVQ_API int kvq_workspace_status(void *workspace, int32_t *status, kvq_stream_t stream);
 
-/* Bytes of the device array behind kvq_decode_attn_noalloc (2 MiB). */
-#define KVQ_NOALLOC_SCRATCH_BYTES (2u * 1024u * 1024u)
+/* Bytes of the device array behind kvq_decode_attn_noalloc (8 MiB). */
+#define KVQ_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
 
 /* kvq_decode_attn (KV mode) for callers that cannot allocate device memory.
  * The source pages have no counterpart: this is a deployment convenience.
@@ -260,11 +283,12 @@ KVQ_API int kvq_workspace_status(void *workspace, int32_t *status, kvq_stream_t 
  *     capture.
  *   Limit: configurations whose kvq_workspace_bytes(cfg, num_ctas) exceeds
  *     KVQ_NOALLOC_SCRATCH_BYTES are rejected with KVQ_ERR_WORKSPACE before
- *     anything is launched (for example B=16, Hkv=8, G=4, Dh=128 needs 0.9 MB).
+ *     anything is launched (for example B=16, Hkv=8, G=4, Dh=128 on 296 CTAs
+ *     needs 3.5 MB).
  *   Sharing: all calls in the process share the one array and it keeps the
  *     last call's contents; calls that overlap on the GPU (different streams,
  *     or several host threads) race on it and give wrong results.  Each call
- *     clears the status word it needs zeroed.
+ *     clears the status word and the merge counters it needs zeroed.
  * Nothing here allocates or frees memory.  Other arguments and errors as
  * kvq_decode_attn; h-mode configs return KVQ_ERR_INVALID_ARG. */
 KVQ_API int kvq_decode_attn_noalloc(const kvq_config *cfg, const kvq_layer *layer, const void *q,

@@ -24,7 +24,8 @@ KVQ_F16, KVQ_F32, KVQ_BF16 = 0, 1, 2
 EXPORTED = ("kvq_cache_bytes", "kvq_layer_buffer_bytes", "kvq_append", "kvq_workspace_bytes",
             "kvq_h_scratch_bytes", "kvq_decode_attn", "kvq_decode_partials", "kvq_merge_partials",
             "kvq_h_reconstruct", "kvq_workspace_status", "kvq_status_string",
-            "kvq_last_error_detail", "kvq_decode_attn_noalloc", "kvq_h_operand_bytes")
+            "kvq_last_error_detail", "kvq_decode_attn_noalloc", "kvq_h_operand_bytes",
+            "kvq_append_decode_attn")
 
 
 class KvqError(RuntimeError):
@@ -62,6 +63,8 @@ def _load():
         "kvq_decode_attn": [cfgp, layp, P, i32, P, i32, ctypes.c_float, P, i32, P, u64, i32, P, P,
                             u64, P],
         "kvq_decode_partials": [cfgp, layp, P, i32, P, i32, ctypes.c_float, P, u64, i32, P],
+        "kvq_append_decode_attn": [cfgp, layp, P, P, i32, P, i32, P, i32, ctypes.c_float, P, i32,
+                                   P, u64, i32, P],
         "kvq_merge_partials": [cfgp, P, P, i32, P, u64, i32, P],
         "kvq_h_operand_bytes": [cfgp, i32, pu64],
         "kvq_h_reconstruct": [cfgp, layp, P, i32, P, P, i32, P, u64, P],
@@ -185,7 +188,8 @@ class LayerCache:
 
 
 class Workspace:
-    """Split-KV partials buffer sized by kvq_workspace_bytes (status word zeroed)."""
+    """Split-KV partials and merge counters, sized by kvq_workspace_bytes and zero-filled
+    (a call leaves it ready for the next; zero it again after a timeout status)."""
 
     def __init__(self, cfg: Config, num_ctas: int = 0, device="cuda"):
         self.nbytes = kvq_workspace_bytes(cfg, num_ctas)
@@ -211,6 +215,21 @@ def kvq_decode_attn(cfg: Config, layer: LayerCache, q: torch.Tensor, d_len: torc
                                 _ptr(out), _dtype_code(out), _ptr(ws.buf), ws.nbytes,
                                 int(num_ctas), _ptr(w_kv), _ptr(kv_scratch), scratch_bytes,
                                 _stream(stream)))
+
+
+def kvq_append_decode_attn(cfg: Config, layer: LayerCache, k_new: torch.Tensor,
+                           v_new: torch.Tensor, q: torch.Tensor, d_len: torch.Tensor, max_len: int,
+                           out: torch.Tensor, ws: Workspace, softmax_scale: float = 0.0,
+                           num_ctas: int = 0, stream=None):
+    """One decode step: quantise k_new/v_new ([B][Hkv][Dh]) into position d_len-1, then attend."""
+    if k_new.dtype != v_new.dtype:
+        raise ValueError("k_new and v_new must share a dtype")
+    _check("kvq_append_decode_attn",
+           _lib.kvq_append_decode_attn(ctypes.byref(cfg.c()), ctypes.byref(layer.c()), _ptr(k_new),
+                                       _ptr(v_new), _dtype_code(k_new), _ptr(q), _dtype_code(q),
+                                       _ptr(d_len), int(max_len), float(softmax_scale), _ptr(out),
+                                       _dtype_code(out), _ptr(ws.buf), ws.nbytes, int(num_ctas),
+                                       _stream(stream)))
 
 
 def kvq_decode_partials(cfg: Config, layer: LayerCache, q: torch.Tensor, d_len: torch.Tensor,

@@ -206,7 +206,7 @@ int resolve_plan(const kvq_config *cfg, int32_t num_ctas, DecodeLaunch *plan, in
 uint64_t workspace_need(const kvq_config *cfg, int ctas)
 {
     const AttnShape a = attn_shape(cfg);
-    return (uint64_t)kWorkspaceHeaderFloats * 4 +
+    return (uint64_t)kWorkspaceHeaderFloats * 4 + counter_ints(cfg->batch, a.hkv) * 4 +
            slot_count(ctas, cfg->batch, a.hkv) * slot_floats(a.G, a.dh) * 4;
 }
 
@@ -384,22 +384,27 @@ int kvq_h_operand_bytes(const kvq_config *cfg, int32_t max_len, uint64_t *bytes)
     return KVQ_OK;
 }
 
-// Validated KV-layout attention: launch the split kernel (do_partials) and/or
-// the merge (do_merge).
+// Validated KV-layout attention.  do_partials && do_merge: one launch that
+// also merges (arrival counters in the workspace); do_partials alone leaves
+// the per-warp partials; do_merge alone launches the merge kernel over them.
+// `app` (optional) fuses the append of each sequence's newest token.
 static int decode_kv_layout(const kvq_config *cfg, const void *k_codes, const void *k_scales,
                             const void *v_codes, const void *v_scales, int cap, const void *q,
                             int32_t q_dtype, const int32_t *d_len, float softmax_scale, void *out,
                             int32_t out_dtype, void *workspace, uint64_t workspace_bytes,
-                            int32_t num_ctas, cudaStream_t stream, bool do_partials, bool do_merge)
+                            int32_t num_ctas, cudaStream_t stream, bool do_partials, bool do_merge,
+                            const FusedAppend *app = nullptr)
 {
     const AttnShape a = attn_shape(cfg);
-    if (q_dtype != KVQ_F16 && a.G > 4) return KVQ_ERR_UNSUPPORTED;
+    // fp16 keys use an f16 MMA whose f32 / bf16 queries take two columns per head
+    if (a.kb == 16 && q_dtype != KVQ_F16 && a.G > 4) return KVQ_ERR_UNSUPPORTED;
     DecodeLaunch plan;
     int ctas = 0;
     int rc = resolve_plan(cfg, num_ctas, &plan, &ctas);
     if (rc) return rc;
     if (workspace_bytes < workspace_need(cfg, ctas)) return KVQ_ERR_WORKSPACE;
-    float *ws = static_cast<float *>(workspace) + kWorkspaceHeaderFloats;
+    int *counters = reinterpret_cast<int *>(static_cast<float *>(workspace) + kWorkspaceHeaderFloats);
+    float *ws = reinterpret_cast<float *>(counters + counter_ints(cfg->batch, a.hkv));
 
     if (do_partials) {
         CUtensorMap tm_k, tm_v;
@@ -414,6 +419,9 @@ static int decode_kv_layout(const kvq_config *cfg, const void *k_codes, const vo
         p.v_scales = static_cast<const __half *>(v_scales);
         p.status = static_cast<int *>(workspace);
         p.ws = ws;
+        p.counters = do_merge ? counters : nullptr;
+        p.out = do_merge ? out : nullptr;
+        p.out_f32 = out_dtype == KVQ_F32;
         p.q_dtype = q_dtype;
         p.batch = cfg->batch;
         p.n_q_heads = a.hq;
@@ -436,8 +444,10 @@ static int decode_kv_layout(const kvq_config *cfg, const void *k_codes, const vo
         const float scale = softmax_scale != 0.f ? softmax_scale : 1.f / std::sqrt((float)a.dh);
         p.tau_log2e = scale * 1.4426950408889634f;
         p.timeout_ns = kTimeoutNs;
+        if (app) p.app = *app;
         cudaError_t e = launch_decode(plan, p, tm_k, tm_v, stream);
         if (e != cudaSuccess) return fail("decode launch", e);
+        return KVQ_OK;
     }
     if (do_merge) {
         MergeParams mp{};
@@ -604,6 +614,44 @@ int kvq_decode_attn(const kvq_config *cfg, const kvq_layer *layer, const void *q
     return decode_kv_layout(cfg, kout, nullptr, vout, nullptr, scap, q, q_dtype, d_len,
                             softmax_scale, out, out_dtype, workspace, workspace_bytes, num_ctas, st,
                             true, true);
+}
+
+int kvq_append_decode_attn(const kvq_config *cfg, const kvq_layer *layer, const void *k_new,
+                           const void *v_new, int32_t in_dtype, const void *q, int32_t q_dtype,
+                           const int32_t *d_len, int32_t max_len_host, float softmax_scale,
+                           void *out, int32_t out_dtype, void *workspace, uint64_t workspace_bytes,
+                           int32_t num_ctas, kvq_stream_t stream)
+{
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (cfg->mode != KVQ_MODE_KV) return KVQ_ERR_INVALID_ARG;
+    if (!layer || !k_new || !v_new || !q || !d_len || !out || !workspace || num_ctas < 0)
+        return KVQ_ERR_INVALID_ARG;
+    if (in_dtype != KVQ_F16 && in_dtype != KVQ_F32 && in_dtype != KVQ_BF16)
+        return KVQ_ERR_INVALID_ARG;
+    if (q_dtype != KVQ_F16 && q_dtype != KVQ_F32 && q_dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
+    if (out_dtype != KVQ_F16 && out_dtype != KVQ_F32) return KVQ_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale) || max_len_host < 0) return KVQ_ERR_INVALID_ARG;
+    if (max_len_host > cfg->capacity) return KVQ_ERR_CAPACITY;
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(q) || !aligned16(out) ||
+        !aligned16(workspace))
+        return KVQ_ERR_ALIGN;
+    rc = check_kv_layer(cfg, layer);
+    if (rc) return rc;
+    FusedAppend app{};
+    app.k_new = k_new;
+    app.v_new = v_new;
+    app.k_codes = static_cast<uint8_t *>(layer->k_codes);
+    app.v_codes = static_cast<uint8_t *>(layer->v_codes);
+    app.k_scales = static_cast<__half *>(layer->k_scales);
+    app.v_scales = static_cast<__half *>(layer->v_scales);
+    app.dtype = in_dtype;
+    app.k_group = cfg->k_bits == 16 ? 32 : cfg->k_group;
+    app.v_group = cfg->v_bits == 16 ? 32 : cfg->v_group;
+    return decode_kv_layout(cfg, layer->k_codes, layer->k_scales, layer->v_codes, layer->v_scales,
+                            cfg->capacity, q, q_dtype, d_len, softmax_scale, out, out_dtype,
+                            workspace, workspace_bytes, num_ctas,
+                            reinterpret_cast<cudaStream_t>(stream), true, true, &app);
 }
 
 int kvq_h_reconstruct(const kvq_config *cfg, const kvq_layer *layer, const void *w_kv,

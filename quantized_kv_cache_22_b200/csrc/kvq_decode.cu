@@ -6,31 +6,43 @@
 // attention kernel (KVSplit discussion: integrate the formats into the
 // FlashAttention kernel), with INT8 / nibble-packed INT4 codes and fp16
 // scales per (token, head) or per group (TinyLoop mode table; KVSplit 8K
-// table).  Output = softmax(tau q.K^T) V, fp32 accumulation.
+// table).  Output = softmax(tau q.K^T) V, fp32 accumulation.  Optionally the
+// new token's K/V are quantised into the cache by the same launch first
+// (quantize-on-append, TinyLoop "KV Cache 模式").
 //
 // Design for sm_100a (not taken from any page):
-//   * Persistent CTAs, work split stream-K style: the units are 64-token tiles
-//     of every (sequence, KV head); CTA c takes units [cN/P, (c+1)N/P).  Every
-//     CTA therefore streams the same number of bytes whatever B, Hkv and the
-//     lengths are.  A CTA's run of tiles inside one (sequence, KV head) is a
-//     "segment"; each segment leaves one partial (m, l, o) in the workspace at
-//     slot (cta + sequence*Hkv + kv_head), which is unique, and a small merge
-//     kernel combines the partials with their log-sum-exp weights.
+//   * Persistent CTAs, work split stream-K style: the units are 128-token
+//     tiles of every (sequence, KV head); CTA c of the P' = min(P, units) CTAs
+//     that get work takes units [cN/P', (c+1)N/P').  Every CTA streams the same
+//     number of bytes whatever B, Hkv and the lengths are.  A CTA's run of
+//     tiles inside one (sequence, KV head) is a "segment"; at its end the
+//     consumer warps combine their partials (m, l, o) in shared memory and
+//     write one per segment to the workspace, at slot (cta + sequence*Hkv +
+//     kv_head), which is unique.  The warp that completes the last of the
+//     partials of a (sequence, KV head) -- an arrival counter tells it --
+//     merges them with their log-sum-exp weights and writes the output, so one
+//     launch does the whole layer.
 //   * One producer warp streams tiles with TMA: codes through 3-D tiled tensor
 //     maps with 128-byte swizzle (bank-conflict-free fragment reads), scales
 //     with 1-D bulk copies, into a multi-stage shared-memory ring guarded by
 //     mbarriers.  Every wait is bounded (about a second) and a give-up sets
-//     the workspace status word instead of hanging.
-//   * Four consumer warps each take 16 tokens of a 64-token stage.  Codes are
-//     turned into fp16 in registers with the exponent-bias trick (a code byte
-//     u placed in the mantissa of 0x6400 reads 1024 + u), so no convert
-//     instruction and no scale multiply touches an element: key scales scale
-//     the 16x8 score tile, value scales are folded into the probabilities.
-//     q.K^T and P.V run on warp-level tensor-core MMA (m16n8k16, f16 in, f32
-//     accumulate) with tokens / head_dim as the M dimension and the G query
-//     heads of the KV group as N.  The constant bias (1024+128 or 1024+8) is
-//     removed in fp32 afterwards using sum(q) and sum(p).
-//   * The online softmax tracks max(s + log2 s_V) so that p * s_V <= 1 fits
+//     the workspace status word instead of hanging.  Before it loads the tile
+//     that holds a sequence's newest token, the producer warp quantises that
+//     token into the cache (the fused append) and fences the writes against
+//     the copy engine.
+//   * Four consumer warps each take 32 tokens of a stage as two 16-token
+//     sub-tiles.  q.K^T runs on int8 tensor-core MMA (m16n8k32): the key codes
+//     feed the MMA as they are stored (4-bit codes after one mask, as 16x the
+//     code), and the query is split per head into two int8 parts, q ~ s (hi +
+//     lo/254), so the products keep ~16 bits of the query.  P.V runs on f16
+//     MMA (m16n8k16, f32 accumulate) with head_dim as M and the G query heads
+//     of the KV group as N: value codes become fp16 in registers with the
+//     exponent-bias trick (a code byte u in the mantissa of 0x6400 reads 1024
+//     + u), value scales are folded into the probabilities, and the constant
+//     bias is removed at the end with the probability sums, which one extra
+//     MMA against a matrix of ones accumulates.  The score tile is turned into
+//     the P operand by two 8x8 transposes (movmatrix).
+//   * The online softmax tracks max(s + log2 s_V) so that p * s_V <= 2^8 fits
 //     fp16 without underflow whatever the value scales are.
 #include <cfloat>
 #include <mutex>
@@ -40,6 +52,7 @@
 
 #include "kvq_internal.h"
 #include "kvq_ptx.cuh"
+#include "kvq_quant.cuh"
 #include "../../include/kvq.h"
 
 namespace kvq {
@@ -48,12 +61,17 @@ namespace {
 constexpr int NW = kDecodeConsumerWarps;
 constexpr int T = kDecodeTileTokens;
 constexpr int NTHR = kDecodeThreads;
+constexpr unsigned FULL = 0xffffffffu;
 
 struct __align__(16) StageMeta {
     int32_t bh;      // sequence * Hkv + kv_head
     int32_t t0;      // first token of the tile
     int32_t len;     // tokens attended by this sequence
-    int32_t flags;   // bit0 first tile of a segment, bit1 last tile, bits 8.. slot
+    int32_t flags;   // bit0 first tile of a segment, bit1 last tile of a segment
+    int32_t slot;    // partial slot of this CTA's segment: cta + bh
+    int32_t ncta;    // CTAs holding a segment of this (sequence, KV head)
+    int32_t cmin;    // the first of them
+    int32_t pad;
 };
 
 // Byte offset of element byte `o` of token `t` inside a stage tile that TMA
@@ -73,30 +91,16 @@ __host__ __device__ constexpr uint32_t sw_off(int t, int o)
     }
 }
 
-// fp16 pair helpers: code bytes / nibbles -> half2 of (bias + code).
-__device__ __forceinline__ uint32_t i8_lo_pair(uint32_t xw) { return prmt(xw, 0x64646464u, 0x4140u); }
-__device__ __forceinline__ uint32_t i8_hi_pair(uint32_t xw) { return prmt(xw, 0x64646464u, 0x4342u); }
+// Token of row g (g < 8) of a 16-token sub-tile's score tile; row g + 8 holds
+// the next token.  The permutation pi(g) = g ^ (g >> 2) keeps both the key-row
+// reads of the score MMA and the value-row reads of the P.V MMA (whose k
+// order follows the score rows through the transpose) free of bank conflicts.
+__host__ __device__ constexpr int row_token(int g) { return 2 * (g ^ (g >> 2)); }
+
+// fp16 pair helpers: value code bytes / nibbles -> half2 of (bias + code).
 __device__ __forceinline__ uint32_t i4_pair(uint32_t w, int k)
 {
     return and_xor(w >> (4 * k), 0x000F000Fu, 0x64086408u);
-}
-
-// Element offset (0..7 inside a lane's 8-element run of a 32-block) feeding
-// k-slot j (0: 2tig, 1: 2tig+1, 2: 2tig+8, 3: 2tig+9) of k-step half hs.
-template <int KB>
-__device__ __forceinline__ int k_elem(int hs, int j)
-{
-    if constexpr (KB == 4) {
-        return 2 * hs + ((j & 1) ? 4 : 0) + (j >> 1);
-    } else {
-        return 4 * hs + j;
-    }
-}
-
-template <typename TQ>
-__device__ __forceinline__ float ld_q(const void *q, int64_t idx)
-{
-    return static_cast<float>(static_cast<const TQ *>(q)[idx]);
 }
 
 __device__ __forceinline__ float load_qf(const void *q, int dtype, int64_t idx)
@@ -106,11 +110,12 @@ __device__ __forceinline__ float load_qf(const void *q, int dtype, int64_t idx)
     return __bfloat162float(static_cast<const __nv_bfloat16 *>(q)[idx]);
 }
 
-__device__ __forceinline__ int tiles_of(int len, int cap)
+__device__ __forceinline__ int clamp_len(int len, int cap)
 {
-    len = len < 0 ? 0 : (len > cap ? cap : len);
-    return (len + T - 1) / T;
+    return len < 0 ? 0 : (len > cap ? cap : len);
 }
+
+__device__ __forceinline__ int tiles_of(int len, int cap) { return (clamp_len(len, cap) + T - 1) / T; }
 
 // 2^x with the hardware approximation (relative error ~2^-22); results below
 // 2^-126 flush to zero, which only drops probabilities that are zero anyway.
@@ -169,22 +174,109 @@ __device__ __forceinline__ uint32_t blk_addr(uint32_t a0, int blk)
     }
 }
 
+__device__ __forceinline__ uint32_t pack_bytes(int a, int b, int c, int d)
+{
+    return (uint32_t)(a & 0xff) | ((uint32_t)(b & 0xff) << 8) | ((uint32_t)(c & 0xff) << 16) |
+           ((uint32_t)(d & 0xff) << 24);
+}
+
+__device__ __forceinline__ float warp_max(float v)
+{
+#pragma unroll
+    for (int off = 16; off; off >>= 1) v = fmaxf(v, __shfl_xor_sync(FULL, v, off));
+    return v;
+}
+__device__ __forceinline__ float warp_sum(float v)
+{
+#pragma unroll
+    for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(FULL, v, off);
+    return v;
+}
+
+// Merge the np CTA partials of one (sequence, KV head), all G query heads at once:
+// slots slot0 .. slot0 + np - 1, each G records of DH + 4 floats holding per
+// query head o[DH], m, l.  out[obase0 + col * DH + d] receives
+//   sum_j o_j[d] 2^(m_j - M) / sum_j l_j 2^(m_j - M),  M = max_j m_j.
+// LPC lanes share one query head (column) and split its DH outputs; the
+// partials are read through L2 (ld.global.cg) because other SMs wrote them in
+// this launch.  One warp.
+template <int DH, int LPC>
+__device__ void merge_segment_lpc(const float *ws, int64_t slot0, int np, int G, void *out,
+                                  int out_f32, int64_t obase0, int lane)
+{
+    constexpr int PER = DH / LPC;       // floats of one partial per lane
+    constexpr int CS = slot_col_floats(DH);
+    const int col = lane / LPC, part = lane % LPC;
+    const bool active = col < G;
+    const int64_t stride = (int64_t)G * CS;
+    const float *base = ws + slot0 * stride + (int64_t)(active ? col : 0) * CS;
+    float M = -INFINITY;
+    if (active)
+        for (int j = part; j < np; j += LPC) M = fmaxf(M, __ldcg(base + j * stride + DH));
+#pragma unroll
+    for (int off = 1; off < LPC; off <<= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, off));
+    float L = 0.f;
+    float o[PER];
+#pragma unroll
+    for (int i = 0; i < PER; i++) o[i] = 0.f;
+    if (active && M != -INFINITY) {
+#pragma unroll 4
+        for (int j = 0; j < np; j++) {
+            const float *src = base + (int64_t)j * stride;
+            const float2 ml = __ldcg(reinterpret_cast<const float2 *>(src + DH));
+            float4 x[PER / 4];
+#pragma unroll
+            for (int i = 0; i < PER / 4; i++)
+                x[i] = __ldcg(reinterpret_cast<const float4 *>(src + part * PER) + i);
+            const float e = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M);
+            L = fmaf(e, ml.y, L);
+#pragma unroll
+            for (int i = 0; i < PER / 4; i++) {
+                o[4 * i] = fmaf(e, x[i].x, o[4 * i]);
+                o[4 * i + 1] = fmaf(e, x[i].y, o[4 * i + 1]);
+                o[4 * i + 2] = fmaf(e, x[i].z, o[4 * i + 2]);
+                o[4 * i + 3] = fmaf(e, x[i].w, o[4 * i + 3]);
+            }
+        }
+    }
+    if (!active) return;
+    const float inv = (L > 0.f) ? 1.f / L : 0.f;
+    const int64_t ob = obase0 + (int64_t)col * DH + part * PER;
+#pragma unroll
+    for (int i = 0; i < PER; i += 2) {
+        if (out_f32)
+            *reinterpret_cast<float2 *>(static_cast<float *>(out) + ob + i) =
+                make_float2(o[i] * inv, o[i + 1] * inv);
+        else
+            *reinterpret_cast<__half2 *>(static_cast<__half *>(out) + ob + i) =
+                __floats2half2_rn(o[i] * inv, o[i + 1] * inv);
+    }
+}
+
+template <int DH>
+__device__ __forceinline__ void merge_segment(const float *ws, int64_t slot0, int np, int G,
+                                              void *out, int out_f32, int64_t obase0, int lane)
+{
+    if (G <= 4)
+        merge_segment_lpc<DH, 8>(ws, slot0, np, G, out, out_f32, obase0, lane);
+    else
+        merge_segment_lpc<DH, 4>(ws, slot0, np, G, out, out_f32, obase0, lane);
+}
+
 template <int DH, int KB, int VB>
 __global__ void __launch_bounds__(NTHR, 2)
     decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                  const DecodeParams p)
+                  const __grid_constant__ DecodeParams p)
 {
     constexpr int NG = DH / 32;                // 32-element blocks along head_dim
     constexpr int RK = DH * KB / 8;            // bytes per key row
     constexpr int RV = DH * VB / 8;
     constexpr int SK = 32 * KB / 8;            // bytes per 32-element block of a key row
     constexpr int SV = 32 * VB / 8;
-    constexpr float BIAS_K = KB == 8 ? 1152.f : (KB == 4 ? 1032.f : 0.f);
     constexpr float BIAS_V = VB == 8 ? 1152.f : (VB == 4 ? 1032.f : 0.f);
     // The running max is only raised when a tile beats it by more than 2^LAZY;
     // weights p * s_V then stay below 2^LAZY, well inside fp16.
     constexpr float LAZY = 8.f;
-    constexpr unsigned FULL = 0xffffffffu;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // align to 1024 B (128-byte swizzle atoms) by pointer arithmetic on the shared
@@ -194,9 +286,9 @@ __global__ void __launch_bounds__(NTHR, 2)
     StageMeta *meta = reinterpret_cast<StageMeta *>(smem + p.off_meta);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + p.off_bar);
     uint64_t *empty = full + p.stages;
-    uint64_t *segbar = empty + p.stages;               // two: [0] partials written, [1] merged
-    int *ctl = reinterpret_cast<int *>(segbar + 2);    // [0] abort, [1] units, [2..3] prefix
-    float *mbuf = reinterpret_cast<float *>(smem + p.off_merge);
+    uint64_t *segbar = empty + p.stages;                // [0] partials in mbuf, [1] mbuf read
+    int *ctl = reinterpret_cast<int *>(segbar + 2);     // [0] abort, [1] units, [2..3] prefix
+    float *mbuf = reinterpret_cast<float *>(smem + p.off_merge);   // [NW][G][DH + 4]
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -204,6 +296,7 @@ __global__ void __launch_bounds__(NTHR, 2)
     const int S = p.stages;
     const int G = p.group_size_g;
     const int cap = p.cap;
+    const int Hkv = p.n_kv_heads;
     volatile int *abort_flag = ctl;
 
     if (tid == 0) {
@@ -218,24 +311,26 @@ __global__ void __launch_bounds__(NTHR, 2)
     }
 
     // ---- work range of this CTA (computed by the producer warp) -------------
-    __shared__ long long sh_u_begin;
+    __shared__ long long sh_u_begin, sh_n, sh_pe;
     __shared__ int sh_b;
     if (warp == NW) {
         long long total = 0;
         for (int b = lane; b < p.batch; b += 32) total += tiles_of(p.d_len[b], cap);
         for (int off = 16; off; off >>= 1) total += __shfl_xor_sync(FULL, total, off);
-        const long long N = total * p.n_kv_heads;
-        const long long P = p.num_ctas;
-        const long long ub = (long long)blockIdx.x * N / P;
-        const long long ue = ((long long)blockIdx.x + 1) * N / P;
+        const long long N = total * Hkv;
+        const long long Pe = N < (long long)p.num_ctas ? N : (long long)p.num_ctas;
+        long long ub = 0, ue = 0;
+        if ((long long)blockIdx.x < Pe) {
+            ub = (long long)blockIdx.x * N / Pe;
+            ue = ((long long)blockIdx.x + 1) * N / Pe;
+        }
         // locate the sequence holding unit ub
         long long acc = 0;
         int fb = -1;
         long long fpre = 0;
-        for (int base = 0; base < p.batch && fb < 0; base += 32) {
+        for (int base = 0; base < p.batch && fb < 0 && ue > ub; base += 32) {
             const int b = base + lane;
-            const long long units =
-                (b < p.batch) ? (long long)tiles_of(p.d_len[b], cap) * p.n_kv_heads : 0;
+            const long long units = (b < p.batch) ? (long long)tiles_of(p.d_len[b], cap) * Hkv : 0;
             long long incl = units;
             for (int off = 1; off < 32; off <<= 1) {
                 const long long v = __shfl_up_sync(FULL, incl, off);
@@ -253,6 +348,8 @@ __global__ void __launch_bounds__(NTHR, 2)
         }
         if (lane == 0) {
             sh_u_begin = ub;
+            sh_n = N;
+            sh_pe = Pe;
             sh_b = fb;
             ctl[1] = (int)(ue > ub && fb >= 0 ? ue - ub : 0);
             reinterpret_cast<long long *>(ctl + 2)[0] = fpre;
@@ -262,13 +359,18 @@ __global__ void __launch_bounds__(NTHR, 2)
     const int n_units = ctl[1];
 
     if (warp == NW) {
-        // ====================== producer ======================
-        if (lane != 0) return;
-        prefetch_tensormap(&tm_k);
-        prefetch_tensormap(&tm_v);
+        // ====================== producer (whole warp) ======================
+        if (lane == 0) {
+            prefetch_tensormap(&tm_k);
+            prefetch_tensormap(&tm_v);
+        }
+        // codes and scales are read once: let them leave L2 first, so that the
+        // partials and the queries stay cached
+        const uint64_t pol = l2_evict_first_policy();
+        const long long N = sh_n, Pe = sh_pe;
         int b = sh_b;
-        const long long pre = reinterpret_cast<long long *>(ctl + 2)[0];
-        int len_b = (b >= 0) ? min(max(p.d_len[b], 0), cap) : 0;
+        long long pre = reinterpret_cast<long long *>(ctl + 2)[0];   // units before sequence b
+        int len_b = (b >= 0) ? clamp_len(p.d_len[b], cap) : 0;
         int tiles_b = (len_b + T - 1) / T;
         const int off = (int)(sh_u_begin - pre);   // unit offset inside sequence b
         int kvh = tiles_b ? off / tiles_b : 0;
@@ -276,48 +378,76 @@ __global__ void __launch_bounds__(NTHR, 2)
         int s = 0;
         uint32_t ph = 0;                            // phase parity of this use of stage s
         int issued = 0;
+        int seg_ncta = 0, seg_cmin = 0;
         for (int i = 0; i < n_units; i++) {
-            if (i >= S) {
-                if (!mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, p.timeout_ns)) {
+            const int bh = b * Hkv + kvh;
+            const int t0 = tile * T;
+            if (i == 0 || tile == 0) {
+                // CTAs whose unit ranges meet this (sequence, KV head)
+                const long long u0 = pre + (long long)kvh * tiles_b, u1 = u0 + tiles_b;
+                const long long cmin = ((u0 + 1) * Pe + N - 1) / N - 1;
+                const long long cmax = (u1 * Pe + N - 1) / N - 1;
+                seg_cmin = (int)cmin;
+                seg_ncta = (int)(cmax - cmin + 1);
+            }
+            if (p.app.k_new != nullptr && tile == tiles_b - 1) {
+                // fused append: the newest token (position len - 1) lies in this
+                // tile; quantise it into the cache before the tile is loaded
+                const int64_t crow = (int64_t)bh * cap + (len_b - 1);
+                quantize_row(p.app.k_new, (int64_t)bh * DH, p.app.dtype, DH, KB, p.app.k_group,
+                             p.app.k_codes + crow * RK,
+                             KB == 16 ? nullptr : p.app.k_scales + crow * (DH / p.app.k_group), lane);
+                quantize_row(p.app.v_new, (int64_t)bh * DH, p.app.dtype, DH, VB, p.app.v_group,
+                             p.app.v_codes + crow * RV,
+                             VB == 16 ? nullptr : p.app.v_scales + crow * (DH / p.app.v_group), lane);
+                fence_proxy_async_global();
+                __syncwarp();
+            }
+            int ok = 1;
+            if (lane == 0 && i >= S) ok = mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, p.timeout_ns);
+            ok = __shfl_sync(FULL, ok, 0);
+            if (!ok) {
+                if (lane == 0) {
                     ctl[0] = 1;
                     atomicExch(p.status, KVQ_ERR_TIMEOUT);
-                    break;
                 }
+                break;
             }
-            const int bh = b * p.n_kv_heads + kvh;
-            const int t0 = tile * T;
-            int flags = 0;
-            if (i == 0 || tile == 0) flags |= 1;
-            if (i == n_units - 1 || tile == tiles_b - 1) flags |= 2;
-            flags |= ((int)blockIdx.x + bh) << 8;
-            StageMeta m;
-            m.bh = bh; m.t0 = t0; m.len = len_b; m.flags = flags;
-            meta[s] = m;
+            if (lane == 0) {
+                int flags = 0;
+                if (i == 0 || tile == 0) flags |= 1;
+                if (i == n_units - 1 || tile == tiles_b - 1) flags |= 2;
+                StageMeta m;
+                m.bh = bh; m.t0 = t0; m.len = len_b; m.flags = flags;
+                m.slot = (int)blockIdx.x + bh;
+                m.ncta = seg_ncta; m.cmin = seg_cmin; m.pad = 0;
+                meta[s] = m;
 
-            uint8_t *st = smem + (size_t)s * p.stage_bytes;
-            const int n_s = min(T, cap - t0);
-            uint32_t bytes = (uint32_t)(T * RK + T * RV);
-            if (KB != 16) bytes += (uint32_t)(n_s * p.ngs_k * 2);
-            if (VB != 16) bytes += (uint32_t)(n_s * p.ngs_v * 2);
-            mbar_arrive_expect_tx(&full[s], bytes);
-            if constexpr (RK <= 128) {
-                tma_load_3d(st, &tm_k, &full[s], 0, t0 / (128 / RK), bh);
-            } else {
-                tma_load_3d(st, &tm_k, &full[s], 0, t0, bh);
-                tma_load_3d(st + T * 128, &tm_k, &full[s], 128, t0, bh);
+                uint8_t *st = smem + (size_t)s * p.stage_bytes;
+                const int n_s = min(T, cap - t0);
+                uint32_t bytes = (uint32_t)(T * RK + T * RV);
+                if (KB != 16) bytes += (uint32_t)(n_s * p.ngs_k * 2);
+                if (VB != 16) bytes += (uint32_t)(n_s * p.ngs_v * 2);
+                mbar_arrive_expect_tx(&full[s], bytes);
+                if constexpr (RK <= 128) {
+                    tma_load_3d_hint(st, &tm_k, &full[s], 0, t0 / (128 / RK), bh, pol);
+                } else {
+                    tma_load_3d_hint(st, &tm_k, &full[s], 0, t0, bh, pol);
+                    tma_load_3d_hint(st + T * 128, &tm_k, &full[s], 128, t0, bh, pol);
+                }
+                if constexpr (RV <= 128) {
+                    tma_load_3d_hint(st + p.off_v, &tm_v, &full[s], 0, t0 / (128 / RV), bh, pol);
+                } else {
+                    tma_load_3d_hint(st + p.off_v, &tm_v, &full[s], 0, t0, bh, pol);
+                    tma_load_3d_hint(st + p.off_v + T * 128, &tm_v, &full[s], 128, t0, bh, pol);
+                }
+                if (KB != 16)
+                    bulk_load_hint(st + p.off_sk, p.k_scales + ((int64_t)bh * cap + t0) * p.ngs_k,
+                                   (uint32_t)(n_s * p.ngs_k * 2), &full[s], pol);
+                if (VB != 16)
+                    bulk_load_hint(st + p.off_sv, p.v_scales + ((int64_t)bh * cap + t0) * p.ngs_v,
+                                   (uint32_t)(n_s * p.ngs_v * 2), &full[s], pol);
             }
-            if constexpr (RV <= 128) {
-                tma_load_3d(st + p.off_v, &tm_v, &full[s], 0, t0 / (128 / RV), bh);
-            } else {
-                tma_load_3d(st + p.off_v, &tm_v, &full[s], 0, t0, bh);
-                tma_load_3d(st + p.off_v + T * 128, &tm_v, &full[s], 128, t0, bh);
-            }
-            if (KB != 16)
-                bulk_load(st + p.off_sk, p.k_scales + ((int64_t)bh * cap + t0) * p.ngs_k,
-                          (uint32_t)(n_s * p.ngs_k * 2), &full[s]);
-            if (VB != 16)
-                bulk_load(st + p.off_sv, p.v_scales + ((int64_t)bh * cap + t0) * p.ngs_v,
-                          (uint32_t)(n_s * p.ngs_v * 2), &full[s]);
             issued = i + 1;
             if (++s == S) {
                 s = 0;
@@ -326,108 +456,158 @@ __global__ void __launch_bounds__(NTHR, 2)
             // advance to the next unit (the length is re-read only when b changes)
             if (++tile == tiles_b) {
                 tile = 0;
-                if (++kvh == p.n_kv_heads) {
+                if (++kvh == Hkv) {
                     kvh = 0;
                     do {
+                        pre += (long long)tiles_b * Hkv;
                         ++b;
-                        len_b = (b < p.batch) ? min(max(p.d_len[b], 0), cap) : T;
+                        len_b = (b < p.batch) ? clamp_len(p.d_len[b], cap) : T;
                         tiles_b = (len_b + T - 1) / T;
                     } while (tiles_b == 0);
                 }
             }
         }
         // never leave with copies in flight: wait for the last issued phases
-        int ss = s;
-        uint32_t pp = ph;
-        for (int j = 0; j < min(S, issued); j++) {
-            if (ss == 0) {
-                ss = S;
-                pp ^= 1u;
+        if (lane == 0) {
+            int ss = s;
+            uint32_t pp = ph;
+            for (int j = 0; j < min(S, issued); j++) {
+                if (ss == 0) {
+                    ss = S;
+                    pp ^= 1u;
+                }
+                --ss;
+                (void)mbar_wait_bounded(&full[ss], pp, abort_flag, p.timeout_ns);
             }
-            --ss;
-            (void)mbar_wait_bounded(&full[ss], pp, abort_flag, p.timeout_ns);
         }
         return;
     }
 
     // ====================== consumers ======================
+    constexpr bool IMMA_K = KB != 16;
     const int gid = lane >> 2;
     const int tig = lane & 3;
-    const bool qsplit = p.q_dtype != KVQ_F16;
+    // fp16 keys keep an f16 MMA; f32 / bf16 queries then use columns 4..7 for
+    // the fp16 residual of the query (G <= 4)
+    const bool qsplit = !IMMA_K && p.q_dtype != KVQ_F16;
     const bool kgrp = p.ngs_k > 1;
     const bool vgrp = p.ngs_v > 1;
     const int colmax = qsplit ? 4 : 8;
     const bool col_ok0 = (2 * tig) < G && (2 * tig) < colmax;
     const bool col_ok1 = (2 * tig + 1) < G && (2 * tig + 1) < colmax;
 
-    // per-lane swizzled offsets of block 0 of the rows this lane reads (relative
-    // to a stage tile), for the two 16-token sub-tiles of the warp
+    // sequences with nothing cached get zeros (fused merge only; the merge
+    // launch writes them otherwise)
+    if (p.counters != nullptr) {
+        const int64_t n_out = (int64_t)p.n_q_heads * DH;
+        for (int b = blockIdx.x; b < p.batch; b += gridDim.x) {
+            if (tiles_of(p.d_len[b], cap) != 0) continue;
+            for (int64_t i = tid; i < n_out; i += 32 * NW) {
+                if (p.out_f32)
+                    static_cast<float *>(p.out)[(int64_t)b * n_out + i] = 0.f;
+                else
+                    static_cast<__half *>(p.out)[(int64_t)b * n_out + i] = __float2half_rn(0.f);
+            }
+        }
+    }
+
+    // Rows of the score tile: row gid is token tw + rt, row gid + 8 token tw + rt + 1.
+    // The P.V MMA takes k-slots 2tig, 2tig+1, 2tig+8, 2tig+9 = tokens
+    // tw + vA, tw + vB, tw + vA + 1, tw + vB + 1 (the transpose of the score rows).
+    const int rt = row_token(gid);
+    const int vA = row_token(2 * tig), vB = row_token(2 * tig + 1);
     uint32_t kofs[2][2], vofs[2][4];
 #pragma unroll
     for (int u = 0; u < 2; u++) {
         const int tw = warp * 32 + u * 16;
-        kofs[u][0] = sw_off<RK>(tw + 2 * gid, tig * (SK / 4));
-        kofs[u][1] = sw_off<RK>(tw + 2 * gid + 1, tig * (SK / 4));
-        const int tv = tw + 2 * tig;
-        vofs[u][0] = p.off_v + sw_off<RV>(tv, gid * (SV / 8));
-        vofs[u][1] = p.off_v + sw_off<RV>(tv + 1, gid * (SV / 8));
-        vofs[u][2] = p.off_v + sw_off<RV>(tv + 8, gid * (SV / 8));
-        vofs[u][3] = p.off_v + sw_off<RV>(tv + 9, gid * (SV / 8));
+        kofs[u][0] = sw_off<RK>(tw + rt, tig * (SK / 4));
+        kofs[u][1] = sw_off<RK>(tw + rt + 1, tig * (SK / 4));
+        vofs[u][0] = p.off_v + sw_off<RV>(tw + vA, gid * (SV / 8));
+        vofs[u][1] = p.off_v + sw_off<RV>(tw + vB, gid * (SV / 8));
+        vofs[u][2] = p.off_v + sw_off<RV>(tw + vA + 1, gid * (SV / 8));
+        vofs[u][3] = p.off_v + sw_off<RV>(tw + vB + 1, gid * (SV / 8));
     }
-    // source lanes of the P transposition (score layout -> B-fragment layout)
-    const int src0 = tig * 4 + (gid >> 1);
-    const int src1 = (tig + 4) * 4 + (gid >> 1);
-    const bool odd = gid & 1;
 
-    uint32_t qb[NG][2][2];              // q B-fragments per (block, k-half)
-    float qbias[NG][2];                 // BIAS_K * sum(q) per block, score cols 2tig, 2tig+1
+    uint32_t qh[NG][2], ql[NG][2];      // int8 query B-fragments (hi / lo parts) per block
+    float sqc[2];                       // score factor of columns 2tig, 2tig+1
+    uint32_t qb[NG][2][2];              // fp16 query B-fragments (fp16 keys)
     float m_run[2], l_run[2];
-    float psum[NG][2];                  // sum of fp16 p*s_V per value block (or [0])
-    float o_acc[2 * NG][4];             // O^T fragments, m-tile = 2*blk + u
-    uint32_t seg_parity = 0;
+    float psum[NG][4];                  // sum of fp16 p*s_V per value group (cols in [0], [1])
+    float o_acc[2 * NG][4];             // O^T fragments, m-tile = 2*blk + h
 
     auto load_q = [&](int bh) {
-        const int b = bh / p.n_kv_heads;
-        const int kvh = bh % p.n_kv_heads;
-        // B-fragment column n = gid: non-split: head n; split: hi (n<4) / lo (n>=4) of head n&3
-        const int head = qsplit ? (gid & 3) : gid;
-        const bool lo_part = qsplit && gid >= 4;
-        const bool valid = head < G;
-        const int64_t qbase = ((int64_t)b * p.n_q_heads + (int64_t)kvh * G + head) * DH;
+        const int b = bh / Hkv;
+        const int kvh = bh % Hkv;
+        if constexpr (IMMA_K) {
+            // q ~ (amax / 127) * (hi + lo / 254) per head, hi, lo in [-127, 127];
+            // lane (gid, tig) holds head gid, elements 32 blk + 8 tig + 0..7
+            const bool valid = gid < G;
+            const int64_t qbase = ((int64_t)b * p.n_q_heads + (int64_t)kvh * G + gid) * DH;
+            float x[NG][8];
+            float amax = 0.f;
 #pragma unroll
-        for (int blk = 0; blk < NG; blk++) {
-            float colsum = 0.f;
+            for (int blk = 0; blk < NG; blk++)
 #pragma unroll
-            for (int hs = 0; hs < 2; hs++) {
-                __half hv[4];
-#pragma unroll
-                for (int j = 0; j < 4; j++) {
-                    const int d = 32 * blk + 8 * tig + k_elem<KB>(hs, j);
-                    const float x = valid ? load_qf(p.q, p.q_dtype, qbase + d) : 0.f;
-                    __half h = __float2half_rn(x);
-                    if (lo_part) h = __float2half_rn(x - __half2float(h));
-                    hv[j] = h;
-                    colsum += __half2float(h);
+                for (int j = 0; j < 8; j++) {
+                    x[blk][j] = valid ? load_qf(p.q, p.q_dtype, qbase + 32 * blk + 8 * tig + j) : 0.f;
+                    amax = fmaxf(amax, fabsf(x[blk][j]));
                 }
-                __half2 b0 = __halves2half2(hv[0], hv[1]);
-                __half2 b1 = __halves2half2(hv[2], hv[3]);
-                qb[blk][hs][0] = *reinterpret_cast<uint32_t *>(&b0);
-                qb[blk][hs][1] = *reinterpret_cast<uint32_t *>(&b1);
-            }
-            colsum += __shfl_xor_sync(FULL, colsum, 1);
-            colsum += __shfl_xor_sync(FULL, colsum, 2);
-            // score cols of this lane are 2tig and 2tig+1; column n lives on lanes with gid = n
-            qbias[blk][0] = BIAS_K * __shfl_sync(FULL, colsum, (2 * tig) * 4);
-            qbias[blk][1] = BIAS_K * __shfl_sync(FULL, colsum, (2 * tig + 1) * 4);
-        }
-        if (!kgrp) {
+            amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 2));
+            const float inv = amax > 0.f ? 127.f / amax : 0.f;
 #pragma unroll
-            for (int c = 0; c < 2; c++) {
-                float t = 0.f;
+            for (int blk = 0; blk < NG; blk++) {
+                int hi[8], lo[8];
 #pragma unroll
-                for (int blk = 0; blk < NG; blk++) t += qbias[blk][c];
-                qbias[0][c] = t;
+                for (int j = 0; j < 8; j++) {
+                    const float y = x[blk][j] * inv;
+                    const float r = rintf(y);
+                    hi[j] = (int)r;
+                    lo[j] = __float2int_rn((y - r) * 254.f);
+                }
+                if constexpr (KB == 8) {
+                    // k-slot 4tig+i <-> element 8tig+i, 16+4tig+i <-> 8tig+4+i
+                    qh[blk][0] = pack_bytes(hi[0], hi[1], hi[2], hi[3]);
+                    qh[blk][1] = pack_bytes(hi[4], hi[5], hi[6], hi[7]);
+                    ql[blk][0] = pack_bytes(lo[0], lo[1], lo[2], lo[3]);
+                    ql[blk][1] = pack_bytes(lo[4], lo[5], lo[6], lo[7]);
+                } else {
+                    // k-slot 4tig+i <-> element 8tig+2i (low nibbles), 16+4tig+i <-> 8tig+2i+1
+                    qh[blk][0] = pack_bytes(hi[0], hi[2], hi[4], hi[6]);
+                    qh[blk][1] = pack_bytes(hi[1], hi[3], hi[5], hi[7]);
+                    ql[blk][0] = pack_bytes(lo[0], lo[2], lo[4], lo[6]);
+                    ql[blk][1] = pack_bytes(lo[1], lo[3], lo[5], lo[7]);
+                }
             }
+            // 4-bit key codes enter the MMA as 16 * code
+            const float f = amax * (1.f / (127.f * 254.f)) * p.tau_log2e * (KB == 4 ? 0.0625f : 1.f);
+            sqc[0] = __shfl_sync(FULL, f, (2 * tig) * 4);
+            sqc[1] = __shfl_sync(FULL, f, (2 * tig + 1) * 4);
+        } else {
+            // B-fragment column n = gid: non-split: head n; split: hi (n<4) / lo (n>=4) of head n&3
+            const int head = qsplit ? (gid & 3) : gid;
+            const bool lo_part = qsplit && gid >= 4;
+            const bool valid = head < G;
+            const int64_t qbase = ((int64_t)b * p.n_q_heads + (int64_t)kvh * G + head) * DH;
+#pragma unroll
+            for (int blk = 0; blk < NG; blk++)
+#pragma unroll
+                for (int hs = 0; hs < 2; hs++) {
+                    __half hv[4];
+#pragma unroll
+                    for (int j = 0; j < 4; j++) {
+                        // k-slots 2tig, 2tig+1, 2tig+8, 2tig+9 <-> elements 8tig + 4hs + j
+                        const int d = 32 * blk + 8 * tig + 4 * hs + j;
+                        const float xq = valid ? load_qf(p.q, p.q_dtype, qbase + d) : 0.f;
+                        __half h = __float2half_rn(xq);
+                        if (lo_part) h = __float2half_rn(xq - __half2float(h));
+                        hv[j] = h;
+                    }
+                    __half2 b0 = __halves2half2(hv[0], hv[1]);
+                    __half2 b1 = __halves2half2(hv[2], hv[3]);
+                    qb[blk][hs][0] = *reinterpret_cast<uint32_t *>(&b0);
+                    qb[blk][hs][1] = *reinterpret_cast<uint32_t *>(&b1);
+                }
         }
 #pragma unroll
         for (int c = 0; c < 2; c++) {
@@ -435,42 +615,32 @@ __global__ void __launch_bounds__(NTHR, 2)
             l_run[c] = 0.f;
         }
 #pragma unroll
-        for (int g = 0; g < NG; g++) psum[g][0] = psum[g][1] = 0.f;
+        for (int g = 0; g < NG; g++) psum[g][0] = psum[g][1] = psum[g][2] = psum[g][3] = 0.f;
 #pragma unroll
         for (int mt = 0; mt < 2 * NG; mt++)
 #pragma unroll
             for (int i = 0; i < 4; i++) o_acc[mt][i] = 0.f;
     };
 
-    // A fragments of block blk, k-half hs, for key rows at a[0] (row gid) and a[1] (row gid+8)
-    auto key_frags = [&](uint32_t ra, uint32_t rb, int blk, uint32_t (&fa)[2][4]) {
+    // A fragments of block blk for the key rows at ra (row gid) and rb (row gid+8)
+    auto key_frags = [&](uint32_t ra, uint32_t rb, int blk, uint32_t (&fa)[4]) {
         if constexpr (KB == 8) {
             const uint2 r0 = lds_u64(sbase, blk_addr<RK, SK>(ra, blk));
             const uint2 r1 = lds_u64(sbase, blk_addr<RK, SK>(rb, blk));
-            const uint32_t x00 = r0.x ^ 0x80808080u, x01 = r0.y ^ 0x80808080u;
-            const uint32_t x10 = r1.x ^ 0x80808080u, x11 = r1.y ^ 0x80808080u;
-            fa[0][0] = i8_lo_pair(x00); fa[0][2] = i8_hi_pair(x00);
-            fa[0][1] = i8_lo_pair(x10); fa[0][3] = i8_hi_pair(x10);
-            fa[1][0] = i8_lo_pair(x01); fa[1][2] = i8_hi_pair(x01);
-            fa[1][1] = i8_lo_pair(x11); fa[1][3] = i8_hi_pair(x11);
-        } else if constexpr (KB == 4) {
+            fa[0] = r0.x; fa[1] = r1.x; fa[2] = r0.y; fa[3] = r1.y;
+        } else {
             const uint32_t r0 = lds_u32(sbase, blk_addr<RK, SK>(ra, blk));
             const uint32_t r1 = lds_u32(sbase, blk_addr<RK, SK>(rb, blk));
-            fa[0][0] = i4_pair(r0, 0); fa[0][2] = i4_pair(r0, 1);
-            fa[0][1] = i4_pair(r1, 0); fa[0][3] = i4_pair(r1, 1);
-            fa[1][0] = i4_pair(r0, 2); fa[1][2] = i4_pair(r0, 3);
-            fa[1][1] = i4_pair(r1, 2); fa[1][3] = i4_pair(r1, 3);
-        } else {
-            const uint4 r0 = lds_u128(sbase, blk_addr<RK, SK>(ra, blk));
-            const uint4 r1 = lds_u128(sbase, blk_addr<RK, SK>(rb, blk));
-            fa[0][0] = r0.x; fa[0][2] = r0.y; fa[0][1] = r1.x; fa[0][3] = r1.y;
-            fa[1][0] = r0.z; fa[1][2] = r0.w; fa[1][1] = r1.z; fa[1][3] = r1.w;
+            fa[0] = (r0 << 4) & 0xF0F0F0F0u; fa[1] = (r1 << 4) & 0xF0F0F0F0u;
+            fa[2] = r0 & 0xF0F0F0F0u;        fa[3] = r1 & 0xF0F0F0F0u;
         }
     };
 
     const uint64_t limit = p.timeout_ns;
+    const uint32_t ONE2 = 0x3C003C00u;   // half2(1, 1)
     int s = 0;
     uint32_t ph = 0;
+    uint32_t seg_parity = 0;
     for (int i = 0; i < n_units; i++) {
         if (!mbar_wait_bounded(&full[s], ph, abort_flag, limit)) {
             ctl[0] = 1;
@@ -479,8 +649,10 @@ __global__ void __launch_bounds__(NTHR, 2)
         }
         StageMeta m;
         {
-            const uint4 mm = *reinterpret_cast<const uint4 *>(&meta[s]);
-            m.bh = (int)mm.x; m.t0 = (int)mm.y; m.len = (int)mm.z; m.flags = (int)mm.w;
+            const uint4 m0 = *reinterpret_cast<const uint4 *>(&meta[s]);
+            const uint4 m1 = *(reinterpret_cast<const uint4 *>(&meta[s]) + 1);
+            m.bh = (int)m0.x; m.t0 = (int)m0.y; m.len = (int)m0.z; m.flags = (int)m0.w;
+            m.slot = (int)m1.x; m.ncta = (int)m1.y; m.cmin = (int)m1.z;
         }
         if (m.flags & 1) load_q(m.bh);
         const uint32_t st = (uint32_t)s * p.stage_bytes;   // stage offset from smem
@@ -494,16 +666,67 @@ __global__ void __launch_bounds__(NTHR, 2)
         bool vt[2][2];
 #pragma unroll
         for (int u = 0; u < 2; u++) {
-            tAu[u] = warp * 32 + u * 16 + 2 * gid;               // score rows: tAu, tAu + 1
+            tAu[u] = warp * 32 + u * 16 + rt;               // score rows: tAu, tAu + 1
             vt[u][0] = m.t0 + tAu[u] < m.len;
             vt[u][1] = m.t0 + tAu[u] + 1 < m.len;
         }
 
         // ---------------- phase 1: scores S^T = K q^T for both sub-tiles ----------
         float s2[2][4];
-        if (!kgrp) {
-            // two partial accumulators per sub-tile (even / odd blocks) halve the
-            // dependent MMA chain
+        if constexpr (IMMA_K) {
+            if (!kgrp) {
+                // hi and lo chains are independent; combined once per tile
+                int ah[2][4], al[2][4];
+#pragma unroll
+                for (int u = 0; u < 2; u++)
+#pragma unroll
+                    for (int e = 0; e < 4; e++) ah[u][e] = al[u][e] = 0;
+#pragma unroll
+                for (int blk = 0; blk < NG; blk++) {
+#pragma unroll
+                    for (int u = 0; u < 2; u++) {
+                        uint32_t fa[4];
+                        key_frags(st + kofs[u][0], st + kofs[u][1], blk, fa);
+                        imma_16832(ah[u], fa[0], fa[1], fa[2], fa[3], qh[blk][0], qh[blk][1]);
+                        imma_16832(al[u], fa[0], fa[1], fa[2], fa[3], ql[blk][0], ql[blk][1]);
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 2; u++) {
+                    const float2 kk = unpack_half2(lds_u32(sbase, ssk + 2 * tAu[u]));
+#pragma unroll
+                    for (int e = 0; e < 4; e++) {
+                        const float ks = (e < 2) ? kk.x : kk.y;
+                        s2[u][e] = (float)(ah[u][e] * 254 + al[u][e]) * (ks * sqc[e & 1]);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int u = 0; u < 2; u++) {
+                    float v[4] = {0.f, 0.f, 0.f, 0.f};
+                    const int tA = tAu[u];
+#pragma unroll
+                    for (int blk = 0; blk < NG; blk++) {
+                        int ah[4] = {0, 0, 0, 0}, al[4] = {0, 0, 0, 0};
+                        uint32_t fa[4];
+                        key_frags(st + kofs[u][0], st + kofs[u][1], blk, fa);
+                        imma_16832(ah, fa[0], fa[1], fa[2], fa[3], qh[blk][0], qh[blk][1]);
+                        imma_16832(al, fa[0], fa[1], fa[2], fa[3], ql[blk][0], ql[blk][1]);
+                        const float k0 = __half2float(__ushort_as_half(
+                            (unsigned short)lds_u16(sbase, ssk + 2 * (tA * p.ngs_k + (blk >> p.kshift)))));
+                        const float k1 = __half2float(__ushort_as_half(
+                            (unsigned short)lds_u16(sbase, ssk + 2 * ((tA + 1) * p.ngs_k + (blk >> p.kshift)))));
+                        v[0] = fmaf(k0, (float)(ah[0] * 254 + al[0]), v[0]);
+                        v[1] = fmaf(k0, (float)(ah[1] * 254 + al[1]), v[1]);
+                        v[2] = fmaf(k1, (float)(ah[2] * 254 + al[2]), v[2]);
+                        v[3] = fmaf(k1, (float)(ah[3] * 254 + al[3]), v[3]);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 4; e++) s2[u][e] = v[e] * sqc[e & 1];
+                }
+            }
+        } else {
+            // fp16 keys: two partial accumulators per sub-tile halve the MMA chain
             float acc[2][2][4];
 #pragma unroll
             for (int u = 0; u < 2; u++)
@@ -513,67 +736,26 @@ __global__ void __launch_bounds__(NTHR, 2)
             for (int blk = 0; blk < NG; blk++) {
 #pragma unroll
                 for (int u = 0; u < 2; u++) {
-                    uint32_t fa[2][4];
-                    key_frags(st + kofs[u][0], st + kofs[u][1], blk, fa);
-#pragma unroll
-                    for (int hs = 0; hs < 2; hs++)
-                        mma_16816(acc[u][blk & 1], fa[hs][0], fa[hs][1], fa[hs][2], fa[hs][3],
-                                  qb[blk][hs][0], qb[blk][hs][1]);
+                    const uint4 r0 = lds_u128(sbase, blk_addr<RK, SK>(st + kofs[u][0], blk));
+                    const uint4 r1 = lds_u128(sbase, blk_addr<RK, SK>(st + kofs[u][1], blk));
+                    mma_16816(acc[u][blk & 1], r0.x, r1.x, r0.y, r1.y, qb[blk][0][0], qb[blk][0][1]);
+                    mma_16816(acc[u][blk & 1], r0.z, r1.z, r0.w, r1.w, qb[blk][1][0], qb[blk][1][1]);
                 }
             }
 #pragma unroll
-            for (int u = 0; u < 2; u++) {
-                float ks0 = p.tau_log2e, ks1 = p.tau_log2e;
-                if (KB != 16) {
-                    const float2 kk = unpack_half2(lds_u32(sbase, ssk + 2 * tAu[u]));
-                    ks0 *= kk.x;
-                    ks1 *= kk.y;
+            for (int u = 0; u < 2; u++)
+#pragma unroll
+                for (int e = 0; e < 4; e++) {
+                    float v = (acc[u][0][e] + acc[u][1][e]) * p.tau_log2e;
+                    if (qsplit) v += __shfl_xor_sync(FULL, v, 2);
+                    s2[u][e] = v;
                 }
-                s2[u][0] = (acc[u][0][0] + acc[u][1][0] - qbias[0][0]) * ks0;
-                s2[u][1] = (acc[u][0][1] + acc[u][1][1] - qbias[0][1]) * ks0;
-                s2[u][2] = (acc[u][0][2] + acc[u][1][2] - qbias[0][0]) * ks1;
-                s2[u][3] = (acc[u][0][3] + acc[u][1][3] - qbias[0][1]) * ks1;
-            }
-        } else {
-#pragma unroll
-            for (int u = 0; u < 2; u++) {
-                float acc[NG][4];
-#pragma unroll
-                for (int blk = 0; blk < NG; blk++) {
-                    acc[blk][0] = acc[blk][1] = acc[blk][2] = acc[blk][3] = 0.f;
-                    uint32_t fa[2][4];
-                    key_frags(st + kofs[u][0], st + kofs[u][1], blk, fa);
-#pragma unroll
-                    for (int hs = 0; hs < 2; hs++)
-                        mma_16816(acc[blk], fa[hs][0], fa[hs][1], fa[hs][2], fa[hs][3],
-                                  qb[blk][hs][0], qb[blk][hs][1]);
-                }
-                float v[4] = {0.f, 0.f, 0.f, 0.f};
-                const int tA = tAu[u];
-#pragma unroll
-                for (int blk = 0; blk < NG; blk++) {
-                    const float k0 = __half2float(__ushort_as_half(
-                        (unsigned short)lds_u16(sbase, ssk + 2 * (tA * p.ngs_k + (blk >> p.kshift)))));
-                    const float k1 = __half2float(__ushort_as_half(
-                        (unsigned short)lds_u16(sbase, ssk + 2 * ((tA + 1) * p.ngs_k + (blk >> p.kshift)))));
-                    v[0] = fmaf(k0, acc[blk][0] - qbias[blk][0], v[0]);
-                    v[1] = fmaf(k0, acc[blk][1] - qbias[blk][1], v[1]);
-                    v[2] = fmaf(k1, acc[blk][2] - qbias[blk][0], v[2]);
-                    v[3] = fmaf(k1, acc[blk][3] - qbias[blk][1], v[3]);
-                }
-#pragma unroll
-                for (int e = 0; e < 4; e++) s2[u][e] = v[e] * p.tau_log2e;
-            }
         }
 #pragma unroll
         for (int u = 0; u < 2; u++) {
-            if (qsplit) {
-#pragma unroll
-                for (int e = 0; e < 4; e++) s2[u][e] += __shfl_xor_sync(FULL, s2[u][e], 2);
-            }
-            // Padding columns (heads >= G, or the hi/lo halves of a split query)
-            // carry finite scores from zero query columns; their outputs are never
-            // written, so only tokens past the length are masked.
+            // Padding columns (heads >= G, or the residual columns of a split
+            // query) carry finite scores from zero query columns; their outputs
+            // are never written, so only tokens past the length are masked.
             s2[u][0] = vt[u][0] ? s2[u][0] : -INFINITY;
             s2[u][1] = vt[u][0] ? s2[u][1] : -INFINITY;
             s2[u][2] = vt[u][1] ? s2[u][2] : -INFINITY;
@@ -656,6 +838,8 @@ __global__ void __launch_bounds__(NTHR, 2)
         }
 
         // ---------------- phase 4: P (fp16, value scale folded) -> B fragments ----
+        // x0 = rows 0..7 of the score tile (tokens tw + row_token(r)), x1 = rows
+        // 8..15; their 8x8 transposes are the B fragments of the P.V MMA.
         uint32_t pb[2][NG][2];
         const int nvb = vgrp ? NG : 1;
 #pragma unroll
@@ -669,17 +853,12 @@ __global__ void __launch_bounds__(NTHR, 2)
 #pragma unroll
             for (int g = 0; g < NG; g++) {
                 if (g < nvb) {
-                    const uint32_t ha = pack_half2(pr[0] * sv[u][0][g], pr[2] * sv[u][1][g]);  // col 2tig
-                    const uint32_t hb = pack_half2(pr[1] * sv[u][0][g], pr[3] * sv[u][1][g]);  // col 2tig+1
-                    const float2 fa = unpack_half2(ha), fb = unpack_half2(hb);
-                    psum[g][0] += fa.x + fa.y;
-                    psum[g][1] += fb.x + fb.y;
-                    const uint32_t x0 = __shfl_sync(FULL, ha, src0);
-                    const uint32_t y0 = __shfl_sync(FULL, hb, src0);
-                    const uint32_t x1 = __shfl_sync(FULL, ha, src1);
-                    const uint32_t y1 = __shfl_sync(FULL, hb, src1);
-                    pb[u][g][0] = odd ? y0 : x0;
-                    pb[u][g][1] = odd ? y1 : x1;
+                    const uint32_t x0 = pack_half2(pr[0] * sv[u][0][g], pr[1] * sv[u][0][g]);
+                    const uint32_t x1 = pack_half2(pr[2] * sv[u][1][g], pr[3] * sv[u][1][g]);
+                    pb[u][g][0] = movmatrix_trans(x0);
+                    pb[u][g][1] = movmatrix_trans(x1);
+                    // column sums of the fp16 weights, for the code bias
+                    if (VB != 16) mma_16816(psum[g], ONE2, ONE2, ONE2, ONE2, pb[u][g][0], pb[u][g][1]);
                 } else {
                     pb[u][g][0] = pb[u][0][0];
                     pb[u][g][1] = pb[u][0][1];
@@ -726,12 +905,12 @@ __global__ void __launch_bounds__(NTHR, 2)
                     }
                 } else {
                     // fp16 values past the length may be anything (NaN included): zero them
-                    const int tg = m.t0 + warp * 32 + u * 16 + 2 * tig;
+                    const int tg = m.t0 + warp * 32 + u * 16;
                     const uint2 z = make_uint2(0u, 0u);
-                    const uint2 wA = tg < m.len ? lds_u64(sbase, blk_addr<RV, SV>(va, blk)) : z;
-                    const uint2 wB = tg + 1 < m.len ? lds_u64(sbase, blk_addr<RV, SV>(vb, blk)) : z;
-                    const uint2 wC = tg + 8 < m.len ? lds_u64(sbase, blk_addr<RV, SV>(vc, blk)) : z;
-                    const uint2 wE = tg + 9 < m.len ? lds_u64(sbase, blk_addr<RV, SV>(ve, blk)) : z;
+                    const uint2 wA = tg + vA < m.len ? lds_u64(sbase, blk_addr<RV, SV>(va, blk)) : z;
+                    const uint2 wB = tg + vB < m.len ? lds_u64(sbase, blk_addr<RV, SV>(vb, blk)) : z;
+                    const uint2 wC = tg + vA + 1 < m.len ? lds_u64(sbase, blk_addr<RV, SV>(vc, blk)) : z;
+                    const uint2 wE = tg + vB + 1 < m.len ? lds_u64(sbase, blk_addr<RV, SV>(ve, blk)) : z;
 #pragma unroll
                     for (int h = 0; h < 2; h++) {
                         const uint32_t A = h ? wA.y : wA.x, Bw = h ? wB.y : wB.x;
@@ -752,9 +931,10 @@ __global__ void __launch_bounds__(NTHR, 2)
             ph ^= 1u;
         }
 
-        // ---------------- segment end: merge the warps, write the partial ---
+        // ---------------- segment end: combine the warps, write the partial ------
         if (m.flags & 2) {
-            float lt[2], ps[NG][2];
+            constexpr int CS = slot_col_floats(DH);
+            float lt[2];
 #pragma unroll
             for (int c = 0; c < 2; c++) {
                 float v = l_run[c];
@@ -762,36 +942,26 @@ __global__ void __launch_bounds__(NTHR, 2)
                 v += __shfl_xor_sync(FULL, v, 8);
                 v += __shfl_xor_sync(FULL, v, 16);
                 lt[c] = v;
-#pragma unroll
-                for (int g = 0; g < NG; g++) {
-                    float w = psum[g][c];
-                    w += __shfl_xor_sync(FULL, w, 4);
-                    w += __shfl_xor_sync(FULL, w, 8);
-                    w += __shfl_xor_sync(FULL, w, 16);
-                    ps[g][c] = w;
-                }
             }
-            // merge buffer: [NW][G][DH + 2] floats: o then (m, l)
-            float *mine = mbuf + (size_t)warp * G * (DH + 2);
+            // this warp's partial into mbuf[warp]: [G][DH + 4] floats, o then (m, l)
+            float *mine = mbuf + (size_t)warp * G * CS;
 #pragma unroll
             for (int c = 0; c < 2; c++) {
                 const int col = 2 * tig + c;
                 if (c == 0 ? col_ok0 : col_ok1) {
-                    float *oc = mine + (size_t)col * (DH + 2);
+                    float *oc = mine + (size_t)col * CS;
 #pragma unroll
                     for (int blk = 0; blk < NG; blk++) {
-                        const float corr = BIAS_V * ps[vgrp ? blk : 0][c];
+                        const float corr = BIAS_V * psum[vgrp ? blk : 0][c];
 #pragma unroll
                         for (int h = 0; h < 2; h++) {
+                            // m-tile 2blk+h: row gid <-> d = 32blk + 4gid + 2h, row gid+8 <-> d + 1
                             const int d = 32 * blk + 4 * gid + 2 * h;
-                            oc[d] = o_acc[2 * blk + h][c] - corr;
-                            oc[d + 1] = o_acc[2 * blk + h][2 + c] - corr;
+                            *reinterpret_cast<float2 *>(oc + d) =
+                                make_float2(o_acc[2 * blk + h][c] - corr, o_acc[2 * blk + h][2 + c] - corr);
                         }
                     }
-                    if (gid == 0) {
-                        oc[DH] = m_run[c];
-                        oc[DH + 1] = lt[c];
-                    }
+                    if (gid == 0) *reinterpret_cast<float2 *>(oc + DH) = make_float2(m_run[c], lt[c]);
                 }
             }
             __syncwarp();
@@ -801,39 +971,33 @@ __global__ void __launch_bounds__(NTHR, 2)
                 atomicExch(p.status, KVQ_ERR_TIMEOUT);
                 break;
             }
-            // combine the NW warps deterministically and write the slot
-            const int slot = m.flags >> 8;
-            float *dst = p.ws + (size_t)slot * G * (DH + 2);
-            for (int idx = tid; idx < G * DH; idx += 32 * NW) {
-                const int col = idx / DH, d = idx % DH;
+            // combine the NW warps (each takes a quarter of the float4 chunks) and
+            // write this CTA's partial of the segment
+            const int ncol = qsplit ? min(G, 4) : G;
+            float *dst = p.ws + (size_t)m.slot * G * CS;
+            for (int k = warp * 32 + lane; k < ncol * (DH / 4); k += 32 * NW) {
+                const int col = k / (DH / 4), d = 4 * (k % (DH / 4));
                 float M = -INFINITY;
 #pragma unroll
-                for (int w = 0; w < NW; w++) M = fmaxf(M, mbuf[((size_t)w * G + col) * (DH + 2) + DH]);
-                float O = 0.f;
-#pragma unroll
-                for (int w = 0; w < NW; w++) {
-                    const float *src = mbuf + ((size_t)w * G + col) * (DH + 2);
-                    const float mw = src[DH];
-                    const float e = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
-                    O += e * src[d];
-                }
-                dst[(size_t)col * (DH + 2) + d] = O;
-            }
-            if (tid < G) {
-                const int col = tid;
-                float M = -INFINITY;
-#pragma unroll
-                for (int w = 0; w < NW; w++) M = fmaxf(M, mbuf[((size_t)w * G + col) * (DH + 2) + DH]);
+                for (int w = 0; w < NW; w++) M = fmaxf(M, mbuf[((size_t)w * G + col) * CS + DH]);
+                float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
                 float L = 0.f;
 #pragma unroll
                 for (int w = 0; w < NW; w++) {
-                    const float *src = mbuf + ((size_t)w * G + col) * (DH + 2);
+                    const float *src = mbuf + ((size_t)w * G + col) * CS;
                     const float mw = src[DH];
-                    L += (mw == -INFINITY) ? 0.f : exp2f(mw - M) * src[DH + 1];
+                    const float e = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+                    const float4 x = *reinterpret_cast<const float4 *>(src + d);
+                    O.x = fmaf(e, x.x, O.x);
+                    O.y = fmaf(e, x.y, O.y);
+                    O.z = fmaf(e, x.z, O.z);
+                    O.w = fmaf(e, x.w, O.w);
+                    L = fmaf(e, src[DH + 1], L);
                 }
-                dst[(size_t)col * (DH + 2) + DH] = M;
-                dst[(size_t)col * (DH + 2) + DH + 1] = L;
+                *reinterpret_cast<float4 *>(dst + (size_t)col * CS + d) = O;
+                if (d == 0) *reinterpret_cast<float2 *>(dst + (size_t)col * CS + DH) = make_float2(M, L);
             }
+            // mbuf is free again once every warp has read it
             __syncwarp();
             if (lane == 0) mbar_arrive(&segbar[1]);
             if (!mbar_wait_bounded(&segbar[1], seg_parity, abort_flag, limit)) {
@@ -842,24 +1006,41 @@ __global__ void __launch_bounds__(NTHR, 2)
                 break;
             }
             seg_parity ^= 1u;
+            if (p.counters != nullptr) {
+                // the warp that completes the last partial of this (sequence, KV
+                // head) merges them (publish: fence, then count the arrival)
+                __threadfence();
+                __syncwarp();
+                int last = 0;
+                if (lane == 0) last = atomicAdd(&p.counters[m.bh], 1) == NW * m.ncta - 1;
+                last = __shfl_sync(FULL, last, 0);
+                if (last) {
+                    __threadfence();
+                    const int b = m.bh / Hkv, kvh = m.bh % Hkv;
+                    merge_segment<DH>(p.ws, (int64_t)m.cmin + m.bh, m.ncta, G, p.out, p.out_f32,
+                                      ((int64_t)b * p.n_q_heads + (int64_t)kvh * G) * DH, lane);
+                    if (lane == 0) p.counters[m.bh] = 0;   // ready for the next launch
+                }
+            }
         }
     }
 }
 
 // ---------------------------------------------------------------------------
-// merge: one warp per (sequence, query head)
+// merge launch (partials left by a decode launch without counters): one warp
+// per (sequence, KV head)
 // ---------------------------------------------------------------------------
 template <int DH>
 __global__ void __launch_bounds__(256) merge_kernel(const MergeParams p)
 {
     const int lane = threadIdx.x & 31;
     const int64_t gw = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (gw >= (int64_t)p.batch * p.n_q_heads) return;
-    const int b = (int)(gw / p.n_q_heads);
-    const int h = (int)(gw % p.n_q_heads);
+    if (gw >= (int64_t)p.batch * p.n_kv_heads) return;
+    const int b = (int)(gw / p.n_kv_heads);
+    const int kvh = (int)(gw % p.n_kv_heads);
     const int G = p.group_size_g;
-    const int kvh = h / G, col = h % G;
     const int cap = p.cap;
+    const int64_t obase0 = ((int64_t)b * p.n_q_heads + (int64_t)kvh * G) * DH;
 
     // units before sequence b, and in total
     long long before = 0, total = 0;
@@ -869,51 +1050,27 @@ __global__ void __launch_bounds__(256) merge_kernel(const MergeParams p)
         if (bb < b) before += t;
     }
     for (int off = 16; off; off >>= 1) {
-        total += __shfl_xor_sync(0xffffffffu, total, off);
-        before += __shfl_xor_sync(0xffffffffu, before, off);
+        total += __shfl_xor_sync(FULL, total, off);
+        before += __shfl_xor_sync(FULL, before, off);
     }
     const int tiles_b = tiles_of(p.d_len[b], cap);
+    if (tiles_b == 0) {
+        for (int i = lane; i < G * DH; i += 32) {
+            if (p.out_f32)
+                static_cast<float *>(p.out)[obase0 + i] = 0.f;
+            else
+                static_cast<__half *>(p.out)[obase0 + i] = __float2half_rn(0.f);
+        }
+        return;
+    }
     const long long N = total * p.n_kv_heads;
-    const long long P = p.num_ctas;
+    const long long Pe = N < (long long)p.num_ctas ? N : (long long)p.num_ctas;
     const long long u0 = before * p.n_kv_heads + (long long)kvh * tiles_b;
     const long long u1 = u0 + tiles_b;
+    const long long cmin = ((u0 + 1) * Pe + N - 1) / N - 1;
+    const long long cmax = (u1 * Pe + N - 1) / N - 1;
     const int bh = b * p.n_kv_heads + kvh;
-
-    constexpr int PER = DH / 32;
-    float o[PER];
-#pragma unroll
-    for (int i = 0; i < PER; i++) o[i] = 0.f;
-    float M = -INFINITY, L = 0.f;
-    if (tiles_b > 0) {
-        const long long c_min = ((u0 + 1) * P + N - 1) / N - 1;
-        const long long c_max = (u1 * P + N - 1) / N - 1;
-        for (int pass = 0; pass < 2; pass++) {
-            for (long long c = c_min; c <= c_max; c++) {
-                const long long cs = c * N / P, ce = (c + 1) * N / P;
-                if (!(max(cs, u0) < min(ce, u1))) continue;
-                const float *slot = p.ws + (size_t)(c + bh) * G * (DH + 2) + (size_t)col * (DH + 2);
-                const float mk = slot[DH];
-                if (pass == 0) {
-                    M = fmaxf(M, mk);
-                } else if (mk != -INFINITY) {
-                    const float e = exp2f(mk - M);
-                    L += e * slot[DH + 1];
-#pragma unroll
-                    for (int i = 0; i < PER; i++) o[i] += e * slot[lane + 32 * i];
-                }
-            }
-        }
-    }
-    const float inv = (L > 0.f) ? 1.f / L : 0.f;
-    const int64_t obase = ((int64_t)b * p.n_q_heads + h) * DH;
-#pragma unroll
-    for (int i = 0; i < PER; i++) {
-        const float v = o[i] * inv;
-        if (p.out_f32)
-            static_cast<float *>(p.out)[obase + lane + 32 * i] = v;
-        else
-            static_cast<__half *>(p.out)[obase + lane + 32 * i] = __float2half_rn(v);
-    }
+    merge_segment<DH>(p.ws, cmin + bh, (int)(cmax - cmin + 1), G, p.out, p.out_f32, obase0, lane);
 }
 
 template <int DH, int KB, int VB>
@@ -952,11 +1109,11 @@ bool plan_decode(int dh, int kb, int vb, int ngs_k, int ngs_v, int G, int max_sm
     L.off_sk = L.off_v + align_up(T * rv, 1024);
     L.off_sv = L.off_sk + align_up(T * (kb == 16 ? 0 : ngs_k) * 2, 16);
     L.stage_bytes = align_up(L.off_sv + T * (vb == 16 ? 0 : ngs_v) * 2, 1024);
-    const uint32_t merge_bytes = (uint32_t)NW * G * (dh + 2) * 4;
-    // tail: meta[S] (16 B each), barriers (2S + 2) * 8, ctl 32 B, merge buffer
+    const uint32_t merge_bytes = (uint32_t)NW * G * slot_col_floats(dh) * 4;
+    // tail: meta[S] (32 B each), barriers (2S + 2) * 8 B, control words 32 B, merge buffer
     for (int S = 8; S >= 2; S--) {
         const uint32_t off_meta = S * L.stage_bytes;
-        const uint32_t off_bar = off_meta + S * 16;
+        const uint32_t off_bar = off_meta + S * (uint32_t)sizeof(StageMeta);
         const uint32_t off_merge = align_up(off_bar + (2 * S + 2) * 8 + 32, 16);
         const uint32_t total = off_merge + merge_bytes + 1024;  // + alignment slack
         // keep two CTAs per SM when possible
@@ -1048,7 +1205,7 @@ cudaError_t launch_decode(const DecodeLaunch &plan, const DecodeParams &p, const
 
 cudaError_t launch_merge(const MergeParams &p, cudaStream_t stream)
 {
-    const int64_t warps = (int64_t)p.batch * p.n_q_heads;
+    const int64_t warps = (int64_t)p.batch * p.n_kv_heads;
     if (warps == 0) return cudaSuccess;
     const unsigned blocks = (unsigned)((warps + 7) / 8);
     (void)cudaGetLastError();  // drop a stale, already-reported error of an earlier call

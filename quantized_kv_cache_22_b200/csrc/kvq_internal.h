@@ -26,13 +26,25 @@ constexpr int kDecodeTileTokens = 32 * kDecodeConsumerWarps;   // tokens per sta
 constexpr int kDecodeThreads = 32 * (kDecodeConsumerWarps + 1);
 constexpr int kWorkspaceHeaderFloats = 64;                      // status word + padding
 
+// The new token's K/V for the append step fused into the decode kernel.
+struct FusedAppend {
+    const void *k_new, *v_new;    // [B][Hkv][Dh] in dtype; null: no append
+    uint8_t *k_codes, *v_codes;   // the layer's cache (same memory the TMA maps read)
+    __half *k_scales, *v_scales;
+    int32_t dtype;                // KVQ_F16 / KVQ_F32 / KVQ_BF16
+    int32_t k_group, v_group;     // elements per scale (32 at 16 bits)
+};
+
 struct DecodeParams {
     const int32_t *d_len;     // [B]
     const void *q;            // [B][Hq][Dh]
     const __half *k_scales;   // [B][Hkv][cap][ngs_k]   (null at 16 bits)
     const __half *v_scales;
-    float *ws;                // partial slots (after the header)
+    float *ws;                // per-warp partial slots
     int *status;              // workspace status word
+    int *counters;            // [B*Hkv] warp arrivals; null: leave the partials for a merge launch
+    void *out;                // [B][Hq][Dh] (fused merge only)
+    int32_t out_f32;
     int32_t q_dtype;
     int32_t batch, n_q_heads, n_kv_heads, group_size_g, cap;
     int32_t ngs_k, ngs_v;     // scales per row
@@ -42,6 +54,7 @@ struct DecodeParams {
     uint32_t stage_bytes, off_v, off_sk, off_sv, off_meta, off_bar, off_merge;
     float tau_log2e;
     uint64_t timeout_ns;
+    FusedAppend app;
 };
 
 struct MergeParams {
@@ -68,11 +81,19 @@ cudaError_t launch_decode(const DecodeLaunch &plan, const DecodeParams &p, const
                           const CUtensorMap &tm_v, cudaStream_t stream);
 cudaError_t launch_merge(const MergeParams &p, cudaStream_t stream);
 
-// Floats of one partial slot and slot count for a launch.
-inline uint64_t slot_floats(int G, int dh) { return (uint64_t)G * (uint64_t)(dh + 2); }
+// Workspace: [header][counters][partial slots].  A partial slot holds, for the
+// G query heads of one KV head, a record of Dh + 4 floats each: o[Dh], m, l and
+// two floats of padding that keep every record 16-byte aligned.  A CTA writes
+// one slot for each (sequence, KV head) segment it works on.
+__host__ __device__ constexpr int slot_col_floats(int dh) { return dh + 4; }
+inline uint64_t slot_floats(int G, int dh) { return (uint64_t)G * (uint64_t)slot_col_floats(dh); }
 inline uint64_t slot_count(int num_ctas, int batch, int n_kv_heads)
 {
     return (uint64_t)num_ctas + (uint64_t)batch * (uint64_t)n_kv_heads;
+}
+inline uint64_t counter_ints(int batch, int n_kv_heads)
+{
+    return ((uint64_t)batch * (uint64_t)n_kv_heads + 63) / 64 * 64;
 }
 
 // ------------------------------------------------------------------ h-mode GEMM

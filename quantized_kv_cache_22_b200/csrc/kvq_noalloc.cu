@@ -12,6 +12,7 @@
 
 #include <cuda_runtime.h>
 
+#include "kvq_internal.h"
 #include "../../include/kvq.h"
 
 namespace {
@@ -57,9 +58,12 @@ extern "C" int kvq_decode_attn_noalloc(const kvq_config *cfg, const kvq_layer *l
     void *ws = nullptr;
     rc = scratch_address(&ws);
     if (rc) return rc;
-    // the status word must start at zero; the partial slots are written before
-    // they are read, so nothing else needs clearing
-    if (cudaMemsetAsync(ws, 0, 4, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    // the status word and the merge's arrival counters must start at zero (a
+    // call that timed out can leave counters behind); the partial slots are
+    // written before they are read, so nothing else needs clearing
+    const uint64_t zero_bytes = (uint64_t)kvq::kWorkspaceHeaderFloats * 4 +
+                                kvq::counter_ints(cfg->batch, cfg->n_kv_heads) * 4;
+    if (cudaMemsetAsync(ws, 0, zero_bytes, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
         return KVQ_ERR_LAUNCH;
     return kvq_decode_attn(cfg, layer, q, q_dtype, d_len, max_len_host, softmax_scale, out,
                            out_dtype, ws, kScratchBytes, num_ctas, nullptr, nullptr, 0, stream);

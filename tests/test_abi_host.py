@@ -80,9 +80,10 @@ def test_workspace_bytes_explicit_ctas_without_device():
     cfg = Config(batch=16, capacity=8192, n_q_heads=32, n_kv_heads=8, head_dim=128)
     a = kvq.kvq_workspace_bytes(cfg, num_ctas=296)
     b = kvq.kvq_workspace_bytes(cfg, num_ctas=300)
-    # header + (ctas + B*Hkv) slots of G*(Dh+2) floats
-    assert a == 256 + (296 + 128) * 4 * 130 * 4
-    assert b - a == 4 * 4 * 130 * 4
+    # header + B*Hkv arrival counters (rounded up to 64) + (CTAs + B*Hkv)
+    # partial slots of G*(Dh+4) floats
+    assert a == 256 + 128 * 4 + (296 + 128) * 4 * 132 * 4
+    assert b - a == 4 * 4 * 132 * 4
 
 
 def _rc(fn, *args):

@@ -20,7 +20,7 @@ from _helpers import TOL, gpu_cache, gpu_decode, oracle_cache, vmax_per_batch
 
 pytestmark = pytest.mark.gpu
 
-LIMIT = 2 * 1024 * 1024  # KVQ_NOALLOC_SCRATCH_BYTES
+LIMIT = 8 * 1024 * 1024  # KVQ_NOALLOC_SCRATCH_BYTES
 
 
 def _noalloc_fn():
@@ -65,7 +65,7 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(cuda_device):
 
 
 def test_noalloc_rejects_configs_beyond_its_scratch(cuda_device):
-    # B*Hkv = 4096 sequences x heads needs far more than 2 MiB of partials
+    # B*Hkv = 4096 sequences x heads needs far more than 8 MiB of partials
     B, Hkv, G, dh, cap = 512, 8, 8, 128, 64
     cfg = Config(batch=B, capacity=cap, n_q_heads=Hkv * G, n_kv_heads=Hkv, head_dim=dh)
     assert kvq.kvq_workspace_bytes(cfg) > LIMIT
