@@ -1,21 +1,28 @@
-"""Build libkvq.so in-tree for sm_100a with nvcc (no JIT, no torch extension)."""
+"""Build libkvq.so in-tree for sm_100a with nvcc (no JIT, no torch extension).
+
+Each .cu file is compiled to an object in parallel (the decode kernel's
+instances are spread over several files), then the objects are linked into
+libkvq.so.  The ptxas report of every file goes to build.log.
+"""
 from __future__ import annotations
 
 import glob
 import os
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libkvq.so")
+OBJ = os.path.join(HERE, "_build")
 
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = [
-    "-O3", "-std=c++17", "-shared", "-Xcompiler", "-fPIC,-fvisibility=hidden",
-    "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
+    "-O3", "-std=c++17", "-Xcompiler", "-fPIC,-fvisibility=hidden", "-lineinfo",
     "-Xptxas", "-v", "--expt-relaxed-constexpr",
-]
+] + ARCH
 
 
 def sources():
@@ -28,19 +35,38 @@ def _stale() -> bool:
     t = os.path.getmtime(LIB)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h"))
     deps.append(os.path.join(ROOT, "include", "kvq.h"))
+    deps.append(os.path.abspath(__file__))
     return any(os.path.getmtime(d) > t for d in deps)
+
+
+def _compile(nvcc: str, src: str):
+    obj = os.path.join(OBJ, os.path.basename(src)[:-3] + ".o")
+    cmd = [nvcc] + NVCC_FLAGS + ["-I", os.path.join(ROOT, "include"), "-c", src, "-o", obj]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    return obj, cmd, res
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and not _stale():
         return LIB
     nvcc = os.environ.get("NVCC", "nvcc")
-    cmd = [nvcc] + NVCC_FLAGS + ["-I", os.path.join(ROOT, "include"), "-o", LIB + ".tmp"] + sources()
-    res = subprocess.run(cmd, capture_output=True, text=True)
-    log = res.stdout + res.stderr
+    os.makedirs(OBJ, exist_ok=True)
+    srcs = sources()
+    with ThreadPoolExecutor(max_workers=min(len(srcs), os.cpu_count() or 4)) as ex:
+        results = list(ex.map(lambda s: _compile(nvcc, s), srcs))
+    log = ""
+    failed = False
+    for obj, cmd, res in results:
+        log += " ".join(cmd) + "\n" + res.stdout + res.stderr
+        failed |= res.returncode != 0
+    if not failed:
+        link = [nvcc, "-shared"] + ARCH + ["-o", LIB + ".tmp"] + [r[0] for r in results]
+        res = subprocess.run(link, capture_output=True, text=True)
+        log += " ".join(link) + "\n" + res.stdout + res.stderr
+        failed = res.returncode != 0
     with open(os.path.join(HERE, "build.log"), "w") as f:
-        f.write(" ".join(cmd) + "\n" + log)
-    if res.returncode != 0:
+        f.write(log)
+    if failed:
         sys.stderr.write(log)
         raise RuntimeError("nvcc failed building libkvq.so")
     if verbose:

@@ -1,0 +1,1102 @@
+// kvq_decode_kernel.cuh -- the split-KV decode attention kernel over a quantised
+// KV cache (instantiated in kvq_decode_k4/k8/k16.cu; host side in kvq_decode.cu).
+//
+// What it computes (the pages' problem statement): one query token per
+// sequence attends over every cached token of its KV head (mni-ml page: keep
+// past K/V, compute only the new token's); K and V are dequantised inside the
+// attention kernel (KVSplit discussion: integrate the formats into the
+// FlashAttention kernel), with INT8 / nibble-packed INT4 codes and fp16
+// scales per (token, head) or per group (TinyLoop mode table; KVSplit 8K
+// table).  Output = softmax(tau q.K^T) V, fp32 accumulation.  Optionally the
+// new token's K/V are quantised into the cache by the same launch first
+// (quantize-on-append, TinyLoop "KV Cache 模式").
+//
+// Design for sm_100a (not taken from any page):
+//   * Persistent CTAs, work split stream-K style: the units are 128-token
+//     tiles of every (sequence, KV head); CTA c of the P' = min(P, units) CTAs
+//     that get work takes units [cN/P', (c+1)N/P').  Every CTA streams the same
+//     number of bytes whatever B, Hkv and the lengths are.  A CTA's run of
+//     tiles inside one (sequence, KV head) is a "segment"; at its end the
+//     consumer warps combine their partials (m, l, o) in shared memory and
+//     write one per segment to the workspace, at slot (cta + sequence*Hkv +
+//     kv_head), which is unique.  The warp that completes the last of the
+//     partials of a (sequence, KV head) -- an arrival counter tells it --
+//     merges them with their log-sum-exp weights and writes the output, so one
+//     launch does the whole layer.
+//   * One producer warp streams tiles with TMA: codes through 3-D tiled tensor
+//     maps with 128-byte swizzle (bank-conflict-free fragment reads), scales
+//     with 1-D bulk copies, into a multi-stage shared-memory ring guarded by
+//     mbarriers.  Every wait is bounded (about a second) and a give-up sets
+//     the workspace status word instead of hanging.  Before it loads the tile
+//     that holds a sequence's newest token, the producer warp quantises that
+//     token into the cache (the fused append) and fences the writes against
+//     the copy engine.
+//   * Four consumer warps each take 32 tokens of a stage as two 16-token
+//     sub-tiles.  q.K^T runs on int8 tensor-core MMA (m16n8k32): the key codes
+//     feed the MMA as they are stored (4-bit codes after one mask, as 16x the
+//     code), and the query is split per head into two int8 parts, q ~ s (hi +
+//     lo/254), so the products keep ~16 bits of the query.  P.V runs on f16
+//     MMA (m16n8k16, f32 accumulate) with head_dim as M and the G query heads
+//     of the KV group as N: value codes become fp16 in registers with the
+//     exponent-bias trick (a code byte u in the mantissa of 0x6400 reads 1024
+//     + u), value scales are folded into the probabilities, and the constant
+//     bias is removed at the end with the probability sums, which one extra
+//     MMA against a matrix of ones accumulates.  The score tile is turned into
+//     the P operand by two 8x8 transposes (movmatrix).
+//   * The online softmax tracks max(s + log2 s_V) so that p * s_V <= 2^8 fits
+//     fp16 without underflow whatever the value scales are.
+#pragma once
+#include <cfloat>
+#include <type_traits>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "kvq_internal.h"
+#include "kvq_ptx.cuh"
+#include "kvq_quant.cuh"
+#include "../../include/kvq.h"
+
+namespace kvq {
+namespace {
+
+constexpr int NW = kDecodeConsumerWarps;
+constexpr int T = kDecodeTileTokens;
+constexpr int NTHR = kDecodeThreads;
+constexpr unsigned FULL = 0xffffffffu;
+
+struct __align__(16) StageMeta {
+    int32_t bh;      // sequence * Hkv + kv_head
+    int32_t t0;      // first token of the tile
+    int32_t len;     // tokens attended by this sequence
+    int32_t flags;   // bit0 first tile of a segment, bit1 last tile of a segment
+    int32_t slot;    // partial slot of this CTA's segment: cta + bh
+    int32_t ncta;    // CTAs holding a segment of this (sequence, KV head)
+    int32_t cmin;    // the first of them
+    int32_t pad;
+};
+
+// Byte offset of element byte `o` of token `t` inside a stage tile that TMA
+// wrote with 128-byte swizzle.  Rows of R <= 128 bytes are packed 128/R tokens
+// per 128-byte line; R = 256 is stored as two 128-byte-wide boxes.
+template <int R>
+__host__ __device__ constexpr uint32_t sw_off(int t, int o)
+{
+    if constexpr (R <= 128) {
+        constexpr int TPL = 128 / R;
+        const int line = t / TPL;
+        const int col = (t % TPL) * R + o;
+        return (uint32_t)(line * 128 + ((((col >> 4) ^ line) & 7) << 4) + (col & 15));
+    } else {
+        const int sub = o >> 7, col = o & 127;
+        return (uint32_t)(sub * (T * 128) + t * 128 + ((((col >> 4) ^ t) & 7) << 4) + (col & 15));
+    }
+}
+
+// Token of row g (g < 8) of a 16-token sub-tile's score tile; row g + 8 holds
+// the next token.  The permutation pi(g) = g ^ (g >> 2) keeps both the key-row
+// reads of the score MMA and the value-row reads of the P.V MMA (whose k
+// order follows the score rows through the transpose) free of bank conflicts.
+__host__ __device__ constexpr int row_token(int g) { return 2 * (g ^ (g >> 2)); }
+
+// fp16 pair helpers: value code bytes / nibbles -> half2 of (bias + code).
+__device__ __forceinline__ uint32_t i4_pair(uint32_t w, int k)
+{
+    return and_xor(w >> (4 * k), 0x000F000Fu, 0x64086408u);
+}
+
+__device__ __forceinline__ float load_qf(const void *q, int dtype, int64_t idx)
+{
+    if (dtype == KVQ_F16) return __half2float(static_cast<const __half *>(q)[idx]);
+    if (dtype == KVQ_F32) return static_cast<const float *>(q)[idx];
+    return __bfloat162float(static_cast<const __nv_bfloat16 *>(q)[idx]);
+}
+
+__device__ __forceinline__ int clamp_len(int len, int cap)
+{
+    return len < 0 ? 0 : (len > cap ? cap : len);
+}
+
+__device__ __forceinline__ int tiles_of(int len, int cap) { return (clamp_len(len, cap) + T - 1) / T; }
+
+// 2^x with the hardware approximation (relative error ~2^-22); results below
+// 2^-126 flush to zero, which only drops probabilities that are zero anyway.
+__device__ __forceinline__ float fast_exp2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Loads from the stage ring.  `b` is the 32-bit shared-window address of the
+// 1024-aligned ring base and `o` a byte offset from it; explicit ld.shared keeps the
+// address arithmetic 32-bit.  volatile keeps every load after the mbarrier wait
+// that guards its stage (the wait is a volatile asm with a memory clobber).
+__device__ __forceinline__ uint32_t lds_u16(uint32_t b, uint32_t o)
+{
+    uint16_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(b + o));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds_u32(uint32_t b, uint32_t o)
+{
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(b + o));
+    return v;
+}
+__device__ __forceinline__ uint2 lds_u64(uint32_t b, uint32_t o)
+{
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(b + o));
+    return v;
+}
+__device__ __forceinline__ uint4 lds_u128(uint32_t b, uint32_t o)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(b + o));
+    return v;
+}
+
+// The same loads at the shared address a + IMM, IMM a compile-time byte offset
+// that the load instruction carries itself.
+template <int IMM>
+__device__ __forceinline__ uint32_t ldsi_u16(uint32_t a)
+{
+    uint16_t v;
+    asm volatile("ld.shared.u16 %0, [%1+%2];" : "=h"(v) : "r"(a), "n"(IMM));
+    return v;
+}
+template <int IMM>
+__device__ __forceinline__ uint32_t ldsi_u32(uint32_t a)
+{
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1+%2];" : "=r"(v) : "r"(a), "n"(IMM));
+    return v;
+}
+template <int IMM>
+__device__ __forceinline__ uint2 ldsi_u64(uint32_t a)
+{
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2+%3];" : "=r"(v.x), "=r"(v.y) : "r"(a), "n"(IMM));
+    return v;
+}
+template <int IMM>
+__device__ __forceinline__ uint4 ldsi_u128(uint32_t a)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4+%5];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(a), "n"(IMM));
+    return v;
+}
+
+// Address of block `blk` of a row whose block-0 address (stage base + per-lane
+// swizzled offset) is `a0`, for a tile of R-byte rows whose 32-element blocks are
+// STR bytes long: the swizzle is linear in the block index, so block blk sits at
+// a0 ^ sw_off<R>(0, blk*STR).  Rows of 256 bytes keep their second half in a
+// second box T*128 bytes further, which is added rather than XORed because the
+// stage base is only 1024-byte aligned.
+template <int R, int STR>
+__device__ __forceinline__ uint32_t blk_addr(uint32_t a0, int blk)
+{
+    if constexpr (R <= 128) {
+        return a0 ^ sw_off<R>(0, blk * STR);
+    } else {
+        const uint32_t x = sw_off<R>(0, blk * STR);
+        return (a0 ^ (x & (T * 128 - 1))) + (x & ~(uint32_t)(T * 128 - 1));
+    }
+}
+
+__device__ __forceinline__ uint32_t pack_bytes(int a, int b, int c, int d)
+{
+    return (uint32_t)(a & 0xff) | ((uint32_t)(b & 0xff) << 8) | ((uint32_t)(c & 0xff) << 16) |
+           ((uint32_t)(d & 0xff) << 24);
+}
+
+__device__ __forceinline__ float warp_max(float v)
+{
+#pragma unroll
+    for (int off = 16; off; off >>= 1) v = fmaxf(v, __shfl_xor_sync(FULL, v, off));
+    return v;
+}
+__device__ __forceinline__ float warp_sum(float v)
+{
+#pragma unroll
+    for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(FULL, v, off);
+    return v;
+}
+
+// Merge the np CTA partials of one (sequence, KV head), all G query heads at once:
+// slots slot0 .. slot0 + np - 1, each G records of DH + 4 floats holding per
+// query head o[DH], m, l.  out[obase0 + col * DH + d] receives
+//   sum_j o_j[d] 2^(m_j - M) / sum_j l_j 2^(m_j - M),  M = max_j m_j.
+// LPC lanes share one query head (column) and split its DH outputs; the
+// partials are read through L2 (ld.global.cg) because other SMs wrote them in
+// this launch.  One warp.
+template <int DH, int LPC>
+__device__ void merge_segment_lpc(const float *ws, int64_t slot0, int np, int G, void *out,
+                                  int out_f32, int64_t obase0, int lane)
+{
+    constexpr int PER = DH / LPC;       // floats of one partial per lane
+    constexpr int CS = slot_col_floats(DH);
+    const int col = lane / LPC, part = lane % LPC;
+    const bool active = col < G;
+    const int64_t stride = (int64_t)G * CS;
+    const float *base = ws + slot0 * stride + (int64_t)(active ? col : 0) * CS;
+    float M = -INFINITY;
+    if (active)
+        for (int j = part; j < np; j += LPC) M = fmaxf(M, __ldcg(base + j * stride + DH));
+#pragma unroll
+    for (int off = 1; off < LPC; off <<= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, off));
+    float L = 0.f;
+    float o[PER];
+#pragma unroll
+    for (int i = 0; i < PER; i++) o[i] = 0.f;
+    if (active && M != -INFINITY) {
+#pragma unroll 4
+        for (int j = 0; j < np; j++) {
+            const float *src = base + (int64_t)j * stride;
+            const float2 ml = __ldcg(reinterpret_cast<const float2 *>(src + DH));
+            float4 x[PER / 4];
+#pragma unroll
+            for (int i = 0; i < PER / 4; i++)
+                x[i] = __ldcg(reinterpret_cast<const float4 *>(src + part * PER) + i);
+            const float e = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M);
+            L = fmaf(e, ml.y, L);
+#pragma unroll
+            for (int i = 0; i < PER / 4; i++) {
+                o[4 * i] = fmaf(e, x[i].x, o[4 * i]);
+                o[4 * i + 1] = fmaf(e, x[i].y, o[4 * i + 1]);
+                o[4 * i + 2] = fmaf(e, x[i].z, o[4 * i + 2]);
+                o[4 * i + 3] = fmaf(e, x[i].w, o[4 * i + 3]);
+            }
+        }
+    }
+    if (!active) return;
+    const float inv = (L > 0.f) ? 1.f / L : 0.f;
+    const int64_t ob = obase0 + (int64_t)col * DH + part * PER;
+#pragma unroll
+    for (int i = 0; i < PER; i += 2) {
+        if (out_f32)
+            *reinterpret_cast<float2 *>(static_cast<float *>(out) + ob + i) =
+                make_float2(o[i] * inv, o[i + 1] * inv);
+        else
+            *reinterpret_cast<__half2 *>(static_cast<__half *>(out) + ob + i) =
+                __floats2half2_rn(o[i] * inv, o[i + 1] * inv);
+    }
+}
+
+template <int DH>
+__device__ __forceinline__ void merge_segment(const float *ws, int64_t slot0, int np, int G,
+                                              void *out, int out_f32, int64_t obase0, int lane)
+{
+    if (G <= 4)
+        merge_segment_lpc<DH, 8>(ws, slot0, np, G, out, out_f32, obase0, lane);
+    else
+        merge_segment_lpc<DH, 4>(ws, slot0, np, G, out, out_f32, obase0, lane);
+}
+
+// KG / VG: keys / values carry one scale per 32/64-element group (else one per
+// (token, head)); compile-time so the per-head case keeps no per-group state.
+template <int DH, int KB, int VB, bool KG, bool VG>
+__global__ void __launch_bounds__(NTHR, 2)
+    decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  const __grid_constant__ DecodeParams p)
+{
+    constexpr int NG = DH / 32;                // 32-element blocks along head_dim
+    constexpr int RK = DH * KB / 8;            // bytes per key row
+    constexpr int RV = DH * VB / 8;
+    constexpr int SK = 32 * KB / 8;            // bytes per 32-element block of a key row
+    constexpr int SV = 32 * VB / 8;
+    constexpr int NVG = VG ? NG : 1;           // value-scale groups tracked per token
+    constexpr float BIAS_V = VB == 8 ? 1152.f : (VB == 4 ? 1032.f : 0.f);
+    // The running max is only raised when a tile beats it by more than 2^LAZY;
+    // weights p * s_V then stay below 2^LAZY, well inside fp16.
+    constexpr float LAZY = 8.f;
+
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // align to 1024 B (128-byte swizzle atoms) by pointer arithmetic on the shared
+    // array itself, so every access below stays a shared-memory access
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(smem);             // 32-bit shared address of the ring
+    StageMeta *meta = reinterpret_cast<StageMeta *>(smem + p.off_meta);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + p.off_bar);
+    uint64_t *empty = full + p.stages;
+    uint64_t *segbar = empty + p.stages;                // [0] partials in mbuf, [1] mbuf read
+    int *ctl = reinterpret_cast<int *>(segbar + 2);     // [0] abort, [1] units, [2..3] prefix
+    float *mbuf = reinterpret_cast<float *>(smem + p.off_merge);   // [NW][G][DH + 4]
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int S = p.stages;
+    const int G = p.group_size_g;
+    const int cap = p.cap;
+    const int Hkv = p.n_kv_heads;
+    volatile int *abort_flag = ctl;
+
+    if (tid == 0) {
+        for (int s = 0; s < S; s++) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], NW);
+        }
+        mbar_init(&segbar[0], NW);
+        mbar_init(&segbar[1], NW);
+        ctl[0] = 0;
+        fence_mbar_init();
+    }
+
+    // ---- work range of this CTA (computed by the producer warp) -------------
+    __shared__ long long sh_u_begin, sh_n, sh_pe;
+    __shared__ int sh_b;
+    if (warp == NW) {
+        long long total = 0;
+        for (int b = lane; b < p.batch; b += 32) total += tiles_of(p.d_len[b], cap);
+        for (int off = 16; off; off >>= 1) total += __shfl_xor_sync(FULL, total, off);
+        const long long N = total * Hkv;
+        const long long Pe = N < (long long)p.num_ctas ? N : (long long)p.num_ctas;
+        long long ub = 0, ue = 0;
+        if ((long long)blockIdx.x < Pe) {
+            ub = (long long)blockIdx.x * N / Pe;
+            ue = ((long long)blockIdx.x + 1) * N / Pe;
+        }
+        // locate the sequence holding unit ub
+        long long acc = 0;
+        int fb = -1;
+        long long fpre = 0;
+        for (int base = 0; base < p.batch && fb < 0 && ue > ub; base += 32) {
+            const int b = base + lane;
+            const long long units = (b < p.batch) ? (long long)tiles_of(p.d_len[b], cap) * Hkv : 0;
+            long long incl = units;
+            for (int off = 1; off < 32; off <<= 1) {
+                const long long v = __shfl_up_sync(FULL, incl, off);
+                if (lane >= off) incl += v;
+            }
+            const long long excl = acc + incl - units;
+            const bool hit = units > 0 && excl <= ub && ub < excl + units;
+            const unsigned m = __ballot_sync(FULL, hit);
+            if (m) {
+                const int src = __ffs(m) - 1;
+                fb = __shfl_sync(FULL, b, src);
+                fpre = __shfl_sync(FULL, excl, src);
+            }
+            acc += __shfl_sync(FULL, incl, 31);
+        }
+        if (lane == 0) {
+            sh_u_begin = ub;
+            sh_n = N;
+            sh_pe = Pe;
+            sh_b = fb;
+            ctl[1] = (int)(ue > ub && fb >= 0 ? ue - ub : 0);
+            reinterpret_cast<long long *>(ctl + 2)[0] = fpre;
+        }
+    }
+    __syncthreads();
+    const int n_units = ctl[1];
+
+    if (warp == NW) {
+        // ====================== producer (whole warp) ======================
+        if (lane == 0) {
+            prefetch_tensormap(&tm_k);
+            prefetch_tensormap(&tm_v);
+        }
+        // codes and scales are read once: let them leave L2 first, so that the
+        // partials and the queries stay cached
+        const uint64_t pol = l2_evict_first_policy();
+        const long long N = sh_n, Pe = sh_pe;
+        int b = sh_b;
+        long long pre = reinterpret_cast<long long *>(ctl + 2)[0];   // units before sequence b
+        int len_b = (b >= 0) ? clamp_len(p.d_len[b], cap) : 0;
+        int tiles_b = (len_b + T - 1) / T;
+        const int off = (int)(sh_u_begin - pre);   // unit offset inside sequence b
+        int kvh = tiles_b ? off / tiles_b : 0;
+        int tile = tiles_b ? off % tiles_b : 0;
+        int s = 0;
+        uint32_t ph = 0;                            // phase parity of this use of stage s
+        int issued = 0;
+        int seg_ncta = 0, seg_cmin = 0;
+        for (int i = 0; i < n_units; i++) {
+            const int bh = b * Hkv + kvh;
+            const int t0 = tile * T;
+            if (i == 0 || tile == 0) {
+                // CTAs whose unit ranges meet this (sequence, KV head)
+                const long long u0 = pre + (long long)kvh * tiles_b, u1 = u0 + tiles_b;
+                const long long cmin = ((u0 + 1) * Pe + N - 1) / N - 1;
+                const long long cmax = (u1 * Pe + N - 1) / N - 1;
+                seg_cmin = (int)cmin;
+                seg_ncta = (int)(cmax - cmin + 1);
+            }
+            if (p.app.k_new != nullptr && tile == tiles_b - 1) {
+                // fused append: the newest token (position len - 1) lies in this
+                // tile; quantise it into the cache before the tile is loaded
+                const int64_t crow = (int64_t)bh * cap + (len_b - 1);
+                quantize_row(p.app.k_new, (int64_t)bh * DH, p.app.dtype, DH, KB, p.app.k_group,
+                             p.app.k_codes + crow * RK,
+                             KB == 16 ? nullptr : p.app.k_scales + crow * (DH / p.app.k_group), lane);
+                quantize_row(p.app.v_new, (int64_t)bh * DH, p.app.dtype, DH, VB, p.app.v_group,
+                             p.app.v_codes + crow * RV,
+                             VB == 16 ? nullptr : p.app.v_scales + crow * (DH / p.app.v_group), lane);
+                fence_proxy_async_global();
+                __syncwarp();
+            }
+            int ok = 1;
+            if (lane == 0 && i >= S) ok = mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, p.timeout_ns);
+            ok = __shfl_sync(FULL, ok, 0);
+            if (!ok) {
+                if (lane == 0) {
+                    ctl[0] = 1;
+                    atomicExch(p.status, KVQ_ERR_TIMEOUT);
+                }
+                break;
+            }
+            if (lane == 0) {
+                int flags = 0;
+                if (i == 0 || tile == 0) flags |= 1;
+                if (i == n_units - 1 || tile == tiles_b - 1) flags |= 2;
+                StageMeta m;
+                m.bh = bh; m.t0 = t0; m.len = len_b; m.flags = flags;
+                m.slot = (int)blockIdx.x + bh;
+                m.ncta = seg_ncta; m.cmin = seg_cmin; m.pad = 0;
+                meta[s] = m;
+
+                uint8_t *st = smem + (size_t)s * p.stage_bytes;
+                const int n_s = min(T, cap - t0);
+                uint32_t bytes = (uint32_t)(T * RK + T * RV);
+                if (KB != 16) bytes += (uint32_t)(n_s * p.ngs_k * 2);
+                if (VB != 16) bytes += (uint32_t)(n_s * p.ngs_v * 2);
+                mbar_arrive_expect_tx(&full[s], bytes);
+                if constexpr (RK <= 128) {
+                    tma_load_3d_hint(st, &tm_k, &full[s], 0, t0 / (128 / RK), bh, pol);
+                } else {
+                    tma_load_3d_hint(st, &tm_k, &full[s], 0, t0, bh, pol);
+                    tma_load_3d_hint(st + T * 128, &tm_k, &full[s], 128, t0, bh, pol);
+                }
+                if constexpr (RV <= 128) {
+                    tma_load_3d_hint(st + p.off_v, &tm_v, &full[s], 0, t0 / (128 / RV), bh, pol);
+                } else {
+                    tma_load_3d_hint(st + p.off_v, &tm_v, &full[s], 0, t0, bh, pol);
+                    tma_load_3d_hint(st + p.off_v + T * 128, &tm_v, &full[s], 128, t0, bh, pol);
+                }
+                if (KB != 16)
+                    bulk_load_hint(st + p.off_sk, p.k_scales + ((int64_t)bh * cap + t0) * p.ngs_k,
+                                   (uint32_t)(n_s * p.ngs_k * 2), &full[s], pol);
+                if (VB != 16)
+                    bulk_load_hint(st + p.off_sv, p.v_scales + ((int64_t)bh * cap + t0) * p.ngs_v,
+                                   (uint32_t)(n_s * p.ngs_v * 2), &full[s], pol);
+            }
+            issued = i + 1;
+            if (++s == S) {
+                s = 0;
+                ph ^= 1u;
+            }
+            // advance to the next unit (the length is re-read only when b changes)
+            if (++tile == tiles_b) {
+                tile = 0;
+                if (++kvh == Hkv) {
+                    kvh = 0;
+                    do {
+                        pre += (long long)tiles_b * Hkv;
+                        ++b;
+                        len_b = (b < p.batch) ? clamp_len(p.d_len[b], cap) : T;
+                        tiles_b = (len_b + T - 1) / T;
+                    } while (tiles_b == 0);
+                }
+            }
+        }
+        // never leave with copies in flight: wait for the last issued phases
+        if (lane == 0) {
+            int ss = s;
+            uint32_t pp = ph;
+            for (int j = 0; j < min(S, issued); j++) {
+                if (ss == 0) {
+                    ss = S;
+                    pp ^= 1u;
+                }
+                --ss;
+                (void)mbar_wait_bounded(&full[ss], pp, abort_flag, p.timeout_ns);
+            }
+        }
+        return;
+    }
+
+    // ====================== consumers ======================
+    constexpr bool IMMA_K = KB != 16;
+    const int gid = lane >> 2;
+    const int tig = lane & 3;
+    // fp16 keys keep an f16 MMA; f32 / bf16 queries then use columns 4..7 for
+    // the fp16 residual of the query (G <= 4)
+    const bool qsplit = !IMMA_K && p.q_dtype != KVQ_F16;
+    constexpr bool kgrp = KG;
+    constexpr bool vgrp = VG;
+    const int colmax = qsplit ? 4 : 8;
+    const bool col_ok0 = (2 * tig) < G && (2 * tig) < colmax;
+    const bool col_ok1 = (2 * tig + 1) < G && (2 * tig + 1) < colmax;
+
+    // sequences with nothing cached get zeros (fused merge only; the merge
+    // launch writes them otherwise)
+    if (p.counters != nullptr) {
+        const int64_t n_out = (int64_t)p.n_q_heads * DH;
+        for (int b = blockIdx.x; b < p.batch; b += gridDim.x) {
+            if (tiles_of(p.d_len[b], cap) != 0) continue;
+            for (int64_t i = tid; i < n_out; i += 32 * NW) {
+                if (p.out_f32)
+                    static_cast<float *>(p.out)[(int64_t)b * n_out + i] = 0.f;
+                else
+                    static_cast<__half *>(p.out)[(int64_t)b * n_out + i] = __float2half_rn(0.f);
+            }
+        }
+    }
+
+    // Rows of the score tile: row gid is token tw + rt, row gid + 8 token tw + rt + 1.
+    // The P.V MMA takes k-slots 2tig, 2tig+1, 2tig+8, 2tig+9 = tokens
+    // tw + vA, tw + vB, tw + vA + 1, tw + vB + 1 (the transpose of the score rows).
+    const int rt = row_token(gid);
+    const int vA = row_token(2 * tig), vB = row_token(2 * tig + 1);
+    uint32_t kofs[2][2], vofs[2][4];
+#pragma unroll
+    for (int u = 0; u < 2; u++) {
+        const int tw = warp * 32 + u * 16;
+        kofs[u][0] = sw_off<RK>(tw + rt, tig * (SK / 4));
+        kofs[u][1] = sw_off<RK>(tw + rt + 1, tig * (SK / 4));
+        vofs[u][0] = p.off_v + sw_off<RV>(tw + vA, gid * (SV / 8));
+        vofs[u][1] = p.off_v + sw_off<RV>(tw + vB, gid * (SV / 8));
+        vofs[u][2] = p.off_v + sw_off<RV>(tw + vA + 1, gid * (SV / 8));
+        vofs[u][3] = p.off_v + sw_off<RV>(tw + vB + 1, gid * (SV / 8));
+    }
+    // Sub-tile 1 lies 16 tokens after sub-tile 0.  For rows of >= 64 bytes the
+    // swizzle phase repeats every 16 tokens, so its addresses are those of
+    // sub-tile 0 plus KU / VU, which the loads carry as immediate offsets;
+    // shorter rows (Dh 64 at 4 bits) keep their own offsets.
+    constexpr bool KREP = RK >= 64, VREP = RV >= 64;
+    constexpr int KU = RK <= 128 ? 16 * RK : 16 * 128;
+    constexpr int VU = RV <= 128 ? 16 * RV : 16 * 128;
+
+    uint32_t qh[NG][2], ql[NG][2];      // int8 query B-fragments (hi / lo parts) per block
+    float sqc[2];                       // score factor of columns 2tig, 2tig+1
+    uint32_t qb[NG][2][2];              // fp16 query B-fragments (fp16 keys)
+    float m_run[2], l_run[2];
+    float psum[NVG][4];                 // sum of fp16 p*s_V per value group (cols in [0], [1])
+    float o_acc[2 * NG][4];             // O^T fragments, m-tile = 2*blk + h
+
+    auto load_q = [&](int bh) {
+        const int b = bh / Hkv;
+        const int kvh = bh % Hkv;
+        if constexpr (IMMA_K) {
+            // q ~ (amax / 127) * (hi + lo / 254) per head, hi, lo in [-127, 127];
+            // lane (gid, tig) holds head gid, elements 32 blk + 8 tig + 0..7
+            const bool valid = gid < G;
+            const int64_t qbase = ((int64_t)b * p.n_q_heads + (int64_t)kvh * G + gid) * DH;
+            float x[NG][8];
+            float amax = 0.f;
+#pragma unroll
+            for (int blk = 0; blk < NG; blk++)
+#pragma unroll
+                for (int j = 0; j < 8; j++) {
+                    x[blk][j] = valid ? load_qf(p.q, p.q_dtype, qbase + 32 * blk + 8 * tig + j) : 0.f;
+                    amax = fmaxf(amax, fabsf(x[blk][j]));
+                }
+            amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 2));
+            const float inv = amax > 0.f ? 127.f / amax : 0.f;
+#pragma unroll
+            for (int blk = 0; blk < NG; blk++) {
+                int hi[8], lo[8];
+#pragma unroll
+                for (int j = 0; j < 8; j++) {
+                    const float y = x[blk][j] * inv;
+                    const float r = rintf(y);
+                    hi[j] = (int)r;
+                    lo[j] = __float2int_rn((y - r) * 254.f);
+                }
+                if constexpr (KB == 8) {
+                    // k-slot 4tig+i <-> element 8tig+i, 16+4tig+i <-> 8tig+4+i
+                    qh[blk][0] = pack_bytes(hi[0], hi[1], hi[2], hi[3]);
+                    qh[blk][1] = pack_bytes(hi[4], hi[5], hi[6], hi[7]);
+                    ql[blk][0] = pack_bytes(lo[0], lo[1], lo[2], lo[3]);
+                    ql[blk][1] = pack_bytes(lo[4], lo[5], lo[6], lo[7]);
+                } else {
+                    // k-slot 4tig+i <-> element 8tig+2i (low nibbles), 16+4tig+i <-> 8tig+2i+1
+                    qh[blk][0] = pack_bytes(hi[0], hi[2], hi[4], hi[6]);
+                    qh[blk][1] = pack_bytes(hi[1], hi[3], hi[5], hi[7]);
+                    ql[blk][0] = pack_bytes(lo[0], lo[2], lo[4], lo[6]);
+                    ql[blk][1] = pack_bytes(lo[1], lo[3], lo[5], lo[7]);
+                }
+            }
+            // 4-bit key codes enter the MMA as 16 * code
+            const float f = amax * (1.f / (127.f * 254.f)) * p.tau_log2e * (KB == 4 ? 0.0625f : 1.f);
+            sqc[0] = __shfl_sync(FULL, f, (2 * tig) * 4);
+            sqc[1] = __shfl_sync(FULL, f, (2 * tig + 1) * 4);
+        } else {
+            // B-fragment column n = gid: non-split: head n; split: hi (n<4) / lo (n>=4) of head n&3
+            const int head = qsplit ? (gid & 3) : gid;
+            const bool lo_part = qsplit && gid >= 4;
+            const bool valid = head < G;
+            const int64_t qbase = ((int64_t)b * p.n_q_heads + (int64_t)kvh * G + head) * DH;
+#pragma unroll
+            for (int blk = 0; blk < NG; blk++)
+#pragma unroll
+                for (int hs = 0; hs < 2; hs++) {
+                    __half hv[4];
+#pragma unroll
+                    for (int j = 0; j < 4; j++) {
+                        // k-slots 2tig, 2tig+1, 2tig+8, 2tig+9 <-> elements 8tig + 4hs + j
+                        const int d = 32 * blk + 8 * tig + 4 * hs + j;
+                        const float xq = valid ? load_qf(p.q, p.q_dtype, qbase + d) : 0.f;
+                        __half h = __float2half_rn(xq);
+                        if (lo_part) h = __float2half_rn(xq - __half2float(h));
+                        hv[j] = h;
+                    }
+                    __half2 b0 = __halves2half2(hv[0], hv[1]);
+                    __half2 b1 = __halves2half2(hv[2], hv[3]);
+                    qb[blk][hs][0] = *reinterpret_cast<uint32_t *>(&b0);
+                    qb[blk][hs][1] = *reinterpret_cast<uint32_t *>(&b1);
+                }
+        }
+#pragma unroll
+        for (int c = 0; c < 2; c++) {
+            m_run[c] = -INFINITY;
+            l_run[c] = 0.f;
+        }
+#pragma unroll
+        for (int g = 0; g < NVG; g++) psum[g][0] = psum[g][1] = psum[g][2] = psum[g][3] = 0.f;
+#pragma unroll
+        for (int mt = 0; mt < 2 * NG; mt++)
+#pragma unroll
+            for (int i = 0; i < 4; i++) o_acc[mt][i] = 0.f;
+    };
+
+    // int8 A fragments of one 32-element key block for the rows at shared
+    // addresses ra (row gid) and rb (row gid + 8), plus IMM bytes
+    auto key_frags = [&](auto imm, uint32_t ra, uint32_t rb, uint32_t (&fa)[4]) {
+        constexpr int IMM = decltype(imm)::value;
+        if constexpr (KB == 8) {
+            const uint2 r0 = ldsi_u64<IMM>(ra);
+            const uint2 r1 = ldsi_u64<IMM>(rb);
+            fa[0] = r0.x; fa[1] = r1.x; fa[2] = r0.y; fa[3] = r1.y;
+        } else {
+            const uint32_t r0 = ldsi_u32<IMM>(ra);
+            const uint32_t r1 = ldsi_u32<IMM>(rb);
+            fa[0] = (r0 << 4) & 0xF0F0F0F0u; fa[1] = (r1 << 4) & 0xF0F0F0F0u;
+            fa[2] = r0 & 0xF0F0F0F0u;        fa[3] = r1 & 0xF0F0F0F0u;
+        }
+    };
+    // key-row addresses of block blk for sub-tile u: {address, immediate}
+    using Imm0 = std::integral_constant<int, 0>;
+    using ImmK = std::integral_constant<int, KREP ? KU : 0>;
+    using ImmV = std::integral_constant<int, VREP ? VU : 0>;
+
+    const uint64_t limit = p.timeout_ns;
+    const uint32_t ONE2 = 0x3C003C00u;   // half2(1, 1)
+    int s = 0;
+    uint32_t ph = 0;
+    uint32_t seg_parity = 0;
+    for (int i = 0; i < n_units; i++) {
+        if (!mbar_wait_bounded(&full[s], ph, abort_flag, limit)) {
+            ctl[0] = 1;
+            atomicExch(p.status, KVQ_ERR_TIMEOUT);
+            break;
+        }
+        StageMeta m;
+        {
+            const uint4 m0 = *reinterpret_cast<const uint4 *>(&meta[s]);
+            const uint4 m1 = *(reinterpret_cast<const uint4 *>(&meta[s]) + 1);
+            m.bh = (int)m0.x; m.t0 = (int)m0.y; m.len = (int)m0.z; m.flags = (int)m0.w;
+            m.slot = (int)m1.x; m.ncta = (int)m1.y; m.cmin = (int)m1.z;
+        }
+        if (m.flags & 1) load_q(m.bh);
+        const uint32_t st = (uint32_t)s * p.stage_bytes;   // stage offset from smem
+        const uint32_t sst = sbase + st;                    // shared address of the stage
+        const uint32_t ssk = st + p.off_sk;   // fp16 key scales of the stage
+        const uint32_t ssv = st + p.off_sv;   // fp16 value scales
+
+        // Work of this warp on the stage: two 16-token sub-tiles u = 0, 1, processed
+        // phase by phase so that the two sub-tiles give the scheduler independent
+        // instruction streams at every step.
+        int tAu[2];
+        bool vt[2][2];
+#pragma unroll
+        for (int u = 0; u < 2; u++) {
+            tAu[u] = warp * 32 + u * 16 + rt;               // score rows: tAu, tAu + 1
+            vt[u][0] = m.t0 + tAu[u] < m.len;
+            vt[u][1] = m.t0 + tAu[u] + 1 < m.len;
+        }
+
+        // ---------------- phase 1: scores S^T = K q^T for both sub-tiles ----------
+        float s2[2][4];
+        if constexpr (IMMA_K) {
+            if constexpr (!kgrp) {
+                // hi and lo chains are independent; combined once per tile
+                int ah[2][4], al[2][4];
+#pragma unroll
+                for (int u = 0; u < 2; u++)
+#pragma unroll
+                    for (int e = 0; e < 4; e++) ah[u][e] = al[u][e] = 0;
+#pragma unroll
+                for (int blk = 0; blk < NG; blk++) {
+                    const uint32_t ra = sst + blk_addr<RK, SK>(kofs[0][0], blk);
+                    const uint32_t rb = sst + blk_addr<RK, SK>(kofs[0][1], blk);
+                    uint32_t fa[2][4];
+                    key_frags(Imm0{}, ra, rb, fa[0]);
+                    if constexpr (KREP)
+                        key_frags(ImmK{}, ra, rb, fa[1]);
+                    else
+                        key_frags(Imm0{}, sst + blk_addr<RK, SK>(kofs[1][0], blk),
+                                  sst + blk_addr<RK, SK>(kofs[1][1], blk), fa[1]);
+#pragma unroll
+                    for (int u = 0; u < 2; u++) {
+                        imma_16832(ah[u], fa[u][0], fa[u][1], fa[u][2], fa[u][3], qh[blk][0], qh[blk][1]);
+                        imma_16832(al[u], fa[u][0], fa[u][1], fa[u][2], fa[u][3], ql[blk][0], ql[blk][1]);
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 2; u++) {
+                    const float2 kk = unpack_half2(lds_u32(sbase, ssk + 2 * tAu[u]));
+#pragma unroll
+                    for (int e = 0; e < 4; e++) {
+                        const float ks = (e < 2) ? kk.x : kk.y;
+                        s2[u][e] = (float)(ah[u][e] * 254 + al[u][e]) * (ks * sqc[e & 1]);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int u = 0; u < 2; u++) {
+                    float v[4] = {0.f, 0.f, 0.f, 0.f};
+                    const int tA = tAu[u];
+#pragma unroll
+                    for (int blk = 0; blk < NG; blk++) {
+                        int ah[4] = {0, 0, 0, 0}, al[4] = {0, 0, 0, 0};
+                        uint32_t fa[4];
+                        key_frags(Imm0{}, sst + blk_addr<RK, SK>(kofs[u][0], blk),
+                                  sst + blk_addr<RK, SK>(kofs[u][1], blk), fa);
+                        imma_16832(ah, fa[0], fa[1], fa[2], fa[3], qh[blk][0], qh[blk][1]);
+                        imma_16832(al, fa[0], fa[1], fa[2], fa[3], ql[blk][0], ql[blk][1]);
+                        const float k0 = __half2float(__ushort_as_half(
+                            (unsigned short)lds_u16(sbase, ssk + 2 * (tA * p.ngs_k + (blk >> p.kshift)))));
+                        const float k1 = __half2float(__ushort_as_half(
+                            (unsigned short)lds_u16(sbase, ssk + 2 * ((tA + 1) * p.ngs_k + (blk >> p.kshift)))));
+                        v[0] = fmaf(k0, (float)(ah[0] * 254 + al[0]), v[0]);
+                        v[1] = fmaf(k0, (float)(ah[1] * 254 + al[1]), v[1]);
+                        v[2] = fmaf(k1, (float)(ah[2] * 254 + al[2]), v[2]);
+                        v[3] = fmaf(k1, (float)(ah[3] * 254 + al[3]), v[3]);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 4; e++) s2[u][e] = v[e] * sqc[e & 1];
+                }
+            }
+        } else {
+            // fp16 keys: two partial accumulators per sub-tile halve the MMA chain
+            float acc[2][2][4];
+#pragma unroll
+            for (int u = 0; u < 2; u++)
+#pragma unroll
+                for (int h = 0; h < 2; h++) acc[u][h][0] = acc[u][h][1] = acc[u][h][2] = acc[u][h][3] = 0.f;
+#pragma unroll
+            for (int blk = 0; blk < NG; blk++) {
+                const uint32_t ra = sst + blk_addr<RK, SK>(kofs[0][0], blk);
+                const uint32_t rb = sst + blk_addr<RK, SK>(kofs[0][1], blk);
+                uint4 r[2][2];
+                r[0][0] = ldsi_u128<0>(ra);
+                r[0][1] = ldsi_u128<0>(rb);
+                r[1][0] = ldsi_u128<ImmK::value>(KREP ? ra : sst + blk_addr<RK, SK>(kofs[1][0], blk));
+                r[1][1] = ldsi_u128<ImmK::value>(KREP ? rb : sst + blk_addr<RK, SK>(kofs[1][1], blk));
+#pragma unroll
+                for (int u = 0; u < 2; u++) {
+                    const uint4 r0 = r[u][0], r1 = r[u][1];
+                    mma_16816(acc[u][blk & 1], r0.x, r1.x, r0.y, r1.y, qb[blk][0][0], qb[blk][0][1]);
+                    mma_16816(acc[u][blk & 1], r0.z, r1.z, r0.w, r1.w, qb[blk][1][0], qb[blk][1][1]);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 2; u++)
+#pragma unroll
+                for (int e = 0; e < 4; e++) {
+                    float v = (acc[u][0][e] + acc[u][1][e]) * p.tau_log2e;
+                    if (qsplit) v += __shfl_xor_sync(FULL, v, 2);
+                    s2[u][e] = v;
+                }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; u++) {
+            // Padding columns (heads >= G, or the residual columns of a split
+            // query) carry finite scores from zero query columns; their outputs
+            // are never written, so only tokens past the length are masked.
+            s2[u][0] = vt[u][0] ? s2[u][0] : -INFINITY;
+            s2[u][1] = vt[u][0] ? s2[u][1] : -INFINITY;
+            s2[u][2] = vt[u][1] ? s2[u][2] : -INFINITY;
+            s2[u][3] = vt[u][1] ? s2[u][3] : -INFINITY;
+        }
+
+        // ---------------- phase 2: value scales of the score rows -----------------
+        float sv[2][2][NVG];   // [sub-tile][row][value group]
+        float lsv[2][2];
+#pragma unroll
+        for (int u = 0; u < 2; u++) {
+            const int tA = tAu[u];
+            if constexpr (VB == 16) {
+                sv[u][0][0] = sv[u][1][0] = 1.f;
+            } else if constexpr (!vgrp) {
+                const float2 vv = unpack_half2(lds_u32(sbase, ssv + 2 * tA));
+                sv[u][0][0] = vv.x;
+                sv[u][1][0] = vv.y;
+            } else {
+#pragma unroll
+                for (int g = 0; g < NG; g++) {
+                    sv[u][0][g] = __half2float(__ushort_as_half(
+                        (unsigned short)lds_u16(sbase, ssv + 2 * (tA * p.ngs_v + (g >> p.vshift)))));
+                    sv[u][1][g] = __half2float(__ushort_as_half(
+                        (unsigned short)lds_u16(sbase, ssv + 2 * ((tA + 1) * p.ngs_v + (g >> p.vshift)))));
+                }
+            }
+            // scales past the length may be stale shared memory: never use them
+#pragma unroll
+            for (int r = 0; r < 2; r++) {
+                float mx = 0.f;
+#pragma unroll
+                for (int g = 0; g < NVG; g++) {
+                    sv[u][r][g] = vt[u][r] ? sv[u][r][g] : 0.f;
+                    mx = fmaxf(mx, sv[u][r][g]);
+                }
+                lsv[u][r] = mx > 0.f ? fmaxf(__log2f(mx), -32.f) : -32.f;
+            }
+        }
+
+        // ---------------- phase 3: online softmax, one lazy check for 32 tokens ---
+        {
+            float loc0 = -INFINITY, loc1 = -INFINITY;
+#pragma unroll
+            for (int u = 0; u < 2; u++) {
+                loc0 = fmaxf(loc0, fmaxf(s2[u][0] + lsv[u][0], s2[u][2] + lsv[u][1]));
+                loc1 = fmaxf(loc1, fmaxf(s2[u][1] + lsv[u][0], s2[u][3] + lsv[u][1]));
+            }
+            const bool need = (loc0 > m_run[0] + LAZY) || (loc1 > m_run[1] + LAZY);
+            if (__any_sync(FULL, need)) {
+#pragma unroll
+                for (int off = 4; off < 32; off <<= 1) {
+                    loc0 = fmaxf(loc0, __shfl_xor_sync(FULL, loc0, off));
+                    loc1 = fmaxf(loc1, __shfl_xor_sync(FULL, loc1, off));
+                }
+                const float mn0 = fmaxf(m_run[0], loc0), mn1 = fmaxf(m_run[1], loc1);
+                const float a0 = (mn0 == -INFINITY) ? 1.f : fast_exp2(m_run[0] - mn0);
+                const float a1 = (mn1 == -INFINITY) ? 1.f : fast_exp2(m_run[1] - mn1);
+                m_run[0] = mn0;
+                m_run[1] = mn1;
+                l_run[0] *= a0;
+                l_run[1] *= a1;
+#pragma unroll
+                for (int g = 0; g < NVG; g++) {
+                    psum[g][0] *= a0;
+                    psum[g][1] *= a1;
+                }
+#pragma unroll
+                for (int mt = 0; mt < 2 * NG; mt++) {
+                    o_acc[mt][0] *= a0;
+                    o_acc[mt][1] *= a1;
+                    o_acc[mt][2] *= a0;
+                    o_acc[mt][3] *= a1;
+                }
+            }
+        }
+
+        // ---------------- phase 4: P (fp16, value scale folded) -> B fragments ----
+        // x0 = rows 0..7 of the score tile (tokens tw + row_token(r)), x1 = rows
+        // 8..15; their 8x8 transposes are the B fragments of the P.V MMA.
+        uint32_t pb[2][NVG][2];
+#pragma unroll
+        for (int u = 0; u < 2; u++) {
+            float pr[4];
+#pragma unroll
+            for (int e = 0; e < 4; e++)
+                pr[e] = (s2[u][e] == -INFINITY) ? 0.f : fast_exp2(s2[u][e] - m_run[e & 1]);
+            l_run[0] += pr[0] + pr[2];
+            l_run[1] += pr[1] + pr[3];
+#pragma unroll
+            for (int g = 0; g < NVG; g++) {
+                const uint32_t x0 = pack_half2(pr[0] * sv[u][0][g], pr[1] * sv[u][0][g]);
+                const uint32_t x1 = pack_half2(pr[2] * sv[u][1][g], pr[3] * sv[u][1][g]);
+                pb[u][g][0] = movmatrix_trans(x0);
+                pb[u][g][1] = movmatrix_trans(x1);
+                // column sums of the fp16 weights, for the code bias
+                if constexpr (VB != 16)
+                    mma_16816(psum[g], ONE2, ONE2, ONE2, ONE2, pb[u][g][0], pb[u][g][1]);
+            }
+        }
+
+        // ---------------- phase 5: O^T += V^T P for both sub-tiles ----------------
+#pragma unroll
+        for (int blk = 0; blk < NG; blk++) {
+            // value-row addresses of this block (sub-tile 0; sub-tile 1 adds VU)
+            uint32_t va[2][4];
+#pragma unroll
+            for (int r = 0; r < 4; r++) {
+                va[0][r] = sst + blk_addr<RV, SV>(vofs[0][r], blk);
+                va[1][r] = VREP ? va[0][r] : sst + blk_addr<RV, SV>(vofs[1][r], blk);
+            }
+#pragma unroll
+            for (int u = 0; u < 2; u++) {
+                const uint32_t b0 = pb[u][VG ? blk : 0][0], b1 = pb[u][VG ? blk : 0][1];
+                if constexpr (VB == 8) {
+                    uint32_t wA, wB, wC, wE;
+                    if (u == 0) {
+                        wA = ldsi_u32<0>(va[0][0]); wB = ldsi_u32<0>(va[0][1]);
+                        wC = ldsi_u32<0>(va[0][2]); wE = ldsi_u32<0>(va[0][3]);
+                    } else {
+                        wA = ldsi_u32<ImmV::value>(va[1][0]); wB = ldsi_u32<ImmV::value>(va[1][1]);
+                        wC = ldsi_u32<ImmV::value>(va[1][2]); wE = ldsi_u32<ImmV::value>(va[1][3]);
+                    }
+#pragma unroll
+                    for (int h = 0; h < 2; h++) {
+                        const uint32_t sel = h ? 0x7632u : 0x5410u;
+                        const uint32_t yAB = prmt(wA, wB, sel), yCE = prmt(wC, wE, sel);
+                        const uint32_t a0 = and_xor(yAB, 0x00FF00FFu, 0x64806480u);
+                        const uint32_t a1 = and_xor(yAB >> 8, 0x00FF00FFu, 0x64806480u);
+                        const uint32_t a2 = and_xor(yCE, 0x00FF00FFu, 0x64806480u);
+                        const uint32_t a3 = and_xor(yCE >> 8, 0x00FF00FFu, 0x64806480u);
+                        mma_16816(o_acc[2 * blk + h], a0, a1, a2, a3, b0, b1);
+                    }
+                } else if constexpr (VB == 4) {
+                    uint32_t hA, hB, hC, hE;
+                    if (u == 0) {
+                        hA = ldsi_u16<0>(va[0][0]); hB = ldsi_u16<0>(va[0][1]);
+                        hC = ldsi_u16<0>(va[0][2]); hE = ldsi_u16<0>(va[0][3]);
+                    } else {
+                        hA = ldsi_u16<ImmV::value>(va[1][0]); hB = ldsi_u16<ImmV::value>(va[1][1]);
+                        hC = ldsi_u16<ImmV::value>(va[1][2]); hE = ldsi_u16<ImmV::value>(va[1][3]);
+                    }
+                    const uint32_t yAB = prmt(hA, hB, 0x5410u), yCE = prmt(hC, hE, 0x5410u);
+#pragma unroll
+                    for (int h = 0; h < 2; h++) {
+                        const uint32_t a0 = i4_pair(yAB, 2 * h);
+                        const uint32_t a1 = i4_pair(yAB, 2 * h + 1);
+                        const uint32_t a2 = i4_pair(yCE, 2 * h);
+                        const uint32_t a3 = i4_pair(yCE, 2 * h + 1);
+                        mma_16816(o_acc[2 * blk + h], a0, a1, a2, a3, b0, b1);
+                    }
+                } else {
+                    // fp16 values past the length may be anything (NaN included): zero them
+                    const int tg = m.t0 + warp * 32 + u * 16;
+                    const uint2 z = make_uint2(0u, 0u);
+                    uint2 w[4];
+#pragma unroll
+                    for (int r = 0; r < 4; r++) {
+                        const int tok = tg + ((r & 1) ? vB : vA) + (r >> 1);
+                        w[r] = z;
+                        if (tok < m.len) w[r] = u == 0 ? ldsi_u64<0>(va[0][r]) : ldsi_u64<ImmV::value>(va[1][r]);
+                    }
+#pragma unroll
+                    for (int h = 0; h < 2; h++) {
+                        const uint32_t A = h ? w[0].y : w[0].x, Bw = h ? w[1].y : w[1].x;
+                        const uint32_t C = h ? w[2].y : w[2].x, E = h ? w[3].y : w[3].x;
+                        const uint32_t a0 = prmt(A, Bw, 0x5410u), a1 = prmt(A, Bw, 0x7632u);
+                        const uint32_t a2 = prmt(C, E, 0x5410u), a3 = prmt(C, E, 0x7632u);
+                        mma_16816(o_acc[2 * blk + h], a0, a1, a2, a3, b0, b1);
+                    }
+                }
+            }
+        }
+
+        // release the stage to the producer
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        if (++s == S) {
+            s = 0;
+            ph ^= 1u;
+        }
+
+        // ---------------- segment end: combine the warps, write the partial ------
+        if (m.flags & 2) {
+            constexpr int CS = slot_col_floats(DH);
+            float lt[2];
+#pragma unroll
+            for (int c = 0; c < 2; c++) {
+                float v = l_run[c];
+                v += __shfl_xor_sync(FULL, v, 4);
+                v += __shfl_xor_sync(FULL, v, 8);
+                v += __shfl_xor_sync(FULL, v, 16);
+                lt[c] = v;
+            }
+            // this warp's partial into mbuf[warp]: [G][DH + 4] floats, o then (m, l)
+            float *mine = mbuf + (size_t)warp * G * CS;
+#pragma unroll
+            for (int c = 0; c < 2; c++) {
+                const int col = 2 * tig + c;
+                if (c == 0 ? col_ok0 : col_ok1) {
+                    float *oc = mine + (size_t)col * CS;
+#pragma unroll
+                    for (int blk = 0; blk < NG; blk++) {
+                        const float corr = BIAS_V * psum[VG ? blk : 0][c];
+#pragma unroll
+                        for (int h = 0; h < 2; h++) {
+                            // m-tile 2blk+h: row gid <-> d = 32blk + 4gid + 2h, row gid+8 <-> d + 1
+                            const int d = 32 * blk + 4 * gid + 2 * h;
+                            *reinterpret_cast<float2 *>(oc + d) =
+                                make_float2(o_acc[2 * blk + h][c] - corr, o_acc[2 * blk + h][2 + c] - corr);
+                        }
+                    }
+                    if (gid == 0) *reinterpret_cast<float2 *>(oc + DH) = make_float2(m_run[c], lt[c]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&segbar[0]);
+            if (!mbar_wait_bounded(&segbar[0], seg_parity, abort_flag, limit)) {
+                ctl[0] = 1;
+                atomicExch(p.status, KVQ_ERR_TIMEOUT);
+                break;
+            }
+            // combine the NW warps (each takes a quarter of the float4 chunks) and
+            // write this CTA's partial of the segment
+            const int ncol = qsplit ? min(G, 4) : G;
+            float *dst = p.ws + (size_t)m.slot * G * CS;
+            for (int k = warp * 32 + lane; k < ncol * (DH / 4); k += 32 * NW) {
+                const int col = k / (DH / 4), d = 4 * (k % (DH / 4));
+                float M = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < NW; w++) M = fmaxf(M, mbuf[((size_t)w * G + col) * CS + DH]);
+                float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+                float L = 0.f;
+#pragma unroll
+                for (int w = 0; w < NW; w++) {
+                    const float *src = mbuf + ((size_t)w * G + col) * CS;
+                    const float mw = src[DH];
+                    const float e = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+                    const float4 x = *reinterpret_cast<const float4 *>(src + d);
+                    O.x = fmaf(e, x.x, O.x);
+                    O.y = fmaf(e, x.y, O.y);
+                    O.z = fmaf(e, x.z, O.z);
+                    O.w = fmaf(e, x.w, O.w);
+                    L = fmaf(e, src[DH + 1], L);
+                }
+                *reinterpret_cast<float4 *>(dst + (size_t)col * CS + d) = O;
+                if (d == 0) *reinterpret_cast<float2 *>(dst + (size_t)col * CS + DH) = make_float2(M, L);
+            }
+            // mbuf is free again once every warp has read it
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&segbar[1]);
+            if (!mbar_wait_bounded(&segbar[1], seg_parity, abort_flag, limit)) {
+                ctl[0] = 1;
+                atomicExch(p.status, KVQ_ERR_TIMEOUT);
+                break;
+            }
+            seg_parity ^= 1u;
+            if (p.counters != nullptr) {
+                // the warp that completes the last partial of this (sequence, KV
+                // head) merges them (publish: fence, then count the arrival)
+                __threadfence();
+                __syncwarp();
+                int last = 0;
+                if (lane == 0) last = atomicAdd(&p.counters[m.bh], 1) == NW * m.ncta - 1;
+                last = __shfl_sync(FULL, last, 0);
+                if (last) {
+                    __threadfence();
+                    const int b = m.bh / Hkv, kvh = m.bh % Hkv;
+                    merge_segment<DH>(p.ws, (int64_t)m.cmin + m.bh, m.ncta, G, p.out, p.out_f32,
+                                      ((int64_t)b * p.n_q_heads + (int64_t)kvh * G) * DH, lane);
+                    if (lane == 0) p.counters[m.bh] = 0;   // ready for the next launch
+                }
+            }
+        }
+    }
+}
+
+}  // namespace
+}  // namespace kvq

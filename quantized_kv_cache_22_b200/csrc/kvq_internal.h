@@ -68,10 +68,18 @@ struct MergeParams {
 // Host helpers implemented in kvq_decode.cu.
 struct DecodeLaunch {
     int dh, kb, vb;
+    bool kg, vg;              // grouped key / value scales
     size_t smem_bytes;
     int stages;
     uint32_t stage_bytes, off_v, off_sk, off_sv, off_meta, off_bar, off_merge;
 };
+
+// Decode kernel instances (kvq_decode_k4/k8/k16.cu), by key width: the kernel
+// for (head_dim, value width, grouped key scales, grouped value scales), or
+// null if there is none.
+void *decode_fn_kb4(int dh, int vb, bool kg, bool vg);
+void *decode_fn_kb8(int dh, int vb, bool kg, bool vg);
+void *decode_fn_kb16(int dh, int vb, bool kg, bool vg);
 
 // Fill in the shared-memory plan; returns false if the shape is unsupported.
 bool plan_decode(int dh, int kb, int vb, int ngs_k, int ngs_v, int G, int max_smem,
