@@ -98,12 +98,6 @@ __host__ __device__ constexpr uint32_t sw_off(int t, int o)
 // order follows the score rows through the transpose) free of bank conflicts.
 __host__ __device__ constexpr int row_token(int g) { return 2 * (g ^ (g >> 2)); }
 
-// fp16 pair helpers: value code bytes / nibbles -> half2 of (bias + code).
-__device__ __forceinline__ uint32_t i4_pair(uint32_t w, int k)
-{
-    return and_xor(w >> (4 * k), 0x000F000Fu, 0x64086408u);
-}
-
 __device__ __forceinline__ float load_qf(const void *q, int dtype, int64_t idx)
 {
     if (dtype == KVQ_F16) return __half2float(static_cast<const __half *>(q)[idx]);
@@ -214,19 +208,6 @@ __device__ __forceinline__ uint32_t pack_bytes(int a, int b, int c, int d)
            ((uint32_t)(d & 0xff) << 24);
 }
 
-__device__ __forceinline__ float warp_max(float v)
-{
-#pragma unroll
-    for (int off = 16; off; off >>= 1) v = fmaxf(v, __shfl_xor_sync(FULL, v, off));
-    return v;
-}
-__device__ __forceinline__ float warp_sum(float v)
-{
-#pragma unroll
-    for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(FULL, v, off);
-    return v;
-}
-
 // Merge the np CTA partials of one (sequence, KV head), all G query heads at once:
 // slots slot0 .. slot0 + np - 1, each G records of DH + 4 floats holding per
 // query head o[DH], m, l.  out[obase0 + col * DH + d] receives
@@ -310,7 +291,7 @@ __global__ void __launch_bounds__(NTHR, 2)
     constexpr int SK = 32 * KB / 8;            // bytes per 32-element block of a key row
     constexpr int SV = 32 * VB / 8;
     constexpr int NVG = VG ? NG : 1;           // value-scale groups tracked per token
-    constexpr float BIAS_V = VB == 8 ? 1152.f : (VB == 4 ? 1032.f : 0.f);
+    constexpr float BIAS_V = VB == 8 ? 1152.f : 0.f;   // 4-bit values: per row, see the segment end
     // The running max is only raised when a tile beats it by more than 2^LAZY;
     // weights p * s_V then stay below 2^LAZY, well inside fp16.
     constexpr float LAZY = 8.f;
@@ -416,6 +397,61 @@ __global__ void __launch_bounds__(NTHR, 2)
         uint32_t ph = 0;                            // phase parity of this use of stage s
         int issued = 0;
         int seg_ncta = 0, seg_cmin = 0;
+
+        // Fused append.  The (sequence, KV head) pairs whose newest token lies in
+        // a tile of this CTA are visited in unit order by a second walker; the
+        // quantisation of the next one is done at the latest right before its
+        // tile is loaded, and earlier whenever the ring is full and the warp
+        // would only wait.  `app_rel` is the pending pair's tile index relative
+        // to this CTA's first unit (n_units when none is left).
+        const bool fuse_app = p.app.k_new != nullptr;
+        int ab = b, akvh = kvh, alen = len_b, atiles = tiles_b;
+        long long apre = pre;
+        int app_rel = n_units;
+        auto find_app = [&]() {
+            app_rel = n_units;
+            while (ab < p.batch) {
+                const long long ulast = apre + (long long)akvh * atiles + atiles - 1;
+                const long long rel = ulast - sh_u_begin;
+                if (rel >= n_units) return;            // beyond this CTA's range
+                if (atiles > 0 && rel >= 0) {
+                    app_rel = (int)rel;
+                    return;
+                }
+                // next (sequence, KV head)
+                if (++akvh == Hkv) {
+                    akvh = 0;
+                    apre += (long long)atiles * Hkv;
+                    ++ab;
+                    alen = (ab < p.batch) ? clamp_len(p.d_len[ab], cap) : 0;
+                    atiles = (alen + T - 1) / T;
+                }
+            }
+        };
+        auto do_app = [&]() {
+            const int bh = ab * Hkv + akvh;
+            const int64_t crow = (int64_t)bh * cap + (alen - 1);
+            quantize_row(p.app.k_new, (int64_t)bh * DH, p.app.dtype, DH, KB, p.app.k_group,
+                         p.app.k_codes + crow * RK,
+                         KB == 16 ? nullptr : p.app.k_scales + crow * (DH / p.app.k_group), lane);
+            quantize_row(p.app.v_new, (int64_t)bh * DH, p.app.dtype, DH, VB, p.app.v_group,
+                         p.app.v_codes + crow * RV,
+                         VB == 16 ? nullptr : p.app.v_scales + crow * (DH / p.app.v_group), lane);
+            // order the writes before the copy engine reads the tile
+            fence_proxy_async_global();
+            __syncwarp();
+            // move on to the next pair
+            if (++akvh == Hkv) {
+                akvh = 0;
+                apre += (long long)atiles * Hkv;
+                ++ab;
+                alen = (ab < p.batch) ? clamp_len(p.d_len[ab], cap) : 0;
+                atiles = (alen + T - 1) / T;
+            }
+            find_app();
+        };
+        if (fuse_app && n_units > 0) find_app();
+
         for (int i = 0; i < n_units; i++) {
             const int bh = b * Hkv + kvh;
             const int t0 = tile * T;
@@ -427,19 +463,9 @@ __global__ void __launch_bounds__(NTHR, 2)
                 seg_cmin = (int)cmin;
                 seg_ncta = (int)(cmax - cmin + 1);
             }
-            if (p.app.k_new != nullptr && tile == tiles_b - 1) {
-                // fused append: the newest token (position len - 1) lies in this
-                // tile; quantise it into the cache before the tile is loaded
-                const int64_t crow = (int64_t)bh * cap + (len_b - 1);
-                quantize_row(p.app.k_new, (int64_t)bh * DH, p.app.dtype, DH, KB, p.app.k_group,
-                             p.app.k_codes + crow * RK,
-                             KB == 16 ? nullptr : p.app.k_scales + crow * (DH / p.app.k_group), lane);
-                quantize_row(p.app.v_new, (int64_t)bh * DH, p.app.dtype, DH, VB, p.app.v_group,
-                             p.app.v_codes + crow * RV,
-                             VB == 16 ? nullptr : p.app.v_scales + crow * (DH / p.app.v_group), lane);
-                fence_proxy_async_global();
-                __syncwarp();
-            }
+            // the newest token of this tile's (sequence, KV head) must be in the
+            // cache before the tile is loaded
+            if (fuse_app && app_rel == i) do_app();
             int ok = 1;
             if (lane == 0 && i >= S) ok = mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, p.timeout_ns);
             ok = __shfl_sync(FULL, ok, 0);
@@ -490,6 +516,8 @@ __global__ void __launch_bounds__(NTHR, 2)
                 s = 0;
                 ph ^= 1u;
             }
+            // ring full: quantise a pending newest token instead of only waiting
+            if (fuse_app && i >= S - 1 && app_rel < n_units) do_app();
             // advance to the next unit (the length is re-read only when b changes)
             if (++tile == tiles_b) {
                 tile = 0;
@@ -966,10 +994,13 @@ __global__ void __launch_bounds__(NTHR, 2)
                     const uint32_t yAB = prmt(hA, hB, 0x5410u), yCE = prmt(hC, hE, 0x5410u);
 #pragma unroll
                     for (int h = 0; h < 2; h++) {
-                        const uint32_t a0 = i4_pair(yAB, 2 * h);
-                        const uint32_t a1 = i4_pair(yAB, 2 * h + 1);
-                        const uint32_t a2 = i4_pair(yCE, 2 * h);
-                        const uint32_t a3 = i4_pair(yCE, 2 * h + 1);
+                        // rows gid take the even nibble (1032 + code), rows gid + 8 the
+                        // odd one in place (1152 + 16 code): no shift for it
+                        const uint32_t xAB = h ? yAB >> 8 : yAB, xCE = h ? yCE >> 8 : yCE;
+                        const uint32_t a0 = and_xor(xAB, 0x000F000Fu, 0x64086408u);
+                        const uint32_t a1 = and_xor(xAB, 0x00F000F0u, 0x64806480u);
+                        const uint32_t a2 = and_xor(xCE, 0x000F000Fu, 0x64086408u);
+                        const uint32_t a3 = and_xor(xCE, 0x00F000F0u, 0x64806480u);
                         mma_16816(o_acc[2 * blk + h], a0, a1, a2, a3, b0, b1);
                     }
                 } else {
@@ -1024,13 +1055,20 @@ __global__ void __launch_bounds__(NTHR, 2)
                     float *oc = mine + (size_t)col * CS;
 #pragma unroll
                     for (int blk = 0; blk < NG; blk++) {
-                        const float corr = BIAS_V * psum[VG ? blk : 0][c];
+                        const float ps = psum[VG ? blk : 0][c];
 #pragma unroll
                         for (int h = 0; h < 2; h++) {
                             // m-tile 2blk+h: row gid <-> d = 32blk + 4gid + 2h, row gid+8 <-> d + 1
                             const int d = 32 * blk + 4 * gid + 2 * h;
-                            *reinterpret_cast<float2 *>(oc + d) =
-                                make_float2(o_acc[2 * blk + h][c] - corr, o_acc[2 * blk + h][2 + c] - corr);
+                            float lo = o_acc[2 * blk + h][c], hi = o_acc[2 * blk + h][2 + c];
+                            if constexpr (VB == 4) {
+                                lo -= 1032.f * ps;                // even nibble: 1032 + code
+                                hi = (hi - 1152.f * ps) * 0.0625f;  // odd nibble: 1152 + 16 code
+                            } else {
+                                lo -= BIAS_V * ps;
+                                hi -= BIAS_V * ps;
+                            }
+                            *reinterpret_cast<float2 *>(oc + d) = make_float2(lo, hi);
                         }
                     }
                     if (gid == 0) *reinterpret_cast<float2 *>(oc + DH) = make_float2(m_run[c], lt[c]);
