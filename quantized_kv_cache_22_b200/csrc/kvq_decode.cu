@@ -176,7 +176,21 @@ cudaError_t launch_decode(const DecodeLaunch &plan, const DecodeParams &p, const
     if (e != cudaSuccess) return e;
     void *args[] = {const_cast<CUtensorMap *>(&tm_k), const_cast<CUtensorMap *>(&tm_v),
                     const_cast<DecodeParams *>(&p)};
-    return cudaLaunchKernel(fn, dim3(p.num_ctas), dim3(NTHR), args, plan.smem_bytes, stream);
+    // Programmatic dependent launch: the kernel may be scheduled while the
+    // previous work on the stream drains; it waits for that work's completion
+    // (griddepcontrol.wait) before its first global-memory access.
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(p.num_ctas);
+    lc.blockDim = dim3(NTHR);
+    lc.dynamicSmemBytes = plan.smem_bytes;
+    lc.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    (void)cudaGetLastError();  // drop a stale, already-reported error of an earlier call
+    return cudaLaunchKernelExC(&lc, fn, args);
 }
 
 cudaError_t launch_merge(const MergeParams &p, cudaStream_t stream)

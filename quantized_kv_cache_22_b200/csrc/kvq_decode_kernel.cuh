@@ -326,7 +326,16 @@ __global__ void __launch_bounds__(NTHR, 2)
         mbar_init(&segbar[1], NW);
         ctl[0] = 0;
         fence_mbar_init();
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
     }
+    // Launched as a programmatic dependent: everything above only touches this
+    // CTA's shared memory and the launch parameters; from here on the kernel
+    // reads and writes global memory, so it first waits for the preceding
+    // grid (whatever it is) to complete.  The next launch may be scheduled now:
+    // it waits the same way before touching memory.
+    grid_dependency_wait();
+    grid_launch_dependents();
 
     // ---- work range of this CTA (computed by the producer warp) -------------
     __shared__ long long sh_u_begin, sh_n, sh_pe;
@@ -378,10 +387,6 @@ __global__ void __launch_bounds__(NTHR, 2)
 
     if (warp == NW) {
         // ====================== producer (whole warp) ======================
-        if (lane == 0) {
-            prefetch_tensormap(&tm_k);
-            prefetch_tensormap(&tm_v);
-        }
         // codes and scales are read once: let them leave L2 first, so that the
         // partials and the queries stay cached
         const uint64_t pol = l2_evict_first_policy();

@@ -159,6 +159,21 @@ __device__ __forceinline__ void bulk_load_hint(void *dst, const void *src, uint3
         : "memory");
 }
 
+// ---------------------------------------------------------------- programmatic launch
+// Wait until the grids this launch depends on have completed and their memory
+// operations are visible (returns at once when there is no such dependency).
+__device__ __forceinline__ void grid_dependency_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Let launches that depend on this grid be scheduled before it completes (they
+// still wait for its completion in grid_dependency_wait).
+__device__ __forceinline__ void grid_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- warp MMA
 // D += A * B, m16n8k16, A row-major 16x16 f16, B col-major 16x8 f16, f32 acc.
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
