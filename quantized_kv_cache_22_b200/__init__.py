@@ -98,19 +98,25 @@ def _check(fn, rc):
 
 
 def _ptr(t):
-    if t is None:
-        return None
-    return ctypes.c_void_p(t.data_ptr())
+    # plain ints: ctypes converts them for c_void_p arguments
+    return None if t is None else t.data_ptr()
+
+
+_DTYPE_CODES = {torch.float16: KVQ_F16, torch.float32: KVQ_F32, torch.bfloat16: KVQ_BF16}
 
 
 def _dtype_code(t: torch.Tensor) -> int:
-    return {torch.float16: KVQ_F16, torch.float32: KVQ_F32, torch.bfloat16: KVQ_BF16}[t.dtype]
+    return _DTYPE_CODES[t.dtype]
 
 
 def _stream(stream):
     if stream is None:
-        stream = torch.cuda.current_stream()
-    return ctypes.c_void_p(stream.cuda_stream)
+        # the current stream's handle without building a Stream object
+        return torch._C._cuda_getCurrentRawStream(torch.cuda.current_device())
+    return stream.cuda_stream
+
+
+_CFG_MEMO = {}   # field tuple -> (KvqConfig, byref); the library only reads the struct
 
 
 @dataclass
@@ -131,11 +137,26 @@ class Config:
     h_bits: int = 4
     h_groups: int = 0
 
+    def _key(self):
+        return (self.mode, self.batch, self.capacity, self.n_layers, self.n_q_heads,
+                self.n_kv_heads, self.head_dim, self.k_bits, self.v_bits,
+                self.k_group or self.head_dim, self.v_group or self.head_dim,
+                self.d_model, self.h_bits, self.h_groups)
+
     def c(self) -> KvqConfig:
-        return KvqConfig(self.mode, self.batch, self.capacity, self.n_layers, self.n_q_heads,
-                         self.n_kv_heads, self.head_dim, self.k_bits, self.v_bits,
-                         self.k_group or self.head_dim, self.v_group or self.head_dim,
-                         self.d_model, self.h_bits, self.h_groups)
+        """A new ``kvq_config`` struct with these fields."""
+        return KvqConfig(*self._key())
+
+    def _ref(self):
+        """byref() of a shared struct with these fields (read-only use by the wrappers)."""
+        key = self._key()
+        r = _CFG_MEMO.get(key)
+        if r is None:
+            if len(_CFG_MEMO) > 256:
+                _CFG_MEMO.clear()
+            c = KvqConfig(*key)
+            r = _CFG_MEMO[key] = (c, ctypes.byref(c))
+        return r[1]
 
 
 # ----------------------------------------------------------------------------- host-only calls
@@ -183,8 +204,19 @@ class LayerCache:
         self.cfg = cfg
 
     def c(self) -> KvqLayer:
+        """A new ``kvq_layer`` struct with these buffers."""
         return KvqLayer(*(None if t is None else t.data_ptr()
                           for t in (self.k_codes, self.k_scales, self.v_codes, self.v_scales)))
+
+    def _ref(self):
+        """byref() of a struct kept for these buffers (read-only use by the wrappers)."""
+        ts = (self.k_codes, self.k_scales, self.v_codes, self.v_scales)
+        memo = self.__dict__.get("_c_memo")
+        if memo is None or any(a is not b for a, b in zip(memo[0], ts)):
+            c = self.c()
+            memo = (ts, c, ctypes.byref(c))
+            self.__dict__["_c_memo"] = memo
+        return memo[2]
 
 
 class Workspace:
@@ -200,7 +232,7 @@ class Workspace:
 
 def kvq_append(cfg: Config, layer: LayerCache, k: torch.Tensor, v, d_pos: torch.Tensor,
                max_pos: int, n_new: int, stream=None):
-    _check("kvq_append", _lib.kvq_append(ctypes.byref(cfg.c()), ctypes.byref(layer.c()), _ptr(k),
+    _check("kvq_append", _lib.kvq_append(cfg._ref(), layer._ref(), _ptr(k),
                                          _ptr(v), _dtype_code(k), _ptr(d_pos), int(max_pos),
                                          int(n_new), _stream(stream)))
 
@@ -210,7 +242,7 @@ def kvq_decode_attn(cfg: Config, layer: LayerCache, q: torch.Tensor, d_len: torc
                     num_ctas: int = 0, w_kv=None, kv_scratch=None, stream=None):
     scratch_bytes = 0 if kv_scratch is None else kv_scratch.numel() * kv_scratch.element_size()
     _check("kvq_decode_attn",
-           _lib.kvq_decode_attn(ctypes.byref(cfg.c()), ctypes.byref(layer.c()), _ptr(q),
+           _lib.kvq_decode_attn(cfg._ref(), layer._ref(), _ptr(q),
                                 _dtype_code(q), _ptr(d_len), int(max_len), float(softmax_scale),
                                 _ptr(out), _dtype_code(out), _ptr(ws.buf), ws.nbytes,
                                 int(num_ctas), _ptr(w_kv), _ptr(kv_scratch), scratch_bytes,
@@ -225,7 +257,7 @@ def kvq_append_decode_attn(cfg: Config, layer: LayerCache, k_new: torch.Tensor,
     if k_new.dtype != v_new.dtype:
         raise ValueError("k_new and v_new must share a dtype")
     _check("kvq_append_decode_attn",
-           _lib.kvq_append_decode_attn(ctypes.byref(cfg.c()), ctypes.byref(layer.c()), _ptr(k_new),
+           _lib.kvq_append_decode_attn(cfg._ref(), layer._ref(), _ptr(k_new),
                                        _ptr(v_new), _dtype_code(k_new), _ptr(q), _dtype_code(q),
                                        _ptr(d_len), int(max_len), float(softmax_scale), _ptr(out),
                                        _dtype_code(out), _ptr(ws.buf), ws.nbytes, int(num_ctas),
@@ -236,7 +268,7 @@ def kvq_decode_partials(cfg: Config, layer: LayerCache, q: torch.Tensor, d_len: 
                         max_len: int, ws: Workspace, softmax_scale: float = 0.0, num_ctas: int = 0,
                         stream=None):
     _check("kvq_decode_partials",
-           _lib.kvq_decode_partials(ctypes.byref(cfg.c()), ctypes.byref(layer.c()), _ptr(q),
+           _lib.kvq_decode_partials(cfg._ref(), layer._ref(), _ptr(q),
                                     _dtype_code(q), _ptr(d_len), int(max_len), float(softmax_scale),
                                     _ptr(ws.buf), ws.nbytes, int(num_ctas), _stream(stream)))
 
@@ -244,13 +276,13 @@ def kvq_decode_partials(cfg: Config, layer: LayerCache, q: torch.Tensor, d_len: 
 def kvq_merge_partials(cfg: Config, d_len: torch.Tensor, out: torch.Tensor, ws: Workspace,
                        num_ctas: int = 0, stream=None):
     _check("kvq_merge_partials",
-           _lib.kvq_merge_partials(ctypes.byref(cfg.c()), _ptr(d_len), _ptr(out), _dtype_code(out),
+           _lib.kvq_merge_partials(cfg._ref(), _ptr(d_len), _ptr(out), _dtype_code(out),
                                    _ptr(ws.buf), ws.nbytes, int(num_ctas), _stream(stream)))
 
 
 def kvq_h_operand_bytes(cfg: Config, max_len: int) -> int:
     v = ctypes.c_uint64()
-    _check("kvq_h_operand_bytes", _lib.kvq_h_operand_bytes(ctypes.byref(cfg.c()), max_len,
+    _check("kvq_h_operand_bytes", _lib.kvq_h_operand_bytes(cfg._ref(), max_len,
                                                            ctypes.byref(v)))
     return v.value
 
@@ -259,7 +291,7 @@ def kvq_h_reconstruct(cfg: Config, layer: LayerCache, w_kv: torch.Tensor, max_le
                       k_out: torch.Tensor, v_out: torch.Tensor, out_capacity: int,
                       operand: torch.Tensor, stream=None):
     _check("kvq_h_reconstruct",
-           _lib.kvq_h_reconstruct(ctypes.byref(cfg.c()), ctypes.byref(layer.c()), _ptr(w_kv),
+           _lib.kvq_h_reconstruct(cfg._ref(), layer._ref(), _ptr(w_kv),
                                   int(max_len), _ptr(k_out), _ptr(v_out), int(out_capacity),
                                   _ptr(operand), operand.numel() * operand.element_size(),
                                   _stream(stream)))

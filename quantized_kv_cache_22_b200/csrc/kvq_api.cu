@@ -89,7 +89,40 @@ EncodeTiledFn encode_fn()
 // Codes of one layer viewed as [bh][cap][R bytes]; a tile of T tokens is one
 // 128-byte-swizzled box (R <= 128: 128/R tokens per 128-byte line) or two
 // 128-byte-wide boxes (R = 256).
+bool encode_codes_map_uncached(CUtensorMap *m, const void *codes, int bh, int cap, int R);
+
+// The descriptor depends only on (address, bh, cap, R): the last few encodings
+// of this thread are kept, so a decode loop over layers does not re-encode.
 bool encode_codes_map(CUtensorMap *m, const void *codes, int bh, int cap, int R)
+{
+    struct Entry {
+        const void *codes;
+        int bh, cap, R;
+        CUtensorMap map;
+    };
+    constexpr int kEntries = 256;
+    thread_local Entry cache[kEntries];
+    thread_local int used = 0, next = 0;
+    for (int i = 0; i < used; i++) {
+        const Entry &e = cache[i];
+        if (e.codes == codes && e.bh == bh && e.cap == cap && e.R == R) {
+            *m = e.map;
+            return true;
+        }
+    }
+    if (!encode_codes_map_uncached(m, codes, bh, cap, R)) return false;
+    Entry &e = cache[next];
+    e.codes = codes;
+    e.bh = bh;
+    e.cap = cap;
+    e.R = R;
+    e.map = *m;
+    next = (next + 1) % kEntries;
+    if (used < kEntries) used++;
+    return true;
+}
+
+bool encode_codes_map_uncached(CUtensorMap *m, const void *codes, int bh, int cap, int R)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
