@@ -58,12 +58,20 @@ def bf16_peaks():
     return 1590.0, 1400.0, "fallback"
 
 
+def decode_kernel_sha() -> str:
+    """sha256 over the decode kernel's device sources (kernel, PTX wrappers, quantiser)."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in ("kvq_decode_kernel.cuh", "kvq_ptx.cuh", "kvq_quant.cuh"):
+        with open(os.path.join(ROOT, "quantized_kv_cache_22_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def decode_traffic(variant: str):
     """DRAM bytes per decode launch from the committed ncu summary, if it was taken on
-    the current decode kernel source (sha256 of kvq_decode.cu); otherwise None."""
-    import hashlib
+    the current decode kernel sources (decode_kernel_sha); otherwise None."""
     f = os.path.join(ROOT, "profiles", "decode_kernel_traffic.txt")
-    src = os.path.join(ROOT, "quantized_kv_cache_22_b200", "csrc", "kvq_decode.cu")
     if not os.path.exists(f):
         return None
     vals = {}
@@ -71,7 +79,7 @@ def decode_traffic(variant: str):
         parts = line.split()
         if len(parts) == 2 and not line.startswith("#"):
             vals[parts[0]] = parts[1]
-    if vals.get("sha256") != hashlib.sha256(open(src, "rb").read()).hexdigest():
+    if vals.get("sha256") != decode_kernel_sha():
         return None
     return float(vals[variant]) if variant in vals else None
 

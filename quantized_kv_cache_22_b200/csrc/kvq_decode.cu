@@ -85,11 +85,11 @@ bool plan_decode(int dh, int kb, int vb, int ngs_k, int ngs_v, int G, int max_sm
     L.off_sv = L.off_sk + align_up(T * (kb == 16 ? 0 : ngs_k) * 2, 16);
     L.stage_bytes = align_up(L.off_sv + T * (vb == 16 ? 0 : ngs_v) * 2, 1024);
     const uint32_t merge_bytes = (uint32_t)NW * G * slot_col_floats(dh) * 4;
-    // tail: meta[S] (32 B each), barriers (2S + 2) * 8 B, control words 32 B, merge buffer
+    // tail: meta[S] (32 B each), barriers (2S + 2) * 8 B, control words 64 B, merge buffer
     for (int S = 8; S >= 2; S--) {
         const uint32_t off_meta = S * L.stage_bytes;
         const uint32_t off_bar = off_meta + S * (uint32_t)sizeof(StageMeta);
-        const uint32_t off_merge = align_up(off_bar + (2 * S + 2) * 8 + 32, 16);
+        const uint32_t off_merge = align_up(off_bar + (2 * S + 2) * 8 + 64, 16);
         const uint32_t total = off_merge + merge_bytes + 1024;  // + alignment slack
         // keep two CTAs per SM when possible
         if (total <= (uint32_t)max_smem / 2 - 1024 || (S == 2 && total <= (uint32_t)max_smem)) {

@@ -305,7 +305,9 @@ __global__ void __launch_bounds__(NTHR, 2)
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + p.off_bar);
     uint64_t *empty = full + p.stages;
     uint64_t *segbar = empty + p.stages;                // [0] partials in mbuf, [1] mbuf read
-    int *ctl = reinterpret_cast<int *>(segbar + 2);     // [0] abort, [1] units, [2..3] prefix
+    // [0] abort, [1] units, [2..3] prefix, [4..8] segment handed to the combiner:
+    // bh, slot, ncta, cmin, end
+    int *ctl = reinterpret_cast<int *>(segbar + 2);
     float *mbuf = reinterpret_cast<float *>(smem + p.off_merge);   // [NW][G][DH + 4]
 
     const int tid = threadIdx.x;
@@ -322,8 +324,8 @@ __global__ void __launch_bounds__(NTHR, 2)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], NW);
         }
-        mbar_init(&segbar[0], NW);
-        mbar_init(&segbar[1], NW);
+        mbar_init(&segbar[0], NW);   // consumers: partials of a segment in mbuf
+        mbar_init(&segbar[1], 1);    // combiner: mbuf read
         ctl[0] = 0;
         fence_mbar_init();
         prefetch_tensormap(&tm_k);
@@ -553,6 +555,68 @@ __global__ void __launch_bounds__(NTHR, 2)
         return;
     }
 
+    if (warp == NW + 1) {
+        // ====================== combiner ======================
+        // Per segment end: combine the consumer warps' partials from mbuf into
+        // this CTA's slot, hand mbuf back, publish, and merge when this CTA's
+        // partial is the last one of its (sequence, KV head).
+        constexpr int CS = slot_col_floats(DH);
+        const int ncol = (KB == 16 && p.q_dtype != KVQ_F16) ? min(G, 4) : G;
+        for (uint32_t k = 0;; k++) {
+            if (!mbar_wait_bounded(&segbar[0], k & 1u, abort_flag, p.timeout_ns)) {
+                if (lane == 0 && *abort_flag == 0) {
+                    ctl[0] = 1;
+                    atomicExch(p.status, KVQ_ERR_TIMEOUT);
+                }
+                return;
+            }
+            const volatile int *seg = ctl + 4;
+            const int bh = seg[0], slot = seg[1], ncta = seg[2], cmin = seg[3], end = seg[4];
+            if (end) return;
+            float *dst = p.ws + (size_t)slot * G * CS;
+            for (int c = lane; c < ncol * (DH / 4); c += 32) {
+                const int col = c / (DH / 4), d = 4 * (c % (DH / 4));
+                float M = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < NW; w++) M = fmaxf(M, mbuf[((size_t)w * G + col) * CS + DH]);
+                float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+                float L = 0.f;
+#pragma unroll
+                for (int w = 0; w < NW; w++) {
+                    const float *src = mbuf + ((size_t)w * G + col) * CS;
+                    const float mw = src[DH];
+                    const float e = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+                    const float4 x = *reinterpret_cast<const float4 *>(src + d);
+                    O.x = fmaf(e, x.x, O.x);
+                    O.y = fmaf(e, x.y, O.y);
+                    O.z = fmaf(e, x.z, O.z);
+                    O.w = fmaf(e, x.w, O.w);
+                    L = fmaf(e, src[DH + 1], L);
+                }
+                *reinterpret_cast<float4 *>(dst + (size_t)col * CS + d) = O;
+                if (d == 0) *reinterpret_cast<float2 *>(dst + (size_t)col * CS + DH) = make_float2(M, L);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&segbar[1]);   // the consumers may refill mbuf
+            if (p.counters != nullptr) {
+                // publish (fence, then count the arrival); the CTA whose arrival
+                // completes the count merges and writes the output
+                __threadfence();
+                __syncwarp();
+                int last = 0;
+                if (lane == 0) last = atomicAdd(&p.counters[bh], 1) == ncta - 1;
+                last = __shfl_sync(FULL, last, 0);
+                if (last) {
+                    __threadfence();
+                    const int b = bh / Hkv, kvh = bh % Hkv;
+                    merge_segment<DH>(p.ws, (int64_t)cmin + bh, ncta, G, p.out, p.out_f32,
+                                      ((int64_t)b * p.n_q_heads + (int64_t)kvh * G) * DH, lane);
+                    if (lane == 0) p.counters[bh] = 0;   // ready for the next launch
+                }
+            }
+        }
+    }
+
     // ====================== consumers ======================
     constexpr bool IMMA_K = KB != 16;
     const int gid = lane >> 2;
@@ -723,11 +787,13 @@ __global__ void __launch_bounds__(NTHR, 2)
     const uint32_t ONE2 = 0x3C003C00u;   // half2(1, 1)
     int s = 0;
     uint32_t ph = 0;
-    uint32_t seg_parity = 0;
+    uint32_t nseg = 0;           // segment ends handed to the combiner
+    bool aborted = false;
     for (int i = 0; i < n_units; i++) {
         if (!mbar_wait_bounded(&full[s], ph, abort_flag, limit)) {
             ctl[0] = 1;
             atomicExch(p.status, KVQ_ERR_TIMEOUT);
+            aborted = true;
             break;
         }
         StageMeta m;
@@ -1039,7 +1105,7 @@ __global__ void __launch_bounds__(NTHR, 2)
             ph ^= 1u;
         }
 
-        // ---------------- segment end: combine the warps, write the partial ------
+        // ---------------- segment end: hand this warp's partial to the combiner ---
         if (m.flags & 2) {
             constexpr int CS = slot_col_floats(DH);
             float lt[2];
@@ -1050,6 +1116,13 @@ __global__ void __launch_bounds__(NTHR, 2)
                 v += __shfl_xor_sync(FULL, v, 8);
                 v += __shfl_xor_sync(FULL, v, 16);
                 lt[c] = v;
+            }
+            // the combiner must have read the previous segment out of mbuf
+            if (nseg > 0 && !mbar_wait_bounded(&segbar[1], (nseg - 1) & 1u, abort_flag, limit)) {
+                ctl[0] = 1;
+                atomicExch(p.status, KVQ_ERR_TIMEOUT);
+                aborted = true;
+                break;
             }
             // this warp's partial into mbuf[warp]: [G][DH + 4] floats, o then (m, l)
             float *mine = mbuf + (size_t)warp * G * CS;
@@ -1079,65 +1152,25 @@ __global__ void __launch_bounds__(NTHR, 2)
                     if (gid == 0) *reinterpret_cast<float2 *>(oc + DH) = make_float2(m_run[c], lt[c]);
                 }
             }
+            if (warp == 0 && lane == 0) {
+                volatile int *seg = ctl + 4;
+                seg[0] = m.bh; seg[1] = m.slot; seg[2] = m.ncta; seg[3] = m.cmin; seg[4] = 0;
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(&segbar[0]);
-            if (!mbar_wait_bounded(&segbar[0], seg_parity, abort_flag, limit)) {
-                ctl[0] = 1;
-                atomicExch(p.status, KVQ_ERR_TIMEOUT);
-                break;
-            }
-            // combine the NW warps (each takes a quarter of the float4 chunks) and
-            // write this CTA's partial of the segment
-            const int ncol = qsplit ? min(G, 4) : G;
-            float *dst = p.ws + (size_t)m.slot * G * CS;
-            for (int k = warp * 32 + lane; k < ncol * (DH / 4); k += 32 * NW) {
-                const int col = k / (DH / 4), d = 4 * (k % (DH / 4));
-                float M = -INFINITY;
-#pragma unroll
-                for (int w = 0; w < NW; w++) M = fmaxf(M, mbuf[((size_t)w * G + col) * CS + DH]);
-                float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-                float L = 0.f;
-#pragma unroll
-                for (int w = 0; w < NW; w++) {
-                    const float *src = mbuf + ((size_t)w * G + col) * CS;
-                    const float mw = src[DH];
-                    const float e = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
-                    const float4 x = *reinterpret_cast<const float4 *>(src + d);
-                    O.x = fmaf(e, x.x, O.x);
-                    O.y = fmaf(e, x.y, O.y);
-                    O.z = fmaf(e, x.z, O.z);
-                    O.w = fmaf(e, x.w, O.w);
-                    L = fmaf(e, src[DH + 1], L);
-                }
-                *reinterpret_cast<float4 *>(dst + (size_t)col * CS + d) = O;
-                if (d == 0) *reinterpret_cast<float2 *>(dst + (size_t)col * CS + DH) = make_float2(M, L);
-            }
-            // mbuf is free again once every warp has read it
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&segbar[1]);
-            if (!mbar_wait_bounded(&segbar[1], seg_parity, abort_flag, limit)) {
-                ctl[0] = 1;
-                atomicExch(p.status, KVQ_ERR_TIMEOUT);
-                break;
-            }
-            seg_parity ^= 1u;
-            if (p.counters != nullptr) {
-                // the warp that completes the last partial of this (sequence, KV
-                // head) merges them (publish: fence, then count the arrival)
-                __threadfence();
-                __syncwarp();
-                int last = 0;
-                if (lane == 0) last = atomicAdd(&p.counters[m.bh], 1) == NW * m.ncta - 1;
-                last = __shfl_sync(FULL, last, 0);
-                if (last) {
-                    __threadfence();
-                    const int b = m.bh / Hkv, kvh = m.bh % Hkv;
-                    merge_segment<DH>(p.ws, (int64_t)m.cmin + m.bh, m.ncta, G, p.out, p.out_f32,
-                                      ((int64_t)b * p.n_q_heads + (int64_t)kvh * G) * DH, lane);
-                    if (lane == 0) p.counters[m.bh] = 0;   // ready for the next launch
-                }
-            }
+            nseg++;
         }
+    }
+    if (!aborted) {
+        // tell the combiner there is no further segment
+        if (nseg > 0 && !mbar_wait_bounded(&segbar[1], (nseg - 1) & 1u, abort_flag, limit)) {
+            ctl[0] = 1;
+            atomicExch(p.status, KVQ_ERR_TIMEOUT);
+            return;
+        }
+        if (warp == 0 && lane == 0) ctl[8] = 1;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&segbar[0]);
     }
 }
 

@@ -23,7 +23,8 @@ cudaError_t launch_append(const AppendParams &k, const AppendParams *v, cudaStre
 // ------------------------------------------------------------------ decode
 constexpr int kDecodeConsumerWarps = 4;
 constexpr int kDecodeTileTokens = 32 * kDecodeConsumerWarps;   // tokens per stage (32 per warp)
-constexpr int kDecodeThreads = 32 * (kDecodeConsumerWarps + 1);
+// consumer warps, one producer warp, one combiner warp
+constexpr int kDecodeThreads = 32 * (kDecodeConsumerWarps + 2);
 constexpr int kWorkspaceHeaderFloats = 64;                      // status word + padding
 
 // The new token's K/V for the append step fused into the decode kernel.
