@@ -19,7 +19,8 @@
  *         --kvq-val) and the 8K-token memory table.
  *   [MNI] "kv-cache-int8-35x-speedup-rust-cuda" (mni-ml/framework): KV cache
  *         keeps past K/V and computes one new K/V per step; INT8 KV.
- *   [OD]  gyaansetu.com on-device LLM page: INT4 keys with INT8 values.
+ *   [OD]  gyaansetu.com on-device LLM page: INT4 keys with INT8 values; a
+ *         sliding window of recent tokens plus anchor tokens.
  *
  * Conventions for every call:
  *   Ownership.  The caller allocates every buffer (cache, inputs, outputs,
@@ -100,6 +101,14 @@ typedef struct kvq_config {
     int32_t h_bits;      /* h-mode: 4, 8 or 16                                    */
     int32_t h_groups;    /* h-mode: fp16 scales per token (the "per-head" scales
                             of [TL]); D / h_groups must be 32, 64 or 128          */
+    int32_t window;      /* KV mode, 0 or a sliding window ([OD] "1536 recent + 64
+                            anchors"): the cache keeps the first n_anchor tokens
+                            and a ring of the most recent `window` tokens, and
+                            capacity must equal n_anchor + window.  Token t (0-
+                            based, counted over the whole sequence) lives in slot
+                            t while t < n_anchor, else in slot n_anchor +
+                            (t - n_anchor) mod window.  0: no window, slot t.     */
+    int32_t n_anchor;    /* KV mode with a window: anchor tokens kept for good    */
 } kvq_config;
 
 /* One layer's cache buffers (device pointers, caller-owned).

@@ -38,7 +38,8 @@ class KvqError(RuntimeError):
 class KvqConfig(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "mode", "batch", "capacity", "n_layers", "n_q_heads", "n_kv_heads", "head_dim",
-        "k_bits", "v_bits", "k_group", "v_group", "d_model", "h_bits", "h_groups")]
+        "k_bits", "v_bits", "k_group", "v_group", "d_model", "h_bits", "h_groups",
+        "window", "n_anchor")]
 
 
 class KvqLayer(ctypes.Structure):
@@ -136,12 +137,14 @@ class Config:
     d_model: int = 0
     h_bits: int = 4
     h_groups: int = 0
+    window: int = 0       # sliding window: ring of recent tokens (capacity = n_anchor + window)
+    n_anchor: int = 0     # tokens kept at the start of the sequence
 
     def _key(self):
         return (self.mode, self.batch, self.capacity, self.n_layers, self.n_q_heads,
                 self.n_kv_heads, self.head_dim, self.k_bits, self.v_bits,
                 self.k_group or self.head_dim, self.v_group or self.head_dim,
-                self.d_model, self.h_bits, self.h_groups)
+                self.d_model, self.h_bits, self.h_groups, self.window, self.n_anchor)
 
     def c(self) -> KvqConfig:
         """A new ``kvq_config`` struct with these fields."""

@@ -50,7 +50,12 @@ int check_cfg(const kvq_config *c)
         if (!valid_bits(c->k_bits) || !valid_bits(c->v_bits)) return KVQ_ERR_UNSUPPORTED;
         if (c->k_bits != 16 && !valid_group(c->k_group, c->head_dim)) return KVQ_ERR_UNSUPPORTED;
         if (c->v_bits != 16 && !valid_group(c->v_group, c->head_dim)) return KVQ_ERR_UNSUPPORTED;
+        if (c->window < 0 || c->n_anchor < 0) return KVQ_ERR_INVALID_ARG;
+        if (c->window == 0 && c->n_anchor != 0) return KVQ_ERR_INVALID_ARG;
+        if (c->window > 0 && (int64_t)c->n_anchor + c->window != c->capacity)
+            return KVQ_ERR_INVALID_ARG;
     } else {
+        if (c->window != 0 || c->n_anchor != 0) return KVQ_ERR_UNSUPPORTED;
         if (c->d_model < 128 || c->d_model % 128 != 0) return KVQ_ERR_UNSUPPORTED;
         if (!valid_bits(c->h_bits)) return KVQ_ERR_UNSUPPORTED;
         if (c->h_bits != 16) {
@@ -322,9 +327,12 @@ int kvq_append(const kvq_config *cfg, const kvq_layer *layer, const void *k, con
     if (!layer || !d_pos || n_new < 0 || max_pos_host < 0) return KVQ_ERR_INVALID_ARG;
     if (in_dtype != KVQ_F16 && in_dtype != KVQ_F32 && in_dtype != KVQ_BF16)
         return KVQ_ERR_INVALID_ARG;
-    if ((int64_t)max_pos_host + n_new > cfg->capacity) return KVQ_ERR_CAPACITY;
+    // with a sliding window positions grow without bound (ring slots)
+    if (cfg->window == 0 && (int64_t)max_pos_host + n_new > cfg->capacity) return KVQ_ERR_CAPACITY;
     if (n_new == 0) return KVQ_OK;
     AppendParams pk{};
+    pk.window = cfg->window;
+    pk.n_anchor = cfg->n_anchor;
     pk.in_dtype = in_dtype;
     pk.batch = cfg->batch;
     pk.n_new = n_new;
@@ -478,6 +486,8 @@ static int decode_kv_layout(const kvq_config *cfg, const void *k_codes, const vo
         p.tau_log2e = scale * 1.4426950408889634f;
         p.timeout_ns = kTimeoutNs;
         if (app) p.app = *app;
+        p.window = cfg->mode == KVQ_MODE_KV ? cfg->window : 0;
+        p.n_anchor = cfg->mode == KVQ_MODE_KV ? cfg->n_anchor : 0;
         cudaError_t e = launch_decode(plan, p, tm_k, tm_v, stream);
         if (e != cudaSuccess) return fail("decode launch", e);
         return KVQ_OK;
@@ -524,7 +534,7 @@ int kvq_decode_partials(const kvq_config *cfg, const kvq_layer *layer, const voi
     if (!layer || !q || !d_len || !workspace || num_ctas < 0) return KVQ_ERR_INVALID_ARG;
     if (q_dtype != KVQ_F16 && q_dtype != KVQ_F32 && q_dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
     if (!std::isfinite(softmax_scale) || max_len_host < 0) return KVQ_ERR_INVALID_ARG;
-    if (max_len_host > cfg->capacity) return KVQ_ERR_CAPACITY;
+    if (max_len_host > cfg->capacity && cfg->window == 0) return KVQ_ERR_CAPACITY;
     if (!aligned16(q) || !aligned16(workspace)) return KVQ_ERR_ALIGN;
     rc = check_kv_layer(cfg, layer);
     if (rc) return rc;
@@ -563,7 +573,7 @@ static int h_reconstruct_impl(const kvq_config *cfg, const kvq_layer *layer, con
     if (cfg->h_bits != 16 && !layer->k_scales) return KVQ_ERR_INVALID_ARG;
     if (max_len_host < 0 || out_capacity < max_len_host || out_capacity % 64 != 0)
         return KVQ_ERR_INVALID_ARG;
-    if (max_len_host > cfg->capacity) return KVQ_ERR_CAPACITY;
+    if (max_len_host > cfg->capacity && cfg->window == 0) return KVQ_ERR_CAPACITY;
     if (!aligned16(layer->k_codes) || !aligned16(w_kv) || !aligned16(k_out) ||
         !aligned16(v_out) || !aligned16(operand) ||
         (layer->k_scales && !aligned16(layer->k_scales)))
@@ -606,7 +616,7 @@ int kvq_decode_attn(const kvq_config *cfg, const kvq_layer *layer, const void *q
     if (out_dtype != KVQ_F16 && out_dtype != KVQ_F32) return KVQ_ERR_INVALID_ARG;
     if (!std::isfinite(softmax_scale)) return KVQ_ERR_INVALID_ARG;
     if (max_len_host < 0) return KVQ_ERR_INVALID_ARG;
-    if (max_len_host > cfg->capacity) return KVQ_ERR_CAPACITY;
+    if (max_len_host > cfg->capacity && cfg->window == 0) return KVQ_ERR_CAPACITY;
     if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return KVQ_ERR_ALIGN;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
@@ -665,7 +675,7 @@ int kvq_append_decode_attn(const kvq_config *cfg, const kvq_layer *layer, const 
     if (q_dtype != KVQ_F16 && q_dtype != KVQ_F32 && q_dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
     if (out_dtype != KVQ_F16 && out_dtype != KVQ_F32) return KVQ_ERR_INVALID_ARG;
     if (!std::isfinite(softmax_scale) || max_len_host < 0) return KVQ_ERR_INVALID_ARG;
-    if (max_len_host > cfg->capacity) return KVQ_ERR_CAPACITY;
+    if (max_len_host > cfg->capacity && cfg->window == 0) return KVQ_ERR_CAPACITY;
     if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(q) || !aligned16(out) ||
         !aligned16(workspace))
         return KVQ_ERR_ALIGN;

@@ -2,7 +2,9 @@
 //
 // One warp quantises one row (one token of one KV head, or one token's h
 // vector) with the row quantiser of kvq_quant.cuh (TinyLoop docs "KV Cache
-// 模式" modes table; KVSplit independent key/value widths and groups).
+// 模式" modes table; KVSplit independent key/value widths and groups).  With a
+// sliding window (on-device page, "Sliding Window Eviction": recent tokens
+// plus anchors) a token goes to its ring slot.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -30,11 +32,19 @@ __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ App
     const int64_t bj = row / p.rows_per_tok;
     const int j = (int)(bj % p.n_new);
     const int b = (int)(bj / p.n_new);
-    const int pos = p.d_pos[b] + j;
-    if (pos < 0 || pos >= p.cap) return;  // the kernel's own bounds check
+    const int first = p.d_pos[b];
+    const int pos = first + j;
+    if (pos < 0) return;
+    int slot = pos;
+    if (p.window > 0) {
+        // a token that a later token of this call overwrites in the ring is skipped
+        if (pos >= p.n_anchor && pos + p.window <= first + p.n_new - 1) return;
+        slot = cache_slot(pos, p.window, p.n_anchor);
+    }
+    if (slot >= p.cap) return;  // the kernel's own bounds check
 
     const int dim = p.dim;
-    const int64_t cache_row = ((int64_t)b * p.rows_per_tok + head) * p.cap + pos;
+    const int64_t cache_row = ((int64_t)b * p.rows_per_tok + head) * p.cap + slot;
     uint8_t *codes_row = p.codes + cache_row * ((int64_t)dim * p.bits / 8);
     __half *scales_row = p.bits == 16 ? nullptr : p.scales + cache_row * (dim / p.group);
     quantize_row(p.x, row * (int64_t)dim, p.in_dtype, dim, p.bits, p.group, codes_row, scales_row,

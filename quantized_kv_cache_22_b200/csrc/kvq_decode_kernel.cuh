@@ -415,10 +415,16 @@ __global__ void __launch_bounds__(NTHR, 2)
         int ab = b, akvh = kvh, alen = len_b, atiles = tiles_b;
         long long apre = pre;
         int app_rel = n_units;
+        // cache slot of sequence ab's newest token (position d_len - 1; with a
+        // sliding window its ring slot, anywhere among the cached tokens)
+        auto newest_slot = [&]() {
+            return p.window > 0 ? cache_slot(p.d_len[ab] - 1, p.window, p.n_anchor) : alen - 1;
+        };
+        int aslot = (ab >= 0 && ab < p.batch && alen > 0) ? newest_slot() : 0;
         auto find_app = [&]() {
             app_rel = n_units;
             while (ab < p.batch) {
-                const long long ulast = apre + (long long)akvh * atiles + atiles - 1;
+                const long long ulast = apre + (long long)akvh * atiles + aslot / T;
                 const long long rel = ulast - sh_u_begin;
                 if (rel >= n_units) return;            // beyond this CTA's range
                 if (atiles > 0 && rel >= 0) {
@@ -432,12 +438,13 @@ __global__ void __launch_bounds__(NTHR, 2)
                     ++ab;
                     alen = (ab < p.batch) ? clamp_len(p.d_len[ab], cap) : 0;
                     atiles = (alen + T - 1) / T;
+                    aslot = alen > 0 ? newest_slot() : 0;
                 }
             }
         };
         auto do_app = [&]() {
             const int bh = ab * Hkv + akvh;
-            const int64_t crow = (int64_t)bh * cap + (alen - 1);
+            const int64_t crow = (int64_t)bh * cap + aslot;
             quantize_row(p.app.k_new, (int64_t)bh * DH, p.app.dtype, DH, KB, p.app.k_group,
                          p.app.k_codes + crow * RK,
                          KB == 16 ? nullptr : p.app.k_scales + crow * (DH / p.app.k_group), lane);
@@ -454,6 +461,7 @@ __global__ void __launch_bounds__(NTHR, 2)
                 ++ab;
                 alen = (ab < p.batch) ? clamp_len(p.d_len[ab], cap) : 0;
                 atiles = (alen + T - 1) / T;
+                aslot = alen > 0 ? newest_slot() : 0;
             }
             find_app();
         };
@@ -470,8 +478,8 @@ __global__ void __launch_bounds__(NTHR, 2)
                 seg_cmin = (int)cmin;
                 seg_ncta = (int)(cmax - cmin + 1);
             }
-            // the newest token of this tile's (sequence, KV head) must be in the
-            // cache before the tile is loaded
+            // the newest token of a (sequence, KV head) must be in the cache
+            // before the tile that holds its slot is loaded
             if (fuse_app && app_rel == i) do_app();
             int ok = 1;
             if (lane == 0 && i >= S) ok = mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, p.timeout_ns);

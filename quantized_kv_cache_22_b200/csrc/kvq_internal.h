@@ -16,7 +16,16 @@ struct AppendParams {
     int32_t in_dtype;       // KVQ_F16 / KVQ_F32 / KVQ_BF16
     int32_t batch, n_new, rows_per_tok, dim, cap;
     int32_t bits, group;
+    int32_t window, n_anchor;   // sliding window (0: slot = position)
 };
+
+// Cache slot of token position t: the first n_anchor tokens stay put, the rest
+// share a ring of `window` slots (window 0: no ring, slot t).
+__host__ __device__ inline int cache_slot(int t, int window, int n_anchor)
+{
+    if (window <= 0 || t < n_anchor) return t;
+    return n_anchor + (t - n_anchor) % window;
+}
 
 cudaError_t launch_append(const AppendParams &k, const AppendParams *v, cudaStream_t stream);
 
@@ -56,6 +65,7 @@ struct DecodeParams {
     float tau_log2e;
     uint64_t timeout_ns;
     FusedAppend app;
+    int32_t window, n_anchor;  // sliding window: slot of the newest token (fused append)
 };
 
 struct MergeParams {

@@ -97,7 +97,8 @@ def test_validation_errors_are_returned_on_the_host():
     # bad configs
     for field, val, want in (("capacity", 40, -2), ("head_dim", 96, -2), ("k_bits", 6, -2),
                              ("n_q_heads", 3, -1), ("batch", 0, -1), ("k_group", 48, -2),
-                             ("mode", 7, -1)):
+                             ("mode", 7, -1), ("window", 100, -1), ("n_anchor", 4, -1),
+                             ("window", -1, -1)):
         c = Config(batch=2, capacity=64, n_q_heads=4, n_kv_heads=2, head_dim=128).c()
         setattr(c, field, val)
         out = ctypes.c_uint64()
@@ -138,3 +139,21 @@ def test_validation_errors_are_returned_on_the_host():
     assert need.value == 1 * 128 * 256 * 2
     assert _rc("kvq_h_reconstruct", ctypes.byref(hc), ctypes.byref(hl), P(64), 10, P(128), P(256),
                64, P(512), ctypes.c_uint64(need.value - 16), None) == -5
+
+
+def test_window_config_validation_and_bytes():
+    # capacity must be n_anchor + window; the cache bytes are those of `capacity` slots
+    ok = Config(batch=2, capacity=1600, n_q_heads=4, n_kv_heads=2, head_dim=128, k_bits=4,
+                v_bits=8, k_group=32, v_group=128, window=1536, n_anchor=64)
+    plain = Config(batch=2, capacity=1600, n_q_heads=4, n_kv_heads=2, head_dim=128, k_bits=4,
+                   v_bits=8, k_group=32, v_group=128)
+    assert kvq.kvq_cache_bytes(ok) == kvq.kvq_cache_bytes(plain)
+    bad = Config(**{**ok.__dict__, "n_anchor": 63})
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.kvq_cache_bytes(bad)
+    assert e.value.status == -1
+    h = Config(batch=1, capacity=64, mode=kvq.KVQ_MODE_H, d_model=2048, h_bits=4, h_groups=16,
+               n_q_heads=16, n_kv_heads=16, head_dim=128, window=48, n_anchor=16)
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.kvq_cache_bytes(h)
+    assert e.value.status == -2
