@@ -416,6 +416,65 @@ def run_hmode(args, world, device):
     return res
 
 
+def run_window(args, world, device):
+    """Sliding-window workload: B=64 sequences that have seen 8192 tokens, each
+    caching 64 anchors + the 1536 most recent (1600 tokens), K4V8; a step of a few
+    layers, one kvq_append_decode_attn per layer (ring slot of the new token)."""
+    import torch
+    import quantized_kv_cache_22_b200 as kvq
+    from quantized_kv_cache_22_b200 import Config, LayerCache, Workspace, inputs
+
+    w = dataclasses.replace(inputs.WORKLOADS[6], n_layers=4)
+    kb, vb, kg, vg = w.kv_variants[0]
+    cfg = Config(batch=w.batch, capacity=w.capacity, n_q_heads=w.n_q_heads,
+                 n_kv_heads=w.n_kv_heads, head_dim=w.head_dim, k_bits=kb, v_bits=vb,
+                 k_group=kg, v_group=vg, n_layers=w.n_layers, window=w.window,
+                 n_anchor=w.n_anchor)
+    L = w.context                                  # tokens seen, the newest at L - 1
+    first_win = L - 1 - w.window                   # window tokens cached before the step
+    caches = []
+    for layer in range(w.n_layers):
+        c = LayerCache(cfg, device)
+        k, v = inputs.kv_tokens(w, layer, w.capacity, device)
+        kvq.kvq_append(cfg, c, k[:, :w.n_anchor].contiguous(), v[:, :w.n_anchor].contiguous(),
+                       torch.zeros(w.batch, dtype=torch.int32, device=device), 0, w.n_anchor)
+        kvq.kvq_append(cfg, c, k[:, w.n_anchor:].contiguous(), v[:, w.n_anchor:].contiguous(),
+                       torch.full((w.batch,), first_win, dtype=torch.int32, device=device),
+                       first_win, w.window)
+        del k, v
+        caches.append(c)
+    st = {"cfg": cfg, "caches": caches,
+          "d_len": torch.full((w.batch,), L, dtype=torch.int32, device=device),
+          "ws": Workspace(cfg, 0, device)}
+    kn, vn, qs = [], [], []
+    for layer in range(w.n_layers):
+        k1, v1 = inputs.kv_tokens(w, layer, 1, device, offset_seed=1)
+        kn.append(k1[:, 0])
+        vn.append(v1[:, 0])
+        qs.append(inputs.queries(w, layer, 0, device))
+    st["k_new"], st["v_new"], st["q"] = torch.stack(kn), torch.stack(vn), torch.stack(qs)
+    st["out"] = torch.empty_like(st["q"])
+    g, ge, ev_s, ev_e, _ = capture_step(w, st)
+    ms, _ = time_graph(g, max(3, min(args.steps, 100)), args.warmup, world, device)
+    for _ in range(args.warmup + 3):
+        ge.replay()
+    torch.cuda.synchronize()
+    dec_ms = reduce_max(statistics.mean(ev_s[i].elapsed_time(ev_e[i]) for i in range(w.n_layers)),
+                        world, device)
+    assert kvq.kvq_workspace_status(st["ws"]) == 0
+    per_layer = kvq.kvq_cache_bytes(cfg)[0] * w.batch * w.capacity
+    hbm_peak, peak_kind = measured_peaks()
+    gbs = per_layer / (dec_ms * 1e-3) / 1e9
+    return {"workload": w.name, "kv": "K4V8", "window": w.window, "n_anchor": w.n_anchor,
+            "tokens_seen": L, "tokens_attended": w.capacity, "layers_timed": w.n_layers,
+            "kv_bytes_per_layer": per_layer, "ms_per_layer": round(ms / w.n_layers, 5),
+            "kv_gbs": round(world * per_layer * w.n_layers / (ms * 1e-3) / 1e9, 1),
+            "roofline": {"bound": "hbm", "kernel": "decode_kernel (ring-slot append + attention "
+                         "+ merge)", "achieved": round(gbs, 1), "peak": hbm_peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": round(gbs / hbm_peak, 4),
+                         "launch_ms": round(dec_ms, 5)}}
+
+
 def run_gpu(args):
     import torch
     import quantized_kv_cache_22_b200 as kvq
@@ -480,9 +539,11 @@ def run_gpu(args):
             torch.cuda.empty_cache()
 
     hmode = run_hmode(args, world, device) if "hmode" in args.sections else None
+    window = run_window(args, world, device) if "window" in args.sections else None
     if not variants:
         if rank == 0:
-            print(json.dumps({"metric": METRIC, "value": None, "hmode": hmode}), flush=True)
+            print(json.dumps({"metric": METRIC, "value": None, "hmode": hmode, "window": window}),
+                  flush=True)
         return
     head = args.variants[0]
     r = results[head]
@@ -520,6 +581,7 @@ def run_gpu(args):
                      for k, v in results.items()},
         "gpu_launches": args.steps * w.n_layers,   # one decode-step kernel per layer
         "hmode": hmode,
+        "window": window,
         "clocks": r["clocks"],
     }
     if "e2e" in r:
@@ -590,8 +652,9 @@ def main():
     ap.add_argument("--variants", default="K8V8,K8V4,K4V4")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--sections", default="kv,hmode",
-                    help="kv: the 8K K/V decode step (headline); hmode: the h-mode workload")
+    ap.add_argument("--sections", default="kv,hmode,window",
+                    help="kv: the 8K K/V decode step (headline); hmode: the h-mode workload; "
+                         "window: the sliding-window workload")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the layer count (small profiling captures only)")
     ap.add_argument("--traffic-bytes", type=float, default=None,

@@ -27,6 +27,11 @@ Workloads (seed = 1000 + index):
   5 h-mode    B=8, S=1024, D=2048, 16 heads x 128; residual ~ N(0,1),
               h = LayerNorm(residual) without affine, eps 1e-5; W_k, W_v bf16
               ~ N(0, 1/D); INT4-h with 16 fp16 scales per token.
+  6 window    sliding-window cache (on-device page: 1536 recent tokens plus the
+              first 64 as anchors; INT4 keys, INT8 values; 24 query / 8 KV
+              heads x 128, 28 layers as the page's 3B model), B=64, 8192 tokens
+              seen, so 1600 cached tokens per sequence; fp16 ~ N(0,1); keys INT4
+              with 32-element groups, values INT8 per (token, head).
 """
 from __future__ import annotations
 
@@ -52,6 +57,8 @@ class Workload:
     outliers: int = 0     # key channels per (layer, kv head) scaled by outlier_scale
     outlier_scale: float = 10.0
     d_model: int = 0      # h-mode
+    window: int = 0       # sliding window (capacity = n_anchor + window)
+    n_anchor: int = 0
 
     @property
     def seed(self) -> int:
@@ -69,6 +76,8 @@ WORKLOADS = {
                 ((8, 8, 128, 128), (8, 4, 128, 128), (4, 4, 128, 128))),
     5: Workload("hmode-int4h-b8-s1k-d2048", 5, 8, 1, 16, 16, 128, 1024, 1024, torch.float16,
                 (), d_model=2048),
+    6: Workload("window-gqa24x8-b64-w1536a64-8k", 6, 64, 28, 24, 8, 128, 8192, 1600,
+                torch.float16, ((4, 8, 32, 128),), window=1536, n_anchor=64),
 }
 
 

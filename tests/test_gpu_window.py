@@ -125,3 +125,51 @@ def test_window_steps_across_the_wrap(cuda_device):
         vmax = vmax_per_batch(oc[2], oc[3], sub, [len(kept)])
         assert_close_to_oracle(out.cpu().numpy(), want, vmax, G, f"L={L}")
     assert kvq.kvq_workspace_status(ws) == 0
+
+
+def test_window_workload_full_size_sampled(cuda_device):
+    """Sliding-window workload at full size (B=64, 8 KV heads, 1536 + 64 slots, 8192
+    tokens seen, K4V8): one decode step, sampled (sequence, KV head) pairs checked."""
+    from quantized_kv_cache_22_b200 import inputs
+    w = inputs.WORKLOADS[6]
+    kb, vb, kg, vg = w.kv_variants[0]
+    cfg = Config(batch=w.batch, capacity=w.capacity, n_q_heads=w.n_q_heads,
+                 n_kv_heads=w.n_kv_heads, head_dim=w.head_dim, k_bits=kb, v_bits=vb,
+                 k_group=kg, v_group=vg, window=w.window, n_anchor=w.n_anchor)
+    L = w.context
+    first_win = L - 1 - w.window
+    k, v = inputs.kv_tokens(w, 0, w.capacity, "cuda")
+    cache = LayerCache(cfg)
+    kvq.kvq_append(cfg, cache, k[:, :w.n_anchor].contiguous(), v[:, :w.n_anchor].contiguous(),
+                   torch.zeros(w.batch, dtype=torch.int32, device="cuda"), 0, w.n_anchor)
+    kvq.kvq_append(cfg, cache, k[:, w.n_anchor:].contiguous(), v[:, w.n_anchor:].contiguous(),
+                   torch.full((w.batch,), first_win, dtype=torch.int32, device="cuda"),
+                   first_win, w.window)
+    k1, v1 = inputs.kv_tokens(w, 0, 1, "cuda", offset_seed=1)
+    q = inputs.queries(w, 0, 0, "cuda")
+    d_len = torch.full((w.batch,), L, dtype=torch.int32, device="cuda")
+    out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    ws = Workspace(cfg)
+    kvq.kvq_append_decode_attn(cfg, cache, k1[:, 0].contiguous(), v1[:, 0].contiguous(), q, d_len,
+                               L, out, ws)
+    torch.cuda.synchronize()
+    assert kvq.kvq_workspace_status(ws) == 0
+    # logical tokens now cached: anchors 0..63, positions first_win+1 .. L-1 (the
+    # token at first_win shared its slot with the newest one)
+    kept_k = torch.cat([k[:, :w.n_anchor], k[:, w.n_anchor + 1:], k1], 1).cpu()
+    kept_v = torch.cat([v[:, :w.n_anchor], v[:, w.n_anchor + 1:], v1], 1).cpu()
+    positions = list(range(w.n_anchor)) + list(range(first_win + 1, L))
+    slots = [_slot(t) for t in positions]
+    gc = read_gpu_cache(cache, cfg)
+    G = w.n_q_heads // w.n_kv_heads
+    got = out.cpu().numpy()
+    for (b, kvh) in ((0, 0), (31, 5), (63, 7)):
+        sub = Config(**{**cfg.__dict__, "batch": 1, "n_kv_heads": 1, "n_q_heads": G,
+                        "window": 0, "n_anchor": 0})
+        oc = oracle_cache(kept_k[b:b + 1, :, kvh:kvh + 1], kept_v[b:b + 1, :, kvh:kvh + 1], sub)
+        for i in range(4):
+            assert np.array_equal(gc[i][b, kvh][slots], oc[i][0, 0]), (b, kvh, i)
+        qq = q[b:b + 1, kvh * G:(kvh + 1) * G].cpu()
+        want = oracle_decode(sub, oc, qq, [w.capacity])
+        vmax = vmax_per_batch(oc[2], oc[3], sub, [w.capacity])
+        assert_close_to_oracle(got[b:b + 1, kvh * G:(kvh + 1) * G], want, vmax, G, f"{(b, kvh)}")
