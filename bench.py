@@ -475,6 +475,63 @@ def run_window(args, world, device):
                          "launch_ms": round(dec_ms, 5)}}
 
 
+def run_paged(args, world, device):
+    """Paged layout of the 8K workload: each layer's cache is a pool of 1024 pages of
+    128 tokens (16 sequences x 64 pages, shuffled by a seeded permutation) behind a
+    block table; a step of four layers, one kvq_append_decode_attn per layer."""
+    import torch
+    import quantized_kv_cache_22_b200 as kvq
+    from quantized_kv_cache_22_b200 import Config, LayerCache, Workspace, inputs
+
+    w = dataclasses.replace(inputs.WORKLOADS[4], n_layers=4)
+    kb, vb, kg, vg = VARIANTS["K8V8"]
+    pages = w.batch * (w.capacity // 128)
+    cfg = Config(batch=w.batch, capacity=w.capacity, n_q_heads=w.n_q_heads,
+                 n_kv_heads=w.n_kv_heads, head_dim=w.head_dim, k_bits=kb, v_bits=vb,
+                 k_group=kg, v_group=vg, n_layers=w.n_layers, page_tokens=128, n_pages=pages)
+    g = torch.Generator().manual_seed(w.seed)
+    table = torch.randperm(pages, generator=g).view(w.batch, -1).to(torch.int32).to(device)
+    L = w.context
+    caches = []
+    for layer in range(w.n_layers):
+        c = LayerCache(cfg, device, block_table=table)
+        k, v = inputs.kv_tokens(w, layer, L - 1, device)
+        kvq.kvq_append(cfg, c, k, v, torch.zeros(w.batch, dtype=torch.int32, device=device), 0,
+                       L - 1)
+        del k, v
+        caches.append(c)
+    st = {"cfg": cfg, "caches": caches,
+          "d_len": torch.full((w.batch,), L, dtype=torch.int32, device=device),
+          "ws": Workspace(cfg, 0, device)}
+    kn, vn, qs = [], [], []
+    for layer in range(w.n_layers):
+        k1, v1 = inputs.kv_tokens(w, layer, 1, device, offset_seed=1)
+        kn.append(k1[:, 0])
+        vn.append(v1[:, 0])
+        qs.append(inputs.queries(w, layer, 0, device))
+    st["k_new"], st["v_new"], st["q"] = torch.stack(kn), torch.stack(vn), torch.stack(qs)
+    st["out"] = torch.empty_like(st["q"])
+    g, ge, ev_s, ev_e, _ = capture_step(w, st)
+    ms, _ = time_graph(g, max(3, min(args.steps, 100)), args.warmup, world, device)
+    for _ in range(args.warmup + 3):
+        ge.replay()
+    torch.cuda.synchronize()
+    dec_ms = reduce_max(statistics.mean(ev_s[i].elapsed_time(ev_e[i]) for i in range(w.n_layers)),
+                        world, device)
+    assert kvq.kvq_workspace_status(st["ws"]) == 0
+    per_layer = kvq.kvq_cache_bytes(cfg)[0] * w.batch * w.context
+    hbm_peak, peak_kind = measured_peaks()
+    gbs = per_layer / (dec_ms * 1e-3) / 1e9
+    return {"workload": w.name + "-paged128", "kv": "K8V8", "page_tokens": 128, "pages": pages,
+            "layers_timed": w.n_layers, "kv_bytes_per_layer": per_layer,
+            "ms_per_layer": round(ms / w.n_layers, 5),
+            "kv_gbs": round(world * per_layer * w.n_layers / (ms * 1e-3) / 1e9, 1),
+            "roofline": {"bound": "hbm", "kernel": "decode_kernel (paged: block-table tiles)",
+                         "achieved": round(gbs, 1), "peak": hbm_peak, "peak_kind": peak_kind,
+                         "unit": "GB/s", "frac": round(gbs / hbm_peak, 4),
+                         "launch_ms": round(dec_ms, 5)}}
+
+
 def run_gpu(args):
     import torch
     import quantized_kv_cache_22_b200 as kvq
@@ -540,10 +597,11 @@ def run_gpu(args):
 
     hmode = run_hmode(args, world, device) if "hmode" in args.sections else None
     window = run_window(args, world, device) if "window" in args.sections else None
+    paged = run_paged(args, world, device) if "paged" in args.sections else None
     if not variants:
         if rank == 0:
-            print(json.dumps({"metric": METRIC, "value": None, "hmode": hmode, "window": window}),
-                  flush=True)
+            print(json.dumps({"metric": METRIC, "value": None, "hmode": hmode, "window": window,
+                              "paged": paged}), flush=True)
         return
     head = args.variants[0]
     r = results[head]
@@ -582,6 +640,7 @@ def run_gpu(args):
         "gpu_launches": args.steps * w.n_layers,   # one decode-step kernel per layer
         "hmode": hmode,
         "window": window,
+        "paged": paged,
         "clocks": r["clocks"],
     }
     if "e2e" in r:
@@ -652,9 +711,9 @@ def main():
     ap.add_argument("--variants", default="K8V8,K8V4,K4V4")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--sections", default="kv,hmode,window",
+    ap.add_argument("--sections", default="kv,hmode,window,paged",
                     help="kv: the 8K K/V decode step (headline); hmode: the h-mode workload; "
-                         "window: the sliding-window workload")
+                         "window: the sliding-window workload; paged: the 8K step on a paged cache")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the layer count (small profiling captures only)")
     ap.add_argument("--traffic-bytes", type=float, default=None,

@@ -109,12 +109,23 @@ typedef struct kvq_config {
                             t while t < n_anchor, else in slot n_anchor +
                             (t - n_anchor) mod window.  0: no window, slot t.     */
     int32_t n_anchor;    /* KV mode with a window: anchor tokens kept for good    */
+    int32_t page_tokens; /* KV mode: 0 (each sequence owns `capacity` contiguous
+                            slots) or 128: paged cache.  The layer's buffers are a
+                            pool of n_pages pages of 128 tokens, [n_pages][Hkv]
+                            [128][...], and kvq_layer.block_table maps logical page
+                            j of sequence b (tokens 128j .. 128j+127) to a pool
+                            page; capacity (a multiple of 128) is then the
+                            logical tokens per sequence.  No sliding window.      */
+    int32_t n_pages;     /* paged cache: pages in each layer's pool               */
 } kvq_config;
 
 /* One layer's cache buffers (device pointers, caller-owned).
  * KV mode:  k_codes  [B][Hkv][capacity][Dh*k_bits/8] bytes
  *           k_scales [B][Hkv][capacity][Dh/k_group] fp16   (NULL at 16 bits)
  *           v_codes / v_scales likewise with v_bits, v_group.
+ *           Paged (page_tokens 128): [n_pages][Hkv][128][...] for each of them,
+ *           logical token t of sequence b at slot t % 128 of pool page
+ *           block_table[b][t / 128].
  * h-mode:   k_codes  [B][capacity][D*h_bits/8] bytes  (the h codes)
  *           k_scales [B][capacity][h_groups] fp16      (NULL at 16 bits)
  *           v_codes = v_scales = NULL. */
@@ -123,6 +134,10 @@ typedef struct kvq_layer {
     void *k_scales;
     void *v_codes;
     void *v_scales;
+    const int32_t *block_table;  /* paged cache: device int32 [B][capacity/128], the
+                                    pool page of each logical page (entries in
+                                    [0, n_pages)); NULL otherwise.  The same table
+                                    usually serves every layer. */
 } kvq_layer;
 
 /* Cache size.  [TL] "記憶體公式": bytes per token per layer are, at
@@ -133,8 +148,9 @@ typedef struct kvq_layer {
  *   KV mode: sum over K and V of Hkv*Dh*bits/8 + Hkv*(Dh/group)*2 (no scale
  *            term at 16 bits);   h-mode: D*h_bits/8 + h_groups*2 (none at 16).
  * Outputs (any may be NULL): bytes per token per layer, per layer
- * (x batch x capacity) and total (x n_layers).  Pure host function: no GPU
- * needed.  Errors: KVQ_ERR_INVALID_ARG / KVQ_ERR_UNSUPPORTED for a bad config. */
+ * (x batch x capacity, or x n_pages x 128 for a paged cache) and total
+ * (x n_layers).  Pure host function: no GPU needed.  Errors:
+ * KVQ_ERR_INVALID_ARG / KVQ_ERR_UNSUPPORTED for a bad config. */
 KVQ_API int kvq_cache_bytes(const kvq_config *cfg, uint64_t *per_token_layer, uint64_t *per_layer,
                     uint64_t *total);
 

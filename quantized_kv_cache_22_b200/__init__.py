@@ -39,12 +39,13 @@ class KvqConfig(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "mode", "batch", "capacity", "n_layers", "n_q_heads", "n_kv_heads", "head_dim",
         "k_bits", "v_bits", "k_group", "v_group", "d_model", "h_bits", "h_groups",
-        "window", "n_anchor")]
+        "window", "n_anchor", "page_tokens", "n_pages")]
 
 
 class KvqLayer(ctypes.Structure):
     _fields_ = [("k_codes", ctypes.c_void_p), ("k_scales", ctypes.c_void_p),
-                ("v_codes", ctypes.c_void_p), ("v_scales", ctypes.c_void_p)]
+                ("v_codes", ctypes.c_void_p), ("v_scales", ctypes.c_void_p),
+                ("block_table", ctypes.c_void_p)]
 
 
 def _load():
@@ -139,12 +140,15 @@ class Config:
     h_groups: int = 0
     window: int = 0       # sliding window: ring of recent tokens (capacity = n_anchor + window)
     n_anchor: int = 0     # tokens kept at the start of the sequence
+    page_tokens: int = 0  # 128: paged cache (a pool of n_pages pages, block table per layer)
+    n_pages: int = 0
 
     def _key(self):
         return (self.mode, self.batch, self.capacity, self.n_layers, self.n_q_heads,
                 self.n_kv_heads, self.head_dim, self.k_bits, self.v_bits,
                 self.k_group or self.head_dim, self.v_group or self.head_dim,
-                self.d_model, self.h_bits, self.h_groups, self.window, self.n_anchor)
+                self.d_model, self.h_bits, self.h_groups, self.window, self.n_anchor,
+                self.page_tokens, self.n_pages)
 
     def c(self) -> KvqConfig:
         """A new ``kvq_config`` struct with these fields."""
@@ -195,9 +199,13 @@ def kvq_h_scratch_bytes(cfg: Config, max_len: int) -> int:
 # ----------------------------------------------------------------------------- device buffers
 
 class LayerCache:
-    """One layer's cache buffers, allocated with torch on `device` (caller-owned memory)."""
+    """One layer's cache buffers, allocated with torch on `device` (caller-owned memory).
+    A paged config allocates the page pool; `block_table` (int32 [B][capacity/128] on
+    the device) then maps each sequence's logical pages to pool pages."""
 
-    def __init__(self, cfg: Config, device="cuda", zero: bool = False):
+    block_table = None
+
+    def __init__(self, cfg: Config, device="cuda", zero: bool = False, block_table=None):
         kc, ks, vc, vs = kvq_layer_buffer_bytes(cfg)
         alloc = torch.zeros if zero else torch.empty
         self.k_codes = alloc(max(kc, 16), dtype=torch.uint8, device=device)
@@ -205,15 +213,17 @@ class LayerCache:
         self.v_codes = alloc(max(vc, 16), dtype=torch.uint8, device=device) if vc else None
         self.v_scales = alloc(max(vs // 2, 8), dtype=torch.float16, device=device) if vs else None
         self.cfg = cfg
+        self.block_table = block_table
 
     def c(self) -> KvqLayer:
         """A new ``kvq_layer`` struct with these buffers."""
         return KvqLayer(*(None if t is None else t.data_ptr()
-                          for t in (self.k_codes, self.k_scales, self.v_codes, self.v_scales)))
+                          for t in (self.k_codes, self.k_scales, self.v_codes, self.v_scales,
+                                    self.block_table)))
 
     def _ref(self):
         """byref() of a struct kept for these buffers (read-only use by the wrappers)."""
-        ts = (self.k_codes, self.k_scales, self.v_codes, self.v_scales)
+        ts = (self.k_codes, self.k_scales, self.v_codes, self.v_scales, self.block_table)
         memo = self.__dict__.get("_c_memo")
         if memo is None or any(a is not b for a, b in zip(memo[0], ts)):
             c = self.c()

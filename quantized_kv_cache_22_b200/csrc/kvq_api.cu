@@ -54,8 +54,16 @@ int check_cfg(const kvq_config *c)
         if (c->window == 0 && c->n_anchor != 0) return KVQ_ERR_INVALID_ARG;
         if (c->window > 0 && (int64_t)c->n_anchor + c->window != c->capacity)
             return KVQ_ERR_INVALID_ARG;
+        if (c->page_tokens != 0) {
+            if (c->page_tokens != kPageTokens) return KVQ_ERR_UNSUPPORTED;
+            if (c->window != 0) return KVQ_ERR_UNSUPPORTED;
+            if (c->n_pages < 1 || c->capacity % kPageTokens != 0) return KVQ_ERR_INVALID_ARG;
+        } else if (c->n_pages != 0) {
+            return KVQ_ERR_INVALID_ARG;
+        }
     } else {
-        if (c->window != 0 || c->n_anchor != 0) return KVQ_ERR_UNSUPPORTED;
+        if (c->window != 0 || c->n_anchor != 0 || c->page_tokens != 0 || c->n_pages != 0)
+            return KVQ_ERR_UNSUPPORTED;
         if (c->d_model < 128 || c->d_model % 128 != 0) return KVQ_ERR_UNSUPPORTED;
         if (!valid_bits(c->h_bits)) return KVQ_ERR_UNSUPPORTED;
         if (c->h_bits != 16) {
@@ -287,7 +295,9 @@ int kvq_cache_bytes(const kvq_config *cfg, uint64_t *per_token_layer, uint64_t *
         b = tensor_row_bytes(cfg->d_model, cfg->h_bits);
         if (cfg->h_bits != 16) b += (uint64_t)cfg->h_groups * 2;
     }
-    const uint64_t layer = b * (uint64_t)cfg->batch * (uint64_t)cfg->capacity;
+    const uint64_t slots = cfg->page_tokens ? (uint64_t)cfg->n_pages * kPageTokens
+                                            : (uint64_t)cfg->batch * (uint64_t)cfg->capacity;
+    const uint64_t layer = b * slots;
     if (per_token_layer) *per_token_layer = b;
     if (per_layer) *per_layer = layer;
     if (total) *total = layer * (uint64_t)cfg->n_layers;
@@ -299,7 +309,8 @@ int kvq_layer_buffer_bytes(const kvq_config *cfg, uint64_t *k_codes, uint64_t *k
 {
     int rc = check_cfg(cfg);
     if (rc) return rc;
-    const uint64_t rows = (uint64_t)cfg->batch * cfg->capacity;
+    const uint64_t rows = cfg->page_tokens ? (uint64_t)cfg->n_pages * kPageTokens
+                                           : (uint64_t)cfg->batch * cfg->capacity;
     uint64_t kc, ks, vc = 0, vs = 0;
     if (cfg->mode == KVQ_MODE_KV) {
         const uint64_t hr = rows * cfg->n_kv_heads;
@@ -333,6 +344,12 @@ int kvq_append(const kvq_config *cfg, const kvq_layer *layer, const void *k, con
     AppendParams pk{};
     pk.window = cfg->window;
     pk.n_anchor = cfg->n_anchor;
+    if (cfg->mode == KVQ_MODE_KV && cfg->page_tokens) {
+        if (!layer->block_table) return KVQ_ERR_INVALID_ARG;
+        pk.block_table = layer->block_table;
+        pk.max_pages = cfg->capacity / kPageTokens;
+        pk.n_pages = cfg->n_pages;
+    }
     pk.in_dtype = in_dtype;
     pk.batch = cfg->batch;
     pk.n_new = n_new;
@@ -434,7 +451,8 @@ static int decode_kv_layout(const kvq_config *cfg, const void *k_codes, const vo
                             int32_t q_dtype, const int32_t *d_len, float softmax_scale, void *out,
                             int32_t out_dtype, void *workspace, uint64_t workspace_bytes,
                             int32_t num_ctas, cudaStream_t stream, bool do_partials, bool do_merge,
-                            const FusedAppend *app = nullptr)
+                            const FusedAppend *app = nullptr,
+                            const int32_t *block_table = nullptr)
 {
     const AttnShape a = attn_shape(cfg);
     // fp16 keys use an f16 MMA whose f32 / bf16 queries take two columns per head
@@ -449,9 +467,11 @@ static int decode_kv_layout(const kvq_config *cfg, const void *k_codes, const vo
 
     if (do_partials) {
         CUtensorMap tm_k, tm_v;
-        const int bh = cfg->batch * a.hkv;
-        if (!encode_codes_map(&tm_k, k_codes, bh, cap, a.dh * a.kb / 8) ||
-            !encode_codes_map(&tm_v, v_codes, bh, cap, a.dh * a.vb / 8))
+        // contiguous: [B*Hkv][cap] rows; paged: the pool, [n_pages*Hkv][128] rows
+        const int zdim = block_table ? cfg->n_pages * a.hkv : cfg->batch * a.hkv;
+        const int ydim = block_table ? kPageTokens : cap;
+        if (!encode_codes_map(&tm_k, k_codes, zdim, ydim, a.dh * a.kb / 8) ||
+            !encode_codes_map(&tm_v, v_codes, zdim, ydim, a.dh * a.vb / 8))
             return fail("tensor map encode", cudaErrorInvalidValue);
         DecodeParams p{};
         p.d_len = d_len;
@@ -488,6 +508,9 @@ static int decode_kv_layout(const kvq_config *cfg, const void *k_codes, const vo
         if (app) p.app = *app;
         p.window = cfg->mode == KVQ_MODE_KV ? cfg->window : 0;
         p.n_anchor = cfg->mode == KVQ_MODE_KV ? cfg->n_anchor : 0;
+        p.block_table = block_table;
+        p.max_pages = block_table ? cap / kPageTokens : 0;
+        p.n_pages = block_table ? cfg->n_pages : 0;
         cudaError_t e = launch_decode(plan, p, tm_k, tm_v, stream);
         if (e != cudaSuccess) return fail("decode launch", e);
         return KVQ_OK;
@@ -514,6 +537,7 @@ static int decode_kv_layout(const kvq_config *cfg, const void *k_codes, const vo
 static int check_kv_layer(const kvq_config *cfg, const kvq_layer *layer)
 {
     if (!layer->k_codes || !layer->v_codes) return KVQ_ERR_INVALID_ARG;
+    if (cfg->page_tokens && !layer->block_table) return KVQ_ERR_INVALID_ARG;
     if ((cfg->k_bits != 16 && !layer->k_scales) || (cfg->v_bits != 16 && !layer->v_scales))
         return KVQ_ERR_INVALID_ARG;
     if (!aligned16(layer->k_codes) || !aligned16(layer->v_codes) ||
@@ -541,7 +565,8 @@ int kvq_decode_partials(const kvq_config *cfg, const kvq_layer *layer, const voi
     return decode_kv_layout(cfg, layer->k_codes, layer->k_scales, layer->v_codes, layer->v_scales,
                             cfg->capacity, q, q_dtype, d_len, softmax_scale, nullptr, KVQ_F32,
                             workspace, workspace_bytes, num_ctas,
-                            reinterpret_cast<cudaStream_t>(stream), true, false);
+                            reinterpret_cast<cudaStream_t>(stream), true, false, nullptr,
+                            cfg->page_tokens ? layer->block_table : nullptr);
 }
 
 int kvq_merge_partials(const kvq_config *cfg, const int32_t *d_len, void *out, int32_t out_dtype,
@@ -627,7 +652,7 @@ int kvq_decode_attn(const kvq_config *cfg, const kvq_layer *layer, const void *q
         return decode_kv_layout(cfg, layer->k_codes, layer->k_scales, layer->v_codes,
                                 layer->v_scales, cfg->capacity, q, q_dtype, d_len, softmax_scale,
                                 out, out_dtype, workspace, workspace_bytes, num_ctas, st, true,
-                                true);
+                                true, nullptr, cfg->page_tokens ? layer->block_table : nullptr);
     }
 
     // h-mode: rebuild K, V into the scratch, then attend over 16-bit K/V.
@@ -694,7 +719,8 @@ int kvq_append_decode_attn(const kvq_config *cfg, const kvq_layer *layer, const 
     return decode_kv_layout(cfg, layer->k_codes, layer->k_scales, layer->v_codes, layer->v_scales,
                             cfg->capacity, q, q_dtype, d_len, softmax_scale, out, out_dtype,
                             workspace, workspace_bytes, num_ctas,
-                            reinterpret_cast<cudaStream_t>(stream), true, true, &app);
+                            reinterpret_cast<cudaStream_t>(stream), true, true, &app,
+                            cfg->page_tokens ? layer->block_table : nullptr);
 }
 
 int kvq_h_reconstruct(const kvq_config *cfg, const kvq_layer *layer, const void *w_kv,

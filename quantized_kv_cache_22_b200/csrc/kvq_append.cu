@@ -4,7 +4,8 @@
 // vector) with the row quantiser of kvq_quant.cuh (TinyLoop docs "KV Cache
 // 模式" modes table; KVSplit independent key/value widths and groups).  With a
 // sliding window (on-device page, "Sliding Window Eviction": recent tokens
-// plus anchors) a token goes to its ring slot.
+// plus anchors) a token goes to its ring slot; in a paged cache to its slot of
+// the pool page the block table names.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -41,10 +42,18 @@ __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ App
         if (pos >= p.n_anchor && pos + p.window <= first + p.n_new - 1) return;
         slot = cache_slot(pos, p.window, p.n_anchor);
     }
-    if (slot >= p.cap) return;  // the kernel's own bounds check
+    if (slot >= p.cap) return;  // the kernel's own bounds checks
 
     const int dim = p.dim;
-    const int64_t cache_row = ((int64_t)b * p.rows_per_tok + head) * p.cap + slot;
+    int64_t cache_row;
+    if (p.block_table != nullptr) {
+        // paged: slot pos % 128 of the pool page holding logical page pos / 128
+        const int page = p.block_table[(int64_t)b * p.max_pages + pos / kPageTokens];
+        if (page < 0 || page >= p.n_pages) return;
+        cache_row = ((int64_t)page * p.rows_per_tok + head) * kPageTokens + pos % kPageTokens;
+    } else {
+        cache_row = ((int64_t)b * p.rows_per_tok + head) * p.cap + slot;
+    }
     uint8_t *codes_row = p.codes + cache_row * ((int64_t)dim * p.bits / 8);
     __half *scales_row = p.bits == 16 ? nullptr : p.scales + cache_row * (dim / p.group);
     quantize_row(p.x, row * (int64_t)dim, p.in_dtype, dim, p.bits, p.group, codes_row, scales_row,

@@ -444,7 +444,13 @@ __global__ void __launch_bounds__(NTHR, 2)
         };
         auto do_app = [&]() {
             const int bh = ab * Hkv + akvh;
-            const int64_t crow = (int64_t)bh * cap + aslot;
+            int64_t crow = (int64_t)bh * cap + aslot;
+            if (p.block_table != nullptr) {
+                // paged: the pool page of the newest token's logical page
+                int page = p.block_table[(int64_t)ab * p.max_pages + aslot / T];
+                page = min(max(page, 0), p.n_pages - 1);
+                crow = ((int64_t)page * Hkv + akvh) * T + aslot % T;
+            }
             quantize_row(p.app.k_new, (int64_t)bh * DH, p.app.dtype, DH, KB, p.app.k_group,
                          p.app.k_codes + crow * RK,
                          KB == 16 ? nullptr : p.app.k_scales + crow * (DH / p.app.k_group), lane);
@@ -501,29 +507,39 @@ __global__ void __launch_bounds__(NTHR, 2)
                 m.ncta = seg_ncta; m.cmin = seg_cmin; m.pad = 0;
                 meta[s] = m;
 
+                // physical tile: (bh, t0) of the contiguous layout, or the pool
+                // page the block table names (whole page, row 0) in a paged one
+                int z = bh, y0 = t0, zcap = cap;
+                if (p.block_table != nullptr) {
+                    int page = p.block_table[(int64_t)b * p.max_pages + tile];
+                    page = min(max(page, 0), p.n_pages - 1);   // stay inside the pool
+                    z = page * Hkv + kvh;
+                    y0 = 0;
+                    zcap = T;
+                }
                 uint8_t *st = smem + (size_t)s * p.stage_bytes;
-                const int n_s = min(T, cap - t0);
+                const int n_s = min(T, zcap - y0);
                 uint32_t bytes = (uint32_t)(T * RK + T * RV);
                 if (KB != 16) bytes += (uint32_t)(n_s * p.ngs_k * 2);
                 if (VB != 16) bytes += (uint32_t)(n_s * p.ngs_v * 2);
                 mbar_arrive_expect_tx(&full[s], bytes);
                 if constexpr (RK <= 128) {
-                    tma_load_3d_hint(st, &tm_k, &full[s], 0, t0 / (128 / RK), bh, pol);
+                    tma_load_3d_hint(st, &tm_k, &full[s], 0, y0 / (128 / RK), z, pol);
                 } else {
-                    tma_load_3d_hint(st, &tm_k, &full[s], 0, t0, bh, pol);
-                    tma_load_3d_hint(st + T * 128, &tm_k, &full[s], 128, t0, bh, pol);
+                    tma_load_3d_hint(st, &tm_k, &full[s], 0, y0, z, pol);
+                    tma_load_3d_hint(st + T * 128, &tm_k, &full[s], 128, y0, z, pol);
                 }
                 if constexpr (RV <= 128) {
-                    tma_load_3d_hint(st + p.off_v, &tm_v, &full[s], 0, t0 / (128 / RV), bh, pol);
+                    tma_load_3d_hint(st + p.off_v, &tm_v, &full[s], 0, y0 / (128 / RV), z, pol);
                 } else {
-                    tma_load_3d_hint(st + p.off_v, &tm_v, &full[s], 0, t0, bh, pol);
-                    tma_load_3d_hint(st + p.off_v + T * 128, &tm_v, &full[s], 128, t0, bh, pol);
+                    tma_load_3d_hint(st + p.off_v, &tm_v, &full[s], 0, y0, z, pol);
+                    tma_load_3d_hint(st + p.off_v + T * 128, &tm_v, &full[s], 128, y0, z, pol);
                 }
                 if (KB != 16)
-                    bulk_load_hint(st + p.off_sk, p.k_scales + ((int64_t)bh * cap + t0) * p.ngs_k,
+                    bulk_load_hint(st + p.off_sk, p.k_scales + ((int64_t)z * zcap + y0) * p.ngs_k,
                                    (uint32_t)(n_s * p.ngs_k * 2), &full[s], pol);
                 if (VB != 16)
-                    bulk_load_hint(st + p.off_sv, p.v_scales + ((int64_t)bh * cap + t0) * p.ngs_v,
+                    bulk_load_hint(st + p.off_sv, p.v_scales + ((int64_t)z * zcap + y0) * p.ngs_v,
                                    (uint32_t)(n_s * p.ngs_v * 2), &full[s], pol);
             }
             issued = i + 1;

@@ -17,7 +17,11 @@ struct AppendParams {
     int32_t batch, n_new, rows_per_tok, dim, cap;
     int32_t bits, group;
     int32_t window, n_anchor;   // sliding window (0: slot = position)
+    const int32_t *block_table; // paged cache: [batch][max_pages] pool page of each logical page
+    int32_t max_pages, n_pages; // (rows_per_tok is the KV heads; pages hold kPageTokens rows)
 };
+
+constexpr int kPageTokens = 128;   // tokens per page of a paged cache (one decode tile)
 
 // Cache slot of token position t: the first n_anchor tokens stay put, the rest
 // share a ring of `window` slots (window 0: no ring, slot t).
@@ -34,6 +38,7 @@ constexpr int kDecodeConsumerWarps = 4;
 constexpr int kDecodeTileTokens = 32 * kDecodeConsumerWarps;   // tokens per stage (32 per warp)
 // consumer warps, one producer warp, one combiner warp
 constexpr int kDecodeThreads = 32 * (kDecodeConsumerWarps + 2);
+static_assert(kPageTokens == kDecodeTileTokens, "a decode tile is one page of a paged cache");
 constexpr int kWorkspaceHeaderFloats = 64;                      // status word + padding
 
 // The new token's K/V for the append step fused into the decode kernel.
@@ -66,6 +71,8 @@ struct DecodeParams {
     uint64_t timeout_ns;
     FusedAppend app;
     int32_t window, n_anchor;  // sliding window: slot of the newest token (fused append)
+    const int32_t *block_table;  // paged cache (null: contiguous per sequence)
+    int32_t max_pages, n_pages;
 };
 
 struct MergeParams {

@@ -157,3 +157,28 @@ def test_window_config_validation_and_bytes():
     with pytest.raises(kvq.KvqError) as e:
         kvq.kvq_cache_bytes(h)
     assert e.value.status == -2
+
+
+def test_paged_config_validation_and_bytes():
+    base = dict(batch=3, capacity=1024, n_q_heads=8, n_kv_heads=2, head_dim=128, k_bits=8,
+                v_bits=4, k_group=128, v_group=32)
+    paged = Config(**base, page_tokens=128, n_pages=30)
+    per_tok = kvq.kvq_cache_bytes(Config(**base))[0]
+    t, layer, _ = kvq.kvq_cache_bytes(paged)
+    assert t == per_tok and layer == per_tok * 30 * 128
+    kc, ks, vc, vs = kvq.kvq_layer_buffer_bytes(paged)
+    assert kc == 30 * 2 * 128 * 128 and ks == 30 * 2 * 128 * 2
+    assert vc == 30 * 2 * 128 * 64 and vs == 30 * 2 * 128 * 4 * 2
+    for over, want in (({"page_tokens": 64}, -2), ({"n_pages": 0}, -1), ({"capacity": 1040}, -1),
+                       ({"window": 896, "n_anchor": 128}, -2)):
+        with pytest.raises(kvq.KvqError) as e:
+            kvq.kvq_cache_bytes(Config(**{**paged.__dict__, **over}))
+        assert e.value.status == want, over
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.kvq_cache_bytes(Config(**base, n_pages=4))
+    assert e.value.status == -1
+    # a paged layer without a block table is rejected before anything runs
+    lay = KvqLayer(16, 16, 32, 48, None)
+    P = ctypes.c_void_p
+    assert _rc("kvq_append", ctypes.byref(paged.c()), ctypes.byref(lay), P(16), P(32), 0, P(64),
+               0, 1, None) == -1
