@@ -93,10 +93,22 @@ __host__ __device__ constexpr uint32_t sw_off(int t, int o)
 }
 
 // Token of row g (g < 8) of a 16-token sub-tile's score tile; row g + 8 holds
-// the next token.  The permutation pi(g) = g ^ (g >> 2) keeps both the key-row
-// reads of the score MMA and the value-row reads of the P.V MMA (whose k
-// order follows the score rows through the transpose) free of bank conflicts.
-__host__ __device__ constexpr int row_token(int g) { return 2 * (g ^ (g >> 2)); }
+// the next token.  The permutation pi keeps the key-row reads of the score MMA
+// and the value-row reads of the P.V MMA (whose k order follows the score rows
+// through the transpose) free of shared-memory bank conflicts under the 128-byte
+// swizzle (checked against a model of the banks for every head_dim-128
+// format): pi(g) = g ^ (g >> 2) when keys are read 4 or 8 bytes per row and
+// block, and pi = (0, 6, 2, 4, 5, 3, 7, 1) when they are read 16 bytes per row
+// (KW), which also needs the two rows of each quarter-warp in different halves
+// of the bank space.
+template <bool KW>
+__host__ __device__ constexpr int row_token(int g)
+{
+    if constexpr (KW)
+        return 2 * (int)((0x17354260u >> (4 * g)) & 7u);
+    else
+        return 2 * (g ^ (g >> 2));
+}
 
 __device__ __forceinline__ float load_qf(const void *q, int dtype, int64_t idx)
 {
@@ -291,6 +303,20 @@ __global__ void __launch_bounds__(NTHR, 2)
     constexpr int SK = 32 * KB / 8;            // bytes per 32-element block of a key row
     constexpr int SV = 32 * VB / 8;
     constexpr int NVG = VG ? NG : 1;           // value-scale groups tracked per token
+    // Value fragments: with one value scale per (token, head) a lane reads 8
+    // consecutive head_dim elements of a row per 64-element half ("wide": one
+    // load feeds four m-tiles); grouped value scales need one P per 32-element
+    // block, so a lane then reads 4 elements per block.  Rows of 32 bytes (Dh 64
+    // at 4 bits) keep the block mapping, which stays free of bank conflicts.
+    constexpr bool VWIDE = !VG && RV >= 64;
+    constexpr int VL = VWIDE ? 2 * SV / 8 : SV / 8;   // value bytes per lane per row and load
+    // Key fragments: with one key scale per (token, head), int8 keys are read 16
+    // bytes per lane and row ("wide": 2 blocks of 32 elements per load at 8
+    // bits, 4 at 4 bits); an int8 MMA block must share one key scale, so
+    // grouped key scales keep one load per block.
+    constexpr bool KWIDE = !KG && KB != 16 && RK >= 64;
+    constexpr int KLW = KWIDE ? 16 : SK / 4;          // key bytes per lane per row and load
+    constexpr int KPL = KWIDE ? 16 * 8 / KB / 8 : 1;  // 32-element blocks per load
     constexpr float BIAS_V = VB == 8 ? 1152.f : 0.f;   // 4-bit values: per row, see the segment end
     // The running max is only raised when a tile beats it by more than 2^LAZY;
     // weights p * s_V then stay below 2^LAZY, well inside fp16.
@@ -341,7 +367,7 @@ __global__ void __launch_bounds__(NTHR, 2)
 
     // ---- work range of this CTA (computed by the producer warp) -------------
     __shared__ long long sh_u_begin, sh_n, sh_pe;
-    __shared__ int sh_b;
+    __shared__ int sh_b, sh_bh0;   // first sequence, and first (sequence, KV head), of the range
     if (warp == NW) {
         long long total = 0;
         for (int b = lane; b < p.batch; b += 32) total += tiles_of(p.d_len[b], cap);
@@ -356,7 +382,7 @@ __global__ void __launch_bounds__(NTHR, 2)
         // locate the sequence holding unit ub
         long long acc = 0;
         int fb = -1;
-        long long fpre = 0;
+        long long fpre = 0, funits = 0;
         for (int base = 0; base < p.batch && fb < 0 && ue > ub; base += 32) {
             const int b = base + lane;
             const long long units = (b < p.batch) ? (long long)tiles_of(p.d_len[b], cap) * Hkv : 0;
@@ -372,6 +398,7 @@ __global__ void __launch_bounds__(NTHR, 2)
                 const int src = __ffs(m) - 1;
                 fb = __shfl_sync(FULL, b, src);
                 fpre = __shfl_sync(FULL, excl, src);
+                funits = __shfl_sync(FULL, units, src);
             }
             acc += __shfl_sync(FULL, incl, 31);
         }
@@ -380,6 +407,7 @@ __global__ void __launch_bounds__(NTHR, 2)
             sh_n = N;
             sh_pe = Pe;
             sh_b = fb;
+            sh_bh0 = fb >= 0 ? fb * Hkv + (int)((ub - fpre) / (funits / Hkv)) : 0;
             ctl[1] = (int)(ue > ub && fb >= 0 ? ue - ub : 0);
             reinterpret_cast<long long *>(ctl + 2)[0] = fpre;
         }
@@ -623,15 +651,19 @@ __global__ void __launch_bounds__(NTHR, 2)
             __syncwarp();
             if (lane == 0) mbar_arrive(&segbar[1]);   // the consumers may refill mbuf
             if (p.counters != nullptr) {
-                // publish (fence, then count the arrival); the CTA whose arrival
-                // completes the count merges and writes the output
-                __threadfence();
+                // publish the warp's writes (warp barrier, then one acq_rel fence
+                // and the arrival count); the CTA whose arrival completes the
+                // count acquires the others' partials the same way and merges
                 __syncwarp();
                 int last = 0;
-                if (lane == 0) last = atomicAdd(&p.counters[bh], 1) == ncta - 1;
+                if (lane == 0) {
+                    fence_acq_rel_gpu();
+                    last = atomicAdd(&p.counters[bh], 1) == ncta - 1;
+                    if (last) fence_acq_rel_gpu();
+                }
                 last = __shfl_sync(FULL, last, 0);
+                __syncwarp();
                 if (last) {
-                    __threadfence();
                     const int b = bh / Hkv, kvh = bh % Hkv;
                     merge_segment<DH>(p.ws, (int64_t)cmin + bh, ncta, G, p.out, p.out_f32,
                                       ((int64_t)b * p.n_q_heads + (int64_t)kvh * G) * DH, lane);
@@ -672,18 +704,18 @@ __global__ void __launch_bounds__(NTHR, 2)
     // Rows of the score tile: row gid is token tw + rt, row gid + 8 token tw + rt + 1.
     // The P.V MMA takes k-slots 2tig, 2tig+1, 2tig+8, 2tig+9 = tokens
     // tw + vA, tw + vB, tw + vA + 1, tw + vB + 1 (the transpose of the score rows).
-    const int rt = row_token(gid);
-    const int vA = row_token(2 * tig), vB = row_token(2 * tig + 1);
+    const int rt = row_token<KWIDE>(gid);
+    const int vA = row_token<KWIDE>(2 * tig), vB = row_token<KWIDE>(2 * tig + 1);
     uint32_t kofs[2][2], vofs[2][4];
 #pragma unroll
     for (int u = 0; u < 2; u++) {
         const int tw = warp * 32 + u * 16;
-        kofs[u][0] = sw_off<RK>(tw + rt, tig * (SK / 4));
-        kofs[u][1] = sw_off<RK>(tw + rt + 1, tig * (SK / 4));
-        vofs[u][0] = p.off_v + sw_off<RV>(tw + vA, gid * (SV / 8));
-        vofs[u][1] = p.off_v + sw_off<RV>(tw + vB, gid * (SV / 8));
-        vofs[u][2] = p.off_v + sw_off<RV>(tw + vA + 1, gid * (SV / 8));
-        vofs[u][3] = p.off_v + sw_off<RV>(tw + vB + 1, gid * (SV / 8));
+        kofs[u][0] = sw_off<RK>(tw + rt, tig * KLW);
+        kofs[u][1] = sw_off<RK>(tw + rt + 1, tig * KLW);
+        vofs[u][0] = p.off_v + sw_off<RV>(tw + vA, gid * VL);
+        vofs[u][1] = p.off_v + sw_off<RV>(tw + vB, gid * VL);
+        vofs[u][2] = p.off_v + sw_off<RV>(tw + vA + 1, gid * VL);
+        vofs[u][3] = p.off_v + sw_off<RV>(tw + vB + 1, gid * VL);
     }
     // Sub-tile 1 lies 16 tokens after sub-tile 0.  For rows of >= 64 bytes the
     // swizzle phase repeats every 16 tokens, so its addresses are those of
@@ -705,7 +737,8 @@ __global__ void __launch_bounds__(NTHR, 2)
         const int kvh = bh % Hkv;
         if constexpr (IMMA_K) {
             // q ~ (amax / 127) * (hi + lo / 254) per head, hi, lo in [-127, 127];
-            // lane (gid, tig) holds head gid, elements 32 blk + 8 tig + 0..7
+            // lane (gid, tig) holds head gid and, for block blk, the 8 elements its
+            // key fragments hold: from (blk / KPL) 32 KPL + 8 KPL tig + 8 (blk % KPL)
             const bool valid = gid < G;
             const int64_t qbase = ((int64_t)b * p.n_q_heads + (int64_t)kvh * G + gid) * DH;
             float x[NG][8];
@@ -714,7 +747,10 @@ __global__ void __launch_bounds__(NTHR, 2)
             for (int blk = 0; blk < NG; blk++)
 #pragma unroll
                 for (int j = 0; j < 8; j++) {
-                    x[blk][j] = valid ? load_qf(p.q, p.q_dtype, qbase + 32 * blk + 8 * tig + j) : 0.f;
+                    x[blk][j] = valid ? load_qf(p.q, p.q_dtype,
+                                                qbase + (blk / KPL) * 32 * KPL + 8 * KPL * tig +
+                                                    8 * (blk % KPL) + j)
+                                      : 0.f;
                     amax = fmaxf(amax, fabsf(x[blk][j]));
                 }
             amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 1));
@@ -813,6 +849,8 @@ __global__ void __launch_bounds__(NTHR, 2)
     uint32_t ph = 0;
     uint32_t nseg = 0;           // segment ends handed to the combiner
     bool aborted = false;
+    // the first segment's query is loaded while its first tile is in flight
+    if (n_units > 0) load_q(sh_bh0);
     for (int i = 0; i < n_units; i++) {
         if (!mbar_wait_bounded(&full[s], ph, abort_flag, limit)) {
             ctl[0] = 1;
@@ -827,7 +865,7 @@ __global__ void __launch_bounds__(NTHR, 2)
             m.bh = (int)m0.x; m.t0 = (int)m0.y; m.len = (int)m0.z; m.flags = (int)m0.w;
             m.slot = (int)m1.x; m.ncta = (int)m1.y; m.cmin = (int)m1.z;
         }
-        if (m.flags & 1) load_q(m.bh);
+        if ((m.flags & 1) && i > 0) load_q(m.bh);
         const uint32_t st = (uint32_t)s * p.stage_bytes;   // stage offset from smem
         const uint32_t sst = sbase + st;                    // shared address of the stage
         const uint32_t ssk = st + p.off_sk;   // fp16 key scales of the stage
@@ -855,6 +893,41 @@ __global__ void __launch_bounds__(NTHR, 2)
                 for (int u = 0; u < 2; u++)
 #pragma unroll
                     for (int e = 0; e < 4; e++) ah[u][e] = al[u][e] = 0;
+                if constexpr (KWIDE) {
+                    // one 16-byte load per row and sub-tile holds KPL blocks
+#pragma unroll
+                    for (int lp = 0; lp < NG / KPL; lp++) {
+                        const uint32_t ra = sst + blk_addr<RK, 4 * KLW>(kofs[0][0], lp);
+                        const uint32_t rb = sst + blk_addr<RK, 4 * KLW>(kofs[0][1], lp);
+                        uint4 r[2][2];
+                        r[0][0] = ldsi_u128<0>(ra);
+                        r[0][1] = ldsi_u128<0>(rb);
+                        r[1][0] = ldsi_u128<ImmK::value>(KREP ? ra : sst + blk_addr<RK, 4 * KLW>(kofs[1][0], lp));
+                        r[1][1] = ldsi_u128<ImmK::value>(KREP ? rb : sst + blk_addr<RK, 4 * KLW>(kofs[1][1], lp));
+#pragma unroll
+                        for (int bi = 0; bi < KPL; bi++) {
+                            const int blk = lp * KPL + bi;
+#pragma unroll
+                            for (int u = 0; u < 2; u++) {
+                                const uint4 r0 = r[u][0], r1 = r[u][1];
+                                uint32_t fa[4];
+                                if constexpr (KB == 8) {
+                                    // block bi: bytes 8bi .. 8bi+7 of the lane's 16
+                                    fa[0] = bi ? r0.z : r0.x; fa[2] = bi ? r0.w : r0.y;
+                                    fa[1] = bi ? r1.z : r1.x; fa[3] = bi ? r1.w : r1.y;
+                                } else {
+                                    // block bi: word bi (8 nibbles) of the lane's 16 bytes
+                                    const uint32_t w0 = bi == 0 ? r0.x : (bi == 1 ? r0.y : (bi == 2 ? r0.z : r0.w));
+                                    const uint32_t w1 = bi == 0 ? r1.x : (bi == 1 ? r1.y : (bi == 2 ? r1.z : r1.w));
+                                    fa[0] = (w0 << 4) & 0xF0F0F0F0u; fa[1] = (w1 << 4) & 0xF0F0F0F0u;
+                                    fa[2] = w0 & 0xF0F0F0F0u;        fa[3] = w1 & 0xF0F0F0F0u;
+                                }
+                                imma_16832(ah[u], fa[0], fa[1], fa[2], fa[3], qh[blk][0], qh[blk][1]);
+                                imma_16832(al[u], fa[0], fa[1], fa[2], fa[3], ql[blk][0], ql[blk][1]);
+                            }
+                        }
+                    }
+                } else {
 #pragma unroll
                 for (int blk = 0; blk < NG; blk++) {
                     const uint32_t ra = sst + blk_addr<RK, SK>(kofs[0][0], blk);
@@ -871,6 +944,7 @@ __global__ void __launch_bounds__(NTHR, 2)
                         imma_16832(ah[u], fa[u][0], fa[u][1], fa[u][2], fa[u][3], qh[blk][0], qh[blk][1]);
                         imma_16832(al[u], fa[u][0], fa[u][1], fa[u][2], fa[u][3], ql[blk][0], ql[blk][1]);
                     }
+                }
                 }
 #pragma unroll
                 for (int u = 0; u < 2; u++) {
@@ -1046,6 +1120,84 @@ __global__ void __launch_bounds__(NTHR, 2)
         }
 
         // ---------------- phase 5: O^T += V^T P for both sub-tiles ----------------
+        if constexpr (VWIDE) {
+            // m-tile 4sb + j: row gid <-> d = 64sb + 8gid + 2j, row gid + 8 <-> d + 1
+#pragma unroll
+            for (int sb = 0; sb < NG / 2; sb++) {
+                uint32_t va[2][4];
+#pragma unroll
+                for (int r = 0; r < 4; r++) {
+                    va[0][r] = sst + blk_addr<RV, 2 * SV>(vofs[0][r], sb);
+                    va[1][r] = VREP ? va[0][r] : sst + blk_addr<RV, 2 * SV>(vofs[1][r], sb);
+                }
+#pragma unroll
+                for (int u = 0; u < 2; u++) {
+                    const uint32_t b0 = pb[u][0][0], b1 = pb[u][0][1];
+                    if constexpr (VB == 8) {
+                        uint2 w[4];
+#pragma unroll
+                        for (int r = 0; r < 4; r++)
+                            w[r] = u == 0 ? ldsi_u64<0>(va[0][r]) : ldsi_u64<ImmV::value>(va[1][r]);
+#pragma unroll
+                        for (int j = 0; j < 4; j++) {
+                            const uint32_t sel = (j & 1) ? 0x7632u : 0x5410u;
+                            const uint32_t A = j < 2 ? w[0].x : w[0].y, Bw = j < 2 ? w[1].x : w[1].y;
+                            const uint32_t C = j < 2 ? w[2].x : w[2].y, E = j < 2 ? w[3].x : w[3].y;
+                            const uint32_t yAB = prmt(A, Bw, sel), yCE = prmt(C, E, sel);
+                            const uint32_t a0 = and_xor(yAB, 0x00FF00FFu, 0x64806480u);
+                            const uint32_t a1 = and_xor(yAB >> 8, 0x00FF00FFu, 0x64806480u);
+                            const uint32_t a2 = and_xor(yCE, 0x00FF00FFu, 0x64806480u);
+                            const uint32_t a3 = and_xor(yCE >> 8, 0x00FF00FFu, 0x64806480u);
+                            mma_16816(o_acc[4 * sb + j], a0, a1, a2, a3, b0, b1);
+                        }
+                    } else if constexpr (VB == 4) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int r = 0; r < 4; r++)
+                            w[r] = u == 0 ? ldsi_u32<0>(va[0][r]) : ldsi_u32<ImmV::value>(va[1][r]);
+#pragma unroll
+                        for (int hb = 0; hb < 2; hb++) {
+                            // bytes 2hb, 2hb+1 of tokens A, B (C, E): elements 4hb .. 4hb+3
+                            const uint32_t sel = hb ? 0x7632u : 0x5410u;
+                            const uint32_t yAB = prmt(w[0], w[1], sel), yCE = prmt(w[2], w[3], sel);
+#pragma unroll
+                            for (int h = 0; h < 2; h++) {
+                                // rows gid take the even nibble (1032 + code), rows gid + 8
+                                // the odd one in place (1152 + 16 code)
+                                const uint32_t xAB = h ? yAB >> 8 : yAB, xCE = h ? yCE >> 8 : yCE;
+                                const uint32_t a0 = and_xor(xAB, 0x000F000Fu, 0x64086408u);
+                                const uint32_t a1 = and_xor(xAB, 0x00F000F0u, 0x64806480u);
+                                const uint32_t a2 = and_xor(xCE, 0x000F000Fu, 0x64086408u);
+                                const uint32_t a3 = and_xor(xCE, 0x00F000F0u, 0x64806480u);
+                                mma_16816(o_acc[4 * sb + 2 * hb + h], a0, a1, a2, a3, b0, b1);
+                            }
+                        }
+                    } else {
+                        // fp16 values past the length may be anything (NaN included): zero them
+                        const int tg = m.t0 + warp * 32 + u * 16;
+                        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                        uint4 w[4];
+#pragma unroll
+                        for (int r = 0; r < 4; r++) {
+                            const int tok = tg + ((r & 1) ? vB : vA) + (r >> 1);
+                            w[r] = z;
+                            if (tok < m.len)
+                                w[r] = u == 0 ? ldsi_u128<0>(va[0][r]) : ldsi_u128<ImmV::value>(va[1][r]);
+                        }
+#pragma unroll
+                        for (int j = 0; j < 4; j++) {
+                            const uint32_t A = j == 0 ? w[0].x : (j == 1 ? w[0].y : (j == 2 ? w[0].z : w[0].w));
+                            const uint32_t Bw = j == 0 ? w[1].x : (j == 1 ? w[1].y : (j == 2 ? w[1].z : w[1].w));
+                            const uint32_t C = j == 0 ? w[2].x : (j == 1 ? w[2].y : (j == 2 ? w[2].z : w[2].w));
+                            const uint32_t E = j == 0 ? w[3].x : (j == 1 ? w[3].y : (j == 2 ? w[3].z : w[3].w));
+                            const uint32_t a0 = prmt(A, Bw, 0x5410u), a1 = prmt(A, Bw, 0x7632u);
+                            const uint32_t a2 = prmt(C, E, 0x5410u), a3 = prmt(C, E, 0x7632u);
+                            mma_16816(o_acc[4 * sb + j], a0, a1, a2, a3, b0, b1);
+                        }
+                    }
+                }
+            }
+        } else {
 #pragma unroll
         for (int blk = 0; blk < NG; blk++) {
             // value-row addresses of this block (sub-tile 0; sub-tile 1 adds VU)
@@ -1121,6 +1273,8 @@ __global__ void __launch_bounds__(NTHR, 2)
             }
         }
 
+        }
+
         // release the stage to the producer
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
@@ -1160,9 +1314,13 @@ __global__ void __launch_bounds__(NTHR, 2)
                         const float ps = psum[VG ? blk : 0][c];
 #pragma unroll
                         for (int h = 0; h < 2; h++) {
-                            // m-tile 2blk+h: row gid <-> d = 32blk + 4gid + 2h, row gid+8 <-> d + 1
-                            const int d = 32 * blk + 4 * gid + 2 * h;
-                            float lo = o_acc[2 * blk + h][c], hi = o_acc[2 * blk + h][2 + c];
+                            // wide: m-tile 4sb + j, row gid <-> d = 64sb + 8gid + 2j;
+                            // block mapping: m-tile 2blk + h, row gid <-> d = 32blk + 4gid + 2h;
+                            // row gid + 8 <-> d + 1
+                            const int mt = 2 * blk + h;
+                            const int d = VWIDE ? 64 * (mt >> 2) + 8 * gid + 2 * (mt & 3)
+                                                : 32 * blk + 4 * gid + 2 * h;
+                            float lo = o_acc[mt][c], hi = o_acc[mt][2 + c];
                             if constexpr (VB == 4) {
                                 lo -= 1032.f * ps;                // even nibble: 1032 + code
                                 hi = (hi - 1152.f * ps) * 0.0625f;  // odd nibble: 1152 + 16 code

@@ -159,6 +159,16 @@ __device__ __forceinline__ void bulk_load_hint(void *dst, const void *src, uint3
         : "memory");
 }
 
+// ---------------------------------------------------------------- memory ordering
+// Acquire-release fence at device scope: orders this thread's earlier memory
+// operations (and those it has observed) before its later ones for every
+// thread of the GPU.  Used by one lane after a warp barrier to publish (or
+// acquire) the whole warp's writes around a flag.
+__device__ __forceinline__ void fence_acq_rel_gpu()
+{
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- programmatic launch
 // Wait until the grids this launch depends on have completed and their memory
 // operations are visible (returns at once when there is no such dependency).
