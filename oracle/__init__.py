@@ -62,6 +62,10 @@ def _load():
     lib.kvqo_f16_to_f32.restype = ctypes.c_float
     lib.kvqo_f32_to_bf16.argtypes = [ctypes.c_float]
     lib.kvqo_f32_to_bf16.restype = ctypes.c_uint16
+    lib.kvqo_f32_to_e4m3.argtypes = [ctypes.c_float]
+    lib.kvqo_f32_to_e4m3.restype = ctypes.c_uint8
+    lib.kvqo_e4m3_to_f32.argtypes = [ctypes.c_uint8]
+    lib.kvqo_e4m3_to_f32.restype = ctypes.c_float
     lib.kvqo_quantize_rows.argtypes = [P, i64, i32, i32, i32, P, P]
     lib.kvqo_dequantize_rows.argtypes = [P, P, i64, i32, i32, i32, P]
     lib.kvqo_attend.argtypes = [P, P, P, i64, i32, f64, P]
@@ -100,32 +104,55 @@ def f32_to_bf16_bits(x: float) -> int:
     return int(_load().kvqo_f32_to_bf16(float(x)))
 
 
+E4M3 = 228   # bit-width code of FP8 e4m3 codes (one byte per element)
+
+
+def f32_to_e4m3(x: float) -> int:
+    """e4m3 byte of x: round to nearest even, saturating at +-448."""
+    return int(_load().kvqo_f32_to_e4m3(float(x)))
+
+
+def e4m3_to_f32(c: int) -> float:
+    return float(_load().kvqo_e4m3_to_f32(int(c)))
+
+
+def _bits_arg(bits):
+    return E4M3 if bits in ("e4m3", E4M3) else int(bits)
+
+
+def _row_bytes(dim: int, bits: int) -> int:
+    return dim if bits == E4M3 else dim * bits // 8
+
+
 # --- quantiser ----------------------------------------------------------------
 
-def quantize_rows(x, group: int, bits: int):
+def quantize_rows(x, group: int, bits):
     """x: [..., dim] float32 (fp16/bf16 inputs must be widened exactly first).
+    bits: 4, 8 or "e4m3".
 
     Returns (codes uint8 [..., dim*bits/8], scales uint16 fp16-bits [..., dim/group]).
     """
+    bits = _bits_arg(bits)
     x = np.ascontiguousarray(x, dtype=np.float32)
     dim = x.shape[-1]
     rows = int(np.prod(x.shape[:-1])) if x.ndim > 1 else 1
-    codes = np.zeros(x.shape[:-1] + (dim * bits // 8,), np.uint8)
+    codes = np.zeros(x.shape[:-1] + (_row_bytes(dim, bits),), np.uint8)
     scales = np.zeros(x.shape[:-1] + (dim // group,), np.uint16)
     _chk(_load().kvqo_quantize_rows(_ptr(x), rows, dim, group, bits, _ptr(codes), _ptr(scales)),
          "quantize_rows")
     return codes, scales
 
 
-def dequantize_rows(codes, scales, dim: int, group: int, bits: int):
+def dequantize_rows(codes, scales, dim: int, group: int, bits):
     """Inverse of quantize_rows in fp64.  bits == 16: codes hold fp16 values."""
+    bits = _bits_arg(bits)
     codes = np.ascontiguousarray(codes)
     if bits == 16:
         codes = codes.view(np.uint8) if codes.dtype != np.uint8 else codes
         rows = codes.size // (dim * 2)
         lead = codes.shape[:-1]
     else:
-        rows = codes.size // (dim * bits // 8)
+        rows = codes.size // _row_bytes(dim, bits)
         lead = codes.shape[:-1]
         scales = np.ascontiguousarray(scales, dtype=np.uint16)
     out = np.zeros(lead + (dim,), np.float64)
@@ -155,6 +182,7 @@ def decode_layer(q, lens, k_codes, k_scales, k_bits, k_group, v_codes, v_scales,
     k_codes: [B, Hkv, cap, row] uint8 (bits 16: [B, Hkv, cap, dh] float16/uint16);
     k_scales: [B, Hkv, cap, dh/group] uint16 or None.  Returns [B, Hq, dh] float64.
     """
+    k_bits, v_bits = _bits_arg(k_bits), _bits_arg(v_bits)
     q = np.ascontiguousarray(q, np.float32)
     B, Hq, dh = q.shape
     lens = np.ascontiguousarray(lens, np.int32)

@@ -29,6 +29,10 @@
  *  - h-mode (TinyLoop docs, "運作原理"): cache h, rebuild K = W_k h and
  *    V = W_v h at every attention call.  Here h^ is dequantised, rounded to
  *    bf16 (the GEMM operand), K/V = W h^ in fp64 with W bf16, rounded to fp16.
+ *  - FP8 e4m3 codes (the mni-ml page's comparison with production stacks:
+ *    vLLM and TensorRT-LLM keep FP8 KV caches): same fp16 scales, with 448
+ *    (the largest finite e4m3 magnitude) in place of qmax and
+ *    code = e4m3_rne(x / s), saturating.  Bit-width code KVQO_E4M3 (228).
  *  - Bytes per token per layer (TinyLoop docs, "記憶體公式" table).
  *
  * Build: gcc -O2 -fopenmp -shared -fPIC -ffp-contract=off (no fast-math: the
@@ -41,6 +45,8 @@
 #ifdef _OPENMP
 #include <omp.h>
 #endif
+
+#define KVQO_E4M3 228   /* bit-width code for FP8 e4m3 codes (8 bits per element) */
 
 /* ------------------------------------------------------------------------ */
 /* Binary16 / bfloat16 conversions written from the IEEE 754 definitions.    */
@@ -147,10 +153,69 @@ float kvqo_bf16_to_f32(uint16_t b)
 }
 
 /* ------------------------------------------------------------------------ */
+/* FP8 e4m3 ("fn": 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits,  */
+/* no infinities; 0x7f / 0xff are NaN; the largest finite magnitude is 448 =  */
+/* 1.75 * 2^8, the smallest subnormal 2^-9).                                  */
+/* ------------------------------------------------------------------------ */
+
+/* Encode a float, rounding to nearest with ties to even; magnitudes that would
+ * round above 448 saturate to 448 (the KV-cache use never wants NaN). */
+uint8_t kvqo_f32_to_e4m3(float f)
+{
+    const uint8_t sign = signbit(f) ? 0x80 : 0x00;
+    if (isnan(f)) return (uint8_t)(sign | 0x7f);
+    const float a = fabsf(f);
+    if (a == 0.0f) return sign;
+    if (a < 0.015625f) {
+        /* below the smallest normal 2^-6: multiples of 2^-9 (a code of 8 is 2^-6,
+         * which is also the encoding of the smallest normal) */
+        const float m = nearbyintf(a * 512.0f);
+        return (uint8_t)(sign | (uint8_t)m);
+    }
+    int ex = 0;
+    (void)frexpf(a, &ex);           /* a = fr * 2^ex, fr in [0.5, 1) */
+    int e = ex - 1;                 /* a in [2^e, 2^(e+1)) */
+    if (e > 8) return (uint8_t)(sign | 0x7e);
+    float m = nearbyintf(ldexpf(a, 3 - e));  /* 8 .. 16: significand in eighths */
+    if (m == 16.0f) {
+        m = 8.0f;
+        e += 1;
+    }
+    const int code = ((e + 7) << 3) | ((int)m - 8);
+    if (code > 0x7e) return (uint8_t)(sign | 0x7e);
+    return (uint8_t)(sign | code);
+}
+
+float kvqo_e4m3_to_f32(uint8_t c)
+{
+    const float sgn = (c & 0x80) ? -1.0f : 1.0f;
+    const int e = (c >> 3) & 0xf, m = c & 7;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) return sgn * ldexpf((float)m, -9);
+    return sgn * ldexpf((float)(8 + m), e - 10);
+}
+
+/* ------------------------------------------------------------------------ */
 /* Quantiser                                                                 */
 /* ------------------------------------------------------------------------ */
 
 static int qmax_of(int bits) { return bits == 8 ? 127 : 7; }
+
+/* FP8 codes: scale s = fp16(absmax / 448), code = e4m3(x / s) (saturating). */
+static void quantize_group_e4m3(const float *x, int n, uint8_t *codes, uint16_t *scale_out)
+{
+    float a = 0.0f;
+    for (int i = 0; i < n; i++) {
+        float v = fabsf(x[i]);
+        if (v > a) a = v;
+    }
+    float s32 = a / 448.0f;
+    uint16_t s16 = kvqo_f32_to_f16(s32);
+    if ((s16 & 0x7fffu) == 0x7c00u) s16 = (uint16_t)((s16 & 0x8000u) | 0x7bffu);
+    float s = kvqo_f16_to_f32(s16);
+    for (int i = 0; i < n; i++) codes[i] = (s == 0.0f) ? 0 : kvqo_f32_to_e4m3(x[i] / s);
+    *scale_out = s16;
+}
 
 /* Quantise one group of n floats.  codes[i] receives the signed code. */
 static void quantize_group(const float *x, int n, int bits, int *codes, uint16_t *scale_out)
@@ -184,6 +249,15 @@ static void quantize_group(const float *x, int n, int bits, int *codes, uint16_t
 int kvqo_quantize_rows(const float *x, int64_t n_rows, int dim, int group, int bits,
                        uint8_t *codes, uint16_t *scales)
 {
+    if (bits == KVQO_E4M3) {
+        if (group <= 0 || dim % group != 0) return -1;
+        const int ng = dim / group;
+        for (int64_t r = 0; r < n_rows; r++)
+            for (int g = 0; g < ng; g++)
+                quantize_group_e4m3(x + r * (int64_t)dim + g * group, group,
+                                    codes + r * (int64_t)dim + g * group, &scales[r * ng + g]);
+        return 0;
+    }
     if (bits != 4 && bits != 8) return -1;
     if (group <= 0 || dim % group != 0) return -1;
     if (bits == 4 && (group % 2 != 0)) return -1;
@@ -226,6 +300,15 @@ int kvqo_dequantize_rows(const uint8_t *codes, const uint16_t *scales, int64_t n
     if (bits == 16) {
         const uint16_t *h = (const uint16_t *)codes;
         for (int64_t i = 0; i < n_rows * (int64_t)dim; i++) out[i] = (double)kvqo_f16_to_f32(h[i]);
+        return 0;
+    }
+    if (bits == KVQO_E4M3) {
+        if (group <= 0 || dim % group != 0) return -1;
+        const int ng = dim / group;
+        for (int64_t r = 0; r < n_rows; r++)
+            for (int i = 0; i < dim; i++)
+                out[r * dim + i] = (double)kvqo_e4m3_to_f32(codes[r * (int64_t)dim + i]) *
+                                   (double)kvqo_f16_to_f32(scales[r * ng + i / group]);
         return 0;
     }
     if (bits != 4 && bits != 8) return -1;
@@ -288,8 +371,10 @@ int kvqo_decode_layer(int B, int Hq, int Hkv, int dh, int cap,
     if (Hkv <= 0 || Hq % Hkv != 0) return -1;
     const int G = Hq / Hkv;
     if (tau <= 0.0) tau = 1.0 / sqrt((double)dh);
-    const int64_t krow = (k_bits == 16) ? (int64_t)dh * 2 : (int64_t)dh * k_bits / 8;
-    const int64_t vrow = (v_bits == 16) ? (int64_t)dh * 2 : (int64_t)dh * v_bits / 8;
+    const int64_t krow = (k_bits == 16) ? (int64_t)dh * 2
+                         : (k_bits == KVQO_E4M3 ? (int64_t)dh : (int64_t)dh * k_bits / 8);
+    const int64_t vrow = (v_bits == 16) ? (int64_t)dh * 2
+                         : (v_bits == KVQO_E4M3 ? (int64_t)dh : (int64_t)dh * v_bits / 8);
     const int kng = (k_bits == 16) ? 0 : dh / k_group;
     const int vng = (v_bits == 16) ? 0 : dh / v_group;
     int rc = 0;

@@ -422,3 +422,73 @@ def test_h_reconstruct_rounds_operand_to_bf16():
     ref = hb @ W.T
     np.testing.assert_allclose(y64, ref, rtol=1e-13, atol=1e-13)
     assert np.array_equal(y16, ref.astype(np.float16).view(np.uint16))
+
+
+# --- FP8 e4m3 codes ------------------------------------------------------------
+
+def test_e4m3_decode_matches_torch_for_every_code():
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    want = codes.view(torch.float8_e4m3fn).float().numpy()
+    got = np.array([oracle.e4m3_to_f32(c) for c in range(256)], np.float32)
+    nan = np.isnan(want)
+    assert np.array_equal(np.isnan(got), nan) and nan.sum() == 2   # 0x7f, 0xff
+    assert np.array_equal(got[~nan], want[~nan])
+    assert oracle.e4m3_to_f32(0x7e) == 448.0 and oracle.e4m3_to_f32(0x01) == 2.0 ** -9
+
+
+def test_e4m3_encode_matches_torch_rounding():
+    # every representable value, every midpoint between neighbours (ties), values
+    # just off the midpoints, random magnitudes over the whole range, saturation
+    vals = np.array([oracle.e4m3_to_f32(c) for c in range(0x7f)], np.float64)
+    mids = (vals[:-1] + vals[1:]) / 2
+    rng = np.random.default_rng(4)
+    x = np.concatenate([vals, mids, mids * (1 + 2.0 ** -20), mids * (1 - 2.0 ** -20),
+                        np.exp(rng.uniform(np.log(2.0 ** -12), np.log(600.0), 4000)),
+                        [448.0, 460.0, 464.0, 470.0, 1e6, 2.0 ** -10, 2.0 ** -10 * 1.01]])
+    x = np.concatenate([x, -x]).astype(np.float32)
+    want = torch.from_numpy(np.clip(x, -448.0, 448.0)).to(torch.float8_e4m3fn).view(torch.uint8)
+    got = np.array([oracle.f32_to_e4m3(v) for v in x], np.uint8)
+    assert np.array_equal(got, want.numpy())
+
+
+def test_e4m3_quantiser_scale_codes_and_error_bound():
+    rng = np.random.default_rng(5)
+    x = (rng.standard_normal((64, 128)) * rng.uniform(0.01, 50, (64, 1))).astype(np.float32)
+    x[3] = 0.0
+    for group in (32, 128):
+        codes, scales = oracle.quantize_rows(x, group, "e4m3")
+        assert codes.shape == (64, 128) and scales.shape == (64, 128 // group)
+        g = x.reshape(64, -1, group)
+        amax = np.abs(g).max(-1)
+        want_s = (amax / np.float32(448.0)).astype(np.float32).astype(np.float16).view(np.uint16)
+        assert np.array_equal(scales, want_s)
+        assert np.all(codes[3] == 0)
+        s = scales.view(np.float16).astype(np.float64)
+        xhat = oracle.dequantize_rows(codes, scales, 128, group, "e4m3").reshape(64, -1, group)
+        y = g / np.where(s == 0, 1, s)[..., None]
+        # half a unit in the last place of e4m3 at |x / s| (normal range: 2^(e-4)),
+        # never below half the smallest subnormal
+        e = np.floor(np.log2(np.maximum(np.abs(y), 2.0 ** -6)))
+        bound = np.maximum(2.0 ** (e - 4), 2.0 ** -10) * s[..., None]
+        assert np.all(np.abs(xhat - g) <= bound * (1 + 1e-6))
+        # the largest element lands within one step of 448
+        top = np.abs(xhat).max(-1)
+        ok = amax > 0
+        assert np.all(np.abs(top[ok] / s[ok] - 448) <= 32)
+
+
+def test_e4m3_decode_layer_matches_dequantised_attention():
+    rng = np.random.default_rng(6)
+    B, H, G, L, dh = 2, 2, 2, 40, 64
+    k = rng.standard_normal((B, H, L, dh)).astype(np.float32)
+    v = rng.standard_normal((B, H, L, dh)).astype(np.float32)
+    q = rng.standard_normal((B, H * G, dh)).astype(np.float32)
+    kc, ks = oracle.quantize_rows(k, 32, "e4m3")
+    vc, vs = oracle.quantize_rows(v, 64, "e4m3")
+    got = oracle.decode_layer(q, np.array([L, 17], np.int32), kc, ks, "e4m3", 32, vc, vs, "e4m3", 64, H)
+    kd = oracle.dequantize_rows(kc, ks, dh, 32, "e4m3")
+    vd = oracle.dequantize_rows(vc, vs, dh, 64, "e4m3")
+    for b, n in ((0, L), (1, 17)):
+        for h in range(H * G):
+            want = oracle.attend(q[b, h], kd[b, h // G, :n], vd[b, h // G, :n], 1 / np.sqrt(dh))
+            assert np.allclose(got[b, h], want, rtol=0, atol=1e-12)
