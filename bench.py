@@ -5,7 +5,8 @@ Workload (default): B=16, 32 layers, 32 query / 8 KV heads, head_dim 128,
 8K context (8191 cached + 1 appended per step), per-(token, head) fp16 scales.
 One step = for every layer: quantize-on-append of the new token's K and V,
 split-KV decode attention, merge of the partials -- captured in one CUDA graph.
-The headline variant is K8V8; K8V4 and K4V4 are reported under "variants".
+The headline variant is K8V8; K8V4, K4V4 and F8 (FP8 e4m3 keys and values)
+are reported under "variants".
 
 value  = KV bytes read per step (codes + scales of every attended token, all
          layers and sequences, summed over ranks) / device time per step.
@@ -37,7 +38,9 @@ sys.path.insert(0, ROOT)
 METRIC = "decode-attn KV GB/s (% of HBM peak) and steps/s at 8K ctx, K8V8/K8V4/K4V4"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
-VARIANTS = {"K8V8": (8, 8, 128, 128), "K8V4": (8, 4, 128, 128), "K4V4": (4, 4, 128, 128)}
+# (k_bits, v_bits, k_group, v_group, kv_format); F8: FP8 e4m3 keys and values
+VARIANTS = {"K8V8": (8, 8, 128, 128, 0), "K8V4": (8, 4, 128, 128, 0), "K4V4": (4, 4, 128, 128, 0),
+            "F8": (8, 8, 128, 128, 1)}
 
 
 def measured_peaks():
@@ -179,10 +182,10 @@ def build_variant(w, fmt, device):
     import quantized_kv_cache_22_b200 as kvq
     from quantized_kv_cache_22_b200 import Config, LayerCache, Workspace, inputs
 
-    kb, vb, kg, vg = fmt
+    kb, vb, kg, vg, kf = fmt
     cfg = Config(batch=w.batch, capacity=w.capacity, n_q_heads=w.n_q_heads,
                  n_kv_heads=w.n_kv_heads, head_dim=w.head_dim, k_bits=kb, v_bits=vb,
-                 k_group=kg, v_group=vg, n_layers=w.n_layers)
+                 k_group=kg, v_group=vg, n_layers=w.n_layers, kv_format=kf)
     L = w.context
     caches = []
     pos0 = torch.zeros(w.batch, dtype=torch.int32, device=device)
@@ -323,24 +326,25 @@ def cpu_oracle_layer(w, fmt, st=None, device=None, reps=1, budget_s=0.0):
     import oracle
     from quantized_kv_cache_22_b200 import inputs
 
-    kb, vb, kg, vg = fmt
+    kb, vb, kg, vg, kf = fmt
+    kb_o, vb_o = ("e4m3", "e4m3") if kf == 1 else (kb, vb)   # the oracle's width arguments
     L = w.context
     gen_dev = device if device is not None else "cpu"
     k, v = inputs.kv_tokens(w, 0, L - 1, gen_dev)
     k1, v1 = inputs.kv_tokens(w, 0, 1, gen_dev, offset_seed=1)
     q = inputs.queries(w, 0, 0, gen_dev)
-    kf = k.float().cpu().numpy().transpose(0, 2, 1, 3)
-    vf = v.float().cpu().numpy().transpose(0, 2, 1, 3)
+    k_f = k.float().cpu().numpy().transpose(0, 2, 1, 3)
+    v_f = v.float().cpu().numpy().transpose(0, 2, 1, 3)
     del k, v
     kc = np.zeros((w.batch, w.n_kv_heads, L, w.head_dim * kb // 8), np.uint8)
     vc = np.zeros((w.batch, w.n_kv_heads, L, w.head_dim * vb // 8), np.uint8)
     ks = np.zeros((w.batch, w.n_kv_heads, L, w.head_dim // kg), np.uint16)
     vs = np.zeros((w.batch, w.n_kv_heads, L, w.head_dim // vg), np.uint16)
-    a, b = oracle.quantize_rows(np.ascontiguousarray(kf), kg, kb)
+    a, b = oracle.quantize_rows(np.ascontiguousarray(k_f), kg, kb_o)
     kc[:, :, : L - 1], ks[:, :, : L - 1] = a, b
-    a, b = oracle.quantize_rows(np.ascontiguousarray(vf), vg, vb)
+    a, b = oracle.quantize_rows(np.ascontiguousarray(v_f), vg, vb_o)
     vc[:, :, : L - 1], vs[:, :, : L - 1] = a, b
-    del kf, vf
+    del k_f, v_f
     k1f = np.ascontiguousarray(k1.float().cpu().numpy().transpose(0, 2, 1, 3))
     v1f = np.ascontiguousarray(v1.float().cpu().numpy().transpose(0, 2, 1, 3))
     qf = q.float().cpu().numpy()
@@ -349,11 +353,11 @@ def cpu_oracle_layer(w, fmt, st=None, device=None, reps=1, budget_s=0.0):
     times = []
     while len(times) < reps or (sum(times) < budget_s and len(times) < 1000):
         t0 = time.perf_counter()
-        a, b = oracle.quantize_rows(k1f, kg, kb)
+        a, b = oracle.quantize_rows(k1f, kg, kb_o)
         kc[:, :, L - 1:], ks[:, :, L - 1:] = a, b
-        a, b = oracle.quantize_rows(v1f, vg, vb)
+        a, b = oracle.quantize_rows(v1f, vg, vb_o)
         vc[:, :, L - 1:], vs[:, :, L - 1:] = a, b
-        oracle.decode_layer(qf, lens, kc, ks, kb, kg, vc, vs, vb, vg, w.n_kv_heads, 0.0, cores)
+        oracle.decode_layer(qf, lens, kc, ks, kb_o, kg, vc, vs, vb_o, vg, w.n_kv_heads, 0.0, cores)
         times.append(time.perf_counter() - t0)
     return times, cores
 
@@ -485,7 +489,7 @@ def run_paged(args, world, device):
     from quantized_kv_cache_22_b200 import Config, LayerCache, Workspace, inputs
 
     w = dataclasses.replace(inputs.WORKLOADS[4], n_layers=4)
-    kb, vb, kg, vg = VARIANTS["K8V8"]
+    kb, vb, kg, vg, _ = VARIANTS["K8V8"]
     pages = w.batch * (w.capacity // 128)
     cfg = Config(batch=w.batch, capacity=w.capacity, n_q_heads=w.n_q_heads,
                  n_kv_heads=w.n_kv_heads, head_dim=w.head_dim, k_bits=kb, v_bits=vb,
@@ -682,7 +686,7 @@ def run_reference(args):
     fmt = VARIANTS[head]
     cfg = kvq.Config(batch=w.batch, capacity=w.capacity, n_q_heads=w.n_q_heads,
                      n_kv_heads=w.n_kv_heads, head_dim=w.head_dim, k_bits=fmt[0], v_bits=fmt[1],
-                     k_group=fmt[2], v_group=fmt[3], n_layers=w.n_layers)
+                     k_group=fmt[2], v_group=fmt[3], n_layers=w.n_layers, kv_format=fmt[4])
     per_layer = kvq.kvq_cache_bytes(cfg)[0] * w.batch * w.context
     times, cores = cpu_oracle_layer(w, fmt, reps=args.warmup + args.steps)
     t = statistics.mean(times[args.warmup:]) if len(times) > args.warmup else statistics.mean(times)
@@ -711,7 +715,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("kvq", "reference"), default="kvq")
     ap.add_argument("--workload", type=int, default=4)
-    ap.add_argument("--variants", default="K8V8,K8V4,K4V4")
+    ap.add_argument("--variants", default="K8V8,K8V4,K4V4,F8")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--sections", default="kv,hmode,window,paged",

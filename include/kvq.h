@@ -75,6 +75,11 @@ enum kvq_mode {
     KVQ_MODE_H = 1    /* the cache stores quantised h = LN(residual) [TL]    */
 };
 
+enum kvq_format {
+    KVQ_FMT_INT = 0,   /* signed integer codes (INT8 / INT4)                       */
+    KVQ_FMT_E4M3 = 1   /* FP8 e4m3 codes, 8 bits                                   */
+};
+
 enum kvq_dtype {
     KVQ_F16 = 0,
     KVQ_F32 = 1,
@@ -117,6 +122,12 @@ typedef struct kvq_config {
                             page; capacity (a multiple of 128) is then the
                             logical tokens per sequence.  No sliding window.      */
     int32_t n_pages;     /* paged cache: pages in each layer's pool               */
+    int32_t kv_format;   /* KV mode: KVQ_FMT_INT (integer codes) or KVQ_FMT_E4M3:
+                            8-bit FP8 e4m3 codes for both keys and values (k_bits =
+                            v_bits = 8), scale s = fp16(absmax / 448) per group,
+                            code = e4m3_rne(x / s) saturating at 448, value =
+                            e4m3(code) * s ([MNI] "Comparison với production
+                            stack": FP8 KV caches of vLLM and TensorRT-LLM).      */
 } kvq_config;
 
 /* One layer's cache buffers (device pointers, caller-owned).

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libkvq.so")
 
 KVQ_OK = 0
 KVQ_MODE_KV, KVQ_MODE_H = 0, 1
+KVQ_FMT_INT, KVQ_FMT_E4M3 = 0, 1
 KVQ_F16, KVQ_F32, KVQ_BF16 = 0, 1, 2
 
 EXPORTED = ("kvq_cache_bytes", "kvq_layer_buffer_bytes", "kvq_append", "kvq_workspace_bytes",
@@ -39,7 +40,7 @@ class KvqConfig(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "mode", "batch", "capacity", "n_layers", "n_q_heads", "n_kv_heads", "head_dim",
         "k_bits", "v_bits", "k_group", "v_group", "d_model", "h_bits", "h_groups",
-        "window", "n_anchor", "page_tokens", "n_pages")]
+        "window", "n_anchor", "page_tokens", "n_pages", "kv_format")]
 
 
 class KvqLayer(ctypes.Structure):
@@ -142,13 +143,14 @@ class Config:
     n_anchor: int = 0     # tokens kept at the start of the sequence
     page_tokens: int = 0  # 128: paged cache (a pool of n_pages pages, block table per layer)
     n_pages: int = 0
+    kv_format: int = 0    # KVQ_FMT_INT, or KVQ_FMT_E4M3 (FP8 e4m3 codes, k_bits = v_bits = 8)
 
     def _key(self):
         return (self.mode, self.batch, self.capacity, self.n_layers, self.n_q_heads,
                 self.n_kv_heads, self.head_dim, self.k_bits, self.v_bits,
                 self.k_group or self.head_dim, self.v_group or self.head_dim,
                 self.d_model, self.h_bits, self.h_groups, self.window, self.n_anchor,
-                self.page_tokens, self.n_pages)
+                self.page_tokens, self.n_pages, self.kv_format)
 
     def c(self) -> KvqConfig:
         """A new ``kvq_config`` struct with these fields."""

@@ -54,6 +54,9 @@ int check_cfg(const kvq_config *c)
         if (c->window == 0 && c->n_anchor != 0) return KVQ_ERR_INVALID_ARG;
         if (c->window > 0 && (int64_t)c->n_anchor + c->window != c->capacity)
             return KVQ_ERR_INVALID_ARG;
+        if (c->kv_format != KVQ_FMT_INT && c->kv_format != KVQ_FMT_E4M3) return KVQ_ERR_INVALID_ARG;
+        if (c->kv_format == KVQ_FMT_E4M3 && (c->k_bits != 8 || c->v_bits != 8))
+            return KVQ_ERR_UNSUPPORTED;
         if (c->page_tokens != 0) {
             if (c->page_tokens != kPageTokens) return KVQ_ERR_UNSUPPORTED;
             if (c->window != 0) return KVQ_ERR_UNSUPPORTED;
@@ -62,7 +65,8 @@ int check_cfg(const kvq_config *c)
             return KVQ_ERR_INVALID_ARG;
         }
     } else {
-        if (c->window != 0 || c->n_anchor != 0 || c->page_tokens != 0 || c->n_pages != 0)
+        if (c->window != 0 || c->n_anchor != 0 || c->page_tokens != 0 || c->n_pages != 0 ||
+            c->kv_format != KVQ_FMT_INT)
             return KVQ_ERR_UNSUPPORTED;
         if (c->d_model < 128 || c->d_model % 128 != 0) return KVQ_ERR_UNSUPPORTED;
         if (!valid_bits(c->h_bits)) return KVQ_ERR_UNSUPPORTED;
@@ -205,6 +209,7 @@ int current_device_props(int *sms, int *max_smem)
 // Shapes of the attention half (KV mode, or h-mode after reconstruction).
 struct AttnShape {
     int hkv, hq, G, dh, kb, vb, kg, vg, ngs_k, ngs_v;
+    bool f8;   // 8-bit codes are FP8 e4m3
 };
 
 AttnShape attn_shape(const kvq_config *c)
@@ -219,6 +224,7 @@ AttnShape attn_shape(const kvq_config *c)
         s.vb = c->v_bits;
         s.kg = c->k_group;
         s.vg = c->v_group;
+        s.f8 = c->kv_format == KVQ_FMT_E4M3;
     } else {
         s.kb = s.vb = 16;
         s.kg = s.vg = s.dh;
@@ -237,7 +243,7 @@ int resolve_plan(const kvq_config *cfg, int32_t num_ctas, DecodeLaunch *plan, in
         int rc = current_device_props(&sms, &max_smem);
         if (rc) return rc;
     }
-    if (!plan_decode(a.dh, a.kb, a.vb, a.ngs_k, a.ngs_v, a.G, max_smem, plan))
+    if (!plan_decode(a.dh, a.kb, a.vb, a.ngs_k, a.ngs_v, a.G, max_smem, plan, a.f8))
         return KVQ_ERR_UNSUPPORTED;
     if (num_ctas > 0) {
         *ctas = num_ctas;
@@ -344,6 +350,7 @@ int kvq_append(const kvq_config *cfg, const kvq_layer *layer, const void *k, con
     AppendParams pk{};
     pk.window = cfg->window;
     pk.n_anchor = cfg->n_anchor;
+    pk.e4m3 = cfg->mode == KVQ_MODE_KV && cfg->kv_format == KVQ_FMT_E4M3;
     if (cfg->mode == KVQ_MODE_KV && cfg->page_tokens) {
         if (!layer->block_table) return KVQ_ERR_INVALID_ARG;
         pk.block_table = layer->block_table;
@@ -455,8 +462,8 @@ static int decode_kv_layout(const kvq_config *cfg, const void *k_codes, const vo
                             const int32_t *block_table = nullptr)
 {
     const AttnShape a = attn_shape(cfg);
-    // fp16 keys use an f16 MMA whose f32 / bf16 queries take two columns per head
-    if (a.kb == 16 && q_dtype != KVQ_F16 && a.G > 4) return KVQ_ERR_UNSUPPORTED;
+    // fp16 and e4m3 keys use an f16 MMA whose f32 / bf16 queries take two columns per head
+    if ((a.kb == 16 || a.f8) && q_dtype != KVQ_F16 && a.G > 4) return KVQ_ERR_UNSUPPORTED;
     DecodeLaunch plan;
     int ctas = 0;
     int rc = resolve_plan(cfg, num_ctas, &plan, &ctas);

@@ -57,7 +57,7 @@ __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ App
     uint8_t *codes_row = p.codes + cache_row * ((int64_t)dim * p.bits / 8);
     __half *scales_row = p.bits == 16 ? nullptr : p.scales + cache_row * (dim / p.group);
     quantize_row(p.x, row * (int64_t)dim, p.in_dtype, dim, p.bits, p.group, codes_row, scales_row,
-                 lane);
+                 lane, p.e4m3 != 0);
 }
 
 }  // namespace

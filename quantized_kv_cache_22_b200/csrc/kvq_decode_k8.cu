@@ -7,7 +7,7 @@ namespace {
 template <int DH, int VB, bool KG, bool VG>
 void *fn()
 {
-    return reinterpret_cast<void *>(&decode_kernel<DH, 8, VB, KG, VG>);
+    return reinterpret_cast<void *>(&decode_kernel<DH, 8, VB, KG, VG, false>);
 }
 
 template <int DH, int VB, bool KG>

@@ -292,7 +292,8 @@ __device__ __forceinline__ void merge_segment(const float *ws, int64_t slot0, in
 
 // KG / VG: keys / values carry one scale per 32/64-element group (else one per
 // (token, head)); compile-time so the per-head case keeps no per-group state.
-template <int DH, int KB, int VB, bool KG, bool VG>
+// F8: the 8-bit codes of keys and values are FP8 e4m3 (KB = VB = 8).
+template <int DH, int KB, int VB, bool KG, bool VG, bool F8>
 __global__ void __launch_bounds__(NTHR, 2)
     decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const __grid_constant__ DecodeParams p)
@@ -308,16 +309,19 @@ __global__ void __launch_bounds__(NTHR, 2)
     // load feeds four m-tiles); grouped value scales need one P per 32-element
     // block, so a lane then reads 4 elements per block.  Rows of 32 bytes (Dh 64
     // at 4 bits) keep the block mapping, which stays free of bank conflicts.
-    constexpr bool VWIDE = !VG && RV >= 64;
+    constexpr bool VWIDE = !VG && RV >= 64 && !F8;
     constexpr int VL = VWIDE ? 2 * SV / 8 : SV / 8;   // value bytes per lane per row and load
     // Key fragments: with one key scale per (token, head), int8 keys are read 16
     // bytes per lane and row ("wide": 2 blocks of 32 elements per load at 8
     // bits, 4 at 4 bits); an int8 MMA block must share one key scale, so
     // grouped key scales keep one load per block.
-    constexpr bool KWIDE = !KG && KB != 16 && RK >= 64;
+    constexpr bool KWIDE = !KG && KB != 16 && RK >= 64 && !F8;
     constexpr int KLW = KWIDE ? 16 : SK / 4;          // key bytes per lane per row and load
     constexpr int KPL = KWIDE ? 16 * 8 / KB / 8 : 1;  // 32-element blocks per load
-    constexpr float BIAS_V = VB == 8 ? 1152.f : 0.f;   // 4-bit values: per row, see the segment end
+    // value codes enter the P.V MMA as (bias + code): 1152 at 8 bits, per row at 4
+    // bits (see the segment end); fp16 and e4m3 values convert exactly, no bias
+    constexpr float BIAS_V = (VB == 8 && !F8) ? 1152.f : 0.f;
+    constexpr bool VBIAS = VB == 4 || (VB == 8 && !F8);
     // The running max is only raised when a tile beats it by more than 2^LAZY;
     // weights p * s_V then stay below 2^LAZY, well inside fp16.
     constexpr float LAZY = 8.f;
@@ -481,10 +485,10 @@ __global__ void __launch_bounds__(NTHR, 2)
             }
             quantize_row(p.app.k_new, (int64_t)bh * DH, p.app.dtype, DH, KB, p.app.k_group,
                          p.app.k_codes + crow * RK,
-                         KB == 16 ? nullptr : p.app.k_scales + crow * (DH / p.app.k_group), lane);
+                         KB == 16 ? nullptr : p.app.k_scales + crow * (DH / p.app.k_group), lane, F8);
             quantize_row(p.app.v_new, (int64_t)bh * DH, p.app.dtype, DH, VB, p.app.v_group,
                          p.app.v_codes + crow * RV,
-                         VB == 16 ? nullptr : p.app.v_scales + crow * (DH / p.app.v_group), lane);
+                         VB == 16 ? nullptr : p.app.v_scales + crow * (DH / p.app.v_group), lane, F8);
             // order the writes before the copy engine reads the tile
             fence_proxy_async_global();
             __syncwarp();
@@ -613,7 +617,7 @@ __global__ void __launch_bounds__(NTHR, 2)
         // this CTA's slot, hand mbuf back, publish, and merge when this CTA's
         // partial is the last one of its (sequence, KV head).
         constexpr int CS = slot_col_floats(DH);
-        const int ncol = (KB == 16 && p.q_dtype != KVQ_F16) ? min(G, 4) : G;
+        const int ncol = ((KB == 16 || F8) && p.q_dtype != KVQ_F16) ? min(G, 4) : G;
         for (uint32_t k = 0;; k++) {
             if (!mbar_wait_bounded(&segbar[0], k & 1u, abort_flag, p.timeout_ns)) {
                 if (lane == 0 && *abort_flag == 0) {
@@ -674,7 +678,7 @@ __global__ void __launch_bounds__(NTHR, 2)
     }
 
     // ====================== consumers ======================
-    constexpr bool IMMA_K = KB != 16;
+    constexpr bool IMMA_K = KB != 16 && !F8;   // else f16 MMA (fp16 keys, or e4m3 converted)
     const int gid = lane >> 2;
     const int tig = lane & 3;
     // fp16 keys keep an f16 MMA; f32 / bf16 queries then use columns 4..7 for
@@ -981,6 +985,82 @@ __global__ void __launch_bounds__(NTHR, 2)
                     for (int e = 0; e < 4; e++) s2[u][e] = v[e] * sqc[e & 1];
                 }
             }
+        } else if constexpr (F8) {
+            // e4m3 keys: each code pair converts exactly to a half2 in registers;
+            // lane tig's 8 bytes of a block are elements 8tig .. 8tig+7, the k-slot
+            // order of the fp16 query fragments
+            auto f8_frags = [&](uint2 r0, uint2 r1, int hs, uint32_t (&fa)[4]) {
+                const uint32_t w0 = hs ? r0.y : r0.x, w1 = hs ? r1.y : r1.x;
+                fa[0] = e4m3x2_to_half2(w0 & 0xFFFFu); fa[1] = e4m3x2_to_half2(w1 & 0xFFFFu);
+                fa[2] = e4m3x2_to_half2(w0 >> 16);     fa[3] = e4m3x2_to_half2(w1 >> 16);
+            };
+            if constexpr (!kgrp) {
+                float acc[2][2][4];
+#pragma unroll
+                for (int u = 0; u < 2; u++)
+#pragma unroll
+                    for (int h = 0; h < 2; h++) acc[u][h][0] = acc[u][h][1] = acc[u][h][2] = acc[u][h][3] = 0.f;
+#pragma unroll
+                for (int blk = 0; blk < NG; blk++) {
+                    const uint32_t ra = sst + blk_addr<RK, SK>(kofs[0][0], blk);
+                    const uint32_t rb = sst + blk_addr<RK, SK>(kofs[0][1], blk);
+                    uint2 r[2][2];
+                    r[0][0] = ldsi_u64<0>(ra);
+                    r[0][1] = ldsi_u64<0>(rb);
+                    r[1][0] = ldsi_u64<ImmK::value>(KREP ? ra : sst + blk_addr<RK, SK>(kofs[1][0], blk));
+                    r[1][1] = ldsi_u64<ImmK::value>(KREP ? rb : sst + blk_addr<RK, SK>(kofs[1][1], blk));
+#pragma unroll
+                    for (int u = 0; u < 2; u++)
+#pragma unroll
+                        for (int hs = 0; hs < 2; hs++) {
+                            uint32_t fa[4];
+                            f8_frags(r[u][0], r[u][1], hs, fa);
+                            mma_16816(acc[u][hs], fa[0], fa[1], fa[2], fa[3], qb[blk][hs][0], qb[blk][hs][1]);
+                        }
+                }
+#pragma unroll
+                for (int u = 0; u < 2; u++) {
+                    const float2 kk = unpack_half2(lds_u32(sbase, ssk + 2 * tAu[u]));
+#pragma unroll
+                    for (int e = 0; e < 4; e++) {
+                        float v = (acc[u][0][e] + acc[u][1][e]) * (((e < 2) ? kk.x : kk.y) * p.tau_log2e);
+                        if (qsplit) v += __shfl_xor_sync(FULL, v, 2);
+                        s2[u][e] = v;
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int u = 0; u < 2; u++) {
+                    float v[4] = {0.f, 0.f, 0.f, 0.f};
+                    const int tA = tAu[u];
+#pragma unroll
+                    for (int blk = 0; blk < NG; blk++) {
+                        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                        const uint2 r0 = ldsi_u64<0>(sst + blk_addr<RK, SK>(kofs[u][0], blk));
+                        const uint2 r1 = ldsi_u64<0>(sst + blk_addr<RK, SK>(kofs[u][1], blk));
+#pragma unroll
+                        for (int hs = 0; hs < 2; hs++) {
+                            uint32_t fa[4];
+                            f8_frags(r0, r1, hs, fa);
+                            mma_16816(acc, fa[0], fa[1], fa[2], fa[3], qb[blk][hs][0], qb[blk][hs][1]);
+                        }
+                        const float k0 = __half2float(__ushort_as_half(
+                            (unsigned short)lds_u16(sbase, ssk + 2 * (tA * p.ngs_k + (blk >> p.kshift)))));
+                        const float k1 = __half2float(__ushort_as_half(
+                            (unsigned short)lds_u16(sbase, ssk + 2 * ((tA + 1) * p.ngs_k + (blk >> p.kshift)))));
+                        v[0] = fmaf(k0, acc[0], v[0]);
+                        v[1] = fmaf(k0, acc[1], v[1]);
+                        v[2] = fmaf(k1, acc[2], v[2]);
+                        v[3] = fmaf(k1, acc[3], v[3]);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 4; e++) {
+                        float x = v[e] * p.tau_log2e;
+                        if (qsplit) x += __shfl_xor_sync(FULL, x, 2);
+                        s2[u][e] = x;
+                    }
+                }
+            }
         } else {
             // fp16 keys: two partial accumulators per sub-tile halve the MMA chain
             float acc[2][2][4];
@@ -1114,7 +1194,7 @@ __global__ void __launch_bounds__(NTHR, 2)
                 pb[u][g][0] = movmatrix_trans(x0);
                 pb[u][g][1] = movmatrix_trans(x1);
                 // column sums of the fp16 weights, for the code bias
-                if constexpr (VB != 16)
+                if constexpr (VBIAS)
                     mma_16816(psum[g], ONE2, ONE2, ONE2, ONE2, pb[u][g][0], pb[u][g][1]);
             }
         }
@@ -1133,7 +1213,28 @@ __global__ void __launch_bounds__(NTHR, 2)
 #pragma unroll
                 for (int u = 0; u < 2; u++) {
                     const uint32_t b0 = pb[u][0][0], b1 = pb[u][0][1];
-                    if constexpr (VB == 8) {
+                    if constexpr (F8) {
+                        // e4m3 values past the length may be stale (a NaN code): zero them
+                        const int tg = m.t0 + warp * 32 + u * 16;
+                        uint2 w[4];
+#pragma unroll
+                        for (int r = 0; r < 4; r++) {
+                            const int tok = tg + ((r & 1) ? vB : vA) + (r >> 1);
+                            w[r] = make_uint2(0u, 0u);
+                            if (tok < m.len) w[r] = u == 0 ? ldsi_u64<0>(va[0][r]) : ldsi_u64<ImmV::value>(va[1][r]);
+                        }
+#pragma unroll
+                        for (int j = 0; j < 4; j++) {
+                            // bytes 2j', 2j'+1 (j' = j mod 2) of tokens A, B interleaved:
+                            // low half (A, B) element 2j', high half the next element
+                            const uint32_t sel = (j & 1) ? 0x7362u : 0x5140u;
+                            const uint32_t A = j < 2 ? w[0].x : w[0].y, Bw = j < 2 ? w[1].x : w[1].y;
+                            const uint32_t C = j < 2 ? w[2].x : w[2].y, E = j < 2 ? w[3].x : w[3].y;
+                            const uint32_t yAB = prmt(A, Bw, sel), yCE = prmt(C, E, sel);
+                            mma_16816(o_acc[4 * sb + j], e4m3x2_to_half2(yAB & 0xFFFFu), e4m3x2_to_half2(yAB >> 16),
+                                      e4m3x2_to_half2(yCE & 0xFFFFu), e4m3x2_to_half2(yCE >> 16), b0, b1);
+                        }
+                    } else if constexpr (VB == 8) {
                         uint2 w[4];
 #pragma unroll
                         for (int r = 0; r < 4; r++)
@@ -1210,7 +1311,25 @@ __global__ void __launch_bounds__(NTHR, 2)
 #pragma unroll
             for (int u = 0; u < 2; u++) {
                 const uint32_t b0 = pb[u][VG ? blk : 0][0], b1 = pb[u][VG ? blk : 0][1];
-                if constexpr (VB == 8) {
+                if constexpr (F8) {
+                    // e4m3 values past the length may be stale (a NaN code): zero them
+                    const int tg = m.t0 + warp * 32 + u * 16;
+                    uint32_t w[4];
+#pragma unroll
+                    for (int r = 0; r < 4; r++) {
+                        const int tok = tg + ((r & 1) ? vB : vA) + (r >> 1);
+                        w[r] = 0u;
+                        if (tok < m.len) w[r] = u == 0 ? ldsi_u32<0>(va[0][r]) : ldsi_u32<ImmV::value>(va[1][r]);
+                    }
+#pragma unroll
+                    for (int h = 0; h < 2; h++) {
+                        // (A, B) byte pairs 2h and 2h+1: rows gid and gid + 8
+                        const uint32_t sel = h ? 0x7362u : 0x5140u;
+                        const uint32_t yAB = prmt(w[0], w[1], sel), yCE = prmt(w[2], w[3], sel);
+                        mma_16816(o_acc[2 * blk + h], e4m3x2_to_half2(yAB & 0xFFFFu), e4m3x2_to_half2(yAB >> 16),
+                                  e4m3x2_to_half2(yCE & 0xFFFFu), e4m3x2_to_half2(yCE >> 16), b0, b1);
+                    }
+                } else if constexpr (VB == 8) {
                     uint32_t wA, wB, wC, wE;
                     if (u == 0) {
                         wA = ldsi_u32<0>(va[0][0]); wB = ldsi_u32<0>(va[0][1]);

@@ -17,6 +17,7 @@ struct AppendParams {
     int32_t batch, n_new, rows_per_tok, dim, cap;
     int32_t bits, group;
     int32_t window, n_anchor;   // sliding window (0: slot = position)
+    int32_t e4m3;               // 8-bit codes are FP8 e4m3
     const int32_t *block_table; // paged cache: [batch][max_pages] pool page of each logical page
     int32_t max_pages, n_pages; // (rows_per_tok is the KV heads; pages hold kPageTokens rows)
 };
@@ -87,6 +88,7 @@ struct MergeParams {
 struct DecodeLaunch {
     int dh, kb, vb;
     bool kg, vg;              // grouped key / value scales
+    bool f8;                  // 8-bit codes are FP8 e4m3
     size_t smem_bytes;
     int stages;
     uint32_t stage_bytes, off_v, off_sk, off_sv, off_meta, off_bar, off_merge;
@@ -98,10 +100,11 @@ struct DecodeLaunch {
 void *decode_fn_kb4(int dh, int vb, bool kg, bool vg);
 void *decode_fn_kb8(int dh, int vb, bool kg, bool vg);
 void *decode_fn_kb16(int dh, int vb, bool kg, bool vg);
+void *decode_fn_f8(int dh, bool kg, bool vg);   // FP8 e4m3 keys and values (kvq_decode_f8.cu)
 
 // Fill in the shared-memory plan; returns false if the shape is unsupported.
 bool plan_decode(int dh, int kb, int vb, int ngs_k, int ngs_v, int G, int max_smem,
-                 DecodeLaunch *plan);
+                 DecodeLaunch *plan, bool f8 = false);
 cudaError_t decode_occupancy(const DecodeLaunch &plan, int *ctas_per_sm);
 cudaError_t launch_decode(const DecodeLaunch &plan, const DecodeParams &p, const CUtensorMap &tm_k,
                           const CUtensorMap &tm_v, cudaStream_t stream);

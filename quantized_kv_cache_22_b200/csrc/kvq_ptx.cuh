@@ -226,6 +226,16 @@ __device__ __forceinline__ void fence_proxy_async_global()
 }
 
 // ---------------------------------------------------------------- bytes
+// Two FP8 e4m3 codes (low 16 bits of x: the first code in the low byte) to a
+// half2 (the first value in the low half); every e4m3 value is exact in fp16.
+__device__ __forceinline__ uint32_t e4m3x2_to_half2(uint32_t x)
+{
+    uint32_t r;
+    const uint16_t h = (uint16_t)x;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(h));
+    return r;
+}
+
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
 {
     uint32_t r;

@@ -12,6 +12,7 @@
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include "../../include/kvq.h"
 
@@ -43,10 +44,12 @@ __device__ __forceinline__ void load4(const void *base, int64_t idx, int dtype, 
 // Scale s = fp16(absmax / qmax) with qmax 127 (8 bits) or 7 (4 bits), an
 // overflow to +inf saturating to 65504; code = clamp(rne(x / s), -qmax, qmax),
 // all codes 0 when s = 0.  4-bit element 2j sits in the low nibble of byte j.
+// e4m3 (8 bits): s = fp16(absmax / 448) and code = e4m3(x / s), rounded to
+// nearest even and saturating at 448.
 // All 32 lanes of the warp must call it with the same arguments.
 __device__ __forceinline__ void quantize_row(const void *x, int64_t in_off, int dtype, int dim,
                                              int bits, int group, uint8_t *codes_row,
-                                             __half *scales_row, int lane)
+                                             __half *scales_row, int lane, bool e4m3 = false)
 {
     const int lanes_per_group = group >> 2;
     for (int base = 0; base < dim; base += 128) {
@@ -71,10 +74,26 @@ __device__ __forceinline__ void quantize_row(const void *x, int64_t in_off, int 
         float a = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
         for (int off = 1; off < lanes_per_group; off <<= 1)
             a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
-        const float s32 = __fdiv_rn(a, (float)qmax);
+        const float s32 = __fdiv_rn(a, e4m3 ? 448.0f : (float)qmax);
         __half s16 = __float2half_rn(s32);
         if (__half_as_ushort(s16) == 0x7c00u) s16 = __ushort_as_half(0x7bffu);
         const float s = __half2float(s16);
+
+        if (e4m3) {
+            if (active) {
+                uint32_t w = 0;
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    const uint32_t c = s != 0.0f
+                        ? (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(v[i], s), __NV_SATFINITE, __NV_E4M3)
+                        : 0u;
+                    w |= c << (8 * i);
+                }
+                *reinterpret_cast<uint32_t *>(codes_row + e0) = w;
+                if ((lane % lanes_per_group) == 0) scales_row[e0 / group] = s16;
+            }
+            continue;
+        }
 
         int c[4];
 #pragma unroll

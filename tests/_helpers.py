@@ -14,6 +14,11 @@ def to_np32(t):
     return t.detach().to("cpu").float().numpy()
 
 
+def obits(cfg: Config, bits: int):
+    """The oracle's bit-width argument for a cache width: "e4m3" for FP8 caches."""
+    return "e4m3" if cfg.kv_format == kvq.KVQ_FMT_E4M3 and bits == 8 else bits
+
+
 def oracle_cache(k, v, cfg: Config):
     """k, v: [B, L, Hkv, dh] tensors -> oracle codes/scales in the cache layout [B, Hkv, cap, ...]."""
     B, L, H, dh = k.shape
@@ -26,7 +31,7 @@ def oracle_cache(k, v, cfg: Config):
             c[:, :, :L] = xf.astype(np.float16)
             out += [c.view(np.uint16), None]
         else:
-            cc, ss = oracle.quantize_rows(xf, grp, bits)
+            cc, ss = oracle.quantize_rows(xf, grp, obits(cfg, bits))
             c = np.zeros((B, H, cap, dh * bits // 8), np.uint8)
             s = np.zeros((B, H, cap, dh // grp), np.uint16)
             c[:, :, :L] = cc
@@ -67,7 +72,7 @@ def vmax_per_batch(vc, vs, cfg: Config, lens):
             out.append(1.0)
             continue
         vd = oracle.dequantize_rows(vc[b, :, :L], None if vs is None else vs[b, :, :L], dh,
-                                    cfg.v_group or dh, cfg.v_bits)
+                                    cfg.v_group or dh, obits(cfg, cfg.v_bits))
         out.append(float(np.abs(vd).max()))
     return np.array(out)
 
@@ -86,8 +91,8 @@ def gpu_decode(cfg: Config, cache, q, lens, out_dtype=torch.float32, num_ctas=0,
 
 def oracle_decode(cfg: Config, oc, q, lens, scale=0.0):
     kc, ks, vc, vs = oc
-    return oracle.decode_layer(to_np32(q), np.array(lens, np.int32), kc, ks, cfg.k_bits,
-                               cfg.k_group or cfg.head_dim, vc, vs, cfg.v_bits,
+    return oracle.decode_layer(to_np32(q), np.array(lens, np.int32), kc, ks, obits(cfg, cfg.k_bits),
+                               cfg.k_group or cfg.head_dim, vc, vs, obits(cfg, cfg.v_bits),
                                cfg.v_group or cfg.head_dim, cfg.n_kv_heads, scale)
 
 

@@ -182,3 +182,22 @@ def test_paged_config_validation_and_bytes():
     P = ctypes.c_void_p
     assert _rc("kvq_append", ctypes.byref(paged.c()), ctypes.byref(lay), P(16), P(32), 0, P(64),
                0, 1, None) == -1
+
+
+def test_fp8_config_validation_and_bytes():
+    # FP8 e4m3 codes take one byte per element like INT8: same cache bytes
+    base = dict(batch=2, capacity=256, n_q_heads=8, n_kv_heads=2, head_dim=128, k_bits=8,
+                v_bits=8, k_group=32, v_group=128)
+    f8 = Config(**base, kv_format=kvq.KVQ_FMT_E4M3)
+    assert kvq.kvq_cache_bytes(f8) == kvq.kvq_cache_bytes(Config(**base))
+    assert kvq.kvq_layer_buffer_bytes(f8) == kvq.kvq_layer_buffer_bytes(Config(**base))
+    for over, want in (({"k_bits": 4}, -2), ({"v_bits": 16}, -2), ({"kv_format": 2}, -1),
+                       ({"kv_format": -1}, -1)):
+        with pytest.raises(kvq.KvqError) as e:
+            kvq.kvq_cache_bytes(Config(**{**f8.__dict__, **over}))
+        assert e.value.status == want, over
+    h = Config(batch=1, capacity=64, mode=kvq.KVQ_MODE_H, d_model=2048, h_bits=4, h_groups=16,
+               n_q_heads=16, n_kv_heads=16, head_dim=128, kv_format=kvq.KVQ_FMT_E4M3)
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.kvq_cache_bytes(h)
+    assert e.value.status == -2

@@ -227,11 +227,11 @@ def test_tiny_workload_prompt_then_252_steps(cuda_device):
     assert kvq.kvq_workspace_status(ws) == 0
 
 
-def _sampled_full_size(widx, fmt, layer, pairs, device="cuda"):
+def _sampled_full_size(widx, fmt, layer, pairs, device="cuda", kv_format=0):
     w = inputs.WORKLOADS[widx]
     cfg = Config(batch=w.batch, capacity=w.capacity, n_q_heads=w.n_q_heads,
                  n_kv_heads=w.n_kv_heads, head_dim=w.head_dim, k_bits=fmt[0], v_bits=fmt[1],
-                 k_group=fmt[2], v_group=fmt[3])
+                 k_group=fmt[2], v_group=fmt[3], kv_format=kv_format)
     L = w.context
     k, v = inputs.kv_tokens(w, layer, L, device)
     cache = gpu_cache(cfg, k, v, device)
