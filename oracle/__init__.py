@@ -13,6 +13,14 @@ Parity status of each function (what pins it, in ``tests/test_oracle_pins.py``):
   f32_to_f16 / f64_to_f16 / bf16: pinned against numpy float16 / torch bfloat16.
   quantize_rows: pinned by the error bound |x - x^| <= s/2, |code| <= qmax,
       absmax -> +-qmax, idempotence, RNE ties and nibble-order fixtures.
+  quantize_rows "e4m3": every code and every tie against torch float8_e4m3fn, the
+      scale formula and the half-ulp error bound.
+  quantize_rows "asym8": an exact arithmetic progression (codes 0..255), one-sided
+      and all-zero groups, the error bound and exact zero, torch's quint8 affine
+      quantiser at the same scale and zero-point; its decode equals the symmetric
+      INT8 decode when the zero-point is 128.
+  quantize_rows_tensor: equal to the per-head INT8 codes at the same scale,
+      clipping, torch's qint8 quantiser.
   attend / decode_layer: pinned by closed forms (L=1, q=0, two tokens, equal
       keys, dominant key), GQA head mapping, permutation/duplication
       invariance, and torch scaled_dot_product_attention in fp64.
@@ -68,6 +76,7 @@ def _load():
     lib.kvqo_e4m3_to_f32.restype = ctypes.c_float
     lib.kvqo_quantize_rows.argtypes = [P, i64, i32, i32, i32, P, P]
     lib.kvqo_dequantize_rows.argtypes = [P, P, i64, i32, i32, i32, P]
+    lib.kvqo_quantize_rows_tensor.argtypes = [P, i64, i32, ctypes.c_uint16, P]
     lib.kvqo_attend.argtypes = [P, P, P, i64, i32, f64, P]
     lib.kvqo_decode_layer.argtypes = [i32, i32, i32, i32, i32, P, P, i32, i32, P, P, i32, i32,
                                       P, P, f64, P, i32]
@@ -105,6 +114,7 @@ def f32_to_bf16_bits(x: float) -> int:
 
 
 E4M3 = 228   # bit-width code of FP8 e4m3 codes (one byte per element)
+ASYM8 = 208  # bit-width code of asymmetric INT8: uint8 codes, (scale, zero-point) fp16 pairs
 
 
 def f32_to_e4m3(x: float) -> int:
@@ -117,30 +127,50 @@ def e4m3_to_f32(c: int) -> float:
 
 
 def _bits_arg(bits):
-    return E4M3 if bits in ("e4m3", E4M3) else int(bits)
+    if bits in ("e4m3", E4M3):
+        return E4M3
+    if bits in ("asym8", ASYM8):
+        return ASYM8
+    return int(bits)
 
 
 def _row_bytes(dim: int, bits: int) -> int:
-    return dim if bits == E4M3 else dim * bits // 8
+    return dim if bits in (E4M3, ASYM8) else dim * bits // 8
+
+
+def _scales_per_group(bits: int) -> int:
+    return 2 if bits == ASYM8 else 1
 
 
 # --- quantiser ----------------------------------------------------------------
 
 def quantize_rows(x, group: int, bits):
     """x: [..., dim] float32 (fp16/bf16 inputs must be widened exactly first).
-    bits: 4, 8 or "e4m3".
+    bits: 4, 8, "e4m3" or "asym8".
 
-    Returns (codes uint8 [..., dim*bits/8], scales uint16 fp16-bits [..., dim/group]).
+    Returns (codes uint8 [..., dim*bits/8], scales uint16 fp16-bits [..., dim/group]);
+    "asym8": codes [..., dim], scales [..., dim/group, 2] = (scale, zero-point) per group.
     """
     bits = _bits_arg(bits)
     x = np.ascontiguousarray(x, dtype=np.float32)
     dim = x.shape[-1]
     rows = int(np.prod(x.shape[:-1])) if x.ndim > 1 else 1
     codes = np.zeros(x.shape[:-1] + (_row_bytes(dim, bits),), np.uint8)
-    scales = np.zeros(x.shape[:-1] + (dim // group,), np.uint16)
+    scales = np.zeros(x.shape[:-1] + (dim // group,) + ((2,) if bits == ASYM8 else ()), np.uint16)
     _chk(_load().kvqo_quantize_rows(_ptr(x), rows, dim, group, bits, _ptr(codes), _ptr(scales)),
          "quantize_rows")
     return codes, scales
+
+
+def quantize_rows_tensor(x, s16: int):
+    """Per-tensor INT8: every element of x with the one fp16 scale s16 (bits);
+    returns int8 codes as uint8 [..., dim]."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    dim = x.shape[-1]
+    codes = np.zeros(x.shape, np.uint8)
+    _chk(_load().kvqo_quantize_rows_tensor(_ptr(x), x.size // dim, dim, int(s16), _ptr(codes)),
+         "quantize_rows_tensor")
+    return codes
 
 
 def dequantize_rows(codes, scales, dim: int, group: int, bits):

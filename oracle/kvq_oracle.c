@@ -33,6 +33,19 @@
  *    vLLM and TensorRT-LLM keep FP8 KV caches): same fp16 scales, with 448
  *    (the largest finite e4m3 magnitude) in place of qmax and
  *    code = e4m3_rne(x / s), saturating.  Bit-width code KVQO_E4M3 (228).
+ *  - Asymmetric INT8 with a zero-point, and per-tensor INT8 (the mni-ml page,
+ *    "Tại sao INT8 mà không mất tốc": scale/zero-point metadata; "Limitations":
+ *    symmetric per-tensor scaling).  Asymmetric, per group of elements, the
+ *    textbook affine scheme with zero inside the range:
+ *      lo = min(0, min x), hi = max(0, max x)
+ *      s16 = fp16_rne((hi - lo) / 255), +inf saturated to 65504
+ *      z = clamp(rne(-lo / s), 0, 255),  q = clamp(rne(x / s) + z, 0, 255)
+ *      x^ = (q - z) * s;  s == 0: z = 0 and q = 0.
+ *    q is stored as a uint8, and each group keeps the pair (s16, fp16(z)).
+ *    Bit-width code KVQO_ASYM8 (208).  Per-tensor: one caller-given fp16
+ *    scale s for a whole tensor, code = clamp(rne(x / s), -127, 127), the
+ *    symmetric INT8 codes (x^ = code * s, the per-head dequantisation with
+ *    every row's scale equal to s).
  *  - Bytes per token per layer (TinyLoop docs, "記憶體公式" table).
  *
  * Build: gcc -O2 -fopenmp -shared -fPIC -ffp-contract=off (no fast-math: the
@@ -47,6 +60,7 @@
 #endif
 
 #define KVQO_E4M3 228   /* bit-width code for FP8 e4m3 codes (8 bits per element) */
+#define KVQO_ASYM8 208  /* bit-width code for asymmetric INT8 (uint8 codes, (scale, zero) pairs) */
 
 /* ------------------------------------------------------------------------ */
 /* Binary16 / bfloat16 conversions written from the IEEE 754 definitions.    */
@@ -217,6 +231,61 @@ static void quantize_group_e4m3(const float *x, int n, uint8_t *codes, uint16_t 
     *scale_out = s16;
 }
 
+/* Asymmetric INT8: lo = min(0, min x), hi = max(0, max x), s = fp16((hi-lo)/255),
+ * z = clamp(rne(-lo/s), 0, 255), q = clamp(rne(x/s) + z, 0, 255). */
+static void quantize_group_asym8(const float *x, int n, uint8_t *codes, uint16_t *scale_out,
+                                 uint16_t *zero_out)
+{
+    float lo = 0.0f, hi = 0.0f;
+    for (int i = 0; i < n; i++) {
+        if (x[i] < lo) lo = x[i];
+        if (x[i] > hi) hi = x[i];
+    }
+    float s32 = (hi - lo) / 255.0f;
+    uint16_t s16 = kvqo_f32_to_f16(s32);
+    if ((s16 & 0x7fffu) == 0x7c00u) s16 = (uint16_t)((s16 & 0x8000u) | 0x7bffu);
+    float s = kvqo_f16_to_f32(s16);
+    int z = 0;
+    if (s != 0.0f) {
+        float zr = nearbyintf(-lo / s);
+        if (zr < 0.0f) zr = 0.0f;
+        if (zr > 255.0f) zr = 255.0f;
+        z = (int)zr;
+    }
+    for (int i = 0; i < n; i++) {
+        if (s == 0.0f) {
+            codes[i] = 0;
+            continue;
+        }
+        float r = nearbyintf(x[i] / s) + (float)z;
+        if (r < 0.0f) r = 0.0f;
+        if (r > 255.0f) r = 255.0f;
+        codes[i] = (uint8_t)(int)r;
+    }
+    *scale_out = s16;
+    *zero_out = kvqo_f32_to_f16((float)z);
+}
+
+/* Per-tensor INT8 with a given fp16 scale s16: code = clamp(rne(x / s), -127, 127),
+ * all codes 0 when s == 0.  n_rows x dim floats, one byte per element. */
+int kvqo_quantize_rows_tensor(const float *x, int64_t n_rows, int dim, uint16_t s16,
+                              uint8_t *codes)
+{
+    const float s = kvqo_f16_to_f32(s16);
+    if (!(s >= 0.0f) || isinf(s)) return -1;
+    for (int64_t i = 0; i < n_rows * (int64_t)dim; i++) {
+        if (s == 0.0f) {
+            codes[i] = 0;
+            continue;
+        }
+        float r = nearbyintf(x[i] / s);
+        if (r > 127.0f) r = 127.0f;
+        if (r < -127.0f) r = -127.0f;
+        codes[i] = (uint8_t)(int8_t)(int)r;
+    }
+    return 0;
+}
+
 /* Quantise one group of n floats.  codes[i] receives the signed code. */
 static void quantize_group(const float *x, int n, int bits, int *codes, uint16_t *scale_out)
 {
@@ -249,6 +318,17 @@ static void quantize_group(const float *x, int n, int bits, int *codes, uint16_t
 int kvqo_quantize_rows(const float *x, int64_t n_rows, int dim, int group, int bits,
                        uint8_t *codes, uint16_t *scales)
 {
+    if (bits == KVQO_ASYM8) {
+        /* scales: [n_rows][dim/group][2] = (s16, fp16(z)) per group */
+        if (group <= 0 || dim % group != 0) return -1;
+        const int ng = dim / group;
+        for (int64_t r = 0; r < n_rows; r++)
+            for (int g = 0; g < ng; g++)
+                quantize_group_asym8(x + r * (int64_t)dim + g * group, group,
+                                     codes + r * (int64_t)dim + g * group,
+                                     &scales[(r * ng + g) * 2], &scales[(r * ng + g) * 2 + 1]);
+        return 0;
+    }
     if (bits == KVQO_E4M3) {
         if (group <= 0 || dim % group != 0) return -1;
         const int ng = dim / group;
@@ -300,6 +380,18 @@ int kvqo_dequantize_rows(const uint8_t *codes, const uint16_t *scales, int64_t n
     if (bits == 16) {
         const uint16_t *h = (const uint16_t *)codes;
         for (int64_t i = 0; i < n_rows * (int64_t)dim; i++) out[i] = (double)kvqo_f16_to_f32(h[i]);
+        return 0;
+    }
+    if (bits == KVQO_ASYM8) {
+        if (group <= 0 || dim % group != 0) return -1;
+        const int ng = dim / group;
+        for (int64_t r = 0; r < n_rows; r++)
+            for (int i = 0; i < dim; i++) {
+                const int64_t gi = (r * ng + i / group) * 2;
+                const double sc = (double)kvqo_f16_to_f32(scales[gi]);
+                const double z = (double)kvqo_f16_to_f32(scales[gi + 1]);
+                out[r * dim + i] = ((double)codes[r * (int64_t)dim + i] - z) * sc;
+            }
         return 0;
     }
     if (bits == KVQO_E4M3) {
@@ -371,12 +463,14 @@ int kvqo_decode_layer(int B, int Hq, int Hkv, int dh, int cap,
     if (Hkv <= 0 || Hq % Hkv != 0) return -1;
     const int G = Hq / Hkv;
     if (tau <= 0.0) tau = 1.0 / sqrt((double)dh);
-    const int64_t krow = (k_bits == 16) ? (int64_t)dh * 2
-                         : (k_bits == KVQO_E4M3 ? (int64_t)dh : (int64_t)dh * k_bits / 8);
-    const int64_t vrow = (v_bits == 16) ? (int64_t)dh * 2
-                         : (v_bits == KVQO_E4M3 ? (int64_t)dh : (int64_t)dh * v_bits / 8);
-    const int kng = (k_bits == 16) ? 0 : dh / k_group;
-    const int vng = (v_bits == 16) ? 0 : dh / v_group;
+    /* one-byte codes: e4m3 and asymmetric INT8 */
+    const int k1 = k_bits == KVQO_E4M3 || k_bits == KVQO_ASYM8;
+    const int v1 = v_bits == KVQO_E4M3 || v_bits == KVQO_ASYM8;
+    const int64_t krow = (k_bits == 16) ? (int64_t)dh * 2 : (k1 ? (int64_t)dh : (int64_t)dh * k_bits / 8);
+    const int64_t vrow = (v_bits == 16) ? (int64_t)dh * 2 : (v1 ? (int64_t)dh : (int64_t)dh * v_bits / 8);
+    /* fp16 values per row in the scale arrays: a pair per group when asymmetric */
+    const int kng = (k_bits == 16) ? 0 : (dh / k_group) * (k_bits == KVQO_ASYM8 ? 2 : 1);
+    const int vng = (v_bits == 16) ? 0 : (dh / v_group) * (v_bits == KVQO_ASYM8 ? 2 : 1);
     int rc = 0;
     (void)n_threads;
 #ifdef _OPENMP

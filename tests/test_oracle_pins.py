@@ -492,3 +492,117 @@ def test_e4m3_decode_layer_matches_dequantised_attention():
         for h in range(H * G):
             want = oracle.attend(q[b, h], kd[b, h // G, :n], vd[b, h // G, :n], 1 / np.sqrt(dh))
             assert np.allclose(got[b, h], want, rtol=0, atol=1e-12)
+
+
+# --- asymmetric INT8 (zero-point) and per-tensor INT8 ----------------------------
+
+def _asym(x, group):
+    codes, sz = oracle.quantize_rows(x, group, "asym8")
+    return codes, sz[..., 0], sz[..., 1]
+
+
+def test_asym8_arithmetic_progression_closed_form():
+    # x_i = (i - 100) / 4, i = 0..255: lo = -25, hi = 38.75, s = 63.75 / 255 = 1/4 exactly,
+    # z = 100 and q_i = i
+    x = ((np.arange(256) - 100) / 4.0).astype(np.float32)[None]
+    codes, s, z = _asym(x, 256)
+    assert np.array_equal(codes[0], np.arange(256))
+    assert s[0, 0] == np.float16(0.25).view(np.uint16) and z[0, 0] == np.float16(100).view(np.uint16)
+    # shuffled order, same codes per element
+    perm = np.random.default_rng(0).permutation(256)
+    c2, _, _ = _asym(np.ascontiguousarray(x[:, perm]), 256)
+    assert np.array_equal(c2[0], perm)
+
+
+def test_asym8_one_sided_groups_and_zero_group():
+    rng = np.random.default_rng(1)
+    pos = rng.uniform(0.5, 3.0, (4, 64)).astype(np.float32)
+    c, s, z = _asym(pos, 64)
+    assert np.all(z == 0) and np.all(c.max(-1) >= 254)          # lo = 0: the max near 255
+    c, s, z = _asym(-pos, 64)
+    assert np.all(z == np.float16(255).view(np.uint16)) and np.all(c.min(-1) <= 1)
+    c, s, z = _asym(np.zeros((2, 64), np.float32), 32)
+    assert not c.any() and not s.any() and not z.any()
+
+
+@pytest.mark.parametrize("group", [32, 64, 128])
+def test_asym8_error_bound_and_exact_zero(group):
+    rng = np.random.default_rng(2 + group)
+    x = (rng.standard_normal((96, 128)) * rng.uniform(0.01, 40, (96, 1))
+         + rng.uniform(-30, 30, (96, 1))).astype(np.float32)
+    x[5, :: 7] = 0.0
+    codes, sz = oracle.quantize_rows(x, group, "asym8")
+    xhat = oracle.dequantize_rows(codes, sz, 128, group, "asym8")
+    s = sz[..., 0].view(np.float16).astype(np.float64)
+    srow = np.repeat(s, group, axis=-1)
+    # unclipped: |x - x^| <= s/2; fp16 rounding of s can clip the ends by at most 1/8 step
+    assert np.all(np.abs(xhat - x) <= 0.625 * srow * (1 + 1e-6))
+    assert np.all(xhat[5, ::7] == 0.0)
+    zr = sz[..., 1].view(np.float16).astype(np.float64)
+    assert np.all(zr == np.round(zr)) and zr.min() >= 0 and zr.max() <= 255
+
+
+def test_asym8_codes_match_torch_affine_quantiser():
+    """torch.quantize_per_tensor (quint8, the oracle's own scale and zero-point per
+    group) computes the same codes, up to one step where x / s sits on a tie (torch
+    multiplies by 1/s)."""
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal((64, 128)) * 3 + 1).astype(np.float32)
+    codes, s, z = _asym(x, 32)
+    n_eq = 0
+    for r in range(64):
+        for g in range(4):
+            sc = float(s[r, g:g + 1].view(np.float16)[0])
+            zp = int(z[r, g:g + 1].view(np.float16)[0])
+            t = torch.quantize_per_tensor(torch.from_numpy(x[r, 32 * g:32 * g + 32].copy()), sc, zp,
+                                          torch.quint8).int_repr().numpy()
+            d = np.abs(t.astype(int) - codes[r, 32 * g:32 * g + 32].astype(int))
+            assert d.max() <= 1
+            n_eq += int((d == 0).sum())
+    assert n_eq >= 0.99 * x.size
+
+
+def test_asym8_decode_with_zero_point_128_equals_symmetric_codes():
+    # symmetric int8 codes c with scale s are the asymmetric codes c + 128 with (s, 128)
+    rng = np.random.default_rng(7)
+    B, H, G, L, dh = 2, 2, 2, 33, 64
+    k = rng.standard_normal((B, H, L, dh)).astype(np.float32)
+    v = rng.standard_normal((B, H, L, dh)).astype(np.float32)
+    q = rng.standard_normal((B, H * G, dh)).astype(np.float32)
+    kc, ks = oracle.quantize_rows(k, 64, 8)
+    vc, vs = oracle.quantize_rows(v, 32, 8)
+    z128 = np.float16(128).view(np.uint16)
+
+    def to_asym(c, s):
+        pairs = np.stack([s, np.full_like(s, z128)], -1)
+        return (c.view(np.int8).astype(np.int16) + 128).astype(np.uint8), pairs
+
+    kca, ksa = to_asym(kc, ks)
+    vca, vsa = to_asym(vc, vs)
+    lens = np.array([L, 9], np.int32)
+    want = oracle.decode_layer(q, lens, kc, ks, 8, 64, vc, vs, 8, 32, H)
+    got = oracle.decode_layer(q, lens, kca, ksa, "asym8", 64, vca, vsa, "asym8", 32, H)
+    assert np.array_equal(got, want)
+
+
+def test_per_tensor_int8_equals_per_head_codes_at_the_same_scale():
+    # rows whose per-head scale is exactly s = 1/16 (absmax 127/16) get the same codes
+    rng = np.random.default_rng(8)
+    x = rng.uniform(-7.9, 7.9, (16, 128)).astype(np.float32)
+    x[:, 3] = 127 / 16
+    s16 = int(np.float16(1 / 16).view(np.uint16))
+    c_head, s_head = oracle.quantize_rows(x, 128, 8)
+    assert np.all(s_head == s16)
+    assert np.array_equal(oracle.quantize_rows_tensor(x, s16), c_head)
+
+
+def test_per_tensor_int8_clips_and_matches_torch_qint8():
+    rng = np.random.default_rng(9)
+    x = (rng.standard_normal((32, 64)) * 4).astype(np.float32)
+    s = 0.03125
+    c = oracle.quantize_rows_tensor(x, int(np.float16(s).view(np.uint16))).view(np.int8)
+    assert c.min() == -127 and c.max() == 127                      # |x| reaches past 127 s
+    xc = np.clip(x, -127 * s, 127 * s)
+    t = torch.quantize_per_tensor(torch.from_numpy(xc), s, 0, torch.qint8).int_repr().numpy()
+    assert np.array_equal(t, c)                                   # s a power of two: no ties differ
+    assert not oracle.quantize_rows_tensor(x, 0).any()
