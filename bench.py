@@ -5,8 +5,9 @@ Workload (default): B=16, 32 layers, 32 query / 8 KV heads, head_dim 128,
 8K context (8191 cached + 1 appended per step), per-(token, head) fp16 scales.
 One step = for every layer: quantize-on-append of the new token's K and V,
 split-KV decode attention, merge of the partials -- captured in one CUDA graph.
-The headline variant is K8V8; K8V4, K4V4 and F8 (FP8 e4m3 keys and values)
-are reported under "variants".
+The headline variant is K8V8; K8V4, K4V4, F8 (FP8 e4m3 keys and values), A8
+(asymmetric INT8 with zero-points) and T8 (per-tensor INT8) are reported under
+"variants".
 
 value  = KV bytes read per step (codes + scales of every attended token, all
          layers and sequences, summed over ranks) / device time per step.
@@ -38,9 +39,17 @@ sys.path.insert(0, ROOT)
 METRIC = "decode-attn KV GB/s (% of HBM peak) and steps/s at 8K ctx, K8V8/K8V4/K4V4"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
-# (k_bits, v_bits, k_group, v_group, kv_format); F8: FP8 e4m3 keys and values
+# (k_bits, v_bits, k_group, v_group, kv_format); F8: FP8 e4m3 keys and values; A8:
+# asymmetric INT8 (scale + zero-point per (token, head)); T8: per-tensor INT8 (one
+# scale per K / V tensor of a layer, set from the tensor's absmax before the prefill)
 VARIANTS = {"K8V8": (8, 8, 128, 128, 0), "K8V4": (8, 4, 128, 128, 0), "K4V4": (4, 4, 128, 128, 0),
-            "F8": (8, 8, 128, 128, 1)}
+            "F8": (8, 8, 128, 128, 1), "A8": (8, 8, 128, 128, 2), "T8": (8, 8, 128, 128, 3)}
+
+
+def tensor_scale_bits(x) -> int:
+    """fp16 bits of a per-tensor INT8 scale max|x| / 127, as a caller would calibrate it."""
+    import numpy as np
+    return int(np.float16(float(x.float().abs().max()) / 127.0).view(np.uint16))
 
 
 def measured_peaks():
@@ -192,6 +201,9 @@ def build_variant(w, fmt, device):
     for layer in range(w.n_layers):
         c = LayerCache(cfg, device)
         k, v = inputs.kv_tokens(w, layer, L - 1, device)
+        if kf == kvq.KVQ_FMT_TENSOR:
+            for t, x in ((c.k_scales, k), (c.v_scales, v)):
+                t.view(torch.int16)[0] = (tensor_scale_bits(x) ^ 0x8000) - 0x8000
         kvq.kvq_append(cfg, c, k, v, pos0, 0, L - 1)
         del k, v
         caches.append(c)
@@ -327,22 +339,31 @@ def cpu_oracle_layer(w, fmt, st=None, device=None, reps=1, budget_s=0.0):
     from quantized_kv_cache_22_b200 import inputs
 
     kb, vb, kg, vg, kf = fmt
-    kb_o, vb_o = ("e4m3", "e4m3") if kf == 1 else (kb, vb)   # the oracle's width arguments
+    # the oracle's width arguments
+    kb_o, vb_o = {1: ("e4m3", "e4m3"), 2: ("asym8", "asym8")}.get(kf, (kb, vb))
     L = w.context
     gen_dev = device if device is not None else "cpu"
     k, v = inputs.kv_tokens(w, 0, L - 1, gen_dev)
     k1, v1 = inputs.kv_tokens(w, 0, 1, gen_dev, offset_seed=1)
     q = inputs.queries(w, 0, 0, gen_dev)
+    s16 = (tensor_scale_bits(k), tensor_scale_bits(v)) if kf == 3 else (0, 0)
     k_f = k.float().cpu().numpy().transpose(0, 2, 1, 3)
     v_f = v.float().cpu().numpy().transpose(0, 2, 1, 3)
     del k, v
+
+    def quant(x, grp, bits_o, sc):
+        if kf == 3:   # per-tensor: the per-head layout with every row's scale equal to sc
+            return (oracle.quantize_rows_tensor(x, sc),
+                    np.full(x.shape[:-1] + (1,), sc, np.uint16))
+        return oracle.quantize_rows(x, grp, bits_o)
+
     kc = np.zeros((w.batch, w.n_kv_heads, L, w.head_dim * kb // 8), np.uint8)
     vc = np.zeros((w.batch, w.n_kv_heads, L, w.head_dim * vb // 8), np.uint8)
-    ks = np.zeros((w.batch, w.n_kv_heads, L, w.head_dim // kg), np.uint16)
-    vs = np.zeros((w.batch, w.n_kv_heads, L, w.head_dim // vg), np.uint16)
-    a, b = oracle.quantize_rows(np.ascontiguousarray(k_f), kg, kb_o)
+    a, b = quant(np.ascontiguousarray(k_f), kg, kb_o, s16[0])
+    ks = np.zeros((w.batch, w.n_kv_heads, L) + b.shape[3:], np.uint16)
     kc[:, :, : L - 1], ks[:, :, : L - 1] = a, b
-    a, b = oracle.quantize_rows(np.ascontiguousarray(v_f), vg, vb_o)
+    a, b = quant(np.ascontiguousarray(v_f), vg, vb_o, s16[1])
+    vs = np.zeros((w.batch, w.n_kv_heads, L) + b.shape[3:], np.uint16)
     vc[:, :, : L - 1], vs[:, :, : L - 1] = a, b
     del k_f, v_f
     k1f = np.ascontiguousarray(k1.float().cpu().numpy().transpose(0, 2, 1, 3))
@@ -353,9 +374,9 @@ def cpu_oracle_layer(w, fmt, st=None, device=None, reps=1, budget_s=0.0):
     times = []
     while len(times) < reps or (sum(times) < budget_s and len(times) < 1000):
         t0 = time.perf_counter()
-        a, b = oracle.quantize_rows(k1f, kg, kb_o)
+        a, b = quant(k1f, kg, kb_o, s16[0])
         kc[:, :, L - 1:], ks[:, :, L - 1:] = a, b
-        a, b = oracle.quantize_rows(v1f, vg, vb_o)
+        a, b = quant(v1f, vg, vb_o, s16[1])
         vc[:, :, L - 1:], vs[:, :, L - 1:] = a, b
         oracle.decode_layer(qf, lens, kc, ks, kb_o, kg, vc, vs, vb_o, vg, w.n_kv_heads, 0.0, cores)
         times.append(time.perf_counter() - t0)
@@ -715,7 +736,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("kvq", "reference"), default="kvq")
     ap.add_argument("--workload", type=int, default=4)
-    ap.add_argument("--variants", default="K8V8,K8V4,K4V4,F8")
+    ap.add_argument("--variants", default="K8V8,K8V4,K4V4,F8,A8,T8")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--sections", default="kv,hmode,window,paged",

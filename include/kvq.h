@@ -76,8 +76,10 @@ enum kvq_mode {
 };
 
 enum kvq_format {
-    KVQ_FMT_INT = 0,   /* signed integer codes (INT8 / INT4)                       */
-    KVQ_FMT_E4M3 = 1   /* FP8 e4m3 codes, 8 bits                                   */
+    KVQ_FMT_INT = 0,    /* signed integer codes (INT8 / INT4), symmetric scales     */
+    KVQ_FMT_E4M3 = 1,   /* FP8 e4m3 codes, 8 bits                                   */
+    KVQ_FMT_ASYM = 2,   /* asymmetric INT8: uint8 codes, scale + zero-point         */
+    KVQ_FMT_TENSOR = 3  /* per-tensor INT8: one caller-set scale per K / V tensor   */
 };
 
 enum kvq_dtype {
@@ -122,18 +124,35 @@ typedef struct kvq_config {
                             page; capacity (a multiple of 128) is then the
                             logical tokens per sequence.  No sliding window.      */
     int32_t n_pages;     /* paged cache: pages in each layer's pool               */
-    int32_t kv_format;   /* KV mode: KVQ_FMT_INT (integer codes) or KVQ_FMT_E4M3:
-                            8-bit FP8 e4m3 codes for both keys and values (k_bits =
-                            v_bits = 8), scale s = fp16(absmax / 448) per group,
-                            code = e4m3_rne(x / s) saturating at 448, value =
-                            e4m3(code) * s ([MNI] "Comparison với production
-                            stack": FP8 KV caches of vLLM and TensorRT-LLM).      */
+    int32_t kv_format;   /* KV mode, k_bits = v_bits = 8 for every format but INT:
+                            KVQ_FMT_INT: symmetric integer codes (above).
+                            KVQ_FMT_E4M3: FP8 e4m3 codes, scale s = fp16(absmax /
+                            448) per group, code = e4m3_rne(x / s) saturating at
+                            448, value = e4m3(code) * s ([MNI] "Comparison với
+                            production stack": FP8 KV caches of vLLM and
+                            TensorRT-LLM).
+                            KVQ_FMT_ASYM: per group lo = min(0, min x), hi =
+                            max(0, max x), s = fp16((hi - lo) / 255), zero-point
+                            z = clamp(rne(-lo / s), 0, 255), code = clamp(rne(x /
+                            s) + z, 0, 255) stored as uint8, value = (code - z) *
+                            s; each group keeps the fp16 pair (s, z) ([MNI] "Tại
+                            sao INT8 mà không mất tốc": scale/zero-point metadata).
+                            KVQ_FMT_TENSOR: one fp16 scale s per K tensor and one
+                            per V tensor of a layer, set by the caller in
+                            k_scales[0] / v_scales[0] before the first append
+                            (e.g. from calibration) and never written by the
+                            library; code = clamp(rne(x / s), -127, 127), value =
+                            code * s ([MNI] "Limitations": symmetric per-tensor
+                            INT8); k_group = v_group = head_dim.                 */
 } kvq_config;
 
 /* One layer's cache buffers (device pointers, caller-owned).
  * KV mode:  k_codes  [B][Hkv][capacity][Dh*k_bits/8] bytes
  *           k_scales [B][Hkv][capacity][Dh/k_group] fp16   (NULL at 16 bits)
  *           v_codes / v_scales likewise with v_bits, v_group.
+ *           KVQ_FMT_ASYM: k_scales [B][Hkv][capacity][Dh/k_group][2] fp16
+ *           (scale, zero-point) pairs.  KVQ_FMT_TENSOR: k_scales and v_scales
+ *           each hold one fp16 scale (caller-set, 16-byte aligned).
  *           Paged (page_tokens 128): [n_pages][Hkv][128][...] for each of them,
  *           logical token t of sequence b at slot t % 128 of pool page
  *           block_table[b][t / 128].
@@ -157,7 +176,9 @@ typedef struct kvq_layer {
  * n_layers * max_seq_len.  Generalised here to separate K/V widths and
  * scale groups ([KS] 8K-token table):
  *   KV mode: sum over K and V of Hkv*Dh*bits/8 + Hkv*(Dh/group)*2 (no scale
- *            term at 16 bits);   h-mode: D*h_bits/8 + h_groups*2 (none at 16).
+ *            term at 16 bits; *4 with a zero-point (KVQ_FMT_ASYM); per-tensor
+ *            scales are no per-token term, 4 bytes per layer);
+ *   h-mode: D*h_bits/8 + h_groups*2 (none at 16).
  * Outputs (any may be NULL): bytes per token per layer, per layer
  * (x batch x capacity, or x n_pages x 128 for a paged cache) and total
  * (x n_layers).  Pure host function: no GPU needed.  Errors:

@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libkvq.so")
 
 KVQ_OK = 0
 KVQ_MODE_KV, KVQ_MODE_H = 0, 1
-KVQ_FMT_INT, KVQ_FMT_E4M3 = 0, 1
+KVQ_FMT_INT, KVQ_FMT_E4M3, KVQ_FMT_ASYM, KVQ_FMT_TENSOR = 0, 1, 2, 3
 KVQ_F16, KVQ_F32, KVQ_BF16 = 0, 1, 2
 
 EXPORTED = ("kvq_cache_bytes", "kvq_layer_buffer_bytes", "kvq_append", "kvq_workspace_bytes",
@@ -143,7 +143,8 @@ class Config:
     n_anchor: int = 0     # tokens kept at the start of the sequence
     page_tokens: int = 0  # 128: paged cache (a pool of n_pages pages, block table per layer)
     n_pages: int = 0
-    kv_format: int = 0    # KVQ_FMT_INT, or KVQ_FMT_E4M3 (FP8 e4m3 codes, k_bits = v_bits = 8)
+    kv_format: int = 0    # KVQ_FMT_INT; or, with k_bits = v_bits = 8, KVQ_FMT_E4M3 (FP8),
+    #                       KVQ_FMT_ASYM (zero-point) or KVQ_FMT_TENSOR (one scale per tensor)
 
     def _key(self):
         return (self.mode, self.batch, self.capacity, self.n_layers, self.n_q_heads,

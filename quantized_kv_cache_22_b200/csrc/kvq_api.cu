@@ -54,8 +54,10 @@ int check_cfg(const kvq_config *c)
         if (c->window == 0 && c->n_anchor != 0) return KVQ_ERR_INVALID_ARG;
         if (c->window > 0 && (int64_t)c->n_anchor + c->window != c->capacity)
             return KVQ_ERR_INVALID_ARG;
-        if (c->kv_format != KVQ_FMT_INT && c->kv_format != KVQ_FMT_E4M3) return KVQ_ERR_INVALID_ARG;
-        if (c->kv_format == KVQ_FMT_E4M3 && (c->k_bits != 8 || c->v_bits != 8))
+        if (c->kv_format < KVQ_FMT_INT || c->kv_format > KVQ_FMT_TENSOR) return KVQ_ERR_INVALID_ARG;
+        if (c->kv_format != KVQ_FMT_INT && (c->k_bits != 8 || c->v_bits != 8))
+            return KVQ_ERR_UNSUPPORTED;
+        if (c->kv_format == KVQ_FMT_TENSOR && (c->k_group != c->head_dim || c->v_group != c->head_dim))
             return KVQ_ERR_UNSUPPORTED;
         if (c->page_tokens != 0) {
             if (c->page_tokens != kPageTokens) return KVQ_ERR_UNSUPPORTED;
@@ -81,6 +83,13 @@ int check_cfg(const kvq_config *c)
 uint64_t tensor_row_bytes(int dim, int bits) { return (uint64_t)dim * bits / 8; }
 
 int scale_groups(int dim, int bits, int group) { return bits == 16 ? 0 : dim / group; }
+
+// fp16 values per (token, head) row in a KV-mode scale array
+int scale_row_vals(const kvq_config *c, int bits, int group)
+{
+    if (bits == 16 || c->kv_format == KVQ_FMT_TENSOR) return 0;
+    return scale_groups(c->head_dim, bits, group) * scale_vals(c->kv_format);
+}
 
 // ---------------------------------------------------------------- TMA encode
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -209,7 +218,7 @@ int current_device_props(int *sms, int *max_smem)
 // Shapes of the attention half (KV mode, or h-mode after reconstruction).
 struct AttnShape {
     int hkv, hq, G, dh, kb, vb, kg, vg, ngs_k, ngs_v;
-    bool f8;   // 8-bit codes are FP8 e4m3
+    int fmt;   // KVQ_FMT_* of the 8-bit codes
 };
 
 AttnShape attn_shape(const kvq_config *c)
@@ -224,13 +233,14 @@ AttnShape attn_shape(const kvq_config *c)
         s.vb = c->v_bits;
         s.kg = c->k_group;
         s.vg = c->v_group;
-        s.f8 = c->kv_format == KVQ_FMT_E4M3;
+        s.fmt = c->kv_format;
     } else {
         s.kb = s.vb = 16;
         s.kg = s.vg = s.dh;
     }
-    s.ngs_k = scale_groups(s.dh, s.kb, s.kg);
-    s.ngs_v = scale_groups(s.dh, s.vb, s.vg);
+    // fp16 values per (token, head) row of the scale arrays
+    s.ngs_k = c->mode == KVQ_MODE_KV ? scale_row_vals(c, s.kb, s.kg) : scale_groups(s.dh, s.kb, s.kg);
+    s.ngs_v = c->mode == KVQ_MODE_KV ? scale_row_vals(c, s.vb, s.vg) : scale_groups(s.dh, s.vb, s.vg);
     return s;
 }
 
@@ -243,7 +253,7 @@ int resolve_plan(const kvq_config *cfg, int32_t num_ctas, DecodeLaunch *plan, in
         int rc = current_device_props(&sms, &max_smem);
         if (rc) return rc;
     }
-    if (!plan_decode(a.dh, a.kb, a.vb, a.ngs_k, a.ngs_v, a.G, max_smem, plan, a.f8))
+    if (!plan_decode(a.dh, a.kb, a.vb, a.ngs_k, a.ngs_v, a.G, max_smem, plan, a.fmt))
         return KVQ_ERR_UNSUPPORTED;
     if (num_ctas > 0) {
         *ctas = num_ctas;
@@ -295,7 +305,7 @@ int kvq_cache_bytes(const kvq_config *cfg, uint64_t *per_token_layer, uint64_t *
         const int grp[2] = {cfg->k_group, cfg->v_group};
         for (int i = 0; i < 2; i++) {
             b += (uint64_t)cfg->n_kv_heads * tensor_row_bytes(cfg->head_dim, bits[i]);
-            b += (uint64_t)cfg->n_kv_heads * scale_groups(cfg->head_dim, bits[i], grp[i]) * 2;
+            b += (uint64_t)cfg->n_kv_heads * scale_row_vals(cfg, bits[i], grp[i]) * 2;
         }
     } else {
         b = tensor_row_bytes(cfg->d_model, cfg->h_bits);
@@ -303,7 +313,8 @@ int kvq_cache_bytes(const kvq_config *cfg, uint64_t *per_token_layer, uint64_t *
     }
     const uint64_t slots = cfg->page_tokens ? (uint64_t)cfg->n_pages * kPageTokens
                                             : (uint64_t)cfg->batch * (uint64_t)cfg->capacity;
-    const uint64_t layer = b * slots;
+    // per-tensor scales: one fp16 for K and one for V per layer
+    const uint64_t layer = b * slots + (cfg->mode == KVQ_MODE_KV && cfg->kv_format == KVQ_FMT_TENSOR ? 4 : 0);
     if (per_token_layer) *per_token_layer = b;
     if (per_layer) *per_layer = layer;
     if (total) *total = layer * (uint64_t)cfg->n_layers;
@@ -321,9 +332,10 @@ int kvq_layer_buffer_bytes(const kvq_config *cfg, uint64_t *k_codes, uint64_t *k
     if (cfg->mode == KVQ_MODE_KV) {
         const uint64_t hr = rows * cfg->n_kv_heads;
         kc = hr * tensor_row_bytes(cfg->head_dim, cfg->k_bits);
-        ks = hr * scale_groups(cfg->head_dim, cfg->k_bits, cfg->k_group) * 2;
+        ks = hr * scale_row_vals(cfg, cfg->k_bits, cfg->k_group) * 2;
         vc = hr * tensor_row_bytes(cfg->head_dim, cfg->v_bits);
-        vs = hr * scale_groups(cfg->head_dim, cfg->v_bits, cfg->v_group) * 2;
+        vs = hr * scale_row_vals(cfg, cfg->v_bits, cfg->v_group) * 2;
+        if (cfg->kv_format == KVQ_FMT_TENSOR) ks = vs = 2;   // one fp16 scale each
     } else {
         kc = rows * tensor_row_bytes(cfg->d_model, cfg->h_bits);
         ks = cfg->h_bits == 16 ? 0 : rows * (uint64_t)cfg->h_groups * 2;
@@ -350,7 +362,7 @@ int kvq_append(const kvq_config *cfg, const kvq_layer *layer, const void *k, con
     AppendParams pk{};
     pk.window = cfg->window;
     pk.n_anchor = cfg->n_anchor;
-    pk.e4m3 = cfg->mode == KVQ_MODE_KV && cfg->kv_format == KVQ_FMT_E4M3;
+    pk.fmt = cfg->mode == KVQ_MODE_KV ? cfg->kv_format : KVQ_FMT_INT;
     if (cfg->mode == KVQ_MODE_KV && cfg->page_tokens) {
         if (!layer->block_table) return KVQ_ERR_INVALID_ARG;
         pk.block_table = layer->block_table;
@@ -463,7 +475,8 @@ static int decode_kv_layout(const kvq_config *cfg, const void *k_codes, const vo
 {
     const AttnShape a = attn_shape(cfg);
     // fp16 and e4m3 keys use an f16 MMA whose f32 / bf16 queries take two columns per head
-    if ((a.kb == 16 || a.f8) && q_dtype != KVQ_F16 && a.G > 4) return KVQ_ERR_UNSUPPORTED;
+    if ((a.kb == 16 || a.fmt == KVQ_FMT_E4M3) && q_dtype != KVQ_F16 && a.G > 4)
+        return KVQ_ERR_UNSUPPORTED;
     DecodeLaunch plan;
     int ctas = 0;
     int rc = resolve_plan(cfg, num_ctas, &plan, &ctas);

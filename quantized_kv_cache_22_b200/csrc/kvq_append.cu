@@ -55,9 +55,11 @@ __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ App
         cache_row = ((int64_t)b * p.rows_per_tok + head) * p.cap + slot;
     }
     uint8_t *codes_row = p.codes + cache_row * ((int64_t)dim * p.bits / 8);
-    __half *scales_row = p.bits == 16 ? nullptr : p.scales + cache_row * (dim / p.group);
+    __half *scales_row = p.bits == 16            ? nullptr
+                         : p.fmt == KVQ_FMT_TENSOR ? p.scales   // the tensor's one scale
+                                                   : p.scales + cache_row * (dim / p.group) * scale_vals(p.fmt);
     quantize_row(p.x, row * (int64_t)dim, p.in_dtype, dim, p.bits, p.group, codes_row, scales_row,
-                 lane, p.e4m3 != 0);
+                 lane, p.fmt);
 }
 
 }  // namespace

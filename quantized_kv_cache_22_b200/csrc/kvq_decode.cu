@@ -56,11 +56,11 @@ __global__ void __launch_bounds__(256) merge_kernel(const MergeParams p)
     merge_segment<DH>(p.ws, cmin + bh, (int)(cmax - cmin + 1), G, p.out, p.out_f32, obase0, lane);
 }
 
-void *pick_decode(int dh, int kb, int vb, bool kg, bool vg, bool f8)
+void *pick_decode(int dh, int kb, int vb, bool kg, bool vg, int fmt)
 {
     if (kb == 16) kg = false;
     if (vb == 16) vg = false;
-    if (f8) return (kb == 8 && vb == 8) ? decode_fn_f8(dh, kg, vg) : nullptr;
+    if (fmt != KVQ_FMT_INT) return (kb == 8 && vb == 8) ? decode_fn_fmt(dh, fmt, kg, vg) : nullptr;
     switch (kb) {
     case 4: return decode_fn_kb4(dh, vb, kg, vg);
     case 8: return decode_fn_kb8(dh, vb, kg, vg);
@@ -74,13 +74,16 @@ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 }  // namespace
 
 bool plan_decode(int dh, int kb, int vb, int ngs_k, int ngs_v, int G, int max_smem,
-                 DecodeLaunch *plan, bool f8)
+                 DecodeLaunch *plan, int fmt)
 {
-    const bool kg = kb != 16 && ngs_k > 1, vg = vb != 16 && ngs_v > 1;
-    if (!pick_decode(dh, kb, vb, kg, vg, f8)) return false;
+    // ngs_k / ngs_v: fp16 values per row in the scale arrays (a pair per group with
+    // a zero-point; none for 16-bit or per-tensor codes)
+    const int sv = scale_vals(fmt);
+    const bool kg = kb != 16 && ngs_k / sv > 1, vg = vb != 16 && ngs_v / sv > 1;
+    if (!pick_decode(dh, kb, vb, kg, vg, fmt)) return false;
     const uint32_t rk = dh * kb / 8, rv = dh * vb / 8;
     DecodeLaunch L{};
-    L.dh = dh; L.kb = kb; L.vb = vb; L.kg = kg; L.vg = vg; L.f8 = f8;
+    L.dh = dh; L.kb = kb; L.vb = vb; L.kg = kg; L.vg = vg; L.fmt = fmt;
     L.off_v = align_up(T * rk, 1024);
     L.off_sk = L.off_v + align_up(T * rv, 1024);
     L.off_sv = L.off_sk + align_up(T * (kb == 16 ? 0 : ngs_k) * 2, 16);
@@ -165,14 +168,14 @@ cudaError_t prepare_fn(void *fn, size_t smem, int *occupancy)
 
 cudaError_t decode_occupancy(const DecodeLaunch &plan, int *ctas_per_sm)
 {
-    return prepare_fn(pick_decode(plan.dh, plan.kb, plan.vb, plan.kg, plan.vg, plan.f8), plan.smem_bytes,
+    return prepare_fn(pick_decode(plan.dh, plan.kb, plan.vb, plan.kg, plan.vg, plan.fmt), plan.smem_bytes,
                       ctas_per_sm);
 }
 
 cudaError_t launch_decode(const DecodeLaunch &plan, const DecodeParams &p, const CUtensorMap &tm_k,
                           const CUtensorMap &tm_v, cudaStream_t stream)
 {
-    void *fn = pick_decode(plan.dh, plan.kb, plan.vb, plan.kg, plan.vg, plan.f8);
+    void *fn = pick_decode(plan.dh, plan.kb, plan.vb, plan.kg, plan.vg, plan.fmt);
     cudaError_t e = prepare_fn(fn, plan.smem_bytes, nullptr);
     if (e != cudaSuccess) return e;
     void *args[] = {const_cast<CUtensorMap *>(&tm_k), const_cast<CUtensorMap *>(&tm_v),

@@ -7,7 +7,7 @@ namespace {
 template <int DH, int VB, bool KG, bool VG>
 void *fn()
 {
-    return reinterpret_cast<void *>(&decode_kernel<DH, 16, VB, KG, VG, false>);
+    return reinterpret_cast<void *>(&decode_kernel<DH, 16, VB, KG, VG, KVQ_FMT_INT>);
 }
 
 template <int DH, int VB, bool KG>

@@ -292,12 +292,17 @@ __device__ __forceinline__ void merge_segment(const float *ws, int64_t slot0, in
 
 // KG / VG: keys / values carry one scale per 32/64-element group (else one per
 // (token, head)); compile-time so the per-head case keeps no per-group state.
-// F8: the 8-bit codes of keys and values are FP8 e4m3 (KB = VB = 8).
-template <int DH, int KB, int VB, bool KG, bool VG, bool F8>
+// FMT: the code format of 8-bit keys and values (KVQ_FMT_*; KB = VB = 8 unless
+// KVQ_FMT_INT): symmetric integer, FP8 e4m3, asymmetric (uint8 codes with a
+// zero-point) or per-tensor (one fixed scale per tensor).
+template <int DH, int KB, int VB, bool KG, bool VG, int FMT>
 __global__ void __launch_bounds__(NTHR, 2)
     decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const __grid_constant__ DecodeParams p)
 {
+    constexpr bool F8 = FMT == KVQ_FMT_E4M3;   // e4m3 codes
+    constexpr bool ZP = FMT == KVQ_FMT_ASYM;   // uint8 codes, (scale, zero-point) per group
+    constexpr bool PT = FMT == KVQ_FMT_TENSOR; // one scale per tensor, no per-token scales
     constexpr int NG = DH / 32;                // 32-element blocks along head_dim
     constexpr int RK = DH * KB / 8;            // bytes per key row
     constexpr int RV = DH * VB / 8;
@@ -318,10 +323,14 @@ __global__ void __launch_bounds__(NTHR, 2)
     constexpr bool KWIDE = !KG && KB != 16 && RK >= 64 && !F8;
     constexpr int KLW = KWIDE ? 16 : SK / 4;          // key bytes per lane per row and load
     constexpr int KPL = KWIDE ? 16 * 8 / KB / 8 : 1;  // 32-element blocks per load
-    // value codes enter the P.V MMA as (bias + code): 1152 at 8 bits, per row at 4
-    // bits (see the segment end); fp16 and e4m3 values convert exactly, no bias
-    constexpr float BIAS_V = (VB == 8 && !F8) ? 1152.f : 0.f;
+    // value codes enter the P.V MMA as (bias + code): 1152 + code at 8 bits (1024
+    // + code for uint8 codes), per row at 4 bits (see the segment end); fp16 and
+    // e4m3 values convert exactly, no bias.  psum = sum of P (times the bias),
+    // from an MMA of P against a constant matrix (ones; 1024 + zero-point for
+    // uint8 codes, so that the zero-point comes off with the bias).
+    constexpr float BIAS_V = (VB == 8 && !F8) ? (ZP ? 1.f : 1152.f) : 0.f;
     constexpr bool VBIAS = VB == 4 || (VB == 8 && !F8);
+    constexpr uint32_t VX = ZP ? 0x64006400u : 0x64806480u;   // byte -> fp16 1024 + byte (^0x80)
     // The running max is only raised when a tile beats it by more than 2^LAZY;
     // weights p * s_V then stay below 2^LAZY, well inside fp16.
     constexpr float LAZY = 8.f;
@@ -483,12 +492,17 @@ __global__ void __launch_bounds__(NTHR, 2)
                 page = min(max(page, 0), p.n_pages - 1);
                 crow = ((int64_t)page * Hkv + akvh) * T + aslot % T;
             }
+            constexpr int SCV = scale_vals(FMT);
             quantize_row(p.app.k_new, (int64_t)bh * DH, p.app.dtype, DH, KB, p.app.k_group,
                          p.app.k_codes + crow * RK,
-                         KB == 16 ? nullptr : p.app.k_scales + crow * (DH / p.app.k_group), lane, F8);
+                         KB == 16 ? nullptr
+                         : PT     ? p.app.k_scales
+                                  : p.app.k_scales + crow * (DH / p.app.k_group) * SCV, lane, FMT);
             quantize_row(p.app.v_new, (int64_t)bh * DH, p.app.dtype, DH, VB, p.app.v_group,
                          p.app.v_codes + crow * RV,
-                         VB == 16 ? nullptr : p.app.v_scales + crow * (DH / p.app.v_group), lane, F8);
+                         VB == 16 ? nullptr
+                         : PT     ? p.app.v_scales
+                                  : p.app.v_scales + crow * (DH / p.app.v_group) * SCV, lane, FMT);
             // order the writes before the copy engine reads the tile
             fence_proxy_async_global();
             __syncwarp();
@@ -552,8 +566,8 @@ __global__ void __launch_bounds__(NTHR, 2)
                 uint8_t *st = smem + (size_t)s * p.stage_bytes;
                 const int n_s = min(T, zcap - y0);
                 uint32_t bytes = (uint32_t)(T * RK + T * RV);
-                if (KB != 16) bytes += (uint32_t)(n_s * p.ngs_k * 2);
-                if (VB != 16) bytes += (uint32_t)(n_s * p.ngs_v * 2);
+                if (KB != 16 && !PT) bytes += (uint32_t)(n_s * p.ngs_k * 2);
+                if (VB != 16 && !PT) bytes += (uint32_t)(n_s * p.ngs_v * 2);
                 mbar_arrive_expect_tx(&full[s], bytes);
                 if constexpr (RK <= 128) {
                     tma_load_3d_hint(st, &tm_k, &full[s], 0, y0 / (128 / RK), z, pol);
@@ -567,10 +581,10 @@ __global__ void __launch_bounds__(NTHR, 2)
                     tma_load_3d_hint(st + p.off_v, &tm_v, &full[s], 0, y0, z, pol);
                     tma_load_3d_hint(st + p.off_v + T * 128, &tm_v, &full[s], 128, y0, z, pol);
                 }
-                if (KB != 16)
+                if (KB != 16 && !PT)
                     bulk_load_hint(st + p.off_sk, p.k_scales + ((int64_t)z * zcap + y0) * p.ngs_k,
                                    (uint32_t)(n_s * p.ngs_k * 2), &full[s], pol);
-                if (VB != 16)
+                if (VB != 16 && !PT)
                     bulk_load_hint(st + p.off_sv, p.v_scales + ((int64_t)z * zcap + y0) * p.ngs_v,
                                    (uint32_t)(n_s * p.ngs_v * 2), &full[s], pol);
             }
@@ -731,6 +745,10 @@ __global__ void __launch_bounds__(NTHR, 2)
 
     uint32_t qh[NG][2], ql[NG][2];      // int8 query B-fragments (hi / lo parts) per block
     float sqc[2];                       // score factor of columns 2tig, 2tig+1
+    // uint8 keys with a zero-point z: q.(c - z) = q.c - z * sum(q), with sum(q) in
+    // the hi/lo units of the MMA (254 sum(hi) + sum(lo)), per head (columns 2tig,
+    // 2tig+1) and per 32-element block when the key scales are grouped
+    int zq[KG ? NG : 1][2];
     uint32_t qb[NG][2][2];              // fp16 query B-fragments (fp16 keys)
     float m_run[2], l_run[2];
     float psum[NVG][4];                 // sum of fp16 p*s_V per value group (cols in [0], [1])
@@ -761,14 +779,29 @@ __global__ void __launch_bounds__(NTHR, 2)
             amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 2));
             const float inv = amax > 0.f ? 127.f / amax : 0.f;
 #pragma unroll
+            int qs_all = 0;
+#pragma unroll
             for (int blk = 0; blk < NG; blk++) {
                 int hi[8], lo[8];
+                int qs_blk = 0;
 #pragma unroll
                 for (int j = 0; j < 8; j++) {
                     const float y = x[blk][j] * inv;
                     const float r = rintf(y);
                     hi[j] = (int)r;
                     lo[j] = __float2int_rn((y - r) * 254.f);
+                    qs_blk += 254 * hi[j] + lo[j];
+                }
+                if constexpr (ZP) {
+                    if constexpr (KG) {
+                        // the block's 32 elements sit in the 4 lanes of the head
+                        qs_blk += __shfl_xor_sync(FULL, qs_blk, 1);
+                        qs_blk += __shfl_xor_sync(FULL, qs_blk, 2);
+                        zq[blk][0] = __shfl_sync(FULL, qs_blk, (2 * tig) * 4);
+                        zq[blk][1] = __shfl_sync(FULL, qs_blk, (2 * tig + 1) * 4);
+                    } else {
+                        qs_all += qs_blk;
+                    }
                 }
                 if constexpr (KB == 8) {
                     // k-slot 4tig+i <-> element 8tig+i, 16+4tig+i <-> 8tig+4+i
@@ -783,6 +816,12 @@ __global__ void __launch_bounds__(NTHR, 2)
                     ql[blk][0] = pack_bytes(lo[0], lo[2], lo[4], lo[6]);
                     ql[blk][1] = pack_bytes(lo[1], lo[3], lo[5], lo[7]);
                 }
+            }
+            if constexpr (ZP && !KG) {
+                qs_all += __shfl_xor_sync(FULL, qs_all, 1);
+                qs_all += __shfl_xor_sync(FULL, qs_all, 2);
+                zq[0][0] = __shfl_sync(FULL, qs_all, (2 * tig) * 4);
+                zq[0][1] = __shfl_sync(FULL, qs_all, (2 * tig + 1) * 4);
             }
             // 4-bit key codes enter the MMA as 16 * code
             const float f = amax * (1.f / (127.f * 254.f)) * p.tau_log2e * (KB == 4 ? 0.0625f : 1.f);
@@ -849,6 +888,9 @@ __global__ void __launch_bounds__(NTHR, 2)
 
     const uint64_t limit = p.timeout_ns;
     const uint32_t ONE2 = 0x3C003C00u;   // half2(1, 1)
+    // per-tensor scales (caller-set, read once)
+    const float k_tensor = PT ? __half2float(p.k_scales[0]) : 0.f;
+    const float v_tensor = PT ? __half2float(p.v_scales[0]) : 0.f;
     int s = 0;
     uint32_t ph = 0;
     uint32_t nseg = 0;           // segment ends handed to the combiner
@@ -926,8 +968,8 @@ __global__ void __launch_bounds__(NTHR, 2)
                                     fa[0] = (w0 << 4) & 0xF0F0F0F0u; fa[1] = (w1 << 4) & 0xF0F0F0F0u;
                                     fa[2] = w0 & 0xF0F0F0F0u;        fa[3] = w1 & 0xF0F0F0F0u;
                                 }
-                                imma_16832(ah[u], fa[0], fa[1], fa[2], fa[3], qh[blk][0], qh[blk][1]);
-                                imma_16832(al[u], fa[0], fa[1], fa[2], fa[3], ql[blk][0], ql[blk][1]);
+                                imma_16832<ZP>(ah[u], fa[0], fa[1], fa[2], fa[3], qh[blk][0], qh[blk][1]);
+                                imma_16832<ZP>(al[u], fa[0], fa[1], fa[2], fa[3], ql[blk][0], ql[blk][1]);
                             }
                         }
                     }
@@ -945,18 +987,33 @@ __global__ void __launch_bounds__(NTHR, 2)
                                   sst + blk_addr<RK, SK>(kofs[1][1], blk), fa[1]);
 #pragma unroll
                     for (int u = 0; u < 2; u++) {
-                        imma_16832(ah[u], fa[u][0], fa[u][1], fa[u][2], fa[u][3], qh[blk][0], qh[blk][1]);
-                        imma_16832(al[u], fa[u][0], fa[u][1], fa[u][2], fa[u][3], ql[blk][0], ql[blk][1]);
+                        imma_16832<ZP>(ah[u], fa[u][0], fa[u][1], fa[u][2], fa[u][3], qh[blk][0], qh[blk][1]);
+                        imma_16832<ZP>(al[u], fa[u][0], fa[u][1], fa[u][2], fa[u][3], ql[blk][0], ql[blk][1]);
                     }
                 }
                 }
 #pragma unroll
                 for (int u = 0; u < 2; u++) {
-                    const float2 kk = unpack_half2(lds_u32(sbase, ssk + 2 * tAu[u]));
+                    float2 kk;
+                    int z0 = 0, z1 = 0;   // zero-points of the two score rows
+                    if constexpr (PT) {
+                        kk = make_float2(k_tensor, k_tensor);
+                    } else if constexpr (ZP) {
+                        // (scale, zero-point) of tokens tA, tA + 1
+                        const uint2 w = lds_u64(sbase, ssk + 4 * tAu[u]);
+                        kk = make_float2(__half2float(__ushort_as_half((unsigned short)(w.x & 0xFFFFu))),
+                                         __half2float(__ushort_as_half((unsigned short)(w.y & 0xFFFFu))));
+                        z0 = __half2int_rn(__ushort_as_half((unsigned short)(w.x >> 16)));
+                        z1 = __half2int_rn(__ushort_as_half((unsigned short)(w.y >> 16)));
+                    } else {
+                        kk = unpack_half2(lds_u32(sbase, ssk + 2 * tAu[u]));
+                    }
 #pragma unroll
                     for (int e = 0; e < 4; e++) {
                         const float ks = (e < 2) ? kk.x : kk.y;
-                        s2[u][e] = (float)(ah[u][e] * 254 + al[u][e]) * (ks * sqc[e & 1]);
+                        int a = ah[u][e] * 254 + al[u][e];
+                        if constexpr (ZP) a -= ((e < 2) ? z0 : z1) * zq[0][e & 1];
+                        s2[u][e] = (float)a * (ks * sqc[e & 1]);
                     }
                 }
             } else {
@@ -970,16 +1027,29 @@ __global__ void __launch_bounds__(NTHR, 2)
                         uint32_t fa[4];
                         key_frags(Imm0{}, sst + blk_addr<RK, SK>(kofs[u][0], blk),
                                   sst + blk_addr<RK, SK>(kofs[u][1], blk), fa);
-                        imma_16832(ah, fa[0], fa[1], fa[2], fa[3], qh[blk][0], qh[blk][1]);
-                        imma_16832(al, fa[0], fa[1], fa[2], fa[3], ql[blk][0], ql[blk][1]);
-                        const float k0 = __half2float(__ushort_as_half(
-                            (unsigned short)lds_u16(sbase, ssk + 2 * (tA * p.ngs_k + (blk >> p.kshift)))));
-                        const float k1 = __half2float(__ushort_as_half(
-                            (unsigned short)lds_u16(sbase, ssk + 2 * ((tA + 1) * p.ngs_k + (blk >> p.kshift)))));
-                        v[0] = fmaf(k0, (float)(ah[0] * 254 + al[0]), v[0]);
-                        v[1] = fmaf(k0, (float)(ah[1] * 254 + al[1]), v[1]);
-                        v[2] = fmaf(k1, (float)(ah[2] * 254 + al[2]), v[2]);
-                        v[3] = fmaf(k1, (float)(ah[3] * 254 + al[3]), v[3]);
+                        imma_16832<ZP>(ah, fa[0], fa[1], fa[2], fa[3], qh[blk][0], qh[blk][1]);
+                        imma_16832<ZP>(al, fa[0], fa[1], fa[2], fa[3], ql[blk][0], ql[blk][1]);
+                        constexpr int SCV = scale_vals(FMT);
+                        const uint32_t o0 = ssk + 2 * (tA * p.ngs_k + SCV * (blk >> p.kshift));
+                        const uint32_t o1 = ssk + 2 * ((tA + 1) * p.ngs_k + SCV * (blk >> p.kshift));
+                        const float k0 = __half2float(__ushort_as_half((unsigned short)lds_u16(sbase, o0)));
+                        const float k1 = __half2float(__ushort_as_half((unsigned short)lds_u16(sbase, o1)));
+                        if constexpr (ZP) {
+                            // minus zero-point x the block's query sum
+                            const int z0 = __half2int_rn(__ushort_as_half((unsigned short)lds_u16(sbase, o0 + 2)));
+                            const int z1 = __half2int_rn(__ushort_as_half((unsigned short)lds_u16(sbase, o1 + 2)));
+                            ah[0] = ah[0] * 254 + al[0] - z0 * zq[blk][0];
+                            ah[1] = ah[1] * 254 + al[1] - z0 * zq[blk][1];
+                            ah[2] = ah[2] * 254 + al[2] - z1 * zq[blk][0];
+                            ah[3] = ah[3] * 254 + al[3] - z1 * zq[blk][1];
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 4; e++) ah[e] = ah[e] * 254 + al[e];
+                        }
+                        v[0] = fmaf(k0, (float)ah[0], v[0]);
+                        v[1] = fmaf(k0, (float)ah[1], v[1]);
+                        v[2] = fmaf(k1, (float)ah[2], v[2]);
+                        v[3] = fmaf(k1, (float)ah[3], v[3]);
                     }
 #pragma unroll
                     for (int e = 0; e < 4; e++) s2[u][e] = v[e] * sqc[e & 1];
@@ -1107,22 +1177,58 @@ __global__ void __launch_bounds__(NTHR, 2)
         // ---------------- phase 2: value scales of the score rows -----------------
         float sv[2][2][NVG];   // [sub-tile][row][value group]
         float lsv[2][2];
+        // uint8 values: A fragments half2(1024 + z) of the P.V k-slot tokens (tw + vA,
+        // tw + vB; tw + vA + 1, tw + vB + 1), zero past the length (stale scales)
+        uint32_t za[2][NVG][2];
 #pragma unroll
         for (int u = 0; u < 2; u++) {
             const int tA = tAu[u];
+            constexpr int SCV = scale_vals(FMT);
             if constexpr (VB == 16) {
                 sv[u][0][0] = sv[u][1][0] = 1.f;
+            } else if constexpr (PT) {
+                sv[u][0][0] = sv[u][1][0] = v_tensor;
             } else if constexpr (!vgrp) {
-                const float2 vv = unpack_half2(lds_u32(sbase, ssv + 2 * tA));
-                sv[u][0][0] = vv.x;
-                sv[u][1][0] = vv.y;
+                if constexpr (ZP) {
+                    const uint2 w = lds_u64(sbase, ssv + 4 * tA);
+                    sv[u][0][0] = __half2float(__ushort_as_half((unsigned short)(w.x & 0xFFFFu)));
+                    sv[u][1][0] = __half2float(__ushort_as_half((unsigned short)(w.y & 0xFFFFu)));
+                } else {
+                    const float2 vv = unpack_half2(lds_u32(sbase, ssv + 2 * tA));
+                    sv[u][0][0] = vv.x;
+                    sv[u][1][0] = vv.y;
+                }
             } else {
 #pragma unroll
                 for (int g = 0; g < NG; g++) {
                     sv[u][0][g] = __half2float(__ushort_as_half(
-                        (unsigned short)lds_u16(sbase, ssv + 2 * (tA * p.ngs_v + (g >> p.vshift)))));
+                        (unsigned short)lds_u16(sbase, ssv + 2 * (tA * p.ngs_v + SCV * (g >> p.vshift)))));
                     sv[u][1][g] = __half2float(__ushort_as_half(
-                        (unsigned short)lds_u16(sbase, ssv + 2 * ((tA + 1) * p.ngs_v + (g >> p.vshift)))));
+                        (unsigned short)lds_u16(sbase, ssv + 2 * ((tA + 1) * p.ngs_v + SCV * (g >> p.vshift)))));
+                }
+            }
+            if constexpr (ZP) {
+                const int tw = warp * 32 + u * 16;
+                const int rem = m.len - m.t0 - tw;   // valid tokens of the sub-tile
+                const uint32_t mlo = (vA < rem ? 0x0000FFFFu : 0u) | (vB < rem ? 0xFFFF0000u : 0u);
+                const uint32_t mhi = (vA + 1 < rem ? 0x0000FFFFu : 0u) | (vB + 1 < rem ? 0xFFFF0000u : 0u);
+                const uint32_t B1024 = 0x64006400u;   // half2(1024, 1024)
+                if constexpr (!vgrp) {
+                    const uint2 wA = lds_u64(sbase, ssv + 4 * (tw + vA));   // (s, z) of tw+vA, tw+vA+1
+                    const uint2 wB = lds_u64(sbase, ssv + 4 * (tw + vB));
+                    za[u][0][0] = hadd2_u32(prmt(wA.x, wB.x, 0x7632u) & mlo, B1024);
+                    za[u][0][1] = hadd2_u32(prmt(wA.y, wB.y, 0x7632u) & mhi, B1024);
+                } else {
+#pragma unroll
+                    for (int g = 0; g < NG; g++) {
+                        const uint32_t zo = 2 * (SCV * (g >> p.vshift) + 1);
+                        const uint32_t a0 = lds_u16(sbase, ssv + 2 * (tw + vA) * p.ngs_v + zo);
+                        const uint32_t b0 = lds_u16(sbase, ssv + 2 * (tw + vB) * p.ngs_v + zo);
+                        const uint32_t a1 = lds_u16(sbase, ssv + 2 * (tw + vA + 1) * p.ngs_v + zo);
+                        const uint32_t b1 = lds_u16(sbase, ssv + 2 * (tw + vB + 1) * p.ngs_v + zo);
+                        za[u][g][0] = hadd2_u32((a0 | (b0 << 16)) & mlo, B1024);
+                        za[u][g][1] = hadd2_u32((a1 | (b1 << 16)) & mhi, B1024);
+                    }
                 }
             }
             // scales past the length may be stale shared memory: never use them
@@ -1194,7 +1300,10 @@ __global__ void __launch_bounds__(NTHR, 2)
                 pb[u][g][0] = movmatrix_trans(x0);
                 pb[u][g][1] = movmatrix_trans(x1);
                 // column sums of the fp16 weights, for the code bias
-                if constexpr (VBIAS)
+                if constexpr (ZP)
+                    mma_16816(psum[g], za[u][g][0], za[u][g][0], za[u][g][1], za[u][g][1], pb[u][g][0],
+                              pb[u][g][1]);
+                else if constexpr (VBIAS)
                     mma_16816(psum[g], ONE2, ONE2, ONE2, ONE2, pb[u][g][0], pb[u][g][1]);
             }
         }
@@ -1245,10 +1354,10 @@ __global__ void __launch_bounds__(NTHR, 2)
                             const uint32_t A = j < 2 ? w[0].x : w[0].y, Bw = j < 2 ? w[1].x : w[1].y;
                             const uint32_t C = j < 2 ? w[2].x : w[2].y, E = j < 2 ? w[3].x : w[3].y;
                             const uint32_t yAB = prmt(A, Bw, sel), yCE = prmt(C, E, sel);
-                            const uint32_t a0 = and_xor(yAB, 0x00FF00FFu, 0x64806480u);
-                            const uint32_t a1 = and_xor(yAB >> 8, 0x00FF00FFu, 0x64806480u);
-                            const uint32_t a2 = and_xor(yCE, 0x00FF00FFu, 0x64806480u);
-                            const uint32_t a3 = and_xor(yCE >> 8, 0x00FF00FFu, 0x64806480u);
+                            const uint32_t a0 = and_xor(yAB, 0x00FF00FFu, VX);
+                            const uint32_t a1 = and_xor(yAB >> 8, 0x00FF00FFu, VX);
+                            const uint32_t a2 = and_xor(yCE, 0x00FF00FFu, VX);
+                            const uint32_t a3 = and_xor(yCE >> 8, 0x00FF00FFu, VX);
                             mma_16816(o_acc[4 * sb + j], a0, a1, a2, a3, b0, b1);
                         }
                     } else if constexpr (VB == 4) {
@@ -1342,10 +1451,10 @@ __global__ void __launch_bounds__(NTHR, 2)
                     for (int h = 0; h < 2; h++) {
                         const uint32_t sel = h ? 0x7632u : 0x5410u;
                         const uint32_t yAB = prmt(wA, wB, sel), yCE = prmt(wC, wE, sel);
-                        const uint32_t a0 = and_xor(yAB, 0x00FF00FFu, 0x64806480u);
-                        const uint32_t a1 = and_xor(yAB >> 8, 0x00FF00FFu, 0x64806480u);
-                        const uint32_t a2 = and_xor(yCE, 0x00FF00FFu, 0x64806480u);
-                        const uint32_t a3 = and_xor(yCE >> 8, 0x00FF00FFu, 0x64806480u);
+                        const uint32_t a0 = and_xor(yAB, 0x00FF00FFu, VX);
+                        const uint32_t a1 = and_xor(yAB >> 8, 0x00FF00FFu, VX);
+                        const uint32_t a2 = and_xor(yCE, 0x00FF00FFu, VX);
+                        const uint32_t a3 = and_xor(yCE >> 8, 0x00FF00FFu, VX);
                         mma_16816(o_acc[2 * blk + h], a0, a1, a2, a3, b0, b1);
                     }
                 } else if constexpr (VB == 4) {

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
 
+#include "../../include/kvq.h"
+
 namespace kvq {
 
 // ------------------------------------------------------------------ append
@@ -12,12 +14,13 @@ struct AppendParams {
     const void *x;          // [B][n_new][rows_per_tok][dim] input
     const int32_t *d_pos;   // [B]
     uint8_t *codes;         // [B][rows_per_tok][cap][row_bytes]
-    __half *scales;         // [B][rows_per_tok][cap][dim/group] (unused at 16 bits)
+    __half *scales;         // [B][rows_per_tok][cap][dim/group] (unused at 16 bits; pairs
+                            // (scale, zero-point) when asymmetric; one scale when per-tensor)
     int32_t in_dtype;       // KVQ_F16 / KVQ_F32 / KVQ_BF16
     int32_t batch, n_new, rows_per_tok, dim, cap;
     int32_t bits, group;
     int32_t window, n_anchor;   // sliding window (0: slot = position)
-    int32_t e4m3;               // 8-bit codes are FP8 e4m3
+    int32_t fmt;                // KVQ_FMT_*: integer, e4m3, asymmetric or per-tensor codes
     const int32_t *block_table; // paged cache: [batch][max_pages] pool page of each logical page
     int32_t max_pages, n_pages; // (rows_per_tok is the KV heads; pages hold kPageTokens rows)
 };
@@ -50,6 +53,9 @@ struct FusedAppend {
     int32_t dtype;                // KVQ_F16 / KVQ_F32 / KVQ_BF16
     int32_t k_group, v_group;     // elements per scale (32 at 16 bits)
 };
+
+// fp16 values per scale group in the scale arrays of a code format
+__host__ __device__ constexpr int scale_vals(int fmt) { return fmt == KVQ_FMT_ASYM ? 2 : 1; }
 
 struct DecodeParams {
     const int32_t *d_len;     // [B]
@@ -88,7 +94,7 @@ struct MergeParams {
 struct DecodeLaunch {
     int dh, kb, vb;
     bool kg, vg;              // grouped key / value scales
-    bool f8;                  // 8-bit codes are FP8 e4m3
+    int fmt;                  // KVQ_FMT_* of the 8-bit codes
     size_t smem_bytes;
     int stages;
     uint32_t stage_bytes, off_v, off_sk, off_sv, off_meta, off_bar, off_merge;
@@ -100,11 +106,12 @@ struct DecodeLaunch {
 void *decode_fn_kb4(int dh, int vb, bool kg, bool vg);
 void *decode_fn_kb8(int dh, int vb, bool kg, bool vg);
 void *decode_fn_kb16(int dh, int vb, bool kg, bool vg);
-void *decode_fn_f8(int dh, bool kg, bool vg);   // FP8 e4m3 keys and values (kvq_decode_f8.cu)
+// e4m3, asymmetric and per-tensor 8-bit keys and values (kvq_decode_fmt.cu)
+void *decode_fn_fmt(int dh, int fmt, bool kg, bool vg);
 
 // Fill in the shared-memory plan; returns false if the shape is unsupported.
 bool plan_decode(int dh, int kb, int vb, int ngs_k, int ngs_v, int G, int max_smem,
-                 DecodeLaunch *plan, bool f8 = false);
+                 DecodeLaunch *plan, int fmt = 0);
 cudaError_t decode_occupancy(const DecodeLaunch &plan, int *ctas_per_sm);
 cudaError_t launch_decode(const DecodeLaunch &plan, const DecodeParams &p, const CUtensorMap &tm_k,
                           const CUtensorMap &tm_v, cudaStream_t stream);

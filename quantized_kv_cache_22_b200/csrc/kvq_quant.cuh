@@ -44,13 +44,20 @@ __device__ __forceinline__ void load4(const void *base, int64_t idx, int dtype, 
 // Scale s = fp16(absmax / qmax) with qmax 127 (8 bits) or 7 (4 bits), an
 // overflow to +inf saturating to 65504; code = clamp(rne(x / s), -qmax, qmax),
 // all codes 0 when s = 0.  4-bit element 2j sits in the low nibble of byte j.
-// e4m3 (8 bits): s = fp16(absmax / 448) and code = e4m3(x / s), rounded to
-// nearest even and saturating at 448.
+// fmt (8 bits only, else KVQ_FMT_INT):
+//   KVQ_FMT_E4M3: s = fp16(absmax / 448) and code = e4m3(x / s), rounded to
+//     nearest even and saturating at 448.
+//   KVQ_FMT_ASYM: lo = min(0, min x), hi = max(0, max x), s = fp16((hi - lo) / 255),
+//     z = clamp(rne(-lo / s), 0, 255), code = clamp(rne(x / s) + z, 0, 255) as a
+//     uint8; the group's scale pair is (s, fp16(z)) (scales_row holds 2 per group).
+//   KVQ_FMT_TENSOR: s = scales_row[0], the tensor's fixed scale (read, never
+//     written), code = clamp(rne(x / s), -127, 127).
 // All 32 lanes of the warp must call it with the same arguments.
 __device__ __forceinline__ void quantize_row(const void *x, int64_t in_off, int dtype, int dim,
                                              int bits, int group, uint8_t *codes_row,
-                                             __half *scales_row, int lane, bool e4m3 = false)
+                                             __half *scales_row, int lane, int fmt = KVQ_FMT_INT)
 {
+    const bool e4m3 = fmt == KVQ_FMT_E4M3;
     const int lanes_per_group = group >> 2;
     for (int base = 0; base < dim; base += 128) {
         const int e0 = base + lane * 4;
@@ -66,6 +73,47 @@ __device__ __forceinline__ void quantize_row(const void *x, int64_t in_off, int 
                 w.x = *reinterpret_cast<uint32_t *>(&lo);
                 w.y = *reinterpret_cast<uint32_t *>(&hi);
                 *reinterpret_cast<uint2 *>(codes_row + (int64_t)e0 * 2) = w;
+            }
+            continue;
+        }
+
+        if (fmt == KVQ_FMT_ASYM) {
+            float lo = fminf(fminf(fminf(v[0], v[1]), fminf(v[2], v[3])), 0.0f);
+            float hi = fmaxf(fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3])), 0.0f);
+            for (int off = 1; off < lanes_per_group; off <<= 1) {
+                lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+                hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+            }
+            __half s16 = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 255.0f));
+            if (__half_as_ushort(s16) == 0x7c00u) s16 = __ushort_as_half(0x7bffu);
+            const float s = __half2float(s16);
+            int z = 0;
+            if (s != 0.0f) z = max(0, min(255, __float2int_rn(__fdiv_rn(-lo, s))));
+            if (active) {
+                uint32_t w = 0;
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    const int q = s != 0.0f ? max(0, min(255, __float2int_rn(__fdiv_rn(v[i], s)) + z)) : 0;
+                    w |= (uint32_t)q << (8 * i);
+                }
+                *reinterpret_cast<uint32_t *>(codes_row + e0) = w;
+                if ((lane % lanes_per_group) == 0) {
+                    scales_row[2 * (e0 / group)] = s16;
+                    scales_row[2 * (e0 / group) + 1] = __int2half_rn(z);
+                }
+            }
+            continue;
+        }
+        if (fmt == KVQ_FMT_TENSOR) {
+            const float s = __half2float(scales_row[0]);
+            if (active) {
+                uint32_t w = 0;
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    const int q = s != 0.0f ? max(-127, min(127, __float2int_rn(__fdiv_rn(v[i], s)))) : 0;
+                    w |= (uint32_t)(q & 0xff) << (8 * i);
+                }
+                *reinterpret_cast<uint32_t *>(codes_row + e0) = w;
             }
             continue;
         }

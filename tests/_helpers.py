@@ -15,17 +15,30 @@ def to_np32(t):
 
 
 def obits(cfg: Config, bits: int):
-    """The oracle's bit-width argument for a cache width: "e4m3" for FP8 caches."""
-    return "e4m3" if cfg.kv_format == kvq.KVQ_FMT_E4M3 and bits == 8 else bits
+    """The oracle's bit-width argument for a cache width: "e4m3" / "asym8" for those
+    8-bit formats (per-tensor INT8 codes are INT8 codes)."""
+    if bits == 8 and cfg.kv_format == kvq.KVQ_FMT_E4M3:
+        return "e4m3"
+    if bits == 8 and cfg.kv_format == kvq.KVQ_FMT_ASYM:
+        return "asym8"
+    return bits
 
 
-def oracle_cache(k, v, cfg: Config):
-    """k, v: [B, L, Hkv, dh] tensors -> oracle codes/scales in the cache layout [B, Hkv, cap, ...]."""
+def oracle_cache(k, v, cfg: Config, tensor_s16=None):
+    """k, v: [B, L, Hkv, dh] tensors -> oracle codes/scales in the cache layout [B, Hkv, cap, ...].
+    Per-tensor INT8: tensor_s16 = (K scale, V scale) fp16 bits; the scales come back
+    broadcast to one per (token, head), the per-head layout of the same values."""
     B, L, H, dh = k.shape
     cap = cfg.capacity
     out = []
-    for x, bits, grp in ((k, cfg.k_bits, cfg.k_group or dh), (v, cfg.v_bits, cfg.v_group or dh)):
+    for i, (x, bits, grp) in enumerate(((k, cfg.k_bits, cfg.k_group or dh),
+                                        (v, cfg.v_bits, cfg.v_group or dh))):
         xf = np.ascontiguousarray(to_np32(x).transpose(0, 2, 1, 3))   # [B, H, L, dh]
+        if cfg.kv_format == kvq.KVQ_FMT_TENSOR:
+            c = np.zeros((B, H, cap, dh), np.uint8)
+            c[:, :, :L] = oracle.quantize_rows_tensor(xf, tensor_s16[i])
+            out += [c, np.full((B, H, cap, 1), tensor_s16[i], np.uint16)]
+            continue
         if bits == 16:
             c = np.zeros((B, H, cap, dh), np.float16)
             c[:, :, :L] = xf.astype(np.float16)
@@ -33,7 +46,7 @@ def oracle_cache(k, v, cfg: Config):
         else:
             cc, ss = oracle.quantize_rows(xf, grp, obits(cfg, bits))
             c = np.zeros((B, H, cap, dh * bits // 8), np.uint8)
-            s = np.zeros((B, H, cap, dh // grp), np.uint16)
+            s = np.zeros((B, H, cap) + ss.shape[3:], np.uint16)
             c[:, :, :L] = cc
             s[:, :, :L] = ss
             out += [c, s]
@@ -49,6 +62,7 @@ def gpu_cache(cfg: Config, k, v, device="cuda"):
 
 
 def read_gpu_cache(cache: LayerCache, cfg: Config):
+    """The GPU cache as numpy arrays in the oracle_cache layout."""
     B, H, cap, dh = cfg.batch, cfg.n_kv_heads, cfg.capacity, cfg.head_dim
     res = []
     for codes, scales, bits, grp in ((cache.k_codes, cache.k_scales, cfg.k_bits, cfg.k_group or dh),
@@ -56,10 +70,15 @@ def read_gpu_cache(cache: LayerCache, cfg: Config):
         c = codes.cpu().numpy()
         if bits == 16:
             res += [c[: B * H * cap * dh * 2].view(np.uint16).reshape(B, H, cap, dh), None]
+            continue
+        c = c[: B * H * cap * dh * bits // 8].reshape(B, H, cap, dh * bits // 8)
+        sc = scales.cpu().numpy().view(np.uint16)
+        if cfg.kv_format == kvq.KVQ_FMT_TENSOR:
+            res += [c, np.full((B, H, cap, 1), sc[0], np.uint16)]
+        elif cfg.kv_format == kvq.KVQ_FMT_ASYM:
+            res += [c, sc[: B * H * cap * (dh // grp) * 2].reshape(B, H, cap, dh // grp, 2)]
         else:
-            res += [c[: B * H * cap * dh * bits // 8].reshape(B, H, cap, dh * bits // 8),
-                    scales.cpu().numpy().view(np.uint16)[: B * H * cap * (dh // grp)].reshape(
-                        B, H, cap, dh // grp)]
+            res += [c, sc[: B * H * cap * (dh // grp)].reshape(B, H, cap, dh // grp)]
     return res
 
 

@@ -191,7 +191,7 @@ def test_fp8_config_validation_and_bytes():
     f8 = Config(**base, kv_format=kvq.KVQ_FMT_E4M3)
     assert kvq.kvq_cache_bytes(f8) == kvq.kvq_cache_bytes(Config(**base))
     assert kvq.kvq_layer_buffer_bytes(f8) == kvq.kvq_layer_buffer_bytes(Config(**base))
-    for over, want in (({"k_bits": 4}, -2), ({"v_bits": 16}, -2), ({"kv_format": 2}, -1),
+    for over, want in (({"k_bits": 4}, -2), ({"v_bits": 16}, -2), ({"kv_format": 4}, -1),
                        ({"kv_format": -1}, -1)):
         with pytest.raises(kvq.KvqError) as e:
             kvq.kvq_cache_bytes(Config(**{**f8.__dict__, **over}))
@@ -201,3 +201,27 @@ def test_fp8_config_validation_and_bytes():
     with pytest.raises(kvq.KvqError) as e:
         kvq.kvq_cache_bytes(h)
     assert e.value.status == -2
+
+
+def test_asym_and_tensor_config_bytes_and_validation():
+    base = dict(batch=2, capacity=256, n_q_heads=8, n_kv_heads=2, head_dim=128, k_bits=8,
+                v_bits=8, k_group=32, v_group=128)
+    sym = kvq.kvq_cache_bytes(Config(**base))[0]
+    asym = Config(**base, kv_format=kvq.KVQ_FMT_ASYM)
+    # a (scale, zero-point) pair per group: the scale bytes double
+    scale_bytes = 2 * (128 // 32 + 128 // 128) * 2
+    assert kvq.kvq_cache_bytes(asym)[0] == sym + scale_bytes
+    kc, ks, vc, vs = kvq.kvq_layer_buffer_bytes(asym)
+    assert ks == 2 * 256 * 2 * 4 * 2 * 2 and vs == 2 * 256 * 2 * 1 * 2 * 2
+    tensor = Config(**{**base, "k_group": 0, "v_group": 0}, kv_format=kvq.KVQ_FMT_TENSOR)
+    per_tok, layer, _ = kvq.kvq_cache_bytes(tensor)
+    assert per_tok == 2 * 2 * 128 and layer == per_tok * 2 * 256 + 4
+    assert kvq.kvq_layer_buffer_bytes(tensor) == (2 * 256 * 2 * 128, 2, 2 * 256 * 2 * 128, 2)
+    for cfg, want in ((Config(**{**base, "k_bits": 4}, kv_format=kvq.KVQ_FMT_ASYM), -2),
+                      (Config(**base, kv_format=kvq.KVQ_FMT_TENSOR), -2),      # grouped
+                      (Config(**{**base, "v_bits": 16, "k_group": 0, "v_group": 0},
+                              kv_format=kvq.KVQ_FMT_TENSOR), -2),
+                      (Config(**base, kv_format=4), -1)):
+        with pytest.raises(kvq.KvqError) as e:
+            kvq.kvq_cache_bytes(cfg)
+        assert e.value.status == want
