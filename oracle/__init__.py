@@ -26,6 +26,9 @@ Parity status of each function (what pins it, in ``tests/test_oracle_pins.py``):
       invariance, and torch scaled_dot_product_attention in fp64.
   h_reconstruct: pinned against a numpy matmul (library primitive) and the
       INT8-h / INT4-h quality bands of the TinyLoop page.
+  h_absorbed_decode: pinned to the reconstruction attention in fp64 (numpy matmuls of
+      W and the dequantised h, then attend), to out = W_v h^ for one token, and to
+      W_v mean(h^) for a zero query.
   bytes_per_token_layer: pinned to the printed TinyLoop, KVSplit and
       on-device figures (tests/golden/).
 """
@@ -77,6 +80,8 @@ def _load():
     lib.kvqo_quantize_rows.argtypes = [P, i64, i32, i32, i32, P, P]
     lib.kvqo_dequantize_rows.argtypes = [P, P, i64, i32, i32, i32, P]
     lib.kvqo_quantize_rows_tensor.argtypes = [P, i64, i32, ctypes.c_uint16, P]
+    lib.kvqo_h_absorbed_decode.argtypes = [i32, i32, i32, i32, i32, i32, P, P, i32, i32, P, P, P,
+                                           f64, P, i32]
     lib.kvqo_attend.argtypes = [P, P, P, i64, i32, f64, P]
     lib.kvqo_decode_layer.argtypes = [i32, i32, i32, i32, i32, P, P, i32, i32, P, P, i32, i32,
                                       P, P, f64, P, i32]
@@ -254,6 +259,30 @@ def h_reconstruct(h_codes, h_scales, D: int, h_groups: int, h_bits: int, w_bf16_
                                     1 if round_bf16 else 0, _ptr(y64), _ptr(y16), n_threads),
          "h_reconstruct")
     return y64, y16
+
+
+def h_absorbed_decode(h_codes, h_scales, h_bits: int, h_groups: int, w_bf16_bits, q, lens,
+                      n_kv_heads: int, tau: float = 0.0, n_threads: int = 0):
+    """h-mode decode attention by query absorption, fp64 (see the C header).
+
+    h_codes: [B, cap, D*bits/8] uint8 (bits 16: fp16 [B, cap, D]); h_scales [B, cap, h_groups];
+    w_bf16_bits: [2*Hkv*Dh, D] uint16; q: [B, Hq, Dh] float32; lens [B].
+    Returns out [B, Hq, Dh] float64.
+    """
+    hc = np.ascontiguousarray(h_codes)
+    hc = hc.view(np.uint8) if hc.dtype != np.uint8 else hc
+    B, cap = h_codes.shape[0], h_codes.shape[1]
+    hs = None if h_bits == 16 else np.ascontiguousarray(h_scales, np.uint16)
+    W = np.ascontiguousarray(w_bf16_bits, np.uint16)
+    q = np.ascontiguousarray(q, np.float32)
+    _, Hq, Dh = q.shape
+    D = W.shape[1]
+    lens = np.ascontiguousarray(lens, np.int32)
+    out = np.zeros((B, Hq, Dh), np.float64)
+    _chk(_load().kvqo_h_absorbed_decode(B, Hq, n_kv_heads, Dh, D, cap, _ptr(hc), _ptr(hs), h_bits,
+                                        h_groups, _ptr(W), _ptr(q), _ptr(lens), tau, _ptr(out),
+                                        n_threads), "h_absorbed_decode")
+    return out
 
 
 def bytes_per_token_layer(mode=0, n_kv_heads=0, head_dim=0, k_bits=16, v_bits=16, k_group=0,

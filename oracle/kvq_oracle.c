@@ -46,6 +46,9 @@
  *    scale s for a whole tensor, code = clamp(rne(x / s), -127, 127), the
  *    symmetric INT8 codes (x^ = code * s, the per-head dequantisation with
  *    every row's scale equal to s).
+ *  - h-mode decode by query absorption: the same attention as the
+ *    reconstruction path, regrouped by linearity (qa = W_k^T q, s = qa . h^,
+ *    out = W_v sum_t p_t h^_t), in fp64 without the bf16 / fp16 roundings.
  *  - Bytes per token per layer (TinyLoop docs, "記憶體公式" table).
  *
  * Build: gcc -O2 -fopenmp -shared -fPIC -ffp-contract=off (no fast-math: the
@@ -551,6 +554,96 @@ int kvqo_h_reconstruct(const uint8_t *h_codes, const uint16_t *h_scales, int64_t
         free(h);
     }
     free(W);
+    return rc ? -1 : 0;
+}
+
+/* h-mode decode by query absorption (an algebraic rewrite of the
+ * reconstruction path of the TinyLoop page, "運作原理": K = W_k h and
+ * V = W_v h are linear in h, so q . K_t = (W_k,j^T q) . h_t and
+ * sum_t p_t V_t = W_v,j (sum_t p_t h_t) for KV head j).  For every sequence b
+ * and query head h (KV head j = h / G), all in fp64 with h^ dequantised
+ * exactly and W the bf16 values:
+ *   qa   = sum_i q[i] W[j Dh + i][:]              (W_k rows of head j)
+ *   s_t  = tau qa . h^_t,  p = softmax(s) over t < lens[b]
+ *   ob   = sum_t p_t h^_t
+ *   out[i] = sum_d W[Hkv Dh + j Dh + i][d] ob[d]  (W_v rows of head j)
+ * No rounding of h^ to bf16 nor of K/V to fp16: the result is the
+ * reconstruction attention in exact arithmetic.  h codes [B][cap][row],
+ * scales [B][cap][h_groups]; q float [B][Hq][Dh]; W bf16 [2 Hkv Dh][D];
+ * out fp64 [B][Hq][Dh]; tau <= 0 means 1/sqrt(Dh); an empty sequence gives
+ * zeros. */
+int kvqo_h_absorbed_decode(int B, int Hq, int Hkv, int Dh, int D, int cap, const uint8_t *h_codes,
+                           const uint16_t *h_scales, int h_bits, int h_groups,
+                           const uint16_t *w_bf16, const float *q, const int32_t *lens, double tau,
+                           double *out, int n_threads)
+{
+    if (Hkv <= 0 || Hq % Hkv != 0 || Hkv * Dh != D || h_groups <= 0 || D % h_groups != 0)
+        return -1;
+    const int G = Hq / Hkv;
+    const int group = D / h_groups;
+    if (tau <= 0.0) tau = 1.0 / sqrt((double)Dh);
+    const int64_t row_bytes = (h_bits == 16) ? (int64_t)D * 2 : (int64_t)D * h_bits / 8;
+    int rc = 0;
+    (void)n_threads;
+#ifdef _OPENMP
+    if (n_threads > 0) omp_set_num_threads(n_threads);
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : rc)
+#endif
+    for (int bh = 0; bh < B * Hq; bh++) {
+        const int b = bh / Hq, h = bh % Hq, j = h / G;
+        int64_t L = lens[b];
+        if (L < 0) L = 0;
+        if (L > cap) L = cap;
+        double *o = out + (int64_t)bh * Dh;
+        for (int i = 0; i < Dh; i++) o[i] = 0.0;
+        if (L == 0) continue;
+        double *H = (double *)malloc(sizeof(double) * (size_t)L * D);
+        double *qa = (double *)malloc(sizeof(double) * (size_t)D);
+        double *ob = (double *)malloc(sizeof(double) * (size_t)D);
+        double *sc = (double *)malloc(sizeof(double) * (size_t)L);
+        if (!H || !qa || !ob || !sc) {
+            rc |= 2;
+        } else {
+            const int64_t slab = (int64_t)b * cap;
+            rc |= kvqo_dequantize_rows(h_codes + slab * row_bytes,
+                                       h_scales ? h_scales + slab * h_groups : NULL, L, D, group,
+                                       h_bits, H) ? 1 : 0;
+            const float *qh = q + (int64_t)bh * Dh;
+            for (int d = 0; d < D; d++) {
+                double acc = 0.0;
+                for (int i = 0; i < Dh; i++)
+                    acc += (double)qh[i] * (double)kvqo_bf16_to_f32(w_bf16[(int64_t)(j * Dh + i) * D + d]);
+                qa[d] = acc;
+            }
+            double m = -INFINITY;
+            for (int64_t t = 0; t < L; t++) {
+                double acc = 0.0;
+                for (int d = 0; d < D; d++) acc += qa[d] * H[t * D + d];
+                sc[t] = tau * acc;
+                if (sc[t] > m) m = sc[t];
+            }
+            double l = 0.0;
+            for (int64_t t = 0; t < L; t++) {
+                sc[t] = exp(sc[t] - m);
+                l += sc[t];
+            }
+            for (int d = 0; d < D; d++) ob[d] = 0.0;
+            for (int64_t t = 0; t < L; t++) {
+                const double p = sc[t] / l;
+                for (int d = 0; d < D; d++) ob[d] += p * H[t * D + d];
+            }
+            for (int i = 0; i < Dh; i++) {
+                const uint16_t *wr = w_bf16 + (int64_t)(Hkv * Dh + j * Dh + i) * D;
+                double acc = 0.0;
+                for (int d = 0; d < D; d++) acc += (double)kvqo_bf16_to_f32(wr[d]) * ob[d];
+                o[i] = acc;
+            }
+        }
+        free(H);
+        free(qa);
+        free(ob);
+        free(sc);
+    }
     return rc ? -1 : 0;
 }
 

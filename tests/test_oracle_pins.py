@@ -606,3 +606,53 @@ def test_per_tensor_int8_clips_and_matches_torch_qint8():
     t = torch.quantize_per_tensor(torch.from_numpy(xc), s, 0, torch.qint8).int_repr().numpy()
     assert np.array_equal(t, c)                                   # s a power of two: no ties differ
     assert not oracle.quantize_rows_tensor(x, 0).any()
+
+
+# --- h-mode query absorption -------------------------------------------------------
+
+def _h_case(bits, seed, B=2, Hkv=2, G=2, Dh=32, cap=20, h_groups=2):
+    rng = np.random.default_rng(seed)
+    D = Hkv * Dh
+    h = rng.standard_normal((B, cap, D)).astype(np.float32)
+    if bits == 16:
+        codes, scales = h.astype(np.float16).view(np.uint16), None
+    else:
+        codes, scales = oracle.quantize_rows(h, D // h_groups, bits)
+    w = torch.from_numpy(rng.standard_normal((2 * D, D)).astype(np.float32) / np.sqrt(D))
+    wb = w.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    q = rng.standard_normal((B, Hkv * G, Dh)).astype(np.float32)
+    hd = oracle.dequantize_rows(codes, scales, D, D // h_groups, bits)     # [B, cap, D] fp64
+    W = w.to(torch.bfloat16).double().numpy()
+    return codes, scales, wb, q, hd, W, D, Dh, G, Hkv
+
+
+@pytest.mark.parametrize("bits", [4, 8, 16])
+def test_h_absorbed_equals_reconstruction_attention_in_fp64(bits):
+    codes, scales, wb, q, hd, W, D, Dh, G, Hkv = _h_case(bits, 11)
+    lens = np.array([20, 7], np.int32)
+    got = oracle.h_absorbed_decode(codes, scales, bits, 2, wb, q, lens, Hkv)
+    for b, L in enumerate(lens):
+        K = hd[b, :L] @ W[:D].T          # [L, Hkv*Dh], numpy matmul
+        V = hd[b, :L] @ W[D:].T
+        for h in range(Hkv * G):
+            j = h // G
+            want = oracle.attend(q[b, h].astype(np.float64), K[:, j * Dh:(j + 1) * Dh],
+                                 V[:, j * Dh:(j + 1) * Dh], 1 / np.sqrt(Dh))
+            assert np.allclose(got[b, h], want, rtol=1e-10, atol=1e-12), (b, h)
+
+
+def test_h_absorbed_single_token_and_zero_query():
+    codes, scales, wb, q, hd, W, D, Dh, G, Hkv = _h_case(4, 12)
+    one = oracle.h_absorbed_decode(codes, scales, 4, 2, wb, q, np.array([1, 0], np.int32), Hkv)
+    V0 = W[D:] @ hd[0, 0]
+    for h in range(Hkv * G):
+        j = h // G
+        assert np.allclose(one[0, h], V0[j * Dh:(j + 1) * Dh], rtol=1e-12, atol=1e-12)
+    assert not one[1].any()                                              # empty sequence
+    zq = oracle.h_absorbed_decode(codes, scales, 4, 2, wb, np.zeros_like(q),
+                                  np.array([20, 9], np.int32), Hkv)
+    for b, L in ((0, 20), (1, 9)):
+        Vm = W[D:] @ hd[b, :L].mean(0)
+        for h in range(Hkv * G):
+            j = h // G
+            assert np.allclose(zq[b, h], Vm[j * Dh:(j + 1) * Dh], rtol=1e-10, atol=1e-12)
