@@ -439,6 +439,39 @@ def run_hmode(args, world, device):
                        "unit": "TFLOP/s", "frac": round(tf / burst, 4),
                        "frac_of_sustained": round(tf / sustained, 4)}
     res["steps_per_s"] = round(world * 1e3 / res["step_ms"], 2)
+
+    # the same attention by query absorption (W_k^T q against the h codes, W_v on
+    # sum p h^): HBM-bound on the h codes + scales and W; the inputs (25 MB) fit in
+    # L2, so every timed call follows a 256 MB L2 flush and is bracketed alone
+    ab_scratch = torch.empty(kvq.kvq_h_absorbed_scratch_bytes(cfg, S) // 4, device=device)
+    flush = torch.empty(256 * 1024 * 1024 // 4, device=device)
+
+    def absorbed():
+        kvq.kvq_h_decode_absorbed(cfg, cache, W, q, d_len, S, out, ab_scratch)
+
+    for _ in range(max(args.warmup, 3)):
+        absorbed()
+    n = max(3, min(args.steps, 100))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n)]
+    for a, b in evs:
+        flush.fill_(1.0)
+        a.record()
+        absorbed()
+        b.record()
+    torch.cuda.synchronize()
+    ams = reduce_max(statistics.mean(a.elapsed_time(b) for a, b in evs), world, device)
+    h_bytes = kvq.kvq_cache_bytes(cfg)[0] * w.batch * S
+    w_bytes = W.numel() * W.element_size()
+    hbm, hkind = measured_peaks()
+    gbs = (h_bytes + w_bytes) / (ams * 1e-3) / 1e9
+    res["absorbed"] = {"kernels": "absorb_q, absorb_scores, absorb_softmax, absorb_pv, absorb_out",
+                       "ms": round(ams, 5), "steps_per_s": round(world * 1e3 / ams, 1),
+                       "bytes": h_bytes + w_bytes, "l2": "flushed before each call",
+                       "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm,
+                                    "peak_kind": hkind, "unit": "GB/s",
+                                    "frac": round(gbs / hbm, 4)},
+                       "speedup_vs_reconstruction_step": round(res["step_ms"] / ams, 2)}
     return res
 
 

@@ -317,6 +317,36 @@ KVQ_API int kvq_h_reconstruct(const kvq_config *cfg, const kvq_layer *layer, con
                               int32_t out_capacity, void *operand, uint64_t operand_bytes,
                               kvq_stream_t stream);
 
+/* h-mode decode attention by query absorption: the attention of
+ * kvq_decode_attn (h-mode) regrouped by the linearity of the reconstruction
+ * ([TL] "運作原理": K = W_k h^, V = W_v h^), without rebuilding K and V:
+ * for sequence b and query head h of KV head j = h / G,
+ *   qa = W_k,j^T q            (W_k,j: rows j*Dh .. j*Dh+Dh-1 of w_kv)
+ *   s_t = softmax_scale * qa . h^_t,  p = softmax(s) over t < d_len[b]
+ *   out = W_v,j (sum_t p_t h^_t)   (W_v,j: rows Hkv*Dh + j*Dh .. of w_kv)
+ * Equal in exact arithmetic to the reconstruction path; it reads the h codes
+ * and W once per step instead of D x 2*Hkv*Dh MACs per cached token.  Here
+ * qa is split per (head, scale group) into two int8 parts for the int8
+ * tensor-core scores (relative error below 2^-15 of the group's largest
+ * element) and p * scale enters the p . h^ product in fp16; everything else
+ * accumulates in fp32.  An empty sequence gets zeros.
+ *   h_bits 4 or 8; Hkv*Dh = D, D a multiple of 256, Dh 64 or 128; Hq <= 32.
+ *   w_kv     device bf16 [2*Hkv*Dh][D] (as kvq_decode_attn)
+ *   q, q_dtype, d_len, max_len_host, softmax_scale, out, out_dtype: as
+ *            kvq_decode_attn (max_len_host bounds d_len[] and sizes the scratch)
+ *   scratch  device, at least kvq_h_absorbed_scratch_bytes(cfg, max_len_host)
+ *            bytes (contents on entry do not matter; calls that overlap on
+ *            the GPU need separate scratch)
+ * Five kernel launches on `stream`.  Errors: INVALID_ARG (KV mode, null or
+ * bad arguments), UNSUPPORTED (shape), CAPACITY, ALIGN (16 bytes), WORKSPACE,
+ * LAUNCH. */
+KVQ_API int kvq_h_absorbed_scratch_bytes(const kvq_config *cfg, int32_t max_len, uint64_t *bytes);
+KVQ_API int kvq_h_decode_absorbed(const kvq_config *cfg, const kvq_layer *layer, const void *w_kv,
+                                  const void *q, int32_t q_dtype, const int32_t *d_len,
+                                  int32_t max_len_host, float softmax_scale, void *out,
+                                  int32_t out_dtype, void *scratch, uint64_t scratch_bytes,
+                                  kvq_stream_t stream);
+
 /* Read and clear the device status word a decode launch leaves in its
  * workspace: KVQ_OK, or KVQ_ERR_TIMEOUT if a kernel gave up a bounded wait
  * (its outputs are then invalid).  Synchronises `stream`. */

@@ -26,7 +26,7 @@ EXPORTED = ("kvq_cache_bytes", "kvq_layer_buffer_bytes", "kvq_append", "kvq_work
             "kvq_h_scratch_bytes", "kvq_decode_attn", "kvq_decode_partials", "kvq_merge_partials",
             "kvq_h_reconstruct", "kvq_workspace_status", "kvq_status_string",
             "kvq_last_error_detail", "kvq_decode_attn_noalloc", "kvq_h_operand_bytes",
-            "kvq_append_decode_attn")
+            "kvq_append_decode_attn", "kvq_h_absorbed_scratch_bytes", "kvq_h_decode_absorbed")
 
 
 class KvqError(RuntimeError):
@@ -72,6 +72,8 @@ def _load():
         "kvq_h_operand_bytes": [cfgp, i32, pu64],
         "kvq_h_reconstruct": [cfgp, layp, P, i32, P, P, i32, P, u64, P],
         "kvq_workspace_status": [P, ctypes.POINTER(i32), P],
+        "kvq_h_absorbed_scratch_bytes": [cfgp, i32, pu64],
+        "kvq_h_decode_absorbed": [cfgp, layp, P, P, i32, P, i32, ctypes.c_float, P, i32, P, u64, P],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -311,6 +313,25 @@ def kvq_h_reconstruct(cfg: Config, layer: LayerCache, w_kv: torch.Tensor, max_le
                                   int(max_len), _ptr(k_out), _ptr(v_out), int(out_capacity),
                                   _ptr(operand), operand.numel() * operand.element_size(),
                                   _stream(stream)))
+
+
+def kvq_h_absorbed_scratch_bytes(cfg: Config, max_len: int) -> int:
+    v = ctypes.c_uint64()
+    _check("kvq_h_absorbed_scratch_bytes",
+           _lib.kvq_h_absorbed_scratch_bytes(cfg._ref(), int(max_len), ctypes.byref(v)))
+    return v.value
+
+
+def kvq_h_decode_absorbed(cfg: Config, layer: LayerCache, w_kv: torch.Tensor, q: torch.Tensor,
+                          d_len: torch.Tensor, max_len: int, out: torch.Tensor,
+                          scratch: torch.Tensor, softmax_scale: float = 0.0, stream=None):
+    """h-mode decode attention by query absorption (W_k^T q against the h codes)."""
+    _check("kvq_h_decode_absorbed",
+           _lib.kvq_h_decode_absorbed(cfg._ref(), layer._ref(), _ptr(w_kv), _ptr(q),
+                                      _dtype_code(q), _ptr(d_len), int(max_len),
+                                      float(softmax_scale), _ptr(out), _dtype_code(out),
+                                      _ptr(scratch), scratch.numel() * scratch.element_size(),
+                                      _stream(stream)))
 
 
 def kvq_workspace_status(ws: Workspace, stream=None) -> int:

@@ -751,6 +751,82 @@ int kvq_h_reconstruct(const kvq_config *cfg, const kvq_layer *layer, const void 
                               operand_bytes, nullptr, stream);
 }
 
+// ------------------------------------------------------------ query absorption
+static int absorbed_shape_check(const kvq_config *cfg)
+{
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (cfg->mode != KVQ_MODE_H) return KVQ_ERR_INVALID_ARG;
+    if (cfg->n_kv_heads * cfg->head_dim != cfg->d_model) return KVQ_ERR_INVALID_ARG;
+    if (cfg->h_bits != 4 && cfg->h_bits != 8) return KVQ_ERR_UNSUPPORTED;
+    if (cfg->head_dim % 32 != 0 || cfg->head_dim > 128 || cfg->d_model % 256 != 0)
+        return KVQ_ERR_UNSUPPORTED;
+    if (cfg->n_q_heads % cfg->n_kv_heads != 0 || cfg->n_q_heads > 32) return KVQ_ERR_UNSUPPORTED;
+    return KVQ_OK;
+}
+
+int kvq_h_absorbed_scratch_bytes(const kvq_config *cfg, int32_t max_len, uint64_t *bytes)
+{
+    int rc = absorbed_shape_check(cfg);
+    if (rc) return rc;
+    if (!bytes || max_len < 0) return KVQ_ERR_INVALID_ARG;
+    if (max_len > cfg->capacity) return KVQ_ERR_CAPACITY;
+    uint64_t off[4];
+    *bytes = absorb_scratch_layout(cfg->batch, cfg->n_q_heads, cfg->d_model, cfg->h_groups, max_len, off);
+    return KVQ_OK;
+}
+
+int kvq_h_decode_absorbed(const kvq_config *cfg, const kvq_layer *layer, const void *w_kv,
+                          const void *q, int32_t q_dtype, const int32_t *d_len,
+                          int32_t max_len_host, float softmax_scale, void *out, int32_t out_dtype,
+                          void *scratch, uint64_t scratch_bytes, kvq_stream_t stream)
+{
+    int rc = absorbed_shape_check(cfg);
+    if (rc) return rc;
+    if (!layer || !layer->k_codes || !layer->k_scales || !w_kv || !q || !d_len || !out || !scratch)
+        return KVQ_ERR_INVALID_ARG;
+    if (q_dtype != KVQ_F16 && q_dtype != KVQ_F32 && q_dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
+    if (out_dtype != KVQ_F16 && out_dtype != KVQ_F32) return KVQ_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale) || max_len_host < 0) return KVQ_ERR_INVALID_ARG;
+    if (max_len_host > cfg->capacity) return KVQ_ERR_CAPACITY;
+    if (!aligned16(layer->k_codes) || !aligned16(layer->k_scales) || !aligned16(w_kv) ||
+        !aligned16(q) || !aligned16(out) || !aligned16(scratch))
+        return KVQ_ERR_ALIGN;
+    uint64_t off[4];
+    const uint64_t need = absorb_scratch_layout(cfg->batch, cfg->n_q_heads, cfg->d_model,
+                                                cfg->h_groups, max_len_host, off);
+    if (scratch_bytes < need) return KVQ_ERR_WORKSPACE;
+    AbsorbParams p{};
+    p.h_codes = static_cast<const uint8_t *>(layer->k_codes);
+    p.h_scales = static_cast<const __half *>(layer->k_scales);
+    p.w = static_cast<const __nv_bfloat16 *>(w_kv);
+    p.q = q;
+    p.d_len = d_len;
+    p.out = out;
+    p.q_dtype = q_dtype;
+    p.out_f32 = out_dtype == KVQ_F32;
+    p.B = cfg->batch;
+    p.Hq = cfg->n_q_heads;
+    p.Hkv = cfg->n_kv_heads;
+    p.Dh = cfg->head_dim;
+    p.D = cfg->d_model;
+    p.cap = cfg->capacity;
+    p.bits = cfg->h_bits;
+    p.ng = cfg->h_groups;
+    p.group = cfg->d_model / cfg->h_groups;
+    const float scale = softmax_scale != 0.f ? softmax_scale : 1.f / std::sqrt((float)cfg->head_dim);
+    p.tau_log2e = scale * 1.4426950408889634f;
+    uint8_t *base = static_cast<uint8_t *>(scratch);
+    p.qfrag = reinterpret_cast<uint4 *>(base + off[0]);
+    p.qfac = reinterpret_cast<float *>(base + off[1]);
+    p.p = reinterpret_cast<float *>(base + off[2]);
+    p.ob = reinterpret_cast<float *>(base + off[3]);
+    p.capP = (max_len_host + 63) / 64 * 64;
+    p.NT = absorb_nt(p.Hq);
+    cudaError_t e = launch_absorbed(p, max_len_host, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KVQ_OK : fail("absorbed decode launch", e);
+}
+
 int kvq_workspace_status(void *workspace, int32_t *status, kvq_stream_t stream)
 {
     if (!workspace || !status) return KVQ_ERR_INVALID_ARG;

@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
+#include <cuda_bf16.h>
 
 #include "../../include/kvq.h"
 
@@ -91,6 +92,29 @@ struct MergeParams {
 };
 
 // Host helpers implemented in kvq_decode.cu.
+// h-mode decode by query absorption (kvq_absorb.cu)
+struct AbsorbParams {
+    const uint8_t *h_codes;       // [B][cap][D*bits/8]
+    const __half *h_scales;       // [B][cap][ng]
+    const __nv_bfloat16 *w;       // [2*Hkv*Dh][D]: W_k rows, then W_v rows
+    const void *q;                // [B][Hq][Dh]
+    const int32_t *d_len;         // [B]
+    void *out;                    // [B][Hq][Dh]
+    int32_t q_dtype, out_f32;
+    int32_t B, Hq, Hkv, Dh, D, cap, bits, group, ng;
+    float tau_log2e;
+    // scratch
+    uint4 *qfrag;                 // [B][D/32][NT][32] int8 hi/lo B fragments of W_k^T q
+    float *qfac;                  // [B][ng][NT*8] score factor per (group, head)
+    float *p;                     // [B][Hq][capP] scores, then probabilities
+    float *ob;                    // [B][Hq][D] sum_t p_t h^_t
+    int32_t capP, NT;
+};
+// scratch bytes and sub-buffer offsets (each 256-byte aligned)
+int absorb_nt(int Hq);   // n-tiles of 8 query heads in the score MMA: 1, 2 or 4
+uint64_t absorb_scratch_layout(int B, int Hq, int D, int ng, int max_len, uint64_t off[4]);
+cudaError_t launch_absorbed(const AbsorbParams &p, int max_len, cudaStream_t stream);
+
 struct DecodeLaunch {
     int dh, kb, vb;
     bool kg, vg;              // grouped key / value scales

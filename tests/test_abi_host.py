@@ -225,3 +225,24 @@ def test_asym_and_tensor_config_bytes_and_validation():
         with pytest.raises(kvq.KvqError) as e:
             kvq.kvq_cache_bytes(cfg)
         assert e.value.status == want
+
+
+def test_absorbed_scratch_bytes_and_validation():
+    cfg = Config(batch=8, capacity=1024, mode=kvq.KVQ_MODE_H, d_model=2048, h_bits=4, h_groups=16,
+                 n_q_heads=16, n_kv_heads=16, head_dim=128)
+    # q fragments B*(D/32)*NT*512 + factors B*ng*NT*8*4 + scores B*Hq*capP*4 + ob B*Hq*D*4
+    want = 8 * 64 * 2 * 512 + 8 * 16 * 16 * 4 + 8 * 16 * 1024 * 4 + 8 * 16 * 2048 * 4
+    assert kvq.kvq_h_absorbed_scratch_bytes(cfg, 1024) == want
+    assert kvq.kvq_h_absorbed_scratch_bytes(cfg, 1000) == want
+    for over, st in (({"h_bits": 16, "h_groups": 0}, -2), ({"n_q_heads": 64}, -2),
+                     ({"n_kv_heads": 8}, -1)):
+        with pytest.raises(kvq.KvqError) as e:
+            kvq.kvq_h_absorbed_scratch_bytes(Config(**{**cfg.__dict__, **over}), 1024)
+        assert e.value.status == st, over
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.kvq_h_absorbed_scratch_bytes(cfg, 1025)
+    assert e.value.status == -3
+    kv = Config(batch=1, capacity=64, n_q_heads=4, n_kv_heads=4, head_dim=128)
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.kvq_h_absorbed_scratch_bytes(kv, 64)
+    assert e.value.status == -1
