@@ -303,7 +303,14 @@ def time_e2e(w, st, steps, warmup, world, device):
     h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v))
     d2h = h_out.numel() * h_out.element_size()
 
+    # each layer's output goes back on a copy stream while the next layers run (the
+    # copy stream waits on the layer's event, the compute stream never waits, so the
+    # programmatic launches between layers stay back to back)
+    copy = torch.cuda.Stream()
+    done = [torch.cuda.Event() for _ in range(w.n_layers)]
+
     def one():
+        cur = torch.cuda.current_stream()
         st["q"].copy_(h_q, non_blocking=True)
         st["k_new"].copy_(h_k, non_blocking=True)
         st["v_new"].copy_(h_v, non_blocking=True)
@@ -311,7 +318,11 @@ def time_e2e(w, st, steps, warmup, world, device):
             kvq.kvq_append_decode_attn(cfg, st["caches"][layer], st["k_new"][layer],
                                        st["v_new"][layer], st["q"][layer], st["d_len"], L,
                                        st["out"][layer], st["ws"])
-        h_out.copy_(st["out"], non_blocking=True)
+            done[layer].record(cur)
+            copy.wait_event(done[layer])
+            with torch.cuda.stream(copy):
+                h_out[layer].copy_(st["out"][layer], non_blocking=True)
+        cur.wait_stream(copy)   # the step ends when its outputs are on the host
 
     for _ in range(warmup):
         one()

@@ -771,8 +771,9 @@ int kvq_h_absorbed_scratch_bytes(const kvq_config *cfg, int32_t max_len, uint64_
     if (rc) return rc;
     if (!bytes || max_len < 0) return KVQ_ERR_INVALID_ARG;
     if (max_len > cfg->capacity) return KVQ_ERR_CAPACITY;
-    uint64_t off[4];
-    *bytes = absorb_scratch_layout(cfg->batch, cfg->n_q_heads, cfg->d_model, cfg->h_groups, max_len, off);
+    uint64_t off[6];
+    *bytes = absorb_scratch_layout(cfg->batch, cfg->n_q_heads, cfg->d_model, cfg->h_groups,
+                                   cfg->h_bits, max_len, off);
     return KVQ_OK;
 }
 
@@ -792,9 +793,9 @@ int kvq_h_decode_absorbed(const kvq_config *cfg, const kvq_layer *layer, const v
     if (!aligned16(layer->k_codes) || !aligned16(layer->k_scales) || !aligned16(w_kv) ||
         !aligned16(q) || !aligned16(out) || !aligned16(scratch))
         return KVQ_ERR_ALIGN;
-    uint64_t off[4];
+    uint64_t off[6];
     const uint64_t need = absorb_scratch_layout(cfg->batch, cfg->n_q_heads, cfg->d_model,
-                                                cfg->h_groups, max_len_host, off);
+                                                cfg->h_groups, cfg->h_bits, max_len_host, off);
     if (scratch_bytes < need) return KVQ_ERR_WORKSPACE;
     AbsorbParams p{};
     p.h_codes = static_cast<const uint8_t *>(layer->k_codes);
@@ -820,9 +821,13 @@ int kvq_h_decode_absorbed(const kvq_config *cfg, const kvq_layer *layer, const v
     p.qfrag = reinterpret_cast<uint4 *>(base + off[0]);
     p.qfac = reinterpret_cast<float *>(base + off[1]);
     p.p = reinterpret_cast<float *>(base + off[2]);
-    p.ob = reinterpret_cast<float *>(base + off[3]);
+    p.stats = reinterpret_cast<float2 *>(base + off[3]);
+    p.obp = reinterpret_cast<float *>(base + off[4]);
     p.capP = (max_len_host + 63) / 64 * 64;
     p.NT = absorb_nt(p.Hq);
+    p.T2 = absorb_t2(p.D, p.bits, p.Hq, p.ng);
+    p.ntile = p.capP / p.T2;
+    p.split = absorb_split(max_len_host);
     cudaError_t e = launch_absorbed(p, max_len_host, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? KVQ_OK : fail("absorbed decode launch", e);
 }
