@@ -87,14 +87,22 @@ __global__ void __launch_bounds__(128) absorb_q_kernel(AbsorbParams p)
     const int q0 = blockIdx.z * 8;
     const int nqc = min(8, nq - q0);
     grid_dependency_wait();
-    for (int k = tid; k < 8 * DH; k += blockDim.x) {
-        const int c = k / DH, i = k % DH;
-        float v = 0.f;
-        if (c < nqc) {
-            const int qi = q0 + c, b = qi / G, h = j * G + qi % G;
-            v = load_qf(p.q, p.q_dtype, ((int64_t)b * p.Hq + h) * DH + i);
+    {
+        float v[8 * DH / 128];                 // all loads in flight before the stores
+#pragma unroll
+        for (int r = 0; r < 8 * DH / 128; r++) {
+            const int k = tid + 128 * r, c = k / DH, i = k % DH;
+            v[r] = 0.f;
+            if (c < nqc) {
+                const int qi = q0 + c, b = qi / G, h = j * G + qi % G;
+                v[r] = load_qf(p.q, p.q_dtype, ((int64_t)b * p.Hq + h) * DH + i);
+            }
         }
-        qs[c][i] = v;
+#pragma unroll
+        for (int r = 0; r < 8 * DH / 128; r++) {
+            const int k = tid + 128 * r;
+            qs[k / DH][k % DH] = v[r];
+        }
     }
     __syncthreads();
     const int rg = tid >> 4, cg = tid & 15;
@@ -208,10 +216,16 @@ __global__ void __launch_bounds__(128) absorb_scores_kernel(AbsorbParams p)
     const uint4 *qsrc = p.qfrag + (size_t)b * KS * NT * 32;
     const uint32_t qb = smem_u32(qf);
     for (int k = tid; k < KS * NT * 32; k += blockDim.x) cp_async16(qb + 16 * k, qsrc + k);
-    for (int k = tid; k < nrow * p.ng; k += blockDim.x)
-        sk[k] = p.h_scales[((int64_t)b * p.cap + t0) * p.ng + k];
-    for (int k = tid; k < p.ng * NT * 8; k += blockDim.x)
-        fac[k] = p.qfac[(int64_t)b * p.ng * NT * 8 + k];
+    // the tile's scales (whole 16-byte pieces by cp.async, a ragged end by plain
+    // loads: nothing past the tile is read) and the factors
+    const __half *ssrc = p.h_scales + ((int64_t)b * p.cap + t0) * p.ng;
+    const uint32_t skb = smem_u32(sk);
+    const int nsk = nrow * p.ng;                        // halves
+    for (int k = tid; k < nsk / 8; k += blockDim.x) cp_async16(skb + 16 * k, ssrc + 8 * k);
+    if (tid < nsk % 8) sk[nsk / 8 * 8 + tid] = ssrc[nsk / 8 * 8 + tid];
+    const uint8_t *fsrc = reinterpret_cast<const uint8_t *>(p.qfac + (int64_t)b * p.ng * NT * 8);
+    const uint32_t fb = smem_u32(fac);
+    for (int k = tid; k < p.ng * NT * 8 * 4 / 16; k += blockDim.x) cp_async16(fb + 16 * k, fsrc + 16 * k);
     cp_async_wait_all();
     __syncthreads();
     grid_launch_dependents();
@@ -353,7 +367,9 @@ __global__ void __launch_bounds__(128) absorb_pv_kernel(AbsorbParams p)
         if (tid < p.Hq) {
             const float2 *st = p.stats + ((int64_t)b * p.Hq + tid) * p.ntile;
             const int nt = (len + p.T2 - 1) / p.T2;
+#pragma unroll 8
             for (int k = 0; k < nt; k++) M = fmaxf(M, st[k].x);
+#pragma unroll 8
             for (int k = 0; k < nt; k++) L += st[k].y * exp2f(st[k].x - M);
         }
         hm[tid] = M;
@@ -381,8 +397,11 @@ __global__ void __launch_bounds__(128) absorb_pv_kernel(AbsorbParams p)
             const int t = k / c16, c = k % c16;
             cp_async16(scb + t * cb + 16 * c, p.h_codes + ((int64_t)b * p.cap + tb0 + t) * rowb + g * cb + 16 * c);
         }
-        for (int t = tid; t < nb; t += blockDim.x)
-            sv[t] = __half2float(p.h_scales[((int64_t)b * p.cap + tb0 + t) * p.ng + g]);
+#pragma unroll
+        for (int r = 0; r < TB / 128; r++) {
+            const int t = tid + 128 * r;
+            if (t < nb) sv[t] = __half2float(p.h_scales[((int64_t)b * p.cap + tb0 + t) * p.ng + g]);
+        }
         cp_async_wait_all();
         __syncthreads();
         for (int c0 = 0; c0 < nb; c0 += TC) {
@@ -492,14 +511,16 @@ __global__ void __launch_bounds__(256) absorb_out_kernel(AbsorbParams p)
     for (int q0 = 0; q0 < nq; q0 += 8) {
         const int nqc = min(8, nq - q0);
         __syncthreads();
+#pragma unroll 4
         for (int k = threadIdx.x; k < nqc * D4; k += blockDim.x) {
             const int c = k / D4, d4 = k % D4;
             const int qi = q0 + c, b = qi / G, h = j * G + qi % G;
             const int ns = (seq_len(p, b) + p.split - 1) / p.split;
             float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
             for (int sidx = 0; sidx < ns; sidx++) {
-                const float4 x = reinterpret_cast<const float4 *>(
-                    p.obp + (((int64_t)sidx * p.B + b) * p.Hq + h) * p.D)[d4];
+                const float4 x = __ldg(reinterpret_cast<const float4 *>(
+                    p.obp + (((int64_t)sidx * p.B + b) * p.Hq + h) * p.D) + d4);
                 v.x += x.x; v.y += x.y; v.z += x.z; v.w += x.w;
             }
             reinterpret_cast<float4 *>(obs)[(size_t)c * D4 + d4] = v;
