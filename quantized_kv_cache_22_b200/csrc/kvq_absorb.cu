@@ -36,13 +36,6 @@ namespace {
 
 constexpr unsigned FULL = 0xffffffffu;
 
-__device__ __forceinline__ float load_qf(const void *q, int dtype, int64_t i)
-{
-    if (dtype == KVQ_F32) return static_cast<const float *>(q)[i];
-    if (dtype == KVQ_F16) return __half2float(static_cast<const __half *>(q)[i]);
-    return __bfloat162float(static_cast<const __nv_bfloat16 *>(q)[i]);
-}
-
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src)
 {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -79,25 +72,52 @@ template <int DH>
 __global__ void __launch_bounds__(128) absorb_q_kernel(AbsorbParams p)
 {
     __shared__ float qs[8][DH];
-    __shared__ float part[8][8][128 + 4];    // [row group][query][column]
+    // the W_k tile [DH][128] bf16 while it is read, then the row-group partials
+    __shared__ __align__(16) float wpart[8 * 8 * (128 + 4)];
+    const __nv_bfloat16 *wt = reinterpret_cast<const __nv_bfloat16 *>(wpart);   // [DH][128]
+    float (*part)[8][128 + 4] = reinterpret_cast<float (*)[8][128 + 4]>(wpart);   // [rg][query][col]
+    static_assert(DH * 128 * 2 <= 8 * 8 * (128 + 4) * 4, "W tile fits the partials buffer");
     const int j = blockIdx.x, tile = blockIdx.y;
     const int tid = threadIdx.x;
     const int G = p.Hq / p.Hkv;
     const int nq = p.B * G;
     const int q0 = blockIdx.z * 8;
     const int nqc = min(8, nq - q0);
+    // W_k does not depend on earlier launches: its copies start before the wait
+    {
+        const uint32_t wb = smem_u32(wpart);
+        const __nv_bfloat16 *src = p.w + (int64_t)j * DH * p.D + tile * 128;
+#pragma unroll
+        for (int r = 0; r < DH * 16 / 128; r++) {
+            const int k = tid + 128 * r, row = k / 16, c = k % 16;
+            cp_async16(wb + row * 256 + 16 * c, src + (int64_t)row * p.D + 8 * c);
+        }
+    }
     grid_dependency_wait();
     {
-        float v[8 * DH / 128];                 // all loads in flight before the stores
+        // all loads in flight before the stores (one dtype branch for the lot)
+        constexpr int R = 8 * DH / 128;
+        float v[R];
+        int64_t idx[R];
 #pragma unroll
-        for (int r = 0; r < 8 * DH / 128; r++) {
+        for (int r = 0; r < R; r++) {
             const int k = tid + 128 * r, c = k / DH, i = k % DH;
-            v[r] = 0.f;
-            if (c < nqc) {
-                const int qi = q0 + c, b = qi / G, h = j * G + qi % G;
-                v[r] = load_qf(p.q, p.q_dtype, ((int64_t)b * p.Hq + h) * DH + i);
-            }
+            const int qi = q0 + min(c, nqc - 1), b = qi / G, h = j * G + qi % G;
+            idx[r] = ((int64_t)b * p.Hq + h) * DH + i;
         }
+        if (p.q_dtype == KVQ_F32) {
+#pragma unroll
+            for (int r = 0; r < R; r++) v[r] = __ldg(static_cast<const float *>(p.q) + idx[r]);
+        } else if (p.q_dtype == KVQ_F16) {
+#pragma unroll
+            for (int r = 0; r < R; r++) v[r] = __half2float(static_cast<const __half *>(p.q)[idx[r]]);
+        } else {
+#pragma unroll
+            for (int r = 0; r < R; r++) v[r] = __bfloat162float(static_cast<const __nv_bfloat16 *>(p.q)[idx[r]]);
+        }
+#pragma unroll
+        for (int r = 0; r < R; r++)
+            if ((tid + 128 * r) / DH >= nqc) v[r] = 0.f;
 #pragma unroll
         for (int r = 0; r < 8 * DH / 128; r++) {
             const int k = tid + 128 * r;
@@ -112,11 +132,11 @@ __global__ void __launch_bounds__(128) absorb_q_kernel(AbsorbParams p)
     for (int c = 0; c < 8; c++)
 #pragma unroll
         for (int e = 0; e < 8; e++) acc[c][e] = 0.f;
-    const uint4 *wp = reinterpret_cast<const uint4 *>(p.w + ((int64_t)j * DH + rg) * p.D + c0);
-    const int64_t rstep = (int64_t)p.D;     // 8 rows, in uint4 units
-#pragma unroll 8
+    cp_async_wait_all();
+    __syncthreads();
+#pragma unroll 4
     for (int k = 0; k < DH / 8; k++) {
-        const uint4 w = __ldg(wp + k * rstep);
+        const uint4 w = *reinterpret_cast<const uint4 *>(wt + (rg + 8 * k) * 128 + cg * 8);
         const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
         float wf[8];
 #pragma unroll
@@ -131,6 +151,7 @@ __global__ void __launch_bounds__(128) absorb_q_kernel(AbsorbParams p)
             for (int e = 0; e < 8; e++) acc[c][e] = fmaf(qv, wf[e], acc[c][e]);
         }
     }
+    __syncthreads();                          // the W tile is consumed: reuse it for the partials
 #pragma unroll
     for (int c = 0; c < 8; c++)
 #pragma unroll
@@ -179,17 +200,19 @@ __global__ void __launch_bounds__(128) absorb_q_kernel(AbsorbParams p)
 }
 
 // ---------------------------------------------------------------- scores
-// Grid (token tiles of T, B), T / 16 warps of 16 tokens x all heads.  The tile's
+// Grid (token tiles of T <= 64, B), 8 warps: warp w takes 16 tokens (w mod 4) x all
+// heads over half of the scale groups (w / 4), the halves summed in shared memory.  The tile's
 // codes (rows padded by 16 bytes: conflict-free fragment loads), this sequence's
 // query fragments, the tile's scales and the factors are staged by cp.async.
 // Scores in log2 units, s[b][h][t] = sum_g s_h(t, g) * qfac[g][h] * (254 acc_hi +
 // acc_lo), written for t < len; the tile's (max, sum 2^(s - max)) per head go to
 // stats[b][h][tile].
 template <int BITS, int NT>
-__global__ void __launch_bounds__(128) absorb_scores_kernel(AbsorbParams p)
+__global__ void __launch_bounds__(256) absorb_scores_kernel(AbsorbParams p)
 {
     extern __shared__ __align__(16) uint8_t sm[];
     __shared__ float red[4][NT * 8];
+    __shared__ float half2s[4][NT * 4][32];    // second group half's partial scores
     __shared__ float tmax[NT * 8];
     const int T = p.T2;
     const int b = blockIdx.y;
@@ -230,7 +253,8 @@ __global__ void __launch_bounds__(128) absorb_scores_kernel(AbsorbParams p)
     __syncthreads();
     grid_launch_dependents();
 
-    const int warp = tid >> 5, lane = tid & 31, gid = lane >> 2, tig = lane & 3;
+    const int wq = tid >> 5, lane = tid & 31, gid = lane >> 2, tig = lane & 3;
+    const int warp = wq & 3, gh = wq >> 2;    // token block, group half
     const int r0 = warp * 16 + gid, r1 = r0 + 8;
     const bool active = warp * 16 < nrow;     // inactive warps still join the reductions
     float s[NT][4];
@@ -238,7 +262,8 @@ __global__ void __launch_bounds__(128) absorb_scores_kernel(AbsorbParams p)
     for (int nt = 0; nt < NT; nt++) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
     if (active) {
         const int ksg = p.group / 32;                   // k-steps per scale group
-        for (int g = 0; g < p.ng; g++) {
+        const int ghn = p.ng / 2;                       // groups per half (ng is even)
+        for (int g = gh * ghn; g < (gh + 1) * ghn; g++) {
             int ah[NT][4], al[NT][4];
 #pragma unroll
             for (int nt = 0; nt < NT; nt++)
@@ -281,8 +306,20 @@ __global__ void __launch_bounds__(128) absorb_scores_kernel(AbsorbParams p)
             }
         }
     }
-    // rows past the length (or of an inactive warp) take no part
-    const bool v0 = active && r0 < nrow, v1 = active && r1 < nrow;
+    // the second half's partial scores join the first half's
+    if (gh == 1)
+#pragma unroll
+        for (int nt = 0; nt < NT; nt++)
+#pragma unroll
+            for (int e = 0; e < 4; e++) half2s[warp][nt * 4 + e][lane] = s[nt][e];
+    __syncthreads();
+    if (gh == 0)
+#pragma unroll
+        for (int nt = 0; nt < NT; nt++)
+#pragma unroll
+            for (int e = 0; e < 4; e++) s[nt][e] += half2s[warp][nt * 4 + e][lane];
+    // rows past the length (or of an inactive warp, or the second half) take no part
+    const bool v0 = gh == 0 && active && r0 < nrow, v1 = gh == 0 && active && r1 < nrow;
 #pragma unroll
     for (int nt = 0; nt < NT; nt++) {
         s[nt][0] = v0 ? s[nt][0] : -INFINITY;
@@ -306,12 +343,12 @@ __global__ void __launch_bounds__(128) absorb_scores_kernel(AbsorbParams p)
         for (int c = 0; c < 2; c++) {
             float m = fmaxf(s[nt][c], s[nt][2 + c]);
             for (int off = 4; off < 32; off <<= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, off));
-            if (gid == 0) red[warp][nt * 8 + 2 * tig + c] = m;
+            if (gid == 0 && gh == 0) red[warp][nt * 8 + 2 * tig + c] = m;
         }
     __syncthreads();
     if (tid < NT * 8) {
         float m = red[0][tid];
-        for (int w = 1; w < (int)(blockDim.x >> 5); w++) m = fmaxf(m, red[w][tid]);
+        for (int w = 1; w < 4; w++) m = fmaxf(m, red[w][tid]);
         tmax[tid] = m;
     }
     __syncthreads();
@@ -323,12 +360,12 @@ __global__ void __launch_bounds__(128) absorb_scores_kernel(AbsorbParams p)
             float l = (s[nt][c] == -INFINITY ? 0.f : exp2f(s[nt][c] - m)) +
                       (s[nt][2 + c] == -INFINITY ? 0.f : exp2f(s[nt][2 + c] - m));
             for (int off = 4; off < 32; off <<= 1) l += __shfl_xor_sync(FULL, l, off);
-            if (gid == 0) red[warp][nt * 8 + 2 * tig + c] = l;
+            if (gid == 0 && gh == 0) red[warp][nt * 8 + 2 * tig + c] = l;
         }
     __syncthreads();
     if (tid < p.Hq) {
         float l = 0.f;
-        for (int w = 0; w < (int)(blockDim.x >> 5); w++) l += red[w][tid];
+        for (int w = 0; w < 4; w++) l += red[w][tid];
         p.stats[((int64_t)b * p.Hq + tid) * p.ntile + blockIdx.x] = make_float2(tmax[tid], l);
     }
 }
@@ -508,14 +545,20 @@ __global__ void __launch_bounds__(256) absorb_out_kernel(AbsorbParams p)
     grid_dependency_wait();
     const uint4 *wr = reinterpret_cast<const uint4 *>(p.w + ((int64_t)p.Hkv * p.Dh + (int64_t)j * p.Dh + i) * p.D);
     const int per = p.D / 256;                      // uint4 per lane over the row
+    __shared__ int qns[8];                          // token splits of each query's sequence
     for (int q0 = 0; q0 < nq; q0 += 8) {
         const int nqc = min(8, nq - q0);
+        __syncthreads();
+        if (threadIdx.x < 8) {
+            const int qi = q0 + min((int)threadIdx.x, nqc - 1);
+            qns[threadIdx.x] = (seq_len(p, qi / G) + p.split - 1) / p.split;
+        }
         __syncthreads();
 #pragma unroll 4
         for (int k = threadIdx.x; k < nqc * D4; k += blockDim.x) {
             const int c = k / D4, d4 = k % D4;
             const int qi = q0 + c, b = qi / G, h = j * G + qi % G;
-            const int ns = (seq_len(p, b) + p.split - 1) / p.split;
+            const int ns = qns[c];
             float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
             for (int sidx = 0; sidx < ns; sidx++) {
@@ -617,7 +660,7 @@ cudaError_t launch_scores(const AbsorbParams &p, int max_len, cudaStream_t st)
     cudaError_t e = set_smem(absorb_scores_kernel<BITS, NT>, smem);
     if (e != cudaSuccess) return e;
     (void)max_len;
-    return launch_pdl(absorb_scores_kernel<BITS, NT>, dim3(p.ntile, p.B), dim3(128), smem, st, p);
+    return launch_pdl(absorb_scores_kernel<BITS, NT>, dim3(p.ntile, p.B), dim3(256), smem, st, p);
 }
 
 template <int BITS, int MT>
