@@ -451,32 +451,31 @@ __global__ void __launch_bounds__(128) absorb_pv_kernel(AbsorbParams p)
                     v = exp2f(ss[h * TB + c0 + t] - hm[h]) * hinv[h] * sv[c0 + t];
                 pt[h * TS + t] = __float2half_rn(v);
             }
+            // Each 8-element run of codes becomes 4 half2 in a permuted element order
+            // (VPERM below), with the exponent-bias conversion: a code sits in the
+            // mantissa of 1024 (sign-flipped: 1152 + c for bytes, 1032 + c for
+            // nibbles) and one half2 subtraction leaves the exact code.
             for (int k = tid; k < TC * (GS / 8); k += blockDim.x) {
                 const int t = k / (GS / 8), d8 = 8 * (k % (GS / 8));
-                int c[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+                uint32_t pk[4] = {0u, 0u, 0u, 0u};
                 if (t < nc) {
                     const uint8_t *row = sc + (size_t)(c0 + t) * cb;
                     if constexpr (BITS == 8) {
+                        // halves (e0, e2), (e1, e3), (e4, e6), (e5, e7)
                         const uint2 w = *reinterpret_cast<const uint2 *>(row + d8);
-#pragma unroll
-                        for (int i = 0; i < 4; i++) {
-                            c[i] = (int)(int8_t)(w.x >> (8 * i));
-                            c[4 + i] = (int)(int8_t)(w.y >> (8 * i));
-                        }
+                        const uint32_t B = 0x64806480u, SUB = 0x64806480u;   // 1152
+                        pk[0] = hsub2_u32(and_xor(w.x, 0x00FF00FFu, B), SUB);
+                        pk[1] = hsub2_u32(and_xor(w.x >> 8, 0x00FF00FFu, B), SUB);
+                        pk[2] = hsub2_u32(and_xor(w.y, 0x00FF00FFu, B), SUB);
+                        pk[3] = hsub2_u32(and_xor(w.y >> 8, 0x00FF00FFu, B), SUB);
                     } else {
-                        const uint32_t w = *reinterpret_cast<const uint32_t *>(row + d8 / 2);
+                        // halves (e0, e4), (e1, e5), (e2, e6), (e3, e7)
+                        const uint32_t w = *reinterpret_cast<const uint32_t *>(row + d8 / 2) ^ 0x88888888u;
+                        const uint32_t SUB = 0x64086408u;                   // 1032
 #pragma unroll
-                        for (int i = 0; i < 8; i++) {
-                            const int nib = (int)((w >> (4 * i)) & 0xFu);
-                            c[i] = nib >= 8 ? nib - 16 : nib;
-                        }
+                        for (int i = 0; i < 4; i++)
+                            pk[i] = hsub2_u32(((w >> (4 * i)) & 0x000F000Fu) | 0x64006400u, SUB);
                     }
-                }
-                uint32_t pk[4];
-#pragma unroll
-                for (int i = 0; i < 4; i++) {
-                    const __half2 h2 = __halves2half2(__int2half_rn(c[2 * i]), __int2half_rn(c[2 * i + 1]));
-                    pk[i] = *reinterpret_cast<const uint32_t *>(&h2);
                 }
                 *reinterpret_cast<uint4 *>(vt + t * VS + d8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
@@ -513,39 +512,49 @@ __global__ void __launch_bounds__(128) absorb_pv_kernel(AbsorbParams p)
     }
     grid_launch_dependents();
     float *ob = p.obp + ((int64_t)split * p.B + b) * p.Hq * p.D;
+    // accumulator columns 2tig, 2tig + 1 hold elements VPERM of the n-tile's 8 columns
+    const int e0 = BITS == 8 ? ((tig & 1) + 4 * (tig >> 1)) : tig;
+    const int e1 = BITS == 8 ? e0 + 2 : tig + 4;
 #pragma unroll
     for (int n = 0; n < 4; n++) {
         if (n >= ntw) break;
-        const int d = g * GS + (warp * ntw + n) * 8 + 2 * tig;
+        const int d = g * GS + (warp * ntw + n) * 8;
 #pragma unroll
         for (int mt = 0; mt < MT; mt++) {
             const int h0 = mt * 16 + gid, h1 = h0 + 8;
-            if (h0 < p.Hq)
-                *reinterpret_cast<float2 *>(ob + (int64_t)h0 * p.D + d) = make_float2(acc[mt][n][0], acc[mt][n][1]);
-            if (h1 < p.Hq)
-                *reinterpret_cast<float2 *>(ob + (int64_t)h1 * p.D + d) = make_float2(acc[mt][n][2], acc[mt][n][3]);
+            if (h0 < p.Hq) {
+                ob[(int64_t)h0 * p.D + d + e0] = acc[mt][n][0];
+                ob[(int64_t)h0 * p.D + d + e1] = acc[mt][n][1];
+            }
+            if (h1 < p.Hq) {
+                ob[(int64_t)h1 * p.D + d + e0] = acc[mt][n][2];
+                ob[(int64_t)h1 * p.D + d + e1] = acc[mt][n][3];
+            }
         }
     }
 }
 
 // ---------------------------------------------------------------- W_v . ob
-// Grid (Hkv, Dh / 8), 8 warps: warp w computes row i = 8 * blockIdx.y + w of
+// Grid (Hkv, Dh / 32), 8 warps: warp w computes rows 32 * blockIdx.y + 4w .. +3 of
 // W_v,j against the ob of every query of KV head j (B * G of them, 8 at a time),
 // ob being the sum of the sequence's token-split partials, staged in shared
-// memory.  The row is read once, 16 bytes per lane and load.
+// memory.  Lane l reads columns 128k + 4l .. +3 (one 16-byte shared load per query
+// feeds 4 rows, conflict-free; 8 bytes of each W row per global load).
 __global__ void __launch_bounds__(256) absorb_out_kernel(AbsorbParams p)
 {
     extern __shared__ __align__(16) float obs[];    // [8][D]
+    __shared__ int qns[8];                          // token splits of each query's sequence
     const int j = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int i = blockIdx.y * 8 + warp;
+    const int i0 = blockIdx.y * 32 + warp * 4;
     const int G = p.Hq / p.Hkv;
     const int nq = p.B * G;
     const int D4 = p.D / 4;
     grid_dependency_wait();
-    const uint4 *wr = reinterpret_cast<const uint4 *>(p.w + ((int64_t)p.Hkv * p.Dh + (int64_t)j * p.Dh + i) * p.D);
-    const int per = p.D / 256;                      // uint4 per lane over the row
-    __shared__ int qns[8];                          // token splits of each query's sequence
+    const uint2 *wr[4];
+#pragma unroll
+    for (int r = 0; r < 4; r++)
+        wr[r] = reinterpret_cast<const uint2 *>(p.w + ((int64_t)p.Hkv * p.Dh + (int64_t)j * p.Dh + i0 + r) * p.D);
     for (int q0 = 0; q0 < nq; q0 += 8) {
         const int nqc = min(8, nq - q0);
         __syncthreads();
@@ -569,51 +578,52 @@ __global__ void __launch_bounds__(256) absorb_out_kernel(AbsorbParams p)
             reinterpret_cast<float4 *>(obs)[(size_t)c * D4 + d4] = v;
         }
         __syncthreads();
-        float acc[8];
+        float acc[4][8];
 #pragma unroll
-        for (int c = 0; c < 8; c++) acc[c] = 0.f;
-        for (int k0 = 0; k0 < per; k0 += 8) {
-            uint4 w[8];
+        for (int r = 0; r < 4; r++)
 #pragma unroll
-            for (int k = 0; k < 8; k++) w[k] = (k0 + k < per) ? __ldg(wr + lane + 32 * (k0 + k)) : make_uint4(0, 0, 0, 0);
+            for (int c = 0; c < 8; c++) acc[r][c] = 0.f;
+        for (int kk = 0; kk < p.D / 128; kk++) {
+            const int d0 = 128 * kk + 4 * lane;
+            float wf[4][4];
 #pragma unroll
-            for (int k = 0; k < 8; k++) {
-                if (k0 + k >= per) break;
-                const int d0 = 8 * (lane + 32 * (k0 + k));
-                const uint32_t ws[4] = {w[k].x, w[k].y, w[k].z, w[k].w};
-                float wf[8];
+            for (int r = 0; r < 4; r++) {
+                const uint2 w = __ldg(wr[r] + d0 / 4);
+                wf[r][0] = __uint_as_float(w.x << 16);
+                wf[r][1] = __uint_as_float(w.x & 0xFFFF0000u);
+                wf[r][2] = __uint_as_float(w.y << 16);
+                wf[r][3] = __uint_as_float(w.y & 0xFFFF0000u);
+            }
 #pragma unroll
-                for (int e = 0; e < 4; e++) {
-                    wf[2 * e] = __uint_as_float(ws[e] << 16);
-                    wf[2 * e + 1] = __uint_as_float(ws[e] & 0xFFFF0000u);
-                }
+            for (int c = 0; c < 8; c++) {
+                if (c >= nqc) break;
+                const float4 o = *reinterpret_cast<const float4 *>(obs + (size_t)c * p.D + d0);
 #pragma unroll
-                for (int c = 0; c < 8; c++) {
-                    if (c >= nqc) break;
-                    const float4 o0 = *reinterpret_cast<const float4 *>(obs + (size_t)c * p.D + d0);
-                    const float4 o1 = *reinterpret_cast<const float4 *>(obs + (size_t)c * p.D + d0 + 4);
-                    float a = acc[c];
-                    a = fmaf(wf[0], o0.x, a); a = fmaf(wf[1], o0.y, a);
-                    a = fmaf(wf[2], o0.z, a); a = fmaf(wf[3], o0.w, a);
-                    a = fmaf(wf[4], o1.x, a); a = fmaf(wf[5], o1.y, a);
-                    a = fmaf(wf[6], o1.z, a); a = fmaf(wf[7], o1.w, a);
-                    acc[c] = a;
+                for (int r = 0; r < 4; r++) {
+                    float a = acc[r][c];
+                    a = fmaf(wf[r][0], o.x, a);
+                    a = fmaf(wf[r][1], o.y, a);
+                    a = fmaf(wf[r][2], o.z, a);
+                    a = fmaf(wf[r][3], o.w, a);
+                    acc[r][c] = a;
                 }
             }
         }
 #pragma unroll
-        for (int c = 0; c < 8; c++) {
-            float v = acc[c];
-            for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(FULL, v, off);
-            if (lane == 0 && c < nqc) {
-                const int qi = q0 + c, b = qi / G, h = j * G + qi % G;
-                const int64_t o = ((int64_t)b * p.Hq + h) * p.Dh + i;
-                if (p.out_f32)
-                    static_cast<float *>(p.out)[o] = v;
-                else
-                    static_cast<__half *>(p.out)[o] = __float2half_rn(v);
+        for (int r = 0; r < 4; r++)
+#pragma unroll
+            for (int c = 0; c < 8; c++) {
+                float v = acc[r][c];
+                for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(FULL, v, off);
+                if (lane == 0 && c < nqc) {
+                    const int qi = q0 + c, b = qi / G, h = j * G + qi % G;
+                    const int64_t o = ((int64_t)b * p.Hq + h) * p.Dh + i0 + r;
+                    if (p.out_f32)
+                        static_cast<float *>(p.out)[o] = v;
+                    else
+                        static_cast<__half *>(p.out)[o] = __float2half_rn(v);
+                }
             }
-        }
     }
 }
 
@@ -739,7 +749,7 @@ cudaError_t launch_absorbed(const AbsorbParams &p, int max_len, cudaStream_t str
     }
     const size_t osm = (size_t)8 * p.D * 4;
     if ((e = set_smem(absorb_out_kernel, osm)) != cudaSuccess) return e;
-    return launch_pdl(absorb_out_kernel, dim3(p.Hkv, p.Dh / 8), dim3(256), osm, stream, p);
+    return launch_pdl(absorb_out_kernel, dim3(p.Hkv, p.Dh / 32), dim3(256), osm, stream, p);
 }
 
 }  // namespace kvq

@@ -245,6 +245,14 @@ __device__ __forceinline__ uint32_t e4m3x2_to_half2(uint32_t x)
     return r;
 }
 
+// half2 difference of two packed half2 words
+__device__ __forceinline__ uint32_t hsub2_u32(uint32_t a, uint32_t b)
+{
+    uint32_t r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
 // half2 sum of two packed half2 words
 __device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b)
 {
