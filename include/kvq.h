@@ -330,7 +330,8 @@ KVQ_API int kvq_h_reconstruct(const kvq_config *cfg, const kvq_layer *layer, con
  * tensor-core scores (relative error below 2^-15 of the group's largest
  * element) and p * scale enters the p . h^ product in fp16; everything else
  * accumulates in fp32.  An empty sequence gets zeros.
- *   h_bits 4 or 8; Hkv*Dh = D, D a multiple of 256, Dh 64 or 128; Hq <= 32.
+ *   h_bits 4 or 8; Hkv*Dh = D, D a multiple of 256 and at most 3584, Dh 64 or
+ *   128; Hq <= 32 (smaller limits where the score tile's shared memory runs out).
  *   w_kv     device bf16 [2*Hkv*Dh][D] (as kvq_decode_attn)
  *   q, q_dtype, d_len, max_len_host, softmax_scale, out, out_dtype: as
  *            kvq_decode_attn (max_len_host bounds d_len[] and sizes the scratch)

@@ -412,6 +412,7 @@ __global__ void __launch_bounds__(128) absorb_pv_kernel(AbsorbParams p)
         hm[tid] = M;
         hinv[tid] = L > 0.f ? 1.f / L : 0.f;
     }
+    grid_launch_dependents();
     const int ntw = GS / 32;                       // n-tiles of 8 columns per warp (1, 2 or 4)
     float acc[MT][4][4];
 #pragma unroll
@@ -510,7 +511,6 @@ __global__ void __launch_bounds__(128) absorb_pv_kernel(AbsorbParams p)
             }
         }
     }
-    grid_launch_dependents();
     float *ob = p.obp + ((int64_t)split * p.B + b) * p.Hq * p.D;
     // accumulator columns 2tig, 2tig + 1 hold elements VPERM of the n-tile's 8 columns
     const int e0 = BITS == 8 ? ((tig & 1) + 4 * (tig >> 1)) : tig;
@@ -535,26 +535,30 @@ __global__ void __launch_bounds__(128) absorb_pv_kernel(AbsorbParams p)
 }
 
 // ---------------------------------------------------------------- W_v . ob
-// Grid (Hkv, Dh / 32), 8 warps: warp w computes rows 32 * blockIdx.y + 4w .. +3 of
+// Grid (Hkv, Dh / 16), 8 warps: warp w computes rows 16 * blockIdx.y + 2w, +1 of
 // W_v,j against the ob of every query of KV head j (B * G of them, 8 at a time),
-// ob being the sum of the sequence's token-split partials, staged in shared
-// memory.  Lane l reads columns 128k + 4l .. +3 (one 16-byte shared load per query
-// feeds 4 rows, conflict-free; 8 bytes of each W row per global load).
+// ob being the sum of the sequence's token-split partials.  The CTA's 16 W_v rows
+// are copied to shared memory (cp.async) before the wait for the previous launch,
+// so that they stream in while it finishes; ob is staged after it.  Lane l reads
+// columns 128k + 4l .. +3: conflict-free 16-byte loads of ob, 8-byte loads of W.
 __global__ void __launch_bounds__(256) absorb_out_kernel(AbsorbParams p)
 {
-    extern __shared__ __align__(16) float obs[];    // [8][D]
+    extern __shared__ __align__(16) float obs[];    // [8][D] fp32, then [16][D] bf16 rows of W_v
     __shared__ int qns[8];                          // token splits of each query's sequence
     const int j = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int i0 = blockIdx.y * 32 + warp * 4;
+    const int rbase = blockIdx.y * 16;
     const int G = p.Hq / p.Hkv;
     const int nq = p.B * G;
     const int D4 = p.D / 4;
+    __nv_bfloat16 *ws = reinterpret_cast<__nv_bfloat16 *>(obs + (size_t)8 * p.D);
+    {
+        const uint32_t wb = smem_u32(ws);
+        const __nv_bfloat16 *src = p.w + ((int64_t)p.Hkv * p.Dh + (int64_t)j * p.Dh + rbase) * p.D;
+        const int pieces = 16 * p.D / 8;            // 16-byte pieces of the 16 rows
+        for (int k = threadIdx.x; k < pieces; k += blockDim.x) cp_async16(wb + 16 * k, src + 8 * k);
+    }
     grid_dependency_wait();
-    const uint2 *wr[4];
-#pragma unroll
-    for (int r = 0; r < 4; r++)
-        wr[r] = reinterpret_cast<const uint2 *>(p.w + ((int64_t)p.Hkv * p.Dh + (int64_t)j * p.Dh + i0 + r) * p.D);
     for (int q0 = 0; q0 < nq; q0 += 8) {
         const int nqc = min(8, nq - q0);
         __syncthreads();
@@ -563,7 +567,7 @@ __global__ void __launch_bounds__(256) absorb_out_kernel(AbsorbParams p)
             qns[threadIdx.x] = (seq_len(p, qi / G) + p.split - 1) / p.split;
         }
         __syncthreads();
-#pragma unroll 4
+#pragma unroll 8
         for (int k = threadIdx.x; k < nqc * D4; k += blockDim.x) {
             const int c = k / D4, d4 = k % D4;
             const int qi = q0 + c, b = qi / G, h = j * G + qi % G;
@@ -577,18 +581,19 @@ __global__ void __launch_bounds__(256) absorb_out_kernel(AbsorbParams p)
             }
             reinterpret_cast<float4 *>(obs)[(size_t)c * D4 + d4] = v;
         }
+        cp_async_wait_all();
         __syncthreads();
-        float acc[4][8];
+        float acc[2][8];
 #pragma unroll
-        for (int r = 0; r < 4; r++)
+        for (int r = 0; r < 2; r++)
 #pragma unroll
             for (int c = 0; c < 8; c++) acc[r][c] = 0.f;
         for (int kk = 0; kk < p.D / 128; kk++) {
             const int d0 = 128 * kk + 4 * lane;
-            float wf[4][4];
+            float wf[2][4];
 #pragma unroll
-            for (int r = 0; r < 4; r++) {
-                const uint2 w = __ldg(wr[r] + d0 / 4);
+            for (int r = 0; r < 2; r++) {
+                const uint2 w = *reinterpret_cast<const uint2 *>(ws + (size_t)(2 * warp + r) * p.D + d0);
                 wf[r][0] = __uint_as_float(w.x << 16);
                 wf[r][1] = __uint_as_float(w.x & 0xFFFF0000u);
                 wf[r][2] = __uint_as_float(w.y << 16);
@@ -599,7 +604,7 @@ __global__ void __launch_bounds__(256) absorb_out_kernel(AbsorbParams p)
                 if (c >= nqc) break;
                 const float4 o = *reinterpret_cast<const float4 *>(obs + (size_t)c * p.D + d0);
 #pragma unroll
-                for (int r = 0; r < 4; r++) {
+                for (int r = 0; r < 2; r++) {
                     float a = acc[r][c];
                     a = fmaf(wf[r][0], o.x, a);
                     a = fmaf(wf[r][1], o.y, a);
@@ -610,14 +615,14 @@ __global__ void __launch_bounds__(256) absorb_out_kernel(AbsorbParams p)
             }
         }
 #pragma unroll
-        for (int r = 0; r < 4; r++)
+        for (int r = 0; r < 2; r++)
 #pragma unroll
             for (int c = 0; c < 8; c++) {
                 float v = acc[r][c];
                 for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(FULL, v, off);
                 if (lane == 0 && c < nqc) {
                     const int qi = q0 + c, b = qi / G, h = j * G + qi % G;
-                    const int64_t o = ((int64_t)b * p.Hq + h) * p.Dh + i0 + r;
+                    const int64_t o = ((int64_t)b * p.Hq + h) * p.Dh + rbase + 2 * warp + r;
                     if (p.out_f32)
                         static_cast<float *>(p.out)[o] = v;
                     else
@@ -687,6 +692,14 @@ cudaError_t launch_pv(const AbsorbParams &p, int max_len, cudaStream_t st)
 
 int absorb_nt(int Hq) { return Hq <= 8 ? 1 : (Hq <= 16 ? 2 : 4); }
 
+// The shape fits the kernels' shared memory: a 16-token score tile with the query
+// fragments, and an 8-query ob chunk with 16 W_v rows.
+bool absorb_fits(int D, int bits, int Hq, int ng)
+{
+    return scores_smem(D, bits, absorb_nt(Hq), ng, 16) <= 227 * 1024 &&
+           (size_t)8 * D * 4 + (size_t)16 * D * 2 <= 227 * 1024;
+}
+
 // Tokens per score tile: 64 (4 warps), fewer when the tile and the fragments
 // outgrow shared memory.
 int absorb_t2(int D, int bits, int Hq, int ng)
@@ -747,9 +760,9 @@ cudaError_t launch_absorbed(const AbsorbParams &p, int max_len, cudaStream_t str
                         : (two ? launch_pv<4, 2>(p, max_len, stream) : launch_pv<4, 1>(p, max_len, stream));
         if (e != cudaSuccess) return e;
     }
-    const size_t osm = (size_t)8 * p.D * 4;
+    const size_t osm = (size_t)8 * p.D * 4 + (size_t)16 * p.D * 2;   // ob chunk + 16 W_v rows
     if ((e = set_smem(absorb_out_kernel, osm)) != cudaSuccess) return e;
-    return launch_pdl(absorb_out_kernel, dim3(p.Hkv, p.Dh / 32), dim3(256), osm, stream, p);
+    return launch_pdl(absorb_out_kernel, dim3(p.Hkv, p.Dh / 16), dim3(256), osm, stream, p);
 }
 
 }  // namespace kvq

@@ -762,6 +762,7 @@ static int absorbed_shape_check(const kvq_config *cfg)
     if (cfg->head_dim % 32 != 0 || cfg->head_dim > 128 || cfg->d_model % 256 != 0)
         return KVQ_ERR_UNSUPPORTED;
     if (cfg->n_q_heads % cfg->n_kv_heads != 0 || cfg->n_q_heads > 32) return KVQ_ERR_UNSUPPORTED;
+    if (!absorb_fits(cfg->d_model, cfg->h_bits, cfg->n_q_heads, cfg->h_groups)) return KVQ_ERR_UNSUPPORTED;
     return KVQ_OK;
 }
 

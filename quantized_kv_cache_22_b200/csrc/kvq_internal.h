@@ -112,6 +112,7 @@ struct AbsorbParams {
     int32_t capP, NT, T2, ntile, split;
 };
 int absorb_nt(int Hq);            // n-tiles of 8 query heads in the score MMA: 1, 2 or 4
+bool absorb_fits(int D, int bits, int Hq, int ng);   // shared memory suffices for the shape
 int absorb_t2(int D, int bits, int Hq, int ng);   // tokens per score tile
 int absorb_split(int max_len);    // tokens per split of the p . h^ kernel
 // scratch bytes; off[0..4] = qfrag, qfac, scores, stats, partial ob (256-byte aligned)
