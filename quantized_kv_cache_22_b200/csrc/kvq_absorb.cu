@@ -232,9 +232,17 @@ __global__ void __launch_bounds__(256) absorb_scores_kernel(AbsorbParams p)
     const int chunks = rowb / 16;
     const uint8_t *src = p.h_codes + ((int64_t)b * p.cap + t0) * rowb;
     const uint32_t tb = smem_u32(tile);
-    for (int k = tid; k < nrow * chunks; k += blockDim.x) {
-        const int r = k / chunks, c = k % chunks;
-        cp_async16(tb + r * rs + 16 * c, src + (size_t)r * rowb + 16 * c);
+    {
+        // (row, piece) walk with one division per thread
+        int r = tid / chunks, c = tid % chunks;
+        while (r < nrow) {
+            cp_async16(tb + r * rs + 16 * c, src + (size_t)r * rowb + 16 * c);
+            c += blockDim.x;
+            while (c >= chunks) {
+                c -= chunks;
+                ++r;
+            }
+        }
     }
     const uint4 *qsrc = p.qfrag + (size_t)b * KS * NT * 32;
     const uint32_t qb = smem_u32(qf);
@@ -378,7 +386,7 @@ __global__ void __launch_bounds__(256) absorb_scores_kernel(AbsorbParams p)
 // as exact fp16 integers [t][d] feed f16 MMAs (M = heads, N = the group's
 // columns, K = tokens; the h fragments by ldmatrix.trans), warp w owning a
 // quarter of the columns.  The split's partial ob goes to obp[split][b][h][d].
-template <int BITS, int MT>
+template <int BITS, int MT, int GS>
 __global__ void __launch_bounds__(128) absorb_pv_kernel(AbsorbParams p)
 {
     constexpr int TB = 256, TC = 64, TS = TC + 8, VS = 128 + 8;
@@ -390,8 +398,7 @@ __global__ void __launch_bounds__(128) absorb_pv_kernel(AbsorbParams p)
     __shared__ float hm[MT * 16], hinv[MT * 16];
     __shared__ float sv[TB];
     const int g = blockIdx.x, b = blockIdx.y, split = blockIdx.z;
-    const int GS = p.group;
-    const int cb = GS * BITS / 8;                  // code bytes of the group per token
+    constexpr int cb = GS * BITS / 8;              // code bytes of the group per token
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gid = lane >> 2, tig = lane & 3;
     grid_dependency_wait();
     const int len = seq_len(p, b);
@@ -413,7 +420,7 @@ __global__ void __launch_bounds__(128) absorb_pv_kernel(AbsorbParams p)
         hinv[tid] = L > 0.f ? 1.f / L : 0.f;
     }
     grid_launch_dependents();
-    const int ntw = GS / 32;                       // n-tiles of 8 columns per warp (1, 2 or 4)
+    constexpr int ntw = GS / 32;                   // n-tiles of 8 columns per warp (1, 2 or 4)
     float acc[MT][4][4];
 #pragma unroll
     for (int mt = 0; mt < MT; mt++)
@@ -425,15 +432,18 @@ __global__ void __launch_bounds__(128) absorb_pv_kernel(AbsorbParams p)
         const int nb = min(TB, t_end - tb0);       // tokens of this block (a multiple of 16 but the last)
         __syncthreads();                           // the previous block's data is consumed
         // raw scores [h][t] (16-byte pieces: 4 tokens) and the group's codes [t][cb]
-        const int n4 = (nb + 3) / 4;
-        for (int k = tid; k < p.Hq * n4; k += blockDim.x) {
-            const int h = k / n4, t4 = 4 * (k % n4);
-            cp_async16(ssb + (h * TB + t4) * 4, p.p + ((int64_t)b * p.Hq + h) * p.capP + tb0 + t4);
+#pragma unroll
+        for (int r = 0; r < MT * 16 * (TB / 4) / 128; r++) {
+            const int k = tid + 128 * r, h = k / (TB / 4), t4 = 4 * (k % (TB / 4));
+            if (h < p.Hq && t4 < nb)
+                cp_async16(ssb + (h * TB + t4) * 4, p.p + ((int64_t)b * p.Hq + h) * p.capP + tb0 + t4);
         }
-        const int c16 = cb / 16;
-        for (int k = tid; k < nb * c16; k += blockDim.x) {
-            const int t = k / c16, c = k % c16;
-            cp_async16(scb + t * cb + 16 * c, p.h_codes + ((int64_t)b * p.cap + tb0 + t) * rowb + g * cb + 16 * c);
+        constexpr int c16 = cb / 16;
+#pragma unroll
+        for (int r = 0; r < TB * c16 / 128; r++) {
+            const int k = tid + 128 * r, t = k / c16, c = k % c16;
+            if (t < nb)
+                cp_async16(scb + t * cb + 16 * c, p.h_codes + ((int64_t)b * p.cap + tb0 + t) * rowb + g * cb + 16 * c);
         }
 #pragma unroll
         for (int r = 0; r < TB / 128; r++) {
@@ -567,19 +577,21 @@ __global__ void __launch_bounds__(256) absorb_out_kernel(AbsorbParams p)
             qns[threadIdx.x] = (seq_len(p, qi / G) + p.split - 1) / p.split;
         }
         __syncthreads();
-#pragma unroll 8
-        for (int k = threadIdx.x; k < nqc * D4; k += blockDim.x) {
-            const int c = k / D4, d4 = k % D4;
+        for (int c = 0; c < nqc; c++) {
             const int qi = q0 + c, b = qi / G, h = j * G + qi % G;
             const int ns = qns[c];
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 *src = reinterpret_cast<const float4 *>(p.obp + ((int64_t)b * p.Hq + h) * p.D);
+            const int64_t sstep = (int64_t)p.B * p.Hq * p.D / 4;   // one split, in float4
+#pragma unroll 2
+            for (int d4 = threadIdx.x; d4 < D4; d4 += blockDim.x) {
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
-            for (int sidx = 0; sidx < ns; sidx++) {
-                const float4 x = __ldg(reinterpret_cast<const float4 *>(
-                    p.obp + (((int64_t)sidx * p.B + b) * p.Hq + h) * p.D) + d4);
-                v.x += x.x; v.y += x.y; v.z += x.z; v.w += x.w;
+                for (int sidx = 0; sidx < ns; sidx++) {
+                    const float4 x = __ldg(src + sidx * sstep + d4);
+                    v.x += x.x; v.y += x.y; v.z += x.z; v.w += x.w;
+                }
+                reinterpret_cast<float4 *>(obs)[(size_t)c * D4 + d4] = v;
             }
-            reinterpret_cast<float4 *>(obs)[(size_t)c * D4 + d4] = v;
         }
         cp_async_wait_all();
         __syncthreads();
@@ -678,14 +690,25 @@ cudaError_t launch_scores(const AbsorbParams &p, int max_len, cudaStream_t st)
     return launch_pdl(absorb_scores_kernel<BITS, NT>, dim3(p.ntile, p.B), dim3(256), smem, st, p);
 }
 
+template <int BITS, int MT, int GS>
+cudaError_t launch_pv_gs(const AbsorbParams &p, int max_len, cudaStream_t st)
+{
+    const size_t smem = pv_smem(BITS, MT);
+    cudaError_t e = set_smem(absorb_pv_kernel<BITS, MT, GS>, smem);
+    if (e != cudaSuccess) return e;
+    const int ns = max(1, (max_len + p.split - 1) / p.split);
+    return launch_pdl(absorb_pv_kernel<BITS, MT, GS>, dim3(p.D / GS, p.B, ns), dim3(128), smem, st, p);
+}
+
 template <int BITS, int MT>
 cudaError_t launch_pv(const AbsorbParams &p, int max_len, cudaStream_t st)
 {
-    const size_t smem = pv_smem(BITS, MT);
-    cudaError_t e = set_smem(absorb_pv_kernel<BITS, MT>, smem);
-    if (e != cudaSuccess) return e;
-    const int ns = max(1, (max_len + p.split - 1) / p.split);
-    return launch_pdl(absorb_pv_kernel<BITS, MT>, dim3(p.D / p.group, p.B, ns), dim3(128), smem, st, p);
+    switch (p.group) {
+    case 32: return launch_pv_gs<BITS, MT, 32>(p, max_len, st);
+    case 64: return launch_pv_gs<BITS, MT, 64>(p, max_len, st);
+    case 128: return launch_pv_gs<BITS, MT, 128>(p, max_len, st);
+    default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace
