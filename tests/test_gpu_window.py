@@ -40,20 +40,24 @@ def _sub_layer(cache, cfg, b):
         if t is None:
             setattr(sub, name, None)
             continue
-        per = rows * (cfg.head_dim * bits // 8 if grp is None else 2 * (cfg.head_dim // grp))
+        pairs = 2 if cfg.kv_format == kvq.KVQ_FMT_ASYM else 1     # (scale, zero-point)
+        per = rows * (cfg.head_dim * bits // 8 if grp is None else 2 * pairs * (cfg.head_dim // grp))
         per //= t.element_size()
         setattr(sub, name, t[b * per:(b + 1) * per])
     return sub
 
 
-@pytest.mark.parametrize("fmt", [(4, 8, 32, 128), (8, 8, 128, 128), (8, 4, 128, 32)])
+@pytest.mark.parametrize("fmt", [(4, 8, 32, 128), (8, 8, 128, 128), (8, 4, 128, 32),
+                                 (8, 8, 128, 32, kvq.KVQ_FMT_E4M3), (8, 8, 32, 128, kvq.KVQ_FMT_ASYM)])
 def test_window_cache_decode_step_matches_oracle(cuda_device, fmt):
     lens = [100, 1600, 1700, 4000]
     B, Hkv, G, dh = len(lens), 2, 4, 128
     cap = N_ANCHOR + WINDOW
-    kb, vb, kg, vg = fmt
+    kb, vb, kg, vg = fmt[:4]
+    kf = fmt[4] if len(fmt) > 4 else kvq.KVQ_FMT_INT
     cfg = Config(batch=B, capacity=cap, n_q_heads=Hkv * G, n_kv_heads=Hkv, head_dim=dh,
-                 k_bits=kb, v_bits=vb, k_group=kg, v_group=vg, window=WINDOW, n_anchor=N_ANCHOR)
+                 k_bits=kb, v_bits=vb, k_group=kg, v_group=vg, window=WINDOW, n_anchor=N_ANCHOR,
+                 kv_format=kf)
     g = torch.Generator().manual_seed(5 + kb + vb)
     Lmax = max(lens)
     k = torch.randn(B, Lmax, Hkv, dh, generator=g).half()
