@@ -451,6 +451,34 @@ def run_hmode(args, world, device):
                        "frac_of_sustained": round(tf / sustained, 4)}
     res["steps_per_s"] = round(world * 1e3 / res["step_ms"], 2)
 
+    # the reconstruction fused into the attention (tcgen05 tiles of K_j | V_j attended
+    # in the GEMM epilogue, nothing written back): tensor-bound like the GEMM
+    fz_scratch = torch.zeros(kvq.kvq_h_fused_scratch_bytes(cfg, S) // 4, device=device)
+
+    def fused():
+        kvq.kvq_h_decode_fused(cfg, cache, W, q, d_len, S, out, fz_scratch)
+
+    for _ in range(max(args.warmup, 3)):
+        fused()
+    torch.cuda.synchronize()
+    fa = torch.cuda.Event(enable_timing=True)
+    fb = torch.cuda.Event(enable_timing=True)
+    nf = max(3, min(args.steps, 100))
+    fa.record()
+    for _ in range(nf):
+        fused()
+    fb.record()
+    fb.synchronize()
+    fms = reduce_max(fa.elapsed_time(fb) / nf, world, device)
+    assert kvq.kvq_workspace_status(fz_scratch) == 0
+    ftf = flops / (fms * 1e-3) / 1e12
+    res["fused"] = {"kernels": "dequant_h, hgemm_kernel<fused>, fused_merge", "ms": round(fms, 5),
+                    "steps_per_s": round(world * 1e3 / fms, 1),
+                    "roofline": {"bound": "tensor", "achieved": round(ftf, 1), "peak": burst,
+                                 "peak_kind": kind + " burst", "unit": "TFLOP/s",
+                                 "frac": round(ftf / burst, 4)},
+                    "speedup_vs_reconstruction_step": round(res["step_ms"] / fms, 2)}
+
     # the same attention by query absorption (W_k^T q against the h codes, W_v on
     # sum p h^): HBM-bound on the h codes + scales and W; the inputs (25 MB) fit in
     # L2, so every timed call follows a 256 MB L2 flush and is bracketed alone

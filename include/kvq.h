@@ -317,6 +317,30 @@ KVQ_API int kvq_h_reconstruct(const kvq_config *cfg, const kvq_layer *layer, con
                               int32_t out_capacity, void *operand, uint64_t operand_bytes,
                               kvq_stream_t stream);
 
+/* h-mode decode attention with the reconstruction fused into it ([TL]
+ * "運作原理": K = W_k h^, V = W_v h^ rebuilt at every call; here never written to
+ * memory): the tcgen05 GEMM computes, per 128-token tile and KV head j, the tile's
+ * K_j and V_j (bf16(h^) operands, fp32 accumulators in tensor memory), and the
+ * epilogue warps attend over them (per 32 tokens: s_t = softmax_scale * q . K_t,
+ * max, sum, o = sum 2^(s - max) V_t); a merge launch combines the partials:
+ *   out = sum_t p_t V_t,  p = softmax(s) over t < d_len[b].
+ * Same arithmetic as kvq_decode_attn's h-mode path except that K and V stay fp32
+ * (no fp16 rounding).  Dh = 128, Hq / Hkv <= 8, h_bits 4, 8 or 16.
+ *   w_kv, q, q_dtype, d_len, max_len_host, softmax_scale, out, out_dtype: as
+ *            kvq_decode_attn
+ *   scratch  device, at least kvq_h_fused_scratch_bytes(cfg, max_len_host) bytes:
+ *            a 256-byte header whose first int32 is a status word like a
+ *            workspace's (zero it once before the first call; read and clear it
+ *            with kvq_workspace_status), then the bf16(h^) operand and the partials
+ * Three launches (operand pre-pass, fused GEMM + attention, merge).  Errors as
+ * kvq_h_decode_absorbed. */
+KVQ_API int kvq_h_fused_scratch_bytes(const kvq_config *cfg, int32_t max_len, uint64_t *bytes);
+KVQ_API int kvq_h_decode_fused(const kvq_config *cfg, const kvq_layer *layer, const void *w_kv,
+                               const void *q, int32_t q_dtype, const int32_t *d_len,
+                               int32_t max_len_host, float softmax_scale, void *out,
+                               int32_t out_dtype, void *scratch, uint64_t scratch_bytes,
+                               kvq_stream_t stream);
+
 /* h-mode decode attention by query absorption: the attention of
  * kvq_decode_attn (h-mode) regrouped by the linearity of the reconstruction
  * ([TL] "運作原理": K = W_k h^, V = W_v h^), without rebuilding K and V:

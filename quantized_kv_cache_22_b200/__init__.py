@@ -26,7 +26,8 @@ EXPORTED = ("kvq_cache_bytes", "kvq_layer_buffer_bytes", "kvq_append", "kvq_work
             "kvq_h_scratch_bytes", "kvq_decode_attn", "kvq_decode_partials", "kvq_merge_partials",
             "kvq_h_reconstruct", "kvq_workspace_status", "kvq_status_string",
             "kvq_last_error_detail", "kvq_decode_attn_noalloc", "kvq_h_operand_bytes",
-            "kvq_append_decode_attn", "kvq_h_absorbed_scratch_bytes", "kvq_h_decode_absorbed")
+            "kvq_append_decode_attn", "kvq_h_absorbed_scratch_bytes", "kvq_h_decode_absorbed",
+            "kvq_h_fused_scratch_bytes", "kvq_h_decode_fused")
 
 
 class KvqError(RuntimeError):
@@ -73,6 +74,8 @@ def _load():
         "kvq_h_reconstruct": [cfgp, layp, P, i32, P, P, i32, P, u64, P],
         "kvq_workspace_status": [P, ctypes.POINTER(i32), P],
         "kvq_h_absorbed_scratch_bytes": [cfgp, i32, pu64],
+        "kvq_h_fused_scratch_bytes": [cfgp, i32, pu64],
+        "kvq_h_decode_fused": [cfgp, layp, P, P, i32, P, i32, ctypes.c_float, P, i32, P, u64, P],
         "kvq_h_decode_absorbed": [cfgp, layp, P, P, i32, P, i32, ctypes.c_float, P, i32, P, u64, P],
     }
     for name, args in sig.items():
@@ -334,8 +337,31 @@ def kvq_h_decode_absorbed(cfg: Config, layer: LayerCache, w_kv: torch.Tensor, q:
                                       _stream(stream)))
 
 
-def kvq_workspace_status(ws: Workspace, stream=None) -> int:
+def kvq_h_fused_scratch_bytes(cfg: Config, max_len: int) -> int:
+    v = ctypes.c_uint64()
+    _check("kvq_h_fused_scratch_bytes",
+           _lib.kvq_h_fused_scratch_bytes(cfg._ref(), int(max_len), ctypes.byref(v)))
+    return v.value
+
+
+def kvq_h_decode_fused(cfg: Config, layer: LayerCache, w_kv: torch.Tensor, q: torch.Tensor,
+                       d_len: torch.Tensor, max_len: int, out: torch.Tensor, scratch: torch.Tensor,
+                       softmax_scale: float = 0.0, stream=None):
+    """h-mode decode attention with the K/V reconstruction fused into the GEMM epilogue.
+    `scratch` starts with a status word (zero it once; read it with kvq_workspace_status)."""
+    _check("kvq_h_decode_fused",
+           _lib.kvq_h_decode_fused(cfg._ref(), layer._ref(), _ptr(w_kv), _ptr(q),
+                                   _dtype_code(q), _ptr(d_len), int(max_len),
+                                   float(softmax_scale), _ptr(out), _dtype_code(out),
+                                   _ptr(scratch), scratch.numel() * scratch.element_size(),
+                                   _stream(stream)))
+
+
+def kvq_workspace_status(ws, stream=None) -> int:
+    """Read and clear the status word of a Workspace (or of a scratch tensor that starts
+    with one, as the fused h-mode path's)."""
     st = ctypes.c_int32()
-    _check("kvq_workspace_status", _lib.kvq_workspace_status(_ptr(ws.buf), ctypes.byref(st),
+    buf = ws.buf if isinstance(ws, Workspace) else ws
+    _check("kvq_workspace_status", _lib.kvq_workspace_status(_ptr(buf), ctypes.byref(st),
                                                              _stream(stream)))
     return st.value

@@ -751,6 +751,93 @@ int kvq_h_reconstruct(const kvq_config *cfg, const kvq_layer *layer, const void 
                               operand_bytes, nullptr, stream);
 }
 
+// ------------------------------------------------------------ fused reconstruction
+static int fused_shape_check(const kvq_config *cfg)
+{
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (cfg->mode != KVQ_MODE_H) return KVQ_ERR_INVALID_ARG;
+    if (cfg->n_kv_heads * cfg->head_dim != cfg->d_model) return KVQ_ERR_INVALID_ARG;
+    if (cfg->head_dim != 128 || cfg->n_q_heads % cfg->n_kv_heads != 0 ||
+        cfg->n_q_heads / cfg->n_kv_heads > 8)
+        return KVQ_ERR_UNSUPPORTED;
+    return KVQ_OK;
+}
+
+static uint64_t fused_part_bytes(const kvq_config *cfg, int max_len)
+{
+    const uint64_t m_tiles = (uint64_t)((max_len + kHTileTokens - 1) / kHTileTokens);
+    return (uint64_t)cfg->batch * cfg->n_q_heads * m_tiles * 4 * (cfg->head_dim + 2) * 4;
+}
+
+int kvq_h_fused_scratch_bytes(const kvq_config *cfg, int32_t max_len, uint64_t *bytes)
+{
+    int rc = fused_shape_check(cfg);
+    if (rc) return rc;
+    if (!bytes || max_len < 0) return KVQ_ERR_INVALID_ARG;
+    if (max_len > cfg->capacity) return KVQ_ERR_CAPACITY;
+    *bytes = 256 + h_operand_need(cfg, max_len) + fused_part_bytes(cfg, max_len);
+    return KVQ_OK;
+}
+
+int kvq_h_decode_fused(const kvq_config *cfg, const kvq_layer *layer, const void *w_kv,
+                       const void *q, int32_t q_dtype, const int32_t *d_len, int32_t max_len_host,
+                       float softmax_scale, void *out, int32_t out_dtype, void *scratch,
+                       uint64_t scratch_bytes, kvq_stream_t stream)
+{
+    int rc = fused_shape_check(cfg);
+    if (rc) return rc;
+    if (!layer || !layer->k_codes || (cfg->h_bits != 16 && !layer->k_scales) || !w_kv || !q ||
+        !d_len || !out || !scratch)
+        return KVQ_ERR_INVALID_ARG;
+    if (q_dtype != KVQ_F16 && q_dtype != KVQ_F32 && q_dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
+    if (out_dtype != KVQ_F16 && out_dtype != KVQ_F32) return KVQ_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale) || max_len_host < 0) return KVQ_ERR_INVALID_ARG;
+    if (max_len_host > cfg->capacity) return KVQ_ERR_CAPACITY;
+    if (!aligned16(layer->k_codes) || (layer->k_scales && !aligned16(layer->k_scales)) ||
+        !aligned16(w_kv) || !aligned16(q) || !aligned16(out) || !aligned16(scratch))
+        return KVQ_ERR_ALIGN;
+    uint64_t need = 0;
+    rc = kvq_h_fused_scratch_bytes(cfg, max_len_host, &need);
+    if (rc) return rc;
+    if (scratch_bytes < need) return KVQ_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (max_len_host == 0) {
+        // nothing cached: every output is zero
+        const size_t ob = (size_t)cfg->batch * cfg->n_q_heads * cfg->head_dim * (out_dtype == KVQ_F32 ? 4 : 2);
+        cudaError_t e = cudaMemsetAsync(out, 0, ob, st);
+        return e == cudaSuccess ? KVQ_OK : fail("zero output", e);
+    }
+    uint8_t *base = static_cast<uint8_t *>(scratch);
+    HGemmParams p{};
+    p.h_codes = static_cast<const uint8_t *>(layer->k_codes);
+    p.h_scales = static_cast<const __half *>(layer->k_scales);
+    p.w = w_kv;
+    p.batch = cfg->batch;
+    p.cap = cfg->capacity;
+    p.d_model = cfg->d_model;
+    p.h_bits = cfg->h_bits;
+    p.h_groups = cfg->h_bits == 16 ? 1 : cfg->h_groups;
+    p.n_kv_heads = cfg->n_kv_heads;
+    p.head_dim = cfg->head_dim;
+    p.len = max_len_host;
+    p.out_cap = 0;
+    p.operand = base + 256;
+    p.status = reinterpret_cast<int *>(base);
+    p.q = q;
+    p.d_len = d_len;
+    p.part = reinterpret_cast<float *>(base + 256 + h_operand_need(cfg, max_len_host));
+    p.out = out;
+    p.q_dtype = q_dtype;
+    p.n_q_heads = cfg->n_q_heads;
+    p.out_f32 = out_dtype == KVQ_F32;
+    const float scale = softmax_scale != 0.f ? softmax_scale : 1.f / std::sqrt((float)cfg->head_dim);
+    p.tau_log2e = scale * 1.4426950408889634f;
+    cudaError_t e = launch_h_reconstruct(p, st);
+    if (e == cudaErrorNotSupported) return KVQ_ERR_UNSUPPORTED;
+    return e == cudaSuccess ? KVQ_OK : fail("fused reconstruction launch", e);
+}
+
 // ------------------------------------------------------------ query absorption
 static int absorbed_shape_check(const kvq_config *cfg)
 {

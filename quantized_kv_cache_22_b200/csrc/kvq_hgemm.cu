@@ -49,6 +49,12 @@ struct GemmArgs {
     int32_t d_model, n_kv_heads, head_dim, len, out_cap, m_tiles, n_tiles, batch;
     uint32_t stage_bytes, stages;
     uint64_t timeout_ns;
+    // fused attention (N tile = K_h | V_h of one KV head h)
+    const void *q;            // [B][Hq][Dh]
+    const int32_t *d_len;     // [B]
+    float *part;              // [B][Hq][m_tiles * 4][Dh + 2]: o, m, l per (tile, warp)
+    int32_t q_dtype, n_q_heads;
+    float tau_log2e;
 };
 
 struct DequantArgs {
@@ -189,6 +195,96 @@ __global__ void __launch_bounds__(256) dequant_h_kernel(const DequantArgs a)
     }
 }
 
+// Fused path, one epilogue warp over its 32 rows (tokens t0 + 32q + lane) of the
+// tile [K_h | V_h] in TMEM (taddr: the warp's lane quarter, column 0).  For each query
+// head of KV head h: s_t = tau log2(e) q . K_t (rows past the length masked), the
+// warp's m = max s, l = sum 2^(s - m) and o = sum_t 2^(s_t - m) V_t, written as one
+// partial (the column sums of o by a transposing butterfly: 31 shuffles per 32 columns).
+__device__ __forceinline__ void fused_epilogue(const GemmArgs &g, uint32_t taddr, int b, int t0,
+                                               int h, int q, int lane, float *qs)
+{
+    constexpr unsigned FULL = 0xffffffffu;
+    const int G = g.n_q_heads / g.n_kv_heads;
+    for (int k = lane; k < G * 128; k += 32) {
+        const int64_t qi = ((int64_t)b * g.n_q_heads + h * G + (k >> 7)) * 128 + (k & 127);
+        float v;
+        if (g.q_dtype == KVQ_F32)
+            v = static_cast<const float *>(g.q)[qi];
+        else if (g.q_dtype == KVQ_F16)
+            v = __half2float(static_cast<const __half *>(g.q)[qi]);
+        else
+            v = __bfloat162float(static_cast<const __nv_bfloat16 *>(g.q)[qi]);
+        qs[k] = v;
+    }
+    __syncwarp();
+    const int len_b = min(max(g.d_len[b], 0), g.len);
+    const bool valid = t0 + 32 * q + lane < len_b;
+    float sc[8];
+#pragma unroll
+    for (int gg = 0; gg < 8; gg++) sc[gg] = 0.f;
+#pragma unroll 1
+    for (int c0 = 0; c0 < 128; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(taddr + (uint32_t)c0, v);
+#pragma unroll
+        for (int gg = 0; gg < 8; gg++) {
+            if (gg >= G) break;
+            float a = sc[gg];
+#pragma unroll
+            for (int j = 0; j < 32; j++) a = fmaf(__uint_as_float(v[j]), qs[gg * 128 + c0 + j], a);
+            sc[gg] = a;
+        }
+    }
+    float mw[8], lw[8], pw[8];
+#pragma unroll
+    for (int gg = 0; gg < 8; gg++) {
+        if (gg >= G) break;
+        const float sv = valid ? sc[gg] * g.tau_log2e : -INFINITY;
+        float m = sv;
+        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, off));
+        const float pv = (m == -INFINITY || !valid) ? 0.f : exp2f(sv - m);
+        float l = pv;
+        for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(FULL, l, off);
+        mw[gg] = m;
+        lw[gg] = l;
+        pw[gg] = pv;
+    }
+    const int P = g.m_tiles * 4;
+    const int slot = (t0 / BM) * 4 + q;
+#pragma unroll 1
+    for (int c0 = 0; c0 < 128; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(taddr + 128u + (uint32_t)c0, v);
+#pragma unroll
+        for (int gg = 0; gg < 8; gg++) {
+            if (gg >= G) break;
+            float x[32];
+#pragma unroll
+            // rows past the length may hold anything (stale scales): zero, not 0 * v
+            for (int j = 0; j < 32; j++) x[j] = valid ? pw[gg] * __uint_as_float(v[j]) : 0.f;
+#pragma unroll
+            for (int w = 16; w >= 1; w >>= 1) {
+                const bool upper = (lane & w) != 0;
+#pragma unroll
+                for (int i = 0; i < w; i++) {
+                    const float send = upper ? x[i] : x[i + w];
+                    const float keep = upper ? x[i + w] : x[i];
+                    x[i] = keep + __shfl_xor_sync(FULL, send, w);
+                }
+            }
+            float *dst = g.part + (((int64_t)b * g.n_q_heads + h * G + gg) * P + slot) * 130;
+            dst[c0 + lane] = x[0];
+            if (c0 == 0 && lane == 0) {
+                dst[128] = mw[gg];
+                dst[129] = lw[gg];
+            }
+        }
+    }
+}
+
+// FUSED: the N tile of KV head h is [K_h | V_h] (W rows h*Dh.. and Hkv*Dh + h*Dh.., two
+// 128-row boxes, Dh = 128) and the epilogue attends over the tile instead of storing it.
+template <bool FUSED>
 __global__ void __launch_bounds__(NTHREADS, 1)
     hgemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_a,
                  const GemmArgs g)
@@ -205,6 +301,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 4);
     int *abort_flag_p = reinterpret_cast<int *>(tmem_slot + 1);
     volatile int *abort_flag = abort_flag_p;
+    // fused: per epilogue warp, the G <= 8 queries of the tile's KV head (fp32)
+    float *qsm = reinterpret_cast<float *>(tmem_slot + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int k_stages = g.d_model / BK;
@@ -264,7 +362,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     uint8_t *st = smem + s * g.stage_bytes;
                     mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES);
                     tma_load_3d(st, &tm_a, &full[s], k * BK, t0, b);
-                    tma_load_2d(st + A_BYTES, &tm_w, &full[s], k * BK, n0);
+                    if constexpr (FUSED) {
+                        // n0 / BN = KV head h: K_h rows, then V_h rows (128-row boxes)
+                        const int h = n0 / BN;
+                        tma_load_2d(st + A_BYTES, &tm_w, &full[s], k * BK, h * g.head_dim);
+                        tma_load_2d(st + A_BYTES + B_BYTES / 2, &tm_w, &full[s], k * BK,
+                                    (g.n_kv_heads + h) * g.head_dim);
+                    } else {
+                        tma_load_2d(st + A_BYTES, &tm_w, &full[s], k * BK, n0);
+                    }
                     ++issued;
                     if (++s == S) {
                         s = 0;
@@ -351,6 +457,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             int n0, b, t0;
             tile_coords(tile, n0, b, t0);
             const int tt = t0 + row;
+            if constexpr (FUSED) {
+                fused_epilogue(g, tmem + (uint32_t)buf * TMEM_COLS + ((uint32_t)(32 * q) << 16), b, t0,
+                               n0 / BN, q, lane, qsm + (size_t)warp * 8 * 128);
+            } else {
 #pragma unroll 1
             for (int c0 = 0; c0 < BN; c0 += 32) {
                 uint32_t v[32];
@@ -372,6 +482,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                 }
             }
+            }
             // all TMEM reads of this buffer are done: hand it back to the MMA warp
             tc_fence_before();
             __syncwarp();
@@ -384,6 +495,39 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     __syncthreads();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem, 2 * TMEM_COLS);
+}
+
+// Merge of the fused path's partials: one warp per (sequence, query head) over its
+// m_tiles * 4 warp partials, out = sum_k o_k 2^(m_k - M) / sum_k l_k 2^(m_k - M).
+__global__ void __launch_bounds__(128) fused_merge_kernel(const float *part, int P, int rows,
+                                                          void *out, int out_f32)
+{
+    const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const float *pr = part + (int64_t)row * P * 130;
+    float M = -INFINITY;
+    for (int k = 0; k < P; k++) M = fmaxf(M, pr[(int64_t)k * 130 + 128]);
+    float L = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
+    if (M != -INFINITY) {
+        for (int k = 0; k < P; k++) {
+            const float m = pr[(int64_t)k * 130 + 128];
+            if (m == -INFINITY) continue;
+            const float e = exp2f(m - M);
+            L = fmaf(e, pr[(int64_t)k * 130 + 129], L);
+#pragma unroll
+            for (int i = 0; i < 4; i++) o[i] = fmaf(e, pr[(int64_t)k * 130 + lane + 32 * i], o[i]);
+        }
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const int64_t idx = (int64_t)row * 128 + lane + 32 * i;
+        if (out_f32)
+            static_cast<float *>(out)[idx] = o[i] * inv;
+        else
+            static_cast<__half *>(out)[idx] = __float2half_rn(o[i] * inv);
+    }
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -410,8 +554,12 @@ EncodeTiledFn encode_fn()
 
 cudaError_t launch_h_reconstruct(const HGemmParams &p, cudaStream_t stream)
 {
+    const bool fused = p.part != nullptr;
     const int N = 2 * p.n_kv_heads * p.head_dim;
     if (p.head_dim % 32 != 0 || N % BN != 0 || p.d_model % BK != 0) return cudaErrorNotSupported;
+    if (fused && (p.head_dim != BN / 2 || p.n_q_heads % p.n_kv_heads != 0 ||
+                  p.n_q_heads / p.n_kv_heads > 8))
+        return cudaErrorNotSupported;
     if (p.h_bits != 16 && (p.d_model / p.h_groups) % 8 != 0) return cudaErrorNotSupported;
     EncodeTiledFn fn = encode_fn();
     if (!fn) return cudaErrorNotSupported;
@@ -440,7 +588,8 @@ cudaError_t launch_h_reconstruct(const HGemmParams &p, cudaStream_t stream)
     {
         cuuint64_t dims[2] = {(cuuint64_t)p.d_model, (cuuint64_t)N};
         cuuint64_t strides[1] = {(cuuint64_t)p.d_model * 2};
-        cuuint32_t box[2] = {BK, BN}, es[2] = {1, 1};
+        // fused: two 128-row boxes per stage (K_h, then V_h)
+        cuuint32_t box[2] = {BK, fused ? (cuuint32_t)(BN / 2) : (cuuint32_t)BN}, es[2] = {1, 1};
         if (fn(&tm_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(p.w), dims, strides,
                box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -468,10 +617,19 @@ cudaError_t launch_h_reconstruct(const HGemmParams &p, cudaStream_t stream)
     g.stage_bytes = A_BYTES + B_BYTES;
     g.stages = 4;
     g.timeout_ns = 1000000000ull;
-    const size_t smem = (size_t)g.stages * g.stage_bytes + 1024 + 8 * (2 * g.stages + 4) + 16;
-    e = cudaFuncSetAttribute(hgemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    g.q = p.q;
+    g.d_len = p.d_len;
+    g.part = p.part;
+    g.q_dtype = p.q_dtype;
+    g.n_q_heads = p.n_q_heads;
+    g.tau_log2e = p.tau_log2e;
+    // + fused: 6 warps x 8 queries x 128 fp32 of query staging
+    const size_t smem = (size_t)g.stages * g.stage_bytes + 1024 + 8 * (2 * g.stages + 4) + 16 +
+                        (fused ? (size_t)NTHREADS / 32 * 8 * 128 * 4 : 0);
+    void *kfn = fused ? reinterpret_cast<void *>(&hgemm_kernel<true>) : reinterpret_cast<void *>(&hgemm_kernel<false>);
+    e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    g.n_tiles = N / BN;
+    g.n_tiles = fused ? p.n_kv_heads : N / BN;
     g.batch = p.batch;
     // persistent: one CTA per SM (the 197 KB ring allows no more), tiles round-robin
     int dev = 0, sms = 148;
@@ -480,8 +638,11 @@ cudaError_t launch_h_reconstruct(const HGemmParams &p, cudaStream_t stream)
     const int tiles = g.n_tiles * m_tiles * p.batch;
     const dim3 grid((unsigned)(tiles < sms ? tiles : sms), 1);
     void *args[] = {&tm_w, &tm_a, &g};
-    return cudaLaunchKernel(reinterpret_cast<void *>(&hgemm_kernel), grid, dim3(NTHREADS), args,
-                            smem, stream);
+    e = cudaLaunchKernel(kfn, grid, dim3(NTHREADS), args, smem, stream);
+    if (e != cudaSuccess || !fused) return e;
+    const int rows = p.batch * p.n_q_heads;
+    fused_merge_kernel<<<(rows + 3) / 4, 128, 0, stream>>>(p.part, m_tiles * 4, rows, p.out, p.out_f32);
+    return cudaGetLastError();
 }
 
 }  // namespace kvq

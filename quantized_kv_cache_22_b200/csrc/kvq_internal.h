@@ -169,6 +169,14 @@ struct HGemmParams {
     void *operand;            // bf16 [B][round_up(len, 128)][D] scratch for h^
     int *status;              // set to KVQ_ERR_TIMEOUT if a wait gives up (may be null)
     int32_t batch, cap, d_model, h_bits, h_groups, n_kv_heads, head_dim, len, out_cap;
+    // fused reconstruction + attention (part != null): no K/V written; the GEMM epilogue
+    // attends over each tile and fused_merge_kernel writes `out`
+    const void *q;            // [B][Hq][Dh]
+    const int32_t *d_len;     // [B]
+    float *part;              // [B][Hq][m_tiles * 4][Dh + 2]
+    void *out;                // [B][Hq][Dh]
+    int32_t q_dtype, n_q_heads, out_f32;
+    float tau_log2e;
 };
 cudaError_t launch_h_reconstruct(const HGemmParams &p, cudaStream_t stream);
 constexpr int kHTileTokens = 128;   // token rows of one reconstruction tile

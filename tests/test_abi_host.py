@@ -248,3 +248,14 @@ def test_absorbed_scratch_bytes_and_validation():
     with pytest.raises(kvq.KvqError) as e:
         kvq.kvq_h_absorbed_scratch_bytes(kv, 64)
     assert e.value.status == -1
+
+
+def test_fused_scratch_bytes_and_validation():
+    cfg = Config(batch=8, capacity=1024, mode=kvq.KVQ_MODE_H, d_model=2048, h_bits=4, h_groups=16,
+                 n_q_heads=16, n_kv_heads=16, head_dim=128)
+    # header 256 + bf16 operand B*round_up(len,128)*D*2 + partials B*Hq*m_tiles*4*(Dh+2)*4
+    assert kvq.kvq_h_fused_scratch_bytes(cfg, 1000) == 256 + 8 * 1024 * 2048 * 2 + 8 * 16 * 8 * 4 * 130 * 4
+    for over, st in (({"n_q_heads": 256}, -2), ({"n_kv_heads": 8}, -1)):
+        with pytest.raises(kvq.KvqError) as e:
+            kvq.kvq_h_fused_scratch_bytes(Config(**{**cfg.__dict__, **over}), 1024)
+        assert e.value.status == st, over
