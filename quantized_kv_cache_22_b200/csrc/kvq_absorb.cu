@@ -172,8 +172,6 @@ __global__ void __launch_bounds__(128) absorb_q_kernel(AbsorbParams p)
     // amax over the scale group's threads (consecutive lanes of a half-warp)
     for (int off = 1; off < p.group / 8; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, off));
     grid_launch_dependents();
-    if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
-        for (int k = tid; k < p.B * p.ng; k += blockDim.x) p.cnt[k] = 0;
     if (q >= nqc) return;
     const float inv = amax > 0.f ? 127.f / amax : 0.f;
     int hi[8], lo[8];
@@ -544,31 +542,6 @@ __global__ void __launch_bounds__(128) absorb_pv_kernel(AbsorbParams p)
             }
         }
     }
-    // The last CTA of (sequence, group) to finish sums the splits' partials, in split
-    // order (deterministic), into split 0's slot.
-    const int ns = (len + p.split - 1) / p.split;
-    if (ns == 1) return;
-    __shared__ int last;
-    __threadfence();                               // release this CTA's partial
-    __syncthreads();
-    if (tid == 0) last = atomicAdd(&p.cnt[b * p.ng + g], 1) == ns - 1;
-    __syncthreads();
-    if (!last) return;
-    __threadfence();                               // acquire the other CTAs' partials
-    const int64_t sstep = (int64_t)p.B * p.Hq * p.D / 4;     // one split, in float4
-    float4 *o0 = reinterpret_cast<float4 *>(p.obp + (int64_t)b * p.Hq * p.D + g * GS);
-#pragma unroll 4
-    for (int k = tid; k < p.Hq * (GS / 4); k += blockDim.x) {
-        const int64_t idx = (int64_t)(k / (GS / 4)) * (p.D / 4) + k % (GS / 4);
-        float4 v = __ldcg(o0 + idx);
-#pragma unroll 4
-        for (int sp = 1; sp < ns; sp++) {
-            const float4 x = __ldcg(o0 + sp * sstep + idx);
-            v.x += x.x; v.y += x.y; v.z += x.z; v.w += x.w;
-        }
-        o0[idx] = v;
-    }
-    if (tid == 0) p.cnt[b * p.ng + g] = 0;         // ready for the next call
 }
 
 // ---------------------------------------------------------------- W_v . ob
@@ -607,11 +580,18 @@ __global__ void __launch_bounds__(256) absorb_out_kernel(AbsorbParams p)
         for (int c = 0; c < nqc; c++) {
             const int qi = q0 + c, b = qi / G, h = j * G + qi % G;
             const int ns = qns[c];
-            // the splits were summed into split 0 by the p . h^ kernel; no split: zeros
             const float4 *src = reinterpret_cast<const float4 *>(p.obp + ((int64_t)b * p.Hq + h) * p.D);
-            for (int d4 = threadIdx.x; d4 < D4; d4 += blockDim.x)
-                reinterpret_cast<float4 *>(obs)[(size_t)c * D4 + d4] =
-                    ns > 0 ? __ldcg(src + d4) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const int64_t sstep = (int64_t)p.B * p.Hq * p.D / 4;   // one split, in float4
+#pragma unroll 2
+            for (int d4 = threadIdx.x; d4 < D4; d4 += blockDim.x) {
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+                for (int sidx = 0; sidx < ns; sidx++) {
+                    const float4 x = __ldg(src + sidx * sstep + d4);
+                    v.x += x.x; v.y += x.y; v.z += x.z; v.w += x.w;
+                }
+                reinterpret_cast<float4 *>(obs)[(size_t)c * D4 + d4] = v;
+            }
         }
         cp_async_wait_all();
         __syncthreads();
@@ -759,21 +739,21 @@ int absorb_split(int max_len)
     return max(256, (per + 255) / 256 * 256);
 }
 
-uint64_t absorb_scratch_layout(int B, int Hq, int D, int ng, int bits, int max_len, uint64_t off[7])
+uint64_t absorb_scratch_layout(int B, int Hq, int D, int ng, int bits, int max_len, uint64_t off[6])
 {
     const int NT = absorb_nt(Hq);
     const uint64_t capP = (uint64_t)((max_len + 63) / 64 * 64);
     const uint64_t ntile = capP / absorb_t2(D, bits, Hq, ng);   // tiles up to capP (T2 divides 64)
     const uint64_t ns = (uint64_t)((max_len + absorb_split(max_len) - 1) / absorb_split(max_len));
-    const uint64_t sz[6] = {(uint64_t)B * (D / 32) * NT * 32 * 16, (uint64_t)B * ng * NT * 8 * 4,
+    const uint64_t sz[5] = {(uint64_t)B * (D / 32) * NT * 32 * 16, (uint64_t)B * ng * NT * 8 * 4,
                             (uint64_t)B * Hq * capP * 4, (uint64_t)B * Hq * (ntile ? ntile : 1) * 8,
-                            (ns ? ns : 1) * B * Hq * D * 4, (uint64_t)B * ng * 4};
+                            (ns ? ns : 1) * B * Hq * D * 4};
     uint64_t o = 0;
-    for (int i = 0; i < 6; i++) {
+    for (int i = 0; i < 5; i++) {
         off[i] = o;
         o += (sz[i] + 255) / 256 * 256;
     }
-    off[6] = o;
+    off[5] = o;
     return o;
 }
 

@@ -859,7 +859,7 @@ int kvq_h_absorbed_scratch_bytes(const kvq_config *cfg, int32_t max_len, uint64_
     if (rc) return rc;
     if (!bytes || max_len < 0) return KVQ_ERR_INVALID_ARG;
     if (max_len > cfg->capacity) return KVQ_ERR_CAPACITY;
-    uint64_t off[7];
+    uint64_t off[6];
     *bytes = absorb_scratch_layout(cfg->batch, cfg->n_q_heads, cfg->d_model, cfg->h_groups,
                                    cfg->h_bits, max_len, off);
     return KVQ_OK;
@@ -881,7 +881,7 @@ int kvq_h_decode_absorbed(const kvq_config *cfg, const kvq_layer *layer, const v
     if (!aligned16(layer->k_codes) || !aligned16(layer->k_scales) || !aligned16(w_kv) ||
         !aligned16(q) || !aligned16(out) || !aligned16(scratch))
         return KVQ_ERR_ALIGN;
-    uint64_t off[7];
+    uint64_t off[6];
     const uint64_t need = absorb_scratch_layout(cfg->batch, cfg->n_q_heads, cfg->d_model,
                                                 cfg->h_groups, cfg->h_bits, max_len_host, off);
     if (scratch_bytes < need) return KVQ_ERR_WORKSPACE;
@@ -911,7 +911,6 @@ int kvq_h_decode_absorbed(const kvq_config *cfg, const kvq_layer *layer, const v
     p.p = reinterpret_cast<float *>(base + off[2]);
     p.stats = reinterpret_cast<float2 *>(base + off[3]);
     p.obp = reinterpret_cast<float *>(base + off[4]);
-    p.cnt = reinterpret_cast<int *>(base + off[5]);
     p.capP = (max_len_host + 63) / 64 * 64;
     p.NT = absorb_nt(p.Hq);
     p.T2 = absorb_t2(p.D, p.bits, p.Hq, p.ng);

@@ -108,17 +108,15 @@ struct AbsorbParams {
     float *qfac;                  // [B][ng][NT*8] score factor per (group, head)
     float *p;                     // [B][Hq][capP] scores (log2 units)
     float2 *stats;                // [B][Hq][ntile] (max, sum 2^(s - max)) per score tile
-    float *obp;                   // [splits][B][Hq][D] partial sum_t p_t h^_t (summed into split 0)
-    int *cnt;                     // [B][ng] arrivals of the splits of (sequence, group)
+    float *obp;                   // [splits][B][Hq][D] partial sum_t p_t h^_t
     int32_t capP, NT, T2, ntile, split;
 };
 int absorb_nt(int Hq);            // n-tiles of 8 query heads in the score MMA: 1, 2 or 4
 bool absorb_fits(int D, int bits, int Hq, int ng);   // shared memory suffices for the shape
 int absorb_t2(int D, int bits, int Hq, int ng);   // tokens per score tile
 int absorb_split(int max_len);    // tokens per split of the p . h^ kernel
-// scratch bytes; off[0..5] = qfrag, qfac, scores, stats, partial ob, split counters
-// (256-byte aligned)
-uint64_t absorb_scratch_layout(int B, int Hq, int D, int ng, int bits, int max_len, uint64_t off[7]);
+// scratch bytes; off[0..4] = qfrag, qfac, scores, stats, partial ob (256-byte aligned)
+uint64_t absorb_scratch_layout(int B, int Hq, int D, int ng, int bits, int max_len, uint64_t off[6]);
 cudaError_t launch_absorbed(const AbsorbParams &p, int max_len, cudaStream_t stream);
 
 struct DecodeLaunch {

@@ -233,7 +233,7 @@ def test_absorbed_scratch_bytes_and_validation():
     # q fragments B*(D/32)*NT*512 + factors B*ng*NT*8*4 + scores B*Hq*capP*4 + tile
     # statistics B*Hq*(capP/64)*8 + partial ob (4 splits of 256 tokens) 4*B*Hq*D*4
     want = (8 * 64 * 2 * 512 + 8 * 16 * 16 * 4 + 8 * 16 * 1024 * 4 + 8 * 16 * 16 * 8 +
-            4 * 8 * 16 * 2048 * 4 + 512)     # + split arrival counters B*ng*4, 256-aligned
+            4 * 8 * 16 * 2048 * 4)
     assert kvq.kvq_h_absorbed_scratch_bytes(cfg, 1024) == want
     assert kvq.kvq_h_absorbed_scratch_bytes(cfg, 1000) == want
     for over, st in (({"h_bits": 16, "h_groups": 0}, -2), ({"n_q_heads": 64}, -2),
