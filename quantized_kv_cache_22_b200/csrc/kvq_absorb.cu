@@ -600,6 +600,7 @@ __global__ void __launch_bounds__(256) absorb_out_kernel(AbsorbParams p)
         for (int r = 0; r < 2; r++)
 #pragma unroll
             for (int c = 0; c < 8; c++) acc[r][c] = 0.f;
+#pragma unroll 2
         for (int kk = 0; kk < p.D / 128; kk++) {
             const int d0 = 128 * kk + 4 * lane;
             float wf[2][4];
