@@ -362,7 +362,8 @@ KVQ_API int kvq_h_decode_fused(const kvq_config *cfg, const kvq_layer *layer, co
  *   scratch  device, at least kvq_h_absorbed_scratch_bytes(cfg, max_len_host)
  *            bytes (contents on entry do not matter; calls that overlap on
  *            the GPU need separate scratch)
- * Five kernel launches on `stream`.  Errors: INVALID_ARG (KV mode, null or
+ * Four kernel launches on `stream`, each a programmatic dependent of the
+ * previous one.  Errors: INVALID_ARG (KV mode, null or
  * bad arguments), UNSUPPORTED (shape), CAPACITY, ALIGN (16 bytes), WORKSPACE,
  * LAUNCH. */
 KVQ_API int kvq_h_absorbed_scratch_bytes(const kvq_config *cfg, int32_t max_len, uint64_t *bytes);
