@@ -150,6 +150,8 @@ __device__ __forceinline__ uint32_t bf2(float lo, float hi)
 // One block per (sequence, token) row, one thread per 8 elements (16 output bytes).
 __global__ void __launch_bounds__(256) dequant_h_kernel(const DequantArgs a)
 {
+    // the GEMM that follows may be scheduled now; it waits for this grid to finish
+    grid_launch_dependents();
     const int row = blockIdx.x;                      // b * len_pad + t
     const int b = row / a.len_pad, t = row % a.len_pad;
     const int nchunk = a.d_model / 8;
@@ -347,6 +349,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (lane == 0) {
             prefetch_tensormap(&tm_w);
             prefetch_tensormap(&tm_a);
+            grid_dependency_wait();          // the operand pre-pass has finished
             uint32_t s = 0, ph = 0;
             int issued = 0;      // stage uses issued so far
             bool stop = false;
@@ -491,6 +494,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
 
     // every role reaches this point; free TMEM after all tcgen05 work is done
+    grid_launch_dependents();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -502,6 +506,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 __global__ void __launch_bounds__(128) fused_merge_kernel(const float *part, int P, int rows,
                                                           void *out, int out_f32)
 {
+    grid_dependency_wait();                          // the GEMM's partials are complete
     const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
@@ -638,11 +643,29 @@ cudaError_t launch_h_reconstruct(const HGemmParams &p, cudaStream_t stream)
     const int tiles = g.n_tiles * m_tiles * p.batch;
     const dim3 grid((unsigned)(tiles < sms ? tiles : sms), 1);
     void *args[] = {&tm_w, &tm_a, &g};
-    e = cudaLaunchKernel(kfn, grid, dim3(NTHREADS), args, smem, stream);
+    // programmatic dependent launches: each kernel may be scheduled while the previous
+    // one drains and waits (griddepcontrol.wait) before touching its outputs
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = grid;
+    lc.blockDim = dim3(NTHREADS);
+    lc.dynamicSmemBytes = smem;
+    lc.stream = stream;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    e = cudaLaunchKernelExC(&lc, kfn, args);
     if (e != cudaSuccess || !fused) return e;
     const int rows = p.batch * p.n_q_heads;
-    fused_merge_kernel<<<(rows + 3) / 4, 128, 0, stream>>>(p.part, m_tiles * 4, rows, p.out, p.out_f32);
-    return cudaGetLastError();
+    const int P = m_tiles * 4;
+    cudaLaunchConfig_t lm = {};
+    lm.gridDim = dim3((rows + 3) / 4);
+    lm.blockDim = dim3(128);
+    lm.stream = stream;
+    lm.attrs = attr;
+    lm.numAttrs = 1;
+    return cudaLaunchKernelEx(&lm, fused_merge_kernel, (const float *)p.part, P, rows, p.out, (int)p.out_f32);
 }
 
 }  // namespace kvq
