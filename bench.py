@@ -303,18 +303,30 @@ def time_e2e(w, st, steps, warmup, world, device):
     h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v))
     d2h = h_out.numel() * h_out.element_size()
 
-    # each layer's output goes back on a copy stream while the next layers run (the
-    # copy stream waits on the layer's event, the compute stream never waits, so the
-    # programmatic launches between layers stay back to back)
+    # Inputs go up on a copy stream in growing chunks of layers (layer 0 alone, then
+    # 1-3, 4-11, 12-): the compute stream waits only at a chunk's first layer, by which
+    # time the chunk has long landed, so the programmatic launches between layers break
+    # three times per step.  Each layer's output goes back on the copy stream as soon
+    # as its kernel ends.  The step ends when its last output is on the host.
     copy = torch.cuda.Stream()
     done = [torch.cuda.Event() for _ in range(w.n_layers)]
+    bounds = [0] + [b for b in (1, 4, 12) if b < w.n_layers] + [w.n_layers]
+    chunks = list(zip(bounds[:-1], bounds[1:]))
+    landed = [torch.cuda.Event() for _ in chunks]
+    first = {a: i for i, (a, _) in enumerate(chunks)}
 
     def one():
         cur = torch.cuda.current_stream()
-        st["q"].copy_(h_q, non_blocking=True)
-        st["k_new"].copy_(h_k, non_blocking=True)
-        st["v_new"].copy_(h_v, non_blocking=True)
+        copy.wait_stream(cur)   # the previous step is done with the input buffers
+        with torch.cuda.stream(copy):
+            for i, (a, b) in enumerate(chunks):
+                st["q"][a:b].copy_(h_q[a:b], non_blocking=True)
+                st["k_new"][a:b].copy_(h_k[a:b], non_blocking=True)
+                st["v_new"][a:b].copy_(h_v[a:b], non_blocking=True)
+                landed[i].record(copy)
         for layer in range(w.n_layers):
+            if layer in first:
+                cur.wait_event(landed[first[layer]])
             kvq.kvq_append_decode_attn(cfg, st["caches"][layer], st["k_new"][layer],
                                        st["v_new"][layer], st["q"][layer], st["d_len"], L,
                                        st["out"][layer], st["ws"])
