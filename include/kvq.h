@@ -378,6 +378,16 @@ KVQ_API int kvq_h_decode_absorbed(const kvq_config *cfg, const kvq_layer *layer,
  * (its outputs are then invalid).  Synchronises `stream`. */
 KVQ_API int kvq_workspace_status(void *workspace, int32_t *status, kvq_stream_t stream);
 
+/* Self-test of failure detection.  Every wait inside the library's kernels is
+ * bounded: after its limit it gives up, the kernel stores KVQ_ERR_TIMEOUT in the
+ * workspace status word, drains and returns, and the context stays usable.  This
+ * call runs that wait on a barrier that nothing completes, for timeout_ns
+ * (1 ns .. 2 s), so that the give-up path can be checked on a GPU without a fault
+ * or a hang: afterwards kvq_workspace_status(workspace) reports KVQ_ERR_TIMEOUT.
+ * Only the first 4 bytes of `workspace` (16-byte aligned device memory) are used.
+ * Errors: INVALID_ARG, ALIGN, LAUNCH. */
+KVQ_API int kvq_selftest_bounded_wait(void *workspace, uint64_t timeout_ns, kvq_stream_t stream);
+
 /* Bytes of the device array behind kvq_decode_attn_noalloc (8 MiB). */
 #define KVQ_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
 

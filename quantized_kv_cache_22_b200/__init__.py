@@ -27,7 +27,7 @@ EXPORTED = ("kvq_cache_bytes", "kvq_layer_buffer_bytes", "kvq_append", "kvq_work
             "kvq_h_reconstruct", "kvq_workspace_status", "kvq_status_string",
             "kvq_last_error_detail", "kvq_decode_attn_noalloc", "kvq_h_operand_bytes",
             "kvq_append_decode_attn", "kvq_h_absorbed_scratch_bytes", "kvq_h_decode_absorbed",
-            "kvq_h_fused_scratch_bytes", "kvq_h_decode_fused")
+            "kvq_h_fused_scratch_bytes", "kvq_h_decode_fused", "kvq_selftest_bounded_wait")
 
 
 class KvqError(RuntimeError):
@@ -75,6 +75,7 @@ def _load():
         "kvq_workspace_status": [P, ctypes.POINTER(i32), P],
         "kvq_h_absorbed_scratch_bytes": [cfgp, i32, pu64],
         "kvq_h_fused_scratch_bytes": [cfgp, i32, pu64],
+        "kvq_selftest_bounded_wait": [P, u64, P],
         "kvq_h_decode_fused": [cfgp, layp, P, P, i32, P, i32, ctypes.c_float, P, i32, P, u64, P],
         "kvq_h_decode_absorbed": [cfgp, layp, P, P, i32, P, i32, ctypes.c_float, P, i32, P, u64, P],
     }
@@ -355,6 +356,13 @@ def kvq_h_decode_fused(cfg: Config, layer: LayerCache, w_kv: torch.Tensor, q: to
                                    float(softmax_scale), _ptr(out), _dtype_code(out),
                                    _ptr(scratch), scratch.numel() * scratch.element_size(),
                                    _stream(stream)))
+
+
+def kvq_selftest_bounded_wait(ws, timeout_ns: int, stream=None):
+    """Run the kernels' bounded wait on a barrier nothing completes (see kvq.h)."""
+    buf = ws.buf if isinstance(ws, Workspace) else ws
+    _check("kvq_selftest_bounded_wait",
+           _lib.kvq_selftest_bounded_wait(_ptr(buf), int(timeout_ns), _stream(stream)))
 
 
 def kvq_workspace_status(ws, stream=None) -> int:

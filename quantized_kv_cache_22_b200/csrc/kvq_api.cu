@@ -920,6 +920,15 @@ int kvq_h_decode_absorbed(const kvq_config *cfg, const kvq_layer *layer, const v
     return e == cudaSuccess ? KVQ_OK : fail("absorbed decode launch", e);
 }
 
+int kvq_selftest_bounded_wait(void *workspace, uint64_t timeout_ns, kvq_stream_t stream)
+{
+    if (!workspace || timeout_ns == 0 || timeout_ns > 2000000000ull) return KVQ_ERR_INVALID_ARG;
+    if (!aligned16(workspace)) return KVQ_ERR_ALIGN;
+    cudaError_t e = launch_bounded_wait_selftest(static_cast<int *>(workspace), timeout_ns,
+                                                 reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KVQ_OK : fail("self-test launch", e);
+}
+
 int kvq_workspace_status(void *workspace, int32_t *status, kvq_stream_t stream)
 {
     if (!workspace || !status) return KVQ_ERR_INVALID_ARG;

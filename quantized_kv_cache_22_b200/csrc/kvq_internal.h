@@ -119,6 +119,9 @@ int absorb_split(int max_len);    // tokens per split of the p . h^ kernel
 uint64_t absorb_scratch_layout(int B, int Hq, int D, int ng, int bits, int max_len, uint64_t off[6]);
 cudaError_t launch_absorbed(const AbsorbParams &p, int max_len, cudaStream_t stream);
 
+// self-test of the bounded wait (kvq_selftest.cu): a wait nothing completes gives up
+cudaError_t launch_bounded_wait_selftest(int *status, uint64_t limit_ns, cudaStream_t stream);
+
 struct DecodeLaunch {
     int dh, kb, vb;
     bool kg, vg;              // grouped key / value scales

@@ -259,3 +259,12 @@ def test_fused_scratch_bytes_and_validation():
         with pytest.raises(kvq.KvqError) as e:
             kvq.kvq_h_fused_scratch_bytes(Config(**{**cfg.__dict__, **over}), 1024)
         assert e.value.status == st, over
+
+
+def test_selftest_bounded_wait_argument_checks():
+    P = ctypes.c_void_p
+    f = kvq.lib().kvq_selftest_bounded_wait
+    assert f(None, 1000, None) == -1                 # no workspace
+    assert f(P(256), 0, None) == -1                  # no limit
+    assert f(P(256), 3_000_000_000, None) == -1      # above 2 s
+    assert f(P(8), 1000, None) == -4                 # not 16-byte aligned
