@@ -388,6 +388,19 @@ KVQ_API int kvq_workspace_status(void *workspace, int32_t *status, kvq_stream_t 
  * Errors: INVALID_ARG, ALIGN, LAUNCH. */
 KVQ_API int kvq_selftest_bounded_wait(void *workspace, uint64_t timeout_ns, kvq_stream_t stream);
 
+/* The same for the decode kernel itself: kvq_decode_attn (KV mode, contiguous
+ * cache) with a wait limit of timeout_ns (1 ns .. 2 s) and a producer warp that
+ * copies nothing, so every consumer's wait for its first tile runs out: the
+ * kernel records KVQ_ERR_TIMEOUT in the workspace status word, its other warps
+ * see the abort flag and return, and `out` is left unwritten.  The workspace must
+ * then be zero-filled again before its next use (as after any timeout).
+ * Arguments as kvq_decode_attn.  Errors as kvq_decode_attn. */
+KVQ_API int kvq_selftest_decode_timeout(const kvq_config *cfg, const kvq_layer *layer,
+                                        const void *q, int32_t q_dtype, const int32_t *d_len,
+                                        void *out, int32_t out_dtype, void *workspace,
+                                        uint64_t workspace_bytes, uint64_t timeout_ns,
+                                        kvq_stream_t stream);
+
 /* Bytes of the device array behind kvq_decode_attn_noalloc (8 MiB). */
 #define KVQ_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
 

@@ -27,7 +27,8 @@ EXPORTED = ("kvq_cache_bytes", "kvq_layer_buffer_bytes", "kvq_append", "kvq_work
             "kvq_h_reconstruct", "kvq_workspace_status", "kvq_status_string",
             "kvq_last_error_detail", "kvq_decode_attn_noalloc", "kvq_h_operand_bytes",
             "kvq_append_decode_attn", "kvq_h_absorbed_scratch_bytes", "kvq_h_decode_absorbed",
-            "kvq_h_fused_scratch_bytes", "kvq_h_decode_fused", "kvq_selftest_bounded_wait")
+            "kvq_h_fused_scratch_bytes", "kvq_h_decode_fused", "kvq_selftest_bounded_wait",
+            "kvq_selftest_decode_timeout")
 
 
 class KvqError(RuntimeError):
@@ -76,6 +77,7 @@ def _load():
         "kvq_h_absorbed_scratch_bytes": [cfgp, i32, pu64],
         "kvq_h_fused_scratch_bytes": [cfgp, i32, pu64],
         "kvq_selftest_bounded_wait": [P, u64, P],
+        "kvq_selftest_decode_timeout": [cfgp, layp, P, i32, P, P, i32, P, u64, u64, P],
         "kvq_h_decode_fused": [cfgp, layp, P, P, i32, P, i32, ctypes.c_float, P, i32, P, u64, P],
         "kvq_h_decode_absorbed": [cfgp, layp, P, P, i32, P, i32, ctypes.c_float, P, i32, P, u64, P],
     }
@@ -363,6 +365,17 @@ def kvq_selftest_bounded_wait(ws, timeout_ns: int, stream=None):
     buf = ws.buf if isinstance(ws, Workspace) else ws
     _check("kvq_selftest_bounded_wait",
            _lib.kvq_selftest_bounded_wait(_ptr(buf), int(timeout_ns), _stream(stream)))
+
+
+def kvq_selftest_decode_timeout(cfg: Config, layer: LayerCache, q: torch.Tensor,
+                                d_len: torch.Tensor, out: torch.Tensor, ws: Workspace,
+                                timeout_ns: int, stream=None):
+    """The decode kernel with a producer that copies nothing: its waits run out (see kvq.h)."""
+    _check("kvq_selftest_decode_timeout",
+           _lib.kvq_selftest_decode_timeout(cfg._ref(), layer._ref(), _ptr(q), _dtype_code(q),
+                                            _ptr(d_len), _ptr(out), _dtype_code(out),
+                                            _ptr(ws.buf), ws.nbytes, int(timeout_ns),
+                                            _stream(stream)))
 
 
 def kvq_workspace_status(ws, stream=None) -> int:

@@ -471,7 +471,7 @@ static int decode_kv_layout(const kvq_config *cfg, const void *k_codes, const vo
                             int32_t out_dtype, void *workspace, uint64_t workspace_bytes,
                             int32_t num_ctas, cudaStream_t stream, bool do_partials, bool do_merge,
                             const FusedAppend *app = nullptr,
-                            const int32_t *block_table = nullptr)
+                            const int32_t *block_table = nullptr, uint64_t stall_ns = 0)
 {
     const AttnShape a = attn_shape(cfg);
     // fp16 and e4m3 keys use an f16 MMA whose f32 / bf16 queries take two columns per head
@@ -524,7 +524,8 @@ static int decode_kv_layout(const kvq_config *cfg, const void *k_codes, const vo
         p.off_merge = plan.off_merge;
         const float scale = softmax_scale != 0.f ? softmax_scale : 1.f / std::sqrt((float)a.dh);
         p.tau_log2e = scale * 1.4426950408889634f;
-        p.timeout_ns = kTimeoutNs;
+        p.timeout_ns = stall_ns ? stall_ns : kTimeoutNs;
+        p.stall = stall_ns ? 1 : 0;
         if (app) p.app = *app;
         p.window = cfg->mode == KVQ_MODE_KV ? cfg->window : 0;
         p.n_anchor = cfg->mode == KVQ_MODE_KV ? cfg->n_anchor : 0;
@@ -918,6 +919,27 @@ int kvq_h_decode_absorbed(const kvq_config *cfg, const kvq_layer *layer, const v
     p.split = absorb_split(max_len_host);
     cudaError_t e = launch_absorbed(p, max_len_host, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? KVQ_OK : fail("absorbed decode launch", e);
+}
+
+int kvq_selftest_decode_timeout(const kvq_config *cfg, const kvq_layer *layer, const void *q,
+                                int32_t q_dtype, const int32_t *d_len, void *out,
+                                int32_t out_dtype, void *workspace, uint64_t workspace_bytes,
+                                uint64_t timeout_ns, kvq_stream_t stream)
+{
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (cfg->mode != KVQ_MODE_KV || cfg->page_tokens) return KVQ_ERR_INVALID_ARG;
+    if (!layer || !q || !d_len || !out || !workspace) return KVQ_ERR_INVALID_ARG;
+    if (timeout_ns == 0 || timeout_ns > 2000000000ull) return KVQ_ERR_INVALID_ARG;
+    if (q_dtype != KVQ_F16 && q_dtype != KVQ_F32 && q_dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
+    if (out_dtype != KVQ_F16 && out_dtype != KVQ_F32) return KVQ_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return KVQ_ERR_ALIGN;
+    rc = check_kv_layer(cfg, layer);
+    if (rc) return rc;
+    return decode_kv_layout(cfg, layer->k_codes, layer->k_scales, layer->v_codes, layer->v_scales,
+                            cfg->capacity, q, q_dtype, d_len, 0.f, out, out_dtype, workspace,
+                            workspace_bytes, 0, reinterpret_cast<cudaStream_t>(stream), true, true,
+                            nullptr, nullptr, timeout_ns);
 }
 
 int kvq_selftest_bounded_wait(void *workspace, uint64_t timeout_ns, kvq_stream_t stream)

@@ -430,6 +430,7 @@ __global__ void __launch_bounds__(NTHR, 2)
 
     if (warp == NW) {
         // ====================== producer (whole warp) ======================
+        if (p.stall) return;   // self-test: nothing is copied, the consumers' waits run out
         // codes and scales are read once: let them leave L2 first, so that the
         // partials and the queries stay cached
         const uint64_t pol = l2_evict_first_policy();

@@ -81,6 +81,8 @@ struct DecodeParams {
     int32_t window, n_anchor;  // sliding window: slot of the newest token (fused append)
     const int32_t *block_table;  // paged cache (null: contiguous per sequence)
     int32_t max_pages, n_pages;
+    int32_t stall;            // self-test only: the producer issues no copy, so every
+                              // consumer wait runs out (kvq_selftest_decode_timeout)
 };
 
 struct MergeParams {
