@@ -779,7 +779,6 @@ __global__ void __launch_bounds__(NTHR, 2)
             amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 1));
             amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 2));
             const float inv = amax > 0.f ? 127.f / amax : 0.f;
-#pragma unroll
             int qs_all = 0;
 #pragma unroll
             for (int blk = 0; blk < NG; blk++) {
@@ -1022,6 +1021,32 @@ __global__ void __launch_bounds__(NTHR, 2)
                 for (int u = 0; u < 2; u++) {
                     float v[4] = {0.f, 0.f, 0.f, 0.f};
                     const int tA = tAu[u];
+                    constexpr int SCV = scale_vals(FMT);
+                    // key scales of rows tA, tA + 1 per block: with 32-element groups
+                    // (no zero-points) a row's NG scales are contiguous, one load per row
+                    float kr0[NG], kr1[NG];
+                    if (!ZP && p.kshift == 0) {
+                        if constexpr (NG == 4) {
+                            const uint2 a = lds_u64(sbase, ssk + 8 * tA), b = lds_u64(sbase, ssk + 8 * (tA + 1));
+                            const float2 a0 = unpack_half2(a.x), a1 = unpack_half2(a.y);
+                            const float2 b0 = unpack_half2(b.x), b1 = unpack_half2(b.y);
+                            kr0[0] = a0.x; kr0[1] = a0.y; kr0[2] = a1.x; kr0[3] = a1.y;
+                            kr1[0] = b0.x; kr1[1] = b0.y; kr1[2] = b1.x; kr1[3] = b1.y;
+                        } else {
+                            const float2 a = unpack_half2(lds_u32(sbase, ssk + 4 * tA));
+                            const float2 b = unpack_half2(lds_u32(sbase, ssk + 4 * (tA + 1)));
+                            kr0[0] = a.x; kr0[1] = a.y;
+                            kr1[0] = b.x; kr1[1] = b.y;
+                        }
+                    } else {
+#pragma unroll
+                        for (int blk = 0; blk < NG; blk++) {
+                            const uint32_t o0 = ssk + 2 * (tA * p.ngs_k + SCV * (blk >> p.kshift));
+                            const uint32_t o1 = ssk + 2 * ((tA + 1) * p.ngs_k + SCV * (blk >> p.kshift));
+                            kr0[blk] = __half2float(__ushort_as_half((unsigned short)lds_u16(sbase, o0)));
+                            kr1[blk] = __half2float(__ushort_as_half((unsigned short)lds_u16(sbase, o1)));
+                        }
+                    }
 #pragma unroll
                     for (int blk = 0; blk < NG; blk++) {
                         int ah[4] = {0, 0, 0, 0}, al[4] = {0, 0, 0, 0};
@@ -1030,13 +1055,11 @@ __global__ void __launch_bounds__(NTHR, 2)
                                   sst + blk_addr<RK, SK>(kofs[u][1], blk), fa);
                         imma_16832<ZP>(ah, fa[0], fa[1], fa[2], fa[3], qh[blk][0], qh[blk][1]);
                         imma_16832<ZP>(al, fa[0], fa[1], fa[2], fa[3], ql[blk][0], ql[blk][1]);
-                        constexpr int SCV = scale_vals(FMT);
-                        const uint32_t o0 = ssk + 2 * (tA * p.ngs_k + SCV * (blk >> p.kshift));
-                        const uint32_t o1 = ssk + 2 * ((tA + 1) * p.ngs_k + SCV * (blk >> p.kshift));
-                        const float k0 = __half2float(__ushort_as_half((unsigned short)lds_u16(sbase, o0)));
-                        const float k1 = __half2float(__ushort_as_half((unsigned short)lds_u16(sbase, o1)));
+                        const float k0 = kr0[blk], k1 = kr1[blk];
                         if constexpr (ZP) {
                             // minus zero-point x the block's query sum
+                            const uint32_t o0 = ssk + 2 * (tA * p.ngs_k + SCV * (blk >> p.kshift));
+                            const uint32_t o1 = ssk + 2 * ((tA + 1) * p.ngs_k + SCV * (blk >> p.kshift));
                             const int z0 = __half2int_rn(__ushort_as_half((unsigned short)lds_u16(sbase, o0 + 2)));
                             const int z1 = __half2int_rn(__ushort_as_half((unsigned short)lds_u16(sbase, o1 + 2)));
                             ah[0] = ah[0] * 254 + al[0] - z0 * zq[blk][0];
