@@ -352,10 +352,11 @@ def time_e2e(w, st, steps, warmup, world, device):
     return ms, h2d, d2h
 
 
-def cpu_oracle_layer(w, fmt, st=None, device=None, reps=1, budget_s=0.0):
+def cpu_oracle_layer(w, fmt, st=None, device=None, reps=1, budget_s=0.0, single=False):
     """Time the oracle on one layer of one decode step: quantize the new token's K/V,
     then fp64 attention for every (sequence, query head) over the 8K context.
-    Runs `reps` times, and more until `budget_s` seconds of CPU work have passed."""
+    Runs `reps` times, and more until `budget_s` seconds of CPU work have passed, on
+    every host core; with `single`, also once on one thread (returned third)."""
     import numpy as np
     import torch
     import oracle
@@ -394,15 +395,21 @@ def cpu_oracle_layer(w, fmt, st=None, device=None, reps=1, budget_s=0.0):
     qf = q.float().cpu().numpy()
     lens = np.full(w.batch, L, np.int32)
     cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
-    times = []
-    while len(times) < reps or (sum(times) < budget_s and len(times) < 1000):
+
+    def one(threads):
         t0 = time.perf_counter()
         a, b = quant(k1f, kg, kb_o, s16[0])
         kc[:, :, L - 1:], ks[:, :, L - 1:] = a, b
         a, b = quant(v1f, vg, vb_o, s16[1])
         vc[:, :, L - 1:], vs[:, :, L - 1:] = a, b
-        oracle.decode_layer(qf, lens, kc, ks, kb_o, kg, vc, vs, vb_o, vg, w.n_kv_heads, 0.0, cores)
-        times.append(time.perf_counter() - t0)
+        oracle.decode_layer(qf, lens, kc, ks, kb_o, kg, vc, vs, vb_o, vg, w.n_kv_heads, 0.0, threads)
+        return time.perf_counter() - t0
+
+    times = []
+    while len(times) < reps or (sum(times) < budget_s and len(times) < 1000):
+        times.append(one(cores))
+    if single:
+        return times, cores, one(1)
     return times, cores
 
 
@@ -758,10 +765,14 @@ def run_gpu(args):
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # a bounded sample: the same layer of the step repeated for ~10 s of CPU work
-        times, cores = cpu_oracle_layer(w, VARIANTS[head], device=device, reps=1, budget_s=10.0)
+        times, cores, t1 = cpu_oracle_layer(w, VARIANTS[head], device=device, reps=1,
+                                            budget_s=10.0, single=True)
         t = statistics.mean(times)
         per_layer = r["kv_bytes_per_step"] / w.n_layers
         line["cpu_baseline"] = {"value": round(per_layer / t / 1e9, 4), "unit": "GB/s",
+                                "single_thread": {"value": round(per_layer / t1 / 1e9, 4),
+                                                  "unit": "GB/s", "cores": 1,
+                                                  "sample": f"1 run of the same layer, {t1:.3f} s"},
                                 "steps_per_s": round(1.0 / (t * w.n_layers), 5),
                                 "cores": cores, "kind": "oracle",
                                 "sample": f"{len(times)} runs of 1 of the {w.n_layers} layers of "
