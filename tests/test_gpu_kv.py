@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 
 FORMATS = [  # (k_bits, v_bits, k_group, v_group)
     (8, 8, 0, 0), (8, 4, 0, 32), (4, 8, 32, 0), (4, 4, 0, 0), (4, 4, 32, 32), (8, 8, 32, 64),
-    (16, 16, 0, 0), (8, 16, 0, 0), (16, 4, 0, 32)]
+    (16, 16, 0, 0), (8, 16, 0, 0), (16, 4, 0, 32), (8, 8, 64, 64), (4, 8, 64, 0)]
 
 
 def _inputs(B, L, Hkv, G, dh, dtype, seed, scale_v=1.0):
