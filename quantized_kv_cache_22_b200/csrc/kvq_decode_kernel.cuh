@@ -610,7 +610,8 @@ __global__ void __launch_bounds__(NTHR, 2)
                 }
             }
         }
-        // never leave with copies in flight: wait for the last issued phases
+        // never leave with copies in flight: wait for the last issued phases, also
+        // after another warp gave up (the copies still target this CTA's memory)
         if (lane == 0) {
             int ss = s;
             uint32_t pp = ph;
@@ -620,7 +621,7 @@ __global__ void __launch_bounds__(NTHR, 2)
                     pp ^= 1u;
                 }
                 --ss;
-                (void)mbar_wait_bounded(&full[ss], pp, abort_flag, p.timeout_ns);
+                (void)mbar_wait_drain(&full[ss], pp, p.timeout_ns);
             }
         }
         return;

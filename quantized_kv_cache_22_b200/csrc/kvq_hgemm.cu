@@ -389,7 +389,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     pp ^= 1u;
                 }
                 --ss;
-                (void)mbar_wait_bounded(&full[ss], pp, abort_flag, limit);
+                (void)mbar_wait_drain(&full[ss], pp, limit);
             }
         }
     } else if (warp == 1) {
@@ -441,7 +441,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     pp ^= 1u;
                 }
                 --ss;
-                (void)mbar_wait_bounded(&empty[ss], pp, abort_flag, limit);
+                (void)mbar_wait_drain(&empty[ss], pp, limit);
             }
         }
     } else {
