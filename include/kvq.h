@@ -425,12 +425,40 @@ KVQ_API int kvq_selftest_decode_timeout(const kvq_config *cfg, const kvq_layer *
  *     last call's contents; calls that overlap on the GPU (different streams,
  *     or several host threads) race on it and give wrong results.  Each call
  *     clears the status word and the merge counters it needs zeroed.
+ *   Status: a bounded wait that gives up inside this call records
+ *     KVQ_ERR_TIMEOUT in the array's status word, not in a caller buffer; read
+ *     it with kvq_noalloc_status after the call and before the next one (the
+ *     next call clears it).
+ *   Device reset: the array's device address is kept per device for the life
+ *     of the process; after cudaDeviceReset (or anything else that destroys
+ *     the primary context) the address may be stale, so neither noalloc entry
+ *     point may be called again in that process.
  * Nothing here allocates or frees memory.  Other arguments and errors as
  * kvq_decode_attn; h-mode configs return KVQ_ERR_INVALID_ARG. */
 KVQ_API int kvq_decode_attn_noalloc(const kvq_config *cfg, const kvq_layer *layer, const void *q,
                                     int32_t q_dtype, const int32_t *d_len, int32_t max_len_host,
                                     float softmax_scale, void *out, int32_t out_dtype,
                                     int32_t num_ctas, kvq_stream_t stream);
+
+/* Read and clear the status word of the device array behind
+ * kvq_decode_attn_noalloc on the current device, like kvq_workspace_status:
+ * enqueues a 4-byte copy and a 4-byte clear on `stream` and synchronises it.
+ * *status = KVQ_OK, or KVQ_ERR_TIMEOUT when a bounded wait of the last noalloc
+ * call gave up (its `out` is then not valid).  Allocates nothing.  The source
+ * pages have no counterpart: it only completes kvq_decode_attn_noalloc. */
+KVQ_API int kvq_noalloc_status(int32_t *status, kvq_stream_t stream);
+
+/* Self-test of the failure path of kvq_decode_attn_noalloc: the same clearing
+ * of the library's array, then the decode kernel of kvq_selftest_decode_timeout
+ * (its producer copies nothing, every consumer wait gives up after timeout_ns)
+ * with that array as the workspace.  Afterwards kvq_noalloc_status reports
+ * KVQ_ERR_TIMEOUT.  No fault, trap or hang is involved.  Arguments and limits
+ * as kvq_selftest_decode_timeout; allocates nothing.  No counterpart on the
+ * source pages. */
+KVQ_API int kvq_selftest_noalloc_timeout(const kvq_config *cfg, const kvq_layer *layer,
+                                         const void *q, int32_t q_dtype, const int32_t *d_len,
+                                         void *out, int32_t out_dtype, uint64_t timeout_ns,
+                                         kvq_stream_t stream);
 
 /* Which step of the last call on this thread that returned KVQ_ERR_LAUNCH
  * failed, and the CUDA error name ("decode launch: cudaErrorX").  Valid until

@@ -28,7 +28,7 @@ EXPORTED = ("kvq_cache_bytes", "kvq_layer_buffer_bytes", "kvq_append", "kvq_work
             "kvq_last_error_detail", "kvq_decode_attn_noalloc", "kvq_h_operand_bytes",
             "kvq_append_decode_attn", "kvq_h_absorbed_scratch_bytes", "kvq_h_decode_absorbed",
             "kvq_h_fused_scratch_bytes", "kvq_h_decode_fused", "kvq_selftest_bounded_wait",
-            "kvq_selftest_decode_timeout")
+            "kvq_selftest_decode_timeout", "kvq_noalloc_status", "kvq_selftest_noalloc_timeout")
 
 
 class KvqError(RuntimeError):
@@ -80,6 +80,9 @@ def _load():
         "kvq_selftest_decode_timeout": [cfgp, layp, P, i32, P, P, i32, P, u64, u64, P],
         "kvq_h_decode_fused": [cfgp, layp, P, P, i32, P, i32, ctypes.c_float, P, i32, P, u64, P],
         "kvq_h_decode_absorbed": [cfgp, layp, P, P, i32, P, i32, ctypes.c_float, P, i32, P, u64, P],
+        "kvq_decode_attn_noalloc": [cfgp, layp, P, i32, P, i32, ctypes.c_float, P, i32, i32, P],
+        "kvq_noalloc_status": [ctypes.POINTER(i32), P],
+        "kvq_selftest_noalloc_timeout": [cfgp, layp, P, i32, P, P, i32, u64, P],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -376,6 +379,34 @@ def kvq_selftest_decode_timeout(cfg: Config, layer: LayerCache, q: torch.Tensor,
                                             _ptr(d_len), _ptr(out), _dtype_code(out),
                                             _ptr(ws.buf), ws.nbytes, int(timeout_ns),
                                             _stream(stream)))
+
+
+def kvq_decode_attn_noalloc(cfg: Config, layer: LayerCache, q: torch.Tensor, d_len: torch.Tensor,
+                            max_len: int, out: torch.Tensor, softmax_scale: float = 0.0,
+                            num_ctas: int = 0, stream=None):
+    """kvq_decode_attn with the library's own fixed device array as the workspace
+    (for callers that may not allocate device memory; see kvq.h)."""
+    _check("kvq_decode_attn_noalloc",
+           _lib.kvq_decode_attn_noalloc(cfg._ref(), layer._ref(), _ptr(q), _dtype_code(q),
+                                        _ptr(d_len), int(max_len), float(softmax_scale), _ptr(out),
+                                        _dtype_code(out), int(num_ctas), _stream(stream)))
+
+
+def kvq_noalloc_status(stream=None) -> int:
+    """Read and clear the status word of the noalloc entry point's device array."""
+    st = ctypes.c_int32()
+    _check("kvq_noalloc_status", _lib.kvq_noalloc_status(ctypes.byref(st), _stream(stream)))
+    return st.value
+
+
+def kvq_selftest_noalloc_timeout(cfg: Config, layer: LayerCache, q: torch.Tensor,
+                                 d_len: torch.Tensor, out: torch.Tensor, timeout_ns: int,
+                                 stream=None):
+    """The stalled-producer decode kernel run on the noalloc array (see kvq.h)."""
+    _check("kvq_selftest_noalloc_timeout",
+           _lib.kvq_selftest_noalloc_timeout(cfg._ref(), layer._ref(), _ptr(q), _dtype_code(q),
+                                             _ptr(d_len), _ptr(out), _dtype_code(out),
+                                             int(timeout_ns), _stream(stream)))
 
 
 def kvq_workspace_status(ws, stream=None) -> int:
