@@ -98,8 +98,9 @@ def test_fused_query_dtypes_scale_fp16_out_and_one_token(cuda_device, qdtype):
     q = (torch.randn(B, cfg.n_q_heads, 128, generator=torch.Generator().manual_seed(6)) * 2).to(qdtype)
     _, got = _gpu(cfg, h, W, q, lens, out_dtype=torch.float16, scale=0.04)
     want, vmax = _oracle(cfg, h, W, q, lens, tau=0.04)
+    # fp16 output, held to the same 2e-3 * max|V^| as every other output
     err = np.abs(got.astype(np.float64) - want).max(axis=(1, 2))
-    assert np.all(err <= 2e-3 * vmax + np.abs(want).max() * 2.0 ** -11), err
+    assert np.all(err <= 2e-3 * vmax), err
 
 
 def test_fused_agrees_with_reconstruction_and_absorbed_paths(cuda_device):
