@@ -71,10 +71,11 @@ def bf16_peaks():
 
 
 def decode_kernel_sha() -> str:
-    """sha256 over the decode kernel's device sources (kernel, PTX wrappers, quantiser)."""
+    """sha256 over the decode kernels' device sources (kernels, PTX wrappers, quantiser)."""
     import hashlib
     h = hashlib.sha256()
-    for name in ("kvq_decode_kernel.cuh", "kvq_ptx.cuh", "kvq_quant.cuh"):
+    for name in ("kvq_decode_kernel.cuh", "kvq_decode_common.cuh", "kvq_decode_tc.cu",
+                 "kvq_ptx.cuh", "kvq_quant.cuh"):
         with open(os.path.join(ROOT, "quantized_kv_cache_22_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()

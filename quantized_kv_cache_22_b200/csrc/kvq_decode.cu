@@ -71,7 +71,57 @@ void *pick_decode(int dh, int kb, int vb, bool kg, bool vg, int fmt)
 
 inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
+// Whether the tensor-core kernel serves the formats it supports (otherwise the
+// warp-MMA kernel does): the faster of the two on the 8K workload.
+constexpr bool kTcDecode = false;
+
 }  // namespace
+
+// The tensor-core kernel takes INT8 / INT4 codes with per-(token, head) value scales,
+// key scales per (token, head) or per 32/64-element group (or per-tensor INT8),
+// head_dim 128 and up to 8 query heads per KV head.  One CTA per
+// SM: the ring gets as many stages as the shared memory holds next to the kernel's
+// double-buffered fp16 value, P, widened-key and query tiles.
+static bool plan_decode_tc(int dh, int kb, int vb, bool kg, bool vg, int ngs_k, int G,
+                           int max_smem, DecodeLaunch *plan, int fmt)
+{
+    if (dh != 128 || vg || G > 8 || !decode_tc_fn(kb, vb, kg, fmt)) return false;
+    DecodeLaunch L{};
+    L.dh = dh; L.kb = kb; L.vb = vb; L.kg = kg; L.vg = false; L.fmt = fmt; L.tc = true;
+    const bool pt = fmt == KVQ_FMT_TENSOR;
+    const uint32_t rk = dh * kb / 8, rv = dh * vb / 8;
+    L.off_v = align_up(T * rk, 1024);
+    L.off_sk = L.off_v + align_up(T * rv, 1024);
+    L.off_sv = L.off_sk + align_up(T * (pt ? 0 : ngs_k) * 2, 16);
+    L.stage_bytes = align_up(L.off_sv + T * (pt ? 0 : 1) * 2, 1024);
+    for (int S = 8; S >= 2; S--) {
+        TcOffsets o{};
+        uint32_t off = S * L.stage_bytes;
+        o.off_kx = off;
+        off += kb == 4 ? 2u * 128u * 128u : 0u;
+        o.off_v16 = off;
+        off += 2u * 128u * 128u * 2u;
+        o.off_pb = off;
+        off += 2u * 2u * 16u * 128u;
+        o.off_qb = off;
+        off += 2u * 16u * 128u;
+        const uint32_t off_meta = off;
+        const uint32_t off_bar = align_up(off_meta + S * (uint32_t)sizeof(StageMeta), 16);
+        o.off_aux = align_up(off_bar + 2u * S * 8u + kTcBarsBytes, 16);
+        const uint32_t total = o.off_aux + kTcAuxBytes + 1024;   // + alignment slack
+        if (total <= (uint32_t)max_smem) {
+            L.stages = S;
+            L.off_meta = off_meta;
+            L.off_bar = off_bar;
+            L.off_merge = 0;
+            L.tco = o;
+            L.smem_bytes = total;
+            *plan = L;
+            return true;
+        }
+    }
+    return false;
+}
 
 bool plan_decode(int dh, int kb, int vb, int ngs_k, int ngs_v, int G, int max_smem,
                  DecodeLaunch *plan, int fmt)
@@ -80,6 +130,7 @@ bool plan_decode(int dh, int kb, int vb, int ngs_k, int ngs_v, int G, int max_sm
     // a zero-point; none for 16-bit or per-tensor codes)
     const int sv = scale_vals(fmt);
     const bool kg = kb != 16 && ngs_k / sv > 1, vg = vb != 16 && ngs_v / sv > 1;
+    if (kTcDecode && plan_decode_tc(dh, kb, vb, kg, vg, ngs_k, G, max_smem, plan, fmt)) return true;
     if (!pick_decode(dh, kb, vb, kg, vg, fmt)) return false;
     const uint32_t rk = dh * kb / 8, rv = dh * vb / 8;
     DecodeLaunch L{};
@@ -129,7 +180,7 @@ std::mutex g_memo_mu;
 std::vector<AttrMemo> g_attr;
 std::vector<OccMemo> g_occ;
 
-cudaError_t prepare_fn(void *fn, size_t smem, int *occupancy)
+cudaError_t prepare_fn(void *fn, size_t smem, int *occupancy, int threads)
 {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -158,7 +209,7 @@ cudaError_t prepare_fn(void *fn, size_t smem, int *occupancy)
             return cudaSuccess;
         }
     int occ = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, NTHR, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, threads, smem);
     if (e != cudaSuccess) return e;
     g_occ.push_back(OccMemo{dev, fn, smem, occ});
     *occupancy = occ;
@@ -166,17 +217,22 @@ cudaError_t prepare_fn(void *fn, size_t smem, int *occupancy)
 }
 }  // namespace
 
+static void *plan_fn(const DecodeLaunch &plan)
+{
+    return plan.tc ? decode_tc_fn(plan.kb, plan.vb, plan.kg, plan.fmt)
+                   : pick_decode(plan.dh, plan.kb, plan.vb, plan.kg, plan.vg, plan.fmt);
+}
+
 cudaError_t decode_occupancy(const DecodeLaunch &plan, int *ctas_per_sm)
 {
-    return prepare_fn(pick_decode(plan.dh, plan.kb, plan.vb, plan.kg, plan.vg, plan.fmt), plan.smem_bytes,
-                      ctas_per_sm);
+    return prepare_fn(plan_fn(plan), plan.smem_bytes, ctas_per_sm, plan.tc ? 192 : NTHR);
 }
 
 cudaError_t launch_decode(const DecodeLaunch &plan, const DecodeParams &p, const CUtensorMap &tm_k,
                           const CUtensorMap &tm_v, cudaStream_t stream)
 {
-    void *fn = pick_decode(plan.dh, plan.kb, plan.vb, plan.kg, plan.vg, plan.fmt);
-    cudaError_t e = prepare_fn(fn, plan.smem_bytes, nullptr);
+    void *fn = plan_fn(plan);
+    cudaError_t e = prepare_fn(fn, plan.smem_bytes, nullptr, 0);
     if (e != cudaSuccess) return e;
     void *args[] = {const_cast<CUtensorMap *>(&tm_k), const_cast<CUtensorMap *>(&tm_v),
                     const_cast<DecodeParams *>(&p)};
@@ -185,7 +241,7 @@ cudaError_t launch_decode(const DecodeLaunch &plan, const DecodeParams &p, const
     // (griddepcontrol.wait) before its first global-memory access.
     cudaLaunchConfig_t lc = {};
     lc.gridDim = dim3(p.num_ctas);
-    lc.blockDim = dim3(NTHR);
+    lc.blockDim = dim3(plan.tc ? 192 : NTHR);
     lc.dynamicSmemBytes = plan.smem_bytes;
     lc.stream = stream;
     cudaLaunchAttribute attr[1];

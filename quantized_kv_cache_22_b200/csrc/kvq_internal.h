@@ -58,6 +58,15 @@ struct FusedAppend {
 // fp16 values per scale group in the scale arrays of a code format
 __host__ __device__ constexpr int scale_vals(int fmt) { return fmt == KVQ_FMT_ASYM ? 2 : 1; }
 
+// Shared-memory regions of the tensor-core decode kernel (kvq_decode_tc.cu) after its
+// stage ring: widened INT4 keys, fp16 value tiles, P tiles, int8 query rows, and the
+// control area (barriers are at off_bar as for the warp-MMA kernel).
+struct TcOffsets {
+    uint32_t off_kx, off_v16, off_pb, off_qb, off_aux;
+};
+constexpr uint32_t kTcBarsBytes = 256;    // the kernel's extra mbarriers
+constexpr uint32_t kTcAuxBytes = 1024;    // factors, max exchange, sums, TMEM address
+
 struct DecodeParams {
     const int32_t *d_len;     // [B]
     const void *q;            // [B][Hq][Dh]
@@ -83,6 +92,7 @@ struct DecodeParams {
     int32_t max_pages, n_pages;
     int32_t stall;            // self-test only: the producer issues no copy, so every
                               // consumer wait runs out (kvq_selftest_decode_timeout)
+    TcOffsets tc;             // tensor-core kernel only
 };
 
 struct MergeParams {
@@ -128,9 +138,11 @@ struct DecodeLaunch {
     int dh, kb, vb;
     bool kg, vg;              // grouped key / value scales
     int fmt;                  // KVQ_FMT_* of the 8-bit codes
+    bool tc;                  // the tensor-core kernel (kvq_decode_tc.cu)
     size_t smem_bytes;
     int stages;
     uint32_t stage_bytes, off_v, off_sk, off_sv, off_meta, off_bar, off_merge;
+    TcOffsets tco;
 };
 
 // Decode kernel instances (kvq_decode_k4/k8/k16.cu), by key width: the kernel
@@ -141,6 +153,10 @@ void *decode_fn_kb8(int dh, int vb, bool kg, bool vg);
 void *decode_fn_kb16(int dh, int vb, bool kg, bool vg);
 // e4m3, asymmetric and per-tensor 8-bit keys and values (kvq_decode_fmt.cu)
 void *decode_fn_fmt(int dh, int fmt, bool kg, bool vg);
+// the tensor-core kernel (head_dim 128; value scales per (token, head), key scales
+// per (token, head) or per 32/64-element group; or per-tensor INT8): INT8 / INT4 keys
+// and values, or null (kvq_decode_tc.cu)
+void *decode_tc_fn(int kb, int vb, bool kg, int fmt);
 
 // Fill in the shared-memory plan; returns false if the shape is unsupported.
 bool plan_decode(int dh, int kb, int vb, int ngs_k, int ngs_v, int G, int max_smem,

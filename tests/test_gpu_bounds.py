@@ -54,7 +54,8 @@ def _guarded_layer(cfg: Config, seed: int, block_table=None):
         if nb == 0:
             setattr(layer, name, None)
             continue
-        gb = Guarded(nb, dt, seed + i)
+        # the interior starts zeroed: rows the test never appends hold code 0, scale 0
+        gb = Guarded(nb, dt, seed + i, zero=True)
         setattr(layer, name, gb.view)
         guards.append((name, gb))
     return layer, guards

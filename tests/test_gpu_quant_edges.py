@@ -112,7 +112,7 @@ def test_edge_groups_fused_append_bit_exact(cuda_device, fmt):
     kb, vb, kg, vg = fmt
     B, L, Hkv, G = 2, 40, 2, 4
     k, v = _kv(kb, vb, B, L, Hkv, 400 + kb * 10 + vb + kg)
-    cfg = Config(batch=B, capacity=L, n_q_heads=Hkv * G, n_kv_heads=Hkv, head_dim=DH,
+    cfg = Config(batch=B, capacity=48, n_q_heads=Hkv * G, n_kv_heads=Hkv, head_dim=DH,
                  k_bits=kb, v_bits=vb, k_group=kg, v_group=vg)
     cache = LayerCache(cfg, zero=True)
     ws = Workspace(cfg)
@@ -131,4 +131,4 @@ def test_edge_groups_fused_append_bit_exact(cuda_device, fmt):
     assert kvq.kvq_workspace_status(ws) == 0
     gc = read_gpu_cache(cache, cfg)
     for i, name in enumerate(("k_codes", "k_scales", "v_codes", "v_scales")):
-        assert np.array_equal(gc[i], oc[i]), name
+        assert np.array_equal(gc[i][:, :, :L], oc[i][:, :, :L]), name

@@ -168,7 +168,8 @@ def test_noalloc_paged_cache(cuda_device):
     table = torch.randperm(n_pages, generator=g)[: B * (cap // 128)].view(B, -1).to(torch.int32)
     cache = LayerCache(cfg, block_table=table.cuda())
     pos = torch.zeros(B, dtype=torch.int32, device="cuda")
-    kvq.kvq_append(cfg, cache, k.cuda(), v.cuda(), pos, 0, max(lens))
+    n = max(lens)
+    kvq.kvq_append(cfg, cache, k[:, :n].contiguous().cuda(), v[:, :n].contiguous().cuda(), pos, 0, n)
     d_len = torch.tensor(lens, dtype=torch.int32, device="cuda")
     out = torch.full((B, Hkv * G, dh), float("nan"), dtype=torch.float32, device="cuda")
     kvq.kvq_decode_attn_noalloc(cfg, cache, q.cuda(), d_len, max(lens), out)
