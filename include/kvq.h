@@ -222,6 +222,31 @@ KVQ_API int kvq_append(const kvq_config *cfg, const kvq_layer *layer, const void
  * device; pass an explicit count to size it without one). */
 KVQ_API int kvq_workspace_bytes(const kvq_config *cfg, int32_t num_ctas, uint64_t *bytes);
 
+/* The decode-attention launch kvq_decode_attn / kvq_append_decode_attn /
+ * kvq_decode_partials make for this config with `num_ctas` CTAs (0 = the
+ * library's choice for the current device, which needs a CUDA device).
+ *   engine     KVQ_ENGINE_WARP_MMA: the warp-level MMA kernel (the default for
+ *              every format); KVQ_ENGINE_TCGEN05: the tcgen05/TMEM kernel (its
+ *              P.V product is an exact integer MMA of the value codes with P in
+ *              fixed point of 2^-24), chosen only when the environment
+ *              variable KVQ_DECODE_TC is "1" at the call and the format is one
+ *              it supports (head_dim 128, INT8/INT4 codes, value scales per
+ *              (token, head), G <= 8).  The variable is read at every call, so
+ *              size the workspace under the same setting as the call.
+ *   num_ctas   persistent CTAs of the launch (the work split over them)
+ *   ctas_per_sm_planned  CTAs per SM its shared memory and registers are sized for
+ *   stages, stage_bytes  depth and bytes of the TMA ring (one 128-token K/V tile
+ *              with its scales per stage); smem_bytes  dynamic shared memory
+ *   threads    threads per CTA
+ * Errors: INVALID_ARG, UNSUPPORTED, DEVICE. */
+#define KVQ_ENGINE_WARP_MMA 0
+#define KVQ_ENGINE_TCGEN05 1
+typedef struct kvq_decode_plan {
+    int32_t engine, num_ctas, ctas_per_sm_planned, stages;
+    int32_t stage_bytes, smem_bytes, threads, reserved;
+} kvq_decode_plan;
+KVQ_API int kvq_decode_plan_info(const kvq_config *cfg, int32_t num_ctas, kvq_decode_plan *info);
+
 /* h-mode scratch bytes for kvq_decode_attn: the reconstructed fp16 K and V for
  * up to max_len tokens of every sequence ([2][B][Hkv][round_up(max_len,64)][Dh]),
  * followed by the bf16 GEMM operand (kvq_h_operand_bytes). */

@@ -28,7 +28,8 @@ EXPORTED = ("kvq_cache_bytes", "kvq_layer_buffer_bytes", "kvq_append", "kvq_work
             "kvq_last_error_detail", "kvq_decode_attn_noalloc", "kvq_h_operand_bytes",
             "kvq_append_decode_attn", "kvq_h_absorbed_scratch_bytes", "kvq_h_decode_absorbed",
             "kvq_h_fused_scratch_bytes", "kvq_h_decode_fused", "kvq_selftest_bounded_wait",
-            "kvq_selftest_decode_timeout", "kvq_noalloc_status", "kvq_selftest_noalloc_timeout")
+            "kvq_selftest_decode_timeout", "kvq_noalloc_status", "kvq_selftest_noalloc_timeout",
+            "kvq_decode_plan_info")
 
 
 class KvqError(RuntimeError):
@@ -43,6 +44,15 @@ class KvqConfig(ctypes.Structure):
         "mode", "batch", "capacity", "n_layers", "n_q_heads", "n_kv_heads", "head_dim",
         "k_bits", "v_bits", "k_group", "v_group", "d_model", "h_bits", "h_groups",
         "window", "n_anchor", "page_tokens", "n_pages", "kv_format")]
+
+
+class KvqDecodePlan(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "engine", "num_ctas", "ctas_per_sm_planned", "stages", "stage_bytes", "smem_bytes",
+        "threads", "reserved")]
+
+
+KVQ_ENGINE_WARP_MMA, KVQ_ENGINE_TCGEN05 = 0, 1
 
 
 class KvqLayer(ctypes.Structure):
@@ -83,6 +93,7 @@ def _load():
         "kvq_decode_attn_noalloc": [cfgp, layp, P, i32, P, i32, ctypes.c_float, P, i32, i32, P],
         "kvq_noalloc_status": [ctypes.POINTER(i32), P],
         "kvq_selftest_noalloc_timeout": [cfgp, layp, P, i32, P, P, i32, u64, P],
+        "kvq_decode_plan_info": [cfgp, i32, ctypes.POINTER(KvqDecodePlan)],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -201,6 +212,14 @@ def kvq_workspace_bytes(cfg: Config, num_ctas: int = 0) -> int:
     _check("kvq_workspace_bytes", _lib.kvq_workspace_bytes(ctypes.byref(cfg.c()), num_ctas,
                                                            ctypes.byref(v)))
     return v.value
+
+
+def kvq_decode_plan_info(cfg: Config, num_ctas: int = 0) -> dict:
+    """The decode launch the library makes for cfg: engine, CTAs, ring depth, shared memory."""
+    v = KvqDecodePlan()
+    _check("kvq_decode_plan_info", _lib.kvq_decode_plan_info(ctypes.byref(cfg.c()), num_ctas,
+                                                             ctypes.byref(v)))
+    return {n: getattr(v, n) for n, _ in KvqDecodePlan._fields_ if n != "reserved"}
 
 
 def kvq_h_scratch_bytes(cfg: Config, max_len: int) -> int:

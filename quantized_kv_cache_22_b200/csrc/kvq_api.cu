@@ -261,6 +261,10 @@ int resolve_plan(const kvq_config *cfg, int32_t num_ctas, DecodeLaunch *plan, in
     }
     int per_sm = 0;
     if (decode_occupancy(*plan, &per_sm) != cudaSuccess || per_sm < 1) return KVQ_ERR_DEVICE;
+    // the occupancy query reports one CTA per SM for the tensor-core kernel although
+    // two of the size it is planned for run side by side (measured: 296 CTAs of the
+    // 8K K8V8 launch take 54.9 us, 148 take 73.8 us), so its plan decides
+    if (plan->tc) per_sm = plan->per_sm;
     *ctas = sms * per_sm;
     return KVQ_OK;
 }
@@ -426,6 +430,27 @@ int kvq_workspace_bytes(const kvq_config *cfg, int32_t num_ctas, uint64_t *bytes
     rc = resolve_plan(cfg, num_ctas, &plan, &ctas);
     if (rc) return rc;
     *bytes = workspace_need(cfg, ctas);
+    return KVQ_OK;
+}
+
+int kvq_decode_plan_info(const kvq_config *cfg, int32_t num_ctas, kvq_decode_plan *info)
+{
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (!info || num_ctas < 0) return KVQ_ERR_INVALID_ARG;
+    if (cfg->mode == KVQ_MODE_H && cfg->n_kv_heads * cfg->head_dim != cfg->d_model)
+        return KVQ_ERR_INVALID_ARG;
+    DecodeLaunch plan;
+    int ctas = 0;
+    rc = resolve_plan(cfg, num_ctas, &plan, &ctas);
+    if (rc) return rc;
+    info->engine = plan.tc ? KVQ_ENGINE_TCGEN05 : KVQ_ENGINE_WARP_MMA;
+    info->num_ctas = ctas;
+    info->ctas_per_sm_planned = plan.per_sm;
+    info->stages = plan.stages;
+    info->stage_bytes = plan.stage_bytes;
+    info->smem_bytes = (int32_t)plan.smem_bytes;
+    info->threads = plan.tc ? 192 : kDecodeThreads;
     return KVQ_OK;
 }
 

@@ -1,6 +1,7 @@
 // kvq_decode.cu -- host side of the decode attention: shared-memory plan,
 // kernel selection, launches, and the merge kernel for partials left by a
 // decode launch without arrival counters.
+#include <cstdlib>
 #include <mutex>
 #include <vector>
 
@@ -71,53 +72,65 @@ void *pick_decode(int dh, int kb, int vb, bool kg, bool vg, int fmt)
 
 inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
-// Whether the tensor-core kernel serves the formats it supports (otherwise the
-// warp-MMA kernel does): the faster of the two on the 8K workload.
-constexpr bool kTcDecode = false;
+// The warp-MMA kernel serves every format by default: on the 8K workload it is as
+// fast as the tensor-core kernel for INT8 keys and values and faster for INT4
+// ones.  KVQ_DECODE_TC=1 in the environment (read at each call) selects the
+// tensor-core kernel for the formats it supports; its integer P.V is exact up to
+// the 2^-25 rounding of P per token.
+static bool tc_selected()
+{
+    const char *e = std::getenv("KVQ_DECODE_TC");
+    return e && e[0] == '1' && e[1] == '\0';
+}
 
 }  // namespace
 
 // The tensor-core kernel takes INT8 / INT4 codes with per-(token, head) value scales,
 // key scales per (token, head) or per 32/64-element group (or per-tensor INT8),
-// head_dim 128 and up to 8 query heads per KV head.  One CTA per
-// SM: the ring gets as many stages as the shared memory holds next to the kernel's
-// double-buffered fp16 value, P, widened-key and query tiles.
+// head_dim 128 and up to 8 query heads per KV head.  Two CTAs per SM when a ring of
+// at least 3 stages fits next to the widened-code, P-digit and query tiles of each,
+// else one CTA per SM with as many stages as fit (2 stages per CTA measured slower).
 static bool plan_decode_tc(int dh, int kb, int vb, bool kg, bool vg, int ngs_k, int G,
                            int max_smem, DecodeLaunch *plan, int fmt)
 {
-    if (dh != 128 || vg || G > 8 || !decode_tc_fn(kb, vb, kg, fmt)) return false;
+    if (dh != 128 || vg || G > 8 || !decode_tc_fn(kb, vb, kg, G, fmt)) return false;
     DecodeLaunch L{};
-    L.dh = dh; L.kb = kb; L.vb = vb; L.kg = kg; L.vg = false; L.fmt = fmt; L.tc = true;
+    L.dh = dh; L.kb = kb; L.vb = vb; L.kg = kg; L.vg = false; L.fmt = fmt; L.tc = true; L.G = G;
     const bool pt = fmt == KVQ_FMT_TENSOR;
     const uint32_t rk = dh * kb / 8, rv = dh * vb / 8;
     L.off_v = align_up(T * rk, 1024);
     L.off_sk = L.off_v + align_up(T * rv, 1024);
     L.off_sv = L.off_sk + align_up(T * (pt ? 0 : ngs_k) * 2, 16);
     L.stage_bytes = align_up(L.off_sv + T * (pt ? 0 : 1) * 2, 1024);
-    for (int S = 8; S >= 2; S--) {
-        TcOffsets o{};
-        uint32_t off = S * L.stage_bytes;
-        o.off_kx = off;
-        off += kb == 4 ? 2u * 128u * 128u : 0u;
-        o.off_v16 = off;
-        off += 2u * 128u * 128u * 2u;
-        o.off_pb = off;
-        off += 2u * 2u * 16u * 128u;
-        o.off_qb = off;
-        off += 2u * 16u * 128u;
-        const uint32_t off_meta = off;
-        const uint32_t off_bar = align_up(off_meta + S * (uint32_t)sizeof(StageMeta), 16);
-        o.off_aux = align_up(off_bar + 2u * S * 8u + kTcBarsBytes, 16);
-        const uint32_t total = o.off_aux + kTcAuxBytes + 1024;   // + alignment slack
-        if (total <= (uint32_t)max_smem) {
-            L.stages = S;
-            L.off_meta = off_meta;
-            L.off_bar = off_bar;
-            L.off_merge = 0;
-            L.tco = o;
-            L.smem_bytes = total;
-            *plan = L;
-            return true;
+    const uint32_t pb = decode_tc_pb_bytes(G);
+    for (int per_sm = 2; per_sm >= 1; per_sm--) {
+        const uint32_t budget = per_sm == 2 ? 233472u / 2 - 1024u - 128u : (uint32_t)max_smem;
+        for (int S = 8; S >= (per_sm == 2 ? 3 : 2); S--) {
+            TcOffsets o{};
+            uint32_t off = S * L.stage_bytes;
+            o.off_kx = off;
+            off += kb == 4 ? 128u * 128u : 0u;
+            o.off_vx = off;
+            off += vb == 4 ? 2u * 128u * 128u : 0u;
+            o.off_pb = off;
+            off += 2u * pb;
+            o.off_qb = off;
+            off += 2u * 16u * 128u;
+            const uint32_t off_meta = off;
+            const uint32_t off_bar = align_up(off_meta + S * (uint32_t)sizeof(StageMeta), 16);
+            o.off_aux = align_up(off_bar + 2u * S * 8u + kTcBarsBytes, 16);
+            const uint32_t total = o.off_aux + kTcAuxBytes + 1024;   // + alignment slack
+            if (total <= budget && total <= (uint32_t)max_smem) {
+                L.stages = S;
+                L.per_sm = per_sm;
+                L.off_meta = off_meta;
+                L.off_bar = off_bar;
+                L.off_merge = 0;
+                L.tco = o;
+                L.smem_bytes = total;
+                *plan = L;
+                return true;
+            }
         }
     }
     return false;
@@ -130,7 +143,7 @@ bool plan_decode(int dh, int kb, int vb, int ngs_k, int ngs_v, int G, int max_sm
     // a zero-point; none for 16-bit or per-tensor codes)
     const int sv = scale_vals(fmt);
     const bool kg = kb != 16 && ngs_k / sv > 1, vg = vb != 16 && ngs_v / sv > 1;
-    if (kTcDecode && plan_decode_tc(dh, kb, vb, kg, vg, ngs_k, G, max_smem, plan, fmt)) return true;
+    if (tc_selected() && plan_decode_tc(dh, kb, vb, kg, vg, ngs_k, G, max_smem, plan, fmt)) return true;
     if (!pick_decode(dh, kb, vb, kg, vg, fmt)) return false;
     const uint32_t rk = dh * kb / 8, rv = dh * vb / 8;
     DecodeLaunch L{};
@@ -140,15 +153,19 @@ bool plan_decode(int dh, int kb, int vb, int ngs_k, int ngs_v, int G, int max_sm
     L.off_sv = L.off_sk + align_up(T * (kb == 16 ? 0 : ngs_k) * 2, 16);
     L.stage_bytes = align_up(L.off_sv + T * (vb == 16 ? 0 : ngs_v) * 2, 1024);
     const uint32_t merge_bytes = (uint32_t)NW * G * slot_col_floats(dh) * 4;
-    // tail: meta[S] (32 B each), barriers (2S + 2) * 8 B, control words 64 B, merge buffer
+    // tail: meta[S] (32 B each), barriers (2S + 2) * 8 B, control words 64 B, merge buffer;
+    // as many stages as fit next to the other CTAs of an SM (228 KB of shared memory,
+    // 1 KB of it reserved per CTA, 128 B left for the kernel's static shared memory),
+    // else as many as fit in one CTA
+    const uint32_t per_cta = 233472u / (uint32_t)kDecodeCtasPerSm - 1024u - 128u;
     for (int S = 8; S >= 2; S--) {
         const uint32_t off_meta = S * L.stage_bytes;
         const uint32_t off_bar = off_meta + S * (uint32_t)sizeof(StageMeta);
         const uint32_t off_merge = align_up(off_bar + (2 * S + 2) * 8 + 64, 16);
         const uint32_t total = off_merge + merge_bytes + 1024;  // + alignment slack
-        // keep two CTAs per SM when possible
-        if (total <= (uint32_t)max_smem / 2 - 1024 || (S == 2 && total <= (uint32_t)max_smem)) {
+        if ((total <= per_cta && total <= (uint32_t)max_smem) || (S == 2 && total <= (uint32_t)max_smem)) {
             L.stages = S;
+            L.per_sm = total <= per_cta ? kDecodeCtasPerSm : 1;
             L.off_meta = off_meta;
             L.off_bar = off_bar;
             L.off_merge = off_merge;
@@ -219,7 +236,7 @@ cudaError_t prepare_fn(void *fn, size_t smem, int *occupancy, int threads)
 
 static void *plan_fn(const DecodeLaunch &plan)
 {
-    return plan.tc ? decode_tc_fn(plan.kb, plan.vb, plan.kg, plan.fmt)
+    return plan.tc ? decode_tc_fn(plan.kb, plan.vb, plan.kg, plan.G, plan.fmt)
                    : pick_decode(plan.dh, plan.kb, plan.vb, plan.kg, plan.vg, plan.fmt);
 }
 

@@ -43,9 +43,10 @@ constexpr int kDecodeConsumerWarps = 4;
 constexpr int kDecodeTileTokens = 32 * kDecodeConsumerWarps;   // tokens per stage (32 per warp)
 // consumer warps, one producer warp, one combiner warp
 constexpr int kDecodeThreads = 32 * (kDecodeConsumerWarps + 2);
-static_assert(kPageTokens == kDecodeTileTokens, "a decode tile is one page of a paged cache");
+// CTAs per SM the decode kernel is compiled for (168 registers per thread) and its
+// shared-memory ring is planned for
+constexpr int kDecodeCtasPerSm = 2;
 constexpr int kWorkspaceHeaderFloats = 64;                      // status word + padding
-
 // The new token's K/V for the append step fused into the decode kernel.
 struct FusedAppend {
     const void *k_new, *v_new;    // [B][Hkv][Dh] in dtype; null: no append
@@ -59,10 +60,10 @@ struct FusedAppend {
 __host__ __device__ constexpr int scale_vals(int fmt) { return fmt == KVQ_FMT_ASYM ? 2 : 1; }
 
 // Shared-memory regions of the tensor-core decode kernel (kvq_decode_tc.cu) after its
-// stage ring: widened INT4 keys, fp16 value tiles, P tiles, int8 query rows, and the
+// stage ring: widened INT4 keys and values, P digit tiles, int8 query rows, and the
 // control area (barriers are at off_bar as for the warp-MMA kernel).
 struct TcOffsets {
-    uint32_t off_kx, off_v16, off_pb, off_qb, off_aux;
+    uint32_t off_kx, off_vx, off_pb, off_qb, off_aux;
 };
 constexpr uint32_t kTcBarsBytes = 256;    // the kernel's extra mbarriers
 constexpr uint32_t kTcAuxBytes = 1024;    // factors, max exchange, sums, TMEM address
@@ -139,6 +140,8 @@ struct DecodeLaunch {
     bool kg, vg;              // grouped key / value scales
     int fmt;                  // KVQ_FMT_* of the 8-bit codes
     bool tc;                  // the tensor-core kernel (kvq_decode_tc.cu)
+    int G;                    // query heads per KV head (tensor-core kernel instance)
+    int per_sm;               // CTAs per SM the plan's shared memory is sized for
     size_t smem_bytes;
     int stages;
     uint32_t stage_bytes, off_v, off_sk, off_sv, off_meta, off_bar, off_merge;
@@ -155,8 +158,10 @@ void *decode_fn_kb16(int dh, int vb, bool kg, bool vg);
 void *decode_fn_fmt(int dh, int fmt, bool kg, bool vg);
 // the tensor-core kernel (head_dim 128; value scales per (token, head), key scales
 // per (token, head) or per 32/64-element group; or per-tensor INT8): INT8 / INT4 keys
-// and values, or null (kvq_decode_tc.cu)
-void *decode_tc_fn(int kb, int vb, bool kg, int fmt);
+// and values with G query heads per KV head, or null (kvq_decode_tc.cu); and the
+// bytes of one of its P digit tiles
+void *decode_tc_fn(int kb, int vb, bool kg, int G, int fmt);
+uint32_t decode_tc_pb_bytes(int G);
 
 // Fill in the shared-memory plan; returns false if the shape is unsupported.
 bool plan_decode(int dh, int kb, int vb, int ngs_k, int ngs_v, int G, int max_smem,

@@ -268,3 +268,31 @@ def test_selftest_bounded_wait_argument_checks():
     assert f(P(256), 0, None) == -1                  # no limit
     assert f(P(256), 3_000_000_000, None) == -1      # above 2 s
     assert f(P(8), 1000, None) == -4                 # not 16-byte aligned
+
+
+def test_decode_plan_info_without_device(monkeypatch):
+    # explicit CTA counts plan without a device: the warp-MMA kernel by default, two
+    # CTAs per SM where a ring of two or more stages fits beside another CTA; the
+    # tcgen05 kernel only when KVQ_DECODE_TC=1 and the format is one it takes
+    def cfg(kb, vb, vg=128, dh=128):
+        return Config(batch=16, capacity=8192, n_q_heads=32, n_kv_heads=8, head_dim=dh,
+                      k_bits=kb, v_bits=vb, k_group=dh, v_group=vg if vb != 16 else dh)
+    monkeypatch.delenv("KVQ_DECODE_TC", raising=False)
+    # (16-bit keys and values: a two-stage ring of 64 KB tiles fits one CTA per SM)
+    for kb, vb, per_sm in ((8, 8, 2), (8, 4, 2), (4, 4, 2), (4, 8, 2), (16, 16, 1)):
+        info = kvq.kvq_decode_plan_info(cfg(kb, vb), 296)
+        assert info["engine"] == kvq.KVQ_ENGINE_WARP_MMA and info["num_ctas"] == 296
+        assert info["ctas_per_sm_planned"] == per_sm and info["threads"] == 192
+        assert info["stages"] >= 2 and info["stage_bytes"] * info["stages"] < info["smem_bytes"]
+        # the plan's shared memory leaves room for that many CTAs on a 228 KB SM
+        assert per_sm * (info["smem_bytes"] + 1024 + 128) <= 233472
+    assert kvq.kvq_decode_plan_info(cfg(4, 4, vg=64, dh=64), 10)["ctas_per_sm_planned"] == 2
+    monkeypatch.setenv("KVQ_DECODE_TC", "1")
+    for kb, vb in ((8, 8), (8, 4), (4, 4), (4, 8)):
+        info = kvq.kvq_decode_plan_info(cfg(kb, vb), 296)
+        assert info["engine"] == kvq.KVQ_ENGINE_TCGEN05 and info["stages"] >= 2
+    # grouped value scales and 16-bit codes stay on the warp-MMA kernel
+    assert kvq.kvq_decode_plan_info(cfg(8, 4, vg=32), 296)["engine"] == kvq.KVQ_ENGINE_WARP_MMA
+    assert kvq.kvq_decode_plan_info(cfg(16, 16), 296)["engine"] == kvq.KVQ_ENGINE_WARP_MMA
+    with pytest.raises(kvq.KvqError):
+        kvq.kvq_decode_plan_info(cfg(8, 8), -1)
