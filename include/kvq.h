@@ -238,12 +238,15 @@ KVQ_API int kvq_workspace_bytes(const kvq_config *cfg, int32_t num_ctas, uint64_
  *   stages, stage_bytes  depth and bytes of the TMA ring (one 128-token K/V tile
  *              with its scales per stage); smem_bytes  dynamic shared memory
  *   threads    threads per CTA
+ *   packed_columns  1 when the warp-MMA kernel packs the score MMA's columns (G <= 4 at
+ *              head_dim 128 with INT4 / INT8 keys): the hi and lo query parts share one
+ *              MMA, and each lane's softmax work covers live columns only
  * Errors: INVALID_ARG, UNSUPPORTED, DEVICE. */
 #define KVQ_ENGINE_WARP_MMA 0
 #define KVQ_ENGINE_TCGEN05 1
 typedef struct kvq_decode_plan {
     int32_t engine, num_ctas, ctas_per_sm_planned, stages;
-    int32_t stage_bytes, smem_bytes, threads, reserved;
+    int32_t stage_bytes, smem_bytes, threads, packed_columns;
 } kvq_decode_plan;
 KVQ_API int kvq_decode_plan_info(const kvq_config *cfg, int32_t num_ctas, kvq_decode_plan *info);
 

@@ -49,7 +49,7 @@ class KvqConfig(ctypes.Structure):
 class KvqDecodePlan(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "engine", "num_ctas", "ctas_per_sm_planned", "stages", "stage_bytes", "smem_bytes",
-        "threads", "reserved")]
+        "threads", "packed_columns")]
 
 
 KVQ_ENGINE_WARP_MMA, KVQ_ENGINE_TCGEN05 = 0, 1
@@ -219,7 +219,7 @@ def kvq_decode_plan_info(cfg: Config, num_ctas: int = 0) -> dict:
     v = KvqDecodePlan()
     _check("kvq_decode_plan_info", _lib.kvq_decode_plan_info(ctypes.byref(cfg.c()), num_ctas,
                                                              ctypes.byref(v)))
-    return {n: getattr(v, n) for n, _ in KvqDecodePlan._fields_ if n != "reserved"}
+    return {n: getattr(v, n) for n, _ in KvqDecodePlan._fields_}
 
 
 def kvq_h_scratch_bytes(cfg: Config, max_len: int) -> int:

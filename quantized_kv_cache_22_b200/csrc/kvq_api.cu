@@ -451,6 +451,7 @@ int kvq_decode_plan_info(const kvq_config *cfg, int32_t num_ctas, kvq_decode_pla
     info->stage_bytes = plan.stage_bytes;
     info->smem_bytes = (int32_t)plan.smem_bytes;
     info->threads = plan.tc ? 192 : kDecodeThreads;
+    info->packed_columns = plan.pk ? 1 : 0;
     return KVQ_OK;
 }
 

@@ -70,6 +70,15 @@ void *pick_decode(int dh, int kb, int vb, bool kg, bool vg, int fmt)
     }
 }
 
+// the packed-column instance for G <= 4, or null
+void *pick_decode_pk(int dh, int kb, int vb, bool kg, bool vg, int fmt, int G)
+{
+    if (dh != 128 || G > 4) return nullptr;
+    if (kb == 4) return decode_fn_pk_kb4(vb, kg, vg, fmt);
+    if (kb == 8) return decode_fn_pk_kb8(vb, kg, vg, fmt);
+    return nullptr;
+}
+
 inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
 // The warp-MMA kernel serves every format by default: on the 8K workload it is as
@@ -147,7 +156,8 @@ bool plan_decode(int dh, int kb, int vb, int ngs_k, int ngs_v, int G, int max_sm
     if (!pick_decode(dh, kb, vb, kg, vg, fmt)) return false;
     const uint32_t rk = dh * kb / 8, rv = dh * vb / 8;
     DecodeLaunch L{};
-    L.dh = dh; L.kb = kb; L.vb = vb; L.kg = kg; L.vg = vg; L.fmt = fmt;
+    L.dh = dh; L.kb = kb; L.vb = vb; L.kg = kg; L.vg = vg; L.fmt = fmt; L.G = G;
+    L.pk = pick_decode_pk(dh, kb, vb, kg, vg, fmt, G) != nullptr;
     L.off_v = align_up(T * rk, 1024);
     L.off_sk = L.off_v + align_up(T * rv, 1024);
     L.off_sv = L.off_sk + align_up(T * (kb == 16 ? 0 : ngs_k) * 2, 16);
@@ -236,8 +246,9 @@ cudaError_t prepare_fn(void *fn, size_t smem, int *occupancy, int threads)
 
 static void *plan_fn(const DecodeLaunch &plan)
 {
-    return plan.tc ? decode_tc_fn(plan.kb, plan.vb, plan.kg, plan.G, plan.fmt)
-                   : pick_decode(plan.dh, plan.kb, plan.vb, plan.kg, plan.vg, plan.fmt);
+    if (plan.tc) return decode_tc_fn(plan.kb, plan.vb, plan.kg, plan.G, plan.fmt);
+    if (plan.pk) return pick_decode_pk(plan.dh, plan.kb, plan.vb, plan.kg, plan.vg, plan.fmt, plan.G);
+    return pick_decode(plan.dh, plan.kb, plan.vb, plan.kg, plan.vg, plan.fmt);
 }
 
 cudaError_t decode_occupancy(const DecodeLaunch &plan, int *ctas_per_sm)

@@ -105,7 +105,15 @@ __device__ __forceinline__ uint32_t pack_bytes(int a, int b, int c, int d)
 // FMT: the code format of 8-bit keys and values (KVQ_FMT_*; KB = VB = 8 unless
 // KVQ_FMT_INT): symmetric integer, FP8 e4m3, asymmetric (uint8 codes with a
 // zero-point) or per-tensor (one fixed scale per tensor).
-template <int DH, int KB, int VB, bool KG, bool VG, int FMT>
+// PK ("packed columns", G <= 4 with int8 keys): the score MMA's eight columns carry
+// the hi parts of the four heads and their lo parts, against sub-tile 0's keys with
+// [hi | lo] and sub-tile 1's with [lo | hi]; one shuffle joins hi and lo, after which
+// lanes tig < 2 own sub-tile 0's scores of their heads and lanes tig >= 2 sub-tile
+// 1's.  Half the score MMAs, and no softmax work on padding columns: every lane
+// carries 4 live scores instead of 8 (4 of them padding).  Both sub-tiles' P then
+// share one transposed fragment, masked per sub-tile for the P.V MMAs, whose output
+// columns 0-3 accumulate sub-tile 0 and 4-7 sub-tile 1 (joined at the segment end).
+template <int DH, int KB, int VB, bool KG, bool VG, int FMT, bool PK = false>
 __global__ void __launch_bounds__(NTHR, 2)
     decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const __grid_constant__ DecodeParams p)
@@ -267,6 +275,8 @@ __global__ void __launch_bounds__(NTHR, 2)
 
     // ====================== consumers ======================
     constexpr bool IMMA_K = KB != 16 && !F8;   // else f16 MMA (fp16 keys, or e4m3 converted)
+    static_assert(!PK || (IMMA_K && !ZP), "packed columns need int8 keys without zero-points");
+    constexpr int NU = PK ? 1 : 2;             // score sub-tiles a lane carries
     const int gid = lane >> 2;
     const int tig = lane & 3;
     // fp16 keys keep an f16 MMA; f32 / bf16 queries then use columns 4..7 for
@@ -275,8 +285,11 @@ __global__ void __launch_bounds__(NTHR, 2)
     constexpr bool kgrp = KG;
     constexpr bool vgrp = VG;
     const int colmax = qsplit ? 4 : 8;
-    const bool col_ok0 = (2 * tig) < G && (2 * tig) < colmax;
-    const bool col_ok1 = (2 * tig + 1) < G && (2 * tig + 1) < colmax;
+    // PK: lane tig holds sub-tile tig >> 1's heads 2 (tig & 1) + c; lanes tig < 2 write
+    const bool col_ok0 = PK ? (tig < 2 && 2 * tig < G) : ((2 * tig) < G && (2 * tig) < colmax);
+    const bool col_ok1 = PK ? (tig < 2 && 2 * tig + 1 < G)
+                            : ((2 * tig + 1) < G && (2 * tig + 1) < colmax);
+    const int ul = tig >> 1;                   // PK: the lane's score sub-tile
 
     // sequences with nothing cached get zeros (fused merge only; the merge
     // launch writes them otherwise)
@@ -335,8 +348,10 @@ __global__ void __launch_bounds__(NTHR, 2)
             // q ~ (amax / 127) * (hi + lo / 254) per head, hi, lo in [-127, 127];
             // lane (gid, tig) holds head gid and, for block blk, the 8 elements its
             // key fragments hold: from (blk / KPL) 32 KPL + 8 KPL tig + 8 (blk % KPL)
-            const bool valid = gid < G;
-            const int64_t qbase = ((int64_t)b * p.n_q_heads + (int64_t)kvh * G + gid) * DH;
+            // PK: columns gid and gid + 4 carry the hi / lo parts of head gid & 3
+            const int qhd = PK ? (gid & 3) : gid;
+            const bool valid = qhd < G;
+            const int64_t qbase = ((int64_t)b * p.n_q_heads + (int64_t)kvh * G + qhd) * DH;
             float x[NG][8];
             float amax = 0.f;
 #pragma unroll
@@ -389,6 +404,16 @@ __global__ void __launch_bounds__(NTHR, 2)
                     ql[blk][0] = pack_bytes(lo[0], lo[2], lo[4], lo[6]);
                     ql[blk][1] = pack_bytes(lo[1], lo[3], lo[5], lo[7]);
                 }
+                if constexpr (PK) {
+                    // qh = [hi | lo] (sub-tile 0's B operand), ql = [lo | hi] (sub-tile 1's)
+                    if (gid >= 4) {
+                        const uint32_t t0 = qh[blk][0], t1 = qh[blk][1];
+                        qh[blk][0] = ql[blk][0];
+                        qh[blk][1] = ql[blk][1];
+                        ql[blk][0] = t0;
+                        ql[blk][1] = t1;
+                    }
+                }
             }
             if constexpr (ZP && !KG) {
                 qs_all += __shfl_xor_sync(FULL, qs_all, 1);
@@ -398,8 +423,9 @@ __global__ void __launch_bounds__(NTHR, 2)
             }
             // 4-bit key codes enter the MMA as 16 * code
             const float f = amax * (1.f / (127.f * 254.f)) * p.tau_log2e * (KB == 4 ? 0.0625f : 1.f);
-            sqc[0] = __shfl_sync(FULL, f, (2 * tig) * 4);
-            sqc[1] = __shfl_sync(FULL, f, (2 * tig + 1) * 4);
+            const int hc = PK ? 2 * (tig & 1) : 2 * tig;   // the lane's first head column
+            sqc[0] = __shfl_sync(FULL, f, hc * 4);
+            sqc[1] = __shfl_sync(FULL, f, (hc + 1) * 4);
         } else {
             // B-fragment column n = gid: non-split: head n; split: hi (n<4) / lo (n>=4) of head n&3
             const int head = qsplit ? (gid & 3) : gid;
@@ -541,8 +567,13 @@ __global__ void __launch_bounds__(NTHR, 2)
                                     fa[0] = (w0 << 4) & 0xF0F0F0F0u; fa[1] = (w1 << 4) & 0xF0F0F0F0u;
                                     fa[2] = w0 & 0xF0F0F0F0u;        fa[3] = w1 & 0xF0F0F0F0u;
                                 }
-                                imma_16832<ZP>(ah[u], fa[0], fa[1], fa[2], fa[3], qh[blk][0], qh[blk][1]);
-                                imma_16832<ZP>(al[u], fa[0], fa[1], fa[2], fa[3], ql[blk][0], ql[blk][1]);
+                                if constexpr (PK) {
+                                    imma_16832<ZP>(ah[u], fa[0], fa[1], fa[2], fa[3], u ? ql[blk][0] : qh[blk][0],
+                                                   u ? ql[blk][1] : qh[blk][1]);
+                                } else {
+                                    imma_16832<ZP>(ah[u], fa[0], fa[1], fa[2], fa[3], qh[blk][0], qh[blk][1]);
+                                    imma_16832<ZP>(al[u], fa[0], fa[1], fa[2], fa[3], ql[blk][0], ql[blk][1]);
+                                }
                             }
                         }
                     }
@@ -560,11 +591,29 @@ __global__ void __launch_bounds__(NTHR, 2)
                                   sst + blk_addr<RK, SK>(kofs[1][1], blk), fa[1]);
 #pragma unroll
                     for (int u = 0; u < 2; u++) {
-                        imma_16832<ZP>(ah[u], fa[u][0], fa[u][1], fa[u][2], fa[u][3], qh[blk][0], qh[blk][1]);
-                        imma_16832<ZP>(al[u], fa[u][0], fa[u][1], fa[u][2], fa[u][3], ql[blk][0], ql[blk][1]);
+                        if constexpr (PK) {
+                            imma_16832<ZP>(ah[u], fa[u][0], fa[u][1], fa[u][2], fa[u][3], u ? ql[blk][0] : qh[blk][0],
+                                           u ? ql[blk][1] : qh[blk][1]);
+                        } else {
+                            imma_16832<ZP>(ah[u], fa[u][0], fa[u][1], fa[u][2], fa[u][3], qh[blk][0], qh[blk][1]);
+                            imma_16832<ZP>(al[u], fa[u][0], fa[u][1], fa[u][2], fa[u][3], ql[blk][0], ql[blk][1]);
+                        }
                     }
                 }
                 }
+                if constexpr (PK) {
+                    // lanes tig < 2: own hi of sub-tile 0 (ah[0]), partner's lo (its ah[0]);
+                    // lanes tig >= 2: own hi of sub-tile 1 (ah[1]), partner's lo (its ah[1])
+                    const float2 kk = PT ? make_float2(k_tensor, k_tensor)
+                                         : unpack_half2(lds_u32(sbase, ssk + 2 * (ul ? tAu[1] : tAu[0])));
+#pragma unroll
+                    for (int e = 0; e < 4; e++) {
+                        const int mine = ul ? ah[1][e] : ah[0][e];
+                        const int send = ul ? ah[0][e] : ah[1][e];
+                        const int a = mine * 254 + __shfl_xor_sync(FULL, send, 2);
+                        s2[0][e] = (float)a * (((e < 2) ? kk.x : kk.y) * sqc[e & 1]);
+                    }
+                } else {
 #pragma unroll
                 for (int u = 0; u < 2; u++) {
                     float2 kk;
@@ -589,7 +638,9 @@ __global__ void __launch_bounds__(NTHR, 2)
                         s2[u][e] = (float)a * (ks * sqc[e & 1]);
                     }
                 }
+                }
             } else {
+                float fk[2][4];   // PK: each sub-tile's single (hi | lo) chain, scaled per block
 #pragma unroll
                 for (int u = 0; u < 2; u++) {
                     float v[4] = {0.f, 0.f, 0.f, 0.f};
@@ -626,9 +677,18 @@ __global__ void __launch_bounds__(NTHR, 2)
                         uint32_t fa[4];
                         key_frags(Imm0{}, sst + blk_addr<RK, SK>(kofs[u][0], blk),
                                   sst + blk_addr<RK, SK>(kofs[u][1], blk), fa);
+                        const float k0 = kr0[blk], k1 = kr1[blk];
+                        if constexpr (PK) {
+                            imma_16832<ZP>(ah, fa[0], fa[1], fa[2], fa[3], u ? ql[blk][0] : qh[blk][0],
+                                           u ? ql[blk][1] : qh[blk][1]);
+                            v[0] = fmaf(k0, (float)ah[0], v[0]);
+                            v[1] = fmaf(k0, (float)ah[1], v[1]);
+                            v[2] = fmaf(k1, (float)ah[2], v[2]);
+                            v[3] = fmaf(k1, (float)ah[3], v[3]);
+                            continue;
+                        }
                         imma_16832<ZP>(ah, fa[0], fa[1], fa[2], fa[3], qh[blk][0], qh[blk][1]);
                         imma_16832<ZP>(al, fa[0], fa[1], fa[2], fa[3], ql[blk][0], ql[blk][1]);
-                        const float k0 = kr0[blk], k1 = kr1[blk];
                         if constexpr (ZP) {
                             // minus zero-point x the block's query sum
                             const uint32_t o0 = ssk + 2 * (tA * p.ngs_k + SCV * (blk >> p.kshift));
@@ -648,8 +708,22 @@ __global__ void __launch_bounds__(NTHR, 2)
                         v[2] = fmaf(k1, (float)ah[2], v[2]);
                         v[3] = fmaf(k1, (float)ah[3], v[3]);
                     }
+                    if constexpr (PK) {
 #pragma unroll
-                    for (int e = 0; e < 4; e++) s2[u][e] = v[e] * sqc[e & 1];
+                        for (int e = 0; e < 4; e++) fk[u][e] = v[e];
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 4; e++) s2[u][e] = v[e] * sqc[e & 1];
+                    }
+                }
+                if constexpr (PK) {
+                    // join hi (own chain) and lo (partner's) as for per-head key scales
+#pragma unroll
+                    for (int e = 0; e < 4; e++) {
+                        const float mine = ul ? fk[1][e] : fk[0][e];
+                        const float send = ul ? fk[0][e] : fk[1][e];
+                        s2[0][e] = fmaf(254.f, mine, __shfl_xor_sync(FULL, send, 2)) * sqc[e & 1];
+                    }
                 }
             }
         } else if constexpr (F8) {
@@ -760,8 +834,14 @@ __global__ void __launch_bounds__(NTHR, 2)
                     s2[u][e] = v;
                 }
         }
+        if constexpr (PK) {
+            // from here on a lane's score rows are those of its own sub-tile
+            tAu[0] = ul ? tAu[1] : tAu[0];
+            vt[0][0] = ul ? vt[1][0] : vt[0][0];
+            vt[0][1] = ul ? vt[1][1] : vt[0][1];
+        }
 #pragma unroll
-        for (int u = 0; u < 2; u++) {
+        for (int u = 0; u < NU; u++) {
             // Padding columns (heads >= G, or the residual columns of a split
             // query) carry finite scores from zero query columns; their outputs
             // are never written, so only tokens past the length are masked.
@@ -778,7 +858,7 @@ __global__ void __launch_bounds__(NTHR, 2)
         // tw + vB; tw + vA + 1, tw + vB + 1), zero past the length (stale scales)
         uint32_t za[2][NVG][2];
 #pragma unroll
-        for (int u = 0; u < 2; u++) {
+        for (int u = 0; u < NU; u++) {
             const int tA = tAu[u];
             constexpr int SCV = scale_vals(FMT);
             if constexpr (VB == 16) {
@@ -845,7 +925,7 @@ __global__ void __launch_bounds__(NTHR, 2)
         {
             float loc0 = -INFINITY, loc1 = -INFINITY;
 #pragma unroll
-            for (int u = 0; u < 2; u++) {
+            for (int u = 0; u < NU; u++) {
                 loc0 = fmaxf(loc0, fmaxf(s2[u][0] + lsv[u][0], s2[u][2] + lsv[u][1]));
                 loc1 = fmaxf(loc1, fmaxf(s2[u][1] + lsv[u][0], s2[u][3] + lsv[u][1]));
             }
@@ -882,6 +962,28 @@ __global__ void __launch_bounds__(NTHR, 2)
         // x0 = rows 0..7 of the score tile (tokens tw + row_token(r)), x1 = rows
         // 8..15; their 8x8 transposes are the B fragments of the P.V MMA.
         uint32_t pb[2][NVG][2];
+        if constexpr (PK) {
+            // one transposed fragment holds both sub-tiles' P: columns (= gid after the
+            // transpose) 0-3 sub-tile 0's heads, 4-7 sub-tile 1's; each sub-tile's P.V
+            // MMA gets it with the other's columns zeroed
+            float pr[4];
+#pragma unroll
+            for (int e = 0; e < 4; e++)
+                pr[e] = (s2[0][e] == -INFINITY) ? 0.f : fast_exp2(s2[0][e] - m_run[e & 1]);
+            l_run[0] += pr[0] + pr[2];
+            l_run[1] += pr[1] + pr[3];
+            const uint32_t keep0 = gid < 4 ? 0xFFFFFFFFu : 0u;
+#pragma unroll
+            for (int g = 0; g < NVG; g++) {
+                const uint32_t t0 = movmatrix_trans(pack_half2(pr[0] * sv[0][0][g], pr[1] * sv[0][0][g]));
+                const uint32_t t1 = movmatrix_trans(pack_half2(pr[2] * sv[0][1][g], pr[3] * sv[0][1][g]));
+                if constexpr (VBIAS) mma_16816(psum[g], ONE2, ONE2, ONE2, ONE2, t0, t1);
+                pb[0][g][0] = t0 & keep0;
+                pb[0][g][1] = t1 & keep0;
+                pb[1][g][0] = t0 & ~keep0;
+                pb[1][g][1] = t1 & ~keep0;
+            }
+        } else {
 #pragma unroll
         for (int u = 0; u < 2; u++) {
             float pr[4];
@@ -903,6 +1005,7 @@ __global__ void __launch_bounds__(NTHR, 2)
                 else if constexpr (VBIAS)
                     mma_16816(psum[g], ONE2, ONE2, ONE2, ONE2, pb[u][g][0], pb[u][g][1]);
             }
+        }
         }
 
         // ---------------- phase 5: O^T += V^T P for both sub-tiles ----------------
@@ -1127,6 +1230,38 @@ __global__ void __launch_bounds__(NTHR, 2)
                 aborted = true;
                 break;
             }
+            float mw[2] = {m_run[0], m_run[1]};
+            if constexpr (PK) {
+                // join the two sub-tiles' partials of each head (lanes tig and tig ^ 2):
+                // remove the code bias from each, then weight by 2^(m - max)
+                float es[2], eo[2];
+#pragma unroll
+                for (int c = 0; c < 2; c++) {
+                    const float mo = __shfl_xor_sync(FULL, m_run[c], 2);
+                    const float lo_ = __shfl_xor_sync(FULL, lt[c], 2);
+                    const float M = fmaxf(m_run[c], mo);
+                    es[c] = (m_run[c] == -INFINITY) ? 0.f : exp2f(m_run[c] - M);
+                    eo[c] = (mo == -INFINITY) ? 0.f : exp2f(mo - M);
+                    lt[c] = lt[c] * es[c] + lo_ * eo[c];
+                    mw[c] = M;
+                }
+#pragma unroll
+                for (int mt = 0; mt < 2 * NG; mt++)
+#pragma unroll
+                    for (int c = 0; c < 2; c++) {
+                        const float ps = psum[VG ? (mt >> 1) : 0][c];
+                        float lo = o_acc[mt][c], hi = o_acc[mt][2 + c];
+                        if constexpr (VB == 4) {
+                            lo -= 1032.f * ps;
+                            hi = (hi - 1152.f * ps) * 0.0625f;
+                        } else {
+                            lo -= BIAS_V * ps;
+                            hi -= BIAS_V * ps;
+                        }
+                        o_acc[mt][c] = lo * es[c] + __shfl_xor_sync(FULL, lo, 2) * eo[c];
+                        o_acc[mt][2 + c] = hi * es[c] + __shfl_xor_sync(FULL, hi, 2) * eo[c];
+                    }
+            }
             // this warp's partial into mbuf[warp]: [G][DH + 4] floats, o then (m, l)
             float *mine = mbuf + (size_t)warp * G * CS;
 #pragma unroll
@@ -1146,7 +1281,9 @@ __global__ void __launch_bounds__(NTHR, 2)
                             const int d = VWIDE ? 64 * (mt >> 2) + 8 * gid + 2 * (mt & 3)
                                                 : 32 * blk + 4 * gid + 2 * h;
                             float lo = o_acc[mt][c], hi = o_acc[mt][2 + c];
-                            if constexpr (VB == 4) {
+                            if constexpr (PK) {
+                                // joined and unbiased above
+                            } else if constexpr (VB == 4) {
                                 lo -= 1032.f * ps;                // even nibble: 1032 + code
                                 hi = (hi - 1152.f * ps) * 0.0625f;  // odd nibble: 1152 + 16 code
                             } else {
@@ -1156,7 +1293,7 @@ __global__ void __launch_bounds__(NTHR, 2)
                             *reinterpret_cast<float2 *>(oc + d) = make_float2(lo, hi);
                         }
                     }
-                    if (gid == 0) *reinterpret_cast<float2 *>(oc + DH) = make_float2(m_run[c], lt[c]);
+                    if (gid == 0) *reinterpret_cast<float2 *>(oc + DH) = make_float2(mw[c], lt[c]);
                 }
             }
             if (warp == 0 && lane == 0) {

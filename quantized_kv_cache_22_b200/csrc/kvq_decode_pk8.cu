@@ -1,0 +1,35 @@
+// kvq_decode_pk8.cu -- decode kernel instances with packed score columns (G <= 4,
+// head_dim 128) for 8-bit keys: symmetric INT4 / INT8 values, and per-tensor INT8
+#include "kvq_decode_kernel.cuh"
+
+namespace kvq {
+namespace {
+
+template <int VB, bool KG, bool VG, int FMT>
+void *fn()
+{
+    return reinterpret_cast<void *>(&decode_kernel<128, 8, VB, KG, VG, FMT, true>);
+}
+
+template <int VB>
+void *by_kg(bool kg, bool vg)
+{
+    if (kg) return vg ? fn<VB, true, true, KVQ_FMT_INT>() : fn<VB, true, false, KVQ_FMT_INT>();
+    return vg ? fn<VB, false, true, KVQ_FMT_INT>() : fn<VB, false, false, KVQ_FMT_INT>();
+}
+
+}  // namespace
+
+void *decode_fn_pk_kb8(int vb, bool kg, bool vg, int fmt)
+{
+    if (fmt == KVQ_FMT_TENSOR)
+        return (vb == 8 && !kg && !vg) ? fn<8, false, false, KVQ_FMT_TENSOR>() : nullptr;
+    if (fmt != KVQ_FMT_INT) return nullptr;
+    switch (vb) {
+    case 4: return by_kg<4>(kg, vg);
+    case 8: return by_kg<8>(kg, vg);
+    default: return nullptr;
+    }
+}
+
+}  // namespace kvq

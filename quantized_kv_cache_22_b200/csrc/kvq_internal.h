@@ -140,6 +140,7 @@ struct DecodeLaunch {
     bool kg, vg;              // grouped key / value scales
     int fmt;                  // KVQ_FMT_* of the 8-bit codes
     bool tc;                  // the tensor-core kernel (kvq_decode_tc.cu)
+    bool pk;                  // warp-MMA kernel with packed score columns (G <= 4)
     int G;                    // query heads per KV head (tensor-core kernel instance)
     int per_sm;               // CTAs per SM the plan's shared memory is sized for
     size_t smem_bytes;
@@ -156,6 +157,10 @@ void *decode_fn_kb8(int dh, int vb, bool kg, bool vg);
 void *decode_fn_kb16(int dh, int vb, bool kg, bool vg);
 // e4m3, asymmetric and per-tensor 8-bit keys and values (kvq_decode_fmt.cu)
 void *decode_fn_fmt(int dh, int fmt, bool kg, bool vg);
+// packed score columns, G <= 4 at head_dim 128 (kvq_decode_pk4/pk8.cu): INT4 / INT8
+// keys and values (fmt KVQ_FMT_INT), or per-tensor INT8
+void *decode_fn_pk_kb4(int vb, bool kg, bool vg, int fmt);
+void *decode_fn_pk_kb8(int vb, bool kg, bool vg, int fmt);
 // the tensor-core kernel (head_dim 128; value scales per (token, head), key scales
 // per (token, head) or per 32/64-element group; or per-tensor INT8): INT8 / INT4 keys
 // and values with G query heads per KV head, or null (kvq_decode_tc.cu); and the

@@ -287,6 +287,14 @@ def test_decode_plan_info_without_device(monkeypatch):
         # the plan's shared memory leaves room for that many CTAs on a 228 KB SM
         assert per_sm * (info["smem_bytes"] + 1024 + 128) <= 233472
     assert kvq.kvq_decode_plan_info(cfg(4, 4, vg=64, dh=64), 10)["ctas_per_sm_planned"] == 2
+    # packed score columns for G <= 4 at head_dim 128 with INT4 / INT8 keys
+    assert kvq.kvq_decode_plan_info(cfg(8, 4), 296)["packed_columns"] == 1
+    assert kvq.kvq_decode_plan_info(cfg(4, 8, vg=32), 296)["packed_columns"] == 1
+    assert kvq.kvq_decode_plan_info(cfg(16, 16), 296)["packed_columns"] == 0
+    assert kvq.kvq_decode_plan_info(cfg(4, 4, vg=64, dh=64), 10)["packed_columns"] == 0
+    g8 = Config(batch=2, capacity=256, n_q_heads=16, n_kv_heads=2, head_dim=128, k_bits=8, v_bits=8,
+                k_group=128, v_group=128)
+    assert kvq.kvq_decode_plan_info(g8, 10)["packed_columns"] == 0
     monkeypatch.setenv("KVQ_DECODE_TC", "1")
     for kb, vb in ((8, 8), (8, 4), (4, 4), (4, 8)):
         info = kvq.kvq_decode_plan_info(cfg(kb, vb), 296)
