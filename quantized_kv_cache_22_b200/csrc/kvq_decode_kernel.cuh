@@ -133,6 +133,9 @@ __global__ void __launch_bounds__(NTHR, 2)
     // block, so a lane then reads 4 elements per block.  Rows of 32 bytes (Dh 64
     // at 4 bits) keep the block mapping, which stays free of bank conflicts.
     constexpr bool VWIDE = !VG && RV >= 64 && !F8;
+    // 4-bit values, wide: one ldmatrix.trans per sub-tile and 64-element half gives
+    // each lane the (k-slot pair, 4 dims) words of four 8-token x 32-dim matrices
+    constexpr bool VLDSM = VWIDE && VB == 4;
     constexpr int VL = VWIDE ? 2 * SV / 8 : SV / 8;   // value bytes per lane per row and load
     // Key fragments: with one key scale per (token, head), int8 keys are read 16
     // bytes per lane and row ("wide": 2 blocks of 32 elements per load at 8
@@ -317,7 +320,12 @@ __global__ void __launch_bounds__(NTHR, 2)
         const int tw = warp * 32 + u * 16;
         kofs[u][0] = sw_off<RK>(tw + rt, tig * KLW);
         kofs[u][1] = sw_off<RK>(tw + rt + 1, tig * KLW);
-        vofs[u][0] = p.off_v + sw_off<RV>(tw + vA, gid * VL);
+        // ldmatrix rows: lane l gives row l % 8 of matrix l / 8 = (token half, 32-dim
+        // window): k-slot l % 8 (+ 8 for the second token half) of the P.V MMA
+        vofs[u][0] = VLDSM
+                         ? p.off_v + sw_off<RV>(tw + row_token<KWIDE>(lane & 7) + ((lane >> 3) & 1),
+                                                16 * (lane >> 4))
+                         : p.off_v + sw_off<RV>(tw + vA, gid * VL);
         vofs[u][1] = p.off_v + sw_off<RV>(tw + vB, gid * VL);
         vofs[u][2] = p.off_v + sw_off<RV>(tw + vA + 1, gid * VL);
         vofs[u][3] = p.off_v + sw_off<RV>(tw + vB + 1, gid * VL);
@@ -1060,6 +1068,28 @@ __global__ void __launch_bounds__(NTHR, 2)
                             const uint32_t a3 = and_xor(yCE >> 8, 0x00FF00FFu, VX);
                             mma_16816(o_acc[4 * sb + j], a0, a1, a2, a3, b0, b1);
                         }
+                    } else if constexpr (VLDSM) {
+                        // y[2wi + h]: token half h, 32-dim window wi; per lane the 4 dims
+                        // 64sb + 32wi + 4gid .. + 3 of its k-slot pair.  m-tile 4sb + 2wi + q
+                        // takes dims 4gid + 2q (rows gid: 1032 + code) and 4gid + 2q + 1
+                        // (rows gid + 8: 1152 + 16 code)
+                        uint32_t y[4];
+                        if (u == 0)
+                            ldsm_x4_trans<0>(va[0][0], y);
+                        else
+                            ldsm_x4_trans<ImmV::value>(va[1][0], y);
+#pragma unroll
+                        for (int wi = 0; wi < 2; wi++)
+#pragma unroll
+                            for (int q = 0; q < 2; q++) {
+                                const uint32_t x0 = q ? y[2 * wi] >> 8 : y[2 * wi];
+                                const uint32_t x1 = q ? y[2 * wi + 1] >> 8 : y[2 * wi + 1];
+                                const uint32_t a0 = and_xor(x0, 0x000F000Fu, 0x64086408u);
+                                const uint32_t a1 = and_xor(x0, 0x00F000F0u, 0x64806480u);
+                                const uint32_t a2 = and_xor(x1, 0x000F000Fu, 0x64086408u);
+                                const uint32_t a3 = and_xor(x1, 0x00F000F0u, 0x64806480u);
+                                mma_16816(o_acc[4 * sb + 2 * wi + q], a0, a1, a2, a3, b0, b1);
+                            }
                     } else if constexpr (VB == 4) {
                         uint32_t w[4];
 #pragma unroll
@@ -1274,12 +1304,14 @@ __global__ void __launch_bounds__(NTHR, 2)
                         const float ps = psum[VG ? blk : 0][c];
 #pragma unroll
                         for (int h = 0; h < 2; h++) {
-                            // wide: m-tile 4sb + j, row gid <-> d = 64sb + 8gid + 2j;
+                            // 4-bit wide (ldmatrix): m-tile 4sb + 2wi + q, row gid <-> d =
+                            // 64sb + 32wi + 4gid + 2q; wide: m-tile 4sb + j, row gid <-> d = 64sb + 8gid + 2j;
                             // block mapping: m-tile 2blk + h, row gid <-> d = 32blk + 4gid + 2h;
                             // row gid + 8 <-> d + 1
                             const int mt = 2 * blk + h;
-                            const int d = VWIDE ? 64 * (mt >> 2) + 8 * gid + 2 * (mt & 3)
-                                                : 32 * blk + 4 * gid + 2 * h;
+                            const int d = VLDSM    ? 64 * (mt >> 2) + 32 * ((mt >> 1) & 1) + 4 * gid + 2 * (mt & 1)
+                                        : VWIDE  ? 64 * (mt >> 2) + 8 * gid + 2 * (mt & 3)
+                                                 : 32 * blk + 4 * gid + 2 * h;
                             float lo = o_acc[mt][c], hi = o_acc[mt][2 + c];
                             if constexpr (PK) {
                                 // joined and unbiased above
