@@ -381,7 +381,9 @@ KVQ_API int kvq_h_decode_fused(const kvq_config *cfg, const kvq_layer *layer, co
  * qa is split per (head, scale group) into two int8 parts for the int8
  * tensor-core scores (relative error below 2^-15 of the group's largest
  * element) and p * scale enters the p . h^ product in fp16; everything else
- * accumulates in fp32.  An empty sequence gets zeros.
+ * accumulates in fp32.  The token splits of sum_t p_t h^_t are added in L2
+ * (fp32 reductions), so the last bits of a result may differ between calls.
+ * An empty sequence gets zeros.
  *   h_bits 4 or 8; Hkv*Dh = D, D a multiple of 256 and at most 3584, Dh 64 or
  *   128; Hq <= 32 (smaller limits where the score tile's shared memory runs out).
  *   w_kv     device bf16 [2*Hkv*Dh][D] (as kvq_decode_attn)

@@ -241,6 +241,13 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x)
     return y;
 }
 
+// Ask for `bytes` (a multiple of 16, at a 16-byte aligned address) of global memory
+// to be brought into L2 by the copy engine; nothing is returned or waited for.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *p, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // Order this thread's earlier generic-proxy global writes before later
 // async-proxy (TMA, bulk copy) accesses.
 __device__ __forceinline__ void fence_proxy_async_global()

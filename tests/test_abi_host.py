@@ -231,9 +231,9 @@ def test_absorbed_scratch_bytes_and_validation():
     cfg = Config(batch=8, capacity=1024, mode=kvq.KVQ_MODE_H, d_model=2048, h_bits=4, h_groups=16,
                  n_q_heads=16, n_kv_heads=16, head_dim=128)
     # q fragments B*(D/32)*NT*512 + factors B*ng*NT*8*4 + scores B*Hq*capP*4 + tile
-    # statistics B*Hq*(capP/64)*8 + partial ob (4 splits of 256 tokens) 4*B*Hq*D*4
+    # statistics B*Hq*(capP/64)*8 + ob B*Hq*D*4 (the token splits add into one)
     want = (8 * 64 * 2 * 512 + 8 * 16 * 16 * 4 + 8 * 16 * 1024 * 4 + 8 * 16 * 16 * 8 +
-            4 * 8 * 16 * 2048 * 4)
+            8 * 16 * 2048 * 4)
     assert kvq.kvq_h_absorbed_scratch_bytes(cfg, 1024) == want
     assert kvq.kvq_h_absorbed_scratch_bytes(cfg, 1000) == want
     for over, st in (({"h_bits": 16, "h_groups": 0}, -2), ({"n_q_heads": 64}, -2),
