@@ -278,7 +278,10 @@ __global__ void __launch_bounds__(NTHR, 2)
 
     // ====================== consumers ======================
     constexpr bool IMMA_K = KB != 16 && !F8;   // else f16 MMA (fp16 keys, or e4m3 converted)
-    static_assert(!PK || (IMMA_K && !ZP), "packed columns need int8 keys without zero-points");
+    // packed columns: int8 keys without zero-points, or e4m3 keys with one scale per
+    // (token, head), whose f16 score MMA then always takes the fp16 query and its
+    // residual (zero for fp16 queries) as the hi / lo parts
+    static_assert(!PK || (IMMA_K && !ZP) || (F8 && !KG), "no packed columns for this format");
     constexpr int NU = PK ? 1 : 2;             // score sub-tiles a lane carries
     const int gid = lane >> 2;
     const int tig = lane & 3;
@@ -345,6 +348,7 @@ __global__ void __launch_bounds__(NTHR, 2)
     // 2tig+1) and per 32-element block when the key scales are grouped
     int zq[KG ? NG : 1][2];
     uint32_t qb[NG][2][2];              // fp16 query B-fragments (fp16 keys)
+    uint32_t qb2[PK && F8 ? NG : 1][2][2];   // PK e4m3: the [lo | hi] fragments of sub-tile 1
     float m_run[2], l_run[2];
     float psum[NVG][4];                 // sum of fp16 p*s_V per value group (cols in [0], [1])
     float o_acc[2 * NG][4];             // O^T fragments, m-tile = 2*blk + h
@@ -435,9 +439,10 @@ __global__ void __launch_bounds__(NTHR, 2)
             sqc[0] = __shfl_sync(FULL, f, hc * 4);
             sqc[1] = __shfl_sync(FULL, f, (hc + 1) * 4);
         } else {
-            // B-fragment column n = gid: non-split: head n; split: hi (n<4) / lo (n>=4) of head n&3
-            const int head = qsplit ? (gid & 3) : gid;
-            const bool lo_part = qsplit && gid >= 4;
+            // B-fragment column n = gid: non-split: head n; split (and PK): hi (n<4) / lo
+            // (n>=4) of head n&3; PK's second set qb2 swaps hi and lo
+            const int head = (qsplit || PK) ? (gid & 3) : gid;
+            const bool lo_part = (qsplit || PK) && gid >= 4;
             const bool valid = head < G;
             const int64_t qbase = ((int64_t)b * p.n_q_heads + (int64_t)kvh * G + head) * DH;
 #pragma unroll
@@ -446,18 +451,26 @@ __global__ void __launch_bounds__(NTHR, 2)
                 for (int hs = 0; hs < 2; hs++) {
                     __half hv[4];
 #pragma unroll
+                    __half hw[4];   // the other part (PK e4m3)
                     for (int j = 0; j < 4; j++) {
                         // k-slots 2tig, 2tig+1, 2tig+8, 2tig+9 <-> elements 8tig + 4hs + j
                         const int d = 32 * blk + 8 * tig + 4 * hs + j;
                         const float xq = valid ? load_qf(p.q, p.q_dtype, qbase + d) : 0.f;
-                        __half h = __float2half_rn(xq);
-                        if (lo_part) h = __float2half_rn(xq - __half2float(h));
-                        hv[j] = h;
+                        const __half hh = __float2half_rn(xq);
+                        const __half hl = __float2half_rn(xq - __half2float(hh));
+                        hv[j] = lo_part ? hl : hh;
+                        hw[j] = lo_part ? hh : hl;
                     }
                     __half2 b0 = __halves2half2(hv[0], hv[1]);
                     __half2 b1 = __halves2half2(hv[2], hv[3]);
                     qb[blk][hs][0] = *reinterpret_cast<uint32_t *>(&b0);
                     qb[blk][hs][1] = *reinterpret_cast<uint32_t *>(&b1);
+                    if constexpr (PK && F8) {
+                        __half2 c0 = __halves2half2(hw[0], hw[1]);
+                        __half2 c1 = __halves2half2(hw[2], hw[3]);
+                        qb2[blk][hs][0] = *reinterpret_cast<uint32_t *>(&c0);
+                        qb2[blk][hs][1] = *reinterpret_cast<uint32_t *>(&c1);
+                    }
                 }
         }
 #pragma unroll
@@ -764,9 +777,26 @@ __global__ void __launch_bounds__(NTHR, 2)
                         for (int hs = 0; hs < 2; hs++) {
                             uint32_t fa[4];
                             f8_frags(r[u][0], r[u][1], hs, fa);
-                            mma_16816(acc[u][hs], fa[0], fa[1], fa[2], fa[3], qb[blk][hs][0], qb[blk][hs][1]);
+                            if constexpr (PK)
+                                mma_16816(acc[u][hs], fa[0], fa[1], fa[2], fa[3],
+                                          u ? qb2[PK && F8 ? blk : 0][hs][0] : qb[blk][hs][0],
+                                          u ? qb2[PK && F8 ? blk : 0][hs][1] : qb[blk][hs][1]);
+                            else
+                                mma_16816(acc[u][hs], fa[0], fa[1], fa[2], fa[3], qb[blk][hs][0], qb[blk][hs][1]);
                         }
                 }
+                if constexpr (PK) {
+                    // as for int8 keys: the lane's own chain holds its heads' hi part, the
+                    // partner's (lane ^ 2) the lo part of the same heads
+                    const float2 kk = unpack_half2(lds_u32(sbase, ssk + 2 * (ul ? tAu[1] : tAu[0])));
+#pragma unroll
+                    for (int e = 0; e < 4; e++) {
+                        const float v0 = acc[0][0][e] + acc[0][1][e], v1 = acc[1][0][e] + acc[1][1][e];
+                        const float mine = ul ? v1 : v0, send = ul ? v0 : v1;
+                        s2[0][e] = (mine + __shfl_xor_sync(FULL, send, 2)) *
+                                   (((e < 2) ? kk.x : kk.y) * p.tau_log2e);
+                    }
+                } else {
 #pragma unroll
                 for (int u = 0; u < 2; u++) {
                     const float2 kk = unpack_half2(lds_u32(sbase, ssk + 2 * tAu[u]));
@@ -776,6 +806,7 @@ __global__ void __launch_bounds__(NTHR, 2)
                         if (qsplit) v += __shfl_xor_sync(FULL, v, 2);
                         s2[u][e] = v;
                     }
+                }
                 }
             } else {
 #pragma unroll
