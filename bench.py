@@ -1038,6 +1038,7 @@ def run_gpu(args):
             "decode_kernel_ms": dec_ms,
             "decode_kernel_gbs": kv_bytes_layer / (dec_ms * 1e-3) / 1e9,
             "clocks": clocks,
+            "plan": kvq.kvq_decode_plan_info(st["cfg"], 0),
         }
         # per decode launch inside the step (the step is only these launches)
         results[name]["in_step_gbs"] = kv_bytes_layer / (ms / w.n_layers * 1e-3) / 1e9
@@ -1093,7 +1094,8 @@ def run_gpu(args):
         "data": "synthetic",
         "config": bench_config(w, head, world),
         "execution": {"graph": "one CUDA graph per step",
-                      "launch": "programmatic dependent launch between layers"},
+                      "launch": "programmatic dependent launch between layers",
+                      "decode_plan": r["plan"]},
         "pct_hbm_measured": round(r["pct_hbm_measured"], 2),
         "pct_hbm_nominal_8tbs": round(r["pct_hbm_nominal_8tbs"], 2),
         "roofline": {"bound": "hbm", "kernel": "decode_kernel (append + split-KV attention + merge)",
