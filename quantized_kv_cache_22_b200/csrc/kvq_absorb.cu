@@ -593,6 +593,152 @@ __global__ void __launch_bounds__(128) absorb_pv_kernel(AbsorbParams p)
     }
 }
 
+
+// ---------------------------------------------------------------- p . h^, group 128
+// The same product for 128-element scale groups, without the shared-memory pass of
+// converted codes and without a CTA barrier per chunk: each warp owns 32 columns of
+// the group and walks the block's tokens on its own.  P~[head][t] = 2^(s_t - M) / L *
+// s_h(t, g) is computed once per staged block of 256 tokens into shared memory (fp16),
+// whence the warps read their A fragments; their B fragments come from
+// ldmatrix.trans of the raw codes (token rows
+// padded by 16 bytes, so that the 8 rows of a matrix fall in 8 different bank
+// groups) and become exact fp16 integers in registers: per 16-bit word of a token
+// pair, a 4-bit code in the mantissa of 1024 (sign flipped: 1032 + c) minus 1032,
+// an 8-bit code as 1152 + c minus 1152.
+template <int BITS, int MT>
+__global__ void __launch_bounds__(128) absorb_pv128_kernel(AbsorbParams p)
+{
+    constexpr int TB = 256;                        // tokens staged per block
+    constexpr int cb = 128 * BITS / 8;             // code bytes of the group per token
+    constexpr int RS = cb + 16;                    // padded row stride of the staged codes
+    constexpr int PS = TB + 8;                     // padded row stride of P~ (halves)
+    extern __shared__ __align__(16) uint8_t sm[];
+    float *ss = reinterpret_cast<float *>(sm);                       // [MT*16][TB]
+    uint8_t *sc = sm + (size_t)MT * 16 * TB * 4;                     // [TB][RS]
+    __half *pt = reinterpret_cast<__half *>(sc + (size_t)TB * RS);   // [MT*16][PS]
+    __shared__ float hm[MT * 16], hinv[MT * 16];
+    __shared__ float sv[TB];
+    const int g = blockIdx.x, b = blockIdx.y, split = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gid = lane >> 2, tig = lane & 3;
+    grid_dependency_wait();
+    const int len = seq_len(p, b);
+    const int t_begin = split * p.split;
+    if (t_begin >= len) return;
+    const int t_end = min(len, t_begin + p.split);
+    if (tid < MT * 16) {
+        float M = -INFINITY, L = 0.f;
+        if (tid < p.Hq) {
+            const float2 *st = p.stats + ((int64_t)b * p.Hq + tid) * p.ntile;
+            const int nt = (len + p.T2 - 1) / p.T2;
+#pragma unroll 8
+            for (int k = 0; k < nt; k++) M = fmaxf(M, st[k].x);
+#pragma unroll 8
+            for (int k = 0; k < nt; k++) L += st[k].y * exp2f(st[k].x - M);
+        }
+        hm[tid] = M;
+        hinv[tid] = L > 0.f ? 1.f / L : 0.f;
+    }
+    grid_launch_dependents();
+    float acc[MT][4][4];
+#pragma unroll
+    for (int mt = 0; mt < MT; mt++)
+#pragma unroll
+        for (int n = 0; n < 4; n++) acc[mt][n][0] = acc[mt][n][1] = acc[mt][n][2] = acc[mt][n][3] = 0.f;
+    const int rowb = p.D * BITS / 8;
+    const uint32_t ssb = smem_u32(ss), scb = smem_u32(sc);
+    // ldmatrix rows of this lane: matrix l / 8 = (k16 step l / 16, token half (l / 8) % 2)
+    const int lrow = 16 * (lane >> 4) + 8 * ((lane >> 3) & 1) + (lane & 7);
+    for (int tb0 = t_begin; tb0 < t_end; tb0 += TB) {
+        const int nb = min(TB, t_end - tb0);
+        __syncthreads();                           // the previous block is consumed
+#pragma unroll
+        for (int r = 0; r < MT * 16 * (TB / 4) / 128; r++) {
+            const int k = tid + 128 * r, h = k / (TB / 4), t4 = 4 * (k % (TB / 4));
+            if (h < p.Hq && t4 < nb)
+                cp_async16(ssb + (h * TB + t4) * 4, p.p + ((int64_t)b * p.Hq + h) * p.capP + tb0 + t4);
+        }
+        constexpr int c16 = cb / 16;
+#pragma unroll
+        for (int r = 0; r < TB * c16 / 128; r++) {
+            const int k = tid + 128 * r, t = k / c16, c = k % c16;
+            if (t < nb)
+                cp_async16(scb + t * RS + 16 * c, p.h_codes + ((int64_t)b * p.cap + tb0 + t) * rowb + g * cb + 16 * c);
+        }
+#pragma unroll
+        for (int r = 0; r < TB / 128; r++) {
+            const int t = tid + 128 * r;
+            sv[t] = t < nb ? __half2float(p.h_scales[((int64_t)b * p.cap + tb0 + t) * p.ng + g]) : 0.f;
+        }
+        cp_async_wait_all();
+        __syncthreads();
+        for (int k = tid; k < MT * 16 * TB / 2; k += 128) {
+            const int h = k / (TB / 2), t = 2 * (k % (TB / 2));
+            float v0 = 0.f, v1 = 0.f;
+            if (h < p.Hq) {
+                const float f = hinv[h], m = hm[h];
+                if (t < nb) v0 = exp2f(ss[h * TB + t] - m) * f * sv[t];
+                if (t + 1 < nb) v1 = exp2f(ss[h * TB + t + 1] - m) * f * sv[t + 1];
+            }
+            *reinterpret_cast<uint32_t *>(pt + h * PS + t) = pack_half2(v0, v1);
+        }
+        __syncthreads();
+        const uint32_t ptb = smem_u32(pt);
+        for (int c0 = 0; c0 < nb; c0 += 32) {
+            // B: y[m] = token pair (2tig, 2tig+1) of matrix m, 16-bit word gid of its 16 bytes
+            uint32_t y[BITS == 4 ? 1 : 2][4];
+#pragma unroll
+            for (int sg = 0; sg < (BITS == 4 ? 1 : 2); sg++)
+                ldsm_x4_trans<0>(scb + (c0 + lrow) * RS + (BITS == 4 ? 16 * warp : 32 * warp + 16 * sg), y[sg]);
+#pragma unroll
+            for (int ks = 0; ks < 2; ks++) {
+                // A: P~ of heads 16mt + gid (+8), tokens c0 + 16ks + 2tig (+1), (+8)
+                uint32_t a[MT][4];
+#pragma unroll
+                for (int mt = 0; mt < MT; mt++)
+#pragma unroll
+                    for (int q = 0; q < 4; q++) {
+                        const int h = 16 * mt + gid + 8 * (q & 1);
+                        const int t = c0 + 16 * ks + 2 * tig + 8 * (q >> 1);
+                        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a[mt][q]) : "r"(ptb + (h * PS + t) * 2));
+                    }
+#pragma unroll
+                for (int n = 0; n < 4; n++) {
+                    uint32_t b0, b1;
+                    if constexpr (BITS == 4) {
+                        // n-tile n: nibble n of each word (columns 4 gid + n)
+                        const uint32_t w0 = (y[0][2 * ks] ^ 0x88888888u) >> (4 * n);
+                        const uint32_t w1 = (y[0][2 * ks + 1] ^ 0x88888888u) >> (4 * n);
+                        b0 = hsub2_u32((w0 & 0x000F000Fu) | 0x64006400u, 0x64086408u);
+                        b1 = hsub2_u32((w1 & 0x000F000Fu) | 0x64006400u, 0x64086408u);
+                    } else {
+                        // n-tile n: piece n / 2, byte n % 2 of each word (columns 2 gid + n % 2)
+                        const uint32_t w0 = (y[n >> 1][2 * ks] ^ 0x80808080u) >> (8 * (n & 1));
+                        const uint32_t w1 = (y[n >> 1][2 * ks + 1] ^ 0x80808080u) >> (8 * (n & 1));
+                        b0 = hsub2_u32((w0 & 0x00FF00FFu) | 0x64006400u, 0x64806480u);
+                        b1 = hsub2_u32((w1 & 0x00FF00FFu) | 0x64006400u, 0x64806480u);
+                    }
+#pragma unroll
+                    for (int mt = 0; mt < MT; mt++)
+                        mma_16816(acc[mt][n], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b0, b1);
+                }
+            }
+        }
+    }
+    // accumulator column 2tig + e of n-tile n: 4-bit, column 4 (2tig + e) + n of the warp's
+    // 32; 8-bit, column 16 (n / 2) + 2 (2tig + e) + n % 2
+    float *ob = p.obp + (int64_t)b * p.Hq * p.D + g * 128 + 32 * warp;
+#pragma unroll
+    for (int mt = 0; mt < MT; mt++)
+#pragma unroll
+        for (int n = 0; n < 4; n++)
+#pragma unroll
+            for (int e = 0; e < 4; e++) {
+                const int h = 16 * mt + gid + 8 * (e >> 1), col = 2 * tig + (e & 1);
+                const int d = BITS == 4 ? 4 * col + n : 16 * (n >> 1) + 2 * col + (n & 1);
+                if (h < p.Hq) atomicAdd(&ob[(int64_t)h * p.D + d], acc[mt][n][e]);
+            }
+}
+
 // ---------------------------------------------------------------- W_v . ob
 // Grid (Hkv, Dh / (8 RW)), 8 warps: warp w computes rows 8 RW blockIdx.y + RW w .. + RW - 1 of
 // W_v,j against the ob of every query of KV head j (B * G of them, 8 at a time).
@@ -740,6 +886,15 @@ cudaError_t launch_pv_gs(const AbsorbParams &p, int max_len, cudaStream_t st)
 template <int BITS, int MT>
 cudaError_t launch_pv(const AbsorbParams &p, int max_len, cudaStream_t st)
 {
+    if (p.group == 128) {
+        const size_t smem = (size_t)MT * 16 * 256 * 4 + (size_t)256 * (128 * BITS / 8 + 16) +
+                            (size_t)MT * 16 * (256 + 8) * 2;
+        cudaError_t e = set_smem(absorb_pv128_kernel<BITS, MT>, smem);
+        if (e != cudaSuccess) return e;
+        const int ns = max(1, (max_len + p.split - 1) / p.split);
+        return launch_pdl(absorb_pv128_kernel<BITS, MT>, dim3(p.D / 128, p.B, ns), dim3(128), smem,
+                          st, p);
+    }
     switch (p.group) {
     case 32: return launch_pv_gs<BITS, MT, 32>(p, max_len, st);
     case 64: return launch_pv_gs<BITS, MT, 64>(p, max_len, st);

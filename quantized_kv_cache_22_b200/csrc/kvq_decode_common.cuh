@@ -124,17 +124,6 @@ __device__ __forceinline__ uint2 ldsi_u64(uint32_t a)
     asm volatile("ld.shared.v2.u32 {%0, %1}, [%2+%3];" : "=r"(v.x), "=r"(v.y) : "r"(a), "n"(IMM));
     return v;
 }
-// Four 8x8 matrices of 16-bit elements, transposed (ldmatrix .trans): lanes 8m ..
-// 8m + 7 give the row addresses of matrix m (16 bytes each, at a + IMM), and lane
-// l receives y[m] = rows 2(l%4), 2(l%4)+1 of column l/4 of matrix m, the lower row
-// in the low half.
-template <int IMM>
-__device__ __forceinline__ void ldsm_x4_trans(uint32_t a, uint32_t (&y)[4])
-{
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4+%5];"
-                 : "=r"(y[0]), "=r"(y[1]), "=r"(y[2]), "=r"(y[3])
-                 : "r"(a), "n"(IMM));
-}
 template <int IMM>
 __device__ __forceinline__ uint4 ldsi_u128(uint32_t a)
 {

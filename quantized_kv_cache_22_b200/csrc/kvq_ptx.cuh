@@ -241,6 +241,17 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x)
     return y;
 }
 
+// Four 8x8 matrices of 16-bit elements, transposed (ldmatrix .trans): lanes 8m ..
+// 8m + 7 give the row addresses of matrix m (16 bytes each, at a + IMM), and lane
+// l receives y[m] = rows 2(l%4), 2(l%4)+1 of column l/4 of matrix m, the lower row
+// in the low half.
+template <int IMM>
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t a, uint32_t (&y)[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4+%5];"
+                 : "=r"(y[0]), "=r"(y[1]), "=r"(y[2]), "=r"(y[3])
+                 : "r"(a), "n"(IMM));
+}
 // Ask for `bytes` (a multiple of 16, at a 16-byte aligned address) of global memory
 // to be brought into L2 by the copy engine; nothing is returned or waited for.
 __device__ __forceinline__ void bulk_prefetch_l2(const void *p, uint32_t bytes)

@@ -72,7 +72,9 @@ def _gpu(cfg, h, W, q, lens, out_dtype=torch.float32, scale=0.0):
 
 @pytest.mark.parametrize("hbits,hgroups,G,Dh,D", [
     (4, 4, 1, 128, 512), (8, 4, 2, 128, 512), (4, 16, 1, 128, 2048), (4, 8, 4, 64, 512),
-    (8, 16, 1, 64, 512), (4, 2, 8, 128, 256)])
+    (8, 16, 1, 64, 512), (4, 2, 8, 128, 256),
+    # 128-element groups with more than 16 query heads (two m-tiles of heads)
+    (4, 4, 3, 64, 512), (8, 4, 3, 64, 512)])
 def test_absorbed_decode_matches_oracle(cuda_device, hbits, hgroups, G, Dh, D):
     B, n, cap = 3, 300, 320
     lens = [300, 1, 129]
