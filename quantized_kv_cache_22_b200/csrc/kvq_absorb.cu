@@ -134,6 +134,13 @@ __global__ void __launch_bounds__(128) absorb_q_kernel(AbsorbParams p)
             cp_async16(wb + row * 256 + 16 * c, src + (int64_t)row * p.D + 8 * c);
         }
     }
+    // element offset of each query row of the chunk in q (no run-time division per load)
+    __shared__ int64_t qoff[8];
+    if (tid < 8) {
+        const int qi = q0 + min(tid, nqc - 1);
+        qoff[tid] = ((int64_t)(qi / G) * p.Hq + j * G + qi % G) * DH;
+    }
+    __syncthreads();
     grid_dependency_wait();
     // ob, which the p . h^ launch accumulates into, starts at zero
     {
@@ -150,9 +157,8 @@ __global__ void __launch_bounds__(128) absorb_q_kernel(AbsorbParams p)
         int64_t idx[R];
 #pragma unroll
         for (int r = 0; r < R; r++) {
-            const int k = tid + 128 * r, c = k / DH, i = k % DH;
-            const int qi = q0 + min(c, nqc - 1), b = qi / G, h = j * G + qi % G;
-            idx[r] = ((int64_t)b * p.Hq + h) * DH + i;
+            const int k = tid + 128 * r;
+            idx[r] = qoff[k / DH] + k % DH;
         }
         if (p.q_dtype == KVQ_F32) {
 #pragma unroll
@@ -455,18 +461,26 @@ __global__ void __launch_bounds__(128) absorb_pv_kernel(AbsorbParams p)
     if (t_begin >= len) return;
     const int t_end = min(len, t_begin + p.split);
     // merged statistics: M = max_k m_k, L = sum_k l_k 2^(m_k - M) over the score tiles
-    if (tid < MT * 16) {
+    {
+        // merged statistics, TPH consecutive threads per head, each over every TPH-th
+        // tile, combined by shuffles
+        constexpr int TPH = 128 / (MT * 16);
+        const int h = tid / TPH, part = tid % TPH;
+        const int nt = (len + p.T2 - 1) / p.T2;
         float M = -INFINITY, L = 0.f;
-        if (tid < p.Hq) {
-            const float2 *st = p.stats + ((int64_t)b * p.Hq + tid) * p.ntile;
-            const int nt = (len + p.T2 - 1) / p.T2;
-#pragma unroll 8
-            for (int k = 0; k < nt; k++) M = fmaxf(M, st[k].x);
-#pragma unroll 8
-            for (int k = 0; k < nt; k++) L += st[k].y * exp2f(st[k].x - M);
+        const float2 *st = p.stats + ((int64_t)b * p.Hq + min(h, p.Hq - 1)) * p.ntile;
+        if (h < p.Hq)
+            for (int k = part; k < nt; k += TPH) M = fmaxf(M, st[k].x);
+#pragma unroll
+        for (int off = 1; off < TPH; off <<= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, off));
+        if (h < p.Hq)
+            for (int k = part; k < nt; k += TPH) L += st[k].y * exp2f(st[k].x - M);
+#pragma unroll
+        for (int off = 1; off < TPH; off <<= 1) L += __shfl_xor_sync(FULL, L, off);
+        if (part == 0) {
+            hm[h] = M;
+            hinv[h] = L > 0.f ? 1.f / L : 0.f;
         }
-        hm[tid] = M;
-        hinv[tid] = L > 0.f ? 1.f / L : 0.f;
     }
     grid_launch_dependents();
     constexpr int ntw = GS / 32;                   // n-tiles of 8 columns per warp (1, 2 or 4)
@@ -625,18 +639,26 @@ __global__ void __launch_bounds__(128) absorb_pv128_kernel(AbsorbParams p)
     const int t_begin = split * p.split;
     if (t_begin >= len) return;
     const int t_end = min(len, t_begin + p.split);
-    if (tid < MT * 16) {
+    {
+        // merged statistics, TPH consecutive threads per head, each over every TPH-th
+        // tile, combined by shuffles
+        constexpr int TPH = 128 / (MT * 16);
+        const int h = tid / TPH, part = tid % TPH;
+        const int nt = (len + p.T2 - 1) / p.T2;
         float M = -INFINITY, L = 0.f;
-        if (tid < p.Hq) {
-            const float2 *st = p.stats + ((int64_t)b * p.Hq + tid) * p.ntile;
-            const int nt = (len + p.T2 - 1) / p.T2;
-#pragma unroll 8
-            for (int k = 0; k < nt; k++) M = fmaxf(M, st[k].x);
-#pragma unroll 8
-            for (int k = 0; k < nt; k++) L += st[k].y * exp2f(st[k].x - M);
+        const float2 *st = p.stats + ((int64_t)b * p.Hq + min(h, p.Hq - 1)) * p.ntile;
+        if (h < p.Hq)
+            for (int k = part; k < nt; k += TPH) M = fmaxf(M, st[k].x);
+#pragma unroll
+        for (int off = 1; off < TPH; off <<= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, off));
+        if (h < p.Hq)
+            for (int k = part; k < nt; k += TPH) L += st[k].y * exp2f(st[k].x - M);
+#pragma unroll
+        for (int off = 1; off < TPH; off <<= 1) L += __shfl_xor_sync(FULL, L, off);
+        if (part == 0) {
+            hm[h] = M;
+            hinv[h] = L > 0.f ? 1.f / L : 0.f;
         }
-        hm[tid] = M;
-        hinv[tid] = L > 0.f ? 1.f / L : 0.f;
     }
     grid_launch_dependents();
     float acc[MT][4][4];
@@ -768,11 +790,13 @@ __global__ void __launch_bounds__(256) absorb_out_kernel(AbsorbParams p)
         const int nqc = min(8, nq - q0);
         __syncthreads();                            // the previous chunk's ob is consumed
         {
+            // per query, its D / 4 pieces (no division by run-time sizes per piece)
             const uint32_t ob_s = smem_u32(obs);
-            for (int k = threadIdx.x; k < nqc * D4; k += blockDim.x) {
-                const int c = k / D4, d4 = k % D4;
+            for (int c = 0; c < nqc; c++) {
                 const int qi = q0 + c, b = qi / G, h = j * G + qi % G;
-                cp_async16(ob_s + 16 * k, p.obp + ((int64_t)b * p.Hq + h) * p.D + 4 * d4);
+                const float *src = p.obp + ((int64_t)b * p.Hq + h) * p.D;
+                for (int d4 = threadIdx.x; d4 < D4; d4 += blockDim.x)
+                    cp_async16(ob_s + 16 * (c * D4 + d4), src + 4 * d4);
             }
         }
         cp_async_wait_all();
@@ -796,7 +820,8 @@ __global__ void __launch_bounds__(256) absorb_out_kernel(AbsorbParams p)
             }
 #pragma unroll
             for (int c = 0; c < 8; c++) {
-                if (c >= nqc) break;
+                // rows of queries past nqc hold the previous chunk's ob or garbage: their
+                // sums are never written
                 const float4 o = *reinterpret_cast<const float4 *>(obs + (size_t)c * p.D + d0);
 #pragma unroll
                 for (int r = 0; r < RW; r++) {
@@ -809,21 +834,45 @@ __global__ void __launch_bounds__(256) absorb_out_kernel(AbsorbParams p)
                 }
             }
         }
+        // Sum each of the NV = 8 RW accumulators over the warp's 32 lanes by halving
+        // exchanges: at offset 16 a lane keeps the half of its values that its lane bit
+        // selects and adds the partner's copy of that half, then the same at offsets
+        // 8, 4, ... until one value is left per lane (LG = log2 NV steps); the remaining
+        // offsets add up the lanes that hold the same value.  The value a lane ends
+        // with is the binary number of its lane bits 4, 3, ... (one per step).
+        constexpr int NV = RW * 8, LG = RW == 2 ? 4 : 3;
+        float vals[NV];
 #pragma unroll
         for (int r = 0; r < RW; r++)
 #pragma unroll
-            for (int c = 0; c < 8; c++) {
-                float v = acc[r][c];
-                for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(FULL, v, off);
-                if (lane == 0 && c < nqc) {
-                    const int qi = q0 + c, b = qi / G, h = j * G + qi % G;
-                    const int64_t o = ((int64_t)b * p.Hq + h) * p.Dh + rbase + RW * warp + r;
-                    if (p.out_f32)
-                        static_cast<float *>(p.out)[o] = v;
-                    else
-                        static_cast<__half *>(p.out)[o] = __float2half_rn(v);
-                }
+            for (int c = 0; c < 8; c++) vals[r * 8 + c] = acc[r][c];
+        int idx = 0;
+#pragma unroll
+        for (int step = 0; step < LG; step++) {
+            const int half = NV >> (step + 1), off = 16 >> step;
+            const bool up = (lane & off) != 0;
+#pragma unroll
+            for (int i = 0; i < half; i++) {
+                const float send = up ? vals[i] : vals[i + half];
+                const float keep = up ? vals[i + half] : vals[i];
+                vals[i] = keep + __shfl_xor_sync(FULL, send, off);
             }
+            idx = 2 * idx + (up ? 1 : 0);
+        }
+        float v = vals[0];
+#pragma unroll
+        for (int off = 16 >> LG; off > 0; off >>= 1) v += __shfl_xor_sync(FULL, v, off);
+        {
+            const int r = idx / 8, c = idx % 8;
+            if ((lane & ((16 >> LG) * 2 - 1)) == 0 && c < nqc) {
+                const int qi = q0 + c, b = qi / G, h = j * G + qi % G;
+                const int64_t o = ((int64_t)b * p.Hq + h) * p.Dh + rbase + RW * warp + r;
+                if (p.out_f32)
+                    static_cast<float *>(p.out)[o] = v;
+                else
+                    static_cast<__half *>(p.out)[o] = __float2half_rn(v);
+            }
+        }
     }
 }
 
