@@ -281,7 +281,7 @@ __global__ void __launch_bounds__(NTHR, 2)
     // packed columns: int8 keys without zero-points, or e4m3 keys with one scale per
     // (token, head), whose f16 score MMA then always takes the fp16 query and its
     // residual (zero for fp16 queries) as the hi / lo parts
-    static_assert(!PK || (IMMA_K && !ZP) || (F8 && !KG), "no packed columns for this format");
+    static_assert(!PK || (IMMA_K && (!ZP || !KG)) || (F8 && !KG), "no packed columns for this format");
     constexpr int NU = PK ? 1 : 2;             // score sub-tiles a lane carries
     const int gid = lane >> 2;
     const int tig = lane & 3;
@@ -430,8 +430,9 @@ __global__ void __launch_bounds__(NTHR, 2)
             if constexpr (ZP && !KG) {
                 qs_all += __shfl_xor_sync(FULL, qs_all, 1);
                 qs_all += __shfl_xor_sync(FULL, qs_all, 2);
-                zq[0][0] = __shfl_sync(FULL, qs_all, (2 * tig) * 4);
-                zq[0][1] = __shfl_sync(FULL, qs_all, (2 * tig + 1) * 4);
+                const int zc = PK ? 2 * (tig & 1) : 2 * tig;   // the lane's first head column
+                zq[0][0] = __shfl_sync(FULL, qs_all, zc * 4);
+                zq[0][1] = __shfl_sync(FULL, qs_all, (zc + 1) * 4);
             }
             // 4-bit key codes enter the MMA as 16 * code
             const float f = amax * (1.f / (127.f * 254.f)) * p.tau_log2e * (KB == 4 ? 0.0625f : 1.f);
@@ -625,13 +626,26 @@ __global__ void __launch_bounds__(NTHR, 2)
                 if constexpr (PK) {
                     // lanes tig < 2: own hi of sub-tile 0 (ah[0]), partner's lo (its ah[0]);
                     // lanes tig >= 2: own hi of sub-tile 1 (ah[1]), partner's lo (its ah[1])
-                    const float2 kk = PT ? make_float2(k_tensor, k_tensor)
-                                         : unpack_half2(lds_u32(sbase, ssk + 2 * (ul ? tAu[1] : tAu[0])));
+                    const int tl = ul ? tAu[1] : tAu[0];
+                    float2 kk;
+                    int z0 = 0, z1 = 0;   // zero-points of the lane's two score rows
+                    if constexpr (PT) {
+                        kk = make_float2(k_tensor, k_tensor);
+                    } else if constexpr (ZP) {
+                        const uint2 w = lds_u64(sbase, ssk + 4 * tl);
+                        kk = make_float2(__half2float(__ushort_as_half((unsigned short)(w.x & 0xFFFFu))),
+                                         __half2float(__ushort_as_half((unsigned short)(w.y & 0xFFFFu))));
+                        z0 = __half2int_rn(__ushort_as_half((unsigned short)(w.x >> 16)));
+                        z1 = __half2int_rn(__ushort_as_half((unsigned short)(w.y >> 16)));
+                    } else {
+                        kk = unpack_half2(lds_u32(sbase, ssk + 2 * tl));
+                    }
 #pragma unroll
                     for (int e = 0; e < 4; e++) {
                         const int mine = ul ? ah[1][e] : ah[0][e];
                         const int send = ul ? ah[0][e] : ah[1][e];
-                        const int a = mine * 254 + __shfl_xor_sync(FULL, send, 2);
+                        int a = mine * 254 + __shfl_xor_sync(FULL, send, 2);
+                        if constexpr (ZP) a -= ((e < 2) ? z0 : z1) * zq[0][e & 1];
                         s2[0][e] = (float)a * (((e < 2) ? kk.x : kk.y) * sqc[e & 1]);
                     }
                 } else {
@@ -894,7 +908,8 @@ __global__ void __launch_bounds__(NTHR, 2)
         float sv[2][2][NVG];   // [sub-tile][row][value group]
         float lsv[2][2];
         // uint8 values: A fragments half2(1024 + z) of the P.V k-slot tokens (tw + vA,
-        // tw + vB; tw + vA + 1, tw + vB + 1), zero past the length (stale scales)
+        // tw + vB; tw + vA + 1, tw + vB + 1), zero past the length (stale scales), set
+        // after the scale loop below
         uint32_t za[2][NVG][2];
 #pragma unroll
         for (int u = 0; u < NU; u++) {
@@ -923,12 +938,30 @@ __global__ void __launch_bounds__(NTHR, 2)
                         (unsigned short)lds_u16(sbase, ssv + 2 * ((tA + 1) * p.ngs_v + SCV * (g >> p.vshift)))));
                 }
             }
-            if constexpr (ZP) {
+            // scales past the length may be stale shared memory: never use them
+#pragma unroll
+            for (int r = 0; r < 2; r++) {
+                float mx = 0.f;
+#pragma unroll
+                for (int g = 0; g < NVG; g++) {
+                    sv[u][r][g] = vt[u][r] ? sv[u][r][g] : 0.f;
+                    mx = fmaxf(mx, sv[u][r][g]);
+                }
+                lsv[u][r] = mx > 0.f ? fmaxf(__log2f(mx), -32.f) : -32.f;
+            }
+        }
+
+        // uint8 values: the za fragments of both sub-tiles (with packed columns too, each
+        // sub-tile's P.V MMA takes its own)
+        if constexpr (ZP) {
+            constexpr int SCV = scale_vals(FMT);
+            const uint32_t B1024 = 0x64006400u;   // half2(1024, 1024)
+#pragma unroll
+            for (int u = 0; u < 2; u++) {
                 const int tw = warp * 32 + u * 16;
                 const int rem = m.len - m.t0 - tw;   // valid tokens of the sub-tile
                 const uint32_t mlo = (vA < rem ? 0x0000FFFFu : 0u) | (vB < rem ? 0xFFFF0000u : 0u);
                 const uint32_t mhi = (vA + 1 < rem ? 0x0000FFFFu : 0u) | (vB + 1 < rem ? 0xFFFF0000u : 0u);
-                const uint32_t B1024 = 0x64006400u;   // half2(1024, 1024)
                 if constexpr (!vgrp) {
                     const uint2 wA = lds_u64(sbase, ssv + 4 * (tw + vA));   // (s, z) of tw+vA, tw+vA+1
                     const uint2 wB = lds_u64(sbase, ssv + 4 * (tw + vB));
@@ -946,17 +979,6 @@ __global__ void __launch_bounds__(NTHR, 2)
                         za[u][g][1] = hadd2_u32((a1 | (b1 << 16)) & mhi, B1024);
                     }
                 }
-            }
-            // scales past the length may be stale shared memory: never use them
-#pragma unroll
-            for (int r = 0; r < 2; r++) {
-                float mx = 0.f;
-#pragma unroll
-                for (int g = 0; g < NVG; g++) {
-                    sv[u][r][g] = vt[u][r] ? sv[u][r][g] : 0.f;
-                    mx = fmaxf(mx, sv[u][r][g]);
-                }
-                lsv[u][r] = mx > 0.f ? fmaxf(__log2f(mx), -32.f) : -32.f;
             }
         }
 
@@ -1016,11 +1038,19 @@ __global__ void __launch_bounds__(NTHR, 2)
             for (int g = 0; g < NVG; g++) {
                 const uint32_t t0 = movmatrix_trans(pack_half2(pr[0] * sv[0][0][g], pr[1] * sv[0][0][g]));
                 const uint32_t t1 = movmatrix_trans(pack_half2(pr[2] * sv[0][1][g], pr[3] * sv[0][1][g]));
-                if constexpr (VBIAS) mma_16816(psum[g], ONE2, ONE2, ONE2, ONE2, t0, t1);
                 pb[0][g][0] = t0 & keep0;
                 pb[0][g][1] = t1 & keep0;
                 pb[1][g][0] = t0 & ~keep0;
                 pb[1][g][1] = t1 & ~keep0;
+                if constexpr (ZP) {
+                    // each sub-tile's zero-points against its own columns
+#pragma unroll
+                    for (int u = 0; u < 2; u++)
+                        mma_16816(psum[g], za[u][g][0], za[u][g][0], za[u][g][1], za[u][g][1], pb[u][g][0],
+                                  pb[u][g][1]);
+                } else if constexpr (VBIAS) {
+                    mma_16816(psum[g], ONE2, ONE2, ONE2, ONE2, t0, t1);
+                }
             }
         } else {
 #pragma unroll

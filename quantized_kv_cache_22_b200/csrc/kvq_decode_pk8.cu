@@ -1,6 +1,6 @@
 // kvq_decode_pk8.cu -- decode kernel instances with packed score columns (G <= 4,
 // head_dim 128) for 8-bit keys: symmetric INT4 / INT8 values, per-tensor INT8, and FP8
-// e4m3 keys and values (key scales per (token, head))
+// e4m3 and asymmetric INT8 keys and values (key scales per (token, head))
 #include "kvq_decode_kernel.cuh"
 
 namespace kvq {
@@ -25,6 +25,10 @@ void *decode_fn_pk_kb8(int vb, bool kg, bool vg, int fmt)
 {
     if (fmt == KVQ_FMT_TENSOR)
         return (vb == 8 && !kg && !vg) ? fn<8, false, false, KVQ_FMT_TENSOR>() : nullptr;
+    if (fmt == KVQ_FMT_ASYM) {
+        if (vb != 8 || kg) return nullptr;
+        return vg ? fn<8, false, true, KVQ_FMT_ASYM>() : fn<8, false, false, KVQ_FMT_ASYM>();
+    }
     if (fmt == KVQ_FMT_E4M3) {
         if (vb != 8 || kg) return nullptr;
         return vg ? fn<8, false, true, KVQ_FMT_E4M3>() : fn<8, false, false, KVQ_FMT_E4M3>();

@@ -296,7 +296,9 @@ def test_decode_plan_info_without_device(monkeypatch):
                 v_bits=8, k_group=128, v_group=128, kv_format=kvq.KVQ_FMT_E4M3)
     assert kvq.kvq_decode_plan_info(f8, 296)["packed_columns"] == 1
     a8 = Config(**{**f8.__dict__, "kv_format": kvq.KVQ_FMT_ASYM})
-    assert kvq.kvq_decode_plan_info(a8, 296)["packed_columns"] == 0
+    assert kvq.kvq_decode_plan_info(a8, 296)["packed_columns"] == 1
+    a8g = Config(**{**a8.__dict__, "k_group": 32})   # grouped zero-points: unpacked
+    assert kvq.kvq_decode_plan_info(a8g, 296)["packed_columns"] == 0
     g8 = Config(batch=2, capacity=256, n_q_heads=16, n_kv_heads=2, head_dim=128, k_bits=8, v_bits=8,
                 k_group=128, v_group=128)
     assert kvq.kvq_decode_plan_info(g8, 10)["packed_columns"] == 0
