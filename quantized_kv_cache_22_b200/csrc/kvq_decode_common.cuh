@@ -54,6 +54,33 @@ __device__ __forceinline__ float load_qf(const void *q, int dtype, int64_t idx)
     return __bfloat162float(static_cast<const __nv_bfloat16 *>(q)[idx]);
 }
 
+// Eight consecutive query elements idx .. idx+7 as float: one 16-byte load (two for
+// fp32).  Every entry point refuses a query base that is not 16-byte aligned, and
+// idx is a multiple of 8.  The dtype test is uniform across the warp.
+__device__ __forceinline__ void load_q8(const void *q, int dtype, int64_t idx, float (&x)[8])
+{
+    if (dtype == KVQ_F32) {
+        const float4 *s = reinterpret_cast<const float4 *>(static_cast<const float *>(q) + idx);
+        const float4 a = __ldg(s), b = __ldg(s + 1);
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+        x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+    } else {
+        const uint4 w = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(q) + idx));
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            if (dtype == KVQ_F16) {
+                x[2 * i] = __half2float(__ushort_as_half((unsigned short)(ws[i] & 0xFFFFu)));
+                x[2 * i + 1] = __half2float(__ushort_as_half((unsigned short)(ws[i] >> 16)));
+            } else {
+                // bfloat16 -> float: the 16 bits become the high half of the word
+                x[2 * i] = __uint_as_float(ws[i] << 16);
+                x[2 * i + 1] = __uint_as_float(ws[i] & 0xFFFF0000u);
+            }
+        }
+    }
+}
+
 __device__ __forceinline__ int clamp_len(int len, int cap)
 {
     return len < 0 ? 0 : (len > cap ? cap : len);

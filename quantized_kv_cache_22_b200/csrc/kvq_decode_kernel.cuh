@@ -367,15 +367,17 @@ __global__ void __launch_bounds__(NTHR, 2)
             float x[NG][8];
             float amax = 0.f;
 #pragma unroll
-            for (int blk = 0; blk < NG; blk++)
+            for (int blk = 0; blk < NG; blk++) {
+                // the lane's 8 elements of the block are contiguous
+                if (valid)
+                    load_q8(p.q, p.q_dtype,
+                            qbase + (blk / KPL) * 32 * KPL + 8 * KPL * tig + 8 * (blk % KPL), x[blk]);
+                else
 #pragma unroll
-                for (int j = 0; j < 8; j++) {
-                    x[blk][j] = valid ? load_qf(p.q, p.q_dtype,
-                                                qbase + (blk / KPL) * 32 * KPL + 8 * KPL * tig +
-                                                    8 * (blk % KPL) + j)
-                                      : 0.f;
-                    amax = fmaxf(amax, fabsf(x[blk][j]));
-                }
+                    for (int j = 0; j < 8; j++) x[blk][j] = 0.f;
+#pragma unroll
+                for (int j = 0; j < 8; j++) amax = fmaxf(amax, fabsf(x[blk][j]));
+            }
             amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 1));
             amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 2));
             const float inv = amax > 0.f ? 127.f / amax : 0.f;

@@ -123,6 +123,7 @@ def test_validation_errors_are_returned_on_the_host():
     assert _rc("kvq_decode_attn", *args(qd=5)) == -1
     assert _rc("kvq_decode_attn", *args(od=2)) == -1
     assert _rc("kvq_decode_attn", *args(out=P(130))) == -4
+    assert _rc("kvq_decode_attn", *args(q=P(18))) == -4   # the kernels load queries 16 bytes at a time
     assert _rc("kvq_decode_attn", *args(w=P(512))) == -1
     assert _rc("kvq_decode_attn", *args(q=None)) == -1
     # h-mode reconstruction argument checks
