@@ -62,11 +62,20 @@ __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d)
            ((uint32_t)(d & 0xff) << 24);
 }
 
+// bf16 hi and lo parts of the pair (a, b): a ~ hi + lo to 16 significant bits
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t &hi, uint32_t &lo)
+{
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+    hi = *reinterpret_cast<const uint32_t *>(&h);
+    lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
 // ---------------------------------------------------------------- qa
-// Grid (Hkv, D / 128, query chunks of 8), 128 threads: thread (rg, cg) sums rows
-// rg, rg + 8, ... of W_k,j over 8 columns (one 16-byte load per row) for the
-// chunk's queries; the 8 row groups are summed in shared memory.  Per query and
-// scale group, qa ~ (amax/127)(hi + lo/254), hi, lo in [-127, 127]; a thread's 8
+// Grid (Hkv, D / 128, query chunks of 8), 128 threads: the CTA's 128 columns of
+// W_k,j^T q for the chunk's queries on tensor cores (see below), then thread
+// (q, cg) quantises 8 columns of query q.  Per query and scale group, qa ~ (amax/127)(hi + lo/254), hi, lo in [-127, 127]; a thread's 8
 // columns are exactly one lane's slot of the score MMA's B fragment (k-slot order
 // of 8-bit or 4-bit codes), written as one 16-byte store {hi0, hi1, lo0, lo1}.
 // The factor amax/(127*254) * tau*log2(e) (/16 for 4-bit codes, which enter the
@@ -74,12 +83,10 @@ __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d)
 template <int DH>
 __global__ void __launch_bounds__(128) absorb_q_kernel(AbsorbParams p)
 {
-    __shared__ float qs[8][DH];
-    // the W_k tile [DH][128] bf16 while it is read, then the row-group partials
-    __shared__ __align__(16) float wpart[8 * 8 * (128 + 4)];
-    const __nv_bfloat16 *wt = reinterpret_cast<const __nv_bfloat16 *>(wpart);   // [DH][128]
-    float (*part)[8][128 + 4] = reinterpret_cast<float (*)[8][128 + 4]>(wpart);   // [rg][query][col]
-    static_assert(DH * 128 * 2 <= 8 * 8 * (128 + 4) * 4, "W tile fits the partials buffer");
+    constexpr int WS = 128 + 8;   // padded row stride of the W tile (conflict-free ldmatrix)
+    __shared__ __align__(16) float qs[8][DH + 8];
+    __shared__ __align__(16) __nv_bfloat16 wt[DH * WS];   // W_k,j [DH][the tile's 128 columns]
+    __shared__ __align__(16) float part[8][128 + 4];      // qa of the chunk [query][column]
     const int j = blockIdx.x, tile = blockIdx.y;
     const int tid = threadIdx.x;
     const int G = p.Hq / p.Hkv;
@@ -126,12 +133,12 @@ __global__ void __launch_bounds__(128) absorb_q_kernel(AbsorbParams p)
     }
     // W_k does not depend on earlier launches: its copies start before the wait
     {
-        const uint32_t wb = smem_u32(wpart);
+        const uint32_t wb = smem_u32(wt);
         const __nv_bfloat16 *src = p.w + (int64_t)j * DH * p.D + tile * 128;
 #pragma unroll
         for (int r = 0; r < DH * 16 / 128; r++) {
             const int k = tid + 128 * r, row = k / 16, c = k % 16;
-            cp_async16(wb + row * 256 + 16 * c, src + (int64_t)row * p.D + 8 * c);
+            cp_async16(wb + row * (2 * WS) + 16 * c, src + (int64_t)row * p.D + 8 * c);
         }
     }
     // element offset of each query row of the chunk in q (no run-time division per load)
@@ -180,49 +187,58 @@ __global__ void __launch_bounds__(128) absorb_q_kernel(AbsorbParams p)
         }
     }
     __syncthreads();
-    const int rg = tid >> 4, cg = tid & 15;
-    const int c0 = tile * 128 + cg * 8;
-    float acc[8][8];
+    // qa^T (the tile's 128 columns x 8 queries) = W^T (columns x DH) q^T (DH x 8 queries) on
+    // bf16 tensor cores, warp w taking columns 32w .. 32w + 31: A fragments by transposed
+    // ldmatrix from the W tile, B fragments from the queries split into bf16 hi and lo
+    // parts (q = hi + lo to 16 significant bits; W_k is bf16 itself), fp32 accumulation.
+    const int warp = tid >> 5, lane = tid & 31, gid = lane >> 2, tig = lane & 3;
+    uint32_t bhi[DH / 16][2], blo[DH / 16][2];
 #pragma unroll
-    for (int c = 0; c < 8; c++)
+    for (int ks = 0; ks < DH / 16; ks++)
 #pragma unroll
-        for (int e = 0; e < 8; e++) acc[c][e] = 0.f;
+        for (int h = 0; h < 2; h++) {
+            const float2 v = *reinterpret_cast<const float2 *>(&qs[gid][16 * ks + 8 * h + 2 * tig]);
+            split_bf16x2(v.x, v.y, bhi[ks][h], blo[ks][h]);
+        }
+    float acc[2][4];
+#pragma unroll
+    for (int mt = 0; mt < 2; mt++) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
     cp_async_wait_all();
     __syncthreads();
-#pragma unroll 4
-    for (int k = 0; k < DH / 8; k++) {
-        const uint4 w = *reinterpret_cast<const uint4 *>(wt + (rg + 8 * k) * 128 + cg * 8);
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-        float wf[8];
+    {
+        // matrices (k 0-7, m 0-7), (k 0-7, m 8-15), (k 8-15, m 0-7), (k 8-15, m 8-15) of the
+        // tile stored [k][m]: lane l gives row (l & 7) + 8 (l >> 4), column 8 ((l >> 3) & 1)
+        const uint32_t a0 = smem_u32(wt) +
+                            2 * (((lane & 7) + 8 * (lane >> 4)) * WS + 32 * warp + 8 * ((lane >> 3) & 1));
 #pragma unroll
-        for (int e = 0; e < 4; e++) {
-            wf[2 * e] = __uint_as_float(ws[e] << 16);
-            wf[2 * e + 1] = __uint_as_float(ws[e] & 0xFFFF0000u);
-        }
+        for (int ks = 0; ks < DH / 16; ks++)
 #pragma unroll
-        for (int c = 0; c < 8; c++) {
-            const float qv = qs[c][rg + 8 * k];
-#pragma unroll
-            for (int e = 0; e < 8; e++) acc[c][e] = fmaf(qv, wf[e], acc[c][e]);
-        }
+            for (int mt = 0; mt < 2; mt++) {
+                uint32_t a[4];
+                ldsm_x4_trans<0>(a0 + 2 * (16 * ks * WS + 16 * mt), a);
+                mma_bf16_16816(acc[mt], a[0], a[1], a[2], a[3], bhi[ks][0], bhi[ks][1]);
+                mma_bf16_16816(acc[mt], a[0], a[1], a[2], a[3], blo[ks][0], blo[ks][1]);
+            }
     }
-    __syncthreads();                          // the W tile is consumed: reuse it for the partials
+    // accumulator rows are columns of the tile, its columns queries
 #pragma unroll
-    for (int c = 0; c < 8; c++)
-#pragma unroll
-        for (int e = 0; e < 8; e++) part[rg][c][cg * 8 + e] = acc[c][e];
+    for (int mt = 0; mt < 2; mt++) {
+        const int c = 32 * warp + 16 * mt + gid;
+        part[2 * tig][c] = acc[mt][0];
+        part[2 * tig + 1][c] = acc[mt][1];
+        part[2 * tig][c + 8] = acc[mt][2];
+        part[2 * tig + 1][c + 8] = acc[mt][3];
+    }
     __syncthreads();
-    // thread (q = tid / 16, cg): the query's 8 columns summed over the row groups
-    const int q = tid >> 4;
+    // thread (q = tid / 16, cg): 8 columns of query q
+    const int q = tid >> 4, cg = tid & 15;
+    const int c0 = tile * 128 + cg * 8;
     float x[8];
     float amax = 0.f;
 #pragma unroll
     for (int e = 0; e < 8; e++) {
-        float v = 0.f;
-#pragma unroll
-        for (int r = 0; r < 8; r++) v += part[r][q][cg * 8 + e];
-        x[e] = v;
-        amax = fmaxf(amax, fabsf(v));
+        x[e] = part[q][cg * 8 + e];
+        amax = fmaxf(amax, fabsf(x[e]));
     }
     // amax over the scale group's threads (consecutive lanes of a half-warp)
     for (int off = 1; off < p.group / 8; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, off));
@@ -246,9 +262,10 @@ __global__ void __launch_bounds__(128) absorb_q_kernel(AbsorbParams p)
                           pack4(lo[0], lo[2], lo[4], lo[6]), pack4(lo[1], lo[3], lo[5], lo[7]));
     }
     const int qi = q0 + q, b = qi / G, h = j * G + qi % G;
-    const int ks = c0 / 32, tig = (c0 % 32) / 8;
-    const int nt = h / 8, lane = (h % 8) * 4 + tig;
-    p.qfrag[(((int64_t)b * (p.D / 32) + ks) * p.NT + nt) * 32 + lane] = frag;
+    // the score MMA's B-fragment slot of these 8 columns: k-step, n-tile, lane
+    const int fks = c0 / 32, ftig = (c0 % 32) / 8;
+    const int nt = h / 8, flane = (h % 8) * 4 + ftig;
+    p.qfrag[(((int64_t)b * (p.D / 32) + fks) * p.NT + nt) * 32 + flane] = frag;
     if (c0 % p.group == 0)
         p.qfac[((int64_t)b * p.ng + c0 / p.group) * (p.NT * 8) + h] =
             amax * (1.f / (127.f * 254.f)) * p.tau_log2e * (p.bits == 4 ? 0.0625f : 1.f);
@@ -762,33 +779,45 @@ __global__ void __launch_bounds__(128) absorb_pv128_kernel(AbsorbParams p)
 }
 
 // ---------------------------------------------------------------- W_v . ob
-// Grid (Hkv, Dh / (8 RW)), 8 warps: warp w computes rows 8 RW blockIdx.y + RW w .. + RW - 1 of
-// W_v,j against the ob of every query of KV head j (B * G of them, 8 at a time).
-// The CTA's 8 RW W_v rows are copied to shared memory (cp.async) before the wait for
-// the previous launch, so that they stream in while it finishes; ob is staged after
-// it, every piece of a chunk of queries in flight at once.  Lane l reads
-// columns 128k + 4l .. +3: conflict-free 16-byte loads of ob, 8-byte loads of W.
-template <int RW>
+// Grid (Hkv, Dh / 16), 8 warps: the CTA's 16 rows of W_v,j against the ob of every
+// query of KV head j (B * G of them, 8 at a time) on bf16 tensor cores, out^T (16 rows
+// x 8 queries) = W (16 x D) ob^T (D x 8): ob enters as bf16 hi and lo parts (16
+// significant bits; W_v is bf16 itself), warp w takes the k-steps (16 columns of D) w,
+// w + 8, ..., and the 8 warps' fp32 partial sums are added in shared memory.  The W_v
+// rows are copied to shared memory (cp.async) before the wait for the previous launch,
+// so that they stream in while it finishes; ob is staged after it, every piece of a
+// chunk of queries in flight at once.  Rows are padded by 16 (W) and 32 (ob) bytes:
+// conflict-free ldmatrix and fragment loads.
 __global__ void __launch_bounds__(256) absorb_out_kernel(AbsorbParams p)
 {
-    extern __shared__ __align__(16) float obs[];    // [8][D] fp32, then [8 RW][D] bf16 rows of W_v
+    // [8][D + 8] fp32 ob, [16][D + 8] bf16 W_v rows, [8 warps][16 rows][8 queries] fp32
+    extern __shared__ __align__(16) float obs[];
+    const int OS = p.D + 8;
     const int j = blockIdx.x;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int rbase = blockIdx.y * 8 * RW;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
+    const int rbase = blockIdx.y * 16;
     const int G = p.Hq / p.Hkv;
     const int nq = p.B * G;
     const int D4 = p.D / 4;
-    __nv_bfloat16 *ws = reinterpret_cast<__nv_bfloat16 *>(obs + (size_t)8 * p.D);
+    __nv_bfloat16 *ws = reinterpret_cast<__nv_bfloat16 *>(obs + (size_t)8 * OS);
+    float *red = reinterpret_cast<float *>(ws + (size_t)16 * OS);
     {
         const uint32_t wb = smem_u32(ws);
         const __nv_bfloat16 *src = p.w + ((int64_t)p.Hkv * p.Dh + (int64_t)j * p.Dh + rbase) * p.D;
-        const int pieces = 8 * RW * p.D / 8;        // 16-byte pieces of the rows
-        for (int k = threadIdx.x; k < pieces; k += blockDim.x) cp_async16(wb + 16 * k, src + 8 * k);
+        const int per_row = p.D / 8;                // 16-byte pieces of a row
+        for (int r = 0; r < 16; r++)
+            for (int c = threadIdx.x; c < per_row; c += blockDim.x)
+                cp_async16(wb + 2 * r * OS + 16 * c, src + (int64_t)r * p.D + 8 * c);
     }
     grid_dependency_wait();
+    // ldmatrix row addresses of the matrices (rows 0-7, k 0-7), (rows 8-15, k 0-7),
+    // (rows 0-7, k 8-15), (rows 8-15, k 8-15): lane l gives row (l & 7) + 8 ((l >> 3) & 1),
+    // column 8 (l >> 4)
+    const uint32_t arow = smem_u32(ws) + 2 * (((lane & 7) + 8 * ((lane >> 3) & 1)) * OS + 8 * (lane >> 4));
+    const int nks = p.D / 16;
     for (int q0 = 0; q0 < nq; q0 += 8) {
         const int nqc = min(8, nq - q0);
-        __syncthreads();                            // the previous chunk's ob is consumed
+        __syncthreads();                            // the previous chunk's ob and sums are consumed
         {
             // per query, its D / 4 pieces (no division by run-time sizes per piece)
             const uint32_t ob_s = smem_u32(obs);
@@ -796,77 +825,40 @@ __global__ void __launch_bounds__(256) absorb_out_kernel(AbsorbParams p)
                 const int qi = q0 + c, b = qi / G, h = j * G + qi % G;
                 const float *src = p.obp + ((int64_t)b * p.Hq + h) * p.D;
                 for (int d4 = threadIdx.x; d4 < D4; d4 += blockDim.x)
-                    cp_async16(ob_s + 16 * (c * D4 + d4), src + 4 * d4);
+                    cp_async16(ob_s + 4 * (c * OS + 4 * d4), src + 4 * d4);
             }
         }
         cp_async_wait_all();
         __syncthreads();
-        float acc[RW][8];
-#pragma unroll
-        for (int r = 0; r < RW; r++)
-#pragma unroll
-            for (int c = 0; c < 8; c++) acc[r][c] = 0.f;
-#pragma unroll 2
-        for (int kk = 0; kk < p.D / 128; kk++) {
-            const int d0 = 128 * kk + 4 * lane;
-            float wf[RW][4];
-#pragma unroll
-            for (int r = 0; r < RW; r++) {
-                const uint2 w = *reinterpret_cast<const uint2 *>(ws + (size_t)(RW * warp + r) * p.D + d0);
-                wf[r][0] = __uint_as_float(w.x << 16);
-                wf[r][1] = __uint_as_float(w.x & 0xFFFF0000u);
-                wf[r][2] = __uint_as_float(w.y << 16);
-                wf[r][3] = __uint_as_float(w.y & 0xFFFF0000u);
-            }
-#pragma unroll
-            for (int c = 0; c < 8; c++) {
-                // rows of queries past nqc hold the previous chunk's ob or garbage: their
-                // sums are never written
-                const float4 o = *reinterpret_cast<const float4 *>(obs + (size_t)c * p.D + d0);
-#pragma unroll
-                for (int r = 0; r < RW; r++) {
-                    float a = acc[r][c];
-                    a = fmaf(wf[r][0], o.x, a);
-                    a = fmaf(wf[r][1], o.y, a);
-                    a = fmaf(wf[r][2], o.z, a);
-                    a = fmaf(wf[r][3], o.w, a);
-                    acc[r][c] = a;
-                }
-            }
+        // B columns of queries past nqc hold the previous chunk's ob or garbage: they
+        // only reach accumulator columns that are never written
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        const float *ob_row = obs + (size_t)gid * OS + 2 * tig;
+#pragma unroll 4
+        for (int ks = warp; ks < nks; ks += 8) {
+            uint32_t a[4];
+            ldsm_x4(arow + 32 * ks, a);
+            const float2 v0 = *reinterpret_cast<const float2 *>(ob_row + 16 * ks);
+            const float2 v1 = *reinterpret_cast<const float2 *>(ob_row + 16 * ks + 8);
+            uint32_t h0, l0, h1, l1;
+            split_bf16x2(v0.x, v0.y, h0, l0);
+            split_bf16x2(v1.x, v1.y, h1, l1);
+            mma_bf16_16816(acc, a[0], a[1], a[2], a[3], h0, h1);
+            mma_bf16_16816(acc, a[0], a[1], a[2], a[3], l0, l1);
         }
-        // Sum each of the NV = 8 RW accumulators over the warp's 32 lanes by halving
-        // exchanges: at offset 16 a lane keeps the half of its values that its lane bit
-        // selects and adds the partner's copy of that half, then the same at offsets
-        // 8, 4, ... until one value is left per lane (LG = log2 NV steps); the remaining
-        // offsets add up the lanes that hold the same value.  The value a lane ends
-        // with is the binary number of its lane bits 4, 3, ... (one per step).
-        constexpr int NV = RW * 8, LG = RW == 2 ? 4 : 3;
-        float vals[NV];
+        // accumulator rows are W_v rows, its columns queries
+        float *rw = red + warp * 128;
+        *reinterpret_cast<float2 *>(rw + gid * 8 + 2 * tig) = make_float2(acc[0], acc[1]);
+        *reinterpret_cast<float2 *>(rw + (gid + 8) * 8 + 2 * tig) = make_float2(acc[2], acc[3]);
+        __syncthreads();
+        if (threadIdx.x < 128) {
+            const int r = threadIdx.x >> 3, c = threadIdx.x & 7;
+            float v = 0.f;
 #pragma unroll
-        for (int r = 0; r < RW; r++)
-#pragma unroll
-            for (int c = 0; c < 8; c++) vals[r * 8 + c] = acc[r][c];
-        int idx = 0;
-#pragma unroll
-        for (int step = 0; step < LG; step++) {
-            const int half = NV >> (step + 1), off = 16 >> step;
-            const bool up = (lane & off) != 0;
-#pragma unroll
-            for (int i = 0; i < half; i++) {
-                const float send = up ? vals[i] : vals[i + half];
-                const float keep = up ? vals[i + half] : vals[i];
-                vals[i] = keep + __shfl_xor_sync(FULL, send, off);
-            }
-            idx = 2 * idx + (up ? 1 : 0);
-        }
-        float v = vals[0];
-#pragma unroll
-        for (int off = 16 >> LG; off > 0; off >>= 1) v += __shfl_xor_sync(FULL, v, off);
-        {
-            const int r = idx / 8, c = idx % 8;
-            if ((lane & ((16 >> LG) * 2 - 1)) == 0 && c < nqc) {
+            for (int w = 0; w < 8; w++) v += red[w * 128 + r * 8 + c];
+            if (c < nqc) {
                 const int qi = q0 + c, b = qi / G, h = j * G + qi % G;
-                const int64_t o = ((int64_t)b * p.Hq + h) * p.Dh + rbase + RW * warp + r;
+                const int64_t o = ((int64_t)b * p.Hq + h) * p.Dh + rbase + r;
                 if (p.out_f32)
                     static_cast<float *>(p.out)[o] = v;
                 else
@@ -875,6 +867,9 @@ __global__ void __launch_bounds__(256) absorb_out_kernel(AbsorbParams p)
         }
     }
 }
+
+// shared-memory bytes of absorb_out_kernel: ob chunk, W_v rows, partial sums
+size_t out_smem(int D) { return (size_t)(D + 8) * (8 * 4 + 16 * 2) + (size_t)8 * 128 * 4; }
 
 // shared-memory bytes of the kernels that size it at run time
 size_t scores_smem(int D, int bits, int NT, int ng, int T)
@@ -960,8 +955,7 @@ int absorb_nt(int Hq) { return Hq <= 8 ? 1 : (Hq <= 16 ? 2 : 4); }
 // fragments, and an 8-query ob chunk with 16 W_v rows.
 bool absorb_fits(int D, int bits, int Hq, int ng)
 {
-    return scores_smem(D, bits, absorb_nt(Hq), ng, 16) <= 227 * 1024 &&
-           (size_t)8 * D * 4 + (size_t)16 * D * 2 <= 227 * 1024;
+    return scores_smem(D, bits, absorb_nt(Hq), ng, 16) <= 227 * 1024 && out_smem(D) <= 227 * 1024;
 }
 
 // Tokens per score tile: 64 (4 warps), fewer when the tile and the fragments
@@ -1023,11 +1017,10 @@ cudaError_t launch_absorbed(const AbsorbParams &p, int max_len, cudaStream_t str
                         : (two ? launch_pv<4, 2>(p, max_len, stream) : launch_pv<4, 1>(p, max_len, stream));
         if (e != cudaSuccess) return e;
     }
-    // 16 W_v rows per CTA (8 rows, with twice the CTAs, measured 0.4 us slower)
-    constexpr int RW = 2;
-    const size_t osm = (size_t)8 * p.D * 4 + (size_t)8 * RW * p.D * 2;   // ob chunk + W_v rows
-    if ((e = set_smem(absorb_out_kernel<RW>, osm)) != cudaSuccess) return e;
-    return launch_pdl(absorb_out_kernel<RW>, dim3(p.Hkv, p.Dh / (8 * RW)), dim3(256), osm, stream, p);
+    // 16 W_v rows per CTA
+    const size_t osm = out_smem(p.D);
+    if ((e = set_smem(absorb_out_kernel, osm)) != cudaSuccess) return e;
+    return launch_pdl(absorb_out_kernel, dim3(p.Hkv, p.Dh / 16), dim3(256), osm, stream, p);
 }
 
 }  // namespace kvq

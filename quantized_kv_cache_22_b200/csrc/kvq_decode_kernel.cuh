@@ -453,8 +453,8 @@ __global__ void __launch_bounds__(NTHR, 2)
 #pragma unroll
                 for (int hs = 0; hs < 2; hs++) {
                     __half hv[4];
-#pragma unroll
                     __half hw[4];   // the other part (PK e4m3)
+#pragma unroll
                     for (int j = 0; j < 4; j++) {
                         // k-slots 2tig, 2tig+1, 2tig+8, 2tig+9 <-> elements 8tig + 4hs + j
                         const int d = 32 * blk + 8 * tig + 4 * hs + j;

@@ -231,6 +231,17 @@ __device__ __forceinline__ void imma_16832(int (&d)[4], uint32_t a0, uint32_t a1
     }
 }
 
+// D += A * B, m16n8k16, A row-major 16x16 bf16, B col-major 16x8 bf16, f32 acc
+// (fragment layout as for f16).
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1)
+{
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // Transpose an 8x8 matrix of 16-bit elements held one row pair per lane (lane
 // l: row l/4, columns 2(l%4), 2(l%4)+1): lane l receives row l/4 of the
 // transpose.
@@ -251,6 +262,15 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t a, uint32_t (&y)[4])
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4+%5];"
                  : "=r"(y[0]), "=r"(y[1]), "=r"(y[2]), "=r"(y[3])
                  : "r"(a), "n"(IMM));
+}
+// Four 8x8 matrices of 16-bit elements (ldmatrix): lanes 8m .. 8m + 7 give the row
+// addresses of matrix m (16 bytes each), and lane l receives y[m] = row l/4,
+// columns 2(l%4), 2(l%4)+1 of matrix m, the lower column in the low half.
+__device__ __forceinline__ void ldsm_x4(uint32_t a, uint32_t (&y)[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(y[0]), "=r"(y[1]), "=r"(y[2]), "=r"(y[3])
+                 : "r"(a));
 }
 // Ask for `bytes` (a multiple of 16, at a 16-byte aligned address) of global memory
 // to be brought into L2 by the copy engine; nothing is returned or waited for.
