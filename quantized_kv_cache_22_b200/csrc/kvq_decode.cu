@@ -51,8 +51,8 @@ __global__ void __launch_bounds__(256) merge_kernel(const MergeParams p)
     const long long Pe = N < (long long)p.num_ctas ? N : (long long)p.num_ctas;
     const long long u0 = before * p.n_kv_heads + (long long)kvh * tiles_b;
     const long long u1 = u0 + tiles_b;
-    const long long cmin = ((u0 + 1) * Pe + N - 1) / N - 1;
-    const long long cmax = (u1 * Pe + N - 1) / N - 1;
+    const long long cmin = range_cta(u0, N, Pe);
+    const long long cmax = range_cta(u1 - 1, N, Pe);
     const int bh = b * p.n_kv_heads + kvh;
     merge_segment<DH>(p.ws, cmin + bh, (int)(cmax - cmin + 1), G, p.out, p.out_f32, obase0, lane);
 }

@@ -235,6 +235,21 @@ __device__ __forceinline__ void merge_segment(const float *ws, int64_t slot0, in
 // sequence-major, then KV-head, then token order; they are split stream-K style
 // over the P' = min(P, units) CTAs that get work: CTA c takes units
 // [c N / P', (c + 1) N / P').  One warp finds this CTA's range; lane 0 writes it.
+// First unit of CTA c's range, c N / P', and the CTA whose range holds unit u,
+// ((u + 1) P' + N - 1) / N - 1: 32-bit divisions when the products fit (a 64-bit
+// division is several times longer, and these sit on the path to a segment's first
+// copy), else 64-bit.
+__device__ __forceinline__ long long range_begin(long long c, long long N, long long Pe)
+{
+    if (N * Pe < (1LL << 32)) return (long long)((uint32_t)(c * N) / (uint32_t)Pe);
+    return c * N / Pe;
+}
+__device__ __forceinline__ long long range_cta(long long u, long long N, long long Pe)
+{
+    if (N * (Pe + 1) < (1LL << 32)) return (long long)((uint32_t)((u + 1) * Pe + N - 1) / (uint32_t)N) - 1;
+    return ((u + 1) * Pe + N - 1) / N - 1;
+}
+
 struct WorkRange {
     long long u_begin;   // first unit of the range
     long long n;         // units in all
@@ -256,8 +271,8 @@ __device__ void decode_work_range(const DecodeParams &p, int lane, WorkRange &wr
     const long long Pe = N < (long long)p.num_ctas ? N : (long long)p.num_ctas;
     long long ub = 0, ue = 0;
     if ((long long)blockIdx.x < Pe) {
-        ub = (long long)blockIdx.x * N / Pe;
-        ue = ((long long)blockIdx.x + 1) * N / Pe;
+        ub = range_begin(blockIdx.x, N, Pe);
+        ue = range_begin((long long)blockIdx.x + 1, N, Pe);
     }
     // locate the sequence holding unit ub
     long long acc = 0;
@@ -411,8 +426,8 @@ __device__ void decode_producer(const DecodeParams &p, const CUtensorMap *tm_k,
         if (i == 0 || tile == 0) {
             // CTAs whose unit ranges meet this (sequence, KV head)
             const long long u0 = pre + (long long)kvh * tiles_b, u1 = u0 + tiles_b;
-            const long long cmin = ((u0 + 1) * Pe + N - 1) / N - 1;
-            const long long cmax = (u1 * Pe + N - 1) / N - 1;
+            const long long cmin = range_cta(u0, N, Pe);
+            const long long cmax = range_cta(u1 - 1, N, Pe);
             seg_cmin = (int)cmin;
             seg_ncta = (int)(cmax - cmin + 1);
         }
