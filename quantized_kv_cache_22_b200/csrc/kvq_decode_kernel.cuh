@@ -190,11 +190,24 @@ __global__ void __launch_bounds__(NTHR, 2)
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
     }
+    // The queries are read right after the work range: ask for this CTA's share of
+    // them to be brought into L2 now, while a preceding launch may still run (a
+    // prefetch only fills L2, which the preceding launch's writes update, and
+    // nothing waits for it).
+    if (tid == 32 * (NW + 1)) {
+        const uint64_t qbytes = (uint64_t)p.batch * p.n_q_heads * DH * (p.q_dtype == KVQ_F32 ? 4 : 2);
+        const uint64_t per = ((qbytes + gridDim.x - 1) / gridDim.x + 15) & ~(uint64_t)15;
+        const uint64_t off = (uint64_t)blockIdx.x * per;
+        if (off < qbytes) {
+            const uint64_t n = qbytes - off < per ? qbytes - off : per;
+            bulk_prefetch_l2(static_cast<const uint8_t *>(p.q) + off, (uint32_t)n);
+        }
+    }
     // Launched as a programmatic dependent: everything above only touches this
-    // CTA's shared memory and the launch parameters; from here on the kernel
-    // reads and writes global memory, so it first waits for the preceding
-    // grid (whatever it is) to complete.  The next launch may be scheduled now:
-    // it waits the same way before touching memory.
+    // CTA's shared memory and the launch parameters (and asks for an L2 prefetch);
+    // from here on the kernel reads and writes global memory, so it first waits for
+    // the preceding grid (whatever it is) to complete.  The next launch may be
+    // scheduled now: it waits the same way before touching memory.
     grid_dependency_wait();
     grid_launch_dependents();
 
