@@ -258,6 +258,7 @@ struct WorkRange {
     int b;               // first sequence of the range (-1: none)
     int bh0;             // first (sequence, KV head) of the range
     int n_units;         // units of the range
+    int tiles_b;         // tiles of each (sequence b, KV head)
 };
 
 __device__ void decode_work_range(const DecodeParams &p, int lane, WorkRange &wr)
@@ -305,6 +306,74 @@ __device__ void decode_work_range(const DecodeParams &p, int lane, WorkRange &wr
         wr.b = fb;
         wr.bh0 = fb >= 0 ? fb * Hkv + (int)((ub - fpre) / (funits / Hkv)) : 0;
         wr.n_units = (int)(ue > ub && fb >= 0 ? ue - ub : 0);
+        wr.tiles_b = (int)(funits / Hkv);
+    }
+}
+
+// The same range from lengths already in registers: lane l holds the lengths of
+// sequences l + 32 k, k < 8 (batch <= kSpecBatch), zero past the batch.  The decode
+// kernel computes it before its wait for the preceding launch, from lengths read
+// through L2 (so that no early copy stays in L1), and reads them again after the
+// wait: when a length changed in between, it computes the range anew.
+constexpr int kSpecBatch = 256;
+
+__device__ __forceinline__ void read_lens(const DecodeParams &p, int lane, int (&dl)[8])
+{
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+        const int b = lane + 32 * k;
+        dl[k] = b < p.batch ? __ldcg(p.d_len + b) : 0;
+    }
+}
+
+__device__ void work_range_from(const DecodeParams &p, int lane, WorkRange &wr, const int (&dl)[8])
+{
+    const int cap = p.cap;
+    const int Hkv = p.n_kv_heads;
+    long long total = 0;
+#pragma unroll
+    for (int k = 0; k < 8; k++) total += tiles_of(dl[k], cap);
+    for (int off = 16; off; off >>= 1) total += __shfl_xor_sync(FULL, total, off);
+    const long long N = total * Hkv;
+    const long long Pe = N < (long long)p.num_ctas ? N : (long long)p.num_ctas;
+    long long ub = 0, ue = 0;
+    if ((long long)blockIdx.x < Pe) {
+        ub = range_begin(blockIdx.x, N, Pe);
+        ue = range_begin((long long)blockIdx.x + 1, N, Pe);
+    }
+    long long acc = 0;
+    int fb = -1;
+    long long fpre = 0, funits = 0;
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+        if (fb >= 0 || ue <= ub) break;
+        const int b = 32 * k + lane;
+        const long long units = (long long)tiles_of(dl[k], cap) * Hkv;
+        long long incl = units;
+        for (int off = 1; off < 32; off <<= 1) {
+            const long long v = __shfl_up_sync(FULL, incl, off);
+            if (lane >= off) incl += v;
+        }
+        const long long excl = acc + incl - units;
+        const bool hit = units > 0 && excl <= ub && ub < excl + units;
+        const unsigned m = __ballot_sync(FULL, hit);
+        if (m) {
+            const int src = __ffs(m) - 1;
+            fb = __shfl_sync(FULL, b, src);
+            fpre = __shfl_sync(FULL, excl, src);
+            funits = __shfl_sync(FULL, units, src);
+        }
+        acc += __shfl_sync(FULL, incl, 31);
+    }
+    if (lane == 0) {
+        wr.u_begin = ub;
+        wr.n = N;
+        wr.pe = Pe;
+        wr.pre = fpre;
+        wr.b = fb;
+        wr.bh0 = fb >= 0 ? fb * Hkv + (int)((ub - fpre) / (funits / Hkv)) : 0;
+        wr.n_units = (int)(ue > ub && fb >= 0 ? ue - ub : 0);
+        wr.tiles_b = (int)(funits / Hkv);
     }
 }
 

@@ -208,12 +208,57 @@ __global__ void __launch_bounds__(NTHR, 2)
     // from here on the kernel reads and writes global memory, so it first waits for
     // the preceding grid (whatever it is) to complete.  The next launch may be
     // scheduled now: it waits the same way before touching memory.
+    // ---- work range of this CTA (computed by the producer warp) -------------
+    // With up to kSpecBatch sequences it is computed before the wait from lengths
+    // read through L2, and the first two tiles of the range are asked into L2 (both
+    // only speculation: the lengths are read again after the wait).
+    __shared__ WorkRange wr;
+    const bool spec = p.batch <= kSpecBatch;
+    int dl[8];
+    if (warp == NW && spec) {
+        read_lens(p, lane, dl);
+        work_range_from(p, lane, wr, dl);
+        __syncwarp();
+        if (lane == 0 && wr.n_units > 0 && p.block_table == nullptr && !p.stall) {
+            const int kvh = wr.bh0 % Hkv;
+            const int tile0 = (int)(wr.u_begin - wr.pre) - kvh * wr.tiles_b;
+            for (int t = tile0; t < tile0 + 2 && t - tile0 < wr.n_units && t < wr.tiles_b; t++) {
+                const int y0 = t * T, z = wr.bh0;
+                constexpr int RK = DH * KB / 8, RV = DH * VB / 8;
+                if constexpr (RK <= 128) {
+                    tma_prefetch_3d(&tm_k, 0, y0 / (128 / RK), z);
+                } else {
+                    tma_prefetch_3d(&tm_k, 0, y0, z);
+                    tma_prefetch_3d(&tm_k, 128, y0, z);
+                }
+                if constexpr (RV <= 128) {
+                    tma_prefetch_3d(&tm_v, 0, y0 / (128 / RV), z);
+                } else {
+                    tma_prefetch_3d(&tm_v, 0, y0, z);
+                    tma_prefetch_3d(&tm_v, 128, y0, z);
+                }
+                const int n_s = min(T, cap - y0);
+                if (KB != 16 && !PT)
+                    bulk_prefetch_l2(p.k_scales + ((int64_t)z * cap + y0) * p.ngs_k, (uint32_t)(n_s * p.ngs_k * 2));
+                if (VB != 16 && !PT)
+                    bulk_prefetch_l2(p.v_scales + ((int64_t)z * cap + y0) * p.ngs_v, (uint32_t)(n_s * p.ngs_v * 2));
+            }
+        }
+    }
     grid_dependency_wait();
     grid_launch_dependents();
-
-    // ---- work range of this CTA (computed by the producer warp) -------------
-    __shared__ WorkRange wr;
-    if (warp == NW) decode_work_range(p, lane, wr);
+    if (warp == NW) {
+        if (spec) {
+            int now[8];
+            read_lens(p, lane, now);
+            bool same = true;
+#pragma unroll
+            for (int k = 0; k < 8; k++) same = same && now[k] == dl[k];
+            if (!__all_sync(FULL, same)) work_range_from(p, lane, wr, now);
+        } else {
+            decode_work_range(p, lane, wr);
+        }
+    }
     __syncthreads();
     const int n_units = wr.n_units;
 

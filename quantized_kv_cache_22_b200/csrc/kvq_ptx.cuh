@@ -120,6 +120,16 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *m, uin
         : "memory");
 }
 
+// Ask for the box of a tiled 3-D tensor map at the given coordinates to be brought
+// into L2 (nothing is written to shared memory, nothing waits for it).
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *m, int x, int y, int z)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(m)),
+                 "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+
 // L2 cache policy that makes the lines a copy brings in the first to be evicted
 // (for data read once, so that it does not push out data that is read again).
 __device__ __forceinline__ uint64_t l2_evict_first_policy()
