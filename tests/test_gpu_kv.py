@@ -142,6 +142,51 @@ def test_decode_split_count_invariance(cuda_device):
         assert np.abs(o - outs[0]).max() <= 2.0 ** -11 * vmax.max()
 
 
+@pytest.mark.parametrize("B", [256, 257])
+def test_decode_batch_at_and_past_early_range_limit(cuda_device, B):
+    """Up to 256 sequences the kernel finds its work range from lengths it reads
+    before the wait for the preceding launch (and reads again after it); past 256 it
+    reads them after the wait only.  Both sides of that limit match the oracle, with
+    ragged lengths (zero included)."""
+    Hkv, G, dh, cap = 1, 2, 64, 48
+    rng = np.random.default_rng(B)
+    lens = [int(x) for x in rng.integers(0, cap + 1, size=B)]
+    lens[0], lens[-1] = 0, cap
+    k, v, q = _inputs(B, cap, Hkv, G, dh, torch.float16, 61)
+    cfg = _cfg(B, cap, Hkv, G, dh, (8, 4, 0, 0))
+    cache = gpu_cache(cfg, k, v)
+    oc = oracle_cache(k, v, cfg)
+    want = oracle_decode(cfg, oc, q, lens)
+    got = gpu_decode(cfg, cache, q, lens)
+    assert np.all(got[0] == 0)
+    assert_close_to_oracle(got, want, vmax_per_batch(oc[2], oc[3], cfg, lens), G, f"B={B}")
+
+
+def test_decode_lengths_rewritten_on_device_between_calls(cuda_device):
+    """A length changed on the device by the launch right before the decode call (the
+    kernel's early read of the lengths may see the old ones) gives the new lengths'
+    result, call after call."""
+    B, Hkv, G, dh, cap = 4, 2, 4, 128, 512
+    k, v, q = _inputs(B, cap, Hkv, G, dh, torch.float16, 67)
+    cfg = _cfg(B, cap, Hkv, G, dh, (8, 8, 0, 0))
+    cache = gpu_cache(cfg, k, v)
+    oc = oracle_cache(k, v, cfg)
+    vmaxs = {}
+    d_len = torch.tensor([512, 300, 1, 129], dtype=torch.int32, device="cuda")
+    out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    ws = Workspace(cfg, 0, torch.device("cuda"))
+    qd = q.cuda()
+    for step, delta in enumerate([0, -37, 90, -200, 64]):
+        d_len.add_(delta).clamp_(0, cap)          # a device kernel right before the call
+        kvq.kvq_decode_attn(cfg, cache, qd, d_len, cap, out, ws)
+        torch.cuda.synchronize()
+        lens = [int(x) for x in d_len.cpu()]
+        want = oracle_decode(cfg, oc, q, lens)
+        assert_close_to_oracle(out.cpu().numpy(), want, vmax_per_batch(oc[2], oc[3], cfg, lens), G,
+                               f"step {step} lens {lens}")
+    assert kvq.kvq_workspace_status(ws) == 0
+
+
 def test_decode_edge_lengths_and_capacity_tail(cuda_device):
     # capacity 80 is not a multiple of the 64-token tile: the last tile runs past it
     B, Hkv, G, dh, cap = 6, 1, 2, 128, 80
