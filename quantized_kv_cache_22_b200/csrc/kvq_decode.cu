@@ -167,6 +167,9 @@ bool plan_decode(int dh, int kb, int vb, int ngs_k, int ngs_v, int G, int max_sm
     // as many stages as fit next to the other CTAs of an SM (228 KB of shared memory,
     // 1 KB of it reserved per CTA, 128 B left for the kernel's static shared memory),
     // else as many as fit in one CTA
+    // (with one CTA per SM the dynamic part may use the opt-in maximum less the kernel's
+    // static shared memory, about 1 KB)
+    max_smem -= 2048;
     const uint32_t per_cta = 233472u / (uint32_t)kDecodeCtasPerSm - 1024u - 128u;
     for (int S = 8; S >= 2; S--) {
         const uint32_t off_meta = S * L.stage_bytes;
