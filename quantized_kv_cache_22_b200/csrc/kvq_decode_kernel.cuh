@@ -45,6 +45,10 @@
 //     the P operand by two 8x8 transposes (movmatrix).
 //   * The online softmax tracks max(s + log2 s_V) so that p * s_V <= 2^8 fits
 //     fp16 without underflow whatever the value scales are.
+//   * In a chain of launches the next layer's CTAs start while this one's last
+//     CTAs finish: each finds its work range and asks its first tiles and its
+//     queries into L2 before the wait for the previous launch, and checks the
+//     lengths it used after it.
 #pragma once
 #include <cfloat>
 #include <type_traits>
@@ -203,15 +207,15 @@ __global__ void __launch_bounds__(NTHR, 2)
             bulk_prefetch_l2(static_cast<const uint8_t *>(p.q) + off, (uint32_t)n);
         }
     }
-    // Launched as a programmatic dependent: everything above only touches this
-    // CTA's shared memory and the launch parameters (and asks for an L2 prefetch);
-    // from here on the kernel reads and writes global memory, so it first waits for
-    // the preceding grid (whatever it is) to complete.  The next launch may be
-    // scheduled now: it waits the same way before touching memory.
+    // Launched as a programmatic dependent: until grid_dependency_wait() below the
+    // preceding grid (whatever it is) may still be writing global memory.  Before
+    // the wait the kernel touches only its shared memory and the launch parameters,
+    // asks for L2 prefetches, and reads the sequence lengths (through L2) to find its
+    // work range speculatively; after the wait it reads the lengths again and finds
+    // the range anew if any changed, so nothing read early is used unchecked.  The
+    // next launch may be scheduled once this one has passed the wait.
     // ---- work range of this CTA (computed by the producer warp) -------------
-    // With up to kSpecBatch sequences it is computed before the wait from lengths
-    // read through L2, and the first two tiles of the range are asked into L2 (both
-    // only speculation: the lengths are read again after the wait).
+    // With more than kSpecBatch sequences it is found after the wait only.
     __shared__ WorkRange wr;
     const bool spec = p.batch <= kSpecBatch;
     int dl[8];
