@@ -165,14 +165,21 @@ bool plan_decode(int dh, int kb, int vb, int ngs_k, int ngs_v, int G, int max_sm
     const uint32_t merge_bytes = (uint32_t)NW * G * slot_col_floats(dh) * 4;
     // tail: meta[S] (32 B each), barriers (2S + 2) * 8 B, control words 64 B, merge buffer;
     // as many stages as fit next to the other CTAs of an SM (228 KB of shared memory,
-    // 1 KB of it reserved per CTA, 128 B left for the kernel's static shared memory),
+    // 1 KB of it reserved per CTA, 1 KB for the kernel's static shared memory),
     // else two stages in one CTA per SM (16-bit K and V at 128-element heads, 64 KB a
     // stage: a third stage measured slower, 29.6-30.3 against 28.5 us for 8 x 1024 tokens
     // of 16 heads)
     // (with one CTA per SM the dynamic part may use the opt-in maximum less the kernel's
     // static shared memory, about 1 KB)
     max_smem -= 2048;
-    const uint32_t per_cta = 233472u / (uint32_t)kDecodeCtasPerSm - 1024u - 128u;
+    // beside another CTA: 228 KB per SM, of which 1 KB is reserved per CTA and 1 KB is
+    // the kernel's static part (the dynamic part starts 1024-byte aligned)
+    const uint32_t per_cta = 233472u / (uint32_t)kDecodeCtasPerSm - 1024u - 1024u;
+    // packed-column int8 keys without zero-points: the consumer warps may quantise a
+    // segment's query rows one head each and share them ([4][2][Dh] bytes, 4 factors,
+    // 2 mbarriers after the merge buffer), where that costs neither a stage nor a CTA
+    const bool qshare = L.pk && kb != 16 && fmt != KVQ_FMT_E4M3 && fmt != KVQ_FMT_ASYM;
+    const uint32_t qs_bytes = 8u * dh + 16u + 16u;
     for (int S = 8; S >= 2; S--) {
         const uint32_t off_meta = S * L.stage_bytes;
         const uint32_t off_bar = off_meta + S * (uint32_t)sizeof(StageMeta);
@@ -185,6 +192,12 @@ bool plan_decode(int dh, int kb, int vb, int ngs_k, int ngs_v, int G, int max_sm
             L.off_bar = off_bar;
             L.off_merge = off_merge;
             L.smem_bytes = total;
+            const uint32_t off_qs = align_up(off_merge + merge_bytes, 16);
+            const uint32_t with_qs = off_qs + qs_bytes + 1024;
+            if (qshare && with_qs <= (uint32_t)max_smem && (with_qs <= per_cta || L.per_sm == 1)) {
+                L.off_qs = off_qs;
+                L.smem_bytes = with_qs;
+            }
             *plan = L;
             return true;
         }

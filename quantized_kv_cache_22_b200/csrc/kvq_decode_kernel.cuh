@@ -189,6 +189,12 @@ __global__ void __launch_bounds__(NTHR, 2)
         }
         mbar_init(&segbar[0], NW);   // consumers: partials of a segment in mbuf
         mbar_init(&segbar[1], 1);    // combiner: mbuf read
+        if (PK && KB != 16 && !F8 && FMT != KVQ_FMT_ASYM && p.off_qs != 0) {
+            // shared query quantisation: [0] every head written, [1] every warp has read
+            uint64_t *qbar = reinterpret_cast<uint64_t *>(smem + p.off_qs + 8 * DH + 16);
+            mbar_init(&qbar[0], NW);
+            mbar_init(&qbar[1], NW);
+        }
         ctl[0] = 0;
         fence_mbar_init();
         prefetch_tensormap(&tm_k);
@@ -551,6 +557,109 @@ __global__ void __launch_bounds__(NTHR, 2)
             for (int i = 0; i < 4; i++) o_acc[mt][i] = 0.f;
     };
 
+    // The same fragments with the quantisation shared (packed-column int8 keys without
+    // zero-points): consumer warp w quantises head w of the segment (lane l: elements
+    // 4l .. 4l+3) into shared memory, and after every warp has written (qbar[0]) each
+    // lane reads its fragments back.  k counts the shared segment starts of this CTA;
+    // a warp writes only after every warp has read the previous segment's (qbar[1]).
+    // The arithmetic is that of load_q, so the fragments are the same bits; like
+    // load_q it starts the segment's softmax state and accumulators afresh.
+    constexpr bool QSHARE = PK && IMMA_K && !ZP;
+    auto share_q = [&](int bh, uint32_t k) -> bool {
+        uint8_t *qsh = smem + p.off_qs;                                  // [4][2][DH] bytes
+        float *qfac = reinterpret_cast<float *>(qsh + 8 * DH);
+        uint64_t *qbar = reinterpret_cast<uint64_t *>(qsh + 8 * DH + 16);
+        const uint32_t qsb = smem_u32(qsh);
+        if (k > 0 && !mbar_wait_bounded(&qbar[1], (k - 1) & 1u, abort_flag, p.timeout_ns)) return false;
+        if (warp < G) {
+            const int b = bh / Hkv, kvh = bh % Hkv;
+            const int64_t base = ((int64_t)b * p.n_q_heads + (int64_t)kvh * G + warp) * DH + 4 * lane;
+            float x[4];
+            if (p.q_dtype == KVQ_F32) {
+                const float4 v = __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(p.q) + base));
+                x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+            } else {
+                const uint2 w = __ldg(reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(p.q) + base));
+                const uint32_t ws[2] = {w.x, w.y};
+#pragma unroll
+                for (int i2 = 0; i2 < 2; i2++) {
+                    if (p.q_dtype == KVQ_F16) {
+                        x[2 * i2] = __half2float(__ushort_as_half((unsigned short)(ws[i2] & 0xFFFFu)));
+                        x[2 * i2 + 1] = __half2float(__ushort_as_half((unsigned short)(ws[i2] >> 16)));
+                    } else {
+                        x[2 * i2] = __uint_as_float(ws[i2] << 16);
+                        x[2 * i2 + 1] = __uint_as_float(ws[i2] & 0xFFFF0000u);
+                    }
+                }
+            }
+            float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, off));
+            const float inv = amax > 0.f ? 127.f / amax : 0.f;
+            int hi[4], lo[4];
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const float y = x[j] * inv;
+                const float r = rintf(y);
+                hi[j] = (int)r;
+                lo[j] = __float2int_rn((y - r) * 254.f);
+            }
+            *reinterpret_cast<uint32_t *>(qsh + warp * 2 * DH + 4 * lane) = pack_bytes(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint32_t *>(qsh + warp * 2 * DH + DH + 4 * lane) = pack_bytes(lo[0], lo[1], lo[2], lo[3]);
+            if (lane == 0)
+                qfac[warp] = amax * (1.f / (127.f * 254.f)) * p.tau_log2e * (KB == 4 ? 0.0625f : 1.f);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&qbar[0]);
+        if (!mbar_wait_bounded(&qbar[0], k & 1u, abort_flag, p.timeout_ns)) return false;
+        const int qhd = gid & 3;
+        const bool valid = qhd < G;
+#pragma unroll
+        for (int blk = 0; blk < NG; blk++) {
+            const int e0 = (blk / KPL) * 32 * KPL + 8 * KPL * tig + 8 * (blk % KPL);
+            uint2 h8 = make_uint2(0u, 0u), l8 = make_uint2(0u, 0u);
+            if (valid) {
+                h8 = lds_u64(qsb, qhd * 2 * DH + e0);
+                l8 = lds_u64(qsb, qhd * 2 * DH + DH + e0);
+            }
+            if constexpr (KB == 8) {
+                // k-slot 4tig+i <-> element 8tig+i, 16+4tig+i <-> 8tig+4+i
+                qh[blk][0] = h8.x; qh[blk][1] = h8.y;
+                ql[blk][0] = l8.x; ql[blk][1] = l8.y;
+            } else {
+                // k-slot 4tig+i <-> element 8tig+2i (low nibbles), 16+4tig+i <-> 8tig+2i+1
+                qh[blk][0] = prmt(h8.x, h8.y, 0x6420u); qh[blk][1] = prmt(h8.x, h8.y, 0x7531u);
+                ql[blk][0] = prmt(l8.x, l8.y, 0x6420u); ql[blk][1] = prmt(l8.x, l8.y, 0x7531u);
+            }
+            // qh = [hi | lo] (sub-tile 0's B operand), ql = [lo | hi] (sub-tile 1's)
+            if (gid >= 4) {
+                const uint32_t t0 = qh[blk][0], t1 = qh[blk][1];
+                qh[blk][0] = ql[blk][0];
+                qh[blk][1] = ql[blk][1];
+                ql[blk][0] = t0;
+                ql[blk][1] = t1;
+            }
+        }
+        const int hc = 2 * (tig & 1);   // the lane's first head column
+        sqc[0] = hc < G ? qfac[hc] : 0.f;
+        sqc[1] = hc + 1 < G ? qfac[hc + 1] : 0.f;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&qbar[1]);
+        // a fresh softmax state and accumulators for the segment
+#pragma unroll
+        for (int c = 0; c < 2; c++) {
+            m_run[c] = -INFINITY;
+            l_run[c] = 0.f;
+        }
+#pragma unroll
+        for (int g = 0; g < NVG; g++) psum[g][0] = psum[g][1] = psum[g][2] = psum[g][3] = 0.f;
+#pragma unroll
+        for (int mt = 0; mt < 2 * NG; mt++)
+#pragma unroll
+            for (int i2 = 0; i2 < 4; i2++) o_acc[mt][i2] = 0.f;
+        return true;
+    };
+
     // int8 A fragments of one 32-element key block for the rows at shared
     // addresses ra (row gid) and rb (row gid + 8), plus IMM bytes
     auto key_frags = [&](auto imm, uint32_t ra, uint32_t rb, uint32_t (&fa)[4]) {
@@ -579,6 +688,7 @@ __global__ void __launch_bounds__(NTHR, 2)
     int s = 0;
     uint32_t ph = 0;
     uint32_t nseg = 0;           // segment ends handed to the combiner
+    uint32_t nqs = 0;            // segment starts with the query quantisation shared
     bool aborted = false;
     // the first segment's query is loaded while its first tile is in flight
     if (n_units > 0) load_q(wr.bh0);
@@ -596,7 +706,18 @@ __global__ void __launch_bounds__(NTHR, 2)
             m.bh = (int)m0.x; m.t0 = (int)m0.y; m.len = (int)m0.z; m.flags = (int)m0.w;
             m.slot = (int)m1.x; m.ncta = (int)m1.y; m.cmin = (int)m1.z;
         }
-        if ((m.flags & 1) && i > 0) load_q(m.bh);
+        if ((m.flags & 1) && i > 0) {
+            if (QSHARE && p.off_qs != 0) {
+                if (!share_q(m.bh, nqs++)) {
+                    ctl[0] = 1;
+                    atomicExch(p.status, KVQ_ERR_TIMEOUT);
+                    aborted = true;
+                    break;
+                }
+            } else {
+                load_q(m.bh);
+            }
+        }
         const uint32_t st = (uint32_t)s * p.stage_bytes;   // stage offset from smem
         const uint32_t sst = sbase + st;                    // shared address of the stage
         const uint32_t ssk = st + p.off_sk;   // fp16 key scales of the stage

@@ -285,8 +285,9 @@ def test_decode_plan_info_without_device(monkeypatch):
         assert info["engine"] == kvq.KVQ_ENGINE_WARP_MMA and info["num_ctas"] == 296
         assert info["ctas_per_sm_planned"] == per_sm and info["threads"] == 192
         assert info["stages"] >= 2 and info["stage_bytes"] * info["stages"] < info["smem_bytes"]
-        # the plan's shared memory leaves room for that many CTAs on a 228 KB SM
-        assert per_sm * (info["smem_bytes"] + 1024 + 128) <= 233472
+        # the plan's shared memory leaves room for that many CTAs on a 228 KB SM (1 KB
+        # reserved per CTA, 1 KB of static shared memory before the aligned dynamic part)
+        assert per_sm * (info["smem_bytes"] + 1024 + 1024) <= 233472
     assert kvq.kvq_decode_plan_info(cfg(4, 4, vg=64, dh=64), 10)["ctas_per_sm_planned"] == 2
     # packed score columns for G <= 4 at head_dim 128 with INT4 / INT8 keys
     assert kvq.kvq_decode_plan_info(cfg(8, 4), 296)["packed_columns"] == 1
