@@ -548,7 +548,9 @@ static int decode_kv_layout(const kvq_config *cfg, const void *k_codes, const vo
         p.off_meta = plan.off_meta;
         p.off_bar = plan.off_bar;
         p.off_merge = plan.off_merge;
-        p.off_qs = plan.off_qs;
+        p.off_qhi = plan.off_qhi;
+        p.off_qlo = plan.off_qlo;
+        p.off_qmisc = plan.off_qmisc;
         p.tc = plan.tco;
         const float scale = softmax_scale != 0.f ? softmax_scale : 1.f / std::sqrt((float)a.dh);
         p.tau_log2e = scale * 1.4426950408889634f;

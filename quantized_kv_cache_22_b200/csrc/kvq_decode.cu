@@ -176,10 +176,14 @@ bool plan_decode(int dh, int kb, int vb, int ngs_k, int ngs_v, int G, int max_sm
     // the kernel's static part (the dynamic part starts 1024-byte aligned)
     const uint32_t per_cta = 233472u / (uint32_t)kDecodeCtasPerSm - 1024u - 1024u;
     // packed-column int8 keys without zero-points: the consumer warps may quantise a
-    // segment's query rows one head each and share them ([4][2][Dh] bytes, 4 factors,
-    // 2 mbarriers after the merge buffer), where that costs neither a stage nor a CTA
+    // segment's query rows one head each and share them (hi and lo bytes, [4][Dh]
+    // each, then 4 factors and 2 mbarriers), where that costs neither a stage nor a
+    // CTA: after the merge buffer, or else in the unused tails of the first three
+    // stages (no copy writes past a stage's scales)
     const bool qshare = L.pk && kb != 16 && fmt != KVQ_FMT_E4M3 && fmt != KVQ_FMT_ASYM;
     const uint32_t qs_bytes = 8u * dh + 16u + 16u;
+    const uint32_t used = align_up(L.off_sv + T * (vb == 16 ? 0 : ngs_v) * 2, 16);
+    const uint32_t tail = L.stage_bytes - used;
     for (int S = 8; S >= 2; S--) {
         const uint32_t off_meta = S * L.stage_bytes;
         const uint32_t off_bar = off_meta + S * (uint32_t)sizeof(StageMeta);
@@ -195,8 +199,14 @@ bool plan_decode(int dh, int kb, int vb, int ngs_k, int ngs_v, int G, int max_sm
             const uint32_t off_qs = align_up(off_merge + merge_bytes, 16);
             const uint32_t with_qs = off_qs + qs_bytes + 1024;
             if (qshare && with_qs <= (uint32_t)max_smem && (with_qs <= per_cta || L.per_sm == 1)) {
-                L.off_qs = off_qs;
+                L.off_qhi = off_qs;
+                L.off_qlo = off_qs + 4u * dh;
+                L.off_qmisc = off_qs + 8u * dh;
                 L.smem_bytes = with_qs;
+            } else if (qshare && S >= 3 && tail >= 4u * dh) {
+                L.off_qhi = used;
+                L.off_qlo = L.stage_bytes + used;
+                L.off_qmisc = 2u * L.stage_bytes + used;
             }
             *plan = L;
             return true;

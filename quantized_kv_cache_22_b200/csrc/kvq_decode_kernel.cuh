@@ -189,9 +189,9 @@ __global__ void __launch_bounds__(NTHR, 2)
         }
         mbar_init(&segbar[0], NW);   // consumers: partials of a segment in mbuf
         mbar_init(&segbar[1], 1);    // combiner: mbuf read
-        if (PK && KB != 16 && !F8 && FMT != KVQ_FMT_ASYM && p.off_qs != 0) {
+        if (PK && KB != 16 && !F8 && FMT != KVQ_FMT_ASYM && p.off_qmisc != 0) {
             // shared query quantisation: [0] every head written, [1] every warp has read
-            uint64_t *qbar = reinterpret_cast<uint64_t *>(smem + p.off_qs + 8 * DH + 16);
+            uint64_t *qbar = reinterpret_cast<uint64_t *>(smem + p.off_qmisc + 16);
             mbar_init(&qbar[0], NW);
             mbar_init(&qbar[1], NW);
         }
@@ -566,10 +566,10 @@ __global__ void __launch_bounds__(NTHR, 2)
     // load_q it starts the segment's softmax state and accumulators afresh.
     constexpr bool QSHARE = PK && IMMA_K && !ZP;
     auto share_q = [&](int bh, uint32_t k) -> bool {
-        uint8_t *qsh = smem + p.off_qs;                                  // [4][2][DH] bytes
-        float *qfac = reinterpret_cast<float *>(qsh + 8 * DH);
-        uint64_t *qbar = reinterpret_cast<uint64_t *>(qsh + 8 * DH + 16);
-        const uint32_t qsb = smem_u32(qsh);
+        uint8_t *qhi = smem + p.off_qhi;                                 // [4][DH] bytes
+        uint8_t *qlo = smem + p.off_qlo;                                 // [4][DH] bytes
+        float *qfac = reinterpret_cast<float *>(smem + p.off_qmisc);
+        uint64_t *qbar = reinterpret_cast<uint64_t *>(smem + p.off_qmisc + 16);
         if (k > 0 && !mbar_wait_bounded(&qbar[1], (k - 1) & 1u, abort_flag, p.timeout_ns)) return false;
         if (warp < G) {
             const int b = bh / Hkv, kvh = bh % Hkv;
@@ -604,8 +604,8 @@ __global__ void __launch_bounds__(NTHR, 2)
                 hi[j] = (int)r;
                 lo[j] = __float2int_rn((y - r) * 254.f);
             }
-            *reinterpret_cast<uint32_t *>(qsh + warp * 2 * DH + 4 * lane) = pack_bytes(hi[0], hi[1], hi[2], hi[3]);
-            *reinterpret_cast<uint32_t *>(qsh + warp * 2 * DH + DH + 4 * lane) = pack_bytes(lo[0], lo[1], lo[2], lo[3]);
+            *reinterpret_cast<uint32_t *>(qhi + warp * DH + 4 * lane) = pack_bytes(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint32_t *>(qlo + warp * DH + 4 * lane) = pack_bytes(lo[0], lo[1], lo[2], lo[3]);
             if (lane == 0)
                 qfac[warp] = amax * (1.f / (127.f * 254.f)) * p.tau_log2e * (KB == 4 ? 0.0625f : 1.f);
         }
@@ -619,8 +619,8 @@ __global__ void __launch_bounds__(NTHR, 2)
             const int e0 = (blk / KPL) * 32 * KPL + 8 * KPL * tig + 8 * (blk % KPL);
             uint2 h8 = make_uint2(0u, 0u), l8 = make_uint2(0u, 0u);
             if (valid) {
-                h8 = lds_u64(qsb, qhd * 2 * DH + e0);
-                l8 = lds_u64(qsb, qhd * 2 * DH + DH + e0);
+                h8 = lds_u64(smem_u32(qhi), qhd * DH + e0);
+                l8 = lds_u64(smem_u32(qlo), qhd * DH + e0);
             }
             if constexpr (KB == 8) {
                 // k-slot 4tig+i <-> element 8tig+i, 16+4tig+i <-> 8tig+4+i
@@ -707,7 +707,7 @@ __global__ void __launch_bounds__(NTHR, 2)
             m.slot = (int)m1.x; m.ncta = (int)m1.y; m.cmin = (int)m1.z;
         }
         if ((m.flags & 1) && i > 0) {
-            if (QSHARE && p.off_qs != 0) {
+            if (QSHARE && p.off_qmisc != 0) {
                 if (!share_q(m.bh, nqs++)) {
                     ctl[0] = 1;
                     atomicExch(p.status, KVQ_ERR_TIMEOUT);

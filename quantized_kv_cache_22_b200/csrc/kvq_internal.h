@@ -86,8 +86,9 @@ struct DecodeParams {
     int32_t stages;
     uint32_t stage_bytes, off_v, off_sk, off_sv, off_meta, off_bar, off_merge;
     // packed-column int8 instances: where the consumer warps share a segment's query
-    // quantisation ([4 heads][hi, lo][Dh] bytes, 4 factors, 2 mbarriers); 0 for none
-    uint32_t off_qs;
+    // quantisation: hi and lo bytes ([4 heads][Dh] each) and 4 factors + 2 mbarriers
+    // (32 bytes); off_qmisc 0 for none
+    uint32_t off_qhi, off_qlo, off_qmisc;
     float tau_log2e;
     uint64_t timeout_ns;
     FusedAppend app;
@@ -149,7 +150,7 @@ struct DecodeLaunch {
     size_t smem_bytes;
     int stages;
     uint32_t stage_bytes, off_v, off_sk, off_sv, off_meta, off_bar, off_merge;
-    uint32_t off_qs;          // shared query quantisation (0: none)
+    uint32_t off_qhi, off_qlo, off_qmisc;   // shared query quantisation (off_qmisc 0: none)
     TcOffsets tco;
 };
 
